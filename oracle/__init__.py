@@ -1,0 +1,123 @@
+"""fp64 CPU oracle for the ViT^3 test-time-training layer forward -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline / reference leg of
+``bench.py`` may import this package.  The CUDA product path never does, and it shares no code
+with it.  Every function takes numpy arrays in the layout documented in ``ttt_oracle.c``
+([B][heads][N][d] for Q, K, V, Z), widens them exactly to float64 and returns float64 results.
+
+Functions and the definitions they follow (page titles and sections; see ``ttt_oracle.c``):
+  linear(...)       L2 loss, one full-batch gradient step on W (d x d), z = W1 q  -- per-pair form
+  linear_gram(...)  the same step written as W0 - eta (2/N) (W0 K K^T - V K^T)
+  dwconv(...)       the same loss with a 3x3 depthwise cross-correlation inner model
+  mlp(...)          the same loss with f(x) = Wb gelu_tanh(Wa x)
+  gelu_tanh(u), gelu_tanh_deriv(u)
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py (closed forms,
+invariants, exact finite differences, autograd and library special cases).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i = ctypes.c_int
+        d = ctypes.c_double
+        lib.oracle_linear.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_linear_gram.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
+        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_dwconv, lib.oracle_mlp):
+            f.restype = ctypes.c_int
+        lib.oracle_gelu_tanh.argtypes = [d]
+        lib.oracle_gelu_tanh.restype = d
+        lib.oracle_gelu_tanh_deriv.argtypes = [d]
+        lib.oracle_gelu_tanh_deriv.restype = d
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    """Exact widening to a contiguous float64 array (bf16 / fp32 values are representable)."""
+    if hasattr(x, "detach"):  # a torch tensor: widen through torch, then hand over to numpy
+        x = x.detach().to("cpu").double().contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads():
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _check(status, name):
+    if status != 0:
+        raise RuntimeError(f"oracle {name} failed with status {status}")
+
+
+def linear(Q, K, V, W0, eta, threads=None, gram=False):
+    """Returns (Z [B][h][N][d], W1 [B][h][d][d]) in float64."""
+    Q, K, V, W0 = _f64(Q), _f64(K), _f64(V), _f64(W0)
+    B, H, N, d = Q.shape
+    assert K.shape == Q.shape and V.shape == Q.shape and W0.shape == (H, d, d)
+    Z = np.empty_like(Q)
+    W1 = np.empty((B, H, d, d))
+    fn = _load().oracle_linear_gram if gram else _load().oracle_linear
+    _check(fn(B, H, N, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1), _p(Z),
+              threads or default_threads()), "linear")
+    return Z, W1
+
+
+def linear_gram(Q, K, V, W0, eta, threads=None):
+    return linear(Q, K, V, W0, eta, threads=threads, gram=True)
+
+
+def dwconv(Q, K, V, W0, eta, Hg, Wg, threads=None):
+    """Q, K, V: [B][h][Hg*Wg][d]; W0: [h][d][3][3].  Returns (Z, W1 [B][h][d][3][3])."""
+    Q, K, V, W0 = _f64(Q), _f64(K), _f64(V), _f64(W0)
+    B, H, N, d = Q.shape
+    assert N == Hg * Wg and K.shape == Q.shape and V.shape == Q.shape and W0.shape == (H, d, 3, 3)
+    Z = np.empty_like(Q)
+    W1 = np.empty((B, H, d, 3, 3))
+    _check(_load().oracle_dwconv(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1),
+                                 _p(Z), threads or default_threads()), "dwconv")
+    return Z, W1
+
+
+def mlp(Q, K, V, Wa, Wb, eta, threads=None):
+    """Wa: [h][hidden][d], Wb: [h][d][hidden].  Returns (Z, Wa1 [B][h][hidden][d], Wb1 [B][h][d][hidden])."""
+    Q, K, V, Wa, Wb = _f64(Q), _f64(K), _f64(V), _f64(Wa), _f64(Wb)
+    B, H, N, d = Q.shape
+    hidden = Wa.shape[1]
+    assert Wa.shape == (H, hidden, d) and Wb.shape == (H, d, hidden)
+    Z = np.empty_like(Q)
+    Wa1 = np.empty((B, H, hidden, d))
+    Wb1 = np.empty((B, H, d, hidden))
+    _check(_load().oracle_mlp(B, H, N, d, hidden, _p(Q), _p(K), _p(V), _p(Wa), _p(Wb), float(eta),
+                              _p(Wa1), _p(Wb1), _p(Z), threads or default_threads()), "mlp")
+    return Z, Wa1, Wb1
+
+
+def gelu_tanh(u):
+    return _load().oracle_gelu_tanh(float(u))
+
+
+def gelu_tanh_deriv(u):
+    return _load().oracle_gelu_tanh_deriv(float(u))
+
+
+def max_threads():
+    return _load().oracle_max_threads()

@@ -1,0 +1,358 @@
+/*
+ * ttt_oracle.c -- plain fp64 CPU oracle for the ViT^3 test-time-training (TTT) layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load this file or the
+ * library built from it.  Only the test suite, the package smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes (one "unit" = one image b and one head h; N = H*W tokens of width d):
+ *   The token sequence is treated as a small dataset of (key -> value) pairs.  An inner model f(.;W)
+ *   is trained on it by ONE full-batch, non-causal gradient step of the L2 reconstruction loss
+ *       L(W) = (1/N) * sum_n || f(k_n; W) - v_n ||^2
+ *   and the updated model is then applied to every query:  z_n = f(q_n; W1),  W1 = W0 - eta*dL/dW(W0).
+ *   Sources (pages on ViT^3 / vision TTT, cited by title and section):
+ *     - "CVPR 2026 Oral | 清華+阿里發布ViT3" (press article), section 序列建模的新視角: keys and
+ *       values form a dataset, the inner model learns to reconstruct v from k by gradient descent
+ *       with e.g. an L2 loss, and the trained model is then applied to the queries.
+ *     - same article, Observation 2 and Fig. 3: one full-batch (B = N) step over all pairs, with no
+ *       ordering between tokens.
+ *     - "Vision-TTT: Efficient and Expressive Visual Representation Learning with Test-Time
+ *       Training" (paper notes), section 关键设计 1: the L2 loss ||W x_K - x_V||^2, its gradient
+ *       2 (W x_K - x_V) x_K^T and the readout z = W x_Q, one d x d matrix per head.
+ *     - press article, Observations 4 and 6 (Fig. 5 parts 1 and 3): the inner model may be a
+ *       2-layer MLP (width ratio up to 4) or a 3x3 depthwise convolution over the token grid.
+ *   Readings where the pages are silent (each also listed in the design notes of the repository):
+ *     - the gradient is the MEAN over the N pairs (factor 2/N), not the sum;
+ *     - the conv head is a cross-correlation with zero padding, stride 1, no bias, one 3x3 kernel
+ *       per channel, tokens in raster order n = y*W + x, channel c = feature c of the head;
+ *     - the MLP head is f(x) = Wb * gelu_tanh(Wa * x) with no biases, and both matrices take one
+ *       simultaneous step from gradients evaluated at the initial weights.
+ *
+ * Memory layout of every array (contiguous, row-major, fp64):
+ *   Q, K, V, Z : [B][heads][N][d]     (token n, feature c at ((b*heads + h)*N + n)*d + c)
+ *   linear W   : [heads][d][d]        W[i][j] maps input feature j to output feature i
+ *   conv W     : [heads][d][3][3]     W[c][a][b] multiplies the input at offset (a-1, b-1)
+ *   mlp Wa     : [heads][hidden][d],  Wb : [heads][d][hidden]
+ *   updated weights are returned per unit: [B][heads][...]
+ *
+ * Every routine is written as the definition states it: explicit loops, no blocking, no reordering.
+ * Units are independent; OpenMP only distributes whole units over threads.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_NOMEM 2
+
+/* ------------------------------------------------------------------------------------------ */
+/* Linear inner model f(x) = W x.                                                               */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One unit, per-pair form: grad = (2/N) sum_n (W0 k_n - v_n) k_n^T  (Vision-TTT notes, 关键设计 1,
+ * the gradient G_t summed over all pairs and divided by N); W1 = W0 - eta*grad; z_n = W1 q_n. */
+static int linear_unit_pairs(int N, int d, const double* Q, const double* K, const double* V,
+                             const double* W0, double eta, double* W1, double* Z)
+{
+    double* grad = (double*)calloc((size_t)d * d, sizeof(double));
+    double* r = (double*)malloc((size_t)d * sizeof(double));
+    if (!grad || !r) { free(grad); free(r); return ORACLE_ERR_NOMEM; }
+    for (int n = 0; n < N; ++n) {
+        const double* k = K + (size_t)n * d;
+        const double* v = V + (size_t)n * d;
+        for (int i = 0; i < d; ++i) {           /* residual r = W0 k - v */
+            double s = 0.0;
+            for (int j = 0; j < d; ++j) s += W0[(size_t)i * d + j] * k[j];
+            r[i] = s - v[i];
+        }
+        for (int i = 0; i < d; ++i)             /* grad += r k^T */
+            for (int j = 0; j < d; ++j) grad[(size_t)i * d + j] += r[i] * k[j];
+    }
+    const double scale = 2.0 / (double)N;
+    for (int i = 0; i < d * d; ++i) W1[i] = W0[i] - eta * scale * grad[i];
+    for (int n = 0; n < N; ++n) {                /* readout z = W1 q */
+        const double* q = Q + (size_t)n * d;
+        for (int i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j) s += W1[(size_t)i * d + j] * q[j];
+            Z[(size_t)n * d + i] = s;
+        }
+    }
+    free(grad); free(r);
+    return ORACLE_OK;
+}
+
+/* One unit, Gram form: G = sum_n k_n k_n^T, C = sum_n v_n k_n^T,
+ * W1 = W0 - eta*(2/N)*(W0 G - C).  Algebraically the same step as the per-pair form
+ * (sum_n (W0 k_n - v_n) k_n^T = W0 G - C); kept as a second, independent routine. */
+static int linear_unit_gram(int N, int d, const double* Q, const double* K, const double* V,
+                            const double* W0, double eta, double* W1, double* Z)
+{
+    double* G = (double*)calloc((size_t)d * d, sizeof(double));
+    double* C = (double*)calloc((size_t)d * d, sizeof(double));
+    if (!G || !C) { free(G); free(C); return ORACLE_ERR_NOMEM; }
+    for (int n = 0; n < N; ++n) {
+        const double* k = K + (size_t)n * d;
+        const double* v = V + (size_t)n * d;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) {
+                G[(size_t)i * d + j] += k[i] * k[j];
+                C[(size_t)i * d + j] += v[i] * k[j];
+            }
+    }
+    const double scale = 2.0 / (double)N;
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) {
+            double wg = 0.0;
+            for (int m = 0; m < d; ++m) wg += W0[(size_t)i * d + m] * G[(size_t)m * d + j];
+            W1[(size_t)i * d + j] = W0[(size_t)i * d + j] - eta * scale * (wg - C[(size_t)i * d + j]);
+        }
+    for (int n = 0; n < N; ++n) {
+        const double* q = Q + (size_t)n * d;
+        for (int i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j) s += W1[(size_t)i * d + j] * q[j];
+            Z[(size_t)n * d + i] = s;
+        }
+    }
+    free(G); free(C);
+    return ORACLE_OK;
+}
+
+static int linear_batch(int gram, int B, int heads, int N, int d, const double* Q, const double* K,
+                        const double* V, const double* W0, double eta, double* W1, double* Z,
+                        int nthreads)
+{
+    if (B < 0 || heads < 0 || N < 1 || d < 1 || !Q || !K || !V || !W0 || !W1 || !Z)
+        return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int h = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        int s = gram ? linear_unit_gram(N, d, Q + off, K + off, V + off, W0 + (size_t)h * d * d,
+                                        eta, W1 + (size_t)u * d * d, Z + off)
+                     : linear_unit_pairs(N, d, Q + off, K + off, V + off, W0 + (size_t)h * d * d,
+                                         eta, W1 + (size_t)u * d * d, Z + off);
+        if (s != ORACLE_OK) {
+#pragma omp atomic write
+            status = s;
+        }
+    }
+    return status;
+}
+
+int oracle_linear(int B, int heads, int N, int d, const double* Q, const double* K, const double* V,
+                  const double* W0, double eta, double* W1, double* Z, int nthreads)
+{
+    return linear_batch(0, B, heads, N, d, Q, K, V, W0, eta, W1, Z, nthreads);
+}
+
+int oracle_linear_gram(int B, int heads, int N, int d, const double* Q, const double* K,
+                       const double* V, const double* W0, double eta, double* W1, double* Z,
+                       int nthreads)
+{
+    return linear_batch(1, B, heads, N, d, Q, K, V, W0, eta, W1, Z, nthreads);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* 3x3 depthwise-convolution inner model over the H x W token grid                             */
+/* (press article, Observation 6 and Fig. 5 part 3; ViT3 news article, 原則六 and section      */
+/* 效果全面驗證: one head uses a 3x3 depthwise convolution).                                     */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Value of channel c of a [N][d] token-major map at grid position (y, x); zero outside the grid. */
+static double grid_at(const double* X, int Hg, int Wg, int d, int c, int y, int x)
+{
+    if (y < 0 || y >= Hg || x < 0 || x >= Wg) return 0.0;
+    return X[((size_t)y * Wg + x) * d + c];
+}
+
+/* One unit.  f(X;W)[c,y,x] = sum_{a,b in 0..2} W[c][a][b] * X[c, y+a-1, x+b-1].
+ * r = f(K;W0) - V;  g[c][a][b] = (2/N) sum_{y,x} r[c,y,x] * K[c, y+a-1, x+b-1];
+ * W1 = W0 - eta*g;  Z = f(Q;W1). */
+static int dwconv_unit(int Hg, int Wg, int d, const double* Q, const double* K, const double* V,
+                       const double* W0, double eta, double* W1, double* Z)
+{
+    const int N = Hg * Wg;
+    double* g = (double*)calloc((size_t)d * 9, sizeof(double));
+    if (!g) return ORACLE_ERR_NOMEM;
+    for (int c = 0; c < d; ++c) {
+        const double* w = W0 + (size_t)c * 9;
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double f = 0.0;
+                for (int a = 0; a < 3; ++a)
+                    for (int b = 0; b < 3; ++b)
+                        f += w[a * 3 + b] * grid_at(K, Hg, Wg, d, c, y + a - 1, x + b - 1);
+                const double r = f - V[((size_t)y * Wg + x) * d + c];
+                for (int a = 0; a < 3; ++a)
+                    for (int b = 0; b < 3; ++b)
+                        g[(size_t)c * 9 + a * 3 + b] += r * grid_at(K, Hg, Wg, d, c, y + a - 1, x + b - 1);
+            }
+    }
+    const double scale = 2.0 / (double)N;
+    for (int i = 0; i < d * 9; ++i) W1[i] = W0[i] - eta * scale * g[i];
+    for (int c = 0; c < d; ++c) {
+        const double* w = W1 + (size_t)c * 9;
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double f = 0.0;
+                for (int a = 0; a < 3; ++a)
+                    for (int b = 0; b < 3; ++b)
+                        f += w[a * 3 + b] * grid_at(Q, Hg, Wg, d, c, y + a - 1, x + b - 1);
+                Z[((size_t)y * Wg + x) * d + c] = f;
+            }
+    }
+    free(g);
+    return ORACLE_OK;
+}
+
+int oracle_dwconv(int B, int heads, int Hg, int Wg, int d, const double* Q, const double* K,
+                  const double* V, const double* W0, double eta, double* W1, double* Z, int nthreads)
+{
+    if (B < 0 || heads < 0 || Hg < 1 || Wg < 1 || d < 1 || !Q || !K || !V || !W0 || !W1 || !Z)
+        return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    const size_t N = (size_t)Hg * Wg;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int h = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        int s = dwconv_unit(Hg, Wg, d, Q + off, K + off, V + off, W0 + (size_t)h * d * 9, eta,
+                            W1 + (size_t)u * d * 9, Z + off);
+        if (s != ORACLE_OK) {
+#pragma omp atomic write
+            status = s;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* One-hidden-layer MLP inner model f(x) = Wb * gelu_tanh(Wa * x)                              */
+/* (press article, Observation 4 and Fig. 5 part 1: a 2-layer MLP inner model, width ratio r up */
+/* to 4; ViT3 news article, 原則四: widening d -> 4d).  The activation is GELU (tanh form).     */
+/* ------------------------------------------------------------------------------------------ */
+
+/* GELU, tanh form (Hendrycks & Gimpel, "Gaussian Error Linear Units", the tanh approximation):
+ *   gelu(u) = u/2 * (1 + tanh( sqrt(2/pi) * (u + 0.044715 u^3) )). */
+double oracle_gelu_tanh(double u)
+{
+    const double c = sqrt(2.0 / M_PI);
+    return 0.5 * u * (1.0 + tanh(c * (u + 0.044715 * u * u * u)));
+}
+
+/* Exact derivative of the expression above:
+ *   d/du = 1/2 (1 + t) + u/2 (1 - t^2) * c * (1 + 3*0.044715 u^2),   t = tanh(c (u + 0.044715 u^3)). */
+double oracle_gelu_tanh_deriv(double u)
+{
+    const double c = sqrt(2.0 / M_PI);
+    const double t = tanh(c * (u + 0.044715 * u * u * u));
+    return 0.5 * (1.0 + t) + 0.5 * u * (1.0 - t * t) * c * (1.0 + 3.0 * 0.044715 * u * u);
+}
+
+/* One unit.  With h_n = Wa k_n, a_n = gelu(h_n), y_n = Wb a_n, r_n = y_n - v_n:
+ *   dL/dWb = (2/N) sum_n r_n a_n^T
+ *   dL/dWa = (2/N) sum_n [ (Wb^T r_n) * gelu'(h_n) ] k_n^T      (* = elementwise)
+ *   Wa1 = Wa - eta dL/dWa,  Wb1 = Wb - eta dL/dWb   (both from gradients at the initial weights)
+ *   z_n = Wb1 gelu(Wa1 q_n). */
+static int mlp_unit(int N, int d, int hidden, const double* Q, const double* K, const double* V,
+                    const double* Wa, const double* Wb, double eta, double* Wa1, double* Wb1,
+                    double* Z)
+{
+    double* gA = (double*)calloc((size_t)hidden * d, sizeof(double));
+    double* gB = (double*)calloc((size_t)d * hidden, sizeof(double));
+    double* h = (double*)malloc((size_t)hidden * sizeof(double));
+    double* a = (double*)malloc((size_t)hidden * sizeof(double));
+    double* r = (double*)malloc((size_t)d * sizeof(double));
+    double* dh = (double*)malloc((size_t)hidden * sizeof(double));
+    if (!gA || !gB || !h || !a || !r || !dh) {
+        free(gA); free(gB); free(h); free(a); free(r); free(dh);
+        return ORACLE_ERR_NOMEM;
+    }
+    for (int n = 0; n < N; ++n) {
+        const double* k = K + (size_t)n * d;
+        const double* v = V + (size_t)n * d;
+        for (int j = 0; j < hidden; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < d; ++i) s += Wa[(size_t)j * d + i] * k[i];
+            h[j] = s;
+            a[j] = oracle_gelu_tanh(s);
+        }
+        for (int i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < hidden; ++j) s += Wb[(size_t)i * hidden + j] * a[j];
+            r[i] = s - v[i];
+        }
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < hidden; ++j) gB[(size_t)i * hidden + j] += r[i] * a[j];
+        for (int j = 0; j < hidden; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < d; ++i) s += Wb[(size_t)i * hidden + j] * r[i];
+            dh[j] = s * oracle_gelu_tanh_deriv(h[j]);
+        }
+        for (int j = 0; j < hidden; ++j)
+            for (int i = 0; i < d; ++i) gA[(size_t)j * d + i] += dh[j] * k[i];
+    }
+    const double scale = 2.0 / (double)N;
+    for (int i = 0; i < hidden * d; ++i) Wa1[i] = Wa[i] - eta * scale * gA[i];
+    for (int i = 0; i < d * hidden; ++i) Wb1[i] = Wb[i] - eta * scale * gB[i];
+    for (int n = 0; n < N; ++n) {
+        const double* q = Q + (size_t)n * d;
+        for (int j = 0; j < hidden; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < d; ++i) s += Wa1[(size_t)j * d + i] * q[i];
+            a[j] = oracle_gelu_tanh(s);
+        }
+        for (int i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < hidden; ++j) s += Wb1[(size_t)i * hidden + j] * a[j];
+            Z[(size_t)n * d + i] = s;
+        }
+    }
+    free(gA); free(gB); free(h); free(a); free(r); free(dh);
+    return ORACLE_OK;
+}
+
+int oracle_mlp(int B, int heads, int N, int d, int hidden, const double* Q, const double* K,
+               const double* V, const double* Wa, const double* Wb, double eta, double* Wa1,
+               double* Wb1, double* Z, int nthreads)
+{
+    if (B < 0 || heads < 0 || N < 1 || d < 1 || hidden < 1 || !Q || !K || !V || !Wa || !Wb ||
+        !Wa1 || !Wb1 || !Z)
+        return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int hh = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        const size_t wsz = (size_t)hidden * d;
+        int s = mlp_unit(N, d, hidden, Q + off, K + off, V + off, Wa + hh * wsz, Wb + hh * wsz, eta,
+                         Wa1 + (size_t)u * wsz, Wb1 + (size_t)u * wsz, Z + off);
+        if (s != ORACLE_OK) {
+#pragma omp atomic write
+            status = s;
+        }
+    }
+    return status;
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,347 @@
+"""Pins for the fp64 oracle: each check ties it to something other than itself.
+
+* exact finite differences: the loss is quadratic in the weights of the linear and conv heads, so a
+  central difference computed in rational arithmetic IS the gradient, with no truncation error;
+* closed forms: with orthogonal keys and eta = N / (2 s) the step lands on the least-squares
+  solution (numpy.linalg.lstsq) whatever W0 is;
+* invariants: eta = 0 gives z = f(q; W0); values that the initial model already reproduces give a
+  zero update; the identity conv kernel with V = K reproduces Q;
+* library special cases: torch conv2d(groups=d), torch gelu(approximate="tanh") and torch float64
+  autograd of the pages' L2 loss;
+* planted mistakes (a transposed gradient, a flipped sign, a 1/N instead of 2/N factor, a dropped
+  update) are shown to fail the pins.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+RNG = np.random.default_rng(1234)
+
+
+# ------------------------------------------------------------------------------------------------
+# helpers: the loss as the pages define it (L2 reconstruction over all pairs, mean over tokens)
+# ------------------------------------------------------------------------------------------------
+def _frac_loss_linear(W, K, V):
+    """(1/N) sum_n ||W k_n - v_n||^2 in exact rational arithmetic."""
+    N, d = len(K), len(K[0])
+    tot = Fraction(0)
+    for n in range(N):
+        for i in range(d):
+            r = sum(W[i][j] * K[n][j] for j in range(d)) - V[n][i]
+            tot += r * r
+    return tot / N
+
+
+def _frac_conv(Wc, X, Hg, Wg, c, y, x):
+    s = Fraction(0)
+    for a in range(3):
+        for b in range(3):
+            yy, xx = y + a - 1, x + b - 1
+            if 0 <= yy < Hg and 0 <= xx < Wg:
+                s += Wc[a][b] * X[yy * Wg + xx][c]
+    return s
+
+
+def _frac_loss_conv(W, K, V, Hg, Wg):
+    d = len(K[0])
+    tot = Fraction(0)
+    for c in range(d):
+        for y in range(Hg):
+            for x in range(Wg):
+                r = _frac_conv(W[c], K, Hg, Wg, c, y, x) - V[y * Wg + x][c]
+                tot += r * r
+    return tot / (Hg * Wg)
+
+
+def _small_ints(shape, lo=-3, hi=4):
+    return RNG.integers(lo, hi, size=shape).astype(np.float64)
+
+
+def _torch_conv_f(X, W, Hg, Wg):
+    """Depthwise 3x3 cross-correlation through torch.conv2d: X [N][d] -> [N][d]."""
+    N, d = X.shape
+    img = X.T.reshape(1, d, Hg, Wg)
+    out = F.conv2d(img, W.reshape(d, 1, 3, 3), padding=1, groups=d)
+    return out.reshape(d, N).T
+
+
+# ------------------------------------------------------------------------------------------------
+# linear head
+# ------------------------------------------------------------------------------------------------
+def test_linear_gradient_exact_rational_fd():
+    d, N, eta = 3, 5, 1.0
+    K = _small_ints((N, d)); V = _small_ints((N, d)); W0 = _small_ints((d, d)); Q = _small_ints((N, d))
+    _, W1 = oracle.linear(Q[None, None], K[None, None], V[None, None], W0[None], eta)
+    grad = (W0 - W1[0, 0]) / eta
+    Kf = [[Fraction(int(v)) for v in row] for row in K]
+    Vf = [[Fraction(int(v)) for v in row] for row in V]
+    Wf = [[Fraction(int(v)) for v in row] for row in W0]
+    for i in range(d):
+        for j in range(d):
+            Wp = [r[:] for r in Wf]; Wm = [r[:] for r in Wf]
+            Wp[i][j] += 1; Wm[i][j] -= 1
+            exact = (_frac_loss_linear(Wp, Kf, Vf) - _frac_loss_linear(Wm, Kf, Vf)) / 2
+            assert abs(grad[i, j] - float(exact)) <= 1e-12 * max(1.0, abs(float(exact)))
+
+
+@pytest.mark.parametrize("d,reps", [(8, 2), (16, 3)])
+def test_linear_least_squares_closed_form(d, reps):
+    """K stacked from `reps` orthogonal d x d bases => sum_n k_n k_n^T = reps * I.  With
+    eta = N / (2 reps) the step gives W1 = V^T K / reps, the least-squares minimiser, for any W0."""
+    blocks = [np.linalg.qr(RNG.standard_normal((d, d)))[0] for _ in range(reps)]
+    K = np.concatenate(blocks, axis=0)                      # [N][d]
+    N = K.shape[0]
+    V = RNG.standard_normal((N, d))
+    W0 = RNG.standard_normal((d, d))
+    Q = RNG.standard_normal((N, d))
+    eta = N / (2.0 * reps)
+    _, W1 = oracle.linear(Q[None, None], K[None, None], V[None, None], W0[None], eta)
+    X, *_ = np.linalg.lstsq(K, V, rcond=None)               # K X ~= V, W = X^T
+    np.testing.assert_allclose(W1[0, 0], X.T, atol=1e-12, rtol=0)
+
+
+def test_linear_eta_zero_is_plain_readout():
+    B, H, N, d = 2, 3, 37, 16
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((H, d, d))
+    Z, W1 = oracle.linear(Q, K, V, W0, 0.0)
+    np.testing.assert_array_equal(W1, np.broadcast_to(W0, W1.shape))
+    ref = np.einsum("bhnj,hij->bhni", Q, W0)
+    np.testing.assert_allclose(Z, ref, atol=1e-13, rtol=0)
+
+
+def test_linear_reproduced_values_give_no_update():
+    B, H, N, d = 1, 2, 50, 8
+    Q, K = RNG.standard_normal((B, H, N, d)), RNG.standard_normal((B, H, N, d))
+    W0 = RNG.standard_normal((H, d, d))
+    V = np.einsum("bhnj,hij->bhni", K, W0)                  # v_n = W0 k_n
+    Z, W1 = oracle.linear(Q, K, V, W0, 1.0)
+    np.testing.assert_allclose(W1, np.broadcast_to(W0, W1.shape), atol=1e-13, rtol=0)
+
+
+def test_linear_matches_torch_autograd():
+    B, H, N, d, eta = 2, 2, 29, 12, 0.7
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((H, d, d))
+    Z, W1 = oracle.linear(Q, K, V, W0, eta)
+    for b in range(B):
+        for h in range(H):
+            W = torch.tensor(W0[h], requires_grad=True)
+            Kt, Vt = torch.tensor(K[b, h]), torch.tensor(V[b, h])
+            loss = ((Kt @ W.T - Vt) ** 2).sum(-1).mean()
+            loss.backward()
+            W1_ref = (W - eta * W.grad).detach().numpy()
+            np.testing.assert_allclose(W1[b, h], W1_ref, atol=1e-12, rtol=0)
+            np.testing.assert_allclose(Z[b, h], Q[b, h] @ W1_ref.T, atol=1e-12, rtol=0)
+
+
+def test_linear_gram_form_equals_pair_form():
+    B, H, N, d = 2, 2, 101, 16
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((H, d, d))
+    Z1, W1 = oracle.linear(Q, K, V, W0, 0.9)
+    Z2, W2 = oracle.linear_gram(Q, K, V, W0, 0.9)
+    np.testing.assert_allclose(W1, W2, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(Z1, Z2, atol=1e-11, rtol=0)
+
+
+def _ls_pin_holds(W1_candidate, K, V, reps):
+    X, *_ = np.linalg.lstsq(K, V, rcond=None)
+    return np.allclose(W1_candidate, X.T, atol=1e-9, rtol=0)
+
+
+@pytest.mark.parametrize("mistake", ["transpose", "sign", "one_over_n", "no_update"])
+def test_planted_mistakes_fail_the_linear_pins(mistake):
+    """Plant a plausible mistake in the oracle's result (on the CPU) and check a pin catches it."""
+    d, reps = 8, 2
+    K = np.concatenate([np.linalg.qr(RNG.standard_normal((d, d)))[0] for _ in range(reps)], axis=0)
+    N = K.shape[0]
+    V = RNG.standard_normal((N, d)); W0 = RNG.standard_normal((d, d)); Q = RNG.standard_normal((N, d))
+    eta = N / (2.0 * reps)
+    _, W1 = oracle.linear(Q[None, None], K[None, None], V[None, None], W0[None], eta)
+    W1 = W1[0, 0]
+    assert _ls_pin_holds(W1, K, V, reps)
+    grad = (W0 - W1) / eta
+    bad = {"transpose": W0 - eta * grad.T, "sign": W0 + eta * grad,
+           "one_over_n": W0 - eta * grad / 2, "no_update": W0}[mistake]
+    assert not _ls_pin_holds(bad, K, V, reps)
+
+
+# ------------------------------------------------------------------------------------------------
+# depthwise 3x3 conv head
+# ------------------------------------------------------------------------------------------------
+def test_dwconv_gradient_exact_rational_fd():
+    Hg, Wg, d, eta = 3, 4, 2, 1.0
+    N = Hg * Wg
+    K = _small_ints((N, d)); V = _small_ints((N, d)); Q = _small_ints((N, d))
+    W0 = _small_ints((d, 3, 3))
+    _, W1 = oracle.dwconv(Q[None, None], K[None, None], V[None, None], W0[None], eta, Hg, Wg)
+    grad = (W0 - W1[0, 0]) / eta
+    Kf = [[Fraction(int(v)) for v in row] for row in K]
+    Vf = [[Fraction(int(v)) for v in row] for row in V]
+    Wf = [[[Fraction(int(v)) for v in r] for r in W0[c]] for c in range(d)]
+    for c in range(d):
+        for a in range(3):
+            for b in range(3):
+                Wp = [[r[:] for r in ch] for ch in Wf]; Wm = [[r[:] for r in ch] for ch in Wf]
+                Wp[c][a][b] += 1; Wm[c][a][b] -= 1
+                exact = (_frac_loss_conv(Wp, Kf, Vf, Hg, Wg) - _frac_loss_conv(Wm, Kf, Vf, Hg, Wg)) / 2
+                assert abs(grad[c, a, b] - float(exact)) <= 1e-12 * max(1.0, abs(float(exact)))
+
+
+@pytest.mark.parametrize("Hg,Wg", [(5, 7), (1, 6), (6, 1), (1, 1)])
+def test_dwconv_eta_zero_is_torch_conv2d(Hg, Wg):
+    d = 8
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 2, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((2, d, 3, 3))
+    Z, W1 = oracle.dwconv(Q, K, V, W0, 0.0, Hg, Wg)
+    for h in range(2):
+        ref = _torch_conv_f(torch.tensor(Q[0, h]), torch.tensor(W0[h]), Hg, Wg).numpy()
+        np.testing.assert_allclose(Z[0, h], ref, atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("Hg,Wg", [(6, 5), (1, 9), (4, 1)])
+def test_dwconv_matches_torch_autograd(Hg, Wg):
+    d, eta = 6, 0.5
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, 3, 3))
+    Z, W1 = oracle.dwconv(Q, K, V, W0, eta, Hg, Wg)
+    W = torch.tensor(W0[0], requires_grad=True)
+    r = _torch_conv_f(torch.tensor(K[0, 0]), W, Hg, Wg) - torch.tensor(V[0, 0])
+    loss = (r ** 2).sum(-1).mean()
+    loss.backward()
+    W1_ref = (W - eta * W.grad).detach()
+    np.testing.assert_allclose(W1[0, 0], W1_ref.numpy(), atol=1e-12, rtol=0)
+    Zref = _torch_conv_f(torch.tensor(Q[0, 0]), W1_ref, Hg, Wg).numpy()
+    np.testing.assert_allclose(Z[0, 0], Zref, atol=1e-12, rtol=0)
+
+
+def test_dwconv_identity_kernel_reproduces_queries():
+    Hg, Wg, d = 7, 5, 8
+    N = Hg * Wg
+    Q, K = RNG.standard_normal((2, 1, N, d)), RNG.standard_normal((2, 1, N, d))
+    W0 = np.zeros((1, d, 3, 3)); W0[:, :, 1, 1] = 1.0
+    Z, W1 = oracle.dwconv(Q, K, K.copy(), W0, 1.0, Hg, Wg)
+    np.testing.assert_array_equal(W1, np.broadcast_to(W0, W1.shape))
+    np.testing.assert_array_equal(Z, Q)
+
+
+def test_dwconv_degenerate_grids_zero_out_missing_taps():
+    d = 4
+    Q, K, V = (RNG.standard_normal((1, 1, 1, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, 3, 3))
+    _, W1 = oracle.dwconv(Q, K, V, W0, 1.0, 1, 1)
+    delta = W1[0, 0] - W0[0]
+    mask = np.ones((3, 3), bool); mask[1, 1] = False
+    assert np.all(delta[:, mask] == 0.0) and np.any(delta[:, 1, 1] != 0.0)
+    Q, K, V = (RNG.standard_normal((1, 1, 9, d)) for _ in range(3))
+    _, W1 = oracle.dwconv(Q, K, V, W0, 1.0, 1, 9)           # a single row: no vertical neighbours
+    delta = W1[0, 0] - W0[0]
+    assert np.all(delta[:, 0, :] == 0.0) and np.all(delta[:, 2, :] == 0.0)
+
+
+def test_dwconv_centre_tap_matches_diagonal_linear_gradient():
+    """A kernel with only the centre tap is the diagonal linear map W = diag(w); the centre-tap
+    gradient must equal the diagonal of the linear head's gradient at that W."""
+    Hg, Wg, d, eta = 6, 6, 8, 1.0
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    w = RNG.standard_normal(d)
+    Wc = np.zeros((1, d, 3, 3)); Wc[0, :, 1, 1] = w
+    _, W1c = oracle.dwconv(Q, K, V, Wc, eta, Hg, Wg)
+    _, W1l = oracle.linear(Q, K, V, np.diag(w)[None], eta)
+    np.testing.assert_allclose((Wc[0, :, 1, 1] - W1c[0, 0, :, 1, 1]),
+                               np.diag(np.diag(w) - W1l[0, 0]), atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------------------------------------------
+# MLP head
+# ------------------------------------------------------------------------------------------------
+def test_gelu_tanh_matches_torch():
+    us = np.concatenate([np.linspace(-8, 8, 401), RNG.standard_normal(200) * 3])
+    ut = torch.tensor(us, requires_grad=True)
+    gt = F.gelu(ut, approximate="tanh")
+    gt.sum().backward()
+    for u, g, dg in zip(us, gt.detach().numpy(), ut.grad.numpy()):
+        assert abs(oracle.gelu_tanh(u) - g) <= 1e-14 * max(1.0, abs(g))
+        assert abs(oracle.gelu_tanh_deriv(u) - dg) <= 1e-13
+
+
+def _torch_mlp(X, Wa, Wb):
+    return F.gelu(X @ Wa.T, approximate="tanh") @ Wb.T
+
+
+def test_mlp_eta_zero_is_plain_readout():
+    B, H, N, d, hid = 1, 2, 23, 8, 32
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    Wa, Wb = RNG.standard_normal((H, hid, d)) / 3, RNG.standard_normal((H, d, hid)) / 6
+    Z, Wa1, Wb1 = oracle.mlp(Q, K, V, Wa, Wb, 0.0)
+    for h in range(H):
+        ref = _torch_mlp(torch.tensor(Q[0, h]), torch.tensor(Wa[h]), torch.tensor(Wb[h])).numpy()
+        np.testing.assert_allclose(Z[0, h], ref, atol=1e-13, rtol=0)
+
+
+def test_mlp_matches_torch_autograd():
+    B, H, N, d, hid, eta = 2, 1, 31, 8, 32, 0.5
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    Wa, Wb = RNG.standard_normal((H, hid, d)) / 3, RNG.standard_normal((H, d, hid)) / 6
+    Z, Wa1, Wb1 = oracle.mlp(Q, K, V, Wa, Wb, eta)
+    for b in range(B):
+        A = torch.tensor(Wa[0], requires_grad=True)
+        Bm = torch.tensor(Wb[0], requires_grad=True)
+        r = _torch_mlp(torch.tensor(K[b, 0]), A, Bm) - torch.tensor(V[b, 0])
+        loss = (r ** 2).sum(-1).mean()
+        loss.backward()
+        A1, B1 = (A - eta * A.grad).detach(), (Bm - eta * Bm.grad).detach()
+        np.testing.assert_allclose(Wa1[b, 0], A1.numpy(), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(Wb1[b, 0], B1.numpy(), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(Z[b, 0], _torch_mlp(torch.tensor(Q[b, 0]), A1, B1).numpy(),
+                                   atol=1e-12, rtol=0)
+
+
+def test_mlp_central_differences():
+    N, d, hid, eta = 17, 4, 8, 1.0
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    Wa, Wb = RNG.standard_normal((1, hid, d)) / 2, RNG.standard_normal((1, d, hid)) / 3
+    _, Wa1, Wb1 = oracle.mlp(Q, K, V, Wa, Wb, eta)
+    gA, gB = (Wa[0] - Wa1[0, 0]) / eta, (Wb[0] - Wb1[0, 0]) / eta
+
+    def loss(A, Bm):
+        H = K[0, 0] @ A.T
+        Aact = 0.5 * H * (1 + np.tanh(np.sqrt(2 / np.pi) * (H + 0.044715 * H ** 3)))
+        return np.mean(np.sum((Aact @ Bm.T - V[0, 0]) ** 2, axis=-1))
+
+    h = 1e-6
+    for (i, j) in [(0, 0), (3, 2), (7, 1), (5, 3)]:
+        Ap, Am = Wa[0].copy(), Wa[0].copy(); Ap[i, j] += h; Am[i, j] -= h
+        assert abs((loss(Ap, Wb[0]) - loss(Am, Wb[0])) / (2 * h) - gA[i, j]) < 1e-7
+    for (i, j) in [(0, 0), (2, 7), (3, 4)]:
+        Bp, Bmm = Wb[0].copy(), Wb[0].copy(); Bp[i, j] += h; Bmm[i, j] -= h
+        assert abs((loss(Wa[0], Bp) - loss(Wa[0], Bmm)) / (2 * h) - gB[i, j]) < 1e-7
+
+
+def test_mlp_reproduced_values_give_no_update():
+    N, d, hid = 40, 8, 32
+    Q, K = RNG.standard_normal((1, 1, N, d)), RNG.standard_normal((1, 1, N, d))
+    Wa, Wb = RNG.standard_normal((1, hid, d)) / 3, RNG.standard_normal((1, d, hid)) / 6
+    V = _torch_mlp(torch.tensor(K[0, 0]), torch.tensor(Wa[0]), torch.tensor(Wb[0])).numpy()[None, None]
+    _, Wa1, Wb1 = oracle.mlp(Q, K, V, Wa, Wb, 1.0)
+    np.testing.assert_allclose(Wa1[0], Wa, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(Wb1[0], Wb, atol=1e-13, rtol=0)
+
+
+def test_threads_do_not_change_results():
+    B, H, N, d = 3, 2, 40, 8
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((H, d, d))
+    Z1, W1 = oracle.linear(Q, K, V, W0, 1.0, threads=1)
+    Z4, W4 = oracle.linear(Q, K, V, W0, 1.0, threads=4)
+    np.testing.assert_array_equal(Z1, Z4)
+    np.testing.assert_array_equal(W1, W4)

@@ -1,0 +1,101 @@
+"""Seeded synthetic inputs for the TTT layer forward.
+
+This module only draws random numbers; it holds none of the layer's arithmetic.  Both the CUDA
+path (tests, bench) and the fp64 oracle read the very same tensors produced here.
+
+Recipe (one torch CPU generator, ``manual_seed(seed)``, float32 draws in this order):
+  Q, K, V  : [B][heads][N][d] standard normal; every q and k row (length d) is then divided by its
+             L2 norm (keys and queries are L2-normalised rows, values stay N(0, 1));
+  weights  : linear W0 [heads_lin][d][d] ~ N(0, 1/d); conv W0 [heads_conv][d][3][3] ~ N(0, 1/9);
+             MLP Wa [heads][4d][d] ~ N(0, 1/d), Wb [heads][d][4d] ~ N(0, 1/(4d));
+then Q, K, V are rounded once to the compute dtype (bf16: round-to-nearest-even) and weights stay
+float32.  Token n of a unit sits at grid position (n // W, n % W) (raster order of the 16x16
+patches of the image).
+
+Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
+224^2 -> 14 x 14 = 196, 1248^2 -> 78 x 78 = 6084, 1280^2 -> 80 x 80 = 6400):
+  lin196_fp32      linear, B 1,  1 head, 14 x 14, fp32, eta 1.0
+  lin196_bf16      linear, B 64, 3 heads, 14 x 14, bf16, eta 1.0   (ViT-Tiny-shaped 224^2 layer)
+  mixed6084_bf16   5 linear heads + 1 depthwise-conv head (the last head), B 8, 78 x 78, bf16, eta 0.5
+  lin6400_bf16     linear, B 4, 12 heads, 80 x 80, bf16, eta 1.0   (ViT-Base-shaped 1280^2 layer)
+  mlp1024_bf16     MLP width 4d = 256, GELU(tanh), B 16, 4 heads, 32 x 32, bf16, eta 0.5
+"""
+from dataclasses import dataclass, field
+import math
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    heads: int            # total heads of the layer
+    H: int                # token grid height
+    W: int                # token grid width
+    dtype: str            # "fp32" or "bf16"
+    eta: float
+    kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp"
+    conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
+    d: int = 64
+    hidden_ratio: int = 4
+
+    @property
+    def N(self):
+        return self.H * self.W
+
+    @property
+    def lin_heads(self):
+        return self.heads - self.conv_heads if self.kind in ("linear", "mixed") else 0
+
+    @property
+    def token_heads(self):
+        return self.batch * self.heads * self.N
+
+
+WORKLOADS = {
+    "lin196_fp32": Workload("lin196_fp32", 1, 1, 14, 14, "fp32", 1.0, "linear"),
+    "lin196_bf16": Workload("lin196_bf16", 64, 3, 14, 14, "bf16", 1.0, "linear"),
+    "mixed6084_bf16": Workload("mixed6084_bf16", 8, 6, 78, 78, "bf16", 0.5, "mixed", conv_heads=1),
+    "lin6400_bf16": Workload("lin6400_bf16", 4, 12, 80, 80, "bf16", 1.0, "linear"),
+    "mlp1024_bf16": Workload("mlp1024_bf16", 16, 4, 32, 32, "bf16", 0.5, "mlp"),
+}
+
+TORCH_DTYPE = {"fp32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _unit_rows(x):
+    return x / x.norm(dim=-1, keepdim=True)
+
+
+def make_inputs(w: Workload, seed: int = 0, device="cpu"):
+    """Returns a dict of tensors: Q, K, V (compute dtype) and the fp32 weights of the workload."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (w.batch, w.heads, w.N, w.d)
+    Q = _unit_rows(torch.randn(shape, generator=g, dtype=torch.float32))
+    K = _unit_rows(torch.randn(shape, generator=g, dtype=torch.float32))
+    V = torch.randn(shape, generator=g, dtype=torch.float32)
+    out = {}
+    if w.kind in ("linear", "mixed"):
+        if w.lin_heads:
+            out["W0_lin"] = torch.randn((w.lin_heads, w.d, w.d), generator=g) / math.sqrt(w.d)
+        if w.conv_heads:
+            out["W0_conv"] = torch.randn((w.conv_heads, w.d, 3, 3), generator=g) / 3.0
+    elif w.kind == "mlp":
+        hid = w.hidden_ratio * w.d
+        out["Wa"] = torch.randn((w.heads, hid, w.d), generator=g) / math.sqrt(w.d)
+        out["Wb"] = torch.randn((w.heads, w.d, hid), generator=g) / math.sqrt(hid)
+    dt = TORCH_DTYPE[w.dtype]
+    out["Q"], out["K"], out["V"] = Q.to(dt), K.to(dt), V.to(dt)
+    if device != "cpu":
+        out = {k: v.to(device) for k, v in out.items()}
+    return out
+
+
+def random_unit(batch, heads, H, W, d=64, dtype="bf16", seed=0, kind="linear", conv_heads=0,
+                hidden_ratio=4, eta=1.0):
+    """Inputs for an arbitrary (test) shape with the same distributions."""
+    w = Workload("custom", batch, heads, H, W, dtype, eta, kind, conv_heads=conv_heads, d=d,
+                 hidden_ratio=hidden_ratio)
+    return w, make_inputs(w, seed)
