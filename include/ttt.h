@@ -1,0 +1,142 @@
+/*
+ * ttt.h -- C ABI of libttt.so: the forward pass of the ViT^3 test-time-training (TTT) token-mixing
+ * layer on NVIDIA B200 (sm_100a).
+ *
+ * The operation (one "unit" = one image b and one head h; N = H*W tokens of width d):
+ *   The unit's key/value pairs are a small training set.  An inner model f(.;W) takes ONE
+ *   full-batch, non-causal gradient step of the L2 reconstruction loss over all N pairs,
+ *       L(W)  = (1/N) sum_n || f(k_n; W) - v_n ||^2,        W1 = W0 - eta * dL/dW (W0),
+ *   and every query is read out through the updated model:  z_n = f(q_n; W1).
+ *   Sources, by page title and section:
+ *     "CVPR 2026 Oral | 清華+阿里發布ViT3" (press article): section 序列建模的新視角 (keys and values
+ *       as a dataset, reconstruction by gradient descent, readout on the queries); Observation 2,
+ *       Fig. 3 (one full-batch step, B = N); Observations 4 and 6, Fig. 5 (MLP and depthwise-conv
+ *       inner models).
+ *     "Vision-TTT: Efficient and Expressive Visual Representation Learning with Test-Time
+ *       Training" (paper notes): section 关键设计 1 (L2 loss ||W x_K - x_V||^2, gradient
+ *       2 (W x_K - x_V) x_K^T, readout z = W x_Q, one d x d state per head).
+ *   The gradient is the mean over the N pairs (factor 2/N); the pages print a per-token gradient
+ *   and leave the batch normalisation open.
+ *
+ * Data layout (all entry points):
+ *   Q, K, V, Z   element (b, h, n, c) at  b*batch_stride + h*head_stride + n*d + c   (elements of
+ *                the call's dtype); token n sits at grid position (n / W, n % W).  Rows of d
+ *                features are contiguous; batch_stride and head_stride let one call work on a
+ *                sub-range of heads of a larger [B][heads_total][N][d] buffer.
+ *   Weights are fp32, contiguous, one set per head shared by every image of the batch.
+ *
+ * Conventions:
+ *   - Device pointers only (Q, K, V, weights, Z, workspace, optional outputs); host pointers are
+ *     rejected with TTT_ERR_INVALID_ARG.  The caller owns every buffer; the library never
+ *     allocates, frees or synchronises.  All work is queued on `stream` (a cudaStream_t; NULL =
+ *     the legacy default stream) and the call returns before it completes.
+ *   - Inputs are read-only.  Z must not overlap Q, K or V.
+ *   - Validation is synchronous: on any error nothing is launched.  Errors raised while the
+ *     kernels run are sticky CUDA errors (reported by the next call, or by ttt_last_error), or a
+ *     device-side wait that ran out (reported by ttt_workspace_status).
+ *   - d must be 64.  Q, K, V, Z must be 16-byte aligned and batch_stride, head_stride multiples of
+ *     8 (bf16) or 4 (fp32) elements.
+ *   - The workspace (size from ttt_workspace_bytes) must be zero-filled once after allocation
+ *     (ttt_workspace_init); every successful call leaves it ready for the next one.  Calls that
+ *     may run at the same time need distinct workspaces.
+ *   - Results are deterministic: the same inputs on the same device give bitwise-equal outputs.
+ *   - Arithmetic: bf16 inputs are multiplied exactly and accumulated in fp32; the updated weights
+ *     are formed in fp32 and rounded once to bf16 for the readout; Z is rounded to the input dtype.
+ *     fp32 inputs are computed in fp32 throughout.
+ */
+#ifndef TTT_H
+#define TTT_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TTT_OK = 0,
+    TTT_ERR_INVALID_ARG = 1,   /* null/host pointer, bad size, overlap, non-finite eta */
+    TTT_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement (e.g. d != 64) */
+    TTT_ERR_ALIGNMENT = 3,     /* pointer or stride alignment rule broken */
+    TTT_ERR_WORKSPACE = 4,     /* workspace missing or smaller than ttt_workspace_bytes() */
+    TTT_ERR_CUDA = 5,          /* a CUDA runtime error (launch failure or a sticky earlier error) */
+    TTT_ERR_TIMEOUT = 6        /* a device-side wait gave up (see ttt_workspace_status) */
+} ttt_status;
+
+typedef enum { TTT_FP32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+typedef enum { TTT_HEAD_LINEAR = 0, TTT_HEAD_DWCONV = 1, TTT_HEAD_MLP = 2 } ttt_head_kind;
+
+typedef struct {
+    int batch;               /* images B >= 1 */
+    int heads;               /* heads handled by this call >= 1 */
+    int H, W;                /* token grid; N = H*W >= 1 */
+    int d;                   /* head width; must be 64 */
+    int hidden;              /* MLP hidden width (multiple of 64, <= 256); ignored by other heads */
+    long long batch_stride;  /* elements between consecutive images in Q, K, V, Z */
+    long long head_stride;   /* elements between consecutive heads in Q, K, V, Z */
+    int dtype;               /* ttt_dtype of Q, K, V and Z */
+} ttt_shape;
+
+/* Bytes of device workspace that a call of head kind `kind` with shape `s` needs (0 on an invalid
+ * shape).  Depends only on the shape, not on the device. */
+size_t ttt_workspace_bytes(int kind, const ttt_shape* s);
+
+/* Zero-fill a workspace on `stream` (call once after allocating it). */
+ttt_status ttt_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reports whether a kernel that used `ws` gave up a bounded device-side
+ * wait (TTT_ERR_TIMEOUT, and the flag is cleared) or finished normally (TTT_OK). */
+ttt_status ttt_workspace_status(void* ws, void* stream);
+
+/* Linear inner model f(x) = W x, W in R^{d x d}.
+ *   Computes per unit  G = sum_n k_n k_n^T,  C = sum_n v_n k_n^T   (fp32),
+ *   W1 = W0 - eta * (2/N) * (W0 G - C)   and   z_n = W1 q_n.
+ *   W0:     [heads][d][d] fp32 (W0[i][j] maps input feature j to output feature i).
+ *   W1_out: optional (NULL = not written) [batch][heads][d][d] fp32, the updated weights.
+ */
+ttt_status ttt_forward_linear(const void* Q, const void* K, const void* V, const float* W0,
+                              void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes,
+                              float* W1_out, void* stream);
+
+/* 3x3 depthwise-convolution inner model over the H x W grid (press article, Observation 6 and
+ * Fig. 5 part 3; one head of ViT^3 uses it): cross-correlation, zero padding, stride 1, no bias,
+ * one kernel per feature channel c:
+ *   f(X;W)[c,y,x] = sum_{a,b=0..2} W[c][a][b] X[c, y+a-1, x+b-1].
+ *   r = f(K;W0) - V;  g[c][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c,y+a-1,x+b-1];  W1 = W0 - eta g;
+ *   Z = f(Q;W1).
+ *   W0:     [heads][d][3][3] fp32.   W1_out: optional [batch][heads][d][3][3] fp32.
+ */
+ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const float* W0,
+                              void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes,
+                              float* W1_out, void* stream);
+
+/* One-hidden-layer MLP inner model f(x) = Wb gelu_tanh(Wa x) (press article, Observation 4 and
+ * Fig. 5 part 1: width ratio up to 4), gelu_tanh(u) = u/2 (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3))).
+ * Both matrices take one simultaneous step from the gradients at (Wa, Wb):
+ *   h = Wa k, a = gelu(h), r = Wb a - v,
+ *   Wb1 = Wb - eta (2/N) sum r a^T,   Wa1 = Wa - eta (2/N) sum [(Wb^T r) * gelu'(h)] k^T,
+ *   z = Wb1 gelu(Wa1 q).
+ *   Wa: [heads][hidden][d] fp32,  Wb: [heads][d][hidden] fp32.
+ *   Wa_out / Wb_out: optional [batch][heads][hidden][d] / [batch][heads][d][hidden] fp32.
+ *   bf16 only (fp32 returns TTT_ERR_UNSUPPORTED).
+ */
+ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const float* Wa,
+                           const float* Wb, void* Z, float eta, const ttt_shape* s, void* ws,
+                           size_t ws_bytes, float* Wa_out, float* Wb_out, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* ttt_status_string(ttt_status st);
+
+/* The first asynchronous CUDA error seen by the library in this process, if any (TTT_ERR_CUDA), else
+ * TTT_OK.  Does not synchronise. */
+ttt_status ttt_last_error(void);
+
+/* ABI version (major*100 + minor). */
+int ttt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H */

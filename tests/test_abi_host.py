@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol that
+include/ttt.h declares, sizes workspaces and rejects invalid requests before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vision_test_token_b200 import build, capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return capi.lib()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "ttt.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttt_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_functions()
+    assert declared, "no declarations parsed"
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(capi.EXPORTED) == declared
+
+
+def test_status_strings_and_version(lib):
+    assert capi.status_string(capi.TTT_OK) == "TTT_OK"
+    assert capi.status_string(capi.TTT_ERR_TIMEOUT) == "TTT_ERR_TIMEOUT"
+    assert capi.ttt_version() >= 100
+
+
+def _shape(**kw):
+    base = dict(batch=8, heads=5, H=78, W=78, d=64, batch_stride=6 * 6084 * 64, head_stride=6084 * 64,
+                dtype=capi.TTT_BF16, hidden=0)
+    base.update(kw)
+    return capi.make_shape(**base)
+
+
+def test_workspace_sizes(lib):
+    s = _shape()
+    n = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, s)
+    # header + counters + bf16 W1 per unit + fp32 partial slots: well below the inputs (149 MB)
+    assert 40 * 64 * 64 * 2 < n < 16 << 20
+    assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(d=32)) == 0
+    assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(batch=0)) == 0
+    assert capi.ttt_workspace_bytes(7, s) == 0
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(d=32), capi.TTT_ERR_UNSUPPORTED),
+    (dict(batch=0), capi.TTT_ERR_INVALID_ARG),
+    (dict(H=0), capi.TTT_ERR_INVALID_ARG),
+    (dict(dtype=5), capi.TTT_ERR_INVALID_ARG),
+    (dict(head_stride=100), capi.TTT_ERR_INVALID_ARG),          # heads would overlap
+    (dict(head_stride=6084 * 64 + 4), capi.TTT_ERR_ALIGNMENT),  # not a 16-byte multiple for bf16
+])
+def test_invalid_shapes_are_rejected_before_any_launch(lib, kw, expected):
+    s = _shape(**kw)
+    st = capi.ttt_forward_linear(None, None, None, None, None, 0.5, s, None, 0, None, None)
+    assert st == expected
+
+
+def test_null_pointers_and_workspace(lib):
+    s = _shape()
+    assert capi.ttt_forward_linear(None, None, None, None, None, 0.5, s, None, 0, None, None) == capi.TTT_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(1 << 20)
+    st = capi.ttt_forward_linear(fake, fake, fake, fake, ctypes.c_void_p(1 << 40), 0.5, s, None, 0, None, None)
+    assert st == capi.TTT_ERR_WORKSPACE
+    st = capi.ttt_forward_linear(fake, fake, fake, fake, ctypes.c_void_p(1 << 40), float("nan"), s, fake, 1 << 30,
+                                 None, None)
+    assert st == capi.TTT_ERR_INVALID_ARG
+
+
+def test_mlp_rejects_unsupported_requests(lib):
+    s = _shape(hidden=256, dtype=capi.TTT_FP32)
+    assert capi.ttt_forward_mlp(None, None, None, None, None, None, 0.5, s, None, 0, None, None, None) == \
+        capi.TTT_ERR_UNSUPPORTED
+    s = _shape(hidden=100)
+    assert capi.ttt_forward_mlp(None, None, None, None, None, None, 0.5, s, None, 0, None, None, None) == \
+        capi.TTT_ERR_INVALID_ARG

@@ -1,0 +1,13 @@
+"""vision_test_token_b200 -- B200-native (sm_100a) forward pass of the ViT^3 test-time-training
+(TTT) token-mixing layer.
+
+The compute lives in ``libttt.so`` (CUDA kernels behind the C ABI of ``include/ttt.h``); this
+package holds its ctypes binding (``capi``), torch-facing wrappers (``layer``), the seeded input
+generator (``inputs``) and the build script (``build``).
+"""
+from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
+from .layer import (forward_dwconv, forward_layer, forward_linear, forward_mlp,  # noqa: F401
+                    workspace, workspace_status)
+
+__all__ = ["WORKLOADS", "Workload", "make_inputs", "forward_linear", "forward_dwconv", "forward_mlp",
+           "forward_layer", "workspace", "workspace_status"]

@@ -1,0 +1,114 @@
+"""ctypes binding of libttt.so: the C ABI declared in include/ttt.h, one Python name per C entry
+point, argument marshalling only.  Importing this module loads the in-tree library and fails
+loudly if it is missing or does not export every declared symbol."""
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libttt.so")
+
+TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_ALIGNMENT = 0, 1, 2, 3
+TTT_ERR_WORKSPACE, TTT_ERR_CUDA, TTT_ERR_TIMEOUT = 4, 5, 6
+TTT_FP32, TTT_BF16 = 0, 1
+TTT_HEAD_LINEAR, TTT_HEAD_DWCONV, TTT_HEAD_MLP = 0, 1, 2
+
+# Every symbol that include/ttt.h declares.
+EXPORTED = (
+    "ttt_workspace_bytes", "ttt_workspace_init", "ttt_workspace_status",
+    "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp",
+    "ttt_status_string", "ttt_last_error", "ttt_version",
+)
+
+
+class TttShape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+        ("d", ctypes.c_int), ("hidden", ctypes.c_int),
+        ("batch_stride", ctypes.c_longlong), ("head_stride", ctypes.c_longlong),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+class TttError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libttt.so (once).  Raises if the library was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libttt.so not found at {LIB_PATH}: run `python -m vision_test_token_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i, f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+        fp = ctypes.POINTER(ctypes.c_float)
+        shp = ctypes.POINTER(TttShape)
+        L.ttt_workspace_bytes.argtypes = [i, shp]
+        L.ttt_workspace_bytes.restype = sz
+        L.ttt_workspace_init.argtypes = [vp, sz, vp]
+        L.ttt_workspace_init.restype = i
+        L.ttt_workspace_status.argtypes = [vp, vp]
+        L.ttt_workspace_status.restype = i
+        L.ttt_forward_linear.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
+        L.ttt_forward_linear.restype = i
+        L.ttt_forward_dwconv.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
+        L.ttt_forward_dwconv.restype = i
+        L.ttt_forward_mlp.argtypes = [vp, vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp, vp]
+        L.ttt_forward_mlp.restype = i
+        L.ttt_status_string.argtypes = [i]
+        L.ttt_status_string.restype = ctypes.c_char_p
+        L.ttt_last_error.argtypes = []
+        L.ttt_last_error.restype = i
+        L.ttt_version.argtypes = []
+        L.ttt_version.restype = i
+        for name in EXPORTED:
+            getattr(L, name)
+        _ = fp
+        _lib = L
+    return _lib
+
+
+def status_string(st):
+    return lib().ttt_status_string(int(st)).decode()
+
+
+def make_shape(batch, heads, H, W, d, batch_stride, head_stride, dtype, hidden=0):
+    return TttShape(batch, heads, H, W, d, hidden, batch_stride, head_stride, dtype)
+
+
+def ttt_workspace_bytes(kind, shape):
+    return lib().ttt_workspace_bytes(kind, ctypes.byref(shape))
+
+
+def ttt_workspace_init(ws, nbytes, stream):
+    return lib().ttt_workspace_init(ws, nbytes, stream)
+
+
+def ttt_workspace_status(ws, stream):
+    return lib().ttt_workspace_status(ws, stream)
+
+
+def ttt_forward_linear(Q, K, V, W0, Z, eta, shape, ws, ws_bytes, W1_out, stream):
+    return lib().ttt_forward_linear(Q, K, V, W0, Z, eta, ctypes.byref(shape), ws, ws_bytes, W1_out, stream)
+
+
+def ttt_forward_dwconv(Q, K, V, W0, Z, eta, shape, ws, ws_bytes, W1_out, stream):
+    return lib().ttt_forward_dwconv(Q, K, V, W0, Z, eta, ctypes.byref(shape), ws, ws_bytes, W1_out, stream)
+
+
+def ttt_forward_mlp(Q, K, V, Wa, Wb, Z, eta, shape, ws, ws_bytes, Wa_out, Wb_out, stream):
+    return lib().ttt_forward_mlp(Q, K, V, Wa, Wb, Z, eta, ctypes.byref(shape), ws, ws_bytes, Wa_out, Wb_out,
+                                 stream)
+
+
+def ttt_last_error():
+    return lib().ttt_last_error()
+
+
+def ttt_version():
+    return lib().ttt_version()

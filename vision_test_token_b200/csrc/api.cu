@@ -1,0 +1,259 @@
+// api.cu -- the C ABI of libttt.so (declared in include/ttt.h): argument validation, tensor-map
+// encoding, workspace helpers and error reporting.  The kernels live in linear.cu, dwconv.cu and
+// mlp.cu; nothing here computes.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "ttt_internal.h"
+
+namespace ttt {
+
+static std::atomic<int> g_sticky{0};   // first asynchronous CUDA error seen (as cudaError_t)
+
+ttt_status check_launch(cudaError_t e) {
+    if (e == cudaSuccess) return TTT_OK;
+    int expected = 0;
+    g_sticky.compare_exchange_strong(expected, (int)e);
+    return TTT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime, so no -lcuda is needed)
+// ------------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_tmap_tokens(CUtensorMap* m, const void* base, const Call& c, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const long long esz = 2;   // bf16
+    // Strides of unused dimensions (size 1) still have to be valid multiples of 16 bytes.
+    const long long hs = (c.heads > 1) ? c.hs : (long long)c.N * c.d;
+    const long long bs = (c.batch > 1) ? c.bs : hs * c.heads;
+    cuuint64_t dims[4] = {(cuuint64_t)c.d, (cuuint64_t)c.N, (cuuint64_t)c.heads, (cuuint64_t)c.batch};
+    cuuint64_t strides[3] = {(cuuint64_t)(c.d * esz), (cuuint64_t)(hs * esz), (cuuint64_t)(bs * esz)};
+    cuuint32_t box[4] = {(cuuint32_t)c.d, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Validation
+// ------------------------------------------------------------------------------------------------
+static ttt_status check_shape(int kind, const ttt_shape* s) {
+    if (!s) return TTT_ERR_INVALID_ARG;
+    if (s->batch < 1 || s->heads < 1 || s->H < 1 || s->W < 1 || s->d < 1) return TTT_ERR_INVALID_ARG;
+    if ((long long)s->H * s->W > (1LL << 30)) return TTT_ERR_INVALID_ARG;
+    if (s->dtype != TTT_FP32 && s->dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if (s->batch_stride < 0 || s->head_stride < 0) return TTT_ERR_INVALID_ARG;
+    if ((long long)s->batch * s->heads > (1LL << 24)) return TTT_ERR_INVALID_ARG;
+    if (s->d != 64) return TTT_ERR_UNSUPPORTED;
+    if (kind == TTT_HEAD_MLP) {
+        if (s->hidden < 64 || s->hidden % 64 != 0) return TTT_ERR_INVALID_ARG;
+        if (s->hidden > 256) return TTT_ERR_UNSUPPORTED;
+        if (s->dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+    }
+    const long long N = (long long)s->H * s->W;
+    const long long span = N * s->d;
+    if (s->heads > 1 && s->head_stride < span) return TTT_ERR_INVALID_ARG;          // heads may not overlap
+    if (s->batch > 1 && s->batch_stride < (long long)(s->heads - 1) * s->head_stride + span)
+        return TTT_ERR_INVALID_ARG;                                                   // images may not overlap
+    const int align_elems = (s->dtype == TTT_BF16) ? 8 : 4;                         // 16 bytes
+    if ((s->heads > 1 && s->head_stride % align_elems) || (s->batch > 1 && s->batch_stride % align_elems))
+        return TTT_ERR_ALIGNMENT;
+    return TTT_OK;
+}
+
+static bool is_device_ptr(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();   // clear the non-sticky error
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+static long long extent_bytes(const ttt_shape* s) {   // bytes spanned by one Q/K/V/Z view
+    const long long esz = (s->dtype == TTT_BF16) ? 2 : 4;
+    const long long N = (long long)s->H * s->W;
+    return ((long long)(s->batch - 1) * s->batch_stride + (long long)(s->heads - 1) * s->head_stride + N * s->d) * esz;
+}
+
+static bool overlaps(const void* a, const void* b, long long n) {
+    const char* x = static_cast<const char*>(a);
+    const char* y = static_cast<const char*>(b);
+    return x < y + n && y < x + n;
+}
+
+static ttt_status prepare(int kind, const void* Q, const void* K, const void* V, const float* W0, const float* W0b,
+                          void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, size_t need,
+                          void* stream, Call* c) {
+    ttt_status st = check_shape(kind, s);
+    if (st != TTT_OK) return st;
+    if (!Q || !K || !V || !W0 || !Z || (kind == TTT_HEAD_MLP && !W0b)) return TTT_ERR_INVALID_ARG;
+    if (!std::isfinite(eta)) return TTT_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < need) return TTT_ERR_WORKSPACE;
+    for (const void* p : {Q, K, V, (const void*)Z})
+        if (reinterpret_cast<uintptr_t>(p) % 16) return TTT_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(W0) % 16 || (W0b && reinterpret_cast<uintptr_t>(W0b) % 16) ||
+        reinterpret_cast<uintptr_t>(ws) % 256)
+        return TTT_ERR_ALIGNMENT;
+    const long long ext = extent_bytes(s);
+    if (overlaps(Z, Q, ext) || overlaps(Z, K, ext) || overlaps(Z, V, ext)) return TTT_ERR_INVALID_ARG;
+    for (const void* p : {Q, K, V, (const void*)Z, (const void*)W0, (const void*)ws})
+        if (!is_device_ptr(p)) return TTT_ERR_INVALID_ARG;
+    if (W0b && !is_device_ptr(W0b)) return TTT_ERR_INVALID_ARG;
+
+    int sticky = g_sticky.load();
+    if (sticky != 0) return TTT_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return check_launch(cudaGetLastError());
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return check_launch(cudaGetLastError());
+
+    c->Q = Q; c->K = K; c->V = V; c->Z = Z;
+    c->W0 = W0; c->W0b = W0b;
+    c->W1_out = nullptr; c->W1b_out = nullptr;
+    c->eta = eta;
+    c->batch = s->batch; c->heads = s->heads; c->H = s->H; c->W = s->W;
+    c->N = s->H * s->W; c->d = s->d; c->hidden = s->hidden;
+    c->hs = (s->heads > 1) ? s->head_stride : (long long)c->N * s->d;
+    c->bs = (s->batch > 1) ? s->batch_stride : c->hs * s->heads;
+    c->dtype = s->dtype;
+    c->ws = static_cast<uint8_t*>(ws);
+    c->ws_bytes = ws_bytes;
+    c->stream = static_cast<cudaStream_t>(stream);
+    c->num_sms = sms;
+    return TTT_OK;
+}
+
+}  // namespace ttt
+
+// ------------------------------------------------------------------------------------------------
+// extern "C" entry points
+// ------------------------------------------------------------------------------------------------
+using namespace ttt;
+
+extern "C" {
+
+size_t ttt_workspace_bytes(int kind, const ttt_shape* s) {
+    if (check_shape(kind, s) != TTT_OK) return 0;
+    switch (kind) {
+        case TTT_HEAD_LINEAR: return linear_ws_bytes(*s);
+        case TTT_HEAD_DWCONV: return dwconv_ws_bytes(*s);
+        case TTT_HEAD_MLP: return mlp_ws_bytes(*s);
+        default: return 0;
+    }
+}
+
+ttt_status ttt_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || ws_bytes < kWsHeader) return TTT_ERR_WORKSPACE;
+    if (!is_device_ptr(ws)) return TTT_ERR_INVALID_ARG;
+    return check_launch(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_workspace_status(void* ws, void* stream) {
+    if (!ws) return TTT_ERR_WORKSPACE;
+    if (!is_device_ptr(ws)) return TTT_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return check_launch(e);
+    if (word & kErrTimeout) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyAsync(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return check_launch(e);
+        return TTT_ERR_TIMEOUT;
+    }
+    return TTT_OK;
+}
+
+ttt_status ttt_forward_linear(const void* Q, const void* K, const void* V, const float* W0, void* Z, float eta,
+                              const ttt_shape* s, void* ws, size_t ws_bytes, float* W1_out, void* stream) {
+    Call c;
+    const size_t need = (check_shape(TTT_HEAD_LINEAR, s) == TTT_OK) ? linear_ws_bytes(*s) : 0;
+    ttt_status st = prepare(TTT_HEAD_LINEAR, Q, K, V, W0, nullptr, Z, eta, s, ws, ws_bytes, need, stream, &c);
+    if (st != TTT_OK) return st;
+    if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
+    c.W1_out = W1_out;
+    return launch_linear(c);
+}
+
+ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const float* W0, void* Z, float eta,
+                              const ttt_shape* s, void* ws, size_t ws_bytes, float* W1_out, void* stream) {
+    Call c;
+    const size_t need = (check_shape(TTT_HEAD_DWCONV, s) == TTT_OK) ? dwconv_ws_bytes(*s) : 0;
+    ttt_status st = prepare(TTT_HEAD_DWCONV, Q, K, V, W0, nullptr, Z, eta, s, ws, ws_bytes, need, stream, &c);
+    if (st != TTT_OK) return st;
+    if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
+    c.W1_out = W1_out;
+    return launch_dwconv(c);
+}
+
+ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const float* Wa, const float* Wb, void* Z,
+                           float eta, const ttt_shape* s, void* ws, size_t ws_bytes, float* Wa_out, float* Wb_out,
+                           void* stream) {
+    Call c;
+    const size_t need = (check_shape(TTT_HEAD_MLP, s) == TTT_OK) ? mlp_ws_bytes(*s) : 0;
+    ttt_status st = prepare(TTT_HEAD_MLP, Q, K, V, Wa, Wb, Z, eta, s, ws, ws_bytes, need, stream, &c);
+    if (st != TTT_OK) return st;
+    for (float* o : {Wa_out, Wb_out})
+        if (o && (reinterpret_cast<uintptr_t>(o) % 16 || !is_device_ptr(o))) return TTT_ERR_INVALID_ARG;
+    c.W1_out = Wa_out;
+    c.W1b_out = Wb_out;
+    return launch_mlp(c);
+}
+
+const char* ttt_status_string(ttt_status st) {
+    switch (st) {
+        case TTT_OK: return "TTT_OK";
+        case TTT_ERR_INVALID_ARG: return "TTT_ERR_INVALID_ARG";
+        case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED";
+        case TTT_ERR_ALIGNMENT: return "TTT_ERR_ALIGNMENT";
+        case TTT_ERR_WORKSPACE: return "TTT_ERR_WORKSPACE";
+        case TTT_ERR_CUDA: return "TTT_ERR_CUDA";
+        case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT";
+    }
+    return "TTT_ERR_UNKNOWN";
+}
+
+ttt_status ttt_last_error(void) { return g_sticky.load() ? TTT_ERR_CUDA : TTT_OK; }
+
+int ttt_version(void) { return 100; }
+
+}  // extern "C"

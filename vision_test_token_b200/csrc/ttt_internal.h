@@ -1,0 +1,58 @@
+// ttt_internal.h -- host-side interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ttt.h"
+
+namespace ttt {
+
+// Workspace header: every workspace starts with kWsHeader bytes; word 0 is the device error word.
+constexpr size_t kWsHeader = 256;
+// Bit set in the error word when a bounded device-side wait gave up.
+constexpr uint32_t kErrTimeout = 1u;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Validated, flattened description of one call.
+struct Call {
+    const void* Q;
+    const void* K;
+    const void* V;
+    void* Z;
+    const float* W0;     // linear / conv weights, or MLP Wa
+    const float* W0b;    // MLP Wb
+    float* W1_out;       // linear / conv updated weights, or MLP Wa_out (nullable)
+    float* W1b_out;      // MLP Wb_out (nullable)
+    float eta;
+    int batch, heads, H, W, N, d, hidden;
+    long long bs, hs;    // element strides
+    int dtype;           // ttt_dtype
+    uint8_t* ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+    int num_sms;
+};
+
+// Encodes a rank-4 bf16 tensor map over [batch][heads][N][64] with a 64 x box_rows box,
+// 128-byte swizzle, zero fill out of bounds.  Returns false on failure.
+bool make_tmap_tokens(CUtensorMap* m, const void* base, const Call& c, int box_rows);
+// Rank-2 bf16 tensor map over a contiguous [rows][cols] matrix with a cols x box_rows box (cols*2 = 128).
+bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);
+
+size_t linear_ws_bytes(const ttt_shape& s);
+ttt_status launch_linear(const Call& c);
+
+size_t dwconv_ws_bytes(const ttt_shape& s);
+ttt_status launch_dwconv(const Call& c);
+
+size_t mlp_ws_bytes(const ttt_shape& s);
+ttt_status launch_mlp(const Call& c);
+
+// Records a launch error in the library's sticky error and maps it to a status.
+ttt_status check_launch(cudaError_t e);
+
+}  // namespace ttt

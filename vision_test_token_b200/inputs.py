@@ -20,7 +20,7 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
   lin6400_bf16     linear, B 4, 12 heads, 80 x 80, bf16, eta 1.0   (ViT-Base-shaped 1280^2 layer)
   mlp1024_bf16     MLP width 4d = 256, GELU(tanh), B 16, 4 heads, 32 x 32, bf16, eta 0.5
 """
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 import math
 
 import torch

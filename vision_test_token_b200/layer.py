@@ -1,0 +1,130 @@
+"""Torch-facing wrappers over the C ABI: they take CUDA tensors, check layouts, hand raw device
+pointers and the current stream to libttt.so and raise on any non-OK status.  PyTorch only
+allocates memory and supplies the stream; every step of the layer runs in the library's kernels.
+
+Tensor layout: Q, K, V (and Z) are [B][heads][N][d] views whose last two dimensions are contiguous
+(row stride d, element stride 1); the batch and head strides may be anything the library accepts,
+so a slice of heads of a larger buffer (e.g. ``X[:, :5]``) is passed without a copy.
+"""
+import torch
+
+from . import capi
+
+_DTYPES = {torch.bfloat16: capi.TTT_BF16, torch.float32: capi.TTT_FP32}
+_ws_cache = {}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _shape_of(Q, H, W, hidden=0):
+    if Q.dim() != 4:
+        raise ValueError("Q/K/V must be [B][heads][N][d]")
+    B, heads, N, d = Q.shape
+    if H * W != N:
+        raise ValueError(f"grid {H}x{W} does not match N={N}")
+    if Q.stride(3) != 1 or Q.stride(2) != d:
+        raise ValueError("token rows of Q/K/V/Z must be contiguous")
+    if Q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {Q.dtype}")
+    return capi.make_shape(B, heads, H, W, d, Q.stride(0), Q.stride(1), _DTYPES[Q.dtype], hidden)
+
+
+def _same_layout(ref, *others):
+    for t in others:
+        if t.shape != ref.shape or t.stride() != ref.stride() or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("Q, K, V and Z must share shape, strides, dtype and device")
+
+
+def workspace(kind, shape, device):
+    """A zero-initialised workspace for (kind, shape) on `device`, cached and reused."""
+    nbytes = capi.ttt_workspace_bytes(kind, shape)
+    if nbytes == 0:
+        raise capi.TttError(capi.TTT_ERR_INVALID_ARG, "ttt_workspace_bytes")
+    key = (kind, str(device), nbytes)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _check(st, where):
+    if st != capi.TTT_OK:
+        raise capi.TttError(st, where)
+
+
+def _out_like(Q, Z):
+    if Z is None:
+        Z = torch.empty_like(Q, memory_format=torch.contiguous_format)
+        if Z.stride() != Q.stride():
+            raise ValueError("pass Z explicitly when Q is a strided view")
+    return Z
+
+
+def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None):
+    """Linear inner model.  W0: [heads][d][d] fp32 CUDA tensor.  Returns Z."""
+    shape = _shape_of(Q, H, W)
+    Z = _out_like(Q, Z)
+    _same_layout(Q, K, V, Z)
+    W0 = W0.contiguous()
+    if ws is None:
+        ws = workspace(capi.TTT_HEAD_LINEAR, shape, Q.device)
+    st = capi.ttt_forward_linear(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, _ptr(ws),
+                                 ws.numel(), _ptr(W1_out), _stream_handle(stream))
+    _check(st, "ttt_forward_linear")
+    return Z
+
+
+def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None):
+    """3x3 depthwise-conv inner model.  W0: [heads][d][3][3] fp32 CUDA tensor.  Returns Z."""
+    shape = _shape_of(Q, H, W)
+    Z = _out_like(Q, Z)
+    _same_layout(Q, K, V, Z)
+    W0 = W0.contiguous()
+    if ws is None:
+        ws = workspace(capi.TTT_HEAD_DWCONV, shape, Q.device)
+    st = capi.ttt_forward_dwconv(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, _ptr(ws),
+                                 ws.numel(), _ptr(W1_out), _stream_handle(stream))
+    _check(st, "ttt_forward_dwconv")
+    return Z
+
+
+def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws=None, stream=None):
+    """One-hidden-layer GELU MLP inner model.  Wa: [heads][hidden][d], Wb: [heads][d][hidden]."""
+    shape = _shape_of(Q, H, W, hidden=Wa.shape[1])
+    Z = _out_like(Q, Z)
+    _same_layout(Q, K, V, Z)
+    Wa, Wb = Wa.contiguous(), Wb.contiguous()
+    if ws is None:
+        ws = workspace(capi.TTT_HEAD_MLP, shape, Q.device)
+    st = capi.ttt_forward_mlp(_ptr(Q), _ptr(K), _ptr(V), _ptr(Wa), _ptr(Wb), _ptr(Z), float(eta), shape,
+                              _ptr(ws), ws.numel(), _ptr(Wa_out), _ptr(Wb_out), _stream_handle(stream))
+    _check(st, "ttt_forward_mlp")
+    return Z
+
+
+def forward_layer(Q, K, V, weights, eta, H, W, conv_heads=0, Z=None, ws_lin=None, ws_conv=None, stream=None):
+    """A layer whose first heads are linear and whose last `conv_heads` heads are depthwise-conv
+    heads: two library calls on the same stream over head slices of the same buffers."""
+    Z = _out_like(Q, Z)
+    heads = Q.shape[1]
+    nl = heads - conv_heads
+    if nl:
+        forward_linear(Q[:, :nl], K[:, :nl], V[:, :nl], weights["W0_lin"], eta, H, W, Z=Z[:, :nl], ws=ws_lin,
+                       stream=stream)
+    if conv_heads:
+        forward_dwconv(Q[:, nl:], K[:, nl:], V[:, nl:], weights["W0_conv"], eta, H, W, Z=Z[:, nl:], ws=ws_conv,
+                       stream=stream)
+    return Z
+
+
+def workspace_status(ws, stream=None):
+    """Synchronises and returns the library status recorded in `ws` (TTT_OK or TTT_ERR_TIMEOUT)."""
+    return capi.ttt_workspace_status(_ptr(ws), _stream_handle(stream))
