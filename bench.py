@@ -1,0 +1,445 @@
+"""Benchmark of the TTT-layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one forward of the whole layer over one batch: for the default workload
+(mixed6084_bf16: 8 images x 6 heads x 78x78 = 6084 tokens, d = 64, bf16, eta = 0.5) the five linear
+heads and the depthwise-conv head, i.e. the Gram/cross accumulation, the deterministic merge and
+update, and the readout of every head.  Inputs are synthetic (seeded, the pages' shapes and
+distributions) and already resident in HBM when the timed region starts; three input sets of
+149.5 MB each (more than the 126 MB L2) are rotated so every step reads cold data.  Steps are replayed
+from CUDA graphs (one graph per input set) and timed with CUDA events on the launching stream.
+
+Metric: token*heads per second (B * heads * N per step), whole job over all ranks.  Under torchrun
+every rank runs the same per-GPU workload on its own GPU (weak scaling; no data-path collective).
+
+--impl reference times the fp64 CPU oracle (the only reference implementation there is) on this
+host's cores for the same workload, metric and unit.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from vision_test_token_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "TTT-layer fwd tokens*heads/s at 6084 tokens"
+UNIT = "token*heads/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="mixed6084_bf16", choices=sorted(WORKLOADS))
+    ap.add_argument("--sets", type=int, default=3, help="rotating input sets (total must exceed L2)")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-oracle", action="store_true", help="skip the CPU-oracle baseline leg")
+    return ap.parse_args()
+
+
+def workload_bytes(w):
+    esz = 2 if w.dtype == "bf16" else 4
+    units = w.batch * w.heads
+    return 4 * units * w.N * w.d * esz          # read Q, K, V once, write Z once
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled during the run
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# distributed plumbing
+# ------------------------------------------------------------------------------------------------
+def dist_init(gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+# the CPU oracle leg (cpu_baseline and --impl reference)
+# ------------------------------------------------------------------------------------------------
+def _np64(t):
+    return t.detach().cpu().double().numpy()
+
+
+def oracle_units(w, x, units, threads):
+    """Runs the oracle on the listed (image, head) units of the workload (inputs already float64)."""
+    import oracle
+    if w.kind == "mlp":
+        for (b, h) in units:
+            oracle.mlp(x["Q"][b:b + 1, h:h + 1], x["K"][b:b + 1, h:h + 1], x["V"][b:b + 1, h:h + 1],
+                       x["Wa"][h:h + 1], x["Wb"][h:h + 1], w.eta, threads=threads)
+        return
+    nl = w.lin_heads
+    imgs = sorted({b for b, _ in units})
+    for b in imgs:
+        hs = [h for bb, h in units if bb == b]
+        lin = [h for h in hs if h < nl]
+        conv = [h for h in hs if h >= nl]
+        if lin:
+            lo, hi = min(lin), max(lin) + 1
+            oracle.linear(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
+                          x["W0_lin"][lo:hi], w.eta, threads=threads)
+        if conv:
+            lo, hi = min(conv), max(conv) + 1
+            oracle.dwconv(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
+                          x["W0_conv"][lo - nl:hi - nl], w.eta, w.H, w.W, threads=threads)
+
+
+def oracle_inputs(w, x, images):
+    return {k: _np64(v[:images] if k in ("Q", "K", "V") else v) for k, v in x.items() if k != "Z"}
+
+
+def time_oracle(w, x, budget_s=12.0):
+    """cpu_baseline: whole images of the workload (all heads, OpenMP over units) until budget_s."""
+    import oracle
+    threads = oracle.default_threads()
+    xs = oracle_inputs(w, x, 1)
+    units = [(0, h) for h in range(w.heads)]
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle_units(w, xs, units, threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": len(units) * w.N * reps / el, "unit": UNIT, "cores": min(threads, len(units)),
+            "kind": "oracle",
+            "sample": f"image 0 of {w.name} ({w.heads} heads x {w.N} tokens) repeated {reps} times, "
+                      f"{el:.1f} s, fp64, OpenMP over the {len(units)} (image, head) units"}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle on this host's cores.  One step = one image of the
+    workload (all heads), or one (image, head) unit per step when K whole images would not finish
+    within about two and a half minutes."""
+    import oracle
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    x = oracle_inputs(w, make_inputs(w, seed=0), 1)
+    threads = oracle.default_threads()
+    all_units = [(0, h) for h in range(w.heads)]
+    t0 = time.perf_counter()
+    oracle_units(w, x, all_units, threads)                  # warm-up: one whole image
+    t_img = time.perf_counter() - t0
+    per_image = args.steps * t_img <= 150.0
+    for _ in range(max(0, min(args.warmup, 3) - 1)):
+        oracle_units(w, x, all_units if per_image else all_units[:1], threads)
+    t0 = time.perf_counter()
+    th = 0
+    for i in range(args.steps):
+        units = all_units if per_image else [all_units[i % len(all_units)]]
+        oracle_units(w, x, units, threads)
+        th += len(units) * w.N
+    el = time.perf_counter() - t0
+    value = th / el
+    sample = (f"{'one image (' + str(w.heads) + ' heads)' if per_image else 'one (image, head) unit, heads in turn'}"
+              f" of {w.name} per step, {args.steps} steps, {el:.1f} s, fp64")
+    cb = {"value": value, "unit": UNIT, "kind": "oracle", "cores": min(threads, w.heads if per_image else 1),
+          "sample": sample}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(1, args.steps) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "tokens": w.N, "d": w.d,
+                       "eta": w.eta, "device": "host CPU"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+def make_step(w, xs, dev):
+    """Returns fn(i) running one layer forward on input set i (all device tensors)."""
+    from vision_test_token_b200 import layer
+    weights = {k: v for k, v in xs[0].items() if k.startswith("W")}
+
+    def step(i):
+        x = xs[i]
+        if w.kind == "mlp":
+            layer.forward_mlp(x["Q"], x["K"], x["V"], weights["Wa"], weights["Wb"], w.eta, w.H, w.W, Z=x["Z"])
+        else:
+            layer.forward_layer(x["Q"], x["K"], x["V"], weights, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=x["Z"])
+    return step
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        fn()
+    return g
+
+
+def time_graphs(graphs, steps, stream):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def run_ours(args):
+    world, rank, local = dist_init(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from vision_test_token_b200 import build as _build, capi, layer
+    _build.build()
+    capi.lib()
+    w = WORKLOADS[args.workload]
+    pk = peaks()
+
+    # input sets (seeded per rank and set), Z buffers, workspaces
+    xs = []
+    for s in range(args.sets):
+        x = make_inputs(w, seed=1000 * rank + s, device=dev)
+        x["Z"] = torch.empty_like(x["Q"])
+        xs.append(x)
+    stream = torch.cuda.Stream(device=dev)
+    step = make_step(w, xs, dev)
+    with torch.cuda.stream(stream):
+        for i in range(3):                      # eager warm-up (workspaces, attributes)
+            step(i % args.sets)
+    stream.synchronize()
+    graphs = [capture(lambda i=i: step(i), stream) for i in range(args.sets)]
+
+    # per-call graphs for the roofline of the linear call and the conv call
+    def call_graphs(which):
+        gs = []
+        for i in range(args.sets):
+            x = xs[i]
+            nl = w.lin_heads
+            if which == "linear":
+                fn = lambda x=x, nl=nl: layer.forward_linear(x["Q"][:, :nl], x["K"][:, :nl], x["V"][:, :nl],
+                                                             x["W0_lin"], w.eta, w.H, w.W, Z=x["Z"][:, :nl])
+            else:
+                fn = lambda x=x, nl=nl: layer.forward_dwconv(x["Q"][:, nl:], x["K"][:, nl:], x["V"][:, nl:],
+                                                             x["W0_conv"], w.eta, w.H, w.W, Z=x["Z"][:, nl:])
+            gs.append(capture(fn, stream))
+        return gs
+
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    sampler.start()
+    time.sleep(0.3)
+    # warm-up (graph replays), then the timed region
+    time_graphs(graphs, max(3, args.warmup), stream)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    el = time_graphs(graphs, args.steps, stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    t_wall1 = time.time()
+    el_max = max_over_ranks(el, world, dev)
+    # keep the GPU loaded a little longer so the clock record covers the load
+    if t_wall1 - t_wall0 < 1.0:
+        soak_steps = int(args.steps * (1.2 / max(t_wall1 - t_wall0, 1e-3)))
+        t_wall0 = time.time()
+        time_graphs(graphs, soak_steps, stream)
+        t_wall1 = time.time()
+    time.sleep(0.25)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    ms_per_step = el_max / args.steps * 1e3
+    th_step = w.token_heads
+    value = th_step * world / (el_max / args.steps)
+
+    # roofline: the dominant call, timed alone (events around its graph replays)
+    roof = None
+    if w.kind == "mixed":
+        gl, gc = call_graphs("linear"), call_graphs("conv")
+        n = max(200, args.steps // 4)
+        time_graphs(gl, 20, stream)
+        t_lin = time_graphs(gl, n, stream) / n
+        time_graphs(gc, 20, stream)
+        t_conv = time_graphs(gc, n, stream) / n
+        esz = 2 if w.dtype == "bf16" else 4
+        lin_bytes = 4 * w.batch * w.lin_heads * w.N * w.d * esz
+        conv_bytes = 4 * w.batch * w.conv_heads * w.N * w.d * esz
+        achieved = lin_bytes / t_lin / 1e9
+        roof = {"bound": "hbm", "kernel": "lin_p1_bf16+lin_p2_bf16 (one ttt_forward_linear call)",
+                "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": None, "peak_source": pk["source"],
+                "algorithmic_bytes": lin_bytes, "us_per_launch": t_lin * 1e6,
+                "conv_call": {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
+                              "achieved_gbs": conv_bytes / t_conv / 1e9}}
+
+    # end to end through the public API: pinned host inputs -> device -> layer -> host result
+    e2e = run_e2e(w, xs[0], dev, stream, args.e2e_steps, world)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads,
+                       "lin_heads": w.lin_heads, "conv_heads": w.conv_heads, "grid": [w.H, w.W],
+                       "tokens": w.N, "d": w.d, "eta": w.eta, "parallelism": f"batch-sharded x{world}",
+                       "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",
+                       "algorithmic_bytes_per_step": workload_bytes(w), "launch": "CUDA graph per input set"},
+            "gbs_per_step": workload_bytes(w) / (el_max / args.steps) / 1e9,
+            "gpu_launches": args.steps * (4 if w.kind == "mixed" else 2),
+            "clocks": clocks, "e2e": e2e}
+    if roof:
+        line["roofline"] = roof
+    if rank == 0 and world == 1 and not args.no_oracle:
+        line["cpu_baseline"] = time_oracle(w, xs[0], budget_s=12.0)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.destroy_process_group()
+
+
+def run_e2e(w, x, dev, stream, steps, world):
+    from vision_test_token_b200 import layer
+    names = ["Q", "K", "V"] + sorted(k for k in x if k.startswith("W"))
+    host = {k: x[k].cpu().pin_memory() for k in names}
+    dev_in = {k: torch.empty_like(x[k]) for k in names}
+    z_host = torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory()
+    z_dev = torch.empty_like(x["Q"])
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = z_host.numel() * z_host.element_size()
+
+    def one():
+        for k in names:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        if w.kind == "mlp":
+            layer.forward_mlp(dev_in["Q"], dev_in["K"], dev_in["V"], dev_in["Wa"], dev_in["Wb"], w.eta, w.H, w.W,
+                              Z=z_dev)
+        else:
+            layer.forward_layer(dev_in["Q"], dev_in["K"], dev_in["V"], dev_in, w.eta, w.H, w.W,
+                                conv_heads=w.conv_heads, Z=z_dev)
+        z_host.copy_(z_dev, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            one()
+        b.record(stream)
+    b.synchronize()
+    el = max_over_ranks(a.elapsed_time(b) / 1e3, world, dev)
+    return {"value": w.token_heads * world * steps / el, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": el / steps * 1e3}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
