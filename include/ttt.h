@@ -125,6 +125,26 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
                            const float* Wb, void* Z, float eta, const ttt_shape* s, void* ws,
                            size_t ws_bytes, float* Wa_out, float* Wb_out, void* stream);
 
+/* Linear-head forward without a caller workspace.  The pages have no counterpart of this entry
+ * point: it exists for callers that cannot allocate device memory themselves -- for example a plugin
+ * inside a host framework that hands it only its input and output buffers and owns the allocator,
+ * or code that runs under a fixed, pre-reserved memory budget and must not call cudaMalloc at run
+ * time (cudaMalloc may synchronise the device and has no bounded latency).
+ *   Same arguments, computation, results and errors as ttt_forward_linear, minus (ws, ws_bytes).
+ *   Scratch: an 8 MiB array that the library holds on every device that loads it, until the process
+ *   exits.  Shapes whose ttt_workspace_bytes(TTT_HEAD_LINEAR, s) exceeds 8 MiB are rejected with
+ *   TTT_ERR_WORKSPACE (e.g. 4 images x 12 heads x 6400 tokens needs about 6 MiB).
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture begins.
+ *   Every call on a device shares that device's one array, which keeps the previous call's contents;
+ *   each call clears the words that must start at zero (a cudaMemsetAsync on `stream`) before its
+ *   kernels run.  Calls whose work may overlap on the same GPU (other streams, other host threads)
+ *   race on the array and must be serialised by the caller.
+ *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ */
+ttt_status ttt_forward_linear_noalloc(const void* Q, const void* K, const void* V, const float* W0, void* Z,
+                                      float eta, const ttt_shape* s, float* W1_out, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(ttt_status st);
 

@@ -1,0 +1,51 @@
+"""GPU test of ttt_forward_linear_noalloc, the linear-head entry point for callers that cannot
+allocate device memory (a plugin handed only its input/output buffers, code with a fixed memory
+budget).  It must give the same result as ttt_forward_linear -- within the parity tolerance of the
+other tests -- on two calls in a row, since the second call finds the first call's leftovers in the
+shared scratch array.  The file is named so that pytest collects it last."""
+import pytest
+import torch
+
+from tests.parity import TOL, rel_max_err
+from vision_test_token_b200 import capi, forward_linear
+from vision_test_token_b200.inputs import random_unit
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(x, eta, H, W, dev):
+    Q, K, V = (x[k].to(dev) for k in ("Q", "K", "V"))
+    W0 = x["W0_lin"].to(dev).contiguous()
+    B, h, N, d = Q.shape
+    Z = torch.full_like(Q, float("nan"))
+    W1 = torch.full((B, h, d, d), float("nan"), device=dev)
+    dtype = capi.TTT_BF16 if Q.dtype == torch.bfloat16 else capi.TTT_FP32
+    shape = capi.make_shape(B, h, H, W, d, Q.stride(0), Q.stride(1), dtype)
+    st = capi.ttt_forward_linear_noalloc(Q.data_ptr(), K.data_ptr(), V.data_ptr(), W0.data_ptr(), Z.data_ptr(),
+                                         float(eta), shape, W1.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == capi.TTT_OK, capi.status_string(st)
+    torch.cuda.synchronize()
+    return Z, W1
+
+
+@pytest.mark.parametrize("dtype,B,h,H,W", [("bf16", 4, 5, 78, 78), ("bf16", 3, 2, 20, 25), ("fp32", 1, 1, 14, 14)])
+def test_noalloc_matches_workspace_entry_point_twice(cuda_dev, dtype, B, h, H, W):
+    _, x = random_unit(B, h, H, W, dtype=dtype, seed=B + h + H)
+    eta = 0.5
+    Q, K, V = (x[k].to(cuda_dev) for k in ("Q", "K", "V"))
+    W1_ref = torch.empty((B, h, 64, 64), device=cuda_dev)
+    Z_ref = forward_linear(Q, K, V, x["W0_lin"].to(cuda_dev), eta, H, W, W1_out=W1_ref)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        Z, W1 = _noalloc(x, eta, H, W, cuda_dev)
+        assert rel_max_err(Z, Z_ref.double().cpu().numpy()) <= TOL[dtype]
+        assert rel_max_err(W1, W1_ref.double().cpu().numpy()) <= TOL[dtype]
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_dev):
+    big = torch.zeros(1, device=cuda_dev)
+    p = big.data_ptr()
+    shape = capi.make_shape(64, 12, 80, 80, 64, 12 * 6400 * 64, 6400 * 64, capi.TTT_BF16)
+    assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, shape) > (8 << 20)
+    st = capi.ttt_forward_linear_noalloc(p, p, p, p, p, 0.5, shape, None, torch.cuda.current_stream().cuda_stream)
+    assert st == capi.TTT_ERR_WORKSPACE

@@ -15,7 +15,7 @@ TTT_HEAD_LINEAR, TTT_HEAD_DWCONV, TTT_HEAD_MLP = 0, 1, 2
 # Every symbol that include/ttt.h declares.
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_workspace_init", "ttt_workspace_status",
-    "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp",
+    "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp", "ttt_forward_linear_noalloc",
     "ttt_status_string", "ttt_last_error", "ttt_version",
 )
 
@@ -56,6 +56,8 @@ def lib():
         L.ttt_workspace_status.restype = i
         L.ttt_forward_linear.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
         L.ttt_forward_linear.restype = i
+        L.ttt_forward_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, vp]
+        L.ttt_forward_linear_noalloc.restype = i
         L.ttt_forward_dwconv.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
         L.ttt_forward_dwconv.restype = i
         L.ttt_forward_mlp.argtypes = [vp, vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp, vp]
@@ -95,6 +97,10 @@ def ttt_workspace_status(ws, stream):
 
 def ttt_forward_linear(Q, K, V, W0, Z, eta, shape, ws, ws_bytes, W1_out, stream):
     return lib().ttt_forward_linear(Q, K, V, W0, Z, eta, ctypes.byref(shape), ws, ws_bytes, W1_out, stream)
+
+
+def ttt_forward_linear_noalloc(Q, K, V, W0, Z, eta, shape, W1_out, stream):
+    return lib().ttt_forward_linear_noalloc(Q, K, V, W0, Z, eta, ctypes.byref(shape), W1_out, stream)
 
 
 def ttt_forward_dwconv(Q, K, V, W0, Z, eta, shape, ws, ws_bytes, W1_out, stream):

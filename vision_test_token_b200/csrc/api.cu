@@ -160,6 +160,12 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
     return TTT_OK;
 }
 
+ttt_status validate_call(int kind, const void* Q, const void* K, const void* V, const float* W0, const float* W0b,
+                         void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, size_t need, void* stream) {
+    Call c;
+    return prepare(kind, Q, K, V, W0, W0b, Z, eta, s, ws, ws_bytes, need, stream, &c);
+}
+
 }  // namespace ttt
 
 // ------------------------------------------------------------------------------------------------

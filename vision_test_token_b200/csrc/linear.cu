@@ -754,6 +754,11 @@ size_t linear_ws_bytes(const ttt_shape& s) {
     return lin::ws_layout((long long)s.batch * s.heads, tpu, s.dtype).total;
 }
 
+size_t linear_ws_control_bytes(const ttt_shape& s) {
+    const int tpu = (s.H * s.W + lin::TOK - 1) / lin::TOK;
+    return lin::ws_layout((long long)s.batch * s.heads, tpu, s.dtype).w1;   // error word, queue, counters, flags
+}
+
 ttt_status launch_linear(const Call& c) {
     using namespace lin;
     const long long units = (long long)c.batch * c.heads;

@@ -44,6 +44,9 @@ bool make_tmap_tokens(CUtensorMap* m, const void* base, const Call& c, int box_r
 bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);
 
 size_t linear_ws_bytes(const ttt_shape& s);
+// Bytes at the start of a linear workspace that must be zero before a call (the rest is written
+// before it is read).
+size_t linear_ws_control_bytes(const ttt_shape& s);
 ttt_status launch_linear(const Call& c);
 
 size_t dwconv_ws_bytes(const ttt_shape& s);
@@ -51,6 +54,10 @@ ttt_status launch_dwconv(const Call& c);
 
 size_t mlp_ws_bytes(const ttt_shape& s);
 ttt_status launch_mlp(const Call& c);
+
+// Full synchronous validation of a call (the checks every entry point runs before launching).
+ttt_status validate_call(int kind, const void* Q, const void* K, const void* V, const float* W0, const float* W0b,
+                         void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, size_t need, void* stream);
 
 // Records a launch error in the library's sticky error and maps it to a status.
 ttt_status check_launch(cudaError_t e);
