@@ -133,7 +133,8 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
  *   Same arguments, computation, results and errors as ttt_forward_linear, minus (ws, ws_bytes).
  *   Scratch: an 8 MiB array that the library holds on every device that loads it, until the process
  *   exits.  Shapes whose ttt_workspace_bytes(TTT_HEAD_LINEAR, s) exceeds 8 MiB are rejected with
- *   TTT_ERR_WORKSPACE (e.g. 4 images x 12 heads x 6400 tokens needs about 6 MiB).
+ *   TTT_ERR_WORKSPACE (bf16 calls need only the 256-byte error word; fp32 calls need about
+ *   5 MiB + 48 KiB per (image, head) unit, so fp32 calls above about 60 units are rejected).
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
  *   device current; make that first call before any stream capture begins.
  *   Every call on a device shares that device's one array, which keeps the previous call's contents;

@@ -47,8 +47,12 @@ def _shape(**kw):
 def test_workspace_sizes(lib):
     s = _shape()
     n = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, s)
-    # header + counters + bf16 W1 per unit + fp32 partial slots: well below the inputs (149 MB)
-    assert 40 * 64 * 64 * 2 < n < 16 << 20
+    # bf16 linear: the cluster kernel keeps its intermediates on chip, only the error word remains
+    assert n == 256
+    nf = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(dtype=capi.TTT_FP32, batch_stride=6 * 6084 * 64))
+    assert 40 * 64 * 64 * 4 < nf < 16 << 20           # fp32: counters, W1 and partial slots
+    nc = capi.ttt_workspace_bytes(capi.TTT_HEAD_DWCONV, s)
+    assert nc == 256                                     # conv: the error word only
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(d=32)) == 0
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(batch=0)) == 0
     assert capi.ttt_workspace_bytes(7, s) == 0

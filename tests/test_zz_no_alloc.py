@@ -45,7 +45,7 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_dev, dtype, B, h, H, W
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_dev):
     big = torch.zeros(1, device=cuda_dev)
     p = big.data_ptr()
-    shape = capi.make_shape(64, 12, 80, 80, 64, 12 * 6400 * 64, 6400 * 64, capi.TTT_BF16)
+    shape = capi.make_shape(64, 12, 80, 80, 64, 12 * 6400 * 64, 6400 * 64, capi.TTT_FP32)
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, shape) > (8 << 20)
     st = capi.ttt_forward_linear_noalloc(p, p, p, p, p, 0.5, shape, None, torch.cuda.current_stream().cuda_stream)
     assert st == capi.TTT_ERR_WORKSPACE

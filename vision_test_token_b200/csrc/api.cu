@@ -56,6 +56,23 @@ bool make_tmap_tokens(CUtensorMap* m, const void* base, const Call& c, int box_r
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_grid(CUtensorMap* m, const void* base, const Call& c, int box_cols, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const long long esz = (c.dtype == TTT_BF16) ? 2 : 4;
+    const long long hs = (c.heads > 1) ? c.hs : (long long)c.N * c.d;
+    const long long bs = (c.batch > 1) ? c.bs : hs * c.heads;
+    cuuint64_t dims[5] = {(cuuint64_t)c.d, (cuuint64_t)c.W, (cuuint64_t)c.H, (cuuint64_t)c.heads, (cuuint64_t)c.batch};
+    cuuint64_t strides[4] = {(cuuint64_t)(c.d * esz), (cuuint64_t)((long long)c.W * c.d * esz), (cuuint64_t)(hs * esz),
+                             (cuuint64_t)(bs * esz)};
+    cuuint32_t box[5] = {(cuuint32_t)c.d, (cuuint32_t)box_cols, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(m, (c.dtype == TTT_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;

@@ -3,31 +3,26 @@
 // Oral | 清華+阿里發布ViT3", Observation 2) written in Gram form:
 //     G = sum_n k_n k_n^T,   C = sum_n v_n k_n^T,   W1 = W0 - eta (2/N) (W0 G - C),   z_n = W1 q_n.
 //
-// bf16 path: ONE persistent kernel (lin_fused_bf16), one CTA per SM, that pulls work items from an
-// ordered queue in global memory (an atomic ticket):
-//   items [0, U*C1)          phase 1: chunk j of unit u (TPC1 tiles of 128 tokens).  The chunk's
-//                            [K | V]^T K  (128 x 64 fp32: rows 0..63 = G_j, rows 64..127 = C_j) is
-//                            accumulated in tensor memory; the epilogue forms P_j = W0 G_j - C_j
-//                            and writes it to partial slot (u, j).
-//   items [U*C1, U*(C1+C2))  phase 2: chunk j of unit u (TPC2 Q tiles): Z = Q W1^T.
-// The CTA that completes the last chunk of a unit (atomic arrival count, no waiting) sums the
-// unit's slots in chunk order -- a fixed order, so results are bitwise deterministic whichever CTA
-// ran which chunk -- forms W1 = W0 - eta (2/N) sum_j P_j in fp32, stores it as bf16 and raises the
-// unit's ready flag.  A
-// phase-2 item waits (bounded) for that flag before loading W1.  Every phase-1 item precedes every
-// phase-2 item in the queue, so the CTAs a phase-2 item waits on have claimed their work already
-// and are running; their MMA and epilogue warps never wait on their own producer's later items.
-// Merges therefore overlap the streaming of other units and the phase boundary costs nothing.
-//
-// Roles (192 threads): warp 0 lane 0 claims items and issues TMA loads (128-byte swizzle); warp 1
-// lane 0 issues tcgen05.mma; warps 2..5 drain tensor memory (partial slots, or bf16 Z tiles stored
-// by TMA) and run merges.  Phase 1 uses one MMA stream for G and C: A = [K | V]^T (M = 128,
-// MN-major straight from the token-major tiles), B = K (N = 64, MN-major), K-dim = tokens.
-// Phase 2: A = Q tile (M = 128 tokens, K-major), B = W1 (bf16, K-major).
+// bf16 path (lin_cluster_bf16): one thread-block cluster of CS CTAs (one CTA per SM) per unit.
+//   Phase 1: each CTA of the cluster streams its share of the unit's 128-token K/V tiles (TMA,
+//     128-byte swizzle) and accumulates [K | V]^T K  (128 x 64 fp32: rows 0..63 = G, rows 64..127
+//     = C) in tensor memory with tcgen05.mma: A = [K | V]^T (M = 128, MN-major straight from the
+//     token-major tiles), B = K (N = 64, MN-major), K-dim = tokens.
+//   Exchange: each CTA puts its partial in shared memory and signals its peers through remote
+//     mbarrier arrivals; every CTA then sums the CS partials over distributed shared memory in rank
+//     order (a fixed order: bitwise deterministic) and forms W1 in fp32, rounded once to bf16 into
+//     the shared-memory B operand of phase 2.  No global-memory round trip, no grid-wide wait.
+//   Phase 2: the CTA streams its share of 256-token Q tiles (they are prefetched while the cluster
+//     reduces) and writes Z = Q W1^T: A = Q tile (M = 128 tokens, K-major), B = W1 (K-major), the
+//     epilogue drains tensor memory to bf16 and stores Z with TMA.
+//   Roles (192 threads): warp 0 lane 0 TMA producer, warp 1 lane 0 MMA issuer, warps 2..5 epilogue
+//   and reduction.  CS is chosen so that all clusters are co-resident (units > SMs: CS = 1 and each
+//   CTA loops over units).
 //
 // fp32 path (lin_p1_f32 / lin_p2_f32): plain fp32 FMA kernels (fp32 accuracy), static partition,
 // the same deterministic last-CTA merge.
 #include <algorithm>
+#include <mutex>
 
 #include "sm100.cuh"
 #include "ttt_internal.h"
@@ -38,14 +33,9 @@ namespace lin {
 constexpr int D = 64;
 constexpr int TOK = 128;                    // tokens per tile
 constexpr int TILE_BYTES = TOK * D * 2;     // one bf16 tile: 16 KB
-constexpr int STAGES = 4;                   // 32 KB each: a K+V tile pair or one Q tile
-constexpr int ACC = 4;                      // tensor-memory accumulators of 64 fp32 columns
-constexpr int WQ = 4;                       // work-descriptor ring
-constexpr int TPC1 = 8;                     // tiles per phase-1 chunk
-constexpr int TPC2 = 4;                     // tiles per phase-2 chunk
 constexpr int kPartialFloats = 2 * D * D;   // [G ; C] = 128 x 64
 constexpr int kThreadsTc = 192;
-constexpr int kW0tPitch = D + 4;           // row pitch of the transposed W0 in shared memory
+constexpr int kW0tPitch = D + 4;           // row pitch of the transposed W0 in shared memory (fp32 path)
 constexpr uint32_t kIdescP1 = idesc_bf16_f32(128, 64, true, true);
 constexpr uint32_t kIdescP2 = idesc_bf16_f32(128, 64, false, false);
 
@@ -174,339 +164,339 @@ __device__ void merge_unit(const MergeOut& m, int u, int h, size_t slot0, int ns
 }
 
 // ------------------------------------------------------------------------------------------------
-// Fused-path phase-1 helpers.  The epilogue of every chunk j turns its accumulator [G_j ; C_j] into
-// P_j = W0 G_j - C_j (64 x 64 fp32), so that W1 = W0 - eta (2/N) sum_j P_j and the unit's merge is a
-// plain ordered sum.  gc holds [G_j ; C_j] in shared memory with its 16-byte chunks XOR-swizzled by
-// (row & 15); w0t holds W0 transposed.
+// bf16: one thread-block cluster per unit
 // ------------------------------------------------------------------------------------------------
+constexpr int STAGES = 4;                   // 32 KB each: a K+V tile pair, or one 256-token Q tile
+constexpr int ACC = 4;                      // phase-2 accumulators (64 columns each)
+constexpr int Q2 = 256;                     // tokens per phase-2 stage
+constexpr int kMaxCluster = 3;                // receive slots of the exchange live in the Z staging area
+
+// [G ; C] rows in shared memory: 16-byte chunks XOR-swizzled by (row & 15) against bank conflicts.
 __device__ __forceinline__ float4* gc_chunk(float* gc, int row, int chunk) {
     return reinterpret_cast<float4*>(gc + row * D) + (chunk ^ (row & 15));
 }
 
-// W0 of head h -> w0t[k][i] = W0[i][k]  (128 threads)
-__device__ __forceinline__ void load_w0t(const float* W0, int h, int tid, float* w0t) {
-    float4 wv[8];
-    const float4* W0h = reinterpret_cast<const float4*>(W0 + (size_t)h * D * D);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) wv[i] = __ldg(W0h + i * 128 + tid);
+// Writes 8 bf16 values as 16-byte chunk `chunk` of row `row` of a 128-byte swizzled K-major operand
+// (64 bf16 per row; chunk position XOR (row & 7)).
+__device__ __forceinline__ void put_bf16_chunk(uint8_t* base, int row, int chunk, const float* v) {
+    uint4 pk;
+    pk.x = pack_bf16x2(v[0], v[1]); pk.y = pack_bf16x2(v[2], v[3]);
+    pk.z = pack_bf16x2(v[4], v[5]); pk.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(base + row * 128 + ((chunk ^ (row & 7)) << 4)) = pk;
+}
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): about 16 significant bits in two bf16 numbers.
+__device__ __forceinline__ void split_bf16(const float* x, float* hi, float* lo) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int e = (i * 128 + tid) * 4;
-        const int row = e / D, col = e % D;
-        w0t[(col + 0) * kW0tPitch + row] = wv[i].x;
-        w0t[(col + 1) * kW0tPitch + row] = wv[i].y;
-        w0t[(col + 2) * kW0tPitch + row] = wv[i].z;
-        w0t[(col + 3) * kW0tPitch + row] = wv[i].w;
+        hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+        lo[i] = x[i] - hi[i];
     }
 }
 
-// P = W0 G - C for this thread's 4 x 8 block (rows i0.., columns j0..), written to dst (64 x 64 fp32).
-__device__ __forceinline__ void chunk_product(const float* gc, const float* w0t, int tid, float* dst) {
-    const int i0 = (tid >> 3) * 4, j0 = (tid & 7) * 8;
-    float acc[4][8];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-#pragma unroll 2
-    for (int k = 0; k < D; ++k) {
-        const float4 wk = *reinterpret_cast<const float4*>(w0t + k * kW0tPitch + i0);
-        const float4 g0 = *gc_chunk(const_cast<float*>(gc), k, j0 / 4);
-        const float4 g1 = *gc_chunk(const_cast<float*>(gc), k, j0 / 4 + 1);
-        const float gk[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        const float wr[4] = {wk.x, wk.y, wk.z, wk.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(wr[a], gk[b], acc[a][b]);
-    }
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int i = i0 + a;
-        const float4 c0 = *gc_chunk(const_cast<float*>(gc), D + i, j0 / 4);
-        const float4 c1 = *gc_chunk(const_cast<float*>(gc), D + i, j0 / 4 + 1);
-        float4* out = reinterpret_cast<float4*>(dst + i * D + j0);
-        out[0] = make_float4(acc[a][0] - c0.x, acc[a][1] - c0.y, acc[a][2] - c0.z, acc[a][3] - c0.w);
-        out[1] = make_float4(acc[a][4] - c1.x, acc[a][5] - c1.y, acc[a][6] - c1.z, acc[a][7] - c1.w);
-    }
-}
-
-// Merge of unit u: S = sum_j P_j over the C1 chunk slots in chunk order, W1 = W0 - eta_scale * S.
-__device__ __forceinline__ void merge_chunks(const MergeOut& m, int u, int nslots, const float* slots, int tid,
-                                             const float* w0t) {
-    constexpr int E4 = D * D / 4 / 128;               // 8 float4 per thread
-    float4 acc[E4];
-#pragma unroll
-    for (int i = 0; i < E4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < nslots; s0 += 3) {
-        float4 v[3][E4];
-#pragma unroll
-        for (int b = 0; b < 3; ++b)
-            if (s0 + b < nslots) {
-                const float4* src = reinterpret_cast<const float4*>(slots + (size_t)(s0 + b) * D * D);
-#pragma unroll
-                for (int i = 0; i < E4; ++i) v[b][i] = __ldcg(src + i * 128 + tid);
-            }
-#pragma unroll
-        for (int b = 0; b < 3; ++b)
-            if (s0 + b < nslots) {
-#pragma unroll
-                for (int i = 0; i < E4; ++i) {
-                    acc[i].x += v[b][i].x; acc[i].y += v[b][i].y; acc[i].z += v[b][i].z; acc[i].w += v[b][i].w;
-                }
-            }
-    }
-#pragma unroll
-    for (int i = 0; i < E4; ++i) {
-        const int e = (i * 128 + tid) * 4;
-        const int row = e / D, col = e % D;
-        const float4 w1 = make_float4(w0t[(col + 0) * kW0tPitch + row] - m.eta_scale * acc[i].x,
-                                      w0t[(col + 1) * kW0tPitch + row] - m.eta_scale * acc[i].y,
-                                      w0t[(col + 2) * kW0tPitch + row] - m.eta_scale * acc[i].z,
-                                      w0t[(col + 3) * kW0tPitch + row] - m.eta_scale * acc[i].w);
-        const size_t off = (size_t)u * D * D + e;
-        if (m.W1_out) *reinterpret_cast<float4*>(m.W1_out + off) = w1;
-        uint2 pk;
-        pk.x = pack_bf16x2(w1.x, w1.y);
-        pk.y = pack_bf16x2(w1.z, w1.w);
-        *reinterpret_cast<uint2*>(m.W1_bf16 + off) = pk;
-    }
-}
-
-// ------------------------------------------------------------------------------------------------
-// bf16: the fused persistent kernel
-// ------------------------------------------------------------------------------------------------
-enum : int { W_STOP = 0, W_P1 = 1, W_P2 = 2 };
-struct Work {
-    int kind, u, t0, t1;
-    unsigned item;
-};
-
-struct FusedParams {
-    int heads, tpu, U, C1, C2;
-    unsigned total;             // U * (C1 + C2)
-    MergeOut m;
-    unsigned* counters;         // [U] phase-1 arrivals
-    uint32_t* ready;            // [U] W1 published
-    unsigned* ctrl;             // [0] next item, [1] finished CTAs
+struct ClusterParams {
+    int heads, U, N, CS;        // units, tokens per unit, CTAs per cluster
+    int tpu1, tpu2;             // 128-token tiles and 256-token tiles per unit
+    float eta_scale;            // eta * 2 / N
+    const float* W0;            // [heads][64][64]
+    float* W1_out;              // nullable [units][64][64]
     uint32_t* err;
 };
 
-__device__ __forceinline__ Work decode_work(const FusedParams& p, unsigned item) {
-    Work w;
-    w.item = item;
-    const unsigned n1 = (unsigned)p.U * (unsigned)p.C1;
-    if (item >= p.total) {
-        w.kind = W_STOP; w.u = 0; w.t0 = 0; w.t1 = 0;
-    } else if (item < n1) {
-        w.kind = W_P1;
-        w.u = (int)(item / p.C1);
-        w.t0 = (int)(item % p.C1) * TPC1;
-        w.t1 = min(p.tpu, w.t0 + TPC1);
-    } else {
-        const unsigned k = item - n1;
-        w.kind = W_P2;
-        w.u = (int)(k / p.C2);
-        w.t0 = (int)(k % p.C2) * TPC2;
-        w.t1 = min(p.tpu, w.t0 + TPC2);
-    }
-    return w;
-}
-
-struct FusedSmem {
+struct ClusterSmem {
     uint8_t stage[STAGES][2 * TILE_BYTES];   // 1024-aligned
-    uint8_t zbuf[2][TILE_BYTES];             // Z staging; doubles as the merge's [G ; C] buffer
-    uint8_t w1[2][D * D * 2];
-    float w0[D * kW0tPitch];
+    uint8_t zbuf[2][TILE_BYTES];             // Z staging; doubles as the receive slots of the peers' P
+    uint8_t w1[D * D * 2];                   // W1, bf16, 128-byte swizzled K-major B operand
+    uint8_t a01[2 * D * D * 2];              // [W0_hi ; W0_lo] (bf16 A operand), then D rows 64.. (fp32)
+    float gc[2 * D * D];                     // G as bf16 hi/lo B operands, then C; C rows become P (sent)
     uint64_t full[STAGES], empty[STAGES];
-    uint64_t acc_full[ACC], acc_empty[ACC];
-    uint64_t w_full[2], w_empty[2];
-    uint64_t work_full[WQ], work_empty[WQ];
-    Work wq[WQ];
+    uint64_t pacc_full, pacc_empty;          // phase-1 accumulator
+    uint64_t acc_full[ACC], acc_empty[ACC];  // phase-2 accumulators
+    uint64_t w_full, w_empty;                // W1 in shared memory
+    uint64_t prod_bar;                       // the W0 G product on the tensor cores is done
+    uint64_t recv_full;                      // the peers' P have landed in zbuf (bytes via complete_tx)
+    uint64_t peer_free;                      // every peer has finished the previous unit: its slots are free
     uint32_t tmem_base;
-    int abort_flag, last_flag, done_flag;
+    int abort_flag;
 };
 
-__device__ __forceinline__ void producer(FusedSmem& s, const FusedParams& p, const CUtensorMap* tmK,
-                                         const CUtensorMap* tmV, const CUtensorMap* tmQ, const CUtensorMap* tmW1,
-                                         const Abort& ab) {
-    int wqi = 0; uint32_t wqph = 0;
-    int st = 0; uint32_t stph = 0;
-    int p2n = 0;
-    for (;;) {
-        const unsigned item = atomicAdd(p.ctrl, 1u);
-        const Work w = decode_work(p, item);
-        if (!mbar_wait(&s.work_empty[wqi], wqph ^ 1u, ab)) return;
-        s.wq[wqi] = w;
-        mbar_arrive(&s.work_full[wqi]);
-        if (++wqi == WQ) { wqi = 0; wqph ^= 1u; }
-        if (w.kind == W_STOP) return;
-        const int b = w.u / p.heads, h = w.u % p.heads;
-        if (w.kind == W_P1) {
-            for (int t = w.t0; t < w.t1; ++t) {
-                if (!mbar_wait(&s.empty[st], stph ^ 1u, ab)) return;
-                mbar_arrive_expect_tx(&s.full[st], 2 * TILE_BYTES);
-                tma_load_4d(s.stage[st], tmK, &s.full[st], 0, t * TOK, h, b);
-                tma_load_4d(s.stage[st] + TILE_BYTES, tmV, &s.full[st], 0, t * TOK, h, b);
-                if (++st == STAGES) { st = 0; stph ^= 1u; }
-            }
-        } else {
-            const int wsl = p2n & 1;
-            for (int t = w.t0; t < w.t1; ++t) {
-                if (!mbar_wait(&s.empty[st], stph ^ 1u, ab)) return;
-                mbar_arrive_expect_tx(&s.full[st], TILE_BYTES);
-                tma_load_4d(s.stage[st], tmQ, &s.full[st], 0, t * TOK, h, b);
-                if (++st == STAGES) { st = 0; stph ^= 1u; }
-                if (t == w.t0) {                               // W1 of the unit, once it is published
-                    if (!mbar_wait(&s.w_empty[wsl], (((uint32_t)p2n >> 1) & 1u) ^ 1u, ab)) return;
-                    if (!wait_flag(p.ready + w.u, ab)) return;
-                    fence_proxy_async_global();
-                    mbar_arrive_expect_tx(&s.w_full[wsl], D * D * 2);
-                    tma_load_2d(s.w1[wsl], tmW1, &s.w_full[wsl], 0, w.u * D);
-                }
-            }
-            ++p2n;
+__device__ __forceinline__ int split_lo(int n, int r, int parts) { return (int)((long long)n * r / parts); }
+
+__device__ __forceinline__ void cl_producer(ClusterSmem& s, const ClusterParams& p, const CUtensorMap* tmK,
+                                            const CUtensorMap* tmV, const CUtensorMap* tmQ, int rank, int cid,
+                                            int ncl, const Abort& ab) {
+    int st = 0; uint32_t ph = 0;
+    for (int u = cid; u < p.U; u += ncl) {
+        const int b = u / p.heads, h = u % p.heads;
+        const int t1b = split_lo(p.tpu1, rank, p.CS), t1e = split_lo(p.tpu1, rank + 1, p.CS);
+        for (int t = t1b; t < t1e; ++t) {
+            if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
+            mbar_arrive_expect_tx(&s.full[st], 2 * TILE_BYTES);
+            tma_load_4d(s.stage[st], tmK, &s.full[st], 0, t * TOK, h, b);
+            tma_load_4d(s.stage[st] + TILE_BYTES, tmV, &s.full[st], 0, t * TOK, h, b);
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
+        }
+        // Q does not depend on W1: it streams in while the cluster reduces and forms W1.
+        const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
+        for (int t = t2b; t < t2e; ++t) {
+            if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
+            mbar_arrive_expect_tx(&s.full[st], 2 * TILE_BYTES);
+            tma_load_4d(s.stage[st], tmQ, &s.full[st], 0, t * Q2, h, b);
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
     }
 }
 
-__device__ __forceinline__ void mma_issuer(FusedSmem& s, uint32_t tmem, const Abort& ab) {
-    int wqi = 0; uint32_t wqph = 0;
-    int st = 0; uint32_t stph = 0;
+__device__ __forceinline__ void cl_mma(ClusterSmem& s, const ClusterParams& p, uint32_t tmem, int rank, int cid,
+                                       int ncl, const Abort& ab) {
+    int st = 0; uint32_t ph = 0;
     int ai = 0; uint32_t aph = 0;
-    int p2n = 0;
-    for (;;) {
-        if (!mbar_wait(&s.work_full[wqi], wqph, ab)) return;
-        const Work w = s.wq[wqi];
-        mbar_arrive(&s.work_empty[wqi]);
-        if (++wqi == WQ) { wqi = 0; wqph ^= 1u; }
-        if (w.kind == W_STOP) return;
-        if (w.kind == W_P1) {
-            if (!mbar_wait(&s.acc_empty[ai], aph ^ 1u, ab)) return;
+    uint32_t k = 0;
+    for (int u = cid; u < p.U; u += ncl, ++k) {
+        if (!mbar_wait(&s.pacc_empty, (k & 1u) ^ 1u, ab)) return;
+        tc_fence_after();
+        const int t1b = split_lo(p.tpu1, rank, p.CS), t1e = split_lo(p.tpu1, rank + 1, p.CS);
+        for (int t = t1b; t < t1e; ++t) {
+            if (!mbar_wait(&s.full[st], ph, ab)) return;
             tc_fence_after();
-            const uint32_t dacc = tmem + (uint32_t)(ai * 64);
-            for (int t = w.t0; t < w.t1; ++t) {
-                if (!mbar_wait(&s.full[st], stph, ab)) return;
-                tc_fence_after();
-                const uint32_t sK = smem_u32(s.stage[st]);
+            const uint32_t sK = smem_u32(s.stage[st]);
 #pragma unroll
-                for (int kk = 0; kk < TOK / 16; ++kk) {
-                    // 16 tokens per MMA = two 8-row groups (2 x 1024 bytes); V sits TILE_BYTES after K
-                    const uint64_t ad = sdesc_sw128(sK + kk * 2048, TILE_BYTES, 1024);
-                    const uint64_t bd = sdesc_sw128(sK + kk * 2048, TILE_BYTES, 1024);
-                    mma_bf16_ss(dacc, ad, bd, kIdescP1, (t > w.t0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&s.empty[st]);
-                if (++st == STAGES) { st = 0; stph ^= 1u; }
+            for (int kk = 0; kk < TOK / 16; ++kk) {
+                // 16 tokens per MMA = two 8-row groups (2 x 1024 bytes); V sits TILE_BYTES after K
+                const uint64_t ad = sdesc_sw128(sK + kk * 2048, TILE_BYTES, 1024);
+                const uint64_t bd = sdesc_sw128(sK + kk * 2048, TILE_BYTES, 1024);
+                mma_bf16_ss(tmem, ad, bd, kIdescP1, (t > t1b || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&s.acc_full[ai]);
-            if (++ai == ACC) { ai = 0; aph ^= 1u; }
-        } else {
-            const int wsl = p2n & 1;
-            if (!mbar_wait(&s.w_full[wsl], ((uint32_t)p2n >> 1) & 1u, ab)) return;
-            const uint32_t sW = smem_u32(s.w1[wsl]);
-            for (int t = w.t0; t < w.t1; ++t) {
+            mma_commit(&s.empty[st]);
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
+        }
+        mma_commit(&s.pacc_full);
+        if (!mbar_wait(&s.w_full, k & 1u, ab)) return;
+        tc_fence_after();
+        const uint32_t sW = smem_u32(s.w1);
+        const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
+        for (int t = t2b; t < t2e; ++t) {
+            if (!mbar_wait(&s.full[st], ph, ab)) return;
+            tc_fence_after();
+            for (int hf = 0; hf < 2; ++hf) {
                 if (!mbar_wait(&s.acc_empty[ai], aph ^ 1u, ab)) return;
-                if (!mbar_wait(&s.full[st], stph, ab)) return;
                 tc_fence_after();
-                const uint32_t sQ = smem_u32(s.stage[st]);
+                const uint32_t sQ = smem_u32(s.stage[st]) + hf * TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = sdesc_sw128(sQ + kk * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(sW + kk * 32, 16, 1024);
-                    mma_bf16_ss(tmem + (uint32_t)(ai * 64), ad, bd, kIdescP2, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + 64u + (uint32_t)(ai * 64), ad, bd, kIdescP2, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&s.empty[st]);
                 mma_commit(&s.acc_full[ai]);
-                if (++st == STAGES) { st = 0; stph ^= 1u; }
                 if (++ai == ACC) { ai = 0; aph ^= 1u; }
             }
-            mma_commit(&s.w_empty[wsl]);
-            ++p2n;
+            mma_commit(&s.empty[st]);
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
+        mma_commit(&s.w_empty);
     }
 }
 
-__device__ __forceinline__ void epilogue(FusedSmem& s, const FusedParams& p, uint32_t tmem, const CUtensorMap* tmZ,
-                                         const Abort& ab) {
+__device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams& p, uint32_t tmem,
+                                            const CUtensorMap* tmZ, int rank, int cid, int ncl, const Abort& ab) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;                                   // tensor-memory lane quarter of this warp
-    const int r = q * 32 + lane;                              // row of the accumulator
+    const int r = q * 32 + lane;                              // accumulator row
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    int wqi = 0; uint32_t wqph = 0;
+    const bool multi = p.CS > 1;
     int ai = 0; uint32_t aph = 0;
     int zn = 0;
-    for (;;) {
-        bool ok = mbar_wait(&s.work_full[wqi], wqph, ab);
+    uint32_t k = 0;
+    bool failed = false;
+    for (int u = cid; u < p.U; u += ncl, ++k) {
+        const int b = u / p.heads, h = u % p.heads;
+        // W0 row (tid >> 1), columns c0w .. c0w+31, kept in registers until W1 is formed
+        const int wrow = tid >> 1, c0w = (tid & 1) * 32;
+        float w0r[32];
+        {
+            const float4* src = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + wrow) * D + c0w);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 v = __ldg(src + i);
+                w0r[4 * i] = v.x; w0r[4 * i + 1] = v.y; w0r[4 * i + 2] = v.z; w0r[4 * i + 3] = v.w;
+            }
+        }
+        // (0) my receive slots (the Z staging area) are free once my Z stores have read it: arm the
+        //     receive barrier, then tell the peers they may push
+        if (tid == 0) bulk_wait_read<0>();
+        // A operand of the product: rows 0..63 = bf16(W0), rows 64..127 = bf16(W0 - bf16(W0))
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float hi[8], lo[8];
+            split_bf16(w0r + 8 * c, hi, lo);
+            put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
+            put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
+        }
+        named_bar_sync(1, 128);
+        if (multi && tid == 0) {
+            mbar_arrive_expect_tx(&s.recv_full, (uint32_t)((p.CS - 1) * D * D * 4));
+            for (int pr = 0; pr < p.CS; ++pr)
+                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
+        }
+        // (1) wait for my phase-1 accumulator and for every peer to be done with the previous unit
+        //     (then my earlier pushes have landed and gc may be overwritten)
+        bool ok = mbar_wait(&s.pacc_full, k & 1u, ab);
+        if (multi) ok = ok && mbar_wait_cluster(&s.peer_free, k & 1u, ab);
+        if (named_bar_or(1, 128, !ok)) { failed = true; break; }
         __syncwarp();
-        const Work w = s.wq[wqi];
-        if (named_bar_or(1, 128, !ok || ab.raised())) break;  // uniform decision of the 4 warps
-        if (tid == 0) mbar_arrive(&s.work_empty[wqi]);
-        if (++wqi == WQ) { wqi = 0; wqph ^= 1u; }
-        if (w.kind == W_STOP) break;
-        const int b = w.u / p.heads, h = w.u % p.heads;
-        if (w.kind == W_P1) {
-            load_w0t(p.m.W0, h, tid, s.w0);                  // overlaps the wait for the accumulator
-            ok = mbar_wait(&s.acc_full[ai], aph, ab);
-            if (tid == 0) bulk_wait_read<0>();                // gc aliases the Z staging area
-            if (named_bar_or(1, 128, !ok)) break;
-            __syncwarp();
+        tc_fence_after();
+        // (2) accumulator rows -> G as bf16 hi/lo B operands (rows r < 64) and C in fp32 (rows 64..)
+        uint8_t* bhi = reinterpret_cast<uint8_t*>(s.gc);
+        uint8_t* blo = bhi + D * D * 2;
+        const bool has_p1 = split_lo(p.tpu1, rank + 1, p.CS) > split_lo(p.tpu1, rank, p.CS);
+        {
+            float v[4][16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + (uint32_t)(j * 16) + lane_off, v[j]);
+            tmem_ld_wait();
+            if (!has_p1) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[j][e] = 0.f;
+            }
+            if (r < D) {                                      // G is symmetric: row r of G = column r
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float hi[8], lo[8];
+                    split_bf16(&v[c / 2][(c & 1) * 8], hi, lo);
+                    put_bf16_chunk(bhi, r, c, hi);
+                    put_bf16_chunk(blo, r, c, lo);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *gc_chunk(s.gc, r, (j * 16 + e) / 4) = make_float4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&s.pacc_empty);
+        fence_proxy_async_smem();                             // the operands are read by the tensor cores
+        named_bar_sync(1, 128);
+        // (3) D = [W0_hi ; W0_lo] (G_hi + G_lo) on the tensor cores (M = 128, N = 64, K = 64 twice)
+        if (tid == 0) {
             tc_fence_after();
-            float* gc = reinterpret_cast<float*>(s.zbuf[0]);
+            const uint32_t sa = smem_u32(s.a01), sh = smem_u32(bhi), sl = smem_u32(blo);
 #pragma unroll
-            for (int j = 0; j < D; j += 16) {
-                float v[16];
-                tmem_ld16(tmem + (uint32_t)(ai * 64 + j) + lane_off, v);
-                tmem_ld_wait();
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sh + kk * 32, 16, 1024),
+                            kIdescP2, kk > 0 ? 1u : 0u);
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) *gc_chunk(gc, r, (j + e) / 4) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            }
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sl + kk * 32, 16, 1024),
+                            kIdescP2, 1u);
+            mma_commit(&s.prod_bar);
+        }
+        ok = mbar_wait(&s.prod_bar, k & 1u, ab);
+        if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+        __syncwarp();
+        tc_fence_after();
+        // (4) P = D[0:64] + D[64:128] - C  (= W0 G - C), written over the C rows of gc
+        float* dlo = reinterpret_cast<float*>(s.a01);          // the A operand is consumed: reuse it
+        {
+            float v[4][16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 320u + (uint32_t)(j * 16) + lane_off, v[j]);
+            tmem_ld_wait();
             tc_fence_before();
-            mbar_arrive(&s.acc_empty[ai]);
-            if (++ai == ACC) { ai = 0; aph ^= 1u; }
-            named_bar_sync(1, 128);
-            chunk_product(gc, s.w0, tid, const_cast<float*>(p.m.partials) + (size_t)w.item * D * D);
-            __threadfence();
-            named_bar_sync(1, 128);
-            if (tid == 0) {
-                const unsigned old = atomicAdd(p.counters + w.u, 1u);
-                s.last_flag = (old + 1u == (unsigned)p.C1) ? 1 : 0;
+            if (r >= D) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *gc_chunk(dlo, r - D, (j * 16 + e) / 4) = make_float4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
             }
             named_bar_sync(1, 128);
-            if (s.last_flag) {
-                __threadfence();
-                merge_chunks(p.m, w.u, p.C1, p.m.partials + (size_t)w.u * p.C1 * D * D, tid, s.w0);
-                fence_proxy_async_global();                   // W1 is read next by TMA (async proxy)
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (tid == 0) {
-                    p.counters[w.u] = 0u;
-                    st_release_gpu(p.ready + w.u, 1u);
+            if (r < D) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4) {
+                        const int c = (j * 16 + e) / 4;
+                        const float4 l = *gc_chunk(dlo, r, c);
+                        float4* cp = gc_chunk(s.gc, D + r, c);
+                        const float4 cv = *cp;
+                        *cp = make_float4(v[j][e] + l.x - cv.x, v[j][e + 1] + l.y - cv.y, v[j][e + 2] + l.z - cv.z,
+                                          v[j][e + 3] + l.w - cv.w);
+                    }
+            }
+        }
+        const float* Pme = s.gc + D * D;                      // rows 64..127 of gc
+        // (5) push P to every peer (bulk copies into the peers' receive slots), then wait for theirs
+        if (multi) {
+            fence_proxy_async_smem();                         // P is read next by the bulk-copy engine
+            named_bar_sync(1, 128);
+            if (tid == 0)
+                for (int pr = 0; pr < p.CS; ++pr) {
+                    if (pr == rank) continue;
+                    const int slot = (rank < pr) ? rank : rank - 1;   // my slot in the peer's receive area
+                    bulk_s2cluster(map_to_rank(smem_u32(s.zbuf[slot]), (uint32_t)pr), Pme, D * D * 4,
+                                   map_to_rank(smem_u32(&s.recv_full), (uint32_t)pr));
+                }
+            ok = mbar_wait_cluster(&s.recv_full, k & 1u, ab);
+        } else {
+            named_bar_sync(1, 128);
+        }
+        // (6) W1 = W0 - eta (2/N) sum_r P_r  (ranks in order: deterministic); W1_out from rank 0
+        ok = ok && mbar_wait(&s.w_empty, (k & 1u) ^ 1u, ab);  // phase 2 of the previous unit is done with w1
+        if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+        {
+            float sum[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sum[e] = 0.f;
+            for (int pr = 0; pr < p.CS; ++pr) {
+                float* src = (pr == rank) ? const_cast<float*>(Pme)
+                                          : reinterpret_cast<float*>(s.zbuf[(pr < rank) ? pr : pr - 1]);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float4 v = *gc_chunk(src, wrow, c0w / 4 + c);
+                    sum[4 * c] += v.x; sum[4 * c + 1] += v.y; sum[4 * c + 2] += v.z; sum[4 * c + 3] += v.w;
                 }
             }
-            named_bar_sync(1, 128);
-        } else {
-            bool fail = false;
-            for (int t = w.t0; t < w.t1; ++t) {
+            float w1[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w1[e] = w0r[e] - p.eta_scale * sum[e];
+            if (p.W1_out && rank == 0) {
+                float4* o = reinterpret_cast<float4*>(p.W1_out + ((size_t)u * D + wrow) * D + c0w);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) o[c] = make_float4(w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) put_bf16_chunk(s.w1, wrow, c0w / 8 + c, w1 + 8 * c);
+        }
+        fence_proxy_async_smem();                             // w1 is read next by the tensor cores
+        named_bar_sync(1, 128);
+        if (tid == 0) mbar_arrive(&s.w_full);
+        // (5) phase 2: Z tiles
+        const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
+        for (int t = t2b; t < t2e && !failed; ++t) {
+            for (int hf = 0; hf < 2; ++hf) {
                 ok = mbar_wait(&s.acc_full[ai], aph, ab);
                 const int zb = zn & 1;
                 if (tid == 0 && zn >= 2) bulk_wait_read<1>();  // staging buffer zb is free again
-                if (named_bar_or(1, 128, !ok)) { fail = true; break; }
+                if (named_bar_or(1, 128, !ok)) { failed = true; break; }
                 __syncwarp();
                 tc_fence_after();
                 uint8_t* zrow = s.zbuf[zb] + r * 128;
 #pragma unroll
                 for (int j = 0; j < D; j += 16) {
                     float v[16];
-                    tmem_ld16(tmem + (uint32_t)(ai * 64 + j) + lane_off, v);
+                    tmem_ld16(tmem + 64u + (uint32_t)(ai * 64 + j) + lane_off, v);
                     tmem_ld_wait();
                     uint4 lo, hi;
                     lo.x = pack_bf16x2(v[0], v[1]);   lo.y = pack_bf16x2(v[2], v[3]);
                     lo.z = pack_bf16x2(v[4], v[5]);   lo.w = pack_bf16x2(v[6], v[7]);
                     hi.x = pack_bf16x2(v[8], v[9]);   hi.y = pack_bf16x2(v[10], v[11]);
                     hi.z = pack_bf16x2(v[12], v[13]); hi.w = pack_bf16x2(v[14], v[15]);
-                    const int c0 = j / 8;                         // 16-byte chunk of columns j..j+7
+                    const int c0 = j / 8;                          // 16-byte chunk of columns j..j+7
                     *reinterpret_cast<uint4*>(zrow + ((c0 ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(zrow + (((c0 + 1) ^ (r & 7)) << 4)) = hi;
                 }
@@ -515,48 +505,67 @@ __device__ __forceinline__ void epilogue(FusedSmem& s, const FusedParams& p, uin
                 if (++ai == ACC) { ai = 0; aph ^= 1u; }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
-                if (tid == 0) {
-                    tma_store_4d(tmZ, s.zbuf[zb], 0, t * TOK, h, b);
+                const int row0 = t * Q2 + hf * TOK;
+                if (tid == 0 && row0 < p.N) {
+                    tma_store_4d(tmZ, s.zbuf[zb], 0, row0, h, b);
                     bulk_commit();
                 }
                 ++zn;
             }
-            if (fail) break;
         }
+        if (failed) break;
+    }
+    // Final handshake: once every peer has finished its last unit, all pushes from this CTA have
+    // landed and nobody will push into it again; only then may it exit.
+    if (multi && !failed) {
+        named_bar_sync(1, 128);
+        if (tid == 0)
+            for (int pr = 0; pr < p.CS; ++pr)
+                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
+        mbar_wait_cluster(&s.peer_free, k & 1u, ab);
     }
     if (tid == 0) bulk_wait<0>();
 }
 
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kThreadsTc, 1)
-lin_fused_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmZ,
-               const __grid_constant__ CUtensorMap tmW1, const FusedParams p) {
+lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmZ,
+                 const ClusterParams p) {
     extern __shared__ uint8_t smem_raw[];
-    FusedSmem& s = *reinterpret_cast<FusedSmem*>(align1024(smem_raw));
+    ClusterSmem& s = *reinterpret_cast<ClusterSmem*>(align1024(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)cluster_ctarank(), cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
     const Abort ab{&s.abort_flag, p.err};
 
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
         for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        mbar_init(&s.pacc_full, 1); mbar_init(&s.pacc_empty, 128);
         for (int i = 0; i < ACC; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&s.w_full[i], 1); mbar_init(&s.w_empty[i], 1); }
-        for (int i = 0; i < WQ; ++i) { mbar_init(&s.work_full[i], 1); mbar_init(&s.work_empty[i], 2); }
+        mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
+        mbar_init(&s.prod_bar, 1);
+        mbar_init(&s.recv_full, 1);
+        mbar_init(&s.peer_free, (uint32_t)(p.CS > 1 ? p.CS - 1 : 1));
         fence_barrier_init();
-        prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmZ); prefetch_tmap(&tmW1);
+        prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
     }
-    if (warp == 1) { tmem_alloc(&s.tmem_base, 256); tmem_relinquish(); }
+    if (warp == 1) { tmem_alloc(&s.tmem_base, 512); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    cluster_sync_all();                  // every CTA's barriers exist before any peer arrives on them
     const uint32_t tmem = s.tmem_base;
 
     if (warp == 0) {
-        if (lane == 0) producer(s, p, &tmK, &tmV, &tmQ, &tmW1, ab);
+        if (lane == 0) cl_producer(s, p, &tmK, &tmV, &tmQ, rank, cid, ncl, ab);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(s, tmem, ab);
+        if (lane == 0) cl_mma(s, p, tmem, rank, cid, ncl, ab);
     } else {
-        epilogue(s, p, tmem, &tmZ, ab);
+        cl_epilogue(s, p, tmem, &tmZ, rank, cid, ncl, ab);
     }
 
     tc_fence_before();
@@ -564,19 +573,7 @@ lin_fused_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
-    }
-    // The last CTA to finish re-arms the queue and the ready flags for the next call.
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned old = atomicAdd(p.ctrl + 1, 1u);
-        s.done_flag = (old + 1u == gridDim.x) ? 1 : 0;
-    }
-    __syncthreads();
-    if (s.done_flag) {
-        __threadfence();
-        for (int u = threadIdx.x; u < p.U; u += blockDim.x) p.ready[u] = 0u;
-        if (threadIdx.x == 0) { p.ctrl[0] = 0u; p.ctrl[1] = 0u; }
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -730,75 +727,114 @@ lin_p2_f32(TokenView Qv, float* Z, long long zbs, long long zhs, const float* W1
 constexpr int kMaxGridF32 = 160;
 
 struct WsLayout {
-    size_t ctrl, counters, ready, w1, partials, total;
+    size_t counters, w1, partials, total;
 };
 
-static WsLayout ws_layout(long long units, int tpu, int dtype) {
+// bf16: the cluster kernel keeps all intermediates on chip; its workspace is the error word only.
+// fp32: counters, W1 and the per-CTA [G ; C] partial slots of the two-kernel path.
+static WsLayout ws_layout(long long units, int dtype) {
     WsLayout L;
-    L.ctrl = kWsHeader;
-    L.counters = L.ctrl + 256;
-    L.ready = align_up(L.counters + (size_t)units * sizeof(unsigned), 256);
-    L.w1 = align_up(L.ready + (size_t)units * sizeof(unsigned), 1024);
-    const size_t w1_elem = (dtype == TTT_BF16) ? 2 : 4;
-    L.partials = align_up(L.w1 + (size_t)units * D * D * w1_elem, 1024);
-    const long long slots = (dtype == TTT_BF16) ? units * ((tpu + TPC1 - 1) / TPC1) : kMaxGridF32 + units;
-    const size_t slot_floats = (dtype == TTT_BF16) ? (size_t)D * D : (size_t)kPartialFloats;   // P_j, or [G ; C]
-    L.total = L.partials + (size_t)slots * slot_floats * sizeof(float);
+    if (dtype == TTT_BF16) {
+        L.counters = L.w1 = L.partials = L.total = kWsHeader;
+        return L;
+    }
+    L.counters = kWsHeader;
+    L.w1 = align_up(L.counters + (size_t)units * sizeof(unsigned), 1024);
+    L.partials = align_up(L.w1 + (size_t)units * D * D * sizeof(float), 1024);
+    L.total = L.partials + (size_t)(kMaxGridF32 + units) * kPartialFloats * sizeof(float);
     return L;
+}
+
+// Largest number of co-resident clusters of `cs` CTAs of the cluster kernel (cached per device).
+static int max_active_clusters(int cs, size_t smem) {
+    static std::mutex mu;
+    static int cache[64][kMaxCluster + 1];
+    static bool init = false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) { cudaGetLastError(); return 0; }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!init) {
+        for (auto& row : cache)
+            for (int& v : row) v = -1;
+        init = true;
+    }
+    if (cache[dev][cs] < 0) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(cs * 64);
+        cfg.blockDim = dim3(kThreadsTc);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = cs; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, (void*)lin_cluster_bf16, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev][cs] = n;
+    }
+    return cache[dev][cs];
 }
 
 }  // namespace lin
 
 size_t linear_ws_bytes(const ttt_shape& s) {
-    const int tpu = (s.H * s.W + lin::TOK - 1) / lin::TOK;
-    return lin::ws_layout((long long)s.batch * s.heads, tpu, s.dtype).total;
+    return lin::ws_layout((long long)s.batch * s.heads, s.dtype).total;
 }
 
 size_t linear_ws_control_bytes(const ttt_shape& s) {
-    const int tpu = (s.H * s.W + lin::TOK - 1) / lin::TOK;
-    return lin::ws_layout((long long)s.batch * s.heads, tpu, s.dtype).w1;   // error word, queue, counters, flags
+    return lin::ws_layout((long long)s.batch * s.heads, s.dtype).w1;   // error word (and fp32 counters)
 }
 
 ttt_status launch_linear(const Call& c) {
     using namespace lin;
     const long long units = (long long)c.batch * c.heads;
     const int tpu = (c.N + TOK - 1) / TOK;
-    const WsLayout L = ws_layout(units, tpu, c.dtype);
+    const WsLayout L = ws_layout(units, c.dtype);
+
+    if (c.dtype == TTT_BF16) {
+        const size_t smem = sizeof(ClusterSmem) + 1024;
+        cudaFuncSetAttribute(lin_cluster_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        // CTAs per cluster: spread each unit over up to kMaxCluster SMs while every cluster stays
+        // co-resident (clusters never wait on one another, but a second wave would double the time).
+        int cs = (int)std::max<long long>(1, std::min<long long>(kMaxCluster, c.num_sms / std::max<long long>(1, units)));
+        while (cs > 1 && max_active_clusters(cs, smem) < (int)std::min<long long>(units, c.num_sms / cs)) --cs;
+        const int ncl = (int)std::min<long long>(units, cs == 1 ? c.num_sms : c.num_sms / cs);
+        ClusterParams p{};
+        p.heads = c.heads;
+        p.U = (int)units;
+        p.N = c.N;
+        p.CS = cs;
+        p.tpu1 = tpu;
+        p.tpu2 = (c.N + Q2 - 1) / Q2;
+        p.eta_scale = c.eta * (2.0f / (float)c.N);
+        p.W0 = c.W0;
+        p.W1_out = c.W1_out;
+        p.err = reinterpret_cast<uint32_t*>(c.ws);
+        CUtensorMap tmK, tmV, tmQ, tmZ;
+        if (!make_tmap_tokens(&tmK, c.K, c, TOK) || !make_tmap_tokens(&tmV, c.V, c, TOK) ||
+            !make_tmap_tokens(&tmQ, c.Q, c, Q2) || !make_tmap_tokens(&tmZ, c.Z, c, TOK))
+            return TTT_ERR_INVALID_ARG;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(ncl * cs));
+        cfg.blockDim = dim3(kThreadsTc);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = c.stream;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = cs; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        return check_launch(cudaLaunchKernelEx(&cfg, lin_cluster_bf16, tmK, tmV, tmQ, tmZ, p));
+    }
 
     MergeOut m{};
     m.eta_scale = c.eta * (2.0f / (float)c.N);
     m.W0 = c.W0;
     m.partials = reinterpret_cast<const float*>(c.ws + L.partials);
     m.W1_out = c.W1_out;
-
-    if (c.dtype == TTT_BF16) {
-        const int C1 = (tpu + TPC1 - 1) / TPC1, C2 = (tpu + TPC2 - 1) / TPC2;
-        const long long total = units * (C1 + C2);
-        if (total >= (1LL << 31)) return TTT_ERR_UNSUPPORTED;
-        m.W1_bf16 = reinterpret_cast<__nv_bfloat16*>(c.ws + L.w1);
-        FusedParams p{};
-        p.heads = c.heads;
-        p.tpu = tpu;
-        p.U = (int)units;
-        p.C1 = C1;
-        p.C2 = C2;
-        p.total = (unsigned)total;
-        p.m = m;
-        p.counters = reinterpret_cast<unsigned*>(c.ws + L.counters);
-        p.ready = reinterpret_cast<uint32_t*>(c.ws + L.ready);
-        p.ctrl = reinterpret_cast<unsigned*>(c.ws + L.ctrl);
-        p.err = reinterpret_cast<uint32_t*>(c.ws);
-        CUtensorMap tmK, tmV, tmQ, tmZ, tmW1;
-        if (!make_tmap_tokens(&tmK, c.K, c, TOK) || !make_tmap_tokens(&tmV, c.V, c, TOK) ||
-            !make_tmap_tokens(&tmQ, c.Q, c, TOK) || !make_tmap_tokens(&tmZ, c.Z, c, TOK) ||
-            !make_tmap_matrix(&tmW1, c.ws + L.w1, units * D, D, D))
-            return TTT_ERR_INVALID_ARG;
-        const size_t smem = sizeof(FusedSmem) + 1024;
-        cudaFuncSetAttribute(lin_fused_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        const int G = (int)std::min<long long>(c.num_sms, total);
-        lin_fused_bf16<<<G, kThreadsTc, smem, c.stream>>>(tmK, tmV, tmQ, tmZ, tmW1, p);
-        return check_launch(cudaGetLastError());
-    }
 
     // fp32
     const long long T = units * tpu;

@@ -40,6 +40,9 @@ struct Call {
 // Encodes a rank-4 bf16 tensor map over [batch][heads][N][64] with a 64 x box_rows box,
 // 128-byte swizzle, zero fill out of bounds.  Returns false on failure.
 bool make_tmap_tokens(CUtensorMap* m, const void* base, const Call& c, int box_rows);
+// Rank-5 tensor map over [batch][heads][H][W][64] (the token grid), no swizzle, zero fill out of bounds,
+// box = 64 channels x box_cols x box_rows of one unit.  Element type from c.dtype.
+bool make_tmap_grid(CUtensorMap* m, const void* base, const Call& c, int box_cols, int box_rows);
 // Rank-2 bf16 tensor map over a contiguous [rows][cols] matrix with a cols x box_rows box (cols*2 = 128).
 bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);
 
