@@ -1,6 +1,507 @@
-// mlp.cu -- placeholder until the MLP kernels land.
+// mlp.cu -- one-hidden-layer MLP inner model of the TTT layer, f(x) = Wb gelu_tanh(Wa x), hidden
+// width 256 = 4d (press article "CVPR 2026 Oral | 清華+阿里發布ViT3", Observation 4 and Fig. 5 part 1:
+// an MLP inner model whose width ratio goes up to 4).  One full-batch step of the L2 loss on both
+// matrices (gradients taken at the initial weights), then the readout:
+//     h = Wa k, a = gelu(h), y = Wb a, r = y - v
+//     gWb = sum_n r a^T,  gWa = sum_n [(Wb^T r) * gelu'(h)] k^T
+//     Wa1 = Wa - eta (2/N) gWa,  Wb1 = Wb - eta (2/N) gWb,  z = Wb1 gelu(Wa1 q)
+// gelu_tanh(u) = u/2 (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))) (the tanh form of Hendrycks & Gimpel).
+//
+// Every product is a dense contraction and runs on tcgen05 (bf16 operands, fp32 accumulation in
+// tensor memory).  One CTA owns a unit (persistent over units).  Per 128-token tile of phase 1:
+//   H  = K Wa^T            M=128 tokens, N=256, K=64       -> TMEM cols 256..511
+//   A  = gelu(H) (bf16, shared memory), gelu'(H) packed bf16x2 back into TMEM cols 256..383
+//   Y  = A Wb^T            M=128, N=64, K=256             -> TMEM cols 384..447
+//   R  = Y - V (bf16, shared memory)
+//   gWb^T += A^T R         M=256 (two 128-row halves), N=64, K=128 tokens (MN-major operands)
+//   dA = R Wb              M=128, N=128 per hidden half, K=64     -> TMEM cols 384..511
+//   dH = dA * gelu'(H) (bf16, shared memory, over A)
+//   gWa  += dH^T K         M=256 (two halves), N=64, K=128 tokens
+// The accumulators gWb^T and gWa stay in TMEM cols 0..255 across the unit's tiles.  Then
+// Wa1, Wb1 are formed in fp32 (optionally written out) and stored as bf16 operands, and phase 2
+// streams Q: H' = Q Wa1^T, A' = gelu(H'), Z = A' Wb1^T, stored with TMA.
+// The same shared-memory buffers serve as K-major operands of one product and MN-major operands of
+// another (both use the 128-byte swizzled layout TMA writes), so nothing is transposed.
+#include <algorithm>
+
+#include "sm100.cuh"
 #include "ttt_internal.h"
+
 namespace ttt {
-size_t mlp_ws_bytes(const ttt_shape&) { return kWsHeader; }
-ttt_status launch_mlp(const Call&) { return TTT_ERR_UNSUPPORTED; }
+namespace mlp {
+
+constexpr int D = 64;
+constexpr int HID = 256;
+constexpr int TOK = 128;
+constexpr int TILE = TOK * D * 2;           // 16 KB bf16 tile
+constexpr int STAGES = 2;                   // each holds a K tile + V tile, or a Q tile
+constexpr int THREADS = 160;                // warp 0: TMA producer, warps 1..4: MMA + elementwise
+constexpr float kGeluC = 0.7978845608028654f;   // sqrt(2 / pi)
+constexpr float kGeluA = 0.044715f;
+
+constexpr uint32_t kIdH = idesc_bf16_f32(128, 256, false, false);
+constexpr uint32_t kIdY = idesc_bf16_f32(128, 64, false, false);
+constexpr uint32_t kIdG = idesc_bf16_f32(128, 64, true, true);
+constexpr uint32_t kIdDA = idesc_bf16_f32(128, 128, false, true);
+
+struct Params {
+    int U, heads, N, tpu;
+    float eta_scale;                        // eta * 2 / N
+    const float* Wa;                        // [heads][256][64]
+    const float* Wb;                        // [heads][64][256]
+    float* Wa_out;                          // nullable [units][256][64]
+    float* Wb_out;                          // nullable [units][64][256]
+    uint32_t* err;
+};
+
+struct Smem {
+    uint8_t stage[STAGES][2 * TILE];        // K | V tiles, or a Q tile (1024-aligned)
+    uint8_t act[4][TOK * 128];              // A (then dH): [token][hidden], 4 panels of 64 hidden
+    uint8_t wa[HID * 128];                  // Wa (bf16): rows = hidden, 64 d per row
+    uint8_t wb[4][D * 128];                 // Wb (bf16): rows = d, 4 panels of 64 hidden
+    uint8_t rz[TOK * 128];                  // R tile (phase 1), Z staging (phase 2)
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t mma_bar;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Byte offset of element (row, col) in a 128-byte swizzled panel of 64 bf16 per row.
+__device__ __forceinline__ uint32_t sw_off(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
+}
+
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// gelu(u) and its derivative, from t = tanh(c (u + a u^3)).
+__device__ __forceinline__ void gelu_and_grad(float u, float& g, float& dg) {
+    const float u2 = u * u;
+    const float t = tanh_fast(kGeluC * fmaf(kGeluA * u2, u, u));
+    g = 0.5f * u * (1.f + t);
+    dg = 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * kGeluC * fmaf(3.f * kGeluA, u2, 1.f);
+}
+__device__ __forceinline__ float gelu_only(float u) {
+    const float t = tanh_fast(kGeluC * fmaf(kGeluA * u * u, u, u));
+    return 0.5f * u * (1.f + t);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+          const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmZ, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& s = *reinterpret_cast<Smem*>(align1024(smem_raw));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Abort ab{&s.abort_flag, p.err};
+
+    if (threadIdx.x == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        mbar_init(&s.mma_bar, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
+    }
+    if (warp == 1) { tmem_alloc(&s.tmem_base, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+
+    if (warp == 0) {                                           // TMA producer
+        if (lane == 0) {
+            int st = 0; uint32_t ph = 0;
+            for (int u = blockIdx.x; u < p.U; u += gridDim.x) {
+                const int b = u / p.heads, h = u % p.heads;
+                for (int t = 0; t < p.tpu; ++t) {
+                    if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
+                    mbar_arrive_expect_tx(&s.full[st], 2 * TILE);
+                    tma_load_4d(s.stage[st], &tmK, &s.full[st], 0, t * TOK, h, b);
+                    tma_load_4d(s.stage[st] + TILE, &tmV, &s.full[st], 0, t * TOK, h, b);
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+                for (int t = 0; t < p.tpu; ++t) {
+                    if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
+                    mbar_arrive_expect_tx(&s.full[st], TILE);
+                    tma_load_4d(s.stage[st], &tmQ, &s.full[st], 0, t * TOK, h, b);
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------------------------------
+        // warps 1..4: tid 0 issues the MMAs, all 128 threads do the elementwise work.  Thread tid
+        // reads and writes accumulator row r (its TMEM lane): a token (or a hidden unit).
+        // ---------------------------------------------------------------------------------------
+        const int tid = threadIdx.x - 32;
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const uint32_t sact = smem_u32(s.act[0]), swa = smem_u32(s.wa), swb = smem_u32(s.wb[0]), srz = smem_u32(s.rz);
+        uint32_t mph = 0;                                       // mma_bar phase
+        int st = 0; uint32_t ph = 0;
+        int zn = 0;
+        bool failed = false;
+
+        // issue-and-wait helper state
+        auto mma_sync = [&](bool& ok) {
+            if (tid == 0) mma_commit(&s.mma_bar);
+            ok = mbar_wait(&s.mma_bar, mph, ab);
+            mph ^= 1u;
+            if (named_bar_or(1, 128, !ok)) return false;
+            __syncwarp();
+            tc_fence_after();
+            return true;
+        };
+
+        for (int u = blockIdx.x; u < p.U && !failed; u += gridDim.x) {
+            const int bi = u / p.heads, h = u % p.heads;
+            // ---- Wa, Wb of the head -> bf16 operands
+            {
+                const float* Wa = p.Wa + (size_t)h * HID * D;
+                const float* Wb = p.Wb + (size_t)h * D * HID;
+                for (int row = tid; row < HID; row += 128) {          // Wa row = hidden unit
+                    for (int c = 0; c < D; c += 8) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = __ldg(Wa + (size_t)row * D + c + e);
+                        uint4 pk;
+                        pk.x = pack_bf16x2(v[0], v[1]); pk.y = pack_bf16x2(v[2], v[3]);
+                        pk.z = pack_bf16x2(v[4], v[5]); pk.w = pack_bf16x2(v[6], v[7]);
+                        *reinterpret_cast<uint4*>(s.wa + sw_off(row, c)) = pk;
+                    }
+                }
+                for (int idx = tid; idx < D * (HID / 8); idx += 128) {   // Wb: (d, 8 hidden) chunks
+                    const int d = idx / (HID / 8), c = (idx % (HID / 8)) * 8;
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = __ldg(Wb + (size_t)d * HID + c + e);
+                    uint4 pk;
+                    pk.x = pack_bf16x2(v[0], v[1]); pk.y = pack_bf16x2(v[2], v[3]);
+                    pk.z = pack_bf16x2(v[4], v[5]); pk.w = pack_bf16x2(v[6], v[7]);
+                    *reinterpret_cast<uint4*>(s.wb[c / 64] + sw_off(d, c % 64)) = pk;
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+            }
+            // ---- phase 1
+            for (int t = 0; t < p.tpu && !failed; ++t) {
+                bool ok = mbar_wait(&s.full[st], ph, ab);
+                if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                const uint32_t sK = smem_u32(s.stage[st]);
+                const uint8_t* vtile = s.stage[st] + TILE;
+                // H = K Wa^T
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16_ss(tmem + 256u, sdesc_sw128(sK + kk * 32, 16, 1024), sdesc_sw128(swa + kk * 32, 16, 1024),
+                                    kIdH, kk > 0 ? 1u : 0u);
+                }
+                if (!mma_sync(ok)) { failed = true; break; }
+                // A = gelu(H) -> act (bf16); gelu'(H) packed bf16x2 -> TMEM cols 256 + hid/2
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {                          // 64 hidden units per chunk
+                    float hv[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 256u + (uint32_t)(c * 64 + j * 16) + lane_off, hv[j]);
+                    tmem_ld_wait();
+                    uint32_t gp[32];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float a[16], dg[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) gelu_and_grad(hv[j][e], a[e], dg[e]);
+#pragma unroll
+                        for (int e = 0; e < 16; e += 8) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(a[e], a[e + 1]); pk.y = pack_bf16x2(a[e + 2], a[e + 3]);
+                            pk.z = pack_bf16x2(a[e + 4], a[e + 5]); pk.w = pack_bf16x2(a[e + 6], a[e + 7]);
+                            *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16 + e)) = pk;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; e += 2) gp[j * 8 + e / 2] = pack_bf16x2(dg[e], dg[e + 1]);
+                    }
+                    uint32_t g0[16], g1[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) { g0[e] = gp[e]; g1[e] = gp[16 + e]; }
+                    tmem_st16(tmem + 256u + (uint32_t)(c * 32) + lane_off, g0);
+                    tmem_st16(tmem + 256u + (uint32_t)(c * 32 + 16) + lane_off, g1);
+                }
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(1, 128);
+                // Y = A Wb^T
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < HID / 16; ++kk)
+                        mma_bf16_ss(tmem + 384u, sdesc_sw128(sact + (kk / 4) * (TOK * 128) + (kk % 4) * 32, 16, 1024),
+                                    sdesc_sw128(swb + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024), kIdY,
+                                    kk > 0 ? 1u : 0u);
+                }
+                if (!mma_sync(ok)) { failed = true; break; }
+                // R = Y - V -> rz (bf16)
+                {
+                    float yv[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 384u + (uint32_t)(j * 16) + lane_off, yv[j]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) {
+                        const uint4 vv = *reinterpret_cast<const uint4*>(vtile + sw_off(r, c));
+                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                        float rr[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            rr[2 * e] = yv[c / 16][(c % 16) + 2 * e] - bf16lo_to_f32(vw[e]);
+                            rr[2 * e + 1] = yv[c / 16][(c % 16) + 2 * e + 1] - bf16hi_to_f32(vw[e]);
+                        }
+                        uint4 pk;
+                        pk.x = pack_bf16x2(rr[0], rr[1]); pk.y = pack_bf16x2(rr[2], rr[3]);
+                        pk.z = pack_bf16x2(rr[4], rr[5]); pk.w = pack_bf16x2(rr[6], rr[7]);
+                        *reinterpret_cast<uint4*>(s.rz + sw_off(r, c)) = pk;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(1, 128);
+                // gWb^T += A^T R (two hidden halves) and dA_0 = R Wb (hidden 0..127)
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+                        for (int kk = 0; kk < TOK / 16; ++kk)
+                            mma_bf16_ss(tmem + (uint32_t)(hb * 64),
+                                        sdesc_sw128(sact + (2 * hb) * (TOK * 128) + kk * 2048, TOK * 128, 1024),
+                                        sdesc_sw128(srz + kk * 2048, 0, 1024), kIdG, (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16_ss(tmem + 384u, sdesc_sw128(srz + kk * 32, 16, 1024),
+                                    sdesc_sw128(swb + kk * 2048, D * 128, 1024), kIdDA, kk > 0 ? 1u : 0u);
+                }
+                if (!mma_sync(ok)) { failed = true; break; }
+                // dH = dA * gelu'(H) for both hidden halves -> act (A is no longer needed)
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    if (half == 1) {
+                        if (tid == 0) {
+                            tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_bf16_ss(tmem + 384u, sdesc_sw128(srz + kk * 32, 16, 1024),
+                                            sdesc_sw128(swb + 2 * (D * 128) + kk * 2048, D * 128, 1024), kIdDA,
+                                            kk > 0 ? 1u : 0u);
+                        }
+                        if (!mma_sync(ok)) { failed = true; break; }
+                    }
+#pragma unroll 1
+                    for (int c = 0; c < 2; ++c) {                       // 64 hidden units per chunk
+                        float da[4][16];
+                        float gq[2][16];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 384u + (uint32_t)(c * 64 + j * 16) + lane_off, da[j]);
+                        tmem_ld16(tmem + 256u + (uint32_t)(half * 64 + c * 32) + lane_off, gq[0]);
+                        tmem_ld16(tmem + 256u + (uint32_t)(half * 64 + c * 32 + 16) + lane_off, gq[1]);
+                        tmem_ld_wait();
+                        const int panel = half * 2 + c;
+#pragma unroll
+                        for (int e = 0; e < 64; e += 8) {
+                            float dh[8];
+#pragma unroll
+                            for (int i = 0; i < 8; i += 2) {
+                                const uint32_t w = __float_as_uint(gq[(e + i) / 32][((e + i) % 32) / 2]);
+                                dh[i] = da[(e + i) / 16][(e + i) % 16] * bf16lo_to_f32(w);
+                                dh[i + 1] = da[(e + i + 1) / 16][(e + i + 1) % 16] * bf16hi_to_f32(w);
+                            }
+                            uint4 pk;
+                            pk.x = pack_bf16x2(dh[0], dh[1]); pk.y = pack_bf16x2(dh[2], dh[3]);
+                            pk.z = pack_bf16x2(dh[4], dh[5]); pk.w = pack_bf16x2(dh[6], dh[7]);
+                            *reinterpret_cast<uint4*>(s.act[panel] + sw_off(r, e)) = pk;
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    named_bar_sync(1, 128);
+                }
+                if (failed) break;
+                // gWa += dH^T K (two hidden halves); frees the K/V stage when done
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+                        for (int kk = 0; kk < TOK / 16; ++kk)
+                            mma_bf16_ss(tmem + 128u + (uint32_t)(hb * 64),
+                                        sdesc_sw128(sact + (2 * hb) * (TOK * 128) + kk * 2048, TOK * 128, 1024),
+                                        sdesc_sw128(sK + kk * 2048, 0, 1024), kIdG, (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&s.empty[st]);
+                }
+                if (!mma_sync(ok)) { failed = true; break; }
+                if (++st == STAGES) { st = 0; ph ^= 1u; }
+            }
+            if (failed) break;
+            // ---- update: Wa1 = Wa - eta (2/N) gWa, Wb1 = Wb - eta (2/N) gWb  (rows hid = r, 128 + r)
+            {
+                const float* Wa = p.Wa + (size_t)h * HID * D;
+                const float* Wb = p.Wb + (size_t)h * D * HID;
+#pragma unroll 1
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int hid = hb * 128 + r;
+                    float ga[4][16], gb[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tmem_ld16(tmem + 128u + (uint32_t)(hb * 64 + j * 16) + lane_off, ga[j]);
+                        tmem_ld16(tmem + (uint32_t)(hb * 64 + j * 16) + lane_off, gb[j]);
+                    }
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) {
+                        float w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            w[e] = __ldg(Wa + (size_t)hid * D + c + e) - p.eta_scale * ga[(c + e) / 16][(c + e) % 16];
+                            if (p.Wa_out) p.Wa_out[((size_t)u * HID + hid) * D + c + e] = w[e];
+                        }
+                        uint4 pk;
+                        pk.x = pack_bf16x2(w[0], w[1]); pk.y = pack_bf16x2(w[2], w[3]);
+                        pk.z = pack_bf16x2(w[4], w[5]); pk.w = pack_bf16x2(w[6], w[7]);
+                        *reinterpret_cast<uint4*>(s.wa + sw_off(hid, c)) = pk;
+                    }
+#pragma unroll
+                    for (int d = 0; d < D; ++d) {
+                        const float w = __ldg(Wb + (size_t)d * HID + hid) - p.eta_scale * gb[d / 16][d % 16];
+                        if (p.Wb_out) p.Wb_out[((size_t)u * D + d) * HID + hid] = w;
+                        *reinterpret_cast<__nv_bfloat16*>(s.wb[hid / 64] + sw_off(d, hid % 64)) = __float2bfloat16_rn(w);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(1, 128);
+            }
+            // ---- phase 2: Z = gelu(Q Wa1^T) Wb1^T
+            for (int t = 0; t < p.tpu && !failed; ++t) {
+                bool ok = mbar_wait(&s.full[st], ph, ab);
+                if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                const uint32_t sQ = smem_u32(s.stage[st]);
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16_ss(tmem + 256u, sdesc_sw128(sQ + kk * 32, 16, 1024), sdesc_sw128(swa + kk * 32, 16, 1024),
+                                    kIdH, kk > 0 ? 1u : 0u);
+                }
+                if (!mma_sync(ok)) { failed = true; break; }
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float hv[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 256u + (uint32_t)(c * 64 + j * 16) + lane_off, hv[j]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int e = 0; e < 16; e += 8) {
+                            float a[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) a[i] = gelu_only(hv[j][e + i]);
+                            uint4 pk;
+                            pk.x = pack_bf16x2(a[0], a[1]); pk.y = pack_bf16x2(a[2], a[3]);
+                            pk.z = pack_bf16x2(a[4], a[5]); pk.w = pack_bf16x2(a[6], a[7]);
+                            *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16 + e)) = pk;
+                        }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(1, 128);
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < HID / 16; ++kk)
+                        mma_bf16_ss(tmem + 384u, sdesc_sw128(sact + (kk / 4) * (TOK * 128) + (kk % 4) * 32, 16, 1024),
+                                    sdesc_sw128(swb + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024), kIdY,
+                                    kk > 0 ? 1u : 0u);
+                    mma_commit(&s.empty[st]);
+                }
+                if (!mma_sync(ok)) { failed = true; break; }
+                if (tid == 0 && zn > 0) bulk_wait_read<0>();          // the previous Z tile has left rz
+                named_bar_sync(1, 128);
+                {
+                    float zv[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 384u + (uint32_t)(j * 16) + lane_off, zv[j]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(zv[c / 16][c % 16], zv[c / 16][c % 16 + 1]);
+                        pk.y = pack_bf16x2(zv[c / 16][c % 16 + 2], zv[c / 16][c % 16 + 3]);
+                        pk.z = pack_bf16x2(zv[c / 16][c % 16 + 4], zv[c / 16][c % 16 + 5]);
+                        pk.w = pack_bf16x2(zv[c / 16][c % 16 + 6], zv[c / 16][c % 16 + 7]);
+                        *reinterpret_cast<uint4*>(s.rz + sw_off(r, c)) = pk;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(1, 128);
+                if (tid == 0) {
+                    tma_store_4d(&tmZ, s.rz, 0, t * TOK, h, bi);
+                    bulk_commit();
+                }
+                ++zn;
+                if (++st == STAGES) { st = 0; ph ^= 1u; }
+            }
+            if (tid == 0) bulk_wait<0>();                          // rz is reused by the next unit
+            named_bar_sync(1, 128);
+        }
+        if (tid == 0) bulk_wait<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace mlp
+
+size_t mlp_ws_bytes(const ttt_shape&) { return kWsHeader; }   // error word only
+
+ttt_status launch_mlp(const Call& c) {
+    using namespace mlp;
+    if (c.dtype != TTT_BF16 || c.hidden != HID) return TTT_ERR_UNSUPPORTED;
+    const long long units = (long long)c.batch * c.heads;
+    Params p{};
+    p.U = (int)units;
+    p.heads = c.heads;
+    p.N = c.N;
+    p.tpu = (c.N + TOK - 1) / TOK;
+    p.eta_scale = c.eta * (2.0f / (float)c.N);
+    p.Wa = c.W0;
+    p.Wb = c.W0b;
+    p.Wa_out = c.W1_out;
+    p.Wb_out = c.W1b_out;
+    p.err = reinterpret_cast<uint32_t*>(c.ws);
+    CUtensorMap tmK, tmV, tmQ, tmZ;
+    if (!make_tmap_tokens(&tmK, c.K, c, TOK) || !make_tmap_tokens(&tmV, c.V, c, TOK) ||
+        !make_tmap_tokens(&tmQ, c.Q, c, TOK) || !make_tmap_tokens(&tmZ, c.Z, c, TOK))
+        return TTT_ERR_INVALID_ARG;
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaFuncSetAttribute(mlp_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int grid = (int)std::min<long long>(units, c.num_sms);
+    mlp_fused<<<grid, THREADS, smem, c.stream>>>(tmK, tmV, tmQ, tmZ, p);
+    return check_launch(cudaGetLastError());
+}
+
 }  // namespace ttt
