@@ -34,6 +34,11 @@ from vision_test_token_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "TTT-layer fwd tokens*heads/s at 6084 tokens"
 UNIT = "token*heads/s"
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised under
+# profiles/ (lin_cluster_bf16_mixed6084.md, mlp_fused_mlp1024.md).  Valid only for the kernel build
+# those captures were taken on; reset to None whenever the kernel changes.
+LIN_TRAFFIC_MIXED6084 = 93.595904e6 + 6.192896e6
+MLP_TRAFFIC_MLP1024 = 25.780736e6 + 0.0
 
 
 def parse():
@@ -339,7 +344,7 @@ def run_ours(args):
     el_max = max_over_ranks(el, world, dev)
     # keep the GPU loaded a little longer so the clock record covers the load
     if t_wall1 - t_wall0 < 1.0:
-        soak_steps = int(args.steps * (1.2 / max(t_wall1 - t_wall0, 1e-3)))
+        soak_steps = min(20000, int(args.steps * (1.2 / max(t_wall1 - t_wall0, 1e-3))))
         t_wall0 = time.time()
         time_graphs(graphs, soak_steps, stream)
         t_wall1 = time.time()
@@ -364,12 +369,25 @@ def run_ours(args):
         lin_bytes = 4 * w.batch * w.lin_heads * w.N * w.d * esz
         conv_bytes = 4 * w.batch * w.conv_heads * w.N * w.d * esz
         achieved = lin_bytes / t_lin / 1e9
-        roof = {"bound": "hbm", "kernel": "lin_p1_bf16+lin_p2_bf16 (one ttt_forward_linear call)",
+        roof = {"bound": "hbm", "kernel": "lin_cluster_bf16 (the whole ttt_forward_linear call)",
                 "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                "traffic": None, "peak_source": pk["source"],
-                "algorithmic_bytes": lin_bytes, "us_per_launch": t_lin * 1e6,
-                "conv_call": {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
-                              "achieved_gbs": conv_bytes / t_conv / 1e9}}
+                "traffic": LIN_TRAFFIC_MIXED6084 if w.name == "mixed6084_bf16" else None,
+                "peak_source": pk["source"], "algorithmic_bytes": lin_bytes, "us_per_launch": t_lin * 1e6,
+                "conv_call": {"kernel": "dw_cluster<bf16>", "us_per_launch": t_conv * 1e6,
+                              "algorithmic_bytes": conv_bytes, "achieved_gbs": conv_bytes / t_conv / 1e9,
+                              "frac": conv_bytes / t_conv / 1e9 / pk["hbm_gbs"]}}
+    elif w.kind == "mlp":
+        n = max(100, args.steps // 4)
+        time_graphs(graphs, 10, stream)
+        t_mlp = time_graphs(graphs, n, stream) / n
+        d, hid = w.d, w.hidden_ratio * w.d
+        flops = w.batch * w.heads * w.N * (2 * d * hid * 5 + 2 * d * hid * 2)   # 5 products in the step, 2 in the readout
+        achieved = flops / t_mlp / 1e12
+        roof = {"bound": "tensor", "kernel": "mlp_fused (the whole ttt_forward_mlp call)", "achieved": achieved,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                "traffic": MLP_TRAFFIC_MLP1024 if w.name == "mlp1024_bf16" else None,
+                "peak_source": pk["source"] + " (bf16 burst)", "algorithmic_flops": flops,
+                "us_per_launch": t_mlp * 1e6}
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host result
     e2e = run_e2e(w, xs[0], dev, stream, args.e2e_steps, world)
@@ -383,7 +401,7 @@ def run_ours(args):
                        "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",
                        "algorithmic_bytes_per_step": workload_bytes(w), "launch": "CUDA graph per input set"},
             "gbs_per_step": workload_bytes(w) / (el_max / args.steps) / 1e9,
-            "gpu_launches": args.steps * (4 if w.kind == "mixed" else 2),
+            "gpu_launches": args.steps * (2 if (w.kind == "mixed" or w.dtype == "fp32") else 1),
             "clocks": clocks, "e2e": e2e}
     if roof:
         line["roofline"] = roof
