@@ -130,17 +130,29 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 # distributed plumbing
 # ------------------------------------------------------------------------------------------------
-def dist_init(gpus):
+def dist_init(gpus, backend="nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).  `backend` is "nccl" on GPUs;
+    the CPU tests use "gloo"."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
+
+
+def shard_batch(global_batch, rank, world):
+    """The contiguous range of images (start, count) that `rank` of `world` processes.  Units are
+    independent, so sharding the batch needs no exchange at all; the first global_batch % world ranks
+    take one image more."""
+    base, extra = divmod(global_batch, world)
+    return rank * base + min(rank, extra), base + (1 if rank < extra else 0)
 
 
 def barrier(world):
@@ -247,7 +259,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(1, args.steps) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "tokens": w.N, "d": w.d,
+            "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads, "tokens": w.N, "d": w.d,
                        "eta": w.eta, "device": "host CPU"},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -299,10 +311,13 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     pk = peaks()
 
-    # input sets (seeded per rank and set), Z buffers, workspaces
+    # this rank's images of the global batch (weak scaling: w.batch images per GPU), one input set per
+    # seed; Z buffers, workspaces
+    first, count = shard_batch(w.batch * world, rank, world)
+    assert count == w.batch
     xs = []
     for s in range(args.sets):
-        x = make_inputs(w, seed=1000 * rank + s, device=dev)
+        x = make_inputs(w, seed=1000 * first + s, device=dev)
         x["Z"] = torch.empty_like(x["Q"])
         xs.append(x)
     stream = torch.cuda.Stream(device=dev)
@@ -395,7 +410,7 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads,
+            "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads,
                        "lin_heads": w.lin_heads, "conv_heads": w.conv_heads, "grid": [w.H, w.W],
                        "tokens": w.N, "d": w.d, "eta": w.eta, "parallelism": f"batch-sharded x{world}",
                        "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",

@@ -8,10 +8,14 @@
 //     128-byte swizzle) and accumulates [K | V]^T K  (128 x 64 fp32: rows 0..63 = G, rows 64..127
 //     = C) in tensor memory with tcgen05.mma: A = [K | V]^T (M = 128, MN-major straight from the
 //     token-major tiles), B = K (N = 64, MN-major), K-dim = tokens.
-//   Exchange: each CTA puts its partial in shared memory and signals its peers through remote
-//     mbarrier arrivals; every CTA then sums the CS partials over distributed shared memory in rank
-//     order (a fixed order: bitwise deterministic) and forms W1 in fp32, rounded once to bf16 into
-//     the shared-memory B operand of phase 2.  No global-memory round trip, no grid-wide wait.
+//   Exchange: each CTA turns its own partial (G_r, C_r) into P_r = W0 G_r - C_r.  The product runs
+//     on the tensor cores with both operands split into bf16 hi + lo parts (M = 128 rows
+//     [W0_hi ; W0_lo], B = G_hi and then G_lo), so that it carries about 16 mantissa bits, close to
+//     fp32.  P_r (16 KB) is pushed with one bulk copy into every other CTA of the cluster (distributed
+//     shared memory, completion counted on the receiver's mbarrier); each CTA then forms
+//     W1 = W0 - eta (2/N) sum_r P_r, summing in rank order (a fixed order: bitwise deterministic),
+//     and rounds W1 once to bf16 into the shared-memory B operand of phase 2.  No global-memory
+//     round trip, no grid-wide wait.
 //   Phase 2: the CTA streams its share of 256-token Q tiles (they are prefetched while the cluster
 //     reduces) and writes Z = Q W1^T: A = Q tile (M = 128 tokens, K-major), B = W1 (K-major), the
 //     epilogue drains tensor memory to bf16 and stores Z with TMA.
