@@ -76,6 +76,11 @@ typedef struct {
     long long batch_stride;  /* elements between consecutive images in Q, K, V, Z */
     long long head_stride;   /* elements between consecutive heads in Q, K, V, Z */
     int dtype;               /* ttt_dtype of Q, K, V and Z */
+    int max_sms;             /* SMs the call may spread its work over; 0 = the whole device.  Two calls
+                                that run at the same time on two streams (e.g. the linear heads and the
+                                conv heads of one layer) each take a share, so that neither waits for
+                                SMs the other holds.  It may change how sums are split over CTAs, hence
+                                the rounding; results are bitwise reproducible for a fixed value. */
 } ttt_shape;
 
 /* Bytes of device workspace that a call of head kind `kind` with shape `s` needs (0 on an invalid
@@ -106,6 +111,8 @@ ttt_status ttt_forward_linear(const void* Q, const void* K, const void* V, const
  *   r = f(K;W0) - V;  g[c][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c,y+a-1,x+b-1];  W1 = W0 - eta g;
  *   Z = f(Q;W1).
  *   W0:     [heads][d][3][3] fp32.   W1_out: optional [batch][heads][d][3][3] fp32.
+ *   The workspace holds per-(image, head) partial sums and counters (about 25 KB per unit at 78 x 78
+ *   tokens); after a TTT_ERR_TIMEOUT it must be zero-filled again (ttt_workspace_init).
  */
 ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const float* W0,
                               void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes,
@@ -145,6 +152,25 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
  */
 ttt_status ttt_forward_linear_noalloc(const void* Q, const void* K, const void* V, const float* W0, void* Z,
                                       float eta, const ttt_shape* s, float* W1_out, void* stream);
+
+/* A layer whose heads [0, heads - conv_heads) are linear heads and whose last conv_heads heads are
+ * depthwise-conv heads (ViT^3 keeps one conv head among its linear heads: press article,
+ * Observation 6), over one [batch][heads][N][d] view described by s (s->heads = all heads):
+ * ttt_forward_linear on the first range and ttt_forward_dwconv on the second, with the same results.
+ * Both kernels run at the same time: the linear kernel is given a share of the SMs in proportion to
+ * its heads' work (a conv head counting as two linear heads); the conv kernel is queued behind it as
+ * a programmatic dependent, starts as soon as every linear CTA is resident, takes the SMs left free
+ * and then those the linear kernel releases.  The call is complete on `stream` when both kernels are.
+ * Results equal those of the two separate calls with the same SM budgets.
+ *   W0_lin: [heads - conv_heads][d][d], W0_conv: [conv_heads][d][3][3] (each may be NULL when its
+ *   range is empty).  W1_lin_out / W1_conv_out: optional, as in the two calls above.
+ *   ws: ttt_layer_workspace_bytes(s, conv_heads) bytes, zero-filled once (ttt_workspace_init); its
+ *   error word is the one ttt_workspace_status reads.
+ */
+size_t ttt_layer_workspace_bytes(const ttt_shape* s, int conv_heads);
+ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const float* W0_lin,
+                             const float* W0_conv, void* Z, float eta, const ttt_shape* s, int conv_heads,
+                             void* ws, size_t ws_bytes, float* W1_lin_out, float* W1_conv_out, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(ttt_status st);

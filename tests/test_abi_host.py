@@ -52,10 +52,32 @@ def test_workspace_sizes(lib):
     nf = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(dtype=capi.TTT_FP32, batch_stride=6 * 6084 * 64))
     assert 40 * 64 * 64 * 4 < nf < 16 << 20           # fp32: counters, W1 and partial slots
     nc = capi.ttt_workspace_bytes(capi.TTT_HEAD_DWCONV, s)
-    assert nc == 256                                     # conv: the error word only
+    # conv: header, control words (queue, done, 40 unit counters, 40 ready flags) padded to 256 B,
+    # then per unit room for one task per row pair (39) x 2 compute groups of 576-float partials,
+    # then W1 per unit
+    assert nc == 256 + 512 + 40 * 39 * 2 * 576 * 4 + 40 * 576 * 4
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(d=32)) == 0
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(batch=0)) == 0
     assert capi.ttt_workspace_bytes(7, s) == 0
+
+
+def test_layer_workspace_sizes(lib):
+    s = _shape(heads=6)
+    # the linear range's workspace (bf16: the error word), then the conv range's (8 units)
+    assert capi.ttt_layer_workspace_bytes(s, 1) == 256 + (256 + 256 + 8 * 39 * 2 * 576 * 4 + 8 * 576 * 4)
+    assert capi.ttt_layer_workspace_bytes(s, 0) == 256
+    assert capi.ttt_layer_workspace_bytes(s, 6) == capi.ttt_workspace_bytes(capi.TTT_HEAD_DWCONV, s)
+    assert capi.ttt_layer_workspace_bytes(s, 7) == 0
+    assert capi.ttt_layer_workspace_bytes(s, -1) == 0
+
+
+def test_layer_rejects_bad_head_split(lib):
+    s = _shape(heads=6)
+    fake = ctypes.c_void_p(1 << 20)
+    for ch in (-1, 7):
+        st = capi.ttt_forward_layer(fake, fake, fake, fake, fake, ctypes.c_void_p(1 << 40), 0.5, s, ch, fake,
+                                    1 << 30, None, None, None)
+        assert st == capi.TTT_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("kw,expected", [
@@ -63,6 +85,7 @@ def test_workspace_sizes(lib):
     (dict(batch=0), capi.TTT_ERR_INVALID_ARG),
     (dict(H=0), capi.TTT_ERR_INVALID_ARG),
     (dict(dtype=5), capi.TTT_ERR_INVALID_ARG),
+    (dict(max_sms=-1), capi.TTT_ERR_INVALID_ARG),
     (dict(head_stride=100), capi.TTT_ERR_INVALID_ARG),          # heads would overlap
     (dict(head_stride=6084 * 64 + 4), capi.TTT_ERR_ALIGNMENT),  # not a 16-byte multiple for bf16
 ])

@@ -14,17 +14,17 @@ from vision_test_token_b200.inputs import random_unit
 pytestmark = pytest.mark.gpu
 
 
-def _run(x, eta, H, W, dev):
+def _run(x, eta, H, W, dev, max_sms=0):
     Q, K, V = (x[k].to(dev) for k in ("Q", "K", "V"))
     B, h = Q.shape[:2]
     W1 = torch.full((B, h, 64, 3, 3), float("nan"), device=dev)
-    Z = forward_dwconv(Q, K, V, x["W0_conv"].to(dev), eta, H, W, W1_out=W1)
+    Z = forward_dwconv(Q, K, V, x["W0_conv"].to(dev), eta, H, W, W1_out=W1, max_sms=max_sms)
     torch.cuda.synchronize()
     return Z, W1
 
 
-def _check(x, eta, H, W, dev, dtype):
-    Z, W1 = _run(x, eta, H, W, dev)
+def _check(x, eta, H, W, dev, dtype, max_sms=0):
+    Z, W1 = _run(x, eta, H, W, dev, max_sms)
     Zr, W1r = oracle.dwconv(x["Q"], x["K"], x["V"], x["W0_conv"], eta, H, W)
     W0 = x["W0_conv"].double().numpy()[None]
     ez, ew = rel_max_err(Z, Zr), rel_update_err(W1, W1r, W0)
@@ -38,7 +38,7 @@ def _conv_inputs(B, h, H, W, dtype, seed):
 
 @pytest.mark.parametrize("B,h,H,W", [
     (1, 1, 1, 1), (1, 1, 1, 9), (1, 1, 9, 1), (2, 1, 5, 7), (3, 2, 14, 14), (2, 1, 33, 17), (8, 1, 78, 78),
-    (1, 3, 80, 80), (40, 1, 6, 6),
+    (1, 3, 80, 80), (40, 1, 6, 6), (5, 1, 2, 30), (1, 1, 7, 170), (2, 1, 4, 161), (300, 1, 3, 5),
 ])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_dwconv_shapes(cuda_dev, B, h, H, W, dtype):
@@ -64,16 +64,26 @@ def test_dwconv_eta_zero_matches_torch_conv2d(cuda_dev):
     assert rel_max_err(Z, ref.numpy()) <= 1e-5
 
 
-def test_mixed6084_layer_full(cuda_dev):
+@pytest.mark.parametrize("max_sms", [1, 2, 3, 24, 25, 0])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_dwconv_sm_budget(cuda_dev, max_sms, dtype):
+    """Any SM budget (cluster sizes 1..8, units looping over fewer clusters) gives the same result
+    within tolerance."""
+    _check(_conv_inputs(8, 1, 78, 78, dtype, seed=17), 0.5, 78, 78, cuda_dev, dtype, max_sms)
+
+
+@pytest.mark.parametrize("concurrent", [True, False])
+def test_mixed6084_layer_full(cuda_dev, concurrent):
     """The full 6084-token layer: 5 linear heads + the depthwise-conv head (last), in the launch
-    configuration the benchmark times (two calls on one stream over head slices)."""
+    configuration the benchmark times (the conv call on a second stream, at the same time as the
+    linear call, each on its share of the SMs) and one call after the other."""
     w = WORKLOADS["mixed6084_bf16"]
     x = make_inputs(w)
     dev = cuda_dev
     Q, K, V = (x[k].to(dev) for k in ("Q", "K", "V"))
     Z = torch.full_like(Q, float("nan"))
     forward_layer(Q, K, V, {k: v.to(dev) for k, v in x.items() if k.startswith("W0")}, w.eta, w.H, w.W,
-                  conv_heads=w.conv_heads, Z=Z)
+                  conv_heads=w.conv_heads, Z=Z, concurrent=concurrent)
     torch.cuda.synchronize()
     nl = w.lin_heads
     Zl, _ = oracle.linear(x["Q"][:, :nl], x["K"][:, :nl], x["V"][:, :nl], x["W0_lin"], w.eta)

@@ -17,18 +17,18 @@ from vision_test_token_b200.inputs import random_unit
 pytestmark = pytest.mark.gpu
 
 
-def _run(x, eta, H, W, dev, with_w1=True):
+def _run(x, eta, H, W, dev, with_w1=True, max_sms=0):
     Q, K, V = (x[k].to(dev) for k in ("Q", "K", "V"))
     W0 = x["W0_lin"].to(dev)
     B, h = Q.shape[:2]
     W1 = torch.full((B, h, 64, 64), float("nan"), device=dev) if with_w1 else None
-    Z = forward_linear(Q, K, V, W0, eta, H, W, W1_out=W1)
+    Z = forward_linear(Q, K, V, W0, eta, H, W, W1_out=W1, max_sms=max_sms)
     torch.cuda.synchronize()
     return Z, W1
 
 
-def _check(x, eta, H, W, dev, dtype):
-    Z, W1 = _run(x, eta, H, W, dev)
+def _check(x, eta, H, W, dev, dtype, max_sms=0):
+    Z, W1 = _run(x, eta, H, W, dev, max_sms=max_sms)
     Zr, W1r = oracle.linear(x["Q"], x["K"], x["V"], x["W0_lin"], eta)
     W0 = x["W0_lin"].double().numpy()[None]
     ez, ew = rel_max_err(Z, Zr), rel_update_err(W1, W1r, W0)
@@ -50,6 +50,14 @@ def test_lin196_bf16_workload(cuda_dev):
 def test_lin6400_bf16_workload_full(cuda_dev):
     w = WORKLOADS["lin6400_bf16"]
     _check(make_inputs(w), w.eta, w.H, w.W, cuda_dev, "bf16")
+
+
+@pytest.mark.parametrize("max_sms", [1, 7, 50, 123])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_sm_budget(cuda_dev, max_sms, dtype):
+    """A bounded SM budget (fewer clusters or CTAs than units, smaller clusters) stays in tolerance."""
+    _, x = random_unit(8, 5, 30, 40, dtype=dtype, seed=max_sms)
+    _check(x, 0.5, 30, 40, cuda_dev, dtype, max_sms=max_sms)
 
 
 @pytest.mark.parametrize("B,h,H,W", [

@@ -16,6 +16,7 @@ TTT_HEAD_LINEAR, TTT_HEAD_DWCONV, TTT_HEAD_MLP = 0, 1, 2
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_workspace_init", "ttt_workspace_status",
     "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp", "ttt_forward_linear_noalloc",
+    "ttt_layer_workspace_bytes", "ttt_forward_layer",
     "ttt_status_string", "ttt_last_error", "ttt_version",
 )
 
@@ -25,7 +26,7 @@ class TttShape(ctypes.Structure):
         ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
         ("d", ctypes.c_int), ("hidden", ctypes.c_int),
         ("batch_stride", ctypes.c_longlong), ("head_stride", ctypes.c_longlong),
-        ("dtype", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("max_sms", ctypes.c_int),
     ]
 
 
@@ -62,6 +63,10 @@ def lib():
         L.ttt_forward_dwconv.restype = i
         L.ttt_forward_mlp.argtypes = [vp, vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp, vp]
         L.ttt_forward_mlp.restype = i
+        L.ttt_layer_workspace_bytes.argtypes = [shp, i]
+        L.ttt_layer_workspace_bytes.restype = sz
+        L.ttt_forward_layer.argtypes = [vp, vp, vp, vp, vp, vp, f, shp, i, vp, sz, vp, vp, vp]
+        L.ttt_forward_layer.restype = i
         L.ttt_status_string.argtypes = [i]
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_last_error.argtypes = []
@@ -79,8 +84,8 @@ def status_string(st):
     return lib().ttt_status_string(int(st)).decode()
 
 
-def make_shape(batch, heads, H, W, d, batch_stride, head_stride, dtype, hidden=0):
-    return TttShape(batch, heads, H, W, d, hidden, batch_stride, head_stride, dtype)
+def make_shape(batch, heads, H, W, d, batch_stride, head_stride, dtype, hidden=0, max_sms=0):
+    return TttShape(batch, heads, H, W, d, hidden, batch_stride, head_stride, dtype, max_sms)
 
 
 def ttt_workspace_bytes(kind, shape):
@@ -110,6 +115,16 @@ def ttt_forward_dwconv(Q, K, V, W0, Z, eta, shape, ws, ws_bytes, W1_out, stream)
 def ttt_forward_mlp(Q, K, V, Wa, Wb, Z, eta, shape, ws, ws_bytes, Wa_out, Wb_out, stream):
     return lib().ttt_forward_mlp(Q, K, V, Wa, Wb, Z, eta, ctypes.byref(shape), ws, ws_bytes, Wa_out, Wb_out,
                                  stream)
+
+
+def ttt_layer_workspace_bytes(shape, conv_heads):
+    return lib().ttt_layer_workspace_bytes(ctypes.byref(shape), conv_heads)
+
+
+def ttt_forward_layer(Q, K, V, W0_lin, W0_conv, Z, eta, shape, conv_heads, ws, ws_bytes, W1_lin_out, W1_conv_out,
+                      stream):
+    return lib().ttt_forward_layer(Q, K, V, W0_lin, W0_conv, Z, eta, ctypes.byref(shape), conv_heads, ws, ws_bytes,
+                                   W1_lin_out, W1_conv_out, stream)
 
 
 def ttt_last_error():

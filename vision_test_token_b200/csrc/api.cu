@@ -94,7 +94,7 @@ static ttt_status check_shape(int kind, const ttt_shape* s) {
     if (s->batch < 1 || s->heads < 1 || s->H < 1 || s->W < 1 || s->d < 1) return TTT_ERR_INVALID_ARG;
     if ((long long)s->H * s->W > (1LL << 30)) return TTT_ERR_INVALID_ARG;
     if (s->dtype != TTT_FP32 && s->dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
-    if (s->batch_stride < 0 || s->head_stride < 0) return TTT_ERR_INVALID_ARG;
+    if (s->batch_stride < 0 || s->head_stride < 0 || s->max_sms < 0) return TTT_ERR_INVALID_ARG;
     if ((long long)s->batch * s->heads > (1LL << 24)) return TTT_ERR_INVALID_ARG;
     if (s->d != 64) return TTT_ERR_UNSUPPORTED;
     if (kind == TTT_HEAD_MLP) {
@@ -173,7 +173,9 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
     c->ws = static_cast<uint8_t*>(ws);
     c->ws_bytes = ws_bytes;
     c->stream = static_cast<cudaStream_t>(stream);
-    c->num_sms = sms;
+    c->num_sms = (s->max_sms > 0 && s->max_sms < sms) ? s->max_sms : sms;
+    c->overlap_previous = 0;
+    c->err_ws = nullptr;
     return TTT_OK;
 }
 
@@ -262,6 +264,79 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
     return launch_mlp(c);
 }
 
+constexpr double kConvHeadWeight = 2.0;
+
+// The layer call works on two head ranges of one [B][heads][N][d] view: heads [0, nl) linear, heads
+// [nl, heads) depthwise conv.  Its workspace is the linear workspace followed by the conv workspace.
+static void layer_shapes(const ttt_shape* s, int conv_heads, ttt_shape* lin, ttt_shape* conv) {
+    *lin = *s;
+    *conv = *s;
+    lin->heads = s->heads - conv_heads;
+    conv->heads = conv_heads;
+}
+
+static size_t layer_lin_ws(const ttt_shape& lin) {
+    return lin.heads > 0 ? align_up(linear_ws_bytes(lin), 256) : 0;
+}
+
+size_t ttt_layer_workspace_bytes(const ttt_shape* s, int conv_heads) {
+    if (check_shape(TTT_HEAD_LINEAR, s) != TTT_OK || conv_heads < 0 || conv_heads > s->heads) return 0;
+    ttt_shape lin, conv;
+    layer_shapes(s, conv_heads, &lin, &conv);
+    return layer_lin_ws(lin) + (conv.heads > 0 ? dwconv_ws_bytes(conv) : 0);
+}
+
+ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const float* W0_lin, const float* W0_conv,
+                             void* Z, float eta, const ttt_shape* s, int conv_heads, void* ws, size_t ws_bytes,
+                             float* W1_lin_out, float* W1_conv_out, void* stream) {
+    ttt_status st = check_shape(TTT_HEAD_LINEAR, s);
+    if (st != TTT_OK) return st;
+    if (conv_heads < 0 || conv_heads > s->heads) return TTT_ERR_INVALID_ARG;
+    ttt_shape lin, conv;
+    layer_shapes(s, conv_heads, &lin, &conv);
+    const size_t lin_ws = layer_lin_ws(lin);
+    const size_t need = ttt_layer_workspace_bytes(s, conv_heads);
+    // the whole view first (pointers, alignment, Z apart from Q/K/V over all heads), then each range
+    Call whole;
+    st = prepare(TTT_HEAD_LINEAR, Q, K, V, lin.heads ? W0_lin : W0_conv, nullptr, Z, eta, s, ws, ws_bytes, need,
+                 stream, &whole);
+    if (st != TTT_OK) return st;
+    for (float* o : {W1_lin_out, W1_conv_out})
+        if (o && (reinterpret_cast<uintptr_t>(o) % 16 || !is_device_ptr(o))) return TTT_ERR_INVALID_ARG;
+    Call cl, cc;
+    const long long esz = (s->dtype == TTT_BF16) ? 2 : 4;
+    const long long off = (long long)lin.heads * whole.hs * esz;    // bytes from head 0 to head nl
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    if (lin.heads) {
+        st = prepare(TTT_HEAD_LINEAR, Q, K, V, W0_lin, nullptr, Z, eta, &lin, w8, lin_ws, linear_ws_bytes(lin),
+                     stream, &cl);
+        if (st != TTT_OK) return st;
+        cl.W1_out = W1_lin_out;
+    }
+    if (conv.heads) {
+        auto shift = [&](const void* p) { return static_cast<const void*>(static_cast<const uint8_t*>(p) + off); };
+        st = prepare(TTT_HEAD_DWCONV, shift(Q), shift(K), shift(V), W0_conv, nullptr,
+                     const_cast<void*>(shift(Z)), eta, &conv, w8 + lin_ws, ws_bytes - lin_ws, dwconv_ws_bytes(conv),
+                     stream, &cc);
+        if (st != TTT_OK) return st;
+        cc.W1_out = W1_conv_out;
+        cc.err_ws = w8;                                              // one error word for the layer
+        // the conv kernel queues behind the linear kernel and takes the SMs it leaves free; as its
+        // CTAs finish, the rest of the conv grid takes over the SMs the linear kernel releases
+        cc.overlap_previous = lin.heads ? 1 : 0;
+    }
+    if (lin.heads && conv.heads) {
+        // The linear kernel gets a share of the SMs in proportion to its heads' work, counting a conv
+        // head as kConvHeadWeight linear heads (a conv head's FMA work per token is about that much
+        // more SM time than a linear head's tensor-core streaming); the conv kernel takes the rest.
+        const double wl = (double)lin.heads, wc = kConvHeadWeight * conv.heads;
+        cl.num_sms = std::max(1, (int)((double)whole.num_sms * wl / (wl + wc)));
+    }
+    if (lin.heads && (st = launch_linear(cl)) != TTT_OK) return st;
+    if (conv.heads) st = launch_dwconv(cc);
+    return st;
+}
+
 const char* ttt_status_string(ttt_status st) {
     switch (st) {
         case TTT_OK: return "TTT_OK";
@@ -277,6 +352,6 @@ const char* ttt_status_string(ttt_status st) {
 
 ttt_status ttt_last_error(void) { return g_sticky.load() ? TTT_ERR_CUDA : TTT_OK; }
 
-int ttt_version(void) { return 100; }
+int ttt_version(void) { return 102; }
 
 }  // extern "C"

@@ -5,25 +5,35 @@
 //     g[c][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c,y+a-1,x+b-1],   W1 = W0 - eta g
 //     Z[c,y,x] = sum_{a,b} W1[c][a][b] Q[c,y+a-1,x+b-1]
 //
-// Not a contraction worth a tensor core (about 7 flop per byte): packed fp32x2 FMA.
+// Not a contraction worth a tensor core (about 7 flop per byte): fp32 FMA in registers.
 //
-// One kernel, one thread-block cluster of CS CTAs per unit (one CTA per SM).  A unit's grid is cut
-// into bands of R output rows of one strip of at most XT columns; each CTA of the cluster takes a
-// contiguous share of the bands.
-//   Phase 1: a producer lane moves each band with two TMA tile loads -- K rows y0-1 .. y0+R with a
-//     one-column halo, V rows y0 .. y0+R-1 -- into a shared-memory stage; the tensor map's
-//     out-of-bounds zero fill supplies the zero padding, so the inner loops carry no bounds checks.
-//     16 compute warps work from shared memory: warp w owns output row w / 8 of the band and an
-//     eighth of its columns, lane l owns channels 2l and 2l+1, and a 3 x 3 register window slides
-//     along the columns.
-//   Exchange: the warps' 64 x 9 gradients are summed in a fixed order into the CTA's partial, which
-//     is pushed with one bulk copy into every other CTA of the cluster (distributed shared memory,
-//     completion on the receiver's mbarrier); each CTA sums the CS partials in rank order (a fixed
-//     order: bitwise deterministic) and forms W1.  Meanwhile the producer keeps loading Q bands.
-//   Phase 2: the same band staging for Q; Z is written straight from registers (128 coalesced
-//     bytes per token and warp).
+// One kernel (dw_queue) of independent CTAs -- no clusters, so it fits whatever SMs are free, e.g.
+// next to the linear-head kernel of the same layer.  A unit's grid is cut into tasks of a few
+// row pairs of one strip of at most XT columns (no more gradient tasks than CTAs).  A CTA's producer lane claims tasks from a
+// global counter: first every gradient task (phase 1) of every unit, then every readout task
+// (phase 2).
+//   Streaming: the producer loads a task's rows as 2-row groups into two shared-memory rings: K (in
+//     phase 2: Q) groups with a one-column halo on both sides, and V groups.  Output row pair j of
+//     the task reads K groups j (rows 2j-1, 2j) and j+1 (rows 2j+1, 2j+2) and V group j.  The tensor
+//     map's out-of-bounds zero fill supplies the zero padding, so the inner loops carry no bounds
+//     checks.
+//   Compute: two groups of 8 warps take alternate row pairs; in a group, warp w owns a column
+//     segment of both rows of the pair, lane l owns channels 2l and 2l+1, and a 4 x 3 register window
+//     slides along the columns (unrolled by 3, so the window never moves between registers).  The
+//     residual is carried negated (s = V - W0 (*) K, from the negated taps), which saves a negation
+//     per token.
+//   Merge: a gradient task's 16 warps fold their 64 x 9 sums in a fixed order into the task's
+//     partial, written to the workspace slot of (unit, task).  The CTA that completes a unit's last
+//     gradient task sums the unit's partials in task order -- a fixed order, so W1 is bitwise
+//     reproducible whichever CTA ran which task -- writes W1 and raises the unit's ready flag.
+//   Readout tasks wait for that flag.  The wait cannot deadlock: tasks are claimed in order, so
+//     every gradient task of the unit was claimed earlier by a CTA that is running it.  Z is written
+//     straight from registers (128 coalesced bytes per token and warp).
+//   The last CTA to finish returns the workspace's counters and flags to zero for the next call.
+//   When launched as a programmatic dependent of the preceding kernel (the linear heads of the same
+//   layer), the kernel starts while that kernel runs and, at its very end, waits for it, so the
+//   stream sees both complete when this one does.
 #include <algorithm>
-#include <mutex>
 
 #include "sm100.cuh"
 #include "ttt_internal.h"
@@ -33,13 +43,15 @@ namespace dw {
 
 constexpr int D = 64;
 constexpr int TAPS = 9;
-constexpr int R = 2;                        // output rows per band
-constexpr int CW = 16;                      // compute warps
-constexpr int WPR = CW / R;                 // compute warps per output row
-constexpr int THREADS = (CW + 1) * 32;      // + one producer warp
+constexpr int GW = 6;                       // warps of a compute group (column segments of a row pair)
+constexpr int CG = 2;                       // compute groups (alternate row pairs)
+constexpr int CW = GW * CG;                 // compute warps
+constexpr int THREADS = (CW + 1) * 32;      // + one producer warp (13 warps: 128 registers a thread)
+constexpr int NK = 6;                       // K / Q ring slots (2-row groups)
+constexpr int NV = 4;                       // V ring slots (2-row groups)
+constexpr int NT = 4;                       // claimed tasks in flight (producer ahead of the compute warps)
 constexpr int kPart = D * TAPS;             // 576 floats: a 64 x 9 gradient or kernel, tap-major
-constexpr int kMaxCluster = 16;
-constexpr int STAGES = 2;
+constexpr int kRed = GW / 2;                // a group's per-warp gradients are folded pairwise into kRed slots
 
 template <typename T>
 struct Elem;
@@ -57,54 +69,83 @@ template <>
 struct Elem<float> {
     using Raw = float2;
     static constexpr int kTokenBytes = D * 4;
-    static constexpr int kXtMax = 40;
+    static constexpr int kXtMax = 38;
     static __device__ __forceinline__ float2 unpack(Raw w) { return w; }
     static __device__ __forceinline__ void store(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
 };
 
 struct Geom {
     int heads, H, W;
-    int Sx, XT, Hb;                  // strips, strip width, bands per strip
-    int bands_per_unit;              // Sx * Hb
+    int Sx, XT;                      // strips, strip width
+    int Hp;                          // row pairs per strip: ceil(H / 2)
+    int tps, tpu;                    // tasks per strip (each a contiguous range of row pairs), per unit
     long long bs, hs;                // element strides of Q/K/V/Z
     int k_pitch;                     // tokens per staged K/Q row (XT + 2)
-    uint32_t k_bytes, v_bytes;       // bytes of the staged K/Q rows and V rows of a band
-    uint32_t stage_bytes;
+    uint32_t kg_bytes, vg_bytes;     // one staged K/Q group (2 x k_pitch tokens), one V group (2 x XT)
 };
 
 struct Params {
     Geom g;
-    int U, CS;
+    int U;                           // units
+    int T1, T;                       // gradient tasks, all tasks
     float eta_scale;                 // eta * 2 / N
     const float* W0;                 // [heads][64][9]
     float* W1_out;                   // nullable [units][64][9]
-    uint32_t* err;
+    uint32_t* err;                   // workspace error word
+    uint32_t* queue;                 // task counter
+    uint32_t* done;                  // CTAs finished
+    uint32_t* unit_count;            // [U] gradient tasks finished per unit
+    uint32_t* ready;                 // [U] W1 of the unit is in w1g
+    float* partials;                 // [U][mtpu][CG][576] negated gradient sums per task and group, tap-major
+    int mtpu;                        // partial slots per unit (one task per row pair, the most a call uses)
+    float* w1g;                      // [U][576] W1 per unit, tap-major
 };
 
-struct Band {
-    int s, y0, xs, xe;               // strip, first output row, output columns [xs, xe)
+// Workspace layout: the 256-byte header (word 0: error word), the control words (queue, done,
+// unit_count[U], ready[U]) padded to 256 bytes, the partials, W1.
+struct WsLayout {
+    size_t ctl, partials, w1g, total;
 };
-
-__device__ __forceinline__ Band decode_band(const Geom& g, int b) {
-    Band r;
-    r.s = b / g.Hb;
-    r.y0 = (b % g.Hb) * R;
-    r.xs = r.s * g.XT;
-    r.xe = min(g.W, r.xs + g.XT);
-    return r;
+static WsLayout ws_layout(long long U, int tpu) {
+    WsLayout l;
+    l.ctl = kWsHeader;
+    l.partials = l.ctl + align_up((size_t)(2 + 2 * U) * 4, 256);
+    l.w1g = l.partials + align_up((size_t)U * tpu * CG * kPart * 4, 256);
+    l.total = l.w1g + (size_t)U * kPart * 4;
+    return l;
 }
 
-struct SmemTail {                            // follows the stages
-    float red[CW][kPart];                    // per-warp gradients (phase 1)
-    float recv[kMaxCluster - 1][kPart];      // the peers' partials
-    float mine[kPart];                       // this CTA's partial (sent to the peers)
-    float w1[kPart];                         // W1 of the unit, tap-major
-    uint64_t full[STAGES], empty[STAGES];
-    uint64_t recv_full, peer_free;
+struct SmemTail {                            // follows the rings
+    float red[CG][kRed][kPart];              // per-warp gradients of each group, folded pairwise
+    uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], tfull[NT], tempty[NT];
+    int task[NT];
+    int flag[CG];                            // per-group decision broadcast
     int abort_flag;
 };
 
-__device__ __forceinline__ int split_lo(int n, int r, int parts) { return (int)((long long)n * r / parts); }
+__host__ __device__ __forceinline__ int split_lo(int n, int r, int parts) { return (int)((long long)n * r / parts); }
+
+struct Task {
+    bool p1;
+    int u, r, sx, pa, n;                     // unit, task index in the unit, strip, first pair, pairs
+};
+
+__device__ __forceinline__ Task decode(const Params& p, int t) {
+    Task k;
+    k.p1 = t < p.T1;
+    const int tt = k.p1 ? t : t - p.T1;
+    k.u = tt / p.g.tpu;
+    k.r = tt % p.g.tpu;
+    k.sx = k.r / p.g.tps;
+    const int c = k.r % p.g.tps;
+    k.pa = split_lo(p.g.Hp, c, p.g.tps);
+    k.n = split_lo(p.g.Hp, c + 1, p.g.tps) - k.pa;
+    return k;
+}
+
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
+}
 
 // Channel pair `lane` of staged row `row`, column `col` (no bounds checks: the halo is staged).
 template <typename T>
@@ -113,305 +154,446 @@ __device__ __forceinline__ float2 staged(const uint8_t* base, int pitch, int row
         base + ((size_t)row * pitch + col) * Elem<T>::kTokenBytes)[lane]);
 }
 
+// The 4 staged rows around an output row pair: rows 0, 1 from one group, rows 2, 3 from the next.
+struct Rows {
+    const uint8_t* a;                // rows y0-1, y0
+    const uint8_t* b;                // rows y0+1, y0+2
+    int pitch;
+};
+
+template <typename T, int C>
+__device__ __forceinline__ void load_col(float2 (&win)[4][3], const Rows& rw, int col, int lane) {
+    win[0][C] = staged<T>(rw.a, rw.pitch, 0, col, lane);
+    win[1][C] = staged<T>(rw.a, rw.pitch, 1, col, lane);
+    win[2][C] = staged<T>(rw.b, rw.pitch, 0, col, lane);
+    win[3][C] = staged<T>(rw.b, rw.pitch, 1, col, lane);
+}
+
+// s = v + sum over the 3 x 3 taps of nw * K at window rows r0 .. r0+2, as three independent
+// 3-term chains (one per tap row) added at the end: a dependency depth of 5 instead of 9.
+template <int L, int M, int R>
+__device__ __forceinline__ float2 neg_residual(const float2 (&win)[4][3], const float2 (&nw)[TAPS], int r0, float2 v) {
+    constexpr int cidx[3] = {L, M, R};
+    const float2 zero = make_float2(0.f, 0.f);
+    float2 t0 = v, t1 = zero, t2 = zero;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+        t0 = ffma2(nw[c], win[r0][cidx[c]], t0);
+        t1 = ffma2(nw[3 + c], win[r0 + 1][cidx[c]], t1);
+        t2 = ffma2(nw[6 + c], win[r0 + 2][cidx[c]], t2);
+    }
+    return make_float2(t0.x + t1.x + t2.x, t0.y + t1.y + t2.y);
+}
+
+// Phase-1 work of output column x (strip-relative) of the row pair: window columns L, M, R hold
+// staged columns x, x+1, x+2 (image columns x-1, x, x+1); R is loaded here.  nw = -W0 taps;
+// gacc accumulates sum s * K with s = V - W0 (*) K = -r.
+template <typename T, bool ROW1, int L, int M, int R>
+__device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[TAPS], float2 (&gacc)[TAPS],
+                                       const Rows& rw, const uint8_t* vg, int XT, int x, int lane) {
+    using E = Elem<T>;
+    load_col<T, R>(win, rw, x + 2, lane);
+    const typename E::Raw* vr = reinterpret_cast<const typename E::Raw*>(vg);
+    constexpr int cidx[3] = {L, M, R};
+    const float2 s0 = neg_residual<L, M, R>(win, nw, 0, E::unpack(vr[(size_t)x * D / 2 + lane]));
+    if (ROW1) {                                            // the second row of the pair lies inside the grid
+        const float2 s1 = neg_residual<L, M, R>(win, nw, 1, E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]));
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                gacc[a * 3 + c] = ffma2(s0, win[a][cidx[c]], gacc[a * 3 + c]);
+                gacc[a * 3 + c] = ffma2(s1, win[a + 1][cidx[c]], gacc[a * 3 + c]);
+            }
+    } else {
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int c = 0; c < 3; ++c) gacc[a * 3 + c] = ffma2(s0, win[a][cidx[c]], gacc[a * 3 + c]);
+    }
+}
+
+template <typename T, bool ROW1>
+__device__ __forceinline__ void p1_pair(const float2 (&nw)[TAPS], float2 (&gacc)[TAPS], const Rows& rw,
+                                        const uint8_t* vg, int XT, int xa, int xb, int lane) {
+    float2 win[4][3];
+    load_col<T, 0>(win, rw, xa, lane);
+    load_col<T, 1>(win, rw, xa + 1, lane);
+    int x = xa;
+    for (; x + 3 <= xb; x += 3) {
+        p1_col<T, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
+        p1_col<T, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
+        p1_col<T, ROW1, 2, 0, 1>(win, nw, gacc, rw, vg, XT, x + 2, lane);
+    }
+    if (x < xb) {
+        p1_col<T, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
+        if (x + 1 < xb) p1_col<T, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
+    }
+}
+
+// Phase-2 work of output column x: z = W1 (*) Q for the rows of the pair.
+template <typename T, bool ROW1, int L, int M, int R>
+__device__ __forceinline__ void p2_col(float2 (&win)[4][3], const float2 (&w)[TAPS], const Rows& rw, T* z0, T* z1,
+                                       int x, int lane) {
+    load_col<T, R>(win, rw, x + 2, lane);
+    constexpr int cidx[3] = {L, M, R};
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            a0 = ffma2(w[a * 3 + c], win[a][cidx[c]], a0);
+            if (ROW1) a1 = ffma2(w[a * 3 + c], win[a + 1][cidx[c]], a1);
+        }
+    Elem<T>::store(z0 + (size_t)x * D, a0);
+    if (ROW1) Elem<T>::store(z1 + (size_t)x * D, a1);
+}
+
+template <typename T, bool ROW1>
+__device__ __forceinline__ void p2_pair(const float2 (&w)[TAPS], const Rows& rw, T* z0, T* z1, int xa, int xb,
+                                        int lane) {
+    float2 win[4][3];
+    load_col<T, 0>(win, rw, xa, lane);
+    load_col<T, 1>(win, rw, xa + 1, lane);
+    int x = xa;
+    for (; x + 3 <= xb; x += 3) {
+        p2_col<T, ROW1, 0, 1, 2>(win, w, rw, z0, z1, x, lane);
+        p2_col<T, ROW1, 1, 2, 0>(win, w, rw, z0, z1, x + 1, lane);
+        p2_col<T, ROW1, 2, 0, 1>(win, w, rw, z0, z1, x + 2, lane);
+    }
+    if (x < xb) {
+        p2_col<T, ROW1, 0, 1, 2>(win, w, rw, z0, z1, x, lane);
+        if (x + 1 < xb) p2_col<T, ROW1, 1, 2, 0>(win, w, rw, z0, z1, x + 1, lane);
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(THREADS, 1)
-dw_cluster(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-           const __grid_constant__ CUtensorMap tmQ, T* __restrict__ Z, const Params p) {
-    using E = Elem<T>;
+dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+         const __grid_constant__ CUtensorMap tmQ, T* __restrict__ Z, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const Geom& g = p.g;
-    uint8_t* stages = base;
-    SmemTail& s = *reinterpret_cast<SmemTail*>(base + (size_t)STAGES * g.stage_bytes);
+    uint8_t* kring = base;
+    uint8_t* vring = kring + (size_t)NK * g.kg_bytes;
+    SmemTail& s = *reinterpret_cast<SmemTail*>(vring + (size_t)NV * g.vg_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rank = (int)cluster_ctarank(), cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
-    const bool multi = p.CS > 1;
     const Abort ab{&s.abort_flag, p.err};
 
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
-        for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], CW); }
-        mbar_init(&s.recv_full, 1);
-        mbar_init(&s.peer_free, (uint32_t)(multi ? p.CS - 1 : 1));
+        // a K group is read by two row pairs, each by GW warps; a V group by one row pair
+        for (int i = 0; i < NK; ++i) { mbar_init(&s.kfull[i], 1); mbar_init(&s.kempty[i], 2 * GW); }
+        for (int i = 0; i < NV; ++i) { mbar_init(&s.vfull[i], 1); mbar_init(&s.vempty[i], GW); }
+        for (int i = 0; i < NT; ++i) { mbar_init(&s.tfull[i], 1); mbar_init(&s.tempty[i], CW); }
         fence_barrier_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ);
     }
     __syncthreads();
-    // every CTA's barriers exist before any peer arrives on them
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-
-    const int b_lo = split_lo(g.bands_per_unit, rank, p.CS), b_hi = split_lo(g.bands_per_unit, rank + 1, p.CS);
 
     if (warp == CW) {                                                // producer
         if (lane == 0) {
-            int st = 0; uint32_t ph = 0;
-            for (int u = cid; u < p.U; u += ncl) {
-                const int bi = u / g.heads, h = u % g.heads;
-                for (int b = b_lo; b < b_hi; ++b) {
-                    const Band bd = decode_band(g, b);
-                    if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
-                    uint8_t* sp = stages + (size_t)st * g.stage_bytes;
-                    mbar_arrive_expect_tx(&s.full[st], g.k_bytes + g.v_bytes);
-                    tma_load_5d(sp, &tmK, &s.full[st], 0, bd.xs - 1, bd.y0 - 1, h, bi);
-                    tma_load_5d(sp + g.k_bytes, &tmV, &s.full[st], 0, bd.xs, bd.y0, h, bi);
-                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+            uint32_t kq = 0, vq = 0, tq = 0;                         // ring sequence numbers
+            auto load_k = [&](const CUtensorMap* tm, int xs, int y, int h, int bi) -> bool {
+                const uint32_t sl = kq % NK, ph = (kq / NK) & 1u;
+                ++kq;
+                if (!mbar_wait(&s.kempty[sl], ph ^ 1u, ab)) return false;
+                mbar_arrive_expect_tx(&s.kfull[sl], g.kg_bytes);
+                tma_load_5d(kring + (size_t)sl * g.kg_bytes, tm, &s.kfull[sl], 0, xs - 1, y, h, bi);
+                return true;
+            };
+            auto load_v = [&](int xs, int y, int h, int bi) -> bool {
+                const uint32_t sl = vq % NV, ph = (vq / NV) & 1u;
+                ++vq;
+                if (!mbar_wait(&s.vempty[sl], ph ^ 1u, ab)) return false;
+                mbar_arrive_expect_tx(&s.vfull[sl], g.vg_bytes);
+                tma_load_5d(vring + (size_t)sl * g.vg_bytes, &tmV, &s.vfull[sl], 0, xs, y, h, bi);
+                return true;
+            };
+            for (;;) {
+                int t = (int)atomicAdd(p.queue, 1u);
+                if (t >= p.T) t = -1;
+                const uint32_t ts = tq % NT, tph = (tq / NT) & 1u;
+                ++tq;
+                if (!mbar_wait(&s.tempty[ts], tph ^ 1u, ab)) break;
+                s.task[ts] = t;
+                mbar_arrive(&s.tfull[ts]);
+                if (t < 0) break;
+                const Task tk = decode(p, t);
+                const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT, y0 = 2 * tk.pa;
+                bool ok = true;
+                if (tk.p1) {                                         // K(0), then K(j+1), V(j)
+                    ok = load_k(&tmK, xs, y0 - 1, h, bi);
+                    for (int j = 0; j < tk.n && ok; ++j)
+                        ok = load_k(&tmK, xs, y0 + 2 * j + 1, h, bi) && load_v(xs, y0 + 2 * j, h, bi);
+                } else {
+                    for (int j = 0; j <= tk.n && ok; ++j) ok = load_k(&tmQ, xs, y0 + 2 * j - 1, h, bi);
                 }
-                // Q does not depend on W1: it streams in while the cluster exchanges its partials.
-                for (int b = b_lo; b < b_hi; ++b) {
-                    const Band bd = decode_band(g, b);
-                    if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
-                    uint8_t* sp = stages + (size_t)st * g.stage_bytes;
-                    mbar_arrive_expect_tx(&s.full[st], g.k_bytes);
-                    tma_load_5d(sp, &tmQ, &s.full[st], 0, bd.xs - 1, bd.y0 - 1, h, bi);
-                    if (++st == STAGES) { st = 0; ph ^= 1u; }
-                }
+                if (!ok) break;
             }
         }
         return;
     }
 
-    // compute warps
+    // compute warps: two groups of GW warps; group g takes the row pairs j = g (mod CG) of every task
+    // (a fixed split, so each partial holds the same sums whichever CTA runs the task) and publishes
+    // its own partial, so the groups never wait for one another
     const int tid = threadIdx.x;                                     // 0 .. CW*32-1
-    const int orow = warp / WPR, oseg = warp % WPR;
-    int st = 0; uint32_t ph = 0;
-    uint32_t k = 0;
+    const int grp = warp / GW, seg = warp % GW, gtid = tid - grp * GW * 32;
+    const uint32_t gbar = 1u + (uint32_t)grp;                        // the group's named barrier
+    uint32_t kq = 0, vq = 0, tq = 0;                                 // ring and task sequence numbers
     bool failed = false;
-    for (int u = cid; u < p.U && !failed; u += ncl, ++k) {
-        const int bi = u / g.heads, h = u % g.heads;
-        if (multi && tid == 0) {                                     // my receive slots are free: arm, then tell the peers
-            mbar_arrive_expect_tx(&s.recv_full, (uint32_t)((p.CS - 1) * kPart * 4));
-            for (int pr = 0; pr < p.CS; ++pr)
-                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
-        }
-        float2 w[TAPS], gacc[TAPS];
+    for (;;) {
+        const uint32_t ts = tq % NT, tph = (tq / NT) & 1u;
+        ++tq;
+        const bool okt = !failed && mbar_wait(&s.tfull[ts], tph, ab);
+        const int t = okt ? s.task[ts] : -1;
+        __syncwarp();
+        if (okt && lane == 0) mbar_arrive(&s.tempty[ts]);
+        // the warps of a group take the same decision: stop on a failure anywhere in the group
+        if (named_bar_or(gbar, GW * 32, failed || !okt)) { failed = true; break; }
+        if (t < 0) break;
+        const Task tk = decode(p, t);
+        const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT;
+        const int cols = min(g.W - xs, g.XT), segw = (cols + GW - 1) / GW;
+        const int xa = seg * segw, xb = min(cols, xa + segw);        // strip-relative output columns
+        const int n = tk.n;
+        if (tk.p1) {
+            // ---- phase-1 task: negated gradient sums over this group's row pairs of the task
+            float2 nw[TAPS], gacc[TAPS];
 #pragma unroll
-        for (int t = 0; t < TAPS; ++t) {
-            w[t] = make_float2(__ldg(p.W0 + ((size_t)h * D + 2 * lane) * TAPS + t),
-                               __ldg(p.W0 + ((size_t)h * D + 2 * lane + 1) * TAPS + t));
-            gacc[t] = make_float2(0.f, 0.f);
-        }
-        // ---- phase 1
-        for (int b = b_lo; b < b_hi; ++b) {
-            const Band bd = decode_band(g, b);
-            const bool okb = mbar_wait(&s.full[st], ph, ab);
-            __syncwarp();
-            const uint8_t* sp = stages + (size_t)st * g.stage_bytes;
-            const int y = bd.y0 + orow;
-            const int cols = bd.xe - bd.xs, segw = (cols + WPR - 1) / WPR;
-            const int xa = oseg * segw, xb = min(cols, xa + segw);      // strip-relative output columns
-            if (okb && y < g.H && xa < xb) {
-                const uint8_t* vrow = sp + g.k_bytes + (size_t)orow * g.XT * E::kTokenBytes;
-                float2 win[3][3];
-#pragma unroll
-                for (int a = 0; a < 3; ++a) {
-                    win[a][0] = staged<T>(sp, g.k_pitch, orow + a, xa, lane);
-                    win[a][1] = staged<T>(sp, g.k_pitch, orow + a, xa + 1, lane);
+            for (int t9 = 0; t9 < TAPS; ++t9) {
+                nw[t9] = make_float2(-__ldg(p.W0 + ((size_t)h * D + 2 * lane) * TAPS + t9),
+                                     -__ldg(p.W0 + ((size_t)h * D + 2 * lane + 1) * TAPS + t9));
+                gacc[t9] = make_float2(0.f, 0.f);
+            }
+            for (int j = 0; j < n; ++j) {
+                if (j % CG != grp || failed) continue;
+                const uint32_t k0 = kq + j, k1 = kq + j + 1, v0 = vq + j;
+                bool okb = mbar_wait(&s.kfull[k0 % NK], (k0 / NK) & 1u, ab);
+                okb = okb && mbar_wait(&s.kfull[k1 % NK], (k1 / NK) & 1u, ab);
+                okb = okb && mbar_wait(&s.vfull[v0 % NV], (v0 / NV) & 1u, ab);
+                if (!okb) { failed = true; continue; }
+                __syncwarp();
+                if (xa < xb) {
+                    const Rows rw{kring + (size_t)(k0 % NK) * g.kg_bytes, kring + (size_t)(k1 % NK) * g.kg_bytes,
+                                  g.k_pitch};
+                    const uint8_t* vg = vring + (size_t)(v0 % NV) * g.vg_bytes;
+                    if (2 * (tk.pa + j) + 1 < g.H) p1_pair<T, true>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
+                    else p1_pair<T, false>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
                 }
-                for (int x = xa; x < xb; ++x) {
-#pragma unroll
-                    for (int a = 0; a < 3; ++a) win[a][2] = staged<T>(sp, g.k_pitch, orow + a, x + 2, lane);
-                    const float2 v =
-                        E::unpack(reinterpret_cast<const typename E::Raw*>(vrow + (size_t)x * E::kTokenBytes)[lane]);
-                    float2 r = make_float2(-v.x, -v.y);
-#pragma unroll
-                    for (int a = 0; a < 3; ++a)
-#pragma unroll
-                        for (int c = 0; c < 3; ++c) r = ffma2(w[a * 3 + c], win[a][c], r);
-#pragma unroll
-                    for (int a = 0; a < 3; ++a)
-#pragma unroll
-                        for (int c = 0; c < 3; ++c) gacc[a * 3 + c] = ffma2(r, win[a][c], gacc[a * 3 + c]);
-#pragma unroll
-                    for (int a = 0; a < 3; ++a) { win[a][0] = win[a][1]; win[a][1] = win[a][2]; }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_n(&s.kempty[k0 % NK], j == 0 ? 2u : 1u);          // group 0 has one reader pair
+                    mbar_arrive_n(&s.kempty[k1 % NK], j == n - 1 ? 2u : 1u);      // so has the last group
+                    mbar_arrive(&s.vempty[v0 % NV]);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.empty[st]);
-            if (++st == STAGES) { st = 0; ph ^= 1u; }
-        }
-        // ---- the CTA's partial, in a fixed order over the warps
-        bool ok = true;
-        if (multi) ok = mbar_wait_cluster(&s.peer_free, k & 1u, ab);  // my last pushes have landed
+            kq += (uint32_t)n + 1; vq += (uint32_t)n;
+            // ---- the group's partial, summed over its warps in a fixed order
+            float(*red)[kPart] = s.red[grp];
+            if (seg >= kRed) {
 #pragma unroll
-        for (int t = 0; t < TAPS; ++t) *reinterpret_cast<float2*>(&s.red[warp][t * D + 2 * lane]) = gacc[t];
-        if (named_bar_or(1, CW * 32, !ok)) { failed = true; break; }
-        for (int e = tid; e < kPart; e += CW * 32) {
-            float acc = 0.f;
+                for (int t9 = 0; t9 < TAPS; ++t9)
+                    *reinterpret_cast<float2*>(&red[seg - kRed][t9 * D + 2 * lane]) = gacc[t9];
+            }
+            named_bar_sync(gbar, GW * 32);
+            if (seg < kRed) {
 #pragma unroll
-            for (int ww = 0; ww < CW; ++ww) acc += s.red[ww][e];
-            s.mine[e] = acc;
-        }
-        // ---- exchange with the cluster, then W1 = W0 - eta (2/N) sum_r partial_r (rank order)
-        if (multi) {
-            fence_proxy_async_smem();                                // `mine` is read by the bulk-copy engine
-            named_bar_sync(1, CW * 32);
-            if (tid == 0)
-                for (int pr = 0; pr < p.CS; ++pr) {
-                    if (pr == rank) continue;
-                    const int slot = (rank < pr) ? rank : rank - 1;
-                    bulk_s2cluster(map_to_rank(smem_u32(s.recv[slot]), (uint32_t)pr), s.mine, kPart * 4,
-                                   map_to_rank(smem_u32(&s.recv_full), (uint32_t)pr));
-                }
-            ok = mbar_wait_cluster(&s.recv_full, k & 1u, ab);
-        }
-        if (named_bar_or(1, CW * 32, !ok)) { failed = true; break; }
-        for (int e = tid; e < kPart; e += CW * 32) {
-            float acc = 0.f;
-            for (int pr = 0; pr < p.CS; ++pr) acc += (pr == rank) ? s.mine[e] : s.recv[(pr < rank) ? pr : pr - 1][e];
-            const int t = e / D, ch = e % D;                        // tap-major index
-            const float w1 = __ldg(p.W0 + ((size_t)h * D + ch) * TAPS + t) - p.eta_scale * acc;
-            s.w1[e] = w1;
-            if (p.W1_out && rank == 0) p.W1_out[((size_t)u * D + ch) * TAPS + t] = w1;
-        }
-        named_bar_sync(1, CW * 32);
-#pragma unroll
-        for (int t = 0; t < TAPS; ++t) w[t] = *reinterpret_cast<const float2*>(&s.w1[t * D + 2 * lane]);
-        // ---- phase 2
-        const long long off = (long long)bi * g.bs + (long long)h * g.hs;
-        for (int b = b_lo; b < b_hi; ++b) {
-            const Band bd = decode_band(g, b);
-            if (!mbar_wait(&s.full[st], ph, ab)) { failed = true; break; }   // no CTA barrier follows
-            __syncwarp();
-            const uint8_t* sp = stages + (size_t)st * g.stage_bytes;
-            const int y = bd.y0 + orow;
-            const int cols = bd.xe - bd.xs, segw = (cols + WPR - 1) / WPR;
-            const int xa = oseg * segw, xb = min(cols, xa + segw);
-            if (y < g.H && xa < xb) {
-                T* zrow = Z + off + ((long long)y * g.W + bd.xs) * D + 2 * lane;
-                float2 win[3][3];
-#pragma unroll
-                for (int a = 0; a < 3; ++a) {
-                    win[a][0] = staged<T>(sp, g.k_pitch, orow + a, xa, lane);
-                    win[a][1] = staged<T>(sp, g.k_pitch, orow + a, xa + 1, lane);
-                }
-                for (int x = xa; x < xb; ++x) {
-#pragma unroll
-                    for (int a = 0; a < 3; ++a) win[a][2] = staged<T>(sp, g.k_pitch, orow + a, x + 2, lane);
-                    float2 z = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int a = 0; a < 3; ++a)
-#pragma unroll
-                        for (int c = 0; c < 3; ++c) z = ffma2(w[a * 3 + c], win[a][c], z);
-                    E::store(zrow + (long long)x * D, z);
-#pragma unroll
-                    for (int a = 0; a < 3; ++a) { win[a][0] = win[a][1]; win[a][1] = win[a][2]; }
+                for (int t9 = 0; t9 < TAPS; ++t9) {
+                    float2* q = reinterpret_cast<float2*>(&red[seg][t9 * D + 2 * lane]);
+                    const float2 o = *q;
+                    *q = make_float2(gacc[t9].x + o.x, gacc[t9].y + o.y);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.empty[st]);
-            if (++st == STAGES) { st = 0; ph ^= 1u; }
+            named_bar_sync(gbar, GW * 32);
+            float* part = p.partials + (((size_t)tk.u * p.mtpu + tk.r) * CG + grp) * kPart;
+            for (int e = gtid; e < kPart; e += GW * 32) {
+                float acc = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < kRed; ++ww) acc += red[ww][e];
+                part[e] = acc;
+            }
+            __threadfence();
+            named_bar_sync(gbar, GW * 32);
+            if (gtid == 0) s.flag[grp] = (atomicAdd(p.unit_count + tk.u, 1u) == (uint32_t)(g.tpu * CG - 1)) ? 1 : 0;
+            named_bar_sync(gbar, GW * 32);
+            if (s.flag[grp]) {
+                // ---- the unit's last partial: W1 = W0 - eta (2/N) g = W0 + eta_scale * (sum of the
+                //      partials in (task, group) order)
+                __threadfence();
+                const float* pu = p.partials + (size_t)tk.u * p.mtpu * CG * kPart;
+                const int R = g.tpu * CG;
+                for (int e4 = gtid; e4 < kPart / 4; e4 += GW * 32) {
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int r0 = 0; r0 < R; r0 += 8) {                // 8 loads in flight, added in order
+                        float4 v[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            v[q] = (r0 + q < R) ? __ldcg(reinterpret_cast<const float4*>(pu + (size_t)(r0 + q) * kPart) + e4)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            if (r0 + q < R) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
+                    }
+                    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = 4 * e4 + i, t9 = e / D, ch = e % D;   // tap-major index
+                        const float w1 = __ldg(p.W0 + ((size_t)h * D + ch) * TAPS + t9) + p.eta_scale * a4[i];
+                        p.w1g[(size_t)tk.u * kPart + e] = w1;
+                        if (p.W1_out) p.W1_out[((size_t)tk.u * D + ch) * TAPS + t9] = w1;
+                    }
+                }
+                __threadfence();
+                named_bar_sync(gbar, GW * 32);
+                if (gtid == 0) st_release_gpu(p.ready + tk.u, 1u);
+            }
+        } else {
+            // ---- phase-2 task: Z = W1 (*) Q over this group's row pairs of the task
+            float2 w[TAPS];
+            if (!wait_flag(p.ready + tk.u, ab)) failed = true;
+#pragma unroll
+            for (int t9 = 0; t9 < TAPS; ++t9)
+                w[t9] = __ldcg(reinterpret_cast<const float2*>(p.w1g + (size_t)tk.u * kPart + t9 * D) + lane);
+            const long long off = (long long)bi * g.bs + (long long)h * g.hs;
+            for (int j = 0; j < n; ++j) {
+                if (j % CG != grp || failed) continue;
+                const uint32_t k0 = kq + j, k1 = kq + j + 1;
+                bool okb = mbar_wait(&s.kfull[k0 % NK], (k0 / NK) & 1u, ab);
+                okb = okb && mbar_wait(&s.kfull[k1 % NK], (k1 / NK) & 1u, ab);
+                if (!okb) { failed = true; continue; }
+                __syncwarp();
+                const int y0 = 2 * (tk.pa + j);
+                if (xa < xb) {
+                    const Rows rw{kring + (size_t)(k0 % NK) * g.kg_bytes, kring + (size_t)(k1 % NK) * g.kg_bytes,
+                                  g.k_pitch};
+                    T* z0 = Z + off + ((long long)y0 * g.W + xs) * D + 2 * lane;
+                    T* z1 = z0 + (long long)g.W * D;
+                    if (y0 + 1 < g.H) p2_pair<T, true>(w, rw, z0, z1, xa, xb, lane);
+                    else p2_pair<T, false>(w, rw, z0, z1, xa, xb, lane);
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_n(&s.kempty[k0 % NK], j == 0 ? 2u : 1u);
+                    mbar_arrive_n(&s.kempty[k1 % NK], j == n - 1 ? 2u : 1u);
+                }
+            }
+            kq += (uint32_t)n + 1;
         }
     }
-    // Final handshake: once every peer has finished its last unit, all of this CTA's pushes have
-    // landed and nobody will push into it again; only then may it exit.
-    if (multi && !failed) {
-        named_bar_sync(1, CW * 32);
-        if (tid == 0)
-            for (int pr = 0; pr < p.CS; ++pr)
-                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
-        mbar_wait_cluster(&s.peer_free, k & 1u, ab);
+    // The last CTA to finish puts the control words back to zero for the next call.
+    named_bar_sync(3, CW * 32);
+    if (tid == 0) {
+        __threadfence();
+        s.flag[0] = (atomicAdd(p.done, 1u) == gridDim.x - 1) ? 1 : 0;
     }
+    named_bar_sync(3, CW * 32);
+    if (s.flag[0]) {
+        __threadfence();
+        for (int i = tid; i < p.U; i += CW * 32) { p.unit_count[i] = 0u; p.ready[i] = 0u; }
+        if (tid == 0) { *p.queue = 0u; *p.done = 0u; }
+    }
+    // As a programmatic dependent of the preceding kernel: complete only after it has completed.
+    pdl_wait_primary();
 }
 
 // ------------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------------
+// Tasks per strip: as many as keep the gradient tasks of the call within `grid` CTAs (one each), so
+// that no CTA runs two of them one after the other; at most one task per row pair.
 template <typename T>
-static Geom make_geom(const Call& c) {
+static Geom make_geom(long long units, int grid, int heads, int H, int W, long long bs, long long hs) {
     constexpr int TB = Elem<T>::kTokenBytes;
     Geom g;
-    g.heads = c.heads;
-    g.H = c.H;
-    g.W = c.W;
-    g.Sx = (c.W + Elem<T>::kXtMax - 1) / Elem<T>::kXtMax;
-    g.XT = (c.W + g.Sx - 1) / g.Sx;
-    g.Hb = (c.H + R - 1) / R;
-    g.bands_per_unit = g.Sx * g.Hb;
-    g.bs = c.bs;
-    g.hs = c.hs;
+    g.heads = heads;
+    g.H = H;
+    g.W = W;
+    g.Sx = (W + Elem<T>::kXtMax - 1) / Elem<T>::kXtMax;
+    g.XT = (W + g.Sx - 1) / g.Sx;
+    g.Hp = (H + 1) / 2;
+    g.tps = (int)std::min<long long>(g.Hp, std::max<long long>(1, grid / std::max<long long>(1, units * g.Sx)));
+    g.tpu = g.Sx * g.tps;
+    g.bs = bs;
+    g.hs = hs;
     g.k_pitch = g.XT + 2;
-    g.k_bytes = (uint32_t)((R + 2) * g.k_pitch * TB);
-    g.v_bytes = (uint32_t)(R * g.XT * TB);
-    g.stage_bytes = (g.k_bytes + g.v_bytes + 127u) & ~127u;
+    g.kg_bytes = (uint32_t)(2 * g.k_pitch * TB);
+    g.vg_bytes = (uint32_t)(2 * g.XT * TB);
     return g;
 }
 
 template <typename T>
-static int max_active_clusters(int cs, size_t smem) {
-    static std::mutex mu;
-    static int cache[64][kMaxCluster + 1];
-    static bool init = false;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) { cudaGetLastError(); return 0; }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!init) {
-        for (auto& row : cache)
-            for (int& v : row) v = -1;
-        init = true;
-    }
-    if (cache[dev][cs] < 0) {
-        cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3(cs * 16);
-        cfg.blockDim = dim3(THREADS);
-        cfg.dynamicSmemBytes = smem;
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = cs; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, (void*)dw_cluster<T>, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            n = 0;
-        }
-        cache[dev][cs] = n;
-    }
-    return cache[dev][cs];
+static size_t smem_bytes(const Geom& g) {
+    return 128 + (size_t)NK * g.kg_bytes + (size_t)NV * g.vg_bytes + sizeof(SmemTail);
+}
+
+// Partial slots a unit may need: one task per row pair of every strip (the workspace is sized for
+// that, so that its size does not depend on the grid).
+static int max_tasks_per_unit(const ttt_shape& s) {
+    const int xt = (s.dtype == TTT_BF16) ? Elem<__nv_bfloat16>::kXtMax : Elem<float>::kXtMax;
+    return ((s.W + xt - 1) / xt) * ((s.H + 1) / 2);
 }
 
 template <typename T>
 static ttt_status launch(const Call& c) {
     const long long units = (long long)c.batch * c.heads;
-    const Geom g = make_geom<T>(c);
-    const size_t smem = 128 + (size_t)STAGES * g.stage_bytes + sizeof(SmemTail);
+    const int grid_max = std::max(1, c.num_sms);
+    const Geom g = make_geom<T>(units, grid_max, c.heads, c.H, c.W, c.bs, c.hs);
+    const size_t smem = smem_bytes<T>(g);
     if (smem > 227 * 1024) return TTT_ERR_UNSUPPORTED;
-    cudaFuncSetAttribute(dw_cluster<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(dw_cluster<T>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    // CTAs per cluster: spread each unit over up to 16 SMs while every cluster stays co-resident.
-    int cs = (int)std::max<long long>(1, std::min<long long>(kMaxCluster, c.num_sms / std::max<long long>(1, units)));
-    cs = std::min(cs, g.bands_per_unit);
-    while (cs > 1 && max_active_clusters<T>(cs, smem) < (int)std::min<long long>(units, c.num_sms / cs)) --cs;
-    const int ncl = (int)std::min<long long>(units, cs == 1 ? c.num_sms : c.num_sms / cs);
+    const WsLayout L = ws_layout(units, g.Sx * g.Hp);
+    if (c.ws_bytes < L.total) return TTT_ERR_WORKSPACE;
+    cudaFuncSetAttribute(dw_queue<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const long long T_all = 2 * units * g.tpu;
+    if (T_all > (1LL << 30)) return TTT_ERR_UNSUPPORTED;
+    const int grid = (int)std::max<long long>(1, std::min<long long>(grid_max, T_all));
 
     CUtensorMap tmK, tmV, tmQ;
-    if (!make_tmap_grid(&tmK, c.K, c, g.XT + 2, R + 2) || !make_tmap_grid(&tmV, c.V, c, g.XT, R) ||
-        !make_tmap_grid(&tmQ, c.Q, c, g.XT + 2, R + 2))
+    if (!make_tmap_grid(&tmK, c.K, c, g.k_pitch, 2) || !make_tmap_grid(&tmV, c.V, c, g.XT, 2) ||
+        !make_tmap_grid(&tmQ, c.Q, c, g.k_pitch, 2))
         return TTT_ERR_INVALID_ARG;
     Params p;
     p.g = g;
     p.U = (int)units;
-    p.CS = cs;
+    p.T1 = (int)(units * g.tpu);
+    p.T = (int)T_all;
     p.eta_scale = c.eta * (2.0f / (float)c.N);
     p.W0 = c.W0;
     p.W1_out = c.W1_out;
-    p.err = reinterpret_cast<uint32_t*>(c.ws);
+    p.err = reinterpret_cast<uint32_t*>(c.err_ws ? c.err_ws : c.ws);
+    uint32_t* ctl = reinterpret_cast<uint32_t*>(c.ws + L.ctl);
+    p.queue = ctl;
+    p.done = ctl + 1;
+    p.unit_count = ctl + 2;
+    p.ready = ctl + 2 + units;
+    p.partials = reinterpret_cast<float*>(c.ws + L.partials);
+    p.mtpu = g.Sx * g.Hp;
+    p.w1g = reinterpret_cast<float*>(c.ws + L.w1g);
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)(ncl * cs));
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = c.stream;
     cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = cs; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return check_launch(cudaLaunchKernelEx(&cfg, dw_cluster<T>, tmK, tmV, tmQ, static_cast<T*>(c.Z), p));
+    cfg.numAttrs = c.overlap_previous ? 1 : 0;
+    return check_launch(cudaLaunchKernelEx(&cfg, dw_queue<T>, tmK, tmV, tmQ, static_cast<T*>(c.Z), p));
 }
 
 }  // namespace dw
 
-// The cluster kernel keeps every intermediate on chip: the workspace is the error word only.
-size_t dwconv_ws_bytes(const ttt_shape&) { return kWsHeader; }
+size_t dwconv_ws_bytes(const ttt_shape& s) {
+    const long long units = (long long)s.batch * s.heads;
+    return dw::ws_layout(units, dw::max_tasks_per_unit(s)).total;
+}
+
+size_t dwconv_ws_control_bytes(const ttt_shape& s) {
+    const long long units = (long long)s.batch * s.heads;
+    return dw::ws_layout(units, dw::max_tasks_per_unit(s)).partials;
+}
 
 ttt_status launch_dwconv(const Call& c) {
     if (c.dtype == TTT_BF16) return dw::launch<__nv_bfloat16>(c);

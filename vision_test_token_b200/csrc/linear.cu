@@ -562,6 +562,9 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     cluster_sync_all();                  // every CTA's barriers exist before any peer arrives on them
+    // A kernel queued behind this one as a programmatic dependent (the conv heads of the same layer)
+    // may start once every CTA of this grid is resident: it takes the SMs this grid leaves free.
+    pdl_launch_dependents();
     const uint32_t tmem = s.tmem_base;
 
     if (warp == 0) {

@@ -34,7 +34,9 @@ struct Call {
     uint8_t* ws;
     size_t ws_bytes;
     cudaStream_t stream;
-    int num_sms;
+    int num_sms;             // SMs the call may spread its work over
+    int overlap_previous;    // launch as a programmatic dependent of the preceding kernel in the stream
+    uint8_t* err_ws;         // workspace whose error word the kernels report to (nullptr: ws itself)
 };
 
 // Encodes a rank-4 bf16 tensor map over [batch][heads][N][64] with a 64 x box_rows box,
@@ -53,6 +55,8 @@ size_t linear_ws_control_bytes(const ttt_shape& s);
 ttt_status launch_linear(const Call& c);
 
 size_t dwconv_ws_bytes(const ttt_shape& s);
+// Bytes at the start of a conv workspace that must be zero before a call (every call leaves them zero).
+size_t dwconv_ws_control_bytes(const ttt_shape& s);
 ttt_status launch_dwconv(const Call& c);
 
 size_t mlp_ws_bytes(const ttt_shape& s);

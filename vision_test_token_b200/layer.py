@@ -23,7 +23,7 @@ def _stream_handle(stream):
     return s.cuda_stream
 
 
-def _shape_of(Q, H, W, hidden=0):
+def _shape_of(Q, H, W, hidden=0, max_sms=0):
     if Q.dim() != 4:
         raise ValueError("Q/K/V must be [B][heads][N][d]")
     B, heads, N, d = Q.shape
@@ -33,7 +33,7 @@ def _shape_of(Q, H, W, hidden=0):
         raise ValueError("token rows of Q/K/V/Z must be contiguous")
     if Q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {Q.dtype}")
-    return capi.make_shape(B, heads, H, W, d, Q.stride(0), Q.stride(1), _DTYPES[Q.dtype], hidden)
+    return capi.make_shape(B, heads, H, W, d, Q.stride(0), Q.stride(1), _DTYPES[Q.dtype], hidden, max_sms)
 
 
 def _same_layout(ref, *others):
@@ -68,9 +68,10 @@ def _out_like(Q, Z):
     return Z
 
 
-def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None):
-    """Linear inner model.  W0: [heads][d][d] fp32 CUDA tensor.  Returns Z."""
-    shape = _shape_of(Q, H, W)
+def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0):
+    """Linear inner model.  W0: [heads][d][d] fp32 CUDA tensor.  Returns Z.  `max_sms` (0 = all)
+    bounds the SMs the call spreads over."""
+    shape = _shape_of(Q, H, W, max_sms=max_sms)
     Z = _out_like(Q, Z)
     _same_layout(Q, K, V, Z)
     W0 = W0.contiguous()
@@ -82,9 +83,9 @@ def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=
     return Z
 
 
-def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None):
+def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0):
     """3x3 depthwise-conv inner model.  W0: [heads][d][3][3] fp32 CUDA tensor.  Returns Z."""
-    shape = _shape_of(Q, H, W)
+    shape = _shape_of(Q, H, W, max_sms=max_sms)
     Z = _out_like(Q, Z)
     _same_layout(Q, K, V, Z)
     W0 = W0.contiguous()
@@ -96,9 +97,9 @@ def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=
     return Z
 
 
-def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws=None, stream=None):
+def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws=None, stream=None, max_sms=0):
     """One-hidden-layer GELU MLP inner model.  Wa: [heads][hidden][d], Wb: [heads][d][hidden]."""
-    shape = _shape_of(Q, H, W, hidden=Wa.shape[1])
+    shape = _shape_of(Q, H, W, hidden=Wa.shape[1], max_sms=max_sms)
     Z = _out_like(Q, Z)
     _same_layout(Q, K, V, Z)
     Wa, Wb = Wa.contiguous(), Wb.contiguous()
@@ -110,18 +111,47 @@ def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws
     return Z
 
 
-def forward_layer(Q, K, V, weights, eta, H, W, conv_heads=0, Z=None, ws_lin=None, ws_conv=None, stream=None):
+def layer_workspace(shape, conv_heads, device):
+    """A zero-initialised workspace for ttt_forward_layer(shape, conv_heads), cached and reused."""
+    nbytes = capi.ttt_layer_workspace_bytes(shape, conv_heads)
+    if nbytes == 0:
+        raise capi.TttError(capi.TTT_ERR_INVALID_ARG, "ttt_layer_workspace_bytes")
+    key = ("layer", str(device), nbytes)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def forward_layer(Q, K, V, weights, eta, H, W, conv_heads=0, Z=None, W1_lin_out=None, W1_conv_out=None, ws=None,
+                  stream=None, concurrent=True, max_sms=0):
     """A layer whose first heads are linear and whose last `conv_heads` heads are depthwise-conv
-    heads: two library calls on the same stream over head slices of the same buffers."""
+    heads, over head ranges of the same buffers.  weights: {"W0_lin": [heads-conv_heads][d][d],
+    "W0_conv": [conv_heads][d][3][3]}.  With `concurrent` (the default) one ttt_forward_layer call
+    runs both kernels at the same time; otherwise ttt_forward_linear and ttt_forward_dwconv run one
+    after the other on the stream."""
     Z = _out_like(Q, Z)
+    _same_layout(Q, K, V, Z)
     heads = Q.shape[1]
     nl = heads - conv_heads
+    W0l = weights["W0_lin"].contiguous() if nl else None
+    W0c = weights["W0_conv"].contiguous() if conv_heads else None
+    if concurrent:
+        shape = _shape_of(Q, H, W, max_sms=max_sms)
+        if ws is None:
+            ws = layer_workspace(shape, conv_heads, Q.device)
+        st = capi.ttt_forward_layer(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0l), _ptr(W0c), _ptr(Z), float(eta), shape,
+                                    conv_heads, _ptr(ws), ws.numel(), _ptr(W1_lin_out), _ptr(W1_conv_out),
+                                    _stream_handle(stream))
+        _check(st, "ttt_forward_layer")
+        return Z
     if nl:
-        forward_linear(Q[:, :nl], K[:, :nl], V[:, :nl], weights["W0_lin"], eta, H, W, Z=Z[:, :nl], ws=ws_lin,
-                       stream=stream)
+        forward_linear(Q[:, :nl], K[:, :nl], V[:, :nl], W0l, eta, H, W, Z=Z[:, :nl], W1_out=W1_lin_out,
+                       stream=stream, max_sms=max_sms)
     if conv_heads:
-        forward_dwconv(Q[:, nl:], K[:, nl:], V[:, nl:], weights["W0_conv"], eta, H, W, Z=Z[:, nl:], ws=ws_conv,
-                       stream=stream)
+        forward_dwconv(Q[:, nl:], K[:, nl:], V[:, nl:], W0c, eta, H, W, Z=Z[:, nl:], W1_out=W1_conv_out,
+                       stream=stream, max_sms=max_sms)
     return Z
 
 
