@@ -567,10 +567,15 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     pdl_launch_dependents();
     const uint32_t tmem = s.tmem_base;
 
+    // Lane 0 of warps 0 and 1 carries the producer and MMA roles; the rest of each warp waits for it
+    // here, so that every warp reaches the block barrier below converged (a block barrier reached by
+    // a partly diverged warp does not hold the warp's other lanes).
     if (warp == 0) {
         if (lane == 0) cl_producer(s, p, &tmK, &tmV, &tmQ, rank, cid, ncl, ab);
+        __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) cl_mma(s, p, tmem, rank, cid, ncl, ab);
+        __syncwarp();
     } else {
         cl_epilogue(s, p, tmem, &tmZ, rank, cid, ncl, ab);
     }

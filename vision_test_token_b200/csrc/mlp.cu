@@ -134,6 +134,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                 }
             }
         }
+        __syncwarp();                                          // the warp reaches the block barrier converged
     } else {
         // ---------------------------------------------------------------------------------------
         // warps 1..4: tid 0 issues the MMAs, all 128 threads do the elementwise work.  Thread tid
