@@ -159,9 +159,10 @@ ttt_status ttt_forward_linear_noalloc(const void* Q, const void* K, const void* 
  * ttt_forward_linear on the first range and ttt_forward_dwconv on the second, with the same results.
  * Both kernels run at the same time: the linear kernel is given a share of the SMs in proportion to
  * its heads' work (a conv head counting as two linear heads); the conv kernel is queued behind it as
- * a programmatic dependent, starts as soon as every linear CTA is resident, takes the SMs left free
- * and then those the linear kernel releases.  The call is complete on `stream` when both kernels are.
- * Results equal those of the two separate calls with the same SM budgets.
+ * a programmatic dependent, starts as soon as every linear CTA is resident and runs on the SMs the
+ * linear kernel leaves free (its work split for that many CTAs).  The call is complete on `stream`
+ * when both kernels are.  Results equal those of the two separate calls given the same SM budgets
+ * (linear: its share; conv: the SMs left to it).
  *   W0_lin: [heads - conv_heads][d][d], W0_conv: [conv_heads][d][3][3] (each may be NULL when its
  *   range is empty).  W1_lin_out / W1_conv_out: optional, as in the two calls above.
  *   ws: ttt_layer_workspace_bytes(s, conv_heads) bytes, zero-filled once (ttt_workspace_init); its

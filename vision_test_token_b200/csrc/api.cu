@@ -176,6 +176,7 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
     c->num_sms = (s->max_sms > 0 && s->max_sms < sms) ? s->max_sms : sms;
     c->overlap_previous = 0;
     c->err_ws = nullptr;
+    c->grid_out = nullptr;
     return TTT_OK;
 }
 
@@ -332,7 +333,13 @@ ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const 
         const double wl = (double)lin.heads, wc = kConvHeadWeight * conv.heads;
         cl.num_sms = std::max(1, (int)((double)whole.num_sms * wl / (wl + wc)));
     }
+    int lin_grid = 0;
+    cl.grid_out = &lin_grid;
     if (lin.heads && (st = launch_linear(cl)) != TTT_OK) return st;
+    // The conv kernel is sized for the SMs the linear kernel leaves free (its tasks are split so that
+    // each of those CTAs runs about one gradient task); with none left, it waits for the linear
+    // kernel's SMs and takes them all.
+    if (conv.heads && lin.heads && lin_grid > 0 && lin_grid < whole.num_sms) cc.num_sms = whole.num_sms - lin_grid;
     if (conv.heads) st = launch_dwconv(cc);
     return st;
 }

@@ -17,15 +17,16 @@
 //     the task reads K groups j (rows 2j-1, 2j) and j+1 (rows 2j+1, 2j+2) and V group j.  The tensor
 //     map's out-of-bounds zero fill supplies the zero padding, so the inner loops carry no bounds
 //     checks.
-//   Compute: two groups of 8 warps take alternate row pairs; in a group, warp w owns a column
-//     segment of both rows of the pair, lane l owns channels 2l and 2l+1, and a 4 x 3 register window
-//     slides along the columns (unrolled by 3, so the window never moves between registers).  The
-//     residual is carried negated (s = V - W0 (*) K, from the negated taps), which saves a negation
-//     per token.
-//   Merge: a gradient task's 16 warps fold their 64 x 9 sums in a fixed order into the task's
-//     partial, written to the workspace slot of (unit, task).  The CTA that completes a unit's last
-//     gradient task sums the unit's partials in task order -- a fixed order, so W1 is bitwise
-//     reproducible whichever CTA ran which task -- writes W1 and raises the unit's ready flag.
+//   Compute: three groups of 5 warps; group g takes the row pairs j = g (mod 3) of every task.  In a
+//     group, warp w owns a column segment of both rows of a pair, lane l owns channels 2l and 2l+1,
+//     and a 4 x 3 register window slides along the columns (unrolled by 3, so the window never moves
+//     between registers).  The residual is carried negated (s = V - W0 (*) K, from the negated taps),
+//     which saves a negation per token.
+//   Merge: each group folds its warps' 64 x 9 sums in a fixed order into its partial for the task,
+//     written to the workspace slot of (unit, task, group); the groups never wait for one another.
+//     The group that writes a unit's last partial sums all of the unit's partials in slot order -- a
+//     fixed order, so W1 is bitwise reproducible whichever CTA ran which task (for a given grid) --
+//     writes W1 and raises the unit's ready flag.
 //   Readout tasks wait for that flag.  The wait cannot deadlock: tasks are claimed in order, so
 //     every gradient task of the unit was claimed earlier by a CTA that is running it.  Z is written
 //     straight from registers (128 coalesced bytes per token and warp).
@@ -43,15 +44,16 @@ namespace dw {
 
 constexpr int D = 64;
 constexpr int TAPS = 9;
-constexpr int GW = 6;                       // warps of a compute group (column segments of a row pair)
-constexpr int CG = 2;                       // compute groups (alternate row pairs)
+constexpr int GW = 5;                       // warps of a compute group (column segments of a row pair)
+constexpr int CG = 3;                       // compute groups (row pairs j = g mod CG)
 constexpr int CW = GW * CG;                 // compute warps
-constexpr int THREADS = (CW + 1) * 32;      // + one producer warp (13 warps: 128 registers a thread)
+constexpr int THREADS = (CW + 1) * 32;      // + one producer warp (16 warps: 128 registers a thread)
 constexpr int NK = 6;                       // K / Q ring slots (2-row groups)
 constexpr int NV = 4;                       // V ring slots (2-row groups)
 constexpr int NT = 4;                       // claimed tasks in flight (producer ahead of the compute warps)
 constexpr int kPart = D * TAPS;             // 576 floats: a 64 x 9 gradient or kernel, tap-major
-constexpr int kRed = GW / 2;                // a group's per-warp gradients are folded pairwise into kRed slots
+constexpr int kRed = (GW + 1) / 2;          // a group's per-warp gradients are folded pairwise into kRed slots
+constexpr uint32_t kExitBar = 1 + CG;       // named barrier of all compute warps (ids 1..CG: the groups)
 
 template <typename T>
 struct Elem;
@@ -185,6 +187,26 @@ __device__ __forceinline__ float2 neg_residual(const float2 (&win)[4][3], const 
     return make_float2(t0.x + t1.x + t2.x, t0.y + t1.y + t2.y);
 }
 
+// Both rows of a pair: s0 from window rows 0..2, s1 from rows 1..3, with their six chains interleaved.
+template <int L, int M, int R>
+__device__ __forceinline__ void neg_residual2(const float2 (&win)[4][3], const float2 (&nw)[TAPS], float2 v0,
+                                              float2 v1, float2& s0, float2& s1) {
+    constexpr int cidx[3] = {L, M, R};
+    const float2 zero = make_float2(0.f, 0.f);
+    float2 a0 = v0, a1 = zero, a2 = zero, b0 = v1, b1 = zero, b2 = zero;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+        a0 = ffma2(nw[c], win[0][cidx[c]], a0);
+        b0 = ffma2(nw[c], win[1][cidx[c]], b0);
+        a1 = ffma2(nw[3 + c], win[1][cidx[c]], a1);
+        b1 = ffma2(nw[3 + c], win[2][cidx[c]], b1);
+        a2 = ffma2(nw[6 + c], win[2][cidx[c]], a2);
+        b2 = ffma2(nw[6 + c], win[3][cidx[c]], b2);
+    }
+    s0 = make_float2(a0.x + a1.x + a2.x, a0.y + a1.y + a2.y);
+    s1 = make_float2(b0.x + b1.x + b2.x, b0.y + b1.y + b2.y);
+}
+
 // Phase-1 work of output column x (strip-relative) of the row pair: window columns L, M, R hold
 // staged columns x, x+1, x+2 (image columns x-1, x, x+1); R is loaded here.  nw = -W0 taps;
 // gacc accumulates sum s * K with s = V - W0 (*) K = -r.
@@ -195,17 +217,22 @@ __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[T
     load_col<T, R>(win, rw, x + 2, lane);
     const typename E::Raw* vr = reinterpret_cast<const typename E::Raw*>(vg);
     constexpr int cidx[3] = {L, M, R};
-    const float2 s0 = neg_residual<L, M, R>(win, nw, 0, E::unpack(vr[(size_t)x * D / 2 + lane]));
     if (ROW1) {                                            // the second row of the pair lies inside the grid
-        const float2 s1 = neg_residual<L, M, R>(win, nw, 1, E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]));
+        // both rows' residual chains side by side (six independent 3-term chains), then the nine
+        // row-0 updates before the nine row-1 updates, so that no update waits on the one before it
+        float2 s0, s1;
+        neg_residual2<L, M, R>(win, nw, E::unpack(vr[(size_t)x * D / 2 + lane]),
+                               E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]), s0, s1);
 #pragma unroll
         for (int a = 0; a < 3; ++a)
 #pragma unroll
-            for (int c = 0; c < 3; ++c) {
-                gacc[a * 3 + c] = ffma2(s0, win[a][cidx[c]], gacc[a * 3 + c]);
-                gacc[a * 3 + c] = ffma2(s1, win[a + 1][cidx[c]], gacc[a * 3 + c]);
-            }
+            for (int c = 0; c < 3; ++c) gacc[a * 3 + c] = ffma2(s0, win[a][cidx[c]], gacc[a * 3 + c]);
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int c = 0; c < 3; ++c) gacc[a * 3 + c] = ffma2(s1, win[a + 1][cidx[c]], gacc[a * 3 + c]);
     } else {
+        const float2 s0 = neg_residual<L, M, R>(win, nw, 0, E::unpack(vr[(size_t)x * D / 2 + lane]));
 #pragma unroll
         for (int a = 0; a < 3; ++a)
 #pragma unroll
@@ -335,7 +362,7 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
         return;
     }
 
-    // compute warps: two groups of GW warps; group g takes the row pairs j = g (mod CG) of every task
+    // compute warps: CG groups of GW warps; group g takes the row pairs j = g (mod CG) of every task
     // (a fixed split, so each partial holds the same sums whichever CTA runs the task) and publishes
     // its own partial, so the groups never wait for one another
     const int tid = threadIdx.x;                                     // 0 .. CW*32-1
@@ -392,17 +419,18 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
             kq += (uint32_t)n + 1; vq += (uint32_t)n;
             // ---- the group's partial, summed over its warps in a fixed order
             float(*red)[kPart] = s.red[grp];
-            if (seg >= kRed) {
+            if (seg >= kRed) {                                       // warps kRed.. store, warps 0.. add
 #pragma unroll
                 for (int t9 = 0; t9 < TAPS; ++t9)
                     *reinterpret_cast<float2*>(&red[seg - kRed][t9 * D + 2 * lane]) = gacc[t9];
             }
             named_bar_sync(gbar, GW * 32);
             if (seg < kRed) {
+                const bool pair = seg + kRed < GW;                   // a partner warp stored into this slot
 #pragma unroll
                 for (int t9 = 0; t9 < TAPS; ++t9) {
                     float2* q = reinterpret_cast<float2*>(&red[seg][t9 * D + 2 * lane]);
-                    const float2 o = *q;
+                    const float2 o = pair ? *q : make_float2(0.f, 0.f);
                     *q = make_float2(gacc[t9].x + o.x, gacc[t9].y + o.y);
                 }
             }
@@ -483,12 +511,12 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
         }
     }
     // The last CTA to finish puts the control words back to zero for the next call.
-    named_bar_sync(3, CW * 32);
+    named_bar_sync(kExitBar, CW * 32);
     if (tid == 0) {
         __threadfence();
         s.flag[0] = (atomicAdd(p.done, 1u) == gridDim.x - 1) ? 1 : 0;
     }
-    named_bar_sync(3, CW * 32);
+    named_bar_sync(kExitBar, CW * 32);
     if (s.flag[0]) {
         __threadfence();
         for (int i = tid; i < p.U; i += CW * 32) { p.unit_count[i] = 0u; p.ready[i] = 0u; }

@@ -831,6 +831,7 @@ ttt_status launch_linear(const Call& c) {
             return TTT_ERR_INVALID_ARG;
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)(ncl * cs));
+        if (c.grid_out) *c.grid_out = ncl * cs;
         cfg.blockDim = dim3(kThreadsTc);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = c.stream;

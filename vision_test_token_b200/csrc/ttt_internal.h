@@ -37,6 +37,7 @@ struct Call {
     int num_sms;             // SMs the call may spread its work over
     int overlap_previous;    // launch as a programmatic dependent of the preceding kernel in the stream
     uint8_t* err_ws;         // workspace whose error word the kernels report to (nullptr: ws itself)
+    int* grid_out;           // nullable: the launch writes the number of CTAs it launched
 };
 
 // Encodes a rank-4 bf16 tensor map over [batch][heads][N][64] with a 64 x box_rows box,
