@@ -37,7 +37,7 @@ UNIT = "token*heads/s"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures summarised under
 # profiles/.  Valid only for the kernel builds those captures were taken on: an entry is removed
 # whenever its kernel changes.  Mixed layer: the two kernels of one step, summed.
-STEP_TRAFFIC = {}
+STEP_TRAFFIC = {"mixed6084_bf16": (93.597696e6 + 3.890688e6) + (18.750720e6 + 0.0)}   # profiles/*_mixed6084.md
 MLP_TRAFFIC = {"mlp1024_bf16": 25.780736e6 + 0.0}
 
 
@@ -430,8 +430,10 @@ def run_ours(args):
                        "tokens": w.N, "d": w.d, "eta": w.eta, "parallelism": f"batch-sharded x{world}",
                        "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",
                        "algorithmic_bytes_per_step": workload_bytes(w),
-                       "launch": "CUDA graph per input set" + ("; the conv call on a second stream, concurrent with the "
-                                                               "linear call" if w.kind == "mixed" else "")},
+                       "launch": "CUDA graph per input set" + ("; one ttt_forward_layer call per step: the conv kernel "
+                                                               "launched behind the linear kernel as a programmatic "
+                                                               "dependent, the two running at the same time"
+                                                               if w.kind == "mixed" else "")},
             "gbs_per_step": workload_bytes(w) / (el_max / args.steps) / 1e9,
             "gpu_launches": args.steps * (2 if (w.kind == "mixed" or w.dtype == "fp32") else 1),
             "clocks": clocks, "e2e": e2e}
