@@ -9,7 +9,7 @@
 //
 // One kernel (dw_queue) of independent CTAs -- no clusters, so it fits whatever SMs are free, e.g.
 // next to the linear-head kernel of the same layer.  A unit's grid is cut into tasks of a few
-// row pairs of one strip of at most XT columns (no more gradient tasks than CTAs).  A CTA's producer lane claims tasks from a
+// row pairs of one strip of at most XT columns (about one gradient task per CTA).  A CTA's producer lane claims tasks from a
 // global counter: first every gradient task (phase 1) of every unit, then every readout task
 // (phase 2).
 //   Streaming: the producer loads a task's rows as 2-row groups into two shared-memory rings: K (in
@@ -54,6 +54,7 @@ constexpr int NT = 4;                       // claimed tasks in flight (producer
 constexpr int kPart = D * TAPS;             // 576 floats: a 64 x 9 gradient or kernel, tap-major
 constexpr int kRed = (GW + 1) / 2;          // a group's per-warp gradients are folded pairwise into kRed slots
 constexpr uint32_t kExitBar = 1 + CG;       // named barrier of all compute warps (ids 1..CG: the groups)
+constexpr int kTasksPerCta = 1;             // gradient tasks per CTA a launch aims for
 
 template <typename T>
 struct Elem;
@@ -529,8 +530,9 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
 // ------------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------------
-// Tasks per strip: as many as keep the gradient tasks of the call within `grid` CTAs (one each), so
-// that no CTA runs two of them one after the other; at most one task per row pair.
+// Tasks per strip: about kTasksPerCta gradient tasks per CTA (at most one task per row pair).  One
+// task per CTA measured best: a task's fixed costs (first loads, the group reductions, the unit
+// merge) are several microseconds, so two half-size tasks per CTA took longer than one.
 template <typename T>
 static Geom make_geom(long long units, int grid, int heads, int H, int W, long long bs, long long hs) {
     constexpr int TB = Elem<T>::kTokenBytes;
@@ -541,7 +543,7 @@ static Geom make_geom(long long units, int grid, int heads, int H, int W, long l
     g.Sx = (W + Elem<T>::kXtMax - 1) / Elem<T>::kXtMax;
     g.XT = (W + g.Sx - 1) / g.Sx;
     g.Hp = (H + 1) / 2;
-    g.tps = (int)std::min<long long>(g.Hp, std::max<long long>(1, grid / std::max<long long>(1, units * g.Sx)));
+    g.tps = (int)std::min<long long>(g.Hp, std::max<long long>(1, kTasksPerCta * grid / std::max<long long>(1, units * g.Sx)));
     g.tpu = g.Sx * g.tps;
     g.bs = bs;
     g.hs = hs;
