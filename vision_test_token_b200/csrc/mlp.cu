@@ -8,7 +8,9 @@
 // gelu_tanh(u) = u/2 (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))) (the tanh form of Hendrycks & Gimpel).
 //
 // Every product is a dense contraction and runs on tcgen05 (bf16 operands, fp32 accumulation in
-// tensor memory).  One CTA owns a unit (persistent over units).  Per 128-token tile of phase 1:
+// tensor memory).  A unit is owned by a cluster of two CTAs, each taking half of the tokens (one CTA
+// per unit, persistent over units, when there are more units than SM pairs).  Per 128-token tile of
+// phase 1:
 //   H  = K Wa^T            M=128 tokens, N=256, K=64       -> TMEM cols 256..511
 //   A  = gelu(H) (bf16, shared memory), gelu'(H) packed bf16x2 back into TMEM cols 256..383
 //   Y  = A Wb^T            M=128, N=64, K=256             -> TMEM cols 384..447
@@ -17,9 +19,12 @@
 //   dA = R Wb              M=128, N=128 per hidden half, K=64     -> TMEM cols 384..511
 //   dH = dA * gelu'(H) (bf16, shared memory, over A)
 //   gWa  += dH^T K         M=256 (two halves), N=64, K=128 tokens
-// The accumulators gWb^T and gWa stay in TMEM cols 0..255 across the unit's tiles.  Then
-// Wa1, Wb1 are formed in fp32 (optionally written out) and stored as bf16 operands, and phase 2
-// streams Q: H' = Q Wa1^T, A' = gelu(H'), Z = A' Wb1^T, stored with TMA.
+// The accumulators gWb^T and gWa stay in TMEM cols 0..255 across the CTA's tiles.  Then the two
+// CTAs exchange partial gradients over distributed shared memory: CTA `rank` owns hidden half `rank`,
+// adds the peer's partial for it (two terms: the same sum in either order), forms that half of Wa1
+// and Wb1 in fp32 (optionally written out) and stores the bf16 operands into both CTAs' shared
+// memory.  Phase 2 streams the CTA's Q tiles: H' = Q Wa1^T, A' = gelu(H'), Z = A' Wb1^T, stored
+// with TMA.
 // The same shared-memory buffers serve as K-major operands of one product and MN-major operands of
 // another (both use the 128-byte swizzled layout TMA writes), so nothing is transposed.
 #include <algorithm>
@@ -46,6 +51,7 @@ constexpr uint32_t kIdDA = idesc_bf16_f32(128, 128, false, true);
 
 struct Params {
     int U, heads, N, tpu;
+    int CS;                                 // CTAs per unit (a cluster): 1 or 2
     float eta_scale;                        // eta * 2 / N
     const float* Wa;                        // [heads][256][64]
     const float* Wb;                        // [heads][64][256]
@@ -62,9 +68,14 @@ struct Smem {
     uint8_t rz[TOK * 128];                  // R tile (phase 1), Z staging (phase 2)
     uint64_t full[STAGES], empty[STAGES];
     uint64_t mma_bar;
+    uint64_t free_bar;                      // the peer has finished phase 1: its act and weights may be written
+    uint64_t xbar;                          // the peer's partial gradients for my hidden half have arrived
+    uint64_t wbar;                          // the peer's half of the updated weight operands has arrived
     uint32_t tmem_base;
     int abort_flag;
 };
+
+__host__ __device__ __forceinline__ int split_lo(int n, int r, int parts) { return (int)((long long)n * r / parts); }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -105,6 +116,9 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
         s.abort_flag = 0;
         for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
         mbar_init(&s.mma_bar, 1);
+        mbar_init(&s.free_bar, 1);
+        mbar_init(&s.xbar, 128);
+        mbar_init(&s.wbar, 128);
         fence_barrier_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
     }
@@ -112,21 +126,28 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // every CTA's barriers exist before its peer arrives on them
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
     const uint32_t tmem = s.tmem_base;
+    const bool multi = p.CS > 1;
+    const int rank = multi ? (int)cluster_ctarank() : 0;
+    const int cid = multi ? (int)cluster_id_x() : (int)blockIdx.x;
+    const int ncl = multi ? (int)cluster_count_x() : (int)gridDim.x;
+    const int t0 = split_lo(p.tpu, rank, p.CS), t1 = split_lo(p.tpu, rank + 1, p.CS);   // this CTA's tiles
 
     if (warp == 0) {                                           // TMA producer
         if (lane == 0) {
             int st = 0; uint32_t ph = 0;
-            for (int u = blockIdx.x; u < p.U; u += gridDim.x) {
+            for (int u = cid; u < p.U; u += ncl) {
                 const int b = u / p.heads, h = u % p.heads;
-                for (int t = 0; t < p.tpu; ++t) {
+                for (int t = t0; t < t1; ++t) {
                     if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
                     mbar_arrive_expect_tx(&s.full[st], 2 * TILE);
                     tma_load_4d(s.stage[st], &tmK, &s.full[st], 0, t * TOK, h, b);
                     tma_load_4d(s.stage[st] + TILE, &tmV, &s.full[st], 0, t * TOK, h, b);
                     if (++st == STAGES) { st = 0; ph ^= 1u; }
                 }
-                for (int t = 0; t < p.tpu; ++t) {
+                for (int t = t0; t < t1; ++t) {
                     if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
                     mbar_arrive_expect_tx(&s.full[st], TILE);
                     tma_load_4d(s.stage[st], &tmQ, &s.full[st], 0, t * TOK, h, b);
@@ -161,7 +182,8 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
             return true;
         };
 
-        for (int u = blockIdx.x; u < p.U && !failed; u += gridDim.x) {
+        uint32_t k = 0;                                         // units done (phase of the exchange barriers)
+        for (int u = cid; u < p.U && !failed; u += ncl, ++k) {
             const int bi = u / p.heads, h = u % p.heads;
             // ---- Wa, Wb of the head -> bf16 operands
             {
@@ -191,8 +213,8 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
             }
-            // ---- phase 1
-            for (int t = 0; t < p.tpu && !failed; ++t) {
+            // ---- phase 1 over this CTA's tiles
+            for (int t = t0; t < t1 && !failed; ++t) {
                 bool ok = mbar_wait(&s.full[st], ph, ab);
                 if (named_bar_or(1, 128, !ok)) { failed = true; break; }
                 const uint32_t sK = smem_u32(s.stage[st]);
@@ -283,7 +305,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                         for (int kk = 0; kk < TOK / 16; ++kk)
                             mma_bf16_ss(tmem + (uint32_t)(hb * 64),
                                         sdesc_sw128(sact + (2 * hb) * (TOK * 128) + kk * 2048, TOK * 128, 1024),
-                                        sdesc_sw128(srz + kk * 2048, 0, 1024), kIdG, (t > 0 || kk > 0) ? 1u : 0u);
+                                        sdesc_sw128(srz + kk * 2048, 0, 1024), kIdG, (t > t0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
                         mma_bf16_ss(tmem + 384u, sdesc_sw128(srz + kk * 32, 16, 1024),
@@ -343,19 +365,66 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                         for (int kk = 0; kk < TOK / 16; ++kk)
                             mma_bf16_ss(tmem + 128u + (uint32_t)(hb * 64),
                                         sdesc_sw128(sact + (2 * hb) * (TOK * 128) + kk * 2048, TOK * 128, 1024),
-                                        sdesc_sw128(sK + kk * 2048, 0, 1024), kIdG, (t > 0 || kk > 0) ? 1u : 0u);
+                                        sdesc_sw128(sK + kk * 2048, 0, 1024), kIdG, (t > t0 || kk > 0) ? 1u : 0u);
                     mma_commit(&s.empty[st]);
                 }
                 if (!mma_sync(ok)) { failed = true; break; }
                 if (++st == STAGES) { st = 0; ph ^= 1u; }
             }
             if (failed) break;
-            // ---- update: Wa1 = Wa - eta (2/N) gWa, Wb1 = Wb - eta (2/N) gWb  (rows hid = r, 128 + r)
+            // ---- update: Wa1 = Wa - eta (2/N) gWa, Wb1 = Wb - eta (2/N) gWb.  With a 2-CTA cluster, CTA
+            //      `rank` owns hidden half `rank` (hidden units 128 rank + r): it receives the peer's
+            //      partial gradients for that half, forms that half of Wa1 (rows) and Wb1 (columns),
+            //      and writes the bf16 operands into its own and the peer's shared memory.  One CTA
+            //      (no cluster) owns both halves.
             {
+                const bool has = t1 > t0;                             // this CTA accumulated any tile
+                const int peer = rank ^ 1;
+                float* recv = reinterpret_cast<float*>(s.act[0]);     // [2][128][64]: gWa, gWb^T of my half
+                // recv element (m, row, col): float4 chunk swizzled by the row (conflict-free stores)
+                auto roff = [](int m, int row, int col) {
+                    return (uint32_t)(((m * 128 + row) * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3)) * 4);
+                };
+                bool ok = true;
+                if (multi) {
+                    // (1) my phase 1 is over: the peer may now write my act and weight operands
+                    if (tid == 0) mbar_arrive_remote(map_to_rank(smem_u32(&s.free_bar), (uint32_t)peer));
+                    // (2) and the peer's phase 1 is over
+                    ok = mbar_wait_cluster(&s.free_bar, k & 1u, ab);
+                    if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                    tc_fence_after();
+                    // (3) push my partials for the peer's half into the peer's act
+                    const int ob = peer;
+                    const uint32_t rb = map_to_rank(smem_u32(recv), (uint32_t)peer);
+#pragma unroll 1
+                    for (int j = 0; j < 4; ++j) {
+                        float ga[16], gb[16];
+                        tmem_ld16(tmem + 128u + (uint32_t)(ob * 64 + j * 16) + lane_off, ga);
+                        tmem_ld16(tmem + (uint32_t)(ob * 64 + j * 16) + lane_off, gb);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4) {
+                            const uint4 va = has ? make_uint4(__float_as_uint(ga[e]), __float_as_uint(ga[e + 1]),
+                                                              __float_as_uint(ga[e + 2]), __float_as_uint(ga[e + 3]))
+                                                 : make_uint4(0u, 0u, 0u, 0u);
+                            const uint4 vb = has ? make_uint4(__float_as_uint(gb[e]), __float_as_uint(gb[e + 1]),
+                                                              __float_as_uint(gb[e + 2]), __float_as_uint(gb[e + 3]))
+                                                 : make_uint4(0u, 0u, 0u, 0u);
+                            st_cluster_v4(rb + roff(0, r, j * 16 + e), va);
+                            st_cluster_v4(rb + roff(1, r, j * 16 + e), vb);
+                        }
+                    }
+                    mbar_arrive_remote(map_to_rank(smem_u32(&s.xbar), (uint32_t)peer));   // after my stores
+                    // (4) the peer's partials for my half
+                    ok = mbar_wait_cluster(&s.xbar, k & 1u, ab);
+                    if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                }
                 const float* Wa = p.Wa + (size_t)h * HID * D;
                 const float* Wb = p.Wb + (size_t)h * D * HID;
+                const uint32_t pwa = multi ? map_to_rank(swa, (uint32_t)peer) : 0u;
+                const uint32_t pwb = multi ? map_to_rank(swb, (uint32_t)peer) : 0u;
 #pragma unroll 1
-                for (int hb = 0; hb < 2; ++hb) {
+                for (int hb = multi ? rank : 0; hb < (multi ? rank + 1 : 2); ++hb) {
                     const int hid = hb * 128 + r;
                     float ga[4][16], gb[4][16];
 #pragma unroll
@@ -364,6 +433,21 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                         tmem_ld16(tmem + (uint32_t)(hb * 64 + j * 16) + lane_off, gb[j]);
                     }
                     tmem_ld_wait();
+                    if (!has) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) { ga[j][e] = 0.f; gb[j][e] = 0.f; }
+                    }
+                    if (multi) {                                      // + the peer's partial (two terms: any order)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                ga[j][e] += *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(recv) + roff(0, r, j * 16 + e));
+                                gb[j][e] += *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(recv) + roff(1, r, j * 16 + e));
+                            }
+                    }
 #pragma unroll
                     for (int c = 0; c < D; c += 8) {
                         float w[8];
@@ -376,20 +460,33 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                         pk.x = pack_bf16x2(w[0], w[1]); pk.y = pack_bf16x2(w[2], w[3]);
                         pk.z = pack_bf16x2(w[4], w[5]); pk.w = pack_bf16x2(w[6], w[7]);
                         *reinterpret_cast<uint4*>(s.wa + sw_off(hid, c)) = pk;
+                        if (multi) st_cluster_v4(pwa + sw_off(hid, c), pk);
                     }
 #pragma unroll
                     for (int d = 0; d < D; ++d) {
                         const float w = __ldg(Wb + (size_t)d * HID + hid) - p.eta_scale * gb[d / 16][d % 16];
                         if (p.Wb_out) p.Wb_out[((size_t)u * D + d) * HID + hid] = w;
-                        *reinterpret_cast<__nv_bfloat16*>(s.wb[hid / 64] + sw_off(d, hid % 64)) = __float2bfloat16_rn(w);
+                        const __nv_bfloat16 wb16 = __float2bfloat16_rn(w);
+                        const uint32_t off = (uint32_t)((hid / 64) * (D * 128)) + sw_off(d, hid % 64);
+                        *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(s.wb[0]) + off) = wb16;
+                        // hidden units 2i, 2i+1 are adjacent in a row: even lanes store both to the peer
+                        const uint32_t mine = (uint32_t)__bfloat16_as_ushort(wb16);
+                        const uint32_t next = __shfl_down_sync(0xffffffffu, mine, 1);
+                        if (multi && (lane & 1) == 0) st_cluster_u32(pwb + off, mine | (next << 16));
                     }
                 }
-                fence_proxy_async_smem();
+                if (multi) {
+                    mbar_arrive_remote(map_to_rank(smem_u32(&s.wbar), (uint32_t)peer));   // after my stores
+                    // (5) the peer's half of the operands
+                    ok = mbar_wait_cluster(&s.wbar, k & 1u, ab);
+                    if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                }
+                fence_proxy_async_smem();                             // the operands are read by the tensor cores
                 tc_fence_before();
                 named_bar_sync(1, 128);
             }
-            // ---- phase 2: Z = gelu(Q Wa1^T) Wb1^T
-            for (int t = 0; t < p.tpu && !failed; ++t) {
+            // ---- phase 2: Z = gelu(Q Wa1^T) Wb1^T over this CTA's tiles
+            for (int t = t0; t < t1 && !failed; ++t) {
                 bool ok = mbar_wait(&s.full[st], ph, ab);
                 if (named_bar_or(1, 128, !ok)) { failed = true; break; }
                 const uint32_t sQ = smem_u32(s.stage[st]);
@@ -468,6 +565,8 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
 
     tc_fence_before();
     __syncthreads();
+    // no CTA of the cluster exits while its peer may still write into its shared memory
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -500,9 +599,22 @@ ttt_status launch_mlp(const Call& c) {
         return TTT_ERR_INVALID_ARG;
     const size_t smem = sizeof(Smem) + 1024;
     cudaFuncSetAttribute(mlp_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const int grid = (int)std::min<long long>(units, c.num_sms);
-    mlp_fused<<<grid, THREADS, smem, c.stream>>>(tmK, tmV, tmQ, tmZ, p);
-    return check_launch(cudaGetLastError());
+    // Two CTAs per unit (a cluster; each takes half of the tokens) while that still gives every unit
+    // its own pair of SMs; otherwise one CTA per unit, persistent over units.
+    const int cs = (c.num_sms >= 2 && p.tpu >= 2 && 2LL * units <= c.num_sms) ? 2 : 1;
+    p.CS = cs;
+    const int ncl = (int)std::max<long long>(1, std::min<long long>(units, c.num_sms / cs));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(ncl * cs));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return check_launch(cudaLaunchKernelEx(&cfg, mlp_fused, tmK, tmV, tmQ, tmZ, p));
 }
 
 }  // namespace ttt

@@ -180,6 +180,14 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
                  : "memory");
     return v;
 }
+// Stores into another CTA's shared memory (address from map_to_rank).
+__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, uint4 v) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
+    asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+}
 // Arrive (release, cluster scope) on an mbarrier that lives in another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
