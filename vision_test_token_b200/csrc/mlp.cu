@@ -185,30 +185,23 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
         uint32_t k = 0;                                         // units done (phase of the exchange barriers)
         for (int u = cid; u < p.U && !failed; u += ncl, ++k) {
             const int bi = u / p.heads, h = u % p.heads;
-            // ---- Wa, Wb of the head -> bf16 operands
+            // ---- Wa, Wb of the head -> bf16 operands (coalesced float4 loads: consecutive threads read
+            //      consecutive 16-byte pieces of a row)
             {
-                const float* Wa = p.Wa + (size_t)h * HID * D;
-                const float* Wb = p.Wb + (size_t)h * D * HID;
-                for (int row = tid; row < HID; row += 128) {          // Wa row = hidden unit
-                    for (int c = 0; c < D; c += 8) {
-                        float v[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = __ldg(Wa + (size_t)row * D + c + e);
-                        uint4 pk;
-                        pk.x = pack_bf16x2(v[0], v[1]); pk.y = pack_bf16x2(v[2], v[3]);
-                        pk.z = pack_bf16x2(v[4], v[5]); pk.w = pack_bf16x2(v[6], v[7]);
-                        *reinterpret_cast<uint4*>(s.wa + sw_off(row, c)) = pk;
-                    }
+                const float4* Wa4 = reinterpret_cast<const float4*>(p.Wa + (size_t)h * HID * D);
+                const float4* Wb4 = reinterpret_cast<const float4*>(p.Wb + (size_t)h * D * HID);
+#pragma unroll 4
+                for (int f = tid; f < HID * D / 4; f += 128) {             // Wa: row = hidden unit, 16 float4 a row
+                    const float4 v = __ldg(Wa4 + f);
+                    const int row = f >> 4, col = (f & 15) * 4;
+                    *reinterpret_cast<uint2*>(s.wa + sw_off(row, col)) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
                 }
-                for (int idx = tid; idx < D * (HID / 8); idx += 128) {   // Wb: (d, 8 hidden) chunks
-                    const int d = idx / (HID / 8), c = (idx % (HID / 8)) * 8;
-                    float v[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __ldg(Wb + (size_t)d * HID + c + e);
-                    uint4 pk;
-                    pk.x = pack_bf16x2(v[0], v[1]); pk.y = pack_bf16x2(v[2], v[3]);
-                    pk.z = pack_bf16x2(v[4], v[5]); pk.w = pack_bf16x2(v[6], v[7]);
-                    *reinterpret_cast<uint4*>(s.wb[c / 64] + sw_off(d, c % 64)) = pk;
+#pragma unroll 4
+                for (int f = tid; f < D * HID / 4; f += 128) {             // Wb: row = d, 64 float4 a row
+                    const float4 v = __ldg(Wb4 + f);
+                    const int d = f >> 6, col = (f & 63) * 4;
+                    *reinterpret_cast<uint2*>(s.wb[col / 64] + sw_off(d, col % 64)) =
+                        make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
@@ -451,9 +444,12 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
 #pragma unroll
                     for (int c = 0; c < D; c += 8) {
                         float w[8];
+                        const float4 w0a = __ldg(reinterpret_cast<const float4*>(Wa + (size_t)hid * D + c));
+                        const float4 w0b = __ldg(reinterpret_cast<const float4*>(Wa + (size_t)hid * D + c + 4));
+                        const float w0[8] = {w0a.x, w0a.y, w0a.z, w0a.w, w0b.x, w0b.y, w0b.z, w0b.w};
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            w[e] = __ldg(Wa + (size_t)hid * D + c + e) - p.eta_scale * ga[(c + e) / 16][(c + e) % 16];
+                            w[e] = w0[e] - p.eta_scale * ga[(c + e) / 16][(c + e) % 16];
                             if (p.Wa_out) p.Wa_out[((size_t)u * HID + hid) * D + c + e] = w[e];
                         }
                         uint4 pk;
