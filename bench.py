@@ -38,7 +38,7 @@ UNIT = "token*heads/s"
 # profiles/.  Valid only for the kernel builds those captures were taken on: an entry is removed
 # whenever its kernel changes.  Mixed layer: the two kernels of one step, summed.
 STEP_TRAFFIC = {"mixed6084_bf16": (93.597696e6 + 3.890688e6) + (18.750720e6 + 0.0)}   # profiles/*_mixed6084.md
-MLP_TRAFFIC = {}
+MLP_TRAFFIC = {"mlp1024_bf16": 25.809664e6 + 0.0}                                   # profiles/mlp_fused_mlp1024.md
 
 
 def parse():
