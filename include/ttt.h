@@ -173,6 +173,15 @@ ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const 
                              const float* W0_conv, void* Z, float eta, const ttt_shape* s, int conv_heads,
                              void* ws, size_t ws_bytes, float* W1_lin_out, float* W1_conv_out, void* stream);
 
+/* Self-test of the failure-detection path (no fault is involved): launches one kernel on `stream`
+ * that waits, for at most limit_ns nanoseconds (1 .. 1e9), on a word of the workspace header that
+ * nothing sets, and then takes the steps every bounded wait of the layer kernels takes when it runs
+ * out: it records TTT_ERR_TIMEOUT in the workspace error word and returns.  ttt_workspace_status(ws)
+ * then reports TTT_ERR_TIMEOUT (and clears it).  ws: any workspace of at least 256 bytes that is
+ * zero-filled (ttt_workspace_init); it must not be in use by another call.
+ * Errors: TTT_ERR_WORKSPACE (ws NULL or too small), TTT_ERR_ALIGNMENT, TTT_ERR_INVALID_ARG. */
+ttt_status ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned long long limit_ns, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(ttt_status st);
 

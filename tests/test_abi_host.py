@@ -113,3 +113,12 @@ def test_mlp_rejects_unsupported_requests(lib):
     s = _shape(hidden=100)
     assert capi.ttt_forward_mlp(None, None, None, None, None, None, 0.5, s, None, 0, None, None, None) == \
         capi.TTT_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    assert capi.ttt_selftest_wait_timeout(None, 256, 1000, None) == capi.TTT_ERR_WORKSPACE
+    assert capi.ttt_selftest_wait_timeout(fake, 100, 1000, None) == capi.TTT_ERR_WORKSPACE
+    assert capi.ttt_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 16), 256, 1000, None) == capi.TTT_ERR_ALIGNMENT
+    assert capi.ttt_selftest_wait_timeout(fake, 256, 0, None) == capi.TTT_ERR_INVALID_ARG
+    assert capi.ttt_selftest_wait_timeout(fake, 256, 2_000_000_000, None) == capi.TTT_ERR_INVALID_ARG

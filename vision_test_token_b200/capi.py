@@ -16,7 +16,7 @@ TTT_HEAD_LINEAR, TTT_HEAD_DWCONV, TTT_HEAD_MLP = 0, 1, 2
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_workspace_init", "ttt_workspace_status",
     "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp", "ttt_forward_linear_noalloc",
-    "ttt_layer_workspace_bytes", "ttt_forward_layer",
+    "ttt_layer_workspace_bytes", "ttt_forward_layer", "ttt_selftest_wait_timeout",
     "ttt_status_string", "ttt_last_error", "ttt_version",
 )
 
@@ -67,6 +67,8 @@ def lib():
         L.ttt_layer_workspace_bytes.restype = sz
         L.ttt_forward_layer.argtypes = [vp, vp, vp, vp, vp, vp, f, shp, i, vp, sz, vp, vp, vp]
         L.ttt_forward_layer.restype = i
+        L.ttt_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_ulonglong, vp]
+        L.ttt_selftest_wait_timeout.restype = i
         L.ttt_status_string.argtypes = [i]
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_last_error.argtypes = []
@@ -125,6 +127,10 @@ def ttt_forward_layer(Q, K, V, W0_lin, W0_conv, Z, eta, shape, conv_heads, ws, w
                       stream):
     return lib().ttt_forward_layer(Q, K, V, W0_lin, W0_conv, Z, eta, ctypes.byref(shape), conv_heads, ws, ws_bytes,
                                    W1_lin_out, W1_conv_out, stream)
+
+
+def ttt_selftest_wait_timeout(ws, ws_bytes, limit_ns, stream):
+    return lib().ttt_selftest_wait_timeout(ws, ws_bytes, limit_ns, stream)
 
 
 def ttt_last_error():
