@@ -26,9 +26,11 @@
 //     written to the workspace slot of (unit, task, group); the groups never wait for one another.
 //     The group that writes a unit's last partial sums all of the unit's partials in slot order -- a
 //     fixed order, so W1 is bitwise reproducible whichever CTA ran which task (for a given grid) --
-//     writes W1 and raises the unit's ready flag.
-//   Readout tasks wait for that flag.  The wait cannot deadlock: tasks are claimed in order, so
-//     every gradient task of the unit was claimed earlier by a CTA that is running it.  Z is written
+//     writes W1 and appends the unit to the merge order.
+//   Readout tasks follow the merge order: readout task slot i serves the i-th unit to finish its
+//     gradients, so no CTA waits for one late unit while another is ready.  The wait for slot i
+//     cannot deadlock: tasks are claimed in order, so every gradient task was claimed earlier by a
+//     CTA that is running it.  Z is written
 //     straight from registers (128 coalesced bytes per token and warp).
 //   The last CTA to finish returns the workspace's counters and flags to zero for the next call.
 //   When launched as a programmatic dependent of the preceding kernel (the linear heads of the same
@@ -97,22 +99,23 @@ struct Params {
     uint32_t* err;                   // workspace error word
     uint32_t* queue;                 // task counter
     uint32_t* done;                  // CTAs finished
-    uint32_t* unit_count;            // [U] gradient tasks finished per unit
-    uint32_t* ready;                 // [U] W1 of the unit is in w1g
+    uint32_t* merged;                // units whose W1 is formed so far
+    uint32_t* unit_count;            // [U] gradient partials written per unit
+    uint32_t* order;                 // [U] slot i: 1 + the i-th unit whose W1 was formed (0: not yet)
     float* partials;                 // [U][mtpu][CG][576] negated gradient sums per task and group, tap-major
     int mtpu;                        // partial slots per unit (one task per row pair, the most a call uses)
     float* w1g;                      // [U][576] W1 per unit, tap-major
 };
 
 // Workspace layout: the 256-byte header (word 0: error word), the control words (queue, done,
-// unit_count[U], ready[U]) padded to 256 bytes, the partials, W1.
+// merged, unit_count[U], order[U]) padded to 256 bytes, the partials, W1.
 struct WsLayout {
     size_t ctl, partials, w1g, total;
 };
 static WsLayout ws_layout(long long U, int tpu) {
     WsLayout l;
     l.ctl = kWsHeader;
-    l.partials = l.ctl + align_up((size_t)(2 + 2 * U) * 4, 256);
+    l.partials = l.ctl + align_up((size_t)(3 + 2 * U) * 4, 256);
     l.w1g = l.partials + align_up((size_t)U * tpu * CG * kPart * 4, 256);
     l.total = l.w1g + (size_t)U * kPart * 4;
     return l;
@@ -122,6 +125,7 @@ struct SmemTail {                            // follows the rings
     float red[CG][kRed][kPart];              // per-warp gradients of each group, folded pairwise
     uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], tfull[NT], tempty[NT];
     int task[NT];
+    int task_u[NT];                          // the unit of the task (for a readout task: resolved from order)
     int flag[CG];                            // per-group decision broadcast
     int abort_flag;
 };
@@ -130,7 +134,8 @@ __host__ __device__ __forceinline__ int split_lo(int n, int r, int parts) { retu
 
 struct Task {
     bool p1;
-    int u, r, sx, pa, n;                     // unit, task index in the unit, strip, first pair, pairs
+    int u, r, sx, pa, n;                     // unit (readout task: its slot in the merge order), task index
+                                             // in the unit, strip, first pair, pairs
 };
 
 __device__ __forceinline__ Task decode(const Params& p, int t) {
@@ -344,10 +349,18 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                 const uint32_t ts = tq % NT, tph = (tq / NT) & 1u;
                 ++tq;
                 if (!mbar_wait(&s.tempty[ts], tph ^ 1u, ab)) break;
+                Task tk = decode(p, t);
+                if (t >= 0 && !tk.p1) {
+                    // readout tasks follow the order in which units finish their gradients: slot
+                    // tk.u is filled once that many units have formed W1 (every gradient task was
+                    // claimed before any readout task, so the wait ends)
+                    if (!wait_flag(p.order + tk.u, ab)) break;
+                    tk.u = (int)ld_acquire_gpu(p.order + tk.u) - 1;
+                }
                 s.task[ts] = t;
+                s.task_u[ts] = t >= 0 ? tk.u : 0;
                 mbar_arrive(&s.tfull[ts]);
                 if (t < 0) break;
-                const Task tk = decode(p, t);
                 const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT, y0 = 2 * tk.pa;
                 bool ok = true;
                 if (tk.p1) {                                         // K(0), then K(j+1), V(j)
@@ -376,12 +389,15 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
         ++tq;
         const bool okt = !failed && mbar_wait(&s.tfull[ts], tph, ab);
         const int t = okt ? s.task[ts] : -1;
+        const int tu = okt ? s.task_u[ts] : 0;
         __syncwarp();
         if (okt && lane == 0) mbar_arrive(&s.tempty[ts]);
         // the warps of a group take the same decision: stop on a failure anywhere in the group
         if (named_bar_or(gbar, GW * 32, failed || !okt)) { failed = true; break; }
         if (t < 0) break;
-        const Task tk = decode(p, t);
+        Task tk = decode(p, t);
+        const int slot = tk.u;                                       // readout task: merge-order slot
+        tk.u = tu;
         const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT;
         const int cols = min(g.W - xs, g.XT), segw = (cols + GW - 1) / GW;
         const int xa = seg * segw, xb = min(cols, xa + segw);        // strip-relative output columns
@@ -476,12 +492,12 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                 }
                 __threadfence();
                 named_bar_sync(gbar, GW * 32);
-                if (gtid == 0) st_release_gpu(p.ready + tk.u, 1u);
+                if (gtid == 0) st_release_gpu(p.order + atomicAdd(p.merged, 1u), (uint32_t)tk.u + 1u);
             }
         } else {
             // ---- phase-2 task: Z = W1 (*) Q over this group's row pairs of the task
             float2 w[TAPS];
-            if (!wait_flag(p.ready + tk.u, ab)) failed = true;
+            if (!wait_flag(p.order + slot, ab)) failed = true;             // (already set: an acquire)
 #pragma unroll
             for (int t9 = 0; t9 < TAPS; ++t9)
                 w[t9] = __ldcg(reinterpret_cast<const float2*>(p.w1g + (size_t)tk.u * kPart + t9 * D) + lane);
@@ -520,8 +536,8 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
     named_bar_sync(kExitBar, CW * 32);
     if (s.flag[0]) {
         __threadfence();
-        for (int i = tid; i < p.U; i += CW * 32) { p.unit_count[i] = 0u; p.ready[i] = 0u; }
-        if (tid == 0) { *p.queue = 0u; *p.done = 0u; }
+        for (int i = tid; i < p.U; i += CW * 32) { p.unit_count[i] = 0u; p.order[i] = 0u; }
+        if (tid == 0) { *p.queue = 0u; *p.done = 0u; *p.merged = 0u; }
     }
     // As a programmatic dependent of the preceding kernel: complete only after it has completed.
     pdl_wait_primary();
@@ -595,8 +611,9 @@ static ttt_status launch(const Call& c) {
     uint32_t* ctl = reinterpret_cast<uint32_t*>(c.ws + L.ctl);
     p.queue = ctl;
     p.done = ctl + 1;
-    p.unit_count = ctl + 2;
-    p.ready = ctl + 2 + units;
+    p.merged = ctl + 2;
+    p.unit_count = ctl + 3;
+    p.order = ctl + 3 + units;
     p.partials = reinterpret_cast<float*>(c.ws + L.partials);
     p.mtpu = g.Sx * g.Hp;
     p.w1g = reinterpret_cast<float*>(c.ws + L.w1g);
