@@ -47,7 +47,6 @@ def lib():
             raise RuntimeError(f"libttt.so not found at {LIB_PATH}: run `python -m vision_test_token_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         vp, sz, i, f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
-        fp = ctypes.POINTER(ctypes.c_float)
         shp = ctypes.POINTER(TttShape)
         L.ttt_workspace_bytes.argtypes = [i, shp]
         L.ttt_workspace_bytes.restype = sz
@@ -77,7 +76,6 @@ def lib():
         L.ttt_version.restype = i
         for name in EXPORTED:
             getattr(L, name)
-        _ = fp
         _lib = L
     return _lib
 
