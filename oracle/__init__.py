@@ -35,9 +35,10 @@ def _load():
         d = ctypes.c_double
         lib.oracle_linear.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_linear_gram.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_linear_dot.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
-        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_dwconv, lib.oracle_mlp):
+        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_dwconv, lib.oracle_mlp):
             f.restype = ctypes.c_int
         lib.oracle_gelu_tanh.argtypes = [d]
         lib.oracle_gelu_tanh.restype = d
@@ -83,6 +84,19 @@ def linear(Q, K, V, W0, eta, threads=None, gram=False):
 
 def linear_gram(Q, K, V, W0, eta, threads=None):
     return linear(Q, K, V, W0, eta, threads=threads, gram=True)
+
+
+def linear_dot(Q, K, V, W0, eta, threads=None):
+    """Linear inner model with the dot-product inner loss L(W) = -(1/N) sum <W k, v>.
+    Returns (Z [B][h][N][d], W1 [B][h][d][d]) in float64."""
+    Q, K, V, W0 = _f64(Q), _f64(K), _f64(V), _f64(W0)
+    B, H, N, d = Q.shape
+    assert K.shape == Q.shape and V.shape == Q.shape and W0.shape == (H, d, d)
+    Z = np.empty_like(Q)
+    W1 = np.empty((B, H, d, d))
+    _check(_load().oracle_linear_dot(B, H, N, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1), _p(Z),
+                                     threads or default_threads()), "linear_dot")
+    return Z, W1
 
 
 def dwconv(Q, K, V, W0, eta, Hg, Wg, threads=None):

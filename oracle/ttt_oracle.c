@@ -162,6 +162,63 @@ int oracle_linear_gram(int B, int heads, int N, int d, const double* Q, const do
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Linear inner model trained with the dot-product inner loss (press article, section            */
+/* ViT3：視覺測試時訓練模型: ViT3's inner training is one full-batch step with a dot-product loss,  */
+/* learning rate 1.0).  The pages do not print the loss; read as the negative mean inner product  */
+/* of prediction and value,                                                                     */
+/*     L(W) = -(1/N) sum_n <W k_n, v_n>,   dL/dW = -(1/N) sum_n v_n k_n^T,                        */
+/*     W1 = W0 - eta dL/dW = W0 + (eta/N) sum_n v_n k_n^T,   z_n = W1 q_n.                        */
+/* Its mixed second derivative d2L/dW dv is not zero (press article, Observation 1).  The update   */
+/* does not depend on W0: there is no Gram term.                                                  */
+/* ------------------------------------------------------------------------------------------ */
+
+static int linear_dot_unit(int N, int d, const double* Q, const double* K, const double* V,
+                           const double* W0, double eta, double* W1, double* Z)
+{
+    double* grad = (double*)calloc((size_t)d * d, sizeof(double));
+    if (!grad) return ORACLE_ERR_NOMEM;
+    for (int n = 0; n < N; ++n) {                /* grad -= v_n k_n^T */
+        const double* k = K + (size_t)n * d;
+        const double* v = V + (size_t)n * d;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) grad[(size_t)i * d + j] -= v[i] * k[j];
+    }
+    const double scale = 1.0 / (double)N;
+    for (int i = 0; i < d * d; ++i) W1[i] = W0[i] - eta * scale * grad[i];
+    for (int n = 0; n < N; ++n) {                /* readout z = W1 q */
+        const double* q = Q + (size_t)n * d;
+        for (int i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j) s += W1[(size_t)i * d + j] * q[j];
+            Z[(size_t)n * d + i] = s;
+        }
+    }
+    free(grad);
+    return ORACLE_OK;
+}
+
+int oracle_linear_dot(int B, int heads, int N, int d, const double* Q, const double* K, const double* V,
+                      const double* W0, double eta, double* W1, double* Z, int nthreads)
+{
+    if (B < 0 || heads < 0 || N < 1 || d < 1 || !Q || !K || !V || !W0 || !W1 || !Z) return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int h = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        int st = linear_dot_unit(N, d, Q + off, K + off, V + off, W0 + (size_t)h * d * d, eta,
+                                 W1 + (size_t)u * d * d, Z + off);
+        if (st != ORACLE_OK) {
+#pragma omp atomic write
+            status = st;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* 3x3 depthwise-convolution inner model over the H x W token grid                             */
 /* (press article, Observation 6 and Fig. 5 part 3; ViT3 news article, 原則六 and section      */
 /* 效果全面驗證: one head uses a 3x3 depthwise convolution).                                     */

@@ -173,6 +173,81 @@ def test_planted_mistakes_fail_the_linear_pins(mistake):
 
 
 # ------------------------------------------------------------------------------------------------
+# linear head, dot-product inner loss  L(W) = -(1/N) sum_n <W k_n, v_n>
+# ------------------------------------------------------------------------------------------------
+def _frac_loss_dot(W, K, V):
+    """-(1/N) sum_n <W k_n, v_n> in exact rational arithmetic."""
+    N, d = len(K), len(K[0])
+    tot = Fraction(0)
+    for n in range(N):
+        for i in range(d):
+            tot += sum(W[i][j] * K[n][j] for j in range(d)) * V[n][i]
+    return -tot / N
+
+
+def _dot_fd_grad(W0, K, V):
+    Kf = [[Fraction(int(v)) for v in row] for row in K]
+    Vf = [[Fraction(int(v)) for v in row] for row in V]
+    Wf = [[Fraction(int(v)) for v in row] for row in W0]
+    d = len(Wf)
+    g = np.zeros((d, d))
+    for i in range(d):
+        for j in range(d):
+            Wp = [r[:] for r in Wf]; Wm = [r[:] for r in Wf]
+            Wp[i][j] += 1; Wm[i][j] -= 1
+            g[i, j] = float((_frac_loss_dot(Wp, Kf, Vf) - _frac_loss_dot(Wm, Kf, Vf)) / 2)
+    return g
+
+
+def test_linear_dot_gradient_exact_rational_fd():
+    d, N, eta = 3, 5, 1.0
+    K = _small_ints((N, d)); V = _small_ints((N, d)); W0 = _small_ints((d, d)); Q = _small_ints((N, d))
+    _, W1 = oracle.linear_dot(Q[None, None], K[None, None], V[None, None], W0[None], eta)
+    grad = (W0 - W1[0, 0]) / eta
+    np.testing.assert_allclose(grad, _dot_fd_grad(W0, K, V), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mistake", ["sign", "two_over_n", "transpose", "l2_gram"])
+def test_planted_mistakes_fail_the_dot_pin(mistake):
+    """A plausible mistake planted in the oracle's gradient (on the CPU) fails the exact-FD pin."""
+    d, N = 3, 5
+    K = _small_ints((N, d)); V = _small_ints((N, d)); W0 = _small_ints((d, d)); Q = _small_ints((N, d))
+    _, W1 = oracle.linear_dot(Q[None, None], K[None, None], V[None, None], W0[None], 1.0)
+    grad = W0 - W1[0, 0]
+    bad = {"sign": -grad, "two_over_n": 2 * grad, "transpose": grad.T,
+           "l2_gram": grad + (W0 @ (K.T @ K)) * 2 / N}[mistake]
+    assert not np.allclose(bad, _dot_fd_grad(W0, K, V), atol=1e-9, rtol=0)
+
+
+def test_linear_dot_eta_zero_and_w0_independent_update():
+    B, H, N, d = 2, 3, 41, 16
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    W0a, W0b = RNG.standard_normal((H, d, d)), RNG.standard_normal((H, d, d))
+    Z, W1 = oracle.linear_dot(Q, K, V, W0a, 0.0)
+    np.testing.assert_array_equal(W1, np.broadcast_to(W0a, W1.shape))
+    np.testing.assert_allclose(Z, np.einsum("bhnj,hij->bhni", Q, W0a), atol=1e-13, rtol=0)
+    _, W1a = oracle.linear_dot(Q, K, V, W0a, 0.8)
+    _, W1b = oracle.linear_dot(Q, K, V, W0b, 0.8)
+    np.testing.assert_allclose(W1a - W0a[None], W1b - W0b[None], atol=1e-12, rtol=0)
+
+
+def test_linear_dot_matches_torch_autograd():
+    B, H, N, d, eta = 2, 2, 23, 12, 1.0
+    Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((H, d, d))
+    Z, W1 = oracle.linear_dot(Q, K, V, W0, eta)
+    for b in range(B):
+        for h in range(H):
+            W = torch.tensor(W0[h], requires_grad=True)
+            Kt, Vt = torch.tensor(K[b, h]), torch.tensor(V[b, h])
+            loss = -((Kt @ W.T) * Vt).sum(-1).mean()
+            loss.backward()
+            W1_ref = (W - eta * W.grad).detach().numpy()
+            np.testing.assert_allclose(W1[b, h], W1_ref, atol=1e-12, rtol=0)
+            np.testing.assert_allclose(Z[b, h], Q[b, h] @ W1_ref.T, atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------------------------------------------
 # depthwise 3x3 conv head
 # ------------------------------------------------------------------------------------------------
 def test_dwconv_gradient_exact_rational_fd():
