@@ -37,8 +37,10 @@ def _load():
         lib.oracle_linear_gram.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_linear_dot.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_dwconv_dot.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
-        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_dwconv, lib.oracle_mlp):
+        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_dwconv,
+                  lib.oracle_dwconv_dot, lib.oracle_mlp):
             f.restype = ctypes.c_int
         lib.oracle_gelu_tanh.argtypes = [d]
         lib.oracle_gelu_tanh.restype = d
@@ -108,6 +110,19 @@ def dwconv(Q, K, V, W0, eta, Hg, Wg, threads=None):
     W1 = np.empty((B, H, d, 3, 3))
     _check(_load().oracle_dwconv(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1),
                                  _p(Z), threads or default_threads()), "dwconv")
+    return Z, W1
+
+
+def dwconv_dot(Q, K, V, W0, eta, Hg, Wg, threads=None):
+    """Conv inner model with the dot-product inner loss L(W) = -(1/N) sum <f(K;W), V>.
+    Q, K, V: [B][h][Hg*Wg][d]; W0: [h][d][3][3].  Returns (Z, W1 [B][h][d][3][3])."""
+    Q, K, V, W0 = _f64(Q), _f64(K), _f64(V), _f64(W0)
+    B, H, N, d = Q.shape
+    assert N == Hg * Wg and K.shape == Q.shape and V.shape == Q.shape and W0.shape == (H, d, 3, 3)
+    Z = np.empty_like(Q)
+    W1 = np.empty((B, H, d, 3, 3))
+    _check(_load().oracle_dwconv_dot(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1),
+                                     _p(Z), threads or default_threads()), "dwconv_dot")
     return Z, W1
 
 

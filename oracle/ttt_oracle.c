@@ -27,6 +27,9 @@
  *       per channel, tokens in raster order n = y*W + x, channel c = feature c of the head;
  *     - the MLP head is f(x) = Wb * gelu_tanh(Wa * x) with no biases, and both matrices take one
  *       simultaneous step from gradients evaluated at the initial weights.
+ *     - the dot-product inner loss of the ViT3 recipe (press article, section on the ViT3 model;
+ *       the loss itself is not printed) is the negative mean inner product of prediction and value,
+ *       L(W) = -(1/N) sum_n <f(k_n; W), v_n>.
  *
  * Memory layout of every array (contiguous, row-major, fp64):
  *   Q, K, V, Z : [B][heads][N][d]     (token n, feature c at ((b*heads + h)*N + n)*d + c)
@@ -286,6 +289,65 @@ int oracle_dwconv(int B, int heads, int Hg, int Wg, int d, const double* Q, cons
         const size_t off = (size_t)u * N * d;
         int s = dwconv_unit(Hg, Wg, d, Q + off, K + off, V + off, W0 + (size_t)h * d * 9, eta,
                             W1 + (size_t)u * d * 9, Z + off);
+        if (s != ORACLE_OK) {
+#pragma omp atomic write
+            status = s;
+        }
+    }
+    return status;
+}
+
+/* The conv inner model trained with the dot-product inner loss (press article, section
+ * ViT3：視覺測試時訓練模型: the ViT3 recipe pairs the dot-product loss with a depthwise-conv inner
+ * model).  Read as L(W) = -(1/N) sum_{c,y,x} f(K;W)[c,y,x] * V[c,y,x], whose gradient is
+ *     g[c][a][b] = -(1/N) sum_{y,x} V[c,y,x] * K[c, y+a-1, x+b-1],
+ * W1 = W0 - eta*g;  Z = f(Q;W1).  The update does not depend on W0. */
+static int dwconv_dot_unit(int Hg, int Wg, int d, const double* Q, const double* K, const double* V,
+                           const double* W0, double eta, double* W1, double* Z)
+{
+    const int N = Hg * Wg;
+    double* g = (double*)calloc((size_t)d * 9, sizeof(double));
+    if (!g) return ORACLE_ERR_NOMEM;
+    for (int c = 0; c < d; ++c)
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                const double v = V[((size_t)y * Wg + x) * d + c];
+                for (int a = 0; a < 3; ++a)
+                    for (int b = 0; b < 3; ++b)
+                        g[(size_t)c * 9 + a * 3 + b] -= v * grid_at(K, Hg, Wg, d, c, y + a - 1, x + b - 1);
+            }
+    const double scale = 1.0 / (double)N;
+    for (int i = 0; i < d * 9; ++i) W1[i] = W0[i] - eta * scale * g[i];
+    for (int c = 0; c < d; ++c) {
+        const double* w = W1 + (size_t)c * 9;
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double f = 0.0;
+                for (int a = 0; a < 3; ++a)
+                    for (int b = 0; b < 3; ++b)
+                        f += w[a * 3 + b] * grid_at(Q, Hg, Wg, d, c, y + a - 1, x + b - 1);
+                Z[((size_t)y * Wg + x) * d + c] = f;
+            }
+    }
+    free(g);
+    return ORACLE_OK;
+}
+
+int oracle_dwconv_dot(int B, int heads, int Hg, int Wg, int d, const double* Q, const double* K,
+                      const double* V, const double* W0, double eta, double* W1, double* Z, int nthreads)
+{
+    if (B < 0 || heads < 0 || Hg < 1 || Wg < 1 || d < 1 || !Q || !K || !V || !W0 || !W1 || !Z)
+        return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    const size_t N = (size_t)Hg * Wg;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int h = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        int s = dwconv_dot_unit(Hg, Wg, d, Q + off, K + off, V + off, W0 + (size_t)h * d * 9, eta,
+                                W1 + (size_t)u * d * 9, Z + off);
         if (s != ORACLE_OK) {
 #pragma omp atomic write
             status = s;

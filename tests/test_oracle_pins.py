@@ -337,6 +337,92 @@ def test_dwconv_centre_tap_matches_diagonal_linear_gradient():
 
 
 # ------------------------------------------------------------------------------------------------
+# depthwise 3x3 conv head, dot-product inner loss  L(W) = -(1/N) sum <f(K;W), V>
+# ------------------------------------------------------------------------------------------------
+def _frac_loss_conv_dot(W, K, V, Hg, Wg):
+    d = len(K[0])
+    tot = Fraction(0)
+    for c in range(d):
+        for y in range(Hg):
+            for x in range(Wg):
+                tot += _frac_conv(W[c], K, Hg, Wg, c, y, x) * V[y * Wg + x][c]
+    return -tot / (Hg * Wg)
+
+
+def _conv_dot_fd_grad(W0, K, V, Hg, Wg):
+    d = W0.shape[0]
+    Kf = [[Fraction(int(v)) for v in row] for row in K]
+    Vf = [[Fraction(int(v)) for v in row] for row in V]
+    Wf = [[[Fraction(int(v)) for v in r] for r in W0[c]] for c in range(d)]
+    g = np.zeros((d, 3, 3))
+    for c in range(d):
+        for a in range(3):
+            for b in range(3):
+                Wp = [[r[:] for r in ch] for ch in Wf]; Wm = [[r[:] for r in ch] for ch in Wf]
+                Wp[c][a][b] += 1; Wm[c][a][b] -= 1
+                g[c, a, b] = float((_frac_loss_conv_dot(Wp, Kf, Vf, Hg, Wg) -
+                                    _frac_loss_conv_dot(Wm, Kf, Vf, Hg, Wg)) / 2)
+    return g
+
+
+def test_dwconv_dot_gradient_exact_rational_fd():
+    Hg, Wg, d, eta = 3, 4, 2, 1.0
+    N = Hg * Wg
+    K = _small_ints((N, d)); V = _small_ints((N, d)); Q = _small_ints((N, d))
+    W0 = _small_ints((d, 3, 3))
+    _, W1 = oracle.dwconv_dot(Q[None, None], K[None, None], V[None, None], W0[None], eta, Hg, Wg)
+    grad = (W0 - W1[0, 0]) / eta
+    np.testing.assert_allclose(grad, _conv_dot_fd_grad(W0, K, V, Hg, Wg), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mistake", ["sign", "two_over_n", "flipped_taps", "l2_residual"])
+def test_planted_mistakes_fail_the_conv_dot_pin(mistake):
+    """A plausible mistake planted in the oracle's conv gradient (on the CPU) fails the exact-FD pin."""
+    Hg, Wg, d = 3, 4, 2
+    N = Hg * Wg
+    K = _small_ints((N, d)); V = _small_ints((N, d)); Q = _small_ints((N, d))
+    W0 = _small_ints((d, 3, 3))
+    _, W1 = oracle.dwconv_dot(Q[None, None], K[None, None], V[None, None], W0[None], 1.0, Hg, Wg)
+    grad = W0 - W1[0, 0]
+    _, W1l2 = oracle.dwconv(Q[None, None], K[None, None], V[None, None], W0[None], 1.0, Hg, Wg)
+    bad = {"sign": -grad, "two_over_n": 2 * grad, "flipped_taps": grad[:, ::-1, ::-1],
+           "l2_residual": W0 - W1l2[0, 0]}[mistake]
+    assert not np.allclose(bad, _conv_dot_fd_grad(W0, K, V, Hg, Wg), atol=1e-9, rtol=0)
+
+
+@pytest.mark.parametrize("Hg,Wg", [(6, 5), (1, 9), (4, 1)])
+def test_dwconv_dot_matches_torch_autograd(Hg, Wg):
+    d, eta = 6, 1.0
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, 3, 3))
+    Z, W1 = oracle.dwconv_dot(Q, K, V, W0, eta, Hg, Wg)
+    W = torch.tensor(W0[0], requires_grad=True)
+    loss = -(_torch_conv_f(torch.tensor(K[0, 0]), W, Hg, Wg) * torch.tensor(V[0, 0])).sum(-1).mean()
+    loss.backward()
+    W1_ref = (W - eta * W.grad).detach()
+    np.testing.assert_allclose(W1[0, 0], W1_ref.numpy(), atol=1e-12, rtol=0)
+    Zref = _torch_conv_f(torch.tensor(Q[0, 0]), W1_ref, Hg, Wg).numpy()
+    np.testing.assert_allclose(Z[0, 0], Zref, atol=1e-12, rtol=0)
+
+
+def test_dwconv_dot_centre_tap_matches_linear_dot_diagonal_and_update_ignores_w0():
+    Hg, Wg, d, eta = 5, 7, 8, 0.9
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    Wa, Wb = RNG.standard_normal((1, d, 3, 3)), RNG.standard_normal((1, d, 3, 3))
+    _, W1a = oracle.dwconv_dot(Q, K, V, Wa, eta, Hg, Wg)
+    _, W1b = oracle.dwconv_dot(Q, K, V, Wb, eta, Hg, Wg)
+    np.testing.assert_allclose(W1a[0, 0] - Wa[0], W1b[0, 0] - Wb[0], atol=1e-12, rtol=0)
+    _, W1l = oracle.linear_dot(Q, K, V, np.zeros((1, d, d)), eta)
+    np.testing.assert_allclose(W1a[0, 0, :, 1, 1] - Wa[0, :, 1, 1], np.diag(W1l[0, 0]), atol=1e-12, rtol=0)
+    _, W1 = oracle.dwconv_dot(Q[:, :, :1], K[:, :, :1], V[:, :, :1], Wa, eta, 1, 1)   # one token
+    delta = W1[0, 0] - Wa[0]
+    mask = np.ones((3, 3), bool); mask[1, 1] = False
+    assert np.all(delta[:, mask] == 0.0)
+
+
+# ------------------------------------------------------------------------------------------------
 # MLP head
 # ------------------------------------------------------------------------------------------------
 def test_gelu_tanh_matches_torch():
