@@ -5,7 +5,8 @@
 One step = one forward of the whole layer over one batch: for the default workload
 (mixed6084_bf16: 8 images x 6 heads x 78x78 = 6084 tokens, d = 64, bf16, eta = 0.5) the five linear
 heads and the depthwise-conv head, i.e. the Gram/cross accumulation, the deterministic merge and
-update, and the readout of every head.  Inputs are synthetic (seeded, the pages' shapes and
+update, and the readout of every head.  --workload mixed6084_dot_bf16 runs the same layer trained
+with the dot-product inner loss (eta = 1.0).  Inputs are synthetic (seeded, the pages' shapes and
 distributions) and already resident in HBM when the timed region starts; three input sets of
 149.5 MB each (more than the 126 MB L2) are rotated so every step reads cold data.  Steps are replayed
 from CUDA graphs (one graph per input set) and timed with CUDA events on the launching stream.
@@ -37,7 +38,9 @@ UNIT = "token*heads/s"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures summarised under
 # profiles/.  Valid only for the kernel builds those captures were taken on: an entry is removed
 # whenever its kernel changes.  Mixed layer: the two kernels of one step, summed.
-STEP_TRAFFIC = {"mixed6084_bf16": (93.596416e6 + 3.737088e6) + (18.751488e6 + 0.0064e6)}   # profiles/*_mixed6084.md
+STEP_TRAFFIC = {"mixed6084_bf16": (93.596416e6 + 3.737088e6) + (18.751488e6 + 0.0064e6),    # profiles/*_mixed6084.md
+                "mixed6084_dot_bf16": (93.595904e6 + 4.063488e6) + (18.747392e6 + 0.002816e6)}
+                # profiles/layer_kernels_mixed6084_dot_bf16.md
 MLP_TRAFFIC = {"mlp1024_bf16": 25.809664e6 + 0.0}                                   # profiles/mlp_fused_mlp1024.md
 
 
@@ -191,14 +194,15 @@ def oracle_units(w, x, units, threads):
         hs = [h for bb, h in units if bb == b]
         lin = [h for h in hs if h < nl]
         conv = [h for h in hs if h >= nl]
+        lin_fn, conv_fn = (oracle.linear_dot, oracle.dwconv_dot) if w.loss == "dot" else (oracle.linear, oracle.dwconv)
         if lin:
             lo, hi = min(lin), max(lin) + 1
-            oracle.linear(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
-                          x["W0_lin"][lo:hi], w.eta, threads=threads)
+            lin_fn(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
+                   x["W0_lin"][lo:hi], w.eta, threads=threads)
         if conv:
             lo, hi = min(conv), max(conv) + 1
-            oracle.dwconv(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
-                          x["W0_conv"][lo - nl:hi - nl], w.eta, w.H, w.W, threads=threads)
+            conv_fn(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
+                    x["W0_conv"][lo - nl:hi - nl], w.eta, w.H, w.W, threads=threads)
 
 
 def oracle_inputs(w, x, images):
@@ -260,7 +264,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(1, args.steps) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads, "tokens": w.N, "d": w.d,
-                       "eta": w.eta, "device": "host CPU"},
+                       "eta": w.eta, "loss": w.loss, "device": "host CPU"},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -279,7 +283,8 @@ def make_step(w, xs, dev):
         if w.kind == "mlp":
             layer.forward_mlp(x["Q"], x["K"], x["V"], weights["Wa"], weights["Wb"], w.eta, w.H, w.W, Z=x["Z"])
         else:
-            layer.forward_layer(x["Q"], x["K"], x["V"], weights, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=x["Z"])
+            layer.forward_layer(x["Q"], x["K"], x["V"], weights, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=x["Z"],
+                                loss=w.loss)
     return step
 
 
@@ -312,10 +317,10 @@ def time_calls_alone(w, xs, stream, n):
         for x in xs:
             if which == "linear":
                 fn = lambda x=x: layer.forward_linear(x["Q"][:, :nl], x["K"][:, :nl], x["V"][:, :nl], x["W0_lin"],
-                                                      w.eta, w.H, w.W, Z=x["Z"][:, :nl])
+                                                      w.eta, w.H, w.W, Z=x["Z"][:, :nl], loss=w.loss)
             else:
                 fn = lambda x=x: layer.forward_dwconv(x["Q"][:, nl:], x["K"][:, nl:], x["V"][:, nl:], x["W0_conv"],
-                                                      w.eta, w.H, w.W, Z=x["Z"][:, nl:])
+                                                      w.eta, w.H, w.W, Z=x["Z"][:, nl:], loss=w.loss)
             with torch.cuda.stream(stream):
                 fn()
             stream.synchronize()
@@ -393,8 +398,9 @@ def run_ours(args):
         t_lin, t_conv = time_calls_alone(w, xs, stream, n=max(200, args.steps // 4))
         step_s = el_max / args.steps
         achieved = workload_bytes(w) / step_s / 1e9
+        conv_name = "dw_queue<bf16, dot>" if w.loss == "dot" else "dw_queue<bf16>"
         roof = {"bound": "hbm",
-                "kernel": "layer step: lin_cluster_bf16 and dw_queue<bf16> running at the same time "
+                "kernel": f"layer step: lin_cluster_bf16 and {conv_name} running at the same time "
                           "(one ttt_forward_layer call)",
                 "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                 "traffic": STEP_TRAFFIC.get(w.name), "peak_source": pk["source"],
@@ -403,7 +409,7 @@ def run_ours(args):
                     "lin_cluster_bf16": {"us_per_launch": t_lin * 1e6, "algorithmic_bytes": lin_bytes,
                                          "achieved_gbs": lin_bytes / t_lin / 1e9,
                                          "frac": lin_bytes / t_lin / 1e9 / pk["hbm_gbs"]},
-                    "dw_queue<bf16>": {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
+                    conv_name: {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
                                        "achieved_gbs": conv_bytes / t_conv / 1e9,
                                        "frac": conv_bytes / t_conv / 1e9 / pk["hbm_gbs"]}}}
     elif w.kind == "mlp":
@@ -427,7 +433,8 @@ def run_ours(args):
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads,
                        "lin_heads": w.lin_heads, "conv_heads": w.conv_heads, "grid": [w.H, w.W],
-                       "tokens": w.N, "d": w.d, "eta": w.eta, "parallelism": f"batch-sharded x{world}",
+                       "tokens": w.N, "d": w.d, "eta": w.eta, "loss": w.loss,
+                       "parallelism": f"batch-sharded x{world}",
                        "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",
                        "algorithmic_bytes_per_step": workload_bytes(w),
                        "launch": "CUDA graph per input set" + ("; one ttt_forward_layer call per step: the conv kernel "
@@ -485,7 +492,7 @@ def run_e2e(w, x, dev, stream, steps, world):
                 layer.forward_mlp(d["Q"], d["K"], d["V"], d["Wa"], d["Wb"], w.eta, w.H, w.W, Z=z_dev[bsel])
             else:
                 layer.forward_layer(d["Q"], d["K"], d["V"], d, w.eta, w.H, w.W, conv_heads=w.conv_heads,
-                                    Z=z_dev[bsel])
+                                    Z=z_dev[bsel], loss=w.loss)
             computed[bsel].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(computed[bsel])

@@ -7,6 +7,7 @@
  *   full-batch, non-causal gradient step of the L2 reconstruction loss over all N pairs,
  *       L(W)  = (1/N) sum_n || f(k_n; W) - v_n ||^2,        W1 = W0 - eta * dL/dW (W0),
  *   and every query is read out through the updated model:  z_n = f(q_n; W1).
+ *   The shape's `loss` field selects the dot-product inner loss instead (see ttt_loss).
  *   Sources, by page title and section:
  *     "CVPR 2026 Oral | 清華+阿里發布ViT3" (press article): section 序列建模的新視角 (keys and values
  *       as a dataset, reconstruction by gradient descent, readout on the queries); Observation 2,
@@ -67,6 +68,17 @@ typedef enum { TTT_FP32 = 0, TTT_BF16 = 1 } ttt_dtype;
 
 typedef enum { TTT_HEAD_LINEAR = 0, TTT_HEAD_DWCONV = 1, TTT_HEAD_MLP = 2 } ttt_head_kind;
 
+/* Inner loss of the one-step training.
+ *   TTT_LOSS_L2:  L(W) = (1/N) sum_n || f(k_n; W) - v_n ||^2  (the formulas of each entry point below).
+ *   TTT_LOSS_DOT: L(W) = -(1/N) sum_n < f(k_n; W), v_n >, the dot-product loss of the ViT^3 recipe
+ *     (press article, section ViT3：視覺測試時訓練模型: one full-batch step, learning rate 1.0,
+ *     dot-product loss; the pages do not print the loss, this is its plain reading).  Its gradient
+ *     has no residual and does not depend on W0:
+ *       linear:  W1 = W0 + eta (1/N) sum_n v_n k_n^T   (= W0 + eta C / N; the Gram term drops out)
+ *       conv:    W1[c][a][b] = W0[c][a][b] + eta (1/N) sum_{y,x} V[c,y,x] K[c,y+a-1,x+b-1]
+ *     The MLP head does not implement it (TTT_ERR_UNSUPPORTED). */
+typedef enum { TTT_LOSS_L2 = 0, TTT_LOSS_DOT = 1 } ttt_loss;
+
 typedef struct {
     int batch;               /* images B >= 1 */
     int heads;               /* heads handled by this call >= 1 */
@@ -81,6 +93,7 @@ typedef struct {
                                 conv heads of one layer) each take a share, so that neither waits for
                                 SMs the other holds.  It may change how sums are split over CTAs, hence
                                 the rounding; results are bitwise reproducible for a fixed value. */
+    int loss;                /* ttt_loss of the inner training step (0 = TTT_LOSS_L2) */
 } ttt_shape;
 
 /* Bytes of device workspace that a call of head kind `kind` with shape `s` needs (0 on an invalid
@@ -96,7 +109,8 @@ ttt_status ttt_workspace_status(void* ws, void* stream);
 
 /* Linear inner model f(x) = W x, W in R^{d x d}.
  *   Computes per unit  G = sum_n k_n k_n^T,  C = sum_n v_n k_n^T   (fp32),
- *   W1 = W0 - eta * (2/N) * (W0 G - C)   and   z_n = W1 q_n.
+ *   W1 = W0 - eta * (2/N) * (W0 G - C)   and   z_n = W1 q_n
+ *   (TTT_LOSS_DOT: W1 = W0 + eta * (1/N) * C; G is not used).
  *   W0:     [heads][d][d] fp32 (W0[i][j] maps input feature j to output feature i).
  *   W1_out: optional (NULL = not written) [batch][heads][d][d] fp32, the updated weights.
  */
@@ -109,7 +123,7 @@ ttt_status ttt_forward_linear(const void* Q, const void* K, const void* V, const
  * one kernel per feature channel c:
  *   f(X;W)[c,y,x] = sum_{a,b=0..2} W[c][a][b] X[c, y+a-1, x+b-1].
  *   r = f(K;W0) - V;  g[c][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c,y+a-1,x+b-1];  W1 = W0 - eta g;
- *   Z = f(Q;W1).
+ *   Z = f(Q;W1).   (TTT_LOSS_DOT: g[c][a][b] = -(1/N) sum_{y,x} V[c,y,x] K[c,y+a-1,x+b-1].)
  *   W0:     [heads][d][3][3] fp32.   W1_out: optional [batch][heads][d][3][3] fp32.
  *   The workspace holds per-(image, head) partial sums and counters (about 25 KB per unit at 78 x 78
  *   tokens); after a TTT_ERR_TIMEOUT it must be zero-filled again (ttt_workspace_init).
@@ -126,7 +140,7 @@ ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const
  *   z = Wb1 gelu(Wa1 q).
  *   Wa: [heads][hidden][d] fp32,  Wb: [heads][d][hidden] fp32.
  *   Wa_out / Wb_out: optional [batch][heads][hidden][d] / [batch][heads][d][hidden] fp32.
- *   bf16 only (fp32 returns TTT_ERR_UNSUPPORTED).
+ *   bf16 and TTT_LOSS_L2 only (fp32 or TTT_LOSS_DOT returns TTT_ERR_UNSUPPORTED).
  */
 ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const float* Wa,
                            const float* Wb, void* Z, float eta, const ttt_shape* s, void* ws,
@@ -162,7 +176,7 @@ ttt_status ttt_forward_linear_noalloc(const void* Q, const void* K, const void* 
  * a programmatic dependent, starts as soon as every linear CTA is resident and runs on the SMs the
  * linear kernel leaves free (its work split for that many CTAs).  The call is complete on `stream`
  * when both kernels are.  Results equal those of the two separate calls given the same SM budgets
- * (linear: its share; conv: the SMs left to it).
+ * (linear: its share; conv: the SMs left to it).  s->loss applies to both ranges.
  *   W0_lin: [heads - conv_heads][d][d], W0_conv: [conv_heads][d][3][3] (each may be NULL when its
  *   range is empty).  W1_lin_out / W1_conv_out: optional, as in the two calls above.
  *   ws: ttt_layer_workspace_bytes(s, conv_heads) bytes, zero-filled once (ttt_workspace_init); its

@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings_and_version(lib):
     assert capi.status_string(capi.TTT_OK) == "TTT_OK"
     assert capi.status_string(capi.TTT_ERR_TIMEOUT) == "TTT_ERR_TIMEOUT"
-    assert capi.ttt_version() >= 100
+    assert capi.ttt_version() >= 103
 
 
 def _shape(**kw):
@@ -86,6 +86,8 @@ def test_layer_rejects_bad_head_split(lib):
     (dict(H=0), capi.TTT_ERR_INVALID_ARG),
     (dict(dtype=5), capi.TTT_ERR_INVALID_ARG),
     (dict(max_sms=-1), capi.TTT_ERR_INVALID_ARG),
+    (dict(loss=2), capi.TTT_ERR_INVALID_ARG),
+    (dict(loss=-1), capi.TTT_ERR_INVALID_ARG),
     (dict(head_stride=100), capi.TTT_ERR_INVALID_ARG),          # heads would overlap
     (dict(head_stride=6084 * 64 + 4), capi.TTT_ERR_ALIGNMENT),  # not a 16-byte multiple for bf16
 ])
@@ -113,6 +115,21 @@ def test_mlp_rejects_unsupported_requests(lib):
     s = _shape(hidden=100)
     assert capi.ttt_forward_mlp(None, None, None, None, None, None, 0.5, s, None, 0, None, None, None) == \
         capi.TTT_ERR_INVALID_ARG
+    s = _shape(hidden=256, loss=capi.TTT_LOSS_DOT)       # the MLP head implements the L2 loss only
+    assert capi.ttt_forward_mlp(None, None, None, None, None, None, 0.5, s, None, 0, None, None, None) == \
+        capi.TTT_ERR_UNSUPPORTED
+    assert capi.ttt_workspace_bytes(capi.TTT_HEAD_MLP, s) == 0
+
+
+def test_dot_loss_shapes_size_like_l2(lib):
+    """The dot-product loss uses the same workspaces as the L2 loss."""
+    for kind in (capi.TTT_HEAD_LINEAR, capi.TTT_HEAD_DWCONV):
+        for dt in (capi.TTT_BF16, capi.TTT_FP32):
+            a = capi.ttt_workspace_bytes(kind, _shape(dtype=dt))
+            b = capi.ttt_workspace_bytes(kind, _shape(dtype=dt, loss=capi.TTT_LOSS_DOT))
+            assert a == b and a > 0
+    s = _shape(heads=6, loss=capi.TTT_LOSS_DOT)
+    assert capi.ttt_layer_workspace_bytes(s, 1) == capi.ttt_layer_workspace_bytes(_shape(heads=6), 1)
 
 
 def test_selftest_rejects_bad_arguments(lib):

@@ -11,6 +11,7 @@ TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_ALIGNMENT = 0, 1, 2, 3
 TTT_ERR_WORKSPACE, TTT_ERR_CUDA, TTT_ERR_TIMEOUT = 4, 5, 6
 TTT_FP32, TTT_BF16 = 0, 1
 TTT_HEAD_LINEAR, TTT_HEAD_DWCONV, TTT_HEAD_MLP = 0, 1, 2
+TTT_LOSS_L2, TTT_LOSS_DOT = 0, 1
 
 # Every symbol that include/ttt.h declares.
 EXPORTED = (
@@ -26,7 +27,7 @@ class TttShape(ctypes.Structure):
         ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
         ("d", ctypes.c_int), ("hidden", ctypes.c_int),
         ("batch_stride", ctypes.c_longlong), ("head_stride", ctypes.c_longlong),
-        ("dtype", ctypes.c_int), ("max_sms", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("max_sms", ctypes.c_int), ("loss", ctypes.c_int),
     ]
 
 
@@ -84,8 +85,8 @@ def status_string(st):
     return lib().ttt_status_string(int(st)).decode()
 
 
-def make_shape(batch, heads, H, W, d, batch_stride, head_stride, dtype, hidden=0, max_sms=0):
-    return TttShape(batch, heads, H, W, d, hidden, batch_stride, head_stride, dtype, max_sms)
+def make_shape(batch, heads, H, W, d, batch_stride, head_stride, dtype, hidden=0, max_sms=0, loss=TTT_LOSS_L2):
+    return TttShape(batch, heads, H, W, d, hidden, batch_stride, head_stride, dtype, max_sms, loss)
 
 
 def ttt_workspace_bytes(kind, shape):

@@ -95,12 +95,14 @@ static ttt_status check_shape(int kind, const ttt_shape* s) {
     if ((long long)s->H * s->W > (1LL << 30)) return TTT_ERR_INVALID_ARG;
     if (s->dtype != TTT_FP32 && s->dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
     if (s->batch_stride < 0 || s->head_stride < 0 || s->max_sms < 0) return TTT_ERR_INVALID_ARG;
+    if (s->loss != TTT_LOSS_L2 && s->loss != TTT_LOSS_DOT) return TTT_ERR_INVALID_ARG;
     if ((long long)s->batch * s->heads > (1LL << 24)) return TTT_ERR_INVALID_ARG;
     if (s->d != 64) return TTT_ERR_UNSUPPORTED;
     if (kind == TTT_HEAD_MLP) {
         if (s->hidden < 64 || s->hidden % 64 != 0) return TTT_ERR_INVALID_ARG;
         if (s->hidden > 256) return TTT_ERR_UNSUPPORTED;
         if (s->dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+        if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
     }
     const long long N = (long long)s->H * s->W;
     const long long span = N * s->d;
@@ -170,6 +172,7 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
     c->hs = (s->heads > 1) ? s->head_stride : (long long)c->N * s->d;
     c->bs = (s->batch > 1) ? s->batch_stride : c->hs * s->heads;
     c->dtype = s->dtype;
+    c->loss = s->loss;
     c->ws = static_cast<uint8_t*>(ws);
     c->ws_bytes = ws_bytes;
     c->stream = static_cast<cudaStream_t>(stream);
@@ -359,6 +362,6 @@ const char* ttt_status_string(ttt_status st) {
 
 ttt_status ttt_last_error(void) { return g_sticky.load() ? TTT_ERR_CUDA : TTT_OK; }
 
-int ttt_version(void) { return 102; }
+int ttt_version(void) { return 103; }
 
 }  // extern "C"

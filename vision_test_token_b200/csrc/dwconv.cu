@@ -4,6 +4,9 @@
 //     r[c,y,x] = sum_{a,b} W0[c][a][b] K[c,y+a-1,x+b-1] - V[c,y,x]           (zero padding)
 //     g[c][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c,y+a-1,x+b-1],   W1 = W0 - eta g
 //     Z[c,y,x] = sum_{a,b} W1[c][a][b] Q[c,y+a-1,x+b-1]
+// With the dot-product inner loss of the ViT^3 recipe (same article, section on the ViT3 model),
+// L = -(1/N) sum <f(K;W), V>, the gradient has no residual: g[c][a][b] = -(1/N) sum V K[shifted]
+// (the kernel's DOT instantiation, half the phase-1 FMAs).
 //
 // Not a contraction worth a tensor core (about 7 flop per byte): fp32 FMA in registers.
 //
@@ -215,8 +218,9 @@ __device__ __forceinline__ void neg_residual2(const float2 (&win)[4][3], const f
 
 // Phase-1 work of output column x (strip-relative) of the row pair: window columns L, M, R hold
 // staged columns x, x+1, x+2 (image columns x-1, x, x+1); R is loaded here.  nw = -W0 taps;
-// gacc accumulates sum s * K with s = V - W0 (*) K = -r.
-template <typename T, bool ROW1, int L, int M, int R>
+// gacc accumulates sum s * K with s = V - W0 (*) K = -r (L2 loss) or s = V (dot-product loss, whose
+// gradient has no residual: nw is unused).
+template <typename T, bool DOT, bool ROW1, int L, int M, int R>
 __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[TAPS], float2 (&gacc)[TAPS],
                                        const Rows& rw, const uint8_t* vg, int XT, int x, int lane) {
     using E = Elem<T>;
@@ -227,8 +231,13 @@ __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[T
         // both rows' residual chains side by side (six independent 3-term chains), then the nine
         // row-0 updates before the nine row-1 updates, so that no update waits on the one before it
         float2 s0, s1;
-        neg_residual2<L, M, R>(win, nw, E::unpack(vr[(size_t)x * D / 2 + lane]),
-                               E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]), s0, s1);
+        if (DOT) {
+            s0 = E::unpack(vr[(size_t)x * D / 2 + lane]);
+            s1 = E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]);
+        } else {
+            neg_residual2<L, M, R>(win, nw, E::unpack(vr[(size_t)x * D / 2 + lane]),
+                                   E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]), s0, s1);
+        }
 #pragma unroll
         for (int a = 0; a < 3; ++a)
 #pragma unroll
@@ -238,7 +247,8 @@ __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[T
 #pragma unroll
             for (int c = 0; c < 3; ++c) gacc[a * 3 + c] = ffma2(s1, win[a + 1][cidx[c]], gacc[a * 3 + c]);
     } else {
-        const float2 s0 = neg_residual<L, M, R>(win, nw, 0, E::unpack(vr[(size_t)x * D / 2 + lane]));
+        const float2 v0 = E::unpack(vr[(size_t)x * D / 2 + lane]);
+        const float2 s0 = DOT ? v0 : neg_residual<L, M, R>(win, nw, 0, v0);
 #pragma unroll
         for (int a = 0; a < 3; ++a)
 #pragma unroll
@@ -246,7 +256,7 @@ __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[T
     }
 }
 
-template <typename T, bool ROW1>
+template <typename T, bool DOT, bool ROW1>
 __device__ __forceinline__ void p1_pair(const float2 (&nw)[TAPS], float2 (&gacc)[TAPS], const Rows& rw,
                                         const uint8_t* vg, int XT, int xa, int xb, int lane) {
     float2 win[4][3];
@@ -254,13 +264,13 @@ __device__ __forceinline__ void p1_pair(const float2 (&nw)[TAPS], float2 (&gacc)
     load_col<T, 1>(win, rw, xa + 1, lane);
     int x = xa;
     for (; x + 3 <= xb; x += 3) {
-        p1_col<T, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
-        p1_col<T, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
-        p1_col<T, ROW1, 2, 0, 1>(win, nw, gacc, rw, vg, XT, x + 2, lane);
+        p1_col<T, DOT, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
+        p1_col<T, DOT, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
+        p1_col<T, DOT, ROW1, 2, 0, 1>(win, nw, gacc, rw, vg, XT, x + 2, lane);
     }
     if (x < xb) {
-        p1_col<T, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
-        if (x + 1 < xb) p1_col<T, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
+        p1_col<T, DOT, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
+        if (x + 1 < xb) p1_col<T, DOT, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
     }
 }
 
@@ -300,7 +310,7 @@ __device__ __forceinline__ void p2_pair(const float2 (&w)[TAPS], const Rows& rw,
     }
 }
 
-template <typename T>
+template <typename T, bool DOT>
 __global__ void __launch_bounds__(THREADS, 1)
 dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
          const __grid_constant__ CUtensorMap tmQ, T* __restrict__ Z, const Params p) {
@@ -407,8 +417,9 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
             float2 nw[TAPS], gacc[TAPS];
 #pragma unroll
             for (int t9 = 0; t9 < TAPS; ++t9) {
-                nw[t9] = make_float2(-__ldg(p.W0 + ((size_t)h * D + 2 * lane) * TAPS + t9),
-                                     -__ldg(p.W0 + ((size_t)h * D + 2 * lane + 1) * TAPS + t9));
+                nw[t9] = DOT ? make_float2(0.f, 0.f)
+                             : make_float2(-__ldg(p.W0 + ((size_t)h * D + 2 * lane) * TAPS + t9),
+                                           -__ldg(p.W0 + ((size_t)h * D + 2 * lane + 1) * TAPS + t9));
                 gacc[t9] = make_float2(0.f, 0.f);
             }
             for (int j = 0; j < n; ++j) {
@@ -423,8 +434,8 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                     const Rows rw{kring + (size_t)(k0 % NK) * g.kg_bytes, kring + (size_t)(k1 % NK) * g.kg_bytes,
                                   g.k_pitch};
                     const uint8_t* vg = vring + (size_t)(v0 % NV) * g.vg_bytes;
-                    if (2 * (tk.pa + j) + 1 < g.H) p1_pair<T, true>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
-                    else p1_pair<T, false>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
+                    if (2 * (tk.pa + j) + 1 < g.H) p1_pair<T, DOT, true>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
+                    else p1_pair<T, DOT, false>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
                 }
                 __syncwarp();
                 if (lane == 0) {
@@ -581,7 +592,7 @@ static int max_tasks_per_unit(const ttt_shape& s) {
     return ((s.W + xt - 1) / xt) * ((s.H + 1) / 2);
 }
 
-template <typename T>
+template <typename T, bool DOT>
 static ttt_status launch(const Call& c) {
     const long long units = (long long)c.batch * c.heads;
     const int grid_max = std::max(1, c.num_sms);
@@ -590,7 +601,7 @@ static ttt_status launch(const Call& c) {
     if (smem > 227 * 1024) return TTT_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(units, g.Sx * g.Hp);
     if (c.ws_bytes < L.total) return TTT_ERR_WORKSPACE;
-    cudaFuncSetAttribute(dw_queue<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(dw_queue<T, DOT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const long long T_all = 2 * units * g.tpu;
     if (T_all > (1LL << 30)) return TTT_ERR_UNSUPPORTED;
     const int grid = (int)std::max<long long>(1, std::min<long long>(grid_max, T_all));
@@ -604,7 +615,9 @@ static ttt_status launch(const Call& c) {
     p.U = (int)units;
     p.T1 = (int)(units * g.tpu);
     p.T = (int)T_all;
-    p.eta_scale = c.eta * (2.0f / (float)c.N);
+    // W1 = W0 + eta_scale * sum s K:  L2 loss s = -r, gradient (2/N) sum r K;  dot-product loss
+    // s = V, gradient -(1/N) sum V K
+    p.eta_scale = c.eta * ((DOT ? 1.0f : 2.0f) / (float)c.N);
     p.W0 = c.W0;
     p.W1_out = c.W1_out;
     p.err = reinterpret_cast<uint32_t*>(c.err_ws ? c.err_ws : c.ws);
@@ -627,7 +640,7 @@ static ttt_status launch(const Call& c) {
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = c.overlap_previous ? 1 : 0;
-    return check_launch(cudaLaunchKernelEx(&cfg, dw_queue<T>, tmK, tmV, tmQ, static_cast<T*>(c.Z), p));
+    return check_launch(cudaLaunchKernelEx(&cfg, dw_queue<T, DOT>, tmK, tmV, tmQ, static_cast<T*>(c.Z), p));
 }
 
 }  // namespace dw
@@ -643,8 +656,9 @@ size_t dwconv_ws_control_bytes(const ttt_shape& s) {
 }
 
 ttt_status launch_dwconv(const Call& c) {
-    if (c.dtype == TTT_BF16) return dw::launch<__nv_bfloat16>(c);
-    return dw::launch<float>(c);
+    const bool dot = c.loss == TTT_LOSS_DOT;
+    if (c.dtype == TTT_BF16) return dot ? dw::launch<__nv_bfloat16, true>(c) : dw::launch<__nv_bfloat16, false>(c);
+    return dot ? dw::launch<float, true>(c) : dw::launch<float, false>(c);
 }
 
 }  // namespace ttt

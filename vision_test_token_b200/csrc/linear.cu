@@ -25,6 +25,10 @@
 //
 // fp32 path (lin_p1_f32 / lin_p2_f32): plain fp32 FMA kernels (fp32 accuracy), static partition,
 // the same deterministic last-CTA merge.
+//
+// Dot-product inner loss (the ViT3 recipe of the same press article, section on the ViT3 model):
+// L = -(1/N) sum <W k_n, v_n> has gradient -(1/N) C, so W1 = W0 + eta (1/N) C.  Both paths skip the
+// W0 G product (bf16: the exchange carries C_r itself) and scale by -eta/N instead of eta 2/N.
 #include <algorithm>
 #include <mutex>
 
@@ -53,7 +57,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 //   gc: 128 x 64 floats of shared memory, w0t: 64 x kW0tPitch floats of shared memory.
 // ------------------------------------------------------------------------------------------------
 struct MergeOut {
-    float eta_scale;            // eta * 2 / N
+    int dot;                    // dot-product loss: no W0 G term
+    float eta_scale;            // eta * 2 / N  (dot-product loss: eta / N)
     const float* W0;            // [heads][64][64]
     const float* partials;      // [slots][128][64]
     float* W1_out;              // nullable [units][64][64]
@@ -115,7 +120,7 @@ __device__ void merge_unit(const MergeOut& m, int u, int h, size_t slot0, int ns
 #pragma unroll
         for (int b = 0; b < CJ; ++b) acc[a][b] = 0.f;
 #pragma unroll 2
-    for (int k = 0; k < D; ++k) {
+    for (int k = 0; k < (m.dot ? 0 : D); ++k) {
         const float4 wk = *reinterpret_cast<const float4*>(w0t + k * kW0tPitch + i0);
         float gk[CJ];
 #pragma unroll
@@ -200,7 +205,8 @@ __device__ __forceinline__ void split_bf16(const float* x, float* hi, float* lo)
 struct ClusterParams {
     int heads, U, N, CS;        // units, tokens per unit, CTAs per cluster
     int tpu1, tpu2;             // 128-token tiles and 256-token tiles per unit
-    float eta_scale;            // eta * 2 / N
+    int dot;                    // dot-product loss: P_r = C_r (no W0 G product)
+    float eta_scale;            // eta * 2 / N  (dot-product loss: -eta / N)
     const float* W0;            // [heads][64][64]
     float* W1_out;              // nullable [units][64][64]
     uint32_t* err;
@@ -330,12 +336,14 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
         //     receive barrier, then tell the peers they may push
         if (tid == 0) bulk_wait_read<0>();
         // A operand of the product: rows 0..63 = bf16(W0), rows 64..127 = bf16(W0 - bf16(W0))
+        if (!p.dot) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float hi[8], lo[8];
-            split_bf16(w0r + 8 * c, hi, lo);
-            put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
-            put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
+            for (int c = 0; c < 4; ++c) {
+                float hi[8], lo[8];
+                split_bf16(w0r + 8 * c, hi, lo);
+                put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
+                put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
+            }
         }
         named_bar_sync(1, 128);
         if (multi && tid == 0) {
@@ -366,12 +374,14 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
                     for (int e = 0; e < 16; ++e) v[j][e] = 0.f;
             }
             if (r < D) {                                      // G is symmetric: row r of G = column r
+                if (!p.dot) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float hi[8], lo[8];
-                    split_bf16(&v[c / 2][(c & 1) * 8], hi, lo);
-                    put_bf16_chunk(bhi, r, c, hi);
-                    put_bf16_chunk(blo, r, c, lo);
+                    for (int c = 0; c < 8; ++c) {
+                        float hi[8], lo[8];
+                        split_bf16(&v[c / 2][(c & 1) * 8], hi, lo);
+                        put_bf16_chunk(bhi, r, c, hi);
+                        put_bf16_chunk(blo, r, c, lo);
+                    }
                 }
             } else {
 #pragma unroll
@@ -385,52 +395,55 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
         mbar_arrive(&s.pacc_empty);
         fence_proxy_async_smem();                             // the operands are read by the tensor cores
         named_bar_sync(1, 128);
-        // (3) D = [W0_hi ; W0_lo] (G_hi + G_lo) on the tensor cores (M = 128, N = 64, K = 64 twice)
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t sa = smem_u32(s.a01), sh = smem_u32(bhi), sl = smem_u32(blo);
+        // (3) D = [W0_hi ; W0_lo] (G_hi + G_lo) on the tensor cores (M = 128, N = 64, K = 64 twice);
+        //     steps (3) and (4) only for the L2 loss (the dot-product loss sends P = C)
+        if (!p.dot) {
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t sa = smem_u32(s.a01), sh = smem_u32(bhi), sl = smem_u32(blo);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sh + kk * 32, 16, 1024),
-                            kIdescP2, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sh + kk * 32, 16, 1024),
+                                kIdescP2, kk > 0 ? 1u : 0u);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sl + kk * 32, 16, 1024),
-                            kIdescP2, 1u);
-            mma_commit(&s.prod_bar);
-        }
-        ok = mbar_wait(&s.prod_bar, k & 1u, ab);
-        if (named_bar_or(1, 128, !ok)) { failed = true; break; }
-        __syncwarp();
-        tc_fence_after();
-        // (4) P = D[0:64] + D[64:128] - C  (= W0 G - C), written over the C rows of gc
-        float* dlo = reinterpret_cast<float*>(s.a01);          // the A operand is consumed: reuse it
-        {
-            float v[4][16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 320u + (uint32_t)(j * 16) + lane_off, v[j]);
-            tmem_ld_wait();
-            tc_fence_before();
-            if (r >= D) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-#pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *gc_chunk(dlo, r - D, (j * 16 + e) / 4) = make_float4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sl + kk * 32, 16, 1024),
+                                kIdescP2, 1u);
+                mma_commit(&s.prod_bar);
             }
-            named_bar_sync(1, 128);
-            if (r < D) {
+            ok = mbar_wait(&s.prod_bar, k & 1u, ab);
+            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+            __syncwarp();
+            tc_fence_after();
+            // (4) P = D[0:64] + D[64:128] - C  (= W0 G - C), written over the C rows of gc
+            float* dlo = reinterpret_cast<float*>(s.a01);          // the A operand is consumed: reuse it
+            {
+                float v[4][16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 320u + (uint32_t)(j * 16) + lane_off, v[j]);
+                tmem_ld_wait();
+                tc_fence_before();
+                if (r >= D) {
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
-                        const int c = (j * 16 + e) / 4;
-                        const float4 l = *gc_chunk(dlo, r, c);
-                        float4* cp = gc_chunk(s.gc, D + r, c);
-                        const float4 cv = *cp;
-                        *cp = make_float4(v[j][e] + l.x - cv.x, v[j][e + 1] + l.y - cv.y, v[j][e + 2] + l.z - cv.z,
-                                          v[j][e + 3] + l.w - cv.w);
-                    }
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            *gc_chunk(dlo, r - D, (j * 16 + e) / 4) = make_float4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
+                }
+                named_bar_sync(1, 128);
+                if (r < D) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4) {
+                            const int c = (j * 16 + e) / 4;
+                            const float4 l = *gc_chunk(dlo, r, c);
+                            float4* cp = gc_chunk(s.gc, D + r, c);
+                            const float4 cv = *cp;
+                            *cp = make_float4(v[j][e] + l.x - cv.x, v[j][e + 1] + l.y - cv.y, v[j][e + 2] + l.z - cv.z,
+                                              v[j][e + 3] + l.w - cv.w);
+                        }
+                }
             }
         }
         const float* Pme = s.gc + D * D;                      // rows 64..127 of gc
@@ -449,7 +462,7 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
         } else {
             named_bar_sync(1, 128);
         }
-        // (6) W1 = W0 - eta (2/N) sum_r P_r  (ranks in order: deterministic); W1_out from rank 0
+        // (6) W1 = W0 - eta_scale sum_r P_r  (ranks in order: deterministic); W1_out from rank 0
         ok = ok && mbar_wait(&s.w_empty, (k & 1u) ^ 1u, ab);  // phase 2 of the previous unit is done with w1
         if (named_bar_or(1, 128, !ok)) { failed = true; break; }
         {
@@ -821,7 +834,8 @@ ttt_status launch_linear(const Call& c) {
         p.CS = cs;
         p.tpu1 = tpu;
         p.tpu2 = (c.N + Q2 - 1) / Q2;
-        p.eta_scale = c.eta * (2.0f / (float)c.N);
+        p.dot = c.loss == TTT_LOSS_DOT;
+        p.eta_scale = p.dot ? -c.eta / (float)c.N : c.eta * (2.0f / (float)c.N);
         p.W0 = c.W0;
         p.W1_out = c.W1_out;
         p.err = reinterpret_cast<uint32_t*>(c.ws);
@@ -844,7 +858,8 @@ ttt_status launch_linear(const Call& c) {
     }
 
     MergeOut m{};
-    m.eta_scale = c.eta * (2.0f / (float)c.N);
+    m.dot = c.loss == TTT_LOSS_DOT;
+    m.eta_scale = m.dot ? c.eta / (float)c.N : c.eta * (2.0f / (float)c.N);
     m.W0 = c.W0;
     m.partials = reinterpret_cast<const float*>(c.ws + L.partials);
     m.W1_out = c.W1_out;

@@ -31,6 +31,7 @@ struct Call {
     int batch, heads, H, W, N, d, hidden;
     long long bs, hs;    // element strides
     int dtype;           // ttt_dtype
+    int loss;            // ttt_loss
     uint8_t* ws;
     size_t ws_bytes;
     cudaStream_t stream;

@@ -19,6 +19,8 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
   mixed6084_bf16   5 linear heads + 1 depthwise-conv head (the last head), B 8, 78 x 78, bf16, eta 0.5
   lin6400_bf16     linear, B 4, 12 heads, 80 x 80, bf16, eta 1.0   (ViT-Base-shaped 1280^2 layer)
   mlp1024_bf16     MLP width 4d = 256, GELU(tanh), B 16, 4 heads, 32 x 32, bf16, eta 0.5
+  mixed6084_dot_bf16  as mixed6084_bf16, trained with the dot-product inner loss and eta 1.0 (the
+                   ViT3 recipe: one full-batch step, learning rate 1.0, dot-product loss)
 """
 from dataclasses import dataclass
 import math
@@ -39,6 +41,7 @@ class Workload:
     conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
     d: int = 64
     hidden_ratio: int = 4
+    loss: str = "l2"      # inner loss: "l2" or "dot"
 
     @property
     def N(self):
@@ -59,6 +62,8 @@ WORKLOADS = {
     "mixed6084_bf16": Workload("mixed6084_bf16", 8, 6, 78, 78, "bf16", 0.5, "mixed", conv_heads=1),
     "lin6400_bf16": Workload("lin6400_bf16", 4, 12, 80, 80, "bf16", 1.0, "linear"),
     "mlp1024_bf16": Workload("mlp1024_bf16", 16, 4, 32, 32, "bf16", 0.5, "mlp"),
+    "mixed6084_dot_bf16": Workload("mixed6084_dot_bf16", 8, 6, 78, 78, "bf16", 1.0, "mixed", conv_heads=1,
+                                   loss="dot"),
 }
 
 TORCH_DTYPE = {"fp32": torch.float32, "bf16": torch.bfloat16}

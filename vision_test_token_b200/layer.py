@@ -11,6 +11,8 @@ import torch
 from . import capi
 
 _DTYPES = {torch.bfloat16: capi.TTT_BF16, torch.float32: capi.TTT_FP32}
+# inner loss of the one-step training: "l2" = (1/N) sum ||f(k) - v||^2, "dot" = -(1/N) sum <f(k), v>
+_LOSSES = {"l2": capi.TTT_LOSS_L2, "dot": capi.TTT_LOSS_DOT}
 _ws_cache = {}
 
 
@@ -23,7 +25,7 @@ def _stream_handle(stream):
     return s.cuda_stream
 
 
-def _shape_of(Q, H, W, hidden=0, max_sms=0):
+def _shape_of(Q, H, W, hidden=0, max_sms=0, loss="l2"):
     if Q.dim() != 4:
         raise ValueError("Q/K/V must be [B][heads][N][d]")
     B, heads, N, d = Q.shape
@@ -33,7 +35,10 @@ def _shape_of(Q, H, W, hidden=0, max_sms=0):
         raise ValueError("token rows of Q/K/V/Z must be contiguous")
     if Q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {Q.dtype}")
-    return capi.make_shape(B, heads, H, W, d, Q.stride(0), Q.stride(1), _DTYPES[Q.dtype], hidden, max_sms)
+    if loss not in _LOSSES:
+        raise ValueError(f"loss must be one of {sorted(_LOSSES)}")
+    return capi.make_shape(B, heads, H, W, d, Q.stride(0), Q.stride(1), _DTYPES[Q.dtype], hidden, max_sms,
+                           _LOSSES[loss])
 
 
 def _same_layout(ref, *others):
@@ -43,16 +48,21 @@ def _same_layout(ref, *others):
 
 
 def workspace(kind, shape, device):
-    """A zero-initialised workspace for (kind, shape) on `device`, cached and reused."""
+    """A zero-initialised workspace for (kind, shape) on `device`, cached and reused.  None when the
+    library sizes none (an invalid or unsupported shape: the call itself then reports why)."""
     nbytes = capi.ttt_workspace_bytes(kind, shape)
     if nbytes == 0:
-        raise capi.TttError(capi.TTT_ERR_INVALID_ARG, "ttt_workspace_bytes")
+        return None
     key = (kind, str(device), nbytes)
     ws = _ws_cache.get(key)
     if ws is None:
         ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         _ws_cache[key] = ws
     return ws
+
+
+def _ws_args(ws):
+    return (None, 0) if ws is None else (_ptr(ws), ws.numel())
 
 
 def _check(st, where):
@@ -68,54 +78,57 @@ def _out_like(Q, Z):
     return Z
 
 
-def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0):
+def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0, loss="l2"):
     """Linear inner model.  W0: [heads][d][d] fp32 CUDA tensor.  Returns Z.  `max_sms` (0 = all)
-    bounds the SMs the call spreads over."""
-    shape = _shape_of(Q, H, W, max_sms=max_sms)
+    bounds the SMs the call spreads over; `loss` is "l2" or "dot" (the inner loss)."""
+    shape = _shape_of(Q, H, W, max_sms=max_sms, loss=loss)
     Z = _out_like(Q, Z)
     _same_layout(Q, K, V, Z)
     W0 = W0.contiguous()
     if ws is None:
         ws = workspace(capi.TTT_HEAD_LINEAR, shape, Q.device)
-    st = capi.ttt_forward_linear(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, _ptr(ws),
-                                 ws.numel(), _ptr(W1_out), _stream_handle(stream))
+    st = capi.ttt_forward_linear(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, *_ws_args(ws),
+                                 _ptr(W1_out), _stream_handle(stream))
     _check(st, "ttt_forward_linear")
     return Z
 
 
-def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0):
+def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0, loss="l2"):
     """3x3 depthwise-conv inner model.  W0: [heads][d][3][3] fp32 CUDA tensor.  Returns Z."""
-    shape = _shape_of(Q, H, W, max_sms=max_sms)
+    shape = _shape_of(Q, H, W, max_sms=max_sms, loss=loss)
     Z = _out_like(Q, Z)
     _same_layout(Q, K, V, Z)
     W0 = W0.contiguous()
     if ws is None:
         ws = workspace(capi.TTT_HEAD_DWCONV, shape, Q.device)
-    st = capi.ttt_forward_dwconv(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, _ptr(ws),
-                                 ws.numel(), _ptr(W1_out), _stream_handle(stream))
+    st = capi.ttt_forward_dwconv(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, *_ws_args(ws),
+                                 _ptr(W1_out), _stream_handle(stream))
     _check(st, "ttt_forward_dwconv")
     return Z
 
 
-def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws=None, stream=None, max_sms=0):
-    """One-hidden-layer GELU MLP inner model.  Wa: [heads][hidden][d], Wb: [heads][d][hidden]."""
-    shape = _shape_of(Q, H, W, hidden=Wa.shape[1], max_sms=max_sms)
+def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws=None, stream=None, max_sms=0,
+                loss="l2"):
+    """One-hidden-layer GELU MLP inner model.  Wa: [heads][hidden][d], Wb: [heads][d][hidden].
+    Only the "l2" loss is implemented (the library rejects "dot" with TTT_ERR_UNSUPPORTED)."""
+    shape = _shape_of(Q, H, W, hidden=Wa.shape[1], max_sms=max_sms, loss=loss)
     Z = _out_like(Q, Z)
     _same_layout(Q, K, V, Z)
     Wa, Wb = Wa.contiguous(), Wb.contiguous()
     if ws is None:
         ws = workspace(capi.TTT_HEAD_MLP, shape, Q.device)
     st = capi.ttt_forward_mlp(_ptr(Q), _ptr(K), _ptr(V), _ptr(Wa), _ptr(Wb), _ptr(Z), float(eta), shape,
-                              _ptr(ws), ws.numel(), _ptr(Wa_out), _ptr(Wb_out), _stream_handle(stream))
+                              *_ws_args(ws), _ptr(Wa_out), _ptr(Wb_out), _stream_handle(stream))
     _check(st, "ttt_forward_mlp")
     return Z
 
 
 def layer_workspace(shape, conv_heads, device):
-    """A zero-initialised workspace for ttt_forward_layer(shape, conv_heads), cached and reused."""
+    """A zero-initialised workspace for ttt_forward_layer(shape, conv_heads), cached and reused (None
+    when the library sizes none)."""
     nbytes = capi.ttt_layer_workspace_bytes(shape, conv_heads)
     if nbytes == 0:
-        raise capi.TttError(capi.TTT_ERR_INVALID_ARG, "ttt_layer_workspace_bytes")
+        return None
     key = ("layer", str(device), nbytes)
     ws = _ws_cache.get(key)
     if ws is None:
@@ -125,7 +138,7 @@ def layer_workspace(shape, conv_heads, device):
 
 
 def forward_layer(Q, K, V, weights, eta, H, W, conv_heads=0, Z=None, W1_lin_out=None, W1_conv_out=None, ws=None,
-                  stream=None, concurrent=True, max_sms=0):
+                  stream=None, concurrent=True, max_sms=0, loss="l2"):
     """A layer whose first heads are linear and whose last `conv_heads` heads are depthwise-conv
     heads, over head ranges of the same buffers.  weights: {"W0_lin": [heads-conv_heads][d][d],
     "W0_conv": [conv_heads][d][3][3]}.  With `concurrent` (the default) one ttt_forward_layer call
@@ -138,20 +151,20 @@ def forward_layer(Q, K, V, weights, eta, H, W, conv_heads=0, Z=None, W1_lin_out=
     W0l = weights["W0_lin"].contiguous() if nl else None
     W0c = weights["W0_conv"].contiguous() if conv_heads else None
     if concurrent:
-        shape = _shape_of(Q, H, W, max_sms=max_sms)
+        shape = _shape_of(Q, H, W, max_sms=max_sms, loss=loss)
         if ws is None:
             ws = layer_workspace(shape, conv_heads, Q.device)
         st = capi.ttt_forward_layer(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0l), _ptr(W0c), _ptr(Z), float(eta), shape,
-                                    conv_heads, _ptr(ws), ws.numel(), _ptr(W1_lin_out), _ptr(W1_conv_out),
+                                    conv_heads, *_ws_args(ws), _ptr(W1_lin_out), _ptr(W1_conv_out),
                                     _stream_handle(stream))
         _check(st, "ttt_forward_layer")
         return Z
     if nl:
         forward_linear(Q[:, :nl], K[:, :nl], V[:, :nl], W0l, eta, H, W, Z=Z[:, :nl], W1_out=W1_lin_out,
-                       stream=stream, max_sms=max_sms)
+                       stream=stream, max_sms=max_sms, loss=loss)
     if conv_heads:
         forward_dwconv(Q[:, nl:], K[:, nl:], V[:, nl:], W0c, eta, H, W, Z=Z[:, nl:], W1_out=W1_conv_out,
-                       stream=stream, max_sms=max_sms)
+                       stream=stream, max_sms=max_sms, loss=loss)
     return Z
 
 
