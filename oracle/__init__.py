@@ -36,10 +36,12 @@ def _load():
         lib.oracle_linear.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_linear_gram.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_linear_dot.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_linear_minibatch.argtypes = [i, i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv_dot.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
-        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_dwconv,
+        for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_linear_minibatch,
+                  lib.oracle_dwconv,
                   lib.oracle_dwconv_dot, lib.oracle_mlp):
             f.restype = ctypes.c_int
         lib.oracle_gelu_tanh.argtypes = [d]
@@ -98,6 +100,22 @@ def linear_dot(Q, K, V, W0, eta, threads=None):
     W1 = np.empty((B, H, d, d))
     _check(_load().oracle_linear_dot(B, H, N, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1), _p(Z),
                                      threads or default_threads()), "linear_dot")
+    return Z, W1
+
+
+def linear_minibatch(Q, K, V, W0, eta, b, mode, threads=None):
+    """Linear inner model trained by mini-batch gradient descent over consecutive batches of b
+    tokens.  mode "prefix": causal prefix sums inside a batch, z_t = W_t q_t; mode "epoch": one
+    mean-gradient step per batch, every query read out with the final weights.
+    Returns (Z [B][h][N][d], W1 [B][h][d][d]: the weights after the last batch) in float64."""
+    Q, K, V, W0 = _f64(Q), _f64(K), _f64(V), _f64(W0)
+    B, H, N, d = Q.shape
+    assert K.shape == Q.shape and V.shape == Q.shape and W0.shape == (H, d, d)
+    m = {"prefix": 0, "epoch": 1}[mode]
+    Z = np.empty_like(Q)
+    W1 = np.empty((B, H, d, d))
+    _check(_load().oracle_linear_minibatch(B, H, N, d, int(b), m, _p(Q), _p(K), _p(V), _p(W0), float(eta),
+                                           _p(W1), _p(Z), threads or default_threads()), "linear_minibatch")
     return Z, W1
 
 

@@ -222,6 +222,98 @@ int oracle_linear_dot(int B, int heads, int N, int d, const double* Q, const dou
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Linear inner model trained by mini-batch gradient descent over consecutive token batches.    */
+/*   The tokens, in raster order, are cut into consecutive mini-batches of b tokens (the last     */
+/*   may be shorter).  In every mini-batch the per-token gradients are taken at the weights W_s   */
+/*   the mini-batch starts from:  G_t = 2 (W_s k_t - v_t) k_t^T  (L2 loss, the notes' G_t).       */
+/*   mode 0, prefix ("Vision-TTT" paper notes, section 关键设计 4): inside a mini-batch the       */
+/*     weights follow the causal prefix sum  W_t = W_s - eta * sum_{s<=t} G_s  and token t reads  */
+/*     out z_t = W_t q_t; the next mini-batch starts from the last W_t.                          */
+/*   mode 1, epoch (press article, Observation 2 and Fig. 3: the dataset cut into 2, 3 or 4       */
+/*     consecutive mini-batches, one parameter update per mini-batch): every mini-batch takes    */
+/*     one step of its mean L2 loss,  W <- W_s - eta (2/|batch|) sum_t (W_s k_t - v_t) k_t^T,    */
+/*     and every query is read out with the weights after the last mini-batch.  With b >= N     */
+/*     this is the full-batch step above.                                                       */
+/* ------------------------------------------------------------------------------------------ */
+
+static int linear_minibatch_unit(int N, int d, int b, int mode, const double* Q, const double* K,
+                                 const double* V, const double* W0, double eta, double* W1, double* Z)
+{
+    double* Ws = (double*)malloc((size_t)d * d * sizeof(double));   /* weights at the batch start */
+    double* Wt = (double*)malloc((size_t)d * d * sizeof(double));   /* running weights */
+    double* R = (double*)malloc((size_t)b * d * sizeof(double));    /* residuals of the batch */
+    if (!Ws || !Wt || !R) { free(Ws); free(Wt); free(R); return ORACLE_ERR_NOMEM; }
+    memcpy(Ws, W0, (size_t)d * d * sizeof(double));
+    for (int start = 0; start < N; start += b) {
+        const int end = (start + b < N) ? start + b : N;
+        const int nb = end - start;
+        for (int t = start; t < end; ++t) {                 /* r_t = W_s k_t - v_t */
+            const double* k = K + (size_t)t * d;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += Ws[(size_t)i * d + j] * k[j];
+                R[(size_t)(t - start) * d + i] = acc - V[(size_t)t * d + i];
+            }
+        }
+        memcpy(Wt, Ws, (size_t)d * d * sizeof(double));
+        /* prefix: step -eta*G_t after each token; epoch: the batch mean, one step */
+        const double step = (mode == 0) ? eta : eta / (double)nb;
+        for (int t = start; t < end; ++t) {
+            const double* k = K + (size_t)t * d;
+            const double* r = R + (size_t)(t - start) * d;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j) Wt[(size_t)i * d + j] -= step * 2.0 * r[i] * k[j];
+            if (mode == 0) {                                 /* z_t = W_t q_t */
+                const double* q = Q + (size_t)t * d;
+                for (int i = 0; i < d; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < d; ++j) acc += Wt[(size_t)i * d + j] * q[j];
+                    Z[(size_t)t * d + i] = acc;
+                }
+            }
+        }
+        memcpy(Ws, Wt, (size_t)d * d * sizeof(double));
+    }
+    if (mode == 1) {                                         /* readout with the final weights */
+        for (int t = 0; t < N; ++t) {
+            const double* q = Q + (size_t)t * d;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += Ws[(size_t)i * d + j] * q[j];
+                Z[(size_t)t * d + i] = acc;
+            }
+        }
+    }
+    memcpy(W1, Ws, (size_t)d * d * sizeof(double));
+    free(Ws); free(Wt); free(R);
+    return ORACLE_OK;
+}
+
+int oracle_linear_minibatch(int B, int heads, int N, int d, int b, int mode, const double* Q,
+                            const double* K, const double* V, const double* W0, double eta,
+                            double* W1, double* Z, int nthreads)
+{
+    if (B < 0 || heads < 0 || N < 1 || d < 1 || b < 1 || (mode != 0 && mode != 1) || !Q || !K || !V ||
+        !W0 || !W1 || !Z)
+        return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int h = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        int st = linear_minibatch_unit(N, d, b, mode, Q + off, K + off, V + off, W0 + (size_t)h * d * d,
+                                       eta, W1 + (size_t)u * d * d, Z + off);
+        if (st != ORACLE_OK) {
+#pragma omp atomic write
+            status = st;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* 3x3 depthwise-convolution inner model over the H x W token grid                             */
 /* (press article, Observation 6 and Fig. 5 part 3; ViT3 news article, 原則六 and section      */
 /* 效果全面驗證: one head uses a 3x3 depthwise convolution).                                     */

@@ -248,6 +248,103 @@ def test_linear_dot_matches_torch_autograd():
 
 
 # ------------------------------------------------------------------------------------------------
+# linear head, mini-batch gradient descent over consecutive token batches
+# ------------------------------------------------------------------------------------------------
+def _per_token_ttt(Q, K, V, W0, eta):
+    """Brute force of per-token sequential TTT (each token one step at the current weights):
+    W_t = W_{t-1} - eta * 2 (W_{t-1} k_t - v_t) k_t^T,  z_t = W_t q_t."""
+    W = W0.copy()
+    Z = np.empty_like(Q)
+    for t in range(Q.shape[0]):
+        W = W - eta * 2.0 * np.outer(W @ K[t] - V[t], K[t])
+        Z[t] = W @ Q[t]
+    return Z, W
+
+
+def test_minibatch_prefix_b1_is_per_token_ttt():
+    """With one token per mini-batch the prefix form is per-token sequential TTT."""
+    N, d, eta = 37, 8, 0.1
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, d)) / np.sqrt(d)
+    Z, W1 = oracle.linear_minibatch(Q, K, V, W0, eta, 1, "prefix")
+    Zr, Wr = _per_token_ttt(Q[0, 0], K[0, 0], V[0, 0], W0[0], eta)
+    np.testing.assert_allclose(Z[0, 0], Zr, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(W1[0, 0], Wr, atol=1e-12, rtol=0)
+
+
+def test_minibatch_prefix_single_batch_matches_full_batch_on_every_prefix():
+    """With b = N every gradient is taken at W0, so W_t is the full-batch step over tokens 0..t with
+    the mean's factor 2/(t+1) absorbed into eta: z_t = W1_full(prefix t, eta (t+1)) q_t."""
+    N, d, eta = 23, 8, 0.05
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, d)) / np.sqrt(d)
+    Z, W1 = oracle.linear_minibatch(Q, K, V, W0, eta, N, "prefix")
+    for t in range(N):
+        _, Wp = oracle.linear(Q[:, :, :t + 1], K[:, :, :t + 1], V[:, :, :t + 1], W0, eta * (t + 1))
+        np.testing.assert_allclose(Z[0, 0, t], Wp[0, 0] @ Q[0, 0, t], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(W1[0, 0], Wp[0, 0], atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("N,b", [(40, 40), (40, 64), (41, 21), (30, 10), (7, 3)])
+def test_minibatch_epoch_chains_full_batch_steps(N, b):
+    """Epoch mode = one full-batch step per consecutive mini-batch (the pinned full-batch oracle run
+    on each chunk in turn from the previous chunk's weights), then the readout of every query with
+    the final weights.  b >= N is exactly the full-batch layer."""
+    d, eta = 8, 0.7
+    Q, K, V = (RNG.standard_normal((2, 1, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, d)) / np.sqrt(d)
+    Z, W1 = oracle.linear_minibatch(Q, K, V, W0, eta, b, "epoch")
+    for img in range(2):
+        W = W0.copy()
+        for s0 in range(0, N, b):
+            sl = slice(s0, min(N, s0 + b))
+            _, Wn = oracle.linear(Q[img:img + 1, :, sl], K[img:img + 1, :, sl], V[img:img + 1, :, sl], W, eta)
+            W = Wn[0]
+        np.testing.assert_allclose(W1[img, 0], W[0], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(Z[img, 0], Q[img, 0] @ W[0].T, atol=1e-12, rtol=0)
+    if b >= N:
+        Zf, W1f = oracle.linear(Q, K, V, W0, eta)
+        np.testing.assert_allclose(Z, Zf, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mode", ["prefix", "epoch"])
+def test_minibatch_invariants(mode):
+    """eta = 0 reads out through W0; values that W0 reproduces exactly give no update at all.  Keys
+    are unit rows (as in the layer's inputs), so that the prefix recurrence contracts and the
+    rounding left in V - W0 K is not amplified from batch to batch."""
+    N, d, b = 45, 8, 16
+    Q, K = RNG.standard_normal((1, 2, N, d)), RNG.standard_normal((1, 2, N, d))
+    K /= np.linalg.norm(K, axis=-1, keepdims=True)
+    W0 = RNG.standard_normal((2, d, d))
+    V = np.einsum("hij,bhnj->bhni", W0, K)
+    for eta, V_ in ((0.0, RNG.standard_normal((1, 2, N, d))), (0.2, V)):
+        Z, W1 = oracle.linear_minibatch(Q, K, V_, W0, eta, b, mode)
+        np.testing.assert_allclose(W1, np.broadcast_to(W0, W1.shape), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(Z, np.einsum("hij,bhnj->bhni", W0, Q), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mistake", ["running_weights", "mean_scale"])
+def test_planted_mistakes_fail_the_minibatch_pins(mistake):
+    """A plausible mistake planted in a CPU copy of the prefix recurrence fails the pins above:
+    gradients taken at the running weights instead of the batch's start weights (fails the b = N
+    prefix pin), or a mean instead of a sum inside the batch (fails the b = 1 pin unless b = 1,
+    so it is checked at b = N)."""
+    N, d, eta = 12, 6, 0.05
+    Q, K, V = (RNG.standard_normal((N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((d, d)) / np.sqrt(d)
+    W = W0.copy()
+    Wt = W0.copy()
+    Z = np.empty_like(Q)
+    for t in range(N):
+        Wg = Wt if mistake == "running_weights" else W
+        scale = eta / N if mistake == "mean_scale" else eta
+        Wt = Wt - scale * 2.0 * np.outer(Wg @ K[t] - V[t], K[t])
+        Z[t] = Wt @ Q[t]
+    Zo, _ = oracle.linear_minibatch(Q[None, None], K[None, None], V[None, None], W0[None], eta, N, "prefix")
+    assert not np.allclose(Z, Zo[0, 0], atol=1e-9, rtol=0)
+
+
+# ------------------------------------------------------------------------------------------------
 # depthwise 3x3 conv head
 # ------------------------------------------------------------------------------------------------
 def test_dwconv_gradient_exact_rational_fd():
