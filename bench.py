@@ -183,6 +183,11 @@ def _np64(t):
 def oracle_units(w, x, units, threads):
     """Runs the oracle on the listed (image, head) units of the workload (inputs already float64)."""
     import oracle
+    if w.kind == "minibatch":
+        for (b, h) in units:
+            oracle.linear_minibatch(x["Q"][b:b + 1, h:h + 1], x["K"][b:b + 1, h:h + 1], x["V"][b:b + 1, h:h + 1],
+                                    x["W0_lin"][h:h + 1], w.eta, w.mb_tokens, w.mb_mode, threads=threads)
+        return
     if w.kind == "mlp":
         for (b, h) in units:
             oracle.mlp(x["Q"][b:b + 1, h:h + 1], x["K"][b:b + 1, h:h + 1], x["V"][b:b + 1, h:h + 1],
@@ -282,6 +287,9 @@ def make_step(w, xs, dev):
         x = xs[i]
         if w.kind == "mlp":
             layer.forward_mlp(x["Q"], x["K"], x["V"], weights["Wa"], weights["Wb"], w.eta, w.H, w.W, Z=x["Z"])
+        elif w.kind == "minibatch":
+            layer.forward_linear_minibatch(x["Q"], x["K"], x["V"], weights["W0_lin"], w.eta, w.H, w.W, w.mb_tokens,
+                                           w.mb_mode, Z=x["Z"])
         else:
             layer.forward_layer(x["Q"], x["K"], x["V"], weights, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=x["Z"],
                                 loss=w.loss)
@@ -412,6 +420,22 @@ def run_ours(args):
                     conv_name: {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
                                        "achieved_gbs": conv_bytes / t_conv / 1e9,
                                        "frac": conv_bytes / t_conv / 1e9 / pk["hbm_gbs"]}}}
+    elif w.kind == "minibatch":
+        # a sequential FP32 recurrence: bound by plain FMA issue, not by HBM.  Algorithmic FLOPs per
+        # (token, head) are the mini-batch TTT terms 6 d^2 + 4 b d; the peak is 148 SMs x 128 FP32
+        # lanes x 2 FLOP per FMA at the SM clock sampled during the run (its maximum if no sample).
+        n = max(100, args.steps // 4)
+        time_graphs(graphs, 10, stream)
+        t_mb = time_graphs(graphs, n, stream) / n
+        flops = w.batch * w.heads * w.N * (6 * w.d * w.d + 4 * w.mb_tokens * w.d)
+        mhz = clocks.get("sm_max_mhz") or 1965.0
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        achieved = flops / t_mb / 1e12
+        roof = {"bound": "alu", "kernel": "lin_minibatch (the whole ttt_forward_linear_minibatch call)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {mhz:.0f} MHz",
+                "algorithmic_flops": flops, "us_per_launch": t_mb * 1e6,
+                "hbm_gbs": workload_bytes(w) / t_mb / 1e9}
     elif w.kind == "mlp":
         n = max(100, args.steps // 4)
         time_graphs(graphs, 10, stream)
@@ -434,6 +458,7 @@ def run_ours(args):
             "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads,
                        "lin_heads": w.lin_heads, "conv_heads": w.conv_heads, "grid": [w.H, w.W],
                        "tokens": w.N, "d": w.d, "eta": w.eta, "loss": w.loss,
+                       **({"mb_tokens": w.mb_tokens, "mb_mode": w.mb_mode} if w.kind == "minibatch" else {}),
                        "parallelism": f"batch-sharded x{world}",
                        "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",
                        "algorithmic_bytes_per_step": workload_bytes(w),
@@ -490,6 +515,9 @@ def run_e2e(w, x, dev, stream, steps, world):
         with torch.cuda.stream(stream):
             if w.kind == "mlp":
                 layer.forward_mlp(d["Q"], d["K"], d["V"], d["Wa"], d["Wb"], w.eta, w.H, w.W, Z=z_dev[bsel])
+            elif w.kind == "minibatch":
+                layer.forward_linear_minibatch(d["Q"], d["K"], d["V"], d["W0_lin"], w.eta, w.H, w.W, w.mb_tokens,
+                                               w.mb_mode, Z=z_dev[bsel])
             else:
                 layer.forward_layer(d["Q"], d["K"], d["V"], d, w.eta, w.H, w.W, conv_heads=w.conv_heads,
                                     Z=z_dev[bsel], loss=w.loss)

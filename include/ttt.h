@@ -167,6 +167,28 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
 ttt_status ttt_forward_linear_noalloc(const void* Q, const void* K, const void* V, const float* W0, void* Z,
                                       float eta, const ttt_shape* s, float* W1_out, void* stream);
 
+/* Mini-batch variants of the linear head's inner training (mode: ttt_minibatch_mode).
+ * The raster-ordered tokens are cut into consecutive mini-batches of batch_tokens tokens (the last
+ * may be shorter); in every mini-batch the per-token gradients are taken at the weights W_s the
+ * mini-batch starts from, G_t = 2 (W_s k_t - v_t) k_t^T.
+ *   TTT_MB_PREFIX ("Vision-TTT" paper notes, section 关键设计 4, b = 16 there): inside a mini-batch
+ *     W_t = W_s - eta * sum_{s <= t} G_s (a causal prefix sum, no 1/b) and z_t = W_t q_t; the next
+ *     mini-batch starts from the last W_t.  batch_tokens = 1 is per-token sequential TTT.
+ *   TTT_MB_EPOCH (press article, Observation 2 and Fig. 3: the dataset cut into 2, 3 or 4
+ *     consecutive mini-batches, one update each): W <- W_s - eta * (2/|batch|) sum (W_s k_t - v_t) k_t^T
+ *     per mini-batch, then z_n = W_final q_n for every token.  batch_tokens >= N gives the results of
+ *     ttt_forward_linear up to rounding.
+ * Computed in fp32 from bf16 or fp32 inputs (Z rounded to the input dtype).
+ *   ws: a workspace of at least 256 bytes, zero-filled once (ttt_workspace_init); its error word
+ *   reports a device-side wait that ran out (ttt_workspace_status).
+ *   W0: [heads][d][d] fp32.  W1_out: optional [batch][heads][d][d] fp32, the weights after the last
+ *   mini-batch.  s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED); s->max_sms bounds the SMs.
+ * Errors: TTT_ERR_INVALID_ARG for batch_tokens < 1 or an unknown mode, and as ttt_forward_linear. */
+typedef enum { TTT_MB_PREFIX = 0, TTT_MB_EPOCH = 1 } ttt_minibatch_mode;
+ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void* V, const float* W0,
+                                        void* Z, float eta, const ttt_shape* s, int batch_tokens, int mode,
+                                        void* ws, size_t ws_bytes, float* W1_out, void* stream);
+
 /* A layer whose heads [0, heads - conv_heads) are linear heads and whose last conv_heads heads are
  * depthwise-conv heads (ViT^3 keeps one conv head among its linear heads: press article,
  * Observation 6), over one [batch][heads][N][d] view described by s (s->heads = all heads):

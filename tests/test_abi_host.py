@@ -139,3 +139,18 @@ def test_selftest_rejects_bad_arguments(lib):
     assert capi.ttt_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 16), 256, 1000, None) == capi.TTT_ERR_ALIGNMENT
     assert capi.ttt_selftest_wait_timeout(fake, 256, 0, None) == capi.TTT_ERR_INVALID_ARG
     assert capi.ttt_selftest_wait_timeout(fake, 256, 2_000_000_000, None) == capi.TTT_ERR_INVALID_ARG
+
+
+def test_minibatch_rejects_bad_arguments(lib):
+    s = _shape()
+    fake = ctypes.c_void_p(1 << 20)
+    call = lambda shape, b, mode: capi.ttt_forward_linear_minibatch(fake, fake, fake, fake, ctypes.c_void_p(1 << 40),
+                                                                   0.5, shape, b, mode, fake, 256, None, None)
+    assert call(s, 0, capi.TTT_MB_PREFIX) == capi.TTT_ERR_INVALID_ARG          # empty mini-batches
+    assert call(s, 16, 2) == capi.TTT_ERR_INVALID_ARG                          # unknown mode
+    assert call(_shape(loss=capi.TTT_LOSS_DOT), 16, capi.TTT_MB_PREFIX) == capi.TTT_ERR_UNSUPPORTED
+    assert call(_shape(d=32), 16, capi.TTT_MB_EPOCH) == capi.TTT_ERR_UNSUPPORTED
+    assert capi.ttt_forward_linear_minibatch(None, None, None, None, None, 0.5, s, 16, capi.TTT_MB_PREFIX, fake, 256,
+                                             None, None) == capi.TTT_ERR_INVALID_ARG
+    assert capi.ttt_forward_linear_minibatch(fake, fake, fake, fake, ctypes.c_void_p(1 << 40), 0.5, s, 16,
+                                             capi.TTT_MB_PREFIX, None, 0, None, None) == capi.TTT_ERR_WORKSPACE

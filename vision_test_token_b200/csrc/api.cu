@@ -143,16 +143,17 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
     if (st != TTT_OK) return st;
     if (!Q || !K || !V || !W0 || !Z || (kind == TTT_HEAD_MLP && !W0b)) return TTT_ERR_INVALID_ARG;
     if (!std::isfinite(eta)) return TTT_ERR_INVALID_ARG;
-    if (!ws || ws_bytes < need) return TTT_ERR_WORKSPACE;
+    if (need > 0 && (!ws || ws_bytes < need)) return TTT_ERR_WORKSPACE;   // need 0: the call takes no workspace
     for (const void* p : {Q, K, V, (const void*)Z})
         if (reinterpret_cast<uintptr_t>(p) % 16) return TTT_ERR_ALIGNMENT;
     if (reinterpret_cast<uintptr_t>(W0) % 16 || (W0b && reinterpret_cast<uintptr_t>(W0b) % 16) ||
-        reinterpret_cast<uintptr_t>(ws) % 256)
+        (ws && reinterpret_cast<uintptr_t>(ws) % 256))
         return TTT_ERR_ALIGNMENT;
     const long long ext = extent_bytes(s);
     if (overlaps(Z, Q, ext) || overlaps(Z, K, ext) || overlaps(Z, V, ext)) return TTT_ERR_INVALID_ARG;
-    for (const void* p : {Q, K, V, (const void*)Z, (const void*)W0, (const void*)ws})
+    for (const void* p : {Q, K, V, (const void*)Z, (const void*)W0})
         if (!is_device_ptr(p)) return TTT_ERR_INVALID_ARG;
+    if (ws && !is_device_ptr(ws)) return TTT_ERR_INVALID_ARG;
     if (W0b && !is_device_ptr(W0b)) return TTT_ERR_INVALID_ARG;
 
     int sticky = g_sticky.load();
@@ -268,6 +269,21 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
     return launch_mlp(c);
 }
 
+ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void* V, const float* W0, void* Z,
+                                        float eta, const ttt_shape* s, int batch_tokens, int mode, void* ws,
+                                        size_t ws_bytes, float* W1_out, void* stream) {
+    ttt_status st = check_shape(TTT_HEAD_LINEAR, s);
+    if (st != TTT_OK) return st;
+    if (batch_tokens < 1 || (mode != TTT_MB_PREFIX && mode != TTT_MB_EPOCH)) return TTT_ERR_INVALID_ARG;
+    if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
+    Call c;
+    st = prepare(TTT_HEAD_LINEAR, Q, K, V, W0, nullptr, Z, eta, s, ws, ws_bytes, kWsHeader, stream, &c);
+    if (st != TTT_OK) return st;
+    if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
+    c.W1_out = W1_out;
+    return launch_linear_minibatch(c, batch_tokens, mode);
+}
+
 constexpr double kConvHeadWeight = 2.0;
 
 // The layer call works on two head ranges of one [B][heads][N][d] view: heads [0, nl) linear, heads
@@ -362,6 +378,6 @@ const char* ttt_status_string(ttt_status st) {
 
 ttt_status ttt_last_error(void) { return g_sticky.load() ? TTT_ERR_CUDA : TTT_OK; }
 
-int ttt_version(void) { return 103; }
+int ttt_version(void) { return 104; }
 
 }  // extern "C"

@@ -221,6 +221,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     }
 }
 
+// Bulk copy (the TMA engine, no tensor map, no multicast) of `bytes` from global memory into this
+// CTA's shared memory; completion is counted (complete_tx) on an mbarrier of this CTA.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // Bulk copy of `bytes` from this CTA's shared memory into another CTA's shared memory of the
 // cluster; completion is signalled (complete_tx) on an mbarrier in the destination CTA.
 __device__ __forceinline__ void bulk_s2cluster(uint32_t dst_caddr, const void* src, uint32_t bytes, uint32_t bar_caddr) {

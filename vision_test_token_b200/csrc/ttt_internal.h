@@ -64,6 +64,10 @@ ttt_status launch_dwconv(const Call& c);
 size_t mlp_ws_bytes(const ttt_shape& s);
 ttt_status launch_mlp(const Call& c);
 
+// Mini-batch linear head (its workspace is the error word only): batch_tokens >= 1, mode
+// TTT_MB_PREFIX or TTT_MB_EPOCH.
+ttt_status launch_linear_minibatch(const Call& c, int batch_tokens, int mode);
+
 // Full synchronous validation of a call (the checks every entry point runs before launching).
 ttt_status validate_call(int kind, const void* Q, const void* K, const void* V, const float* W0, const float* W0b,
                          void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, size_t need, void* stream);

@@ -21,6 +21,8 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
   mlp1024_bf16     MLP width 4d = 256, GELU(tanh), B 16, 4 heads, 32 x 32, bf16, eta 0.5
   mixed6084_dot_bf16  as mixed6084_bf16, trained with the dot-product inner loss and eta 1.0 (the
                    ViT3 recipe: one full-batch step, learning rate 1.0, dot-product loss)
+  mb16_6084_bf16   linear, B 8, 6 heads, 78 x 78, bf16, trained by mini-batch gradient descent in
+                   consecutive batches of 16 tokens (causal prefix inside a batch), eta 0.25
 """
 from dataclasses import dataclass
 import math
@@ -37,11 +39,13 @@ class Workload:
     W: int                # token grid width
     dtype: str            # "fp32" or "bf16"
     eta: float
-    kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp"
+    kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp", "minibatch" (linear)
     conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
     d: int = 64
     hidden_ratio: int = 4
     loss: str = "l2"      # inner loss: "l2" or "dot"
+    mb_tokens: int = 0    # kind "minibatch": tokens per mini-batch
+    mb_mode: str = "prefix"
 
     @property
     def N(self):
@@ -49,7 +53,7 @@ class Workload:
 
     @property
     def lin_heads(self):
-        return self.heads - self.conv_heads if self.kind in ("linear", "mixed") else 0
+        return self.heads - self.conv_heads if self.kind in ("linear", "mixed", "minibatch") else 0
 
     @property
     def token_heads(self):
@@ -64,6 +68,7 @@ WORKLOADS = {
     "mlp1024_bf16": Workload("mlp1024_bf16", 16, 4, 32, 32, "bf16", 0.5, "mlp"),
     "mixed6084_dot_bf16": Workload("mixed6084_dot_bf16", 8, 6, 78, 78, "bf16", 1.0, "mixed", conv_heads=1,
                                    loss="dot"),
+    "mb16_6084_bf16": Workload("mb16_6084_bf16", 8, 6, 78, 78, "bf16", 0.25, "minibatch", mb_tokens=16),
 }
 
 TORCH_DTYPE = {"fp32": torch.float32, "bf16": torch.bfloat16}
@@ -82,7 +87,7 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
     K = _unit_rows(torch.randn(shape, generator=g, dtype=torch.float32))
     V = torch.randn(shape, generator=g, dtype=torch.float32)
     out = {}
-    if w.kind in ("linear", "mixed"):
+    if w.kind in ("linear", "mixed", "minibatch"):
         if w.lin_heads:
             out["W0_lin"] = torch.randn((w.lin_heads, w.d, w.d), generator=g) / math.sqrt(w.d)
         if w.conv_heads:

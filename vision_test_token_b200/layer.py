@@ -93,6 +93,40 @@ def forward_linear(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=
     return Z
 
 
+_MB_MODES = {"prefix": capi.TTT_MB_PREFIX, "epoch": capi.TTT_MB_EPOCH}
+
+
+def _error_word_workspace(device):
+    """The 256-byte zero-filled workspace (an error word) of the calls that need no other scratch."""
+    key = ("error_word", str(device))
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(256, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def forward_linear_minibatch(Q, K, V, W0, eta, H, W, batch_tokens, mode="prefix", Z=None, W1_out=None, ws=None,
+                             stream=None, max_sms=0):
+    """Linear inner model trained by mini-batch gradient descent over consecutive batches of
+    `batch_tokens` tokens.  mode "prefix": causal prefix sums inside a mini-batch, z_t = W_t q_t;
+    mode "epoch": one mean-gradient step per mini-batch, every query read out with the final
+    weights.  W1_out (optional, [B][heads][d][d] fp32) receives the weights after the last batch."""
+    if mode not in _MB_MODES:
+        raise ValueError(f"mode must be one of {sorted(_MB_MODES)}")
+    shape = _shape_of(Q, H, W, max_sms=max_sms)
+    Z = _out_like(Q, Z)
+    _same_layout(Q, K, V, Z)
+    W0 = W0.contiguous()
+    if ws is None:
+        ws = _error_word_workspace(Q.device)
+    st = capi.ttt_forward_linear_minibatch(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape,
+                                           int(batch_tokens), _MB_MODES[mode], *_ws_args(ws), _ptr(W1_out),
+                                           _stream_handle(stream))
+    _check(st, "ttt_forward_linear_minibatch")
+    return Z
+
+
 def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0, loss="l2"):
     """3x3 depthwise-conv inner model.  W0: [heads][d][3][3] fp32 CUDA tensor.  Returns Z."""
     shape = _shape_of(Q, H, W, max_sms=max_sms, loss=loss)
