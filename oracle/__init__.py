@@ -37,10 +37,12 @@ def _load():
         lib.oracle_linear_gram.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_linear_dot.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_linear_minibatch.argtypes = [i, i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_linear_backward.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, dp, dp, dp, dp, i]
         lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv_dot.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
         for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_linear_minibatch,
+                  lib.oracle_linear_backward,
                   lib.oracle_dwconv,
                   lib.oracle_dwconv_dot, lib.oracle_mlp):
             f.restype = ctypes.c_int
@@ -117,6 +119,22 @@ def linear_minibatch(Q, K, V, W0, eta, b, mode, threads=None):
     _check(_load().oracle_linear_minibatch(B, H, N, d, int(b), m, _p(Q), _p(K), _p(V), _p(W0), float(eta),
                                            _p(W1), _p(Z), threads or default_threads()), "linear_minibatch")
     return Z, W1
+
+
+def linear_backward(Q, K, V, W0, eta, dZ, threads=None):
+    """Backward pass of the full-batch linear head (L2 loss) for the upstream gradient dZ.
+    Returns (dQ, dK, dV [B][h][N][d], dW0 [h][d][d] summed over images, deta: a float summed over
+    every unit) in float64."""
+    Q, K, V, W0, dZ = _f64(Q), _f64(K), _f64(V), _f64(W0), _f64(dZ)
+    B, H, N, d = Q.shape
+    assert K.shape == Q.shape and V.shape == Q.shape and dZ.shape == Q.shape and W0.shape == (H, d, d)
+    dQ, dK, dV = np.empty_like(Q), np.empty_like(Q), np.empty_like(Q)
+    dW0 = np.empty((H, d, d))
+    deta = np.zeros(1)
+    _check(_load().oracle_linear_backward(B, H, N, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(dZ), _p(dQ),
+                                          _p(dK), _p(dV), _p(dW0), _p(deta), threads or default_threads()),
+           "linear_backward")
+    return dQ, dK, dV, dW0, float(deta[0])
 
 
 def dwconv(Q, K, V, W0, eta, Hg, Wg, threads=None):

@@ -222,6 +222,112 @@ int oracle_linear_dot(int B, int heads, int N, int d, const double* Q, const dou
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Backward pass of the linear head (press article, Observation 1: the layer is trained end to   */
+/* end through its inner step, the outer gradient flowing through the inner update).  Given the */
+/* upstream gradient dZ of the forward above (L2 loss, full batch), the chain rule through       */
+/*     G = sum k k^T,  C = sum v k^T,  W1 = W0 - s (W0 G - C),  z = W1 q,   s = 2 eta / N        */
+/* gives                                                                                         */
+/*     dW1 = sum dz q^T,   dq = W1^T dz,                                                          */
+/*     dW0 = dW1 (I - s G),   dC = s dW1,   dG = -s W0^T dW1,                                     */
+/*     dv = dC k,   dk = dC^T v + (dG + dG^T) k,   deta = -(2/N) sum_ij dW1_ij (W0 G - C)_ij.     */
+/* W0 and eta are shared by every unit: dW0 is summed over the images of each head and deta over */
+/* every unit, in index order.                                                                   */
+/* ------------------------------------------------------------------------------------------ */
+
+static int linear_backward_unit(int N, int d, const double* Q, const double* K, const double* V,
+                                const double* W0, double eta, const double* dZ, double* dQ, double* dK,
+                                double* dV, double* dW0, double* deta)
+{
+    const size_t dd = (size_t)d * d;
+    double* buf = (double*)calloc(8 * dd, sizeof(double));
+    if (!buf) return ORACLE_ERR_NOMEM;
+    double *G = buf, *C = buf + dd, *dW1 = buf + 2 * dd, *W1 = buf + 3 * dd, *P = buf + 4 * dd;
+    double *dC = buf + 5 * dd, *dG = buf + 6 * dd;
+    const double s = 2.0 * eta / (double)N;
+    for (int n = 0; n < N; ++n) {
+        const double *k = K + (size_t)n * d, *v = V + (size_t)n * d, *q = Q + (size_t)n * d;
+        const double* dz = dZ + (size_t)n * d;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) {
+                G[(size_t)i * d + j] += k[i] * k[j];
+                C[(size_t)i * d + j] += v[i] * k[j];
+                dW1[(size_t)i * d + j] += dz[i] * q[j];
+            }
+    }
+    for (int i = 0; i < d; ++i)                              /* P = W0 G - C,  W1 = W0 - s P */
+        for (int j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (int m = 0; m < d; ++m) acc += W0[(size_t)i * d + m] * G[(size_t)m * d + j];
+            P[(size_t)i * d + j] = acc - C[(size_t)i * d + j];
+            W1[(size_t)i * d + j] = W0[(size_t)i * d + j] - s * P[(size_t)i * d + j];
+        }
+    double de = 0.0;
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) {
+            double acc = 0.0, g = 0.0;
+            for (int m = 0; m < d; ++m) {
+                acc += dW1[(size_t)i * d + m] * G[(size_t)m * d + j];   /* (dW1 G)_ij */
+                g += W0[(size_t)m * d + i] * dW1[(size_t)m * d + j];    /* (W0^T dW1)_ij */
+            }
+            dW0[(size_t)i * d + j] += dW1[(size_t)i * d + j] - s * acc;
+            dC[(size_t)i * d + j] = s * dW1[(size_t)i * d + j];
+            dG[(size_t)i * d + j] = -s * g;
+            de += dW1[(size_t)i * d + j] * P[(size_t)i * d + j];
+        }
+    *deta += -(2.0 / (double)N) * de;
+    for (int n = 0; n < N; ++n) {
+        const double *k = K + (size_t)n * d, *v = V + (size_t)n * d, *dz = dZ + (size_t)n * d;
+        for (int j = 0; j < d; ++j) {
+            double aq = 0.0, ak = 0.0, av = 0.0;
+            for (int i = 0; i < d; ++i) {
+                aq += W1[(size_t)i * d + j] * dz[i];                                   /* W1^T dz */
+                ak += dC[(size_t)i * d + j] * v[i]                                     /* dC^T v */
+                      + (dG[(size_t)j * d + i] + dG[(size_t)i * d + j]) * k[i];         /* (dG + dG^T) k */
+                av += dC[(size_t)j * d + i] * k[i];                                    /* dC k */
+            }
+            dQ[(size_t)n * d + j] = aq;
+            dK[(size_t)n * d + j] = ak;
+            dV[(size_t)n * d + j] = av;
+        }
+    }
+    free(buf);
+    return ORACLE_OK;
+}
+
+/* dW0: [heads][d][d] (summed over images), deta: one value (summed over units).  Units run one at a
+ * time per head in image order so that both sums have a fixed order; heads run in parallel. */
+int oracle_linear_backward(int B, int heads, int N, int d, const double* Q, const double* K, const double* V,
+                           const double* W0, double eta, const double* dZ, double* dQ, double* dK, double* dV,
+                           double* dW0, double* deta, int nthreads)
+{
+    if (B < 0 || heads < 0 || N < 1 || d < 1 || !Q || !K || !V || !W0 || !dZ || !dQ || !dK || !dV || !dW0 ||
+        !deta)
+        return ORACLE_ERR_ARG;
+    double* deta_h = (double*)calloc(heads > 0 ? (size_t)heads : 1, sizeof(double));
+    if (!deta_h) return ORACLE_ERR_NOMEM;
+    memset(dW0, 0, (size_t)heads * d * d * sizeof(double));
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int h = 0; h < heads; ++h) {
+        for (int b = 0; b < B; ++b) {
+            const size_t off = ((size_t)b * heads + h) * N * d;
+            int st = linear_backward_unit(N, d, Q + off, K + off, V + off, W0 + (size_t)h * d * d, eta, dZ + off,
+                                          dQ + off, dK + off, dV + off, dW0 + (size_t)h * d * d, &deta_h[h]);
+            if (st != ORACLE_OK) {
+#pragma omp atomic write
+                status = st;
+            }
+        }
+    }
+    double total = 0.0;
+    for (int h = 0; h < heads; ++h) total += deta_h[h];
+    *deta = total;
+    free(deta_h);
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Linear inner model trained by mini-batch gradient descent over consecutive token batches.    */
 /*   The tokens, in raster order, are cut into consecutive mini-batches of b tokens (the last     */
 /*   may be shorter).  In every mini-batch the per-token gradients are taken at the weights W_s   */

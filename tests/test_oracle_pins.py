@@ -345,6 +345,98 @@ def test_planted_mistakes_fail_the_minibatch_pins(mistake):
 
 
 # ------------------------------------------------------------------------------------------------
+# backward pass of the linear head
+# ------------------------------------------------------------------------------------------------
+def _bwd_case(B=2, H=2, N=9, d=5, seed=0):
+    r = np.random.default_rng(100 + seed)
+    Q, K, V, dZ = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    W0 = r.standard_normal((H, d, d)) / np.sqrt(d)
+    return Q, K, V, W0, dZ
+
+
+def _fwd_loss(Q, K, V, W0, eta, dZ):
+    """L = sum dZ * Z with Z from the pinned forward oracle."""
+    Z, _ = oracle.linear(Q, K, V, W0, eta)
+    return float(np.sum(dZ * Z))
+
+
+def test_linear_backward_matches_central_differences_of_the_forward_oracle():
+    """Every gradient the backward oracle returns equals the central difference of the pinned
+    forward oracle's L = sum dZ * Z, on a few entries of each input and on eta."""
+    Q, K, V, W0, dZ = _bwd_case()
+    eta, h = 0.7, 1e-5
+    dQ, dK, dV, dW0, deta = oracle.linear_backward(Q, K, V, W0, eta, dZ)
+    grads = {"Q": dQ, "K": dK, "V": dV, "W0": dW0}
+    args = {"Q": Q, "K": K, "V": V, "W0": W0}
+    r = np.random.default_rng(5)
+    for name, g in grads.items():
+        for _ in range(6):
+            idx = tuple(int(r.integers(0, n)) for n in args[name].shape)
+            plus = {k: v.copy() for k, v in args.items()}
+            minus = {k: v.copy() for k, v in args.items()}
+            plus[name][idx] += h
+            minus[name][idx] -= h
+            fd = (_fwd_loss(plus["Q"], plus["K"], plus["V"], plus["W0"], eta, dZ) -
+                  _fwd_loss(minus["Q"], minus["K"], minus["V"], minus["W0"], eta, dZ)) / (2 * h)
+            assert abs(g[idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, g[idx], fd)
+    fd = (_fwd_loss(Q, K, V, W0, eta + h, dZ) - _fwd_loss(Q, K, V, W0, eta - h, dZ)) / (2 * h)
+    assert abs(deta - fd) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_linear_backward_matches_torch_autograd():
+    Q, K, V, W0, dZ = _bwd_case(B=2, H=3, N=17, d=8, seed=1)
+    eta = 0.4
+    dQ, dK, dV, dW0, deta = oracle.linear_backward(Q, K, V, W0, eta, dZ)
+    tQ, tK, tV, tW = (torch.tensor(a, requires_grad=True) for a in (Q, K, V, W0))
+    te = torch.tensor(eta, dtype=torch.float64, requires_grad=True)
+    N = Q.shape[2]
+    r = (tK @ tW.transpose(-1, -2)[None]) - tV                       # [B][H][N][d]: W0 k - v
+    grad = 2.0 / N * (r.transpose(-1, -2) @ tK)                      # (2/N) sum (W0 k - v) k^T
+    W1 = tW[None] - te * grad
+    Z = tQ @ W1.transpose(-1, -2)
+    (Z * torch.tensor(dZ)).sum().backward()
+    np.testing.assert_allclose(dQ, tQ.grad.numpy(), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(dK, tK.grad.numpy(), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(dV, tV.grad.numpy(), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(dW0, tW.grad.numpy(), atol=1e-10, rtol=0)
+    assert abs(deta - te.grad.item()) <= 1e-10 * max(1.0, abs(deta))
+
+
+def test_linear_backward_special_cases():
+    """dZ = 0 gives zero gradients; eta = 0 makes the layer z = W0 q, so dQ = W0^T dz, dK = dV = 0
+    and dW0 = sum over images of dZ^T Q."""
+    Q, K, V, W0, dZ = _bwd_case(B=3, H=2, N=11, d=6, seed=2)
+    out = oracle.linear_backward(Q, K, V, W0, 0.9, np.zeros_like(dZ))
+    for a in out[:4]:
+        assert np.all(a == 0.0)
+    assert out[4] == 0.0
+    dQ, dK, dV, dW0, _ = oracle.linear_backward(Q, K, V, W0, 0.0, dZ)
+    np.testing.assert_allclose(dQ, np.einsum("hij,bhni->bhnj", W0, dZ), atol=1e-12, rtol=0)
+    assert np.all(dK == 0.0) and np.all(dV == 0.0)
+    np.testing.assert_allclose(dW0, np.einsum("bhni,bhnj->hij", dZ, Q), atol=1e-12, rtol=0)
+
+
+def test_planted_mistake_fails_the_backward_pin():
+    """Dropping the transposed half of the Gram gradient (dG k instead of (dG + dG^T) k), planted in
+    a CPU copy of the key gradient, disagrees with the central differences."""
+    Q, K, V, W0, dZ = _bwd_case(B=1, H=1, N=7, d=4, seed=3)
+    eta, h = 0.7, 1e-5
+    dQ, dK, dV, _, _ = oracle.linear_backward(Q, K, V, W0, eta, dZ)
+    N = Q.shape[2]
+    s = 2 * eta / N
+    dW1 = dZ[0, 0].T @ Q[0, 0]
+    dG = -s * W0[0].T @ dW1
+    bad = dK[0, 0] - (K[0, 0] @ dG)                      # remove the dG^T k half
+    idx = (0, 0, 3, 2)
+    plus, minus = K.copy(), K.copy()
+    plus[idx] += h
+    minus[idx] -= h
+    fd = (_fwd_loss(Q, plus, V, W0, eta, dZ) - _fwd_loss(Q, minus, V, W0, eta, dZ)) / (2 * h)
+    assert abs(dK[idx] - fd) <= 1e-6 * max(1.0, abs(fd))
+    assert abs(bad[3, 2] - fd) > 1e-4
+
+
+# ------------------------------------------------------------------------------------------------
 # depthwise 3x3 conv head
 # ------------------------------------------------------------------------------------------------
 def test_dwconv_gradient_exact_rational_fd():
