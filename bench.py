@@ -34,6 +34,7 @@ import torch  # noqa: E402
 from vision_test_token_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "TTT-layer fwd tokens*heads/s at 6084 tokens"
+METRIC_BWD = "TTT-layer bwd (linear heads) tokens*heads/s at 6084 tokens"
 UNIT = "token*heads/s"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures summarised under
 # profiles/.  Valid only for the kernel builds those captures were taken on: an entry is removed
@@ -183,6 +184,12 @@ def _np64(t):
 def oracle_units(w, x, units, threads):
     """Runs the oracle on the listed (image, head) units of the workload (inputs already float64)."""
     import oracle
+    if w.kind == "backward":
+        for (b, h) in units:
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            oracle.linear_backward(x["Q"][sl], x["K"][sl], x["V"][sl], x["W0_lin"][h:h + 1], w.eta, x["dZ"][sl],
+                                   threads=threads)
+        return
     if w.kind == "minibatch":
         for (b, h) in units:
             oracle.linear_minibatch(x["Q"][b:b + 1, h:h + 1], x["K"][b:b + 1, h:h + 1], x["V"][b:b + 1, h:h + 1],
@@ -211,7 +218,8 @@ def oracle_units(w, x, units, threads):
 
 
 def oracle_inputs(w, x, images):
-    return {k: _np64(v[:images] if k in ("Q", "K", "V") else v) for k, v in x.items() if k != "Z"}
+    return {k: _np64(v[:images] if k in ("Q", "K", "V", "dZ") else v) for k, v in x.items()
+            if k not in ("Z", "grads")}
 
 
 def time_oracle(w, x, budget_s=12.0):
@@ -265,7 +273,7 @@ def run_reference(args):
               f" of {w.name} per step, {args.steps} steps, {el:.1f} s, fp64")
     cb = {"value": value, "unit": UNIT, "kind": "oracle", "cores": min(threads, w.heads if per_image else 1),
           "sample": sample}
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+    line = {"impl": "reference", "metric": METRIC_BWD if w.kind == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(1, args.steps) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads, "tokens": w.N, "d": w.d,
@@ -290,6 +298,8 @@ def make_step(w, xs, dev):
         elif w.kind == "minibatch":
             layer.forward_linear_minibatch(x["Q"], x["K"], x["V"], weights["W0_lin"], w.eta, w.H, w.W, w.mb_tokens,
                                            w.mb_mode, Z=x["Z"])
+        elif w.kind == "backward":
+            layer.backward_linear(x["Q"], x["K"], x["V"], weights["W0_lin"], w.eta, w.H, w.W, x["dZ"], out=x["grads"])
         else:
             layer.forward_layer(x["Q"], x["K"], x["V"], weights, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=x["Z"],
                                 loss=w.loss)
@@ -356,6 +366,9 @@ def run_ours(args):
     for s in range(args.sets):
         x = make_inputs(w, seed=1000 * first + s, device=dev)
         x["Z"] = torch.empty_like(x["Q"])
+        if w.kind == "backward":
+            x["grads"] = (torch.empty_like(x["Q"]), torch.empty_like(x["Q"]), torch.empty_like(x["Q"]),
+                          torch.empty((w.heads, w.d, w.d), device=dev), torch.empty(1, device=dev))
         xs.append(x)
     stream = torch.cuda.Stream(device=dev)
     step = make_step(w, xs, dev)
@@ -420,6 +433,23 @@ def run_ours(args):
                     conv_name: {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
                                        "achieved_gbs": conv_bytes / t_conv / 1e9,
                                        "frac": conv_bytes / t_conv / 1e9 / pk["hbm_gbs"]}}}
+    elif w.kind == "backward":
+        # plain FP32 FMA kernels: 14 d^2 FLOP per token and head (6 d^2 for G, C, dW1; 8 d^2 for dq, dk,
+        # dv); algorithmic bytes: read Q, K, V, dZ and write dQ, dK, dV once (7 N d elements per unit)
+        n = max(100, args.steps // 4)
+        time_graphs(graphs, 10, stream)
+        t_b = time_graphs(graphs, n, stream) / n
+        flops = w.batch * w.heads * w.N * 14 * w.d * w.d
+        esz = 2 if w.dtype == "bf16" else 4
+        nbytes = 7 * w.batch * w.heads * w.N * w.d * esz
+        mhz = clocks.get("sm_max_mhz") or 1965.0
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        achieved = flops / t_b / 1e12
+        roof = {"bound": "alu", "kernel": "lin_bwd_p1 + lin_bwd_p2 + lin_bwd_sum (the whole ttt_backward_linear call)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {mhz:.0f} MHz",
+                "algorithmic_flops": flops, "algorithmic_bytes": nbytes, "us_per_launch": t_b * 1e6,
+                "hbm_gbs": nbytes / t_b / 1e9, "hbm_frac": nbytes / t_b / 1e9 / pk["hbm_gbs"]}
     elif w.kind == "minibatch":
         # a sequential FP32 recurrence: bound by plain FMA issue, not by HBM.  Algorithmic FLOPs per
         # (token, head) are the mini-batch TTT terms 6 d^2 + 4 b d; the peak is 148 SMs x 128 FP32
@@ -452,7 +482,7 @@ def run_ours(args):
     # end to end through the public API: pinned host inputs -> device -> layer -> host result
     e2e = run_e2e(w, xs[0], dev, stream, args.e2e_steps, world)
 
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    line = {"metric": METRIC_BWD if w.kind == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads,
@@ -467,7 +497,8 @@ def run_ours(args):
                                                                "dependent, the two running at the same time"
                                                                if w.kind == "mixed" else "")},
             "gbs_per_step": workload_bytes(w) / (el_max / args.steps) / 1e9,
-            "gpu_launches": args.steps * (2 if (w.kind == "mixed" or w.dtype == "fp32") else 1),
+            "gpu_launches": args.steps * (3 if w.kind == "backward" else 2 if (w.kind == "mixed" or w.dtype == "fp32")
+                                          else 1),
             "clocks": clocks, "e2e": e2e}
     if roof:
         line["roofline"] = roof
@@ -488,13 +519,15 @@ def run_e2e(w, x, dev, stream, steps, world):
     host-to-device copy of step i+1 overlaps the compute and the device-to-host copy of step i (PCIe
     moves both directions at once).  Every step's copies are inside the timed region."""
     from vision_test_token_b200 import layer
-    names = ["Q", "K", "V"] + sorted(k for k in x if k.startswith("W"))
+    names = ["Q", "K", "V"] + (["dZ"] if w.kind == "backward" else []) + sorted(k for k in x if k.startswith("W"))
     host = {k: x[k].cpu().pin_memory() for k in names}
     dev_in = [{k: torch.empty_like(x[k]) for k in names} for _ in range(2)]
-    z_dev = [torch.empty_like(x["Q"]) for _ in range(2)]
-    z_host = [torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory() for _ in range(2)]
+    n_out = 3 if w.kind == "backward" else 1                 # dQ, dK, dV, or Z
+    z_dev = [[torch.empty_like(x["Q"]) for _ in range(n_out)] for _ in range(2)]
+    z_host = [[torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory() for _ in range(n_out)] for _ in range(2)]
+    small = [(torch.empty((w.heads, w.d, w.d), device=dev), torch.empty(1, device=dev)) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = z_host[0].numel() * z_host[0].element_size()
+    d2h = sum(t.numel() * t.element_size() for t in z_host[0])
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev = lambda: torch.cuda.Event()
     loaded, computed, drained = [ev(), ev()], [ev(), ev()], [ev(), ev()]
@@ -514,17 +547,21 @@ def run_e2e(w, x, dev, stream, steps, world):
             stream.wait_event(drained[bsel])                 # step i-2's Z has left this buffer
         with torch.cuda.stream(stream):
             if w.kind == "mlp":
-                layer.forward_mlp(d["Q"], d["K"], d["V"], d["Wa"], d["Wb"], w.eta, w.H, w.W, Z=z_dev[bsel])
+                layer.forward_mlp(d["Q"], d["K"], d["V"], d["Wa"], d["Wb"], w.eta, w.H, w.W, Z=z_dev[bsel][0])
             elif w.kind == "minibatch":
                 layer.forward_linear_minibatch(d["Q"], d["K"], d["V"], d["W0_lin"], w.eta, w.H, w.W, w.mb_tokens,
-                                               w.mb_mode, Z=z_dev[bsel])
+                                               w.mb_mode, Z=z_dev[bsel][0])
+            elif w.kind == "backward":
+                layer.backward_linear(d["Q"], d["K"], d["V"], d["W0_lin"], w.eta, w.H, w.W, d["dZ"],
+                                      out=(*z_dev[bsel], *small[bsel]))
             else:
                 layer.forward_layer(d["Q"], d["K"], d["V"], d, w.eta, w.H, w.W, conv_heads=w.conv_heads,
-                                    Z=z_dev[bsel], loss=w.loss)
+                                    Z=z_dev[bsel][0], loss=w.loss)
             computed[bsel].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(computed[bsel])
-            z_host[bsel].copy_(z_dev[bsel], non_blocking=True)
+            for zh, zd in zip(z_host[bsel], z_dev[bsel]):
+                zh.copy_(zd, non_blocking=True)
             drained[bsel].record(s_out)
         started[bsel] = True
 

@@ -66,7 +66,12 @@ typedef enum {
 
 typedef enum { TTT_FP32 = 0, TTT_BF16 = 1 } ttt_dtype;
 
-typedef enum { TTT_HEAD_LINEAR = 0, TTT_HEAD_DWCONV = 1, TTT_HEAD_MLP = 2 } ttt_head_kind;
+typedef enum {
+    TTT_HEAD_LINEAR = 0,
+    TTT_HEAD_DWCONV = 1,
+    TTT_HEAD_MLP = 2,
+    TTT_HEAD_LINEAR_BACKWARD = 3   /* the workspace of ttt_backward_linear */
+} ttt_head_kind;
 
 /* Inner loss of the one-step training.
  *   TTT_LOSS_L2:  L(W) = (1/N) sum_n || f(k_n; W) - v_n ||^2  (the formulas of each entry point below).
@@ -188,6 +193,24 @@ typedef enum { TTT_MB_PREFIX = 0, TTT_MB_EPOCH = 1 } ttt_minibatch_mode;
 ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void* V, const float* W0,
                                         void* Z, float eta, const ttt_shape* s, int batch_tokens, int mode,
                                         void* ws, size_t ws_bytes, float* W1_out, void* stream);
+
+/* Backward pass of the full-batch linear head (L2 loss): the outer gradient through the inner update
+ * that trains the layer end to end (press article, Observation 1).  With s = 2 eta / N and the
+ * forward of ttt_forward_linear, for the upstream gradient dZ of Z:
+ *   dW1 = sum dz q^T,  dq = W1^T dz,  dC = s dW1,  dG = -s W0^T dW1,
+ *   dv = dC k,  dk = dC^T v + (dG + dG^T) k,  dW0 = dW1 (I - s G),
+ *   deta = -(2/N) sum_ij dW1_ij (W0 G - C)_ij.
+ *   dZ: same layout and dtype as Q.  dQ, dK, dV: outputs, same layout and dtype as Q; they may not
+ *   overlap Q, K, V, dZ or one another.
+ *   dW0_out: optional [heads][d][d] fp32, summed over the images of each head in image order.
+ *   deta_out: optional, one fp32, summed over every (image, head) unit in index order.
+ *   ws: ttt_workspace_bytes(TTT_HEAD_LINEAR_BACKWARD, s) bytes, zero-filled once
+ *   (ttt_workspace_init); it holds per-unit partial sums and matrices.
+ * Computed in fp32 from bf16 or fp32 inputs (outputs rounded to the input dtype); deterministic.
+ * s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED). */
+ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
+                               float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
+                               void* dV, float* dW0_out, float* deta_out, void* stream);
 
 /* A layer whose heads [0, heads - conv_heads) are linear heads and whose last conv_heads heads are
  * depthwise-conv heads (ViT^3 keeps one conv head among its linear heads: press article,

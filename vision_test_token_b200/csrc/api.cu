@@ -205,6 +205,7 @@ size_t ttt_workspace_bytes(int kind, const ttt_shape* s) {
         case TTT_HEAD_LINEAR: return linear_ws_bytes(*s);
         case TTT_HEAD_DWCONV: return dwconv_ws_bytes(*s);
         case TTT_HEAD_MLP: return mlp_ws_bytes(*s);
+        case TTT_HEAD_LINEAR_BACKWARD: return linear_backward_ws_bytes(*s);
         default: return 0;
     }
 }
@@ -282,6 +283,34 @@ ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void
     if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
     c.W1_out = W1_out;
     return launch_linear_minibatch(c, batch_tokens, mode);
+}
+
+ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
+                               float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
+                               void* dV, float* dW0_out, float* deta_out, void* stream) {
+    ttt_status st = check_shape(TTT_HEAD_LINEAR_BACKWARD, s);
+    if (st != TTT_OK) return st;
+    if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
+    if (!dZ || !dK || !dV) return TTT_ERR_INVALID_ARG;
+    Call c;
+    // Q, K, V, W0, the workspace and dQ (as the output Z: apart from Q, K and V)
+    st = prepare(TTT_HEAD_LINEAR_BACKWARD, Q, K, V, W0, nullptr, dQ, eta, s, ws, ws_bytes, linear_backward_ws_bytes(*s),
+                 stream, &c);
+    if (st != TTT_OK) return st;
+    for (const void* p : {dZ, (const void*)dK, (const void*)dV}) {
+        if (reinterpret_cast<uintptr_t>(p) % 16) return TTT_ERR_ALIGNMENT;
+        if (!is_device_ptr(p)) return TTT_ERR_INVALID_ARG;
+    }
+    const long long ext = extent_bytes(s);
+    const void* ins[] = {Q, K, V, dZ};
+    const void* outs[] = {dQ, dK, dV};
+    for (const void* o : outs)
+        for (const void* in : ins)
+            if (overlaps(o, in, ext)) return TTT_ERR_INVALID_ARG;
+    if (overlaps(dQ, dK, ext) || overlaps(dQ, dV, ext) || overlaps(dK, dV, ext)) return TTT_ERR_INVALID_ARG;
+    if (dW0_out && (reinterpret_cast<uintptr_t>(dW0_out) % 16 || !is_device_ptr(dW0_out))) return TTT_ERR_INVALID_ARG;
+    if (deta_out && (reinterpret_cast<uintptr_t>(deta_out) % 4 || !is_device_ptr(deta_out))) return TTT_ERR_INVALID_ARG;
+    return launch_linear_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
 }
 
 constexpr double kConvHeadWeight = 2.0;
@@ -378,6 +407,6 @@ const char* ttt_status_string(ttt_status st) {
 
 ttt_status ttt_last_error(void) { return g_sticky.load() ? TTT_ERR_CUDA : TTT_OK; }
 
-int ttt_version(void) { return 104; }
+int ttt_version(void) { return 105; }
 
 }  // extern "C"

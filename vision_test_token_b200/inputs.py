@@ -8,8 +8,10 @@ Recipe (one torch CPU generator, ``manual_seed(seed)``, float32 draws in this or
              L2 norm (keys and queries are L2-normalised rows, values stay N(0, 1));
   weights  : linear W0 [heads_lin][d][d] ~ N(0, 1/d); conv W0 [heads_conv][d][3][3] ~ N(0, 1/9);
              MLP Wa [heads][4d][d] ~ N(0, 1/d), Wb [heads][d][4d] ~ N(0, 1/(4d));
-then Q, K, V are rounded once to the compute dtype (bf16: round-to-nearest-even) and weights stay
-float32.  Token n of a unit sits at grid position (n // W, n % W) (raster order of the 16x16
+  dZ       : (kind "backward", the upstream gradient of Z) [B][heads][N][d] standard normal, drawn
+             after the weights;
+then Q, K, V (and dZ) are rounded once to the compute dtype (bf16: round-to-nearest-even) and
+weights stay float32.  Token n of a unit sits at grid position (n // W, n % W) (raster order of the 16x16
 patches of the image).
 
 Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
@@ -23,6 +25,8 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
                    ViT3 recipe: one full-batch step, learning rate 1.0, dot-product loss)
   mb16_6084_bf16   linear, B 8, 6 heads, 78 x 78, bf16, trained by mini-batch gradient descent in
                    consecutive batches of 16 tokens (causal prefix inside a batch), eta 0.25
+  bwd6084_bf16     backward pass of the linear heads of mixed6084_bf16: B 8, 5 heads, 78 x 78,
+                   bf16, eta 0.5
 """
 from dataclasses import dataclass
 import math
@@ -39,7 +43,8 @@ class Workload:
     W: int                # token grid width
     dtype: str            # "fp32" or "bf16"
     eta: float
-    kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp", "minibatch" (linear)
+    kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp", "minibatch" (linear),
+                          # "backward" (linear)
     conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
     d: int = 64
     hidden_ratio: int = 4
@@ -53,7 +58,7 @@ class Workload:
 
     @property
     def lin_heads(self):
-        return self.heads - self.conv_heads if self.kind in ("linear", "mixed", "minibatch") else 0
+        return self.heads - self.conv_heads if self.kind in ("linear", "mixed", "minibatch", "backward") else 0
 
     @property
     def token_heads(self):
@@ -69,6 +74,7 @@ WORKLOADS = {
     "mixed6084_dot_bf16": Workload("mixed6084_dot_bf16", 8, 6, 78, 78, "bf16", 1.0, "mixed", conv_heads=1,
                                    loss="dot"),
     "mb16_6084_bf16": Workload("mb16_6084_bf16", 8, 6, 78, 78, "bf16", 0.25, "minibatch", mb_tokens=16),
+    "bwd6084_bf16": Workload("bwd6084_bf16", 8, 5, 78, 78, "bf16", 0.5, "backward"),
 }
 
 TORCH_DTYPE = {"fp32": torch.float32, "bf16": torch.bfloat16}
@@ -87,7 +93,7 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
     K = _unit_rows(torch.randn(shape, generator=g, dtype=torch.float32))
     V = torch.randn(shape, generator=g, dtype=torch.float32)
     out = {}
-    if w.kind in ("linear", "mixed", "minibatch"):
+    if w.kind in ("linear", "mixed", "minibatch", "backward"):
         if w.lin_heads:
             out["W0_lin"] = torch.randn((w.lin_heads, w.d, w.d), generator=g) / math.sqrt(w.d)
         if w.conv_heads:
@@ -97,6 +103,8 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
         out["Wa"] = torch.randn((w.heads, hid, w.d), generator=g) / math.sqrt(w.d)
         out["Wb"] = torch.randn((w.heads, w.d, hid), generator=g) / math.sqrt(hid)
     dt = TORCH_DTYPE[w.dtype]
+    if w.kind == "backward":
+        out["dZ"] = torch.randn(shape, generator=g, dtype=torch.float32).to(dt)
     out["Q"], out["K"], out["V"] = Q.to(dt), K.to(dt), V.to(dt)
     if device != "cpu":
         out = {k: v.to(device) for k, v in out.items()}
