@@ -14,8 +14,11 @@
 //               [G ; C ; dW1] (192 x 64) and writes it to a partial slot; the CTA that completes a
 //               unit sums the unit's slots in slot order (deterministic) and forms W1, dC, dC^T,
 //               dG + dG^T, the unit's dW0 and deta.
-//   lin_bwd_p2  one CTA per 128-token tile (a programmatic dependent of p1): the four 64 x 64
-//               matrices and the tile's dz, k, v rows in shared memory; dq, dk, dv per token.
+//   lin_bwd_p2  one CTA per 32 tokens (a programmatic dependent of p1): the four 64 x 64 matrices and
+//               the tokens' dz, k, v rows in shared memory; 8 lanes per token compute its dq, dk, dv.
+// The lanes that share a row of outputs take interleaved groups of 4 columns, so that their float4
+// reads of shared memory are contiguous (no bank conflicts), and both kernels keep their shared
+// memory under half an SM's, so that two CTAs share every SM.
 //   lin_bwd_sum dW0 over images and deta over units, in index order.
 #include <algorithm>
 
@@ -28,32 +31,30 @@ namespace bwd {
 constexpr int D = 64;
 constexpr int TOK = 128;                     // tokens per tile
 constexpr int CHUNK = 32;                    // tokens staged in shared memory at a time (p1)
-constexpr int P1_THREADS = 384;              // (row of [G ; C ; dW1], half of its columns)
-constexpr int P2_THREADS = 256;              // (token of the tile, half of the outputs)
+constexpr int P1_THREADS = 384;              // (row of [G ; C ; dW1], one of 2 interleaved column sets)
+constexpr int P2_TOK = 32;                   // tokens per phase-2 CTA
+constexpr int P2_LANES = 8;                  // lanes per token in phase 2
+constexpr int P2_THREADS = P2_TOK * P2_LANES;
 constexpr int kRows = 3 * D;                 // [G ; C ; dW1]
 constexpr int kPartial = kRows * D;          // floats per partial slot
 constexpr int kMats = 4;                     // W1, dC, dC^T, dG + dG^T per unit
-constexpr int kMaxGrid = 160;
+constexpr int kMaxGrid = 320;               // phase-1 CTAs: two per SM
 constexpr int MP = D + 4;                    // padded pitch of the 64 x 64 matrices in shared memory
 constexpr int RP = D + 1;                    // padded pitch of token rows
 
 template <typename E> struct Io;
 template <> struct Io<float> {
     static __device__ __forceinline__ float ld(const float* p) { return __ldg(p); }
-    // 32 consecutive outputs (128-byte aligned)
-    static __device__ __forceinline__ void st32(float* p, const float (&g)[32]) {
-#pragma unroll
-        for (int a = 0; a < 32; a += 4) *reinterpret_cast<float4*>(p + a) = make_float4(g[a], g[a + 1], g[a + 2], g[a + 3]);
+    // 4 consecutive outputs (16-byte aligned)
+    static __device__ __forceinline__ void st4(float* p, float a, float b, float c, float d) {
+        *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
     }
 };
 template <> struct Io<__nv_bfloat16> {
     static __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(p[0]); }
-    // 32 consecutive outputs (64-byte aligned), rounded to bf16
-    static __device__ __forceinline__ void st32(__nv_bfloat16* p, const float (&g)[32]) {
-#pragma unroll
-        for (int a = 0; a < 32; a += 8)
-            *reinterpret_cast<uint4*>(p + a) = make_uint4(pack_bf16x2(g[a], g[a + 1]), pack_bf16x2(g[a + 2], g[a + 3]),
-                                                          pack_bf16x2(g[a + 4], g[a + 5]), pack_bf16x2(g[a + 6], g[a + 7]));
+    // 4 consecutive outputs (8-byte aligned), rounded to bf16
+    static __device__ __forceinline__ void st4(__nv_bfloat16* p, float a, float b, float c, float d) {
+        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
     }
 };
 
@@ -92,11 +93,19 @@ struct Params {
 // ------------------------------------------------------------------------------------------------
 // phase 1: token sums and the per-unit merge
 // ------------------------------------------------------------------------------------------------
-struct P1Smem {
+struct P1Stage {                             // token chunk (the sums)
     float k[CHUNK][D], v[CHUNK][D], q[CHUNK][D], dz[CHUNK][D];
-    float acc[kRows][D];                     // the unit's summed [G ; C ; dW1] (merge)
-    float w0[D][MP];                         // W0 of the head (merge)
-    float p[D][MP];                          // P = W0 G - C (merge)
+};
+struct P1Merge {                             // the merge (the staging tiles are idle by then)
+    float acc[kRows][D];                     // the unit's summed [G ; C ; dW1]
+    float w0[D][MP];                         // W0 of the head
+    float p[D][MP];                          // P = W0 G - C
+};
+struct P1Smem {
+    union {
+        P1Stage st;
+        P1Merge mg;
+    };
     float red[P1_THREADS / 32];
     int last;
 };
@@ -109,20 +118,22 @@ __device__ void merge_unit(const Params& p, P1Smem& s, int u, int slot0, int nsl
     for (int e = tid; e < kPartial; e += P1_THREADS) {
         float a = 0.f;
         for (int j = 0; j < nslots; ++j) a += __ldcg(p.partials + (size_t)(slot0 + j) * kPartial + e);
-        (&s.acc[0][0])[e] = a;
+        (&s.mg.acc[0][0])[e] = a;
     }
-    for (int e = tid; e < D * D; e += P1_THREADS) s.w0[e / D][e % D] = __ldg(p.W0 + (size_t)h * D * D + e);
+    for (int e = tid; e < D * D; e += P1_THREADS) s.mg.w0[e / D][e % D] = __ldg(p.W0 + (size_t)h * D * D + e);
     __syncthreads();
-    const float (*G)[D] = s.acc;             // rows 0..63
-    const float (*C)[D] = s.acc + D;         // rows 64..127
-    const float (*dW1)[D] = s.acc + 2 * D;   // rows 128..191
+    const float (*G)[D] = s.mg.acc;          // rows 0..63
+    const float (*C)[D] = s.mg.acc + D;      // rows 64..127
+    const float (*dW1)[D] = s.mg.acc + 2 * D;   // rows 128..191
+    const float (*w0)[MP] = s.mg.w0;
+    float (*P)[MP] = s.mg.p;
     // P = W0 G - C (a warp's lanes take consecutive j: rows of G are read contiguously)
     for (int e = tid; e < D * D; e += P1_THREADS) {
         const int i = e / D, j = e % D;
         float a = 0.f;
 #pragma unroll 8
-        for (int m = 0; m < D; ++m) a = fmaf(s.w0[i][m], G[m][j], a);
-        s.p[i][j] = a - C[i][j];
+        for (int m = 0; m < D; ++m) a = fmaf(w0[i][m], G[m][j], a);
+        P[i][j] = a - C[i][j];
     }
     __syncthreads();
     float* M = p.mats + (size_t)u * kMats * D * D;
@@ -133,16 +144,16 @@ __device__ void merge_unit(const Params& p, P1Smem& s, int u, int slot0, int nsl
         float dg = 0.f, dgt = 0.f, dwg = 0.f;
 #pragma unroll 8
         for (int m = 0; m < D; ++m) {
-            dg = fmaf(s.w0[m][i], dW1[m][j], dg);    // (W0^T dW1)_ij
-            dgt = fmaf(s.w0[m][j], dW1[m][i], dgt);  // (W0^T dW1)_ji
+            dg = fmaf(w0[m][i], dW1[m][j], dg);      // (W0^T dW1)_ij
+            dgt = fmaf(w0[m][j], dW1[m][i], dgt);    // (W0^T dW1)_ji
             dwg = fmaf(dW1[i][m], G[m][j], dwg);     // (dW1 G)_ij
         }
-        M[0 * D * D + e] = s.w0[i][j] - p.s * s.p[i][j];    // W1
+        M[0 * D * D + e] = w0[i][j] - p.s * P[i][j];        // W1
         M[1 * D * D + e] = p.s * g;                         // dC
         M[2 * D * D + j * D + i] = p.s * g;                 // dC^T
         M[3 * D * D + e] = -p.s * (dg + dgt);               // dG + dG^T
         p.dW0_unit[(size_t)u * D * D + e] = g - p.s * dwg;  // dW0 of this unit
-        part = fmaf(g, s.p[i][j], part);
+        part = fmaf(g, P[i][j], part);
     }
     // deta of the unit: fixed-order block sum
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -165,7 +176,7 @@ lin_bwd_p1(const Params p) {
     const E* Vp = static_cast<const E*>(p.V);
     const E* Qp = static_cast<const E*>(p.Q);
     const E* Zp = static_cast<const E*>(p.dZ);
-    const int r = tid >> 1, j0 = (tid & 1) * 32;       // row of [G ; C ; dW1], first column
+    const int r = tid >> 1, j0 = (tid & 1) * 4;        // row of [G ; C ; dW1]; columns 8 c + j0 .. + 3
     pdl_launch_dependents();
     const long long t_begin = p.part.start(c), t_end = p.part.start(c + 1);
     long long t = t_begin;
@@ -182,30 +193,31 @@ lin_bwd_p1(const Params p) {
                 const int tk = e / D, cc = e % D, n = n0 + tk;
                 const bool in = n < n_end;
                 const size_t o = p.view.row(u, in ? n : 0) + cc;
-                s.k[tk][cc] = in ? Io<E>::ld(Kp + o) : 0.f;
-                s.v[tk][cc] = in ? Io<E>::ld(Vp + o) : 0.f;
-                s.q[tk][cc] = in ? Io<E>::ld(Qp + o) : 0.f;
-                s.dz[tk][cc] = in ? Io<E>::ld(Zp + o) : 0.f;
+                s.st.k[tk][cc] = in ? Io<E>::ld(Kp + o) : 0.f;
+                s.st.v[tk][cc] = in ? Io<E>::ld(Vp + o) : 0.f;
+                s.st.q[tk][cc] = in ? Io<E>::ld(Qp + o) : 0.f;
+                s.st.dz[tk][cc] = in ? Io<E>::ld(Zp + o) : 0.f;
             }
             __syncthreads();
             for (int tk = 0; tk < CHUNK; ++tk) {
-                const float x = (r < D) ? s.k[tk][r] : (r < 2 * D) ? s.v[tk][r - D] : s.dz[tk][r - 2 * D];
-                const float* y = (r < 2 * D) ? s.k[tk] : s.q[tk];
+                const float x = (r < D) ? s.st.k[tk][r] : (r < 2 * D) ? s.st.v[tk][r - D] : s.st.dz[tk][r - 2 * D];
+                const float* y = (r < 2 * D) ? s.st.k[tk] : s.st.q[tk];
 #pragma unroll
-                for (int jj = 0; jj < 32; jj += 4) {
-                    const float4 yv = *reinterpret_cast<const float4*>(y + j0 + jj);
-                    acc[jj + 0] = fmaf(x, yv.x, acc[jj + 0]);
-                    acc[jj + 1] = fmaf(x, yv.y, acc[jj + 1]);
-                    acc[jj + 2] = fmaf(x, yv.z, acc[jj + 2]);
-                    acc[jj + 3] = fmaf(x, yv.w, acc[jj + 3]);
+                for (int cg = 0; cg < 8; ++cg) {
+                    const float4 yv = *reinterpret_cast<const float4*>(y + 8 * cg + j0);
+                    acc[4 * cg + 0] = fmaf(x, yv.x, acc[4 * cg + 0]);
+                    acc[4 * cg + 1] = fmaf(x, yv.y, acc[4 * cg + 1]);
+                    acc[4 * cg + 2] = fmaf(x, yv.z, acc[4 * cg + 2]);
+                    acc[4 * cg + 3] = fmaf(x, yv.w, acc[4 * cg + 3]);
                 }
             }
             __syncthreads();
         }
         float* dst = p.partials + (size_t)(c + u) * kPartial + (size_t)r * D + j0;
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 4)
-            *reinterpret_cast<float4*>(dst + jj) = make_float4(acc[jj], acc[jj + 1], acc[jj + 2], acc[jj + 3]);
+        for (int cg = 0; cg < 8; ++cg)
+            *reinterpret_cast<float4*>(dst + 8 * cg) =
+                make_float4(acc[4 * cg], acc[4 * cg + 1], acc[4 * cg + 2], acc[4 * cg + 3]);
         __threadfence();
         __syncthreads();
         const int cf = p.part.cta_of((long long)u * p.tpu), cl = p.part.cta_of((long long)(u + 1) * p.tpu - 1);
@@ -229,22 +241,22 @@ lin_bwd_p1(const Params p) {
 // phase 2: dq, dk, dv per token
 // ------------------------------------------------------------------------------------------------
 struct P2Smem {
-    float m[kMats][D][MP];                   // W1, dC, dC^T, dG + dG^T
-    float dz[TOK][RP], k[TOK][RP], v[TOK][RP];
+    float m[kMats][D][D];                    // W1, dC, dC^T, dG + dG^T
+    float dz[P2_TOK][RP], k[P2_TOK][RP], v[P2_TOK][RP];
 };
 
 template <typename E>
 __global__ void __launch_bounds__(P2_THREADS)
-lin_bwd_p2(const Params p) {
+lin_bwd_p2(const Params p, int tiles_per_unit) {
     extern __shared__ uint8_t smem_raw[];
     P2Smem& s = *reinterpret_cast<P2Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int tid = threadIdx.x;
     const long long tile = blockIdx.x;
-    const int u = (int)(tile / p.tpu), n0 = (int)(tile % p.tpu) * TOK;
+    const int u = (int)(tile / tiles_per_unit), n0 = (int)(tile % tiles_per_unit) * P2_TOK;
     const E* Kp = static_cast<const E*>(p.K);
     const E* Vp = static_cast<const E*>(p.V);
     const E* Zp = static_cast<const E*>(p.dZ);
-    for (int e = tid; e < TOK * D; e += P2_THREADS) {
+    for (int e = tid; e < P2_TOK * D; e += P2_THREADS) {
         const int tk = e / D, cc = e % D, n = n0 + tk;
         const bool in = n < p.N;
         const size_t o = p.view.row(u, in ? n : 0) + cc;
@@ -253,24 +265,25 @@ lin_bwd_p2(const Params p) {
         s.v[tk][cc] = in ? Io<E>::ld(Vp + o) : 0.f;
     }
     pdl_wait_primary();                      // the unit's matrices come from phase 1
-    const float* M = p.mats + (size_t)u * kMats * D * D;
-    for (int e = tid; e < kMats * D * D; e += P2_THREADS) {
-        const int mi = e / (D * D), rc = e % (D * D);
-        s.m[mi][rc / D][rc % D] = __ldcg(M + e);
-    }
+    const float4* M4 = reinterpret_cast<const float4*>(p.mats + (size_t)u * kMats * D * D);
+    float4* m4 = reinterpret_cast<float4*>(&s.m[0][0][0]);
+    for (int e = tid; e < kMats * D * D / 4; e += P2_THREADS) m4[e] = __ldcg(M4 + e);
     __syncthreads();
-    const int row = tid >> 1, a0 = (tid & 1) * 32;       // token of the tile, first output feature
-    float gq[32], gk[32], gv[32];
+    // token row of the CTA; output columns 32 h + 4 j4 .. + 3 for h = 0, 1
+    const int row = tid / P2_LANES, j4 = (tid % P2_LANES) * 4;
+    float gq[8], gk[8], gv[8];
 #pragma unroll
-    for (int a = 0; a < 32; ++a) { gq[a] = 0.f; gk[a] = 0.f; gv[a] = 0.f; }
+    for (int a = 0; a < 8; ++a) { gq[a] = 0.f; gk[a] = 0.f; gv[a] = 0.f; }
+#pragma unroll 4
     for (int i = 0; i < D; ++i) {
         const float z = s.dz[row][i], kk = s.k[row][i], vv = s.v[row][i];
 #pragma unroll
-        for (int a = 0; a < 32; a += 4) {
-            const float4 w1 = *reinterpret_cast<const float4*>(&s.m[0][i][a0 + a]);    // W1[i][.]
-            const float4 dc = *reinterpret_cast<const float4*>(&s.m[1][i][a0 + a]);    // dC[i][.]
-            const float4 dct = *reinterpret_cast<const float4*>(&s.m[2][i][a0 + a]);   // dC^T[i][.]
-            const float4 dg = *reinterpret_cast<const float4*>(&s.m[3][i][a0 + a]);    // (dG + dG^T)[i][.]
+        for (int h = 0; h < 2; ++h) {
+            const int c = 32 * h + j4, a = 4 * h;
+            const float4 w1 = *reinterpret_cast<const float4*>(&s.m[0][i][c]);    // W1[i][.]
+            const float4 dc = *reinterpret_cast<const float4*>(&s.m[1][i][c]);    // dC[i][.]
+            const float4 dct = *reinterpret_cast<const float4*>(&s.m[2][i][c]);   // dC^T[i][.]
+            const float4 dg = *reinterpret_cast<const float4*>(&s.m[3][i][c]);    // (dG + dG^T)[i][.]
             gq[a] = fmaf(w1.x, z, gq[a]); gq[a + 1] = fmaf(w1.y, z, gq[a + 1]);
             gq[a + 2] = fmaf(w1.z, z, gq[a + 2]); gq[a + 3] = fmaf(w1.w, z, gq[a + 3]);
             gk[a] = fmaf(dc.x, vv, fmaf(dg.x, kk, gk[a]));
@@ -283,10 +296,14 @@ lin_bwd_p2(const Params p) {
     }
     const int n = n0 + row;
     if (n < p.N) {
-        const size_t o = p.view.row(u, n) + a0;
-        Io<E>::st32(static_cast<E*>(p.dQ) + o, gq);
-        Io<E>::st32(static_cast<E*>(p.dK) + o, gk);
-        Io<E>::st32(static_cast<E*>(p.dV) + o, gv);
+        const size_t o = p.view.row(u, n);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = 32 * h + j4, a = 4 * h;
+            Io<E>::st4(static_cast<E*>(p.dQ) + o + c, gq[a], gq[a + 1], gq[a + 2], gq[a + 3]);
+            Io<E>::st4(static_cast<E*>(p.dK) + o + c, gk[a], gk[a + 1], gk[a + 2], gk[a + 3]);
+            Io<E>::st4(static_cast<E*>(p.dV) + o + c, gv[a], gv[a + 1], gv[a + 2], gv[a + 3]);
+        }
     }
 }
 
@@ -342,7 +359,7 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
     p.tpu = tpu;
     p.units = (int)units;
     const long long T = units * tpu;
-    const int G = (int)std::max<long long>(1, std::min<long long>(std::min(c.num_sms, kMaxGrid), T));
+    const int G = (int)std::max<long long>(1, std::min<long long>(std::min(2 * c.num_sms, kMaxGrid), T));
     p.part = Partition{T, G};
     p.s = c.eta * (2.0f / (float)c.N);
     p.eta_grad_scale = -2.0f / (float)c.N;
@@ -364,14 +381,15 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    const int tiles2 = (c.N + P2_TOK - 1) / P2_TOK;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)T);
+    cfg.gridDim = dim3((unsigned)(units * tiles2));
     cfg.blockDim = dim3(P2_THREADS);
     cfg.dynamicSmemBytes = sm2;
     cfg.stream = c.stream;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2<E>, p));
+    st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2<E>, p, tiles2));
     if (st != TTT_OK || (!dW0_out && !deta_out)) return st;
     lin_bwd_sum<<<c.heads, 256, 0, c.stream>>>(p, c.batch);
     return check_launch(cudaGetLastError());
