@@ -39,7 +39,7 @@ UNIT = "token*heads/s"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures summarised under
 # profiles/.  Valid only for the kernel builds those captures were taken on: an entry is removed
 # whenever its kernel changes.  Mixed layer: the two kernels of one step, summed.
-STEP_TRAFFIC = {"mixed6084_bf16": (93.596416e6 + 3.737088e6) + (18.751488e6 + 0.0064e6),    # profiles/*_mixed6084.md
+STEP_TRAFFIC = {"mixed6084_bf16": (93.597184e6 + 3.062272e6) + (18.751488e6 + 0.0),   # profiles/traffic_mixed6084_bf16.md
                 "mixed6084_dot_bf16": (93.595904e6 + 4.063488e6) + (18.747392e6 + 0.002816e6)}
                 # profiles/layer_kernels_mixed6084_dot_bf16.md
 MLP_TRAFFIC = {"mlp1024_bf16": 25.809664e6 + 0.0}                                   # profiles/mlp_fused_mlp1024.md
