@@ -56,3 +56,28 @@ def test_oracle_regression_record():
     np.testing.assert_allclose(Z[0, 0, 0], g["mlp"]["Z_row0"], rtol=1e-13, atol=1e-15)
     assert abs(Wa1.sum() - g["mlp"]["Wa1_sum"]) < 1e-11
     assert abs(Wb1.sum() - g["mlp"]["Wb1_sum"]) < 1e-11
+
+
+def test_oracle_regression_record_of_the_variants():
+    """The dot-loss, mini-batch and backward oracles reproduce their recorded values."""
+    g = _load("oracle_regression.json")
+    _, x = random_unit(1, 1, 3, 4, d=8, dtype="fp32", seed=g["linear_dot"]["seed"])
+    Z, W1 = oracle.linear_dot(x["Q"], x["K"], x["V"], x["W0_lin"], g["linear_dot"]["eta"])
+    np.testing.assert_allclose(Z[0, 0, 0], g["linear_dot"]["Z_row0"], rtol=1e-13, atol=1e-15)
+    assert abs(W1.sum() - g["linear_dot"]["W1_sum"]) < 1e-12
+    _, x = random_unit(1, 1, 3, 4, d=8, dtype="fp32", seed=g["dwconv_dot"]["seed"], kind="mixed", conv_heads=1)
+    Z, W1 = oracle.dwconv_dot(x["Q"], x["K"], x["V"], x["W0_conv"], g["dwconv_dot"]["eta"], 3, 4)
+    np.testing.assert_allclose(Z[0, 0, 0], g["dwconv_dot"]["Z_row0"], rtol=1e-13, atol=1e-15)
+    assert abs(W1.sum() - g["dwconv_dot"]["W1_sum"]) < 1e-12
+    for mode in ("prefix", "epoch"):
+        rec = g["linear_minibatch_" + mode]
+        _, x = random_unit(1, 1, 3, 4, d=8, dtype="fp32", seed=rec["seed"])
+        Z, W1 = oracle.linear_minibatch(x["Q"], x["K"], x["V"], x["W0_lin"], rec["eta"], rec["b"], mode)
+        np.testing.assert_allclose(Z[0, 0, 0], rec["Z_row0"], rtol=1e-13, atol=1e-15)
+        assert abs(W1.sum() - rec["W1_sum"]) < 1e-12
+    rec = g["linear_backward"]
+    _, x = random_unit(2, 1, 3, 4, d=8, dtype="fp32", seed=rec["seed"], kind="backward")
+    dQ, dK, dV, dW0, deta = oracle.linear_backward(x["Q"], x["K"], x["V"], x["W0_lin"], rec["eta"], x["dZ"])
+    for name, a in (("dQ_row0", dQ), ("dK_row0", dK), ("dV_row0", dV)):
+        np.testing.assert_allclose(a[0, 0, 0], rec[name], rtol=1e-13, atol=1e-15)
+    assert abs(dW0.sum() - rec["dW0_sum"]) < 1e-12 and abs(deta - rec["deta"]) < 1e-12 * max(1.0, abs(deta))
