@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for the ViT^3 test-time-training layer forward -- TEST INFRASTRUCTURE ONLY.
+"""fp64 CPU oracle for the ViT^3 test-time-training layer -- TEST INFRASTRUCTURE ONLY.
 
 Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline / reference leg of
 ``bench.py`` may import this package.  The CUDA product path never does, and it shares no code
@@ -10,6 +10,13 @@ Functions and the definitions they follow (page titles and sections; see ``ttt_o
   linear_gram(...)  the same step written as W0 - eta (2/N) (W0 K K^T - V K^T)
   dwconv(...)       the same loss with a 3x3 depthwise cross-correlation inner model
   mlp(...)          the same loss with f(x) = Wb gelu_tanh(Wa x)
+  linear_dot(...), dwconv_dot(...)
+                    the linear and conv heads under the dot-product inner loss -(1/N) sum <f(k), v>
+  linear_minibatch(...)
+                    the linear head trained by mini-batch gradient descent over consecutive token
+                    batches (prefix: causal prefix sums inside a batch; epoch: one mean step per batch)
+  linear_backward(...)
+                    the chain rule through the full-batch linear step: dQ, dK, dV, dW0, deta
   gelu_tanh(u), gelu_tanh_deriv(u)
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py (closed forms,

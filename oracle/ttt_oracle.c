@@ -1,5 +1,6 @@
 /*
- * ttt_oracle.c -- plain fp64 CPU oracle for the ViT^3 test-time-training (TTT) layer forward.
+ * ttt_oracle.c -- plain fp64 CPU oracle for the ViT^3 test-time-training (TTT) layer: its forward
+ * pass, the variants of its inner training, and the backward pass of its linear head.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load this file or the
  * library built from it.  Only the test suite, the package smoke check and the CPU-baseline leg of
@@ -30,6 +31,12 @@
  *     - the dot-product inner loss of the ViT3 recipe (press article, section on the ViT3 model;
  *       the loss itself is not printed) is the negative mean inner product of prediction and value,
  *       L(W) = -(1/N) sum_n <f(k_n; W), v_n>.
+ *     - the mini-batch variants take every in-batch gradient at the weights the mini-batch starts
+ *       from; inside a batch the notes' prefix sum carries no 1/b, while the press article's
+ *       B = N/k ablation takes one step of each batch's mean loss and reads out with the final
+ *       weights;
+ *     - the backward pass differentiates the full-batch linear step; W0 and eta are shared by
+ *       every unit, so their gradients are summed (over images, over units).
  *
  * Memory layout of every array (contiguous, row-major, fp64):
  *   Q, K, V, Z : [B][heads][N][d]     (token n, feature c at ((b*heads + h)*N + n)*d + c)
