@@ -154,3 +154,22 @@ def test_minibatch_rejects_bad_arguments(lib):
                                              None, None) == capi.TTT_ERR_INVALID_ARG
     assert capi.ttt_forward_linear_minibatch(fake, fake, fake, fake, ctypes.c_void_p(1 << 40), 0.5, s, 16,
                                              capi.TTT_MB_PREFIX, None, 0, None, None) == capi.TTT_ERR_WORKSPACE
+
+
+def test_backward_workspace_and_validation(lib):
+    s = _shape()
+    n = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR_BACKWARD, s)
+    units = 8 * 5
+    # counters, then partial slots for up to 320 CTAs + one per unit ([G ; C ; dW1] = 192 x 64 fp32),
+    # the unit matrices (4 x 64 x 64), each unit's dW0 and deta
+    assert n > (320 + units) * 192 * 64 * 4 + units * 5 * 64 * 64 * 4
+    assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR_BACKWARD, _shape(batch=0)) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    far = ctypes.c_void_p(1 << 40)
+    call = lambda shape, dZ=fake, ws=fake, nbytes=1 << 30: capi.ttt_backward_linear(
+        fake, fake, fake, fake, dZ, 0.5, shape, ws, nbytes, far, far, far, None, None, None)
+    assert call(_shape(loss=capi.TTT_LOSS_DOT)) == capi.TTT_ERR_UNSUPPORTED     # L2 only
+    assert call(s, dZ=None) == capi.TTT_ERR_INVALID_ARG
+    assert call(s, ws=None, nbytes=0) == capi.TTT_ERR_WORKSPACE
+    assert call(s, nbytes=n - 1) == capi.TTT_ERR_WORKSPACE
+    assert call(_shape(d=32)) == capi.TTT_ERR_UNSUPPORTED
