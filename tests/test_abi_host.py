@@ -173,3 +173,20 @@ def test_backward_workspace_and_validation(lib):
     assert call(s, ws=None, nbytes=0) == capi.TTT_ERR_WORKSPACE
     assert call(s, nbytes=n - 1) == capi.TTT_ERR_WORKSPACE
     assert call(_shape(d=32)) == capi.TTT_ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/ttt.h is a C header: a C99 translation unit that includes it and takes the address of
+    every declared function compiles with gcc in pedantic mode."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    names = _declared_functions()
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "ttt.h"\n' + "".join(f"void (*p_{n})(void) = (void (*)(void)){n};\n" for n in names) +
+                   "int main(void) { ttt_shape s = {0}; (void)s; return 0; }\n")
+    r = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Werror", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
