@@ -419,7 +419,7 @@ def run_ours(args):
         t_lin, t_conv = time_calls_alone(w, xs, stream, n=max(200, args.steps // 4))
         step_s = el_max / args.steps
         achieved = workload_bytes(w) / step_s / 1e9
-        conv_name = "dw_queue<bf16, dot>" if w.loss == "dot" else "dw_queue<bf16>"
+        conv_name = "dw_band<bf16, dot>" if w.loss == "dot" else "dw_band<bf16>"
         roof = {"bound": "hbm",
                 "kernel": f"layer step: lin_cluster_bf16 and {conv_name} running at the same time "
                           "(one ttt_forward_layer call)",

@@ -156,21 +156,30 @@ ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const fl
  * inside a host framework that hands it only its input and output buffers and owns the allocator,
  * or code that runs under a fixed, pre-reserved memory budget and must not call cudaMalloc at run
  * time (cudaMalloc may synchronise the device and has no bounded latency).
- *   Same arguments, computation, results and errors as ttt_forward_linear, minus (ws, ws_bytes).
+ *   Same arguments, computation, results and validation errors as ttt_forward_linear, minus
+ *   (ws, ws_bytes).
  *   Scratch: an 8 MiB array that the library holds on every device that loads it, until the process
  *   exits.  Shapes whose ttt_workspace_bytes(TTT_HEAD_LINEAR, s) exceeds 8 MiB are rejected with
  *   TTT_ERR_WORKSPACE (bf16 calls need only the 256-byte error word; fp32 calls need about
  *   5 MiB + 48 KiB per (image, head) unit, so fp32 calls above about 60 units are rejected).
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
- *   device current; make that first call before any stream capture begins.
+ *   device current, and looks it up again when the device's context has changed (after a
+ *   cudaDeviceReset); make that first call before any stream capture begins.
  *   Every call on a device shares that device's one array, which keeps the previous call's contents;
- *   each call clears the words that must start at zero (a cudaMemsetAsync on `stream`) before its
- *   kernels run.  Calls whose work may overlap on the same GPU (other streams, other host threads)
- *   race on the array and must be serialised by the caller.
+ *   each call clears the control words that must start at zero (a cudaMemsetAsync on `stream`)
+ *   before its kernels run, and keeps the error word.  Calls whose work may overlap on the same GPU
+ *   (other streams, other host threads) race on the array and must be serialised by the caller.
+ *   A device-side wait that runs out is reported by ttt_noalloc_status (below), not by the call.
  *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  */
 ttt_status ttt_forward_linear_noalloc(const void* Q, const void* K, const void* V, const float* W0, void* Z,
                                       float eta, const ttt_shape* s, float* W1_out, void* stream);
+
+/* The error word of the current device's ttt_forward_linear_noalloc scratch (no counterpart on the
+ * pages either): synchronises `stream`, then reports TTT_ERR_TIMEOUT (and clears it) if a kernel of
+ * an earlier noalloc call on this device gave up a bounded device-side wait -- its Z and W1_out are
+ * then incomplete -- else TTT_OK.  Allocates nothing. */
+ttt_status ttt_noalloc_status(void* stream);
 
 /* Mini-batch variants of the linear head's inner training (mode: ttt_minibatch_mode).
  * The raster-ordered tokens are cut into consecutive mini-batches of batch_tokens tokens (the last
@@ -240,6 +249,13 @@ ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const 
  * zero-filled (ttt_workspace_init); it must not be in use by another call.
  * Errors: TTT_ERR_WORKSPACE (ws NULL or too small), TTT_ERR_ALIGNMENT, TTT_ERR_INVALID_ARG. */
 ttt_status ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned long long limit_ns, void* stream);
+
+/* Bound, in nanoseconds (1 .. 1e9; 1e9 at load), of every device-side wait of the kernels launched
+ * by later calls in this process (a wait on a tile, on a partner warp or on another CTA's result).
+ * A wait that runs out records TTT_ERR_TIMEOUT in the call's workspace error word and the kernel
+ * returns; no fault is involved.  Shortening it is meant for tests of that failure path.  Returns
+ * TTT_ERR_INVALID_ARG outside the range. */
+ttt_status ttt_set_wait_limit(unsigned long long limit_ns);
 
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(ttt_status st);

@@ -52,7 +52,7 @@ def test_workspace_sizes(lib):
     nf = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(dtype=capi.TTT_FP32, batch_stride=6 * 6084 * 64))
     assert 40 * 64 * 64 * 4 < nf < 16 << 20           # fp32: counters, W1 and partial slots
     nc = capi.ttt_workspace_bytes(capi.TTT_HEAD_DWCONV, s)
-    # conv: header, control words (queue, done, 40 unit counters, 40 ready flags) padded to 256 B,
+    # conv: header, control words (done, 40 unit counters, 40 ready flags) padded to 256 B,
     # then per unit room for one task per row pair (39) x 3 compute groups of 576-float partials,
     # then W1 per unit
     assert nc == 256 + 512 + 40 * 39 * 3 * 576 * 4 + 40 * 576 * 4

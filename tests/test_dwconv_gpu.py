@@ -67,8 +67,9 @@ def test_dwconv_eta_zero_matches_torch_conv2d(cuda_dev):
 @pytest.mark.parametrize("max_sms", [1, 2, 3, 24, 25, 0])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_dwconv_sm_budget(cuda_dev, max_sms, dtype):
-    """Any SM budget (cluster sizes 1..8, units looping over fewer clusters) gives the same result
-    within tolerance."""
+    """Any SM budget gives the same result within tolerance: one CTA looping over every (unit, band)
+    task, a few CTAs each taking several tasks (their gradients first, then their readouts), bands
+    of one row pair, and the whole device."""
     _check(_conv_inputs(8, 1, 78, 78, dtype, seed=17), 0.5, 78, 78, cuda_dev, dtype, max_sms)
 
 

@@ -17,9 +17,9 @@ TTT_MB_PREFIX, TTT_MB_EPOCH = 0, 1
 # Every symbol that include/ttt.h declares.
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_workspace_init", "ttt_workspace_status",
-    "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp", "ttt_forward_linear_noalloc",
+    "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_mlp", "ttt_forward_linear_noalloc", "ttt_noalloc_status",
     "ttt_forward_linear_minibatch", "ttt_backward_linear",
-    "ttt_layer_workspace_bytes", "ttt_forward_layer", "ttt_selftest_wait_timeout",
+    "ttt_layer_workspace_bytes", "ttt_forward_layer", "ttt_selftest_wait_timeout", "ttt_set_wait_limit",
     "ttt_status_string", "ttt_last_error", "ttt_version",
 )
 
@@ -60,6 +60,8 @@ def lib():
         L.ttt_forward_linear.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
         L.ttt_forward_linear.restype = i
         L.ttt_forward_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, vp]
+        L.ttt_noalloc_status.argtypes = [vp]
+        L.ttt_noalloc_status.restype = i
         L.ttt_forward_linear_noalloc.restype = i
         L.ttt_forward_linear_minibatch.argtypes = [vp, vp, vp, vp, vp, f, shp, i, i, vp, sz, vp, vp]
         L.ttt_forward_linear_minibatch.restype = i
@@ -75,6 +77,8 @@ def lib():
         L.ttt_forward_layer.restype = i
         L.ttt_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_ulonglong, vp]
         L.ttt_selftest_wait_timeout.restype = i
+        L.ttt_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+        L.ttt_set_wait_limit.restype = i
         L.ttt_status_string.argtypes = [i]
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_last_error.argtypes = []
@@ -115,6 +119,10 @@ def ttt_forward_linear_noalloc(Q, K, V, W0, Z, eta, shape, W1_out, stream):
     return lib().ttt_forward_linear_noalloc(Q, K, V, W0, Z, eta, ctypes.byref(shape), W1_out, stream)
 
 
+def ttt_noalloc_status(stream):
+    return lib().ttt_noalloc_status(stream)
+
+
 def ttt_forward_linear_minibatch(Q, K, V, W0, Z, eta, shape, batch_tokens, mode, ws, ws_bytes, W1_out, stream):
     return lib().ttt_forward_linear_minibatch(Q, K, V, W0, Z, eta, ctypes.byref(shape), batch_tokens, mode, ws,
                                               ws_bytes, W1_out, stream)
@@ -146,6 +154,10 @@ def ttt_forward_layer(Q, K, V, W0_lin, W0_conv, Z, eta, shape, conv_heads, ws, w
 
 def ttt_selftest_wait_timeout(ws, ws_bytes, limit_ns, stream):
     return lib().ttt_selftest_wait_timeout(ws, ws_bytes, limit_ns, stream)
+
+
+def ttt_set_wait_limit(limit_ns):
+    return lib().ttt_set_wait_limit(limit_ns)
 
 
 def ttt_last_error():

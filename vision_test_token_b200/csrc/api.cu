@@ -11,6 +11,9 @@
 namespace ttt {
 
 static std::atomic<int> g_sticky{0};   // first asynchronous CUDA error seen (as cudaError_t)
+static std::atomic<unsigned long long> g_wait_ns{1000000000ull};   // bound of each device-side wait
+
+unsigned long long wait_limit_ns() { return g_wait_ns.load(); }
 
 ttt_status check_launch(cudaError_t e) {
     if (e == cudaSuccess) return TTT_OK;
@@ -181,6 +184,7 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
     c->overlap_previous = 0;
     c->err_ws = nullptr;
     c->grid_out = nullptr;
+    c->wait_ns = wait_limit_ns();
     return TTT_OK;
 }
 
@@ -188,6 +192,32 @@ ttt_status validate_call(int kind, const void* Q, const void* K, const void* V, 
                          void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, size_t need, void* stream) {
     Call c;
     return prepare(kind, Q, K, V, W0, W0b, Z, eta, s, ws, ws_bytes, need, stream, &c);
+}
+
+ttt_status prepare_linear(const void* Q, const void* K, const void* V, const float* W0, void* Z, float eta,
+                          const ttt_shape* s, void* ws, size_t ws_bytes, float* W1_out, void* stream, Call* c) {
+    const size_t need = (check_shape(TTT_HEAD_LINEAR, s) == TTT_OK) ? linear_ws_bytes(*s) : 0;
+    ttt_status st = prepare(TTT_HEAD_LINEAR, Q, K, V, W0, nullptr, Z, eta, s, ws, ws_bytes, need, stream, c);
+    if (st != TTT_OK) return st;
+    if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
+    c->W1_out = W1_out;
+    return TTT_OK;
+}
+
+ttt_status read_error_word(void* ws, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return check_launch(e);
+    if (word & kErrTimeout) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyAsync(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return check_launch(e);
+        return TTT_ERR_TIMEOUT;
+    }
+    return TTT_OK;
 }
 
 }  // namespace ttt
@@ -219,29 +249,14 @@ ttt_status ttt_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 ttt_status ttt_workspace_status(void* ws, void* stream) {
     if (!ws) return TTT_ERR_WORKSPACE;
     if (!is_device_ptr(ws)) return TTT_ERR_INVALID_ARG;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint32_t word = 0;
-    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) return check_launch(e);
-    if (word & kErrTimeout) {
-        const uint32_t zero = 0;
-        e = cudaMemcpyAsync(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-        if (e != cudaSuccess) return check_launch(e);
-        return TTT_ERR_TIMEOUT;
-    }
-    return TTT_OK;
+    return read_error_word(ws, stream);
 }
 
 ttt_status ttt_forward_linear(const void* Q, const void* K, const void* V, const float* W0, void* Z, float eta,
                               const ttt_shape* s, void* ws, size_t ws_bytes, float* W1_out, void* stream) {
     Call c;
-    const size_t need = (check_shape(TTT_HEAD_LINEAR, s) == TTT_OK) ? linear_ws_bytes(*s) : 0;
-    ttt_status st = prepare(TTT_HEAD_LINEAR, Q, K, V, W0, nullptr, Z, eta, s, ws, ws_bytes, need, stream, &c);
+    const ttt_status st = prepare_linear(Q, K, V, W0, Z, eta, s, ws, ws_bytes, W1_out, stream, &c);
     if (st != TTT_OK) return st;
-    if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
-    c.W1_out = W1_out;
     return launch_linear(c);
 }
 
@@ -384,9 +399,9 @@ ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const 
     int lin_grid = 0;
     cl.grid_out = &lin_grid;
     if (lin.heads && (st = launch_linear(cl)) != TTT_OK) return st;
-    // The conv kernel is sized for the SMs the linear kernel leaves free (its tasks are split so that
-    // each of those CTAs runs about one gradient task); with none left, it waits for the linear
-    // kernel's SMs and takes them all.
+    // The conv kernel is queued behind the linear kernel as a programmatic dependent and sized for
+    // the SMs the linear grid leaves free; with none left, it takes the whole device and its CTAs
+    // start as the linear CTAs finish.
     if (conv.heads && lin.heads && lin_grid > 0 && lin_grid < whole.num_sms) cc.num_sms = whole.num_sms - lin_grid;
     if (conv.heads) st = launch_dwconv(cc);
     return st;
@@ -407,6 +422,12 @@ const char* ttt_status_string(ttt_status st) {
 
 ttt_status ttt_last_error(void) { return g_sticky.load() ? TTT_ERR_CUDA : TTT_OK; }
 
-int ttt_version(void) { return 105; }
+ttt_status ttt_set_wait_limit(unsigned long long limit_ns) {
+    if (limit_ns == 0 || limit_ns > 1000000000ull) return TTT_ERR_INVALID_ARG;
+    g_wait_ns.store(limit_ns);
+    return TTT_OK;
+}
+
+int ttt_version(void) { return 200; }
 
 }  // extern "C"

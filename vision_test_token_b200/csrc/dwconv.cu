@@ -8,32 +8,30 @@
 // L = -(1/N) sum <f(K;W), V>, the gradient has no residual: g[c][a][b] = -(1/N) sum V K[shifted]
 // (the kernel's DOT instantiation, half the phase-1 FMAs).
 //
-// Not a contraction worth a tensor core (about 7 flop per byte): fp32 FMA in registers.
+// Not a contraction worth a tensor core (about 7 flop per byte, and no sharing across channels): fp32
+// FMA in registers.
 //
-// One kernel (dw_queue) of independent CTAs -- no clusters, so it fits whatever SMs are free, e.g.
-// next to the linear-head kernel of the same layer.  A unit's grid is cut into tasks of a few
-// row pairs of one strip of at most XT columns (about one gradient task per CTA).  A CTA's producer lane claims tasks from a
-// global counter: first every gradient task (phase 1) of every unit, then every readout task
-// (phase 2).
-//   Streaming: the producer loads a task's rows as 2-row groups into two shared-memory rings: K (in
-//     phase 2: Q) groups with a one-column halo on both sides, and V groups.  Output row pair j of
-//     the task reads K groups j (rows 2j-1, 2j) and j+1 (rows 2j+1, 2j+2) and V group j.  The tensor
-//     map's out-of-bounds zero fill supplies the zero padding, so the inner loops carry no bounds
-//     checks.
+// One kernel (dw_band) of independent CTAs -- no clusters, so it fits whatever SMs are free, e.g. next
+// to the linear-head kernel of the same layer.  A unit's grid is cut into tasks: a band of row pairs
+// of one strip of at most XT columns; a launch makes about one task per CTA.  CTA c takes tasks c,
+// c + grid, ...: first the gradient (phase 1) of each of its tasks, then the readout (phase 2) of
+// each, so a CTA only waits for other CTAs after all of its own phase-1 work is done.
+//   Streaming: the producer lane loads the task's rows as 2-row groups into two shared-memory rings:
+//     K groups with a one-column halo on both sides, and V groups; then, without waiting for W1, the
+//     Q groups of the readout into the K ring (so Q streams in while the unit's gradients are merged).
+//     Output row pair j reads K groups j (rows 2j-1, 2j) and j+1 (rows 2j+1, 2j+2) and V group j.  The
+//     tensor map's out-of-bounds zero fill supplies the zero padding, so the inner loops carry no
+//     bounds checks.
 //   Compute: three groups of 5 warps; group g takes the row pairs j = g (mod 3) of every task.  In a
 //     group, warp w owns a column segment of both rows of a pair, lane l owns channels 2l and 2l+1,
 //     and a 4 x 3 register window slides along the columns (unrolled by 3, so the window never moves
-//     between registers).  The residual is carried negated (s = V - W0 (*) K, from the negated taps),
-//     which saves a negation per token.
+//     between registers), fed by explicit shared-memory loads.  The residual is carried negated
+//     (s = V - W0 (*) K, from the negated taps), which saves a negation per token.
 //   Merge: each group folds its warps' 64 x 9 sums in a fixed order into its partial for the task,
-//     written to the workspace slot of (unit, task, group); the groups never wait for one another.
-//     The group that writes a unit's last partial sums all of the unit's partials in slot order -- a
-//     fixed order, so W1 is bitwise reproducible whichever CTA ran which task (for a given grid) --
-//     writes W1 and appends the unit to the merge order.
-//   Readout tasks follow the merge order: readout task slot i serves the i-th unit to finish its
-//     gradients, so no CTA waits for one late unit while another is ready.  The wait for slot i
-//     cannot deadlock: tasks are claimed in order, so every gradient task was claimed earlier by a
-//     CTA that is running it.  Z is written
+//     written to the workspace slot of (unit, task, group).  The group that writes a unit's last
+//     partial sums all of the unit's partials in slot order -- a fixed order, so W1 is bitwise
+//     reproducible whichever CTA ran which task (for a given grid) -- writes W1 and raises the unit's
+//     ready flag; the readout of the unit's tasks waits for that flag (bounded).  Z is written
 //     straight from registers (128 coalesced bytes per token and warp).
 //   The last CTA to finish returns the workspace's counters and flags to zero for the next call.
 //   When launched as a programmatic dependent of the preceding kernel (the linear heads of the same
@@ -55,30 +53,29 @@ constexpr int CW = GW * CG;                 // compute warps
 constexpr int THREADS = (CW + 1) * 32;      // + one producer warp (16 warps: 128 registers a thread)
 constexpr int NK = 6;                       // K / Q ring slots (2-row groups)
 constexpr int NV = 4;                       // V ring slots (2-row groups)
-constexpr int NT = 4;                       // claimed tasks in flight (producer ahead of the compute warps)
 constexpr int kPart = D * TAPS;             // 576 floats: a 64 x 9 gradient or kernel, tap-major
 constexpr int kRed = (GW + 1) / 2;          // a group's per-warp gradients are folded pairwise into kRed slots
-constexpr uint32_t kExitBar = 1 + CG;       // named barrier of all compute warps (ids 1..CG: the groups)
-constexpr int kTasksPerCta = 1;             // gradient tasks per CTA a launch aims for
+constexpr int kTasksPerCta = 1;             // tasks a launch aims for per CTA
 
 template <typename T>
 struct Elem;
 template <>
 struct Elem<__nv_bfloat16> {                 // two bf16 channels in one 32-bit word
-    using Raw = uint32_t;
     static constexpr int kTokenBytes = D * 2;
     static constexpr int kXtMax = 80;
-    static __device__ __forceinline__ float2 unpack(Raw w) { return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w)); }
+    static __device__ __forceinline__ float2 lds(uint32_t addr) {
+        const uint32_t w = lds_u32(addr);
+        return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+    }
     static __device__ __forceinline__ void store(__nv_bfloat16* p, float2 v) {
         *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(v.x, v.y);
     }
 };
 template <>
 struct Elem<float> {
-    using Raw = float2;
     static constexpr int kTokenBytes = D * 4;
     static constexpr int kXtMax = 38;
-    static __device__ __forceinline__ float2 unpack(Raw w) { return w; }
+    static __device__ __forceinline__ float2 lds(uint32_t addr) { return lds_f2(addr); }
     static __device__ __forceinline__ void store(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
 };
 
@@ -86,7 +83,7 @@ struct Geom {
     int heads, H, W;
     int Sx, XT;                      // strips, strip width
     int Hp;                          // row pairs per strip: ceil(H / 2)
-    int tps, tpu;                    // tasks per strip (each a contiguous range of row pairs), per unit
+    int tps, tpu;                    // tasks per strip (each a contiguous band of row pairs), per unit
     long long bs, hs;                // element strides of Q/K/V/Z
     int k_pitch;                     // tokens per staged K/Q row (XT + 2)
     uint32_t kg_bytes, vg_bytes;     // one staged K/Q group (2 x k_pitch tokens), one V group (2 x XT)
@@ -95,30 +92,29 @@ struct Geom {
 struct Params {
     Geom g;
     int U;                           // units
-    int T1, T;                       // gradient tasks, all tasks
-    float eta_scale;                 // eta * 2 / N
+    int T;                           // tasks (each: its gradient, then its readout)
+    float eta_scale;                 // eta * 2 / N  (dot-product loss: eta / N)
     const float* W0;                 // [heads][64][9]
     float* W1_out;                   // nullable [units][64][9]
     uint32_t* err;                   // workspace error word
-    uint32_t* queue;                 // task counter
     uint32_t* done;                  // CTAs finished
-    uint32_t* merged;                // units whose W1 is formed so far
     uint32_t* unit_count;            // [U] gradient partials written per unit
-    uint32_t* order;                 // [U] slot i: 1 + the i-th unit whose W1 was formed (0: not yet)
+    uint32_t* ready;                 // [U] 1 once the unit's W1 is formed
     float* partials;                 // [U][mtpu][CG][576] negated gradient sums per task and group, tap-major
     int mtpu;                        // partial slots per unit (one task per row pair, the most a call uses)
     float* w1g;                      // [U][576] W1 per unit, tap-major
+    unsigned long long wait_ns;      // bound of every device-side wait
 };
 
-// Workspace layout: the 256-byte header (word 0: error word), the control words (queue, done,
-// merged, unit_count[U], order[U]) padded to 256 bytes, the partials, W1.
+// Workspace layout: the 256-byte header (word 0: error word), the control words (done,
+// unit_count[U], ready[U]) padded to 256 bytes, the partials, W1.
 struct WsLayout {
     size_t ctl, partials, w1g, total;
 };
 static WsLayout ws_layout(long long U, int tpu) {
     WsLayout l;
     l.ctl = kWsHeader;
-    l.partials = l.ctl + align_up((size_t)(3 + 2 * U) * 4, 256);
+    l.partials = l.ctl + align_up((size_t)(1 + 2 * U) * 4, 256);
     l.w1g = l.partials + align_up((size_t)U * tpu * CG * kPart * 4, 256);
     l.total = l.w1g + (size_t)U * kPart * 4;
     return l;
@@ -126,27 +122,22 @@ static WsLayout ws_layout(long long U, int tpu) {
 
 struct SmemTail {                            // follows the rings
     float red[CG][kRed][kPart];              // per-warp gradients of each group, folded pairwise
-    uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], tfull[NT], tempty[NT];
-    int task[NT];
-    int task_u[NT];                          // the unit of the task (for a readout task: resolved from order)
+    uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV];
     int flag[CG];                            // per-group decision broadcast
+    int last;
     int abort_flag;
 };
 
 __host__ __device__ __forceinline__ int split_lo(int n, int r, int parts) { return (int)((long long)n * r / parts); }
 
 struct Task {
-    bool p1;
-    int u, r, sx, pa, n;                     // unit (readout task: its slot in the merge order), task index
-                                             // in the unit, strip, first pair, pairs
+    int u, r, sx, pa, n;                     // unit, task index in the unit, strip, first pair, pairs
 };
 
 __device__ __forceinline__ Task decode(const Params& p, int t) {
     Task k;
-    k.p1 = t < p.T1;
-    const int tt = k.p1 ? t : t - p.T1;
-    k.u = tt / p.g.tpu;
-    k.r = tt % p.g.tpu;
+    k.u = t / p.g.tpu;
+    k.r = t % p.g.tpu;
     k.sx = k.r / p.g.tps;
     const int c = k.r % p.g.tps;
     k.pa = split_lo(p.g.Hp, c, p.g.tps);
@@ -158,26 +149,21 @@ __device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
 
-// Channel pair `lane` of staged row `row`, column `col` (no bounds checks: the halo is staged).
-template <typename T>
-__device__ __forceinline__ float2 staged(const uint8_t* base, int pitch, int row, int col, int lane) {
-    return Elem<T>::unpack(reinterpret_cast<const typename Elem<T>::Raw*>(
-        base + ((size_t)row * pitch + col) * Elem<T>::kTokenBytes)[lane]);
-}
-
-// The 4 staged rows around an output row pair: rows 0, 1 from one group, rows 2, 3 from the next.
+// The 4 staged rows around an output row pair: rows 0, 1 from one group, rows 2, 3 from the next
+// (32-bit shared addresses of the lane's channel pair in column 0 of each group).
 struct Rows {
-    const uint8_t* a;                // rows y0-1, y0
-    const uint8_t* b;                // rows y0+1, y0+2
-    int pitch;
+    uint32_t a;                      // rows y0-1, y0
+    uint32_t b;                      // rows y0+1, y0+2
+    uint32_t row_bytes;              // bytes of one staged row (k_pitch tokens)
 };
 
 template <typename T, int C>
-__device__ __forceinline__ void load_col(float2 (&win)[4][3], const Rows& rw, int col, int lane) {
-    win[0][C] = staged<T>(rw.a, rw.pitch, 0, col, lane);
-    win[1][C] = staged<T>(rw.a, rw.pitch, 1, col, lane);
-    win[2][C] = staged<T>(rw.b, rw.pitch, 0, col, lane);
-    win[3][C] = staged<T>(rw.b, rw.pitch, 1, col, lane);
+__device__ __forceinline__ void load_col(float2 (&win)[4][3], const Rows& rw, int col) {
+    const uint32_t o = (uint32_t)col * Elem<T>::kTokenBytes;
+    win[0][C] = Elem<T>::lds(rw.a + o);
+    win[1][C] = Elem<T>::lds(rw.a + rw.row_bytes + o);
+    win[2][C] = Elem<T>::lds(rw.b + o);
+    win[3][C] = Elem<T>::lds(rw.b + rw.row_bytes + o);
 }
 
 // s = v + sum over the 3 x 3 taps of nw * K at window rows r0 .. r0+2, as three independent
@@ -219,24 +205,24 @@ __device__ __forceinline__ void neg_residual2(const float2 (&win)[4][3], const f
 // Phase-1 work of output column x (strip-relative) of the row pair: window columns L, M, R hold
 // staged columns x, x+1, x+2 (image columns x-1, x, x+1); R is loaded here.  nw = -W0 taps;
 // gacc accumulates sum s * K with s = V - W0 (*) K = -r (L2 loss) or s = V (dot-product loss, whose
-// gradient has no residual: nw is unused).
+// gradient has no residual: nw is unused).  vg: shared address of the lane's channels in V column 0
+// of the group's first row; vrow: bytes of one staged V row.
 template <typename T, bool DOT, bool ROW1, int L, int M, int R>
 __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[TAPS], float2 (&gacc)[TAPS],
-                                       const Rows& rw, const uint8_t* vg, int XT, int x, int lane) {
+                                       const Rows& rw, uint32_t vg, uint32_t vrow, int x) {
     using E = Elem<T>;
-    load_col<T, R>(win, rw, x + 2, lane);
-    const typename E::Raw* vr = reinterpret_cast<const typename E::Raw*>(vg);
+    load_col<T, R>(win, rw, x + 2);
+    const uint32_t vo = vg + (uint32_t)x * E::kTokenBytes;
     constexpr int cidx[3] = {L, M, R};
     if (ROW1) {                                            // the second row of the pair lies inside the grid
         // both rows' residual chains side by side (six independent 3-term chains), then the nine
         // row-0 updates before the nine row-1 updates, so that no update waits on the one before it
         float2 s0, s1;
         if (DOT) {
-            s0 = E::unpack(vr[(size_t)x * D / 2 + lane]);
-            s1 = E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]);
+            s0 = E::lds(vo);
+            s1 = E::lds(vo + vrow);
         } else {
-            neg_residual2<L, M, R>(win, nw, E::unpack(vr[(size_t)x * D / 2 + lane]),
-                                   E::unpack(vr[(size_t)(XT + x) * D / 2 + lane]), s0, s1);
+            neg_residual2<L, M, R>(win, nw, E::lds(vo), E::lds(vo + vrow), s0, s1);
         }
 #pragma unroll
         for (int a = 0; a < 3; ++a)
@@ -247,7 +233,7 @@ __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[T
 #pragma unroll
             for (int c = 0; c < 3; ++c) gacc[a * 3 + c] = ffma2(s1, win[a + 1][cidx[c]], gacc[a * 3 + c]);
     } else {
-        const float2 v0 = E::unpack(vr[(size_t)x * D / 2 + lane]);
+        const float2 v0 = E::lds(vo);
         const float2 s0 = DOT ? v0 : neg_residual<L, M, R>(win, nw, 0, v0);
 #pragma unroll
         for (int a = 0; a < 3; ++a)
@@ -258,27 +244,27 @@ __device__ __forceinline__ void p1_col(float2 (&win)[4][3], const float2 (&nw)[T
 
 template <typename T, bool DOT, bool ROW1>
 __device__ __forceinline__ void p1_pair(const float2 (&nw)[TAPS], float2 (&gacc)[TAPS], const Rows& rw,
-                                        const uint8_t* vg, int XT, int xa, int xb, int lane) {
+                                        uint32_t vg, uint32_t vrow, int xa, int xb) {
     float2 win[4][3];
-    load_col<T, 0>(win, rw, xa, lane);
-    load_col<T, 1>(win, rw, xa + 1, lane);
+    load_col<T, 0>(win, rw, xa);
+    load_col<T, 1>(win, rw, xa + 1);
     int x = xa;
     for (; x + 3 <= xb; x += 3) {
-        p1_col<T, DOT, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
-        p1_col<T, DOT, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
-        p1_col<T, DOT, ROW1, 2, 0, 1>(win, nw, gacc, rw, vg, XT, x + 2, lane);
+        p1_col<T, DOT, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, vrow, x);
+        p1_col<T, DOT, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, vrow, x + 1);
+        p1_col<T, DOT, ROW1, 2, 0, 1>(win, nw, gacc, rw, vg, vrow, x + 2);
     }
     if (x < xb) {
-        p1_col<T, DOT, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, XT, x, lane);
-        if (x + 1 < xb) p1_col<T, DOT, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, XT, x + 1, lane);
+        p1_col<T, DOT, ROW1, 0, 1, 2>(win, nw, gacc, rw, vg, vrow, x);
+        if (x + 1 < xb) p1_col<T, DOT, ROW1, 1, 2, 0>(win, nw, gacc, rw, vg, vrow, x + 1);
     }
 }
 
 // Phase-2 work of output column x: z = W1 (*) Q for the rows of the pair.
 template <typename T, bool ROW1, int L, int M, int R>
 __device__ __forceinline__ void p2_col(float2 (&win)[4][3], const float2 (&w)[TAPS], const Rows& rw, T* z0, T* z1,
-                                       int x, int lane) {
-    load_col<T, R>(win, rw, x + 2, lane);
+                                       int x) {
+    load_col<T, R>(win, rw, x + 2);
     constexpr int cidx[3] = {L, M, R};
     float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -293,42 +279,41 @@ __device__ __forceinline__ void p2_col(float2 (&win)[4][3], const float2 (&w)[TA
 }
 
 template <typename T, bool ROW1>
-__device__ __forceinline__ void p2_pair(const float2 (&w)[TAPS], const Rows& rw, T* z0, T* z1, int xa, int xb,
-                                        int lane) {
+__device__ __forceinline__ void p2_pair(const float2 (&w)[TAPS], const Rows& rw, T* z0, T* z1, int xa, int xb) {
     float2 win[4][3];
-    load_col<T, 0>(win, rw, xa, lane);
-    load_col<T, 1>(win, rw, xa + 1, lane);
+    load_col<T, 0>(win, rw, xa);
+    load_col<T, 1>(win, rw, xa + 1);
     int x = xa;
     for (; x + 3 <= xb; x += 3) {
-        p2_col<T, ROW1, 0, 1, 2>(win, w, rw, z0, z1, x, lane);
-        p2_col<T, ROW1, 1, 2, 0>(win, w, rw, z0, z1, x + 1, lane);
-        p2_col<T, ROW1, 2, 0, 1>(win, w, rw, z0, z1, x + 2, lane);
+        p2_col<T, ROW1, 0, 1, 2>(win, w, rw, z0, z1, x);
+        p2_col<T, ROW1, 1, 2, 0>(win, w, rw, z0, z1, x + 1);
+        p2_col<T, ROW1, 2, 0, 1>(win, w, rw, z0, z1, x + 2);
     }
     if (x < xb) {
-        p2_col<T, ROW1, 0, 1, 2>(win, w, rw, z0, z1, x, lane);
-        if (x + 1 < xb) p2_col<T, ROW1, 1, 2, 0>(win, w, rw, z0, z1, x + 1, lane);
+        p2_col<T, ROW1, 0, 1, 2>(win, w, rw, z0, z1, x);
+        if (x + 1 < xb) p2_col<T, ROW1, 1, 2, 0>(win, w, rw, z0, z1, x + 1);
     }
 }
 
 template <typename T, bool DOT>
 __global__ void __launch_bounds__(THREADS, 1)
-dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-         const __grid_constant__ CUtensorMap tmQ, T* __restrict__ Z, const Params p) {
+dw_band(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+        const __grid_constant__ CUtensorMap tmQ, T* __restrict__ Z, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    // 128-byte aligned start, derived from the shared array by pointer arithmetic only
+    uint8_t* base = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     const Geom& g = p.g;
     uint8_t* kring = base;
     uint8_t* vring = kring + (size_t)NK * g.kg_bytes;
     SmemTail& s = *reinterpret_cast<SmemTail*>(vring + (size_t)NV * g.vg_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Abort ab{&s.abort_flag, p.err};
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
 
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
         // a K group is read by two row pairs, each by GW warps; a V group by one row pair
         for (int i = 0; i < NK; ++i) { mbar_init(&s.kfull[i], 1); mbar_init(&s.kempty[i], 2 * GW); }
         for (int i = 0; i < NV; ++i) { mbar_init(&s.vfull[i], 1); mbar_init(&s.vempty[i], GW); }
-        for (int i = 0; i < NT; ++i) { mbar_init(&s.tfull[i], 1); mbar_init(&s.tempty[i], CW); }
         fence_barrier_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ);
     }
@@ -336,84 +321,67 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
 
     if (warp == CW) {                                                // producer
         if (lane == 0) {
-            uint32_t kq = 0, vq = 0, tq = 0;                         // ring sequence numbers
+            uint32_t kq = 0, vq = 0;                                 // loads issued into each ring
             auto load_k = [&](const CUtensorMap* tm, int xs, int y, int h, int bi) -> bool {
                 const uint32_t sl = kq % NK, ph = (kq / NK) & 1u;
-                ++kq;
                 if (!mbar_wait(&s.kempty[sl], ph ^ 1u, ab)) return false;
                 mbar_arrive_expect_tx(&s.kfull[sl], g.kg_bytes);
                 tma_load_5d(kring + (size_t)sl * g.kg_bytes, tm, &s.kfull[sl], 0, xs - 1, y, h, bi);
+                ++kq;
                 return true;
             };
             auto load_v = [&](int xs, int y, int h, int bi) -> bool {
                 const uint32_t sl = vq % NV, ph = (vq / NV) & 1u;
-                ++vq;
                 if (!mbar_wait(&s.vempty[sl], ph ^ 1u, ab)) return false;
                 mbar_arrive_expect_tx(&s.vfull[sl], g.vg_bytes);
                 tma_load_5d(vring + (size_t)sl * g.vg_bytes, &tmV, &s.vfull[sl], 0, xs, y, h, bi);
+                ++vq;
                 return true;
             };
-            for (;;) {
-                int t = (int)atomicAdd(p.queue, 1u);
-                if (t >= p.T) t = -1;
-                const uint32_t ts = tq % NT, tph = (tq / NT) & 1u;
-                ++tq;
-                if (!mbar_wait(&s.tempty[ts], tph ^ 1u, ab)) break;
-                Task tk = decode(p, t);
-                if (t >= 0 && !tk.p1) {
-                    // readout tasks follow the order in which units finish their gradients: slot
-                    // tk.u is filled once that many units have formed W1 (every gradient task was
-                    // claimed before any readout task, so the wait ends)
-                    if (!wait_flag(p.order + tk.u, ab)) break;
-                    tk.u = (int)ld_acquire_gpu(p.order + tk.u) - 1;
-                }
-                s.task[ts] = t;
-                s.task_u[ts] = t >= 0 ? tk.u : 0;
-                mbar_arrive(&s.tfull[ts]);
-                if (t < 0) break;
+            bool ok = true;
+            // phase 1 of every task of this CTA (K(0), then K(j+1), V(j)), then the readout rows of
+            // every task: Q streams in while the gradients are merged
+            for (int t = blockIdx.x; t < p.T && ok; t += gridDim.x) {
+                const Task tk = decode(p, t);
                 const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT, y0 = 2 * tk.pa;
-                bool ok = true;
-                if (tk.p1) {                                         // K(0), then K(j+1), V(j)
-                    ok = load_k(&tmK, xs, y0 - 1, h, bi);
-                    for (int j = 0; j < tk.n && ok; ++j)
-                        ok = load_k(&tmK, xs, y0 + 2 * j + 1, h, bi) && load_v(xs, y0 + 2 * j, h, bi);
-                } else {
-                    for (int j = 0; j <= tk.n && ok; ++j) ok = load_k(&tmQ, xs, y0 + 2 * j - 1, h, bi);
-                }
-                if (!ok) break;
+                ok = load_k(&tmK, xs, y0 - 1, h, bi);
+                for (int j = 0; j < tk.n && ok; ++j)
+                    ok = load_k(&tmK, xs, y0 + 2 * j + 1, h, bi) && load_v(xs, y0 + 2 * j, h, bi);
             }
+            for (int t = blockIdx.x; t < p.T && ok; t += gridDim.x) {
+                const Task tk = decode(p, t);
+                const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT, y0 = 2 * tk.pa;
+                for (int j = 0; j <= tk.n && ok; ++j) ok = load_k(&tmQ, xs, y0 + 2 * j - 1, h, bi);
+            }
+            // Before the CTA may exit, every load issued into the rings has landed (on a normal exit
+            // they were all consumed already; after a wait gave up, some may still be in flight).
+            for (uint32_t q = kq > (uint32_t)NK ? kq - NK : 0u; q < kq; ++q)
+                mbar_drain(&s.kfull[q % NK], (q / NK) & 1u, ab.limit);
+            for (uint32_t q = vq > (uint32_t)NV ? vq - NV : 0u; q < vq; ++q)
+                mbar_drain(&s.vfull[q % NV], (q / NV) & 1u, ab.limit);
         }
-        return;
-    }
-
-    // compute warps: CG groups of GW warps; group g takes the row pairs j = g (mod CG) of every task
-    // (a fixed split, so each partial holds the same sums whichever CTA runs the task) and publishes
-    // its own partial, so the groups never wait for one another
-    const int tid = threadIdx.x;                                     // 0 .. CW*32-1
-    const int grp = warp / GW, seg = warp % GW, gtid = tid - grp * GW * 32;
-    const uint32_t gbar = 1u + (uint32_t)grp;                        // the group's named barrier
-    uint32_t kq = 0, vq = 0, tq = 0;                                 // ring and task sequence numbers
-    bool failed = false;
-    for (;;) {
-        const uint32_t ts = tq % NT, tph = (tq / NT) & 1u;
-        ++tq;
-        const bool okt = !failed && mbar_wait(&s.tfull[ts], tph, ab);
-        const int t = okt ? s.task[ts] : -1;
-        const int tu = okt ? s.task_u[ts] : 0;
-        __syncwarp();
-        if (okt && lane == 0) mbar_arrive(&s.tempty[ts]);
-        // the warps of a group take the same decision: stop on a failure anywhere in the group
-        if (named_bar_or(gbar, GW * 32, failed || !okt)) { failed = true; break; }
-        if (t < 0) break;
-        Task tk = decode(p, t);
-        const int slot = tk.u;                                       // readout task: merge-order slot
-        tk.u = tu;
-        const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT;
-        const int cols = min(g.W - xs, g.XT), segw = (cols + GW - 1) / GW;
-        const int xa = seg * segw, xb = min(cols, xa + segw);        // strip-relative output columns
-        const int n = tk.n;
-        if (tk.p1) {
-            // ---- phase-1 task: negated gradient sums over this group's row pairs of the task
+        __syncwarp();                                                // the warp reaches the block barrier converged
+    } else {
+        // compute warps: CG groups of GW warps; group g takes the row pairs j = g (mod CG) of every task
+        // (a fixed split, so each partial holds the same sums whichever CTA runs the task) and publishes
+        // its own partial, so the groups never wait for one another
+        const int tid = threadIdx.x;                                 // 0 .. CW*32-1
+        const int grp = warp / GW, seg = warp % GW, gtid = tid - grp * GW * 32;
+        const uint32_t gbar = 1u + (uint32_t)grp;                    // the group's named barrier
+        const uint32_t kring_s = smem_u32(kring), vring_s = smem_u32(vring);
+        const uint32_t krow = (uint32_t)g.k_pitch * Elem<T>::kTokenBytes;
+        const uint32_t vrow = (uint32_t)g.XT * Elem<T>::kTokenBytes;
+        const uint32_t lane_b = (uint32_t)lane * (Elem<T>::kTokenBytes / 32);
+        uint32_t kq = 0, vq = 0;                                     // ring sequence numbers
+        bool failed = false;
+        // ---- phase 1 of every task of this CTA
+        for (int t = blockIdx.x; t < p.T && !failed; t += gridDim.x) {
+            const Task tk = decode(p, t);
+            const int h = tk.u % g.heads, xs = tk.sx * g.XT;
+            const int cols = min(g.W - xs, g.XT), segw = (cols + GW - 1) / GW;
+            const int xa = seg * segw, xb = min(cols, xa + segw);    // strip-relative output columns
+            const int n = tk.n;
+            // negated gradient sums over this group's row pairs of the task
             float2 nw[TAPS], gacc[TAPS];
 #pragma unroll
             for (int t9 = 0; t9 < TAPS; ++t9) {
@@ -431,11 +399,11 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                 if (!okb) { failed = true; continue; }
                 __syncwarp();
                 if (xa < xb) {
-                    const Rows rw{kring + (size_t)(k0 % NK) * g.kg_bytes, kring + (size_t)(k1 % NK) * g.kg_bytes,
-                                  g.k_pitch};
-                    const uint8_t* vg = vring + (size_t)(v0 % NV) * g.vg_bytes;
-                    if (2 * (tk.pa + j) + 1 < g.H) p1_pair<T, DOT, true>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
-                    else p1_pair<T, DOT, false>(nw, gacc, rw, vg, g.XT, xa, xb, lane);
+                    const Rows rw{kring_s + (k0 % NK) * g.kg_bytes + lane_b, kring_s + (k1 % NK) * g.kg_bytes + lane_b,
+                                  krow};
+                    const uint32_t vg = vring_s + (v0 % NV) * g.vg_bytes + lane_b;
+                    if (2 * (tk.pa + j) + 1 < g.H) p1_pair<T, DOT, true>(nw, gacc, rw, vg, vrow, xa, xb);
+                    else p1_pair<T, DOT, false>(nw, gacc, rw, vg, vrow, xa, xb);
                 }
                 __syncwarp();
                 if (lane == 0) {
@@ -445,6 +413,8 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                 }
             }
             kq += (uint32_t)n + 1; vq += (uint32_t)n;
+            // the group stops on a failure anywhere in it (a uniform decision)
+            if (named_bar_or(gbar, GW * 32, failed)) { failed = true; break; }
             // ---- the group's partial, summed over its warps in a fixed order
             float(*red)[kPart] = s.red[grp];
             if (seg >= kRed) {                                       // warps kRed.. store, warps 0.. add
@@ -503,12 +473,22 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                 }
                 __threadfence();
                 named_bar_sync(gbar, GW * 32);
-                if (gtid == 0) st_release_gpu(p.order + atomicAdd(p.merged, 1u), (uint32_t)tk.u + 1u);
+                if (gtid == 0) st_release_gpu(p.ready + tk.u, 1u);
             }
-        } else {
-            // ---- phase-2 task: Z = W1 (*) Q over this group's row pairs of the task
+        }
+        // ---- phase 2 of every task of this CTA: Z = W1 (*) Q over this group's row pairs
+        for (int t = blockIdx.x; t < p.T && !failed; t += gridDim.x) {
+            const Task tk = decode(p, t);
+            const int bi = tk.u / g.heads, h = tk.u % g.heads, xs = tk.sx * g.XT;
+            const int cols = min(g.W - xs, g.XT), segw = (cols + GW - 1) / GW;
+            const int xa = seg * segw, xb = min(cols, xa + segw);
+            const int n = tk.n;
+            // the unit's W1 (lane 0 waits, bounded; the warp follows its decision)
+            int okw = 1;
+            if (lane == 0) okw = wait_flag(p.ready + tk.u, ab) ? 1 : 0;
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (!okw) failed = true;
             float2 w[TAPS];
-            if (!wait_flag(p.order + slot, ab)) failed = true;             // (already set: an acquire)
 #pragma unroll
             for (int t9 = 0; t9 < TAPS; ++t9)
                 w[t9] = __ldcg(reinterpret_cast<const float2*>(p.w1g + (size_t)tk.u * kPart + t9 * D) + lane);
@@ -522,12 +502,12 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
                 __syncwarp();
                 const int y0 = 2 * (tk.pa + j);
                 if (xa < xb) {
-                    const Rows rw{kring + (size_t)(k0 % NK) * g.kg_bytes, kring + (size_t)(k1 % NK) * g.kg_bytes,
-                                  g.k_pitch};
+                    const Rows rw{kring_s + (k0 % NK) * g.kg_bytes + lane_b, kring_s + (k1 % NK) * g.kg_bytes + lane_b,
+                                  krow};
                     T* z0 = Z + off + ((long long)y0 * g.W + xs) * D + 2 * lane;
                     T* z1 = z0 + (long long)g.W * D;
-                    if (y0 + 1 < g.H) p2_pair<T, true>(w, rw, z0, z1, xa, xb, lane);
-                    else p2_pair<T, false>(w, rw, z0, z1, xa, xb, lane);
+                    if (y0 + 1 < g.H) p2_pair<T, true>(w, rw, z0, z1, xa, xb);
+                    else p2_pair<T, false>(w, rw, z0, z1, xa, xb);
                 }
                 __syncwarp();
                 if (lane == 0) {
@@ -539,16 +519,16 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
         }
     }
     // The last CTA to finish puts the control words back to zero for the next call.
-    named_bar_sync(kExitBar, CW * 32);
-    if (tid == 0) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
         __threadfence();
-        s.flag[0] = (atomicAdd(p.done, 1u) == gridDim.x - 1) ? 1 : 0;
+        s.last = (atomicAdd(p.done, 1u) == gridDim.x - 1) ? 1 : 0;
     }
-    named_bar_sync(kExitBar, CW * 32);
-    if (s.flag[0]) {
+    __syncthreads();
+    if (s.last) {
         __threadfence();
-        for (int i = tid; i < p.U; i += CW * 32) { p.unit_count[i] = 0u; p.order[i] = 0u; }
-        if (tid == 0) { *p.queue = 0u; *p.done = 0u; *p.merged = 0u; }
+        for (int i = threadIdx.x; i < p.U; i += blockDim.x) { p.unit_count[i] = 0u; p.ready[i] = 0u; }
+        if (threadIdx.x == 0) *p.done = 0u;
     }
     // As a programmatic dependent of the preceding kernel: complete only after it has completed.
     pdl_wait_primary();
@@ -557,9 +537,7 @@ dw_queue(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtens
 // ------------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------------
-// Tasks per strip: about kTasksPerCta gradient tasks per CTA (at most one task per row pair).  One
-// task per CTA measured best: a task's fixed costs (first loads, the group reductions, the unit
-// merge) are several microseconds, so two half-size tasks per CTA took longer than one.
+// Tasks per strip: about kTasksPerCta tasks per CTA (at most one task per row pair).
 template <typename T>
 static Geom make_geom(long long units, int grid, int heads, int H, int W, long long bs, long long hs) {
     constexpr int TB = Elem<T>::kTokenBytes;
@@ -601,8 +579,8 @@ static ttt_status launch(const Call& c) {
     if (smem > 227 * 1024) return TTT_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(units, g.Sx * g.Hp);
     if (c.ws_bytes < L.total) return TTT_ERR_WORKSPACE;
-    cudaFuncSetAttribute(dw_queue<T, DOT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const long long T_all = 2 * units * g.tpu;
+    cudaFuncSetAttribute(dw_band<T, DOT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const long long T_all = units * g.tpu;
     if (T_all > (1LL << 30)) return TTT_ERR_UNSUPPORTED;
     const int grid = (int)std::max<long long>(1, std::min<long long>(grid_max, T_all));
 
@@ -613,7 +591,6 @@ static ttt_status launch(const Call& c) {
     Params p;
     p.g = g;
     p.U = (int)units;
-    p.T1 = (int)(units * g.tpu);
     p.T = (int)T_all;
     // W1 = W0 + eta_scale * sum s K:  L2 loss s = -r, gradient (2/N) sum r K;  dot-product loss
     // s = V, gradient -(1/N) sum V K
@@ -622,14 +599,13 @@ static ttt_status launch(const Call& c) {
     p.W1_out = c.W1_out;
     p.err = reinterpret_cast<uint32_t*>(c.err_ws ? c.err_ws : c.ws);
     uint32_t* ctl = reinterpret_cast<uint32_t*>(c.ws + L.ctl);
-    p.queue = ctl;
-    p.done = ctl + 1;
-    p.merged = ctl + 2;
-    p.unit_count = ctl + 3;
-    p.order = ctl + 3 + units;
+    p.done = ctl;
+    p.unit_count = ctl + 1;
+    p.ready = ctl + 1 + units;
     p.partials = reinterpret_cast<float*>(c.ws + L.partials);
     p.mtpu = g.Sx * g.Hp;
     p.w1g = reinterpret_cast<float*>(c.ws + L.w1g);
+    p.wait_ns = c.wait_ns;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(THREADS);
@@ -640,7 +616,7 @@ static ttt_status launch(const Call& c) {
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = c.overlap_previous ? 1 : 0;
-    return check_launch(cudaLaunchKernelEx(&cfg, dw_queue<T, DOT>, tmK, tmV, tmQ, static_cast<T*>(c.Z), p));
+    return check_launch(cudaLaunchKernelEx(&cfg, dw_band<T, DOT>, tmK, tmV, tmQ, static_cast<T*>(c.Z), p));
 }
 
 }  // namespace dw

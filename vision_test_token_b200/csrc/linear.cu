@@ -210,6 +210,7 @@ struct ClusterParams {
     const float* W0;            // [heads][64][64]
     float* W1_out;              // nullable [units][64][64]
     uint32_t* err;
+    unsigned long long wait_ns; // bound of every device-side wait
 };
 
 struct ClusterSmem {
@@ -225,7 +226,9 @@ struct ClusterSmem {
     uint64_t prod_bar;                       // the W0 G product on the tensor cores is done
     uint64_t recv_full;                      // the peers' P have landed in zbuf (bytes via complete_tx)
     uint64_t peer_free;                      // every peer has finished the previous unit: its slots are free
+    uint64_t drain_bar, pdrain_bar;          // the MMAs of the MMA lane / of the epilogue's products (exit)
     uint32_t tmem_base;
+    uint32_t recv_armed;                     // phases of recv_full armed so far
     int abort_flag;
 };
 
@@ -235,25 +238,33 @@ __device__ __forceinline__ void cl_producer(ClusterSmem& s, const ClusterParams&
                                             const CUtensorMap* tmV, const CUtensorMap* tmQ, int rank, int cid,
                                             int ncl, const Abort& ab) {
     int st = 0; uint32_t ph = 0;
-    for (int u = cid; u < p.U; u += ncl) {
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int u = cid; u < p.U && ok; u += ncl) {
         const int b = u / p.heads, h = u % p.heads;
         const int t1b = split_lo(p.tpu1, rank, p.CS), t1e = split_lo(p.tpu1, rank + 1, p.CS);
-        for (int t = t1b; t < t1e; ++t) {
-            if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
+        for (int t = t1b; t < t1e && ok; ++t) {
+            if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
             mbar_arrive_expect_tx(&s.full[st], 2 * TILE_BYTES);
             tma_load_4d(s.stage[st], tmK, &s.full[st], 0, t * TOK, h, b);
             tma_load_4d(s.stage[st] + TILE_BYTES, tmV, &s.full[st], 0, t * TOK, h, b);
+            ++issued;
             if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
         // Q does not depend on W1: it streams in while the cluster reduces and forms W1.
         const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
-        for (int t = t2b; t < t2e; ++t) {
-            if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) return;
+        for (int t = t2b; t < t2e && ok; ++t) {
+            if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
             mbar_arrive_expect_tx(&s.full[st], 2 * TILE_BYTES);
             tma_load_4d(s.stage[st], tmQ, &s.full[st], 0, t * Q2, h, b);
+            ++issued;
             if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
     }
+    // Before the CTA may exit, every tile load it issued has landed (on a normal exit they were all
+    // consumed already; after a wait gave up, some may still be in flight).
+    for (uint32_t k = issued > (uint32_t)STAGES ? issued - STAGES : 0u; k < issued; ++k)
+        mbar_drain(&s.full[k % STAGES], (k / STAGES) & 1u, ab.limit);
 }
 
 __device__ __forceinline__ void cl_mma(ClusterSmem& s, const ClusterParams& p, uint32_t tmem, int rank, int cid,
@@ -347,6 +358,7 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
         }
         named_bar_sync(1, 128);
         if (multi && tid == 0) {
+            ++s.recv_armed;
             mbar_arrive_expect_tx(&s.recv_full, (uint32_t)((p.CS - 1) * D * D * 4));
             for (int pr = 0; pr < p.CS; ++pr)
                 if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
@@ -503,11 +515,13 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
                 __syncwarp();
                 tc_fence_after();
                 uint8_t* zrow = s.zbuf[zb] + r * 128;
+                float va[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 64u + (uint32_t)(ai * 64 + j * 16) + lane_off, va[j]);
+                tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < D; j += 16) {
-                    float v[16];
-                    tmem_ld16(tmem + 64u + (uint32_t)(ai * 64 + j) + lane_off, v);
-                    tmem_ld_wait();
+                    const float* v = va[j / 16];
                     uint4 lo, hi;
                     lo.x = pack_bf16x2(v[0], v[1]);   lo.y = pack_bf16x2(v[2], v[3]);
                     lo.z = pack_bf16x2(v[4], v[5]);   lo.w = pack_bf16x2(v[6], v[7]);
@@ -541,7 +555,13 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
                 if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
         mbar_wait_cluster(&s.peer_free, k & 1u, ab);
     }
-    if (tid == 0) bulk_wait<0>();
+    if (tid == 0) {
+        bulk_wait<0>();
+        if (!p.dot) {                                         // the product MMAs this thread issued
+            mma_commit(&s.pdrain_bar);
+            mbar_drain(&s.pdrain_bar, 0u, ab.limit);
+        }
+    }
 }
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -556,11 +576,13 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     ClusterSmem& s = *reinterpret_cast<ClusterSmem*>(align1024(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_ctarank(), cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
-    const Abort ab{&s.abort_flag, p.err};
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
 
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
+        s.recv_armed = 0;
         for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        mbar_init(&s.drain_bar, 1); mbar_init(&s.pdrain_bar, 1);
         mbar_init(&s.pacc_full, 1); mbar_init(&s.pacc_empty, 128);
         for (int i = 0; i < ACC; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
         mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
@@ -587,7 +609,12 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (lane == 0) cl_producer(s, p, &tmK, &tmV, &tmQ, rank, cid, ncl, ab);
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) cl_mma(s, p, tmem, rank, cid, ncl, ab);
+        if (lane == 0) {
+            cl_mma(s, p, tmem, rank, cid, ncl, ab);
+            // every MMA this thread issued has completed before tensor memory is freed
+            mma_commit(&s.drain_bar);
+            mbar_drain(&s.drain_bar, 0u, ab.limit);
+        }
         __syncwarp();
     } else {
         cl_epilogue(s, p, tmem, &tmZ, rank, cid, ncl, ab);
@@ -595,11 +622,20 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
+    if (p.CS > 1) {
+        // No CTA leaves while a peer may still push into it: every CTA of the cluster gets here after
+        // issuing its last push, and then each waits (bounded) for the pushes it was promised to land.
+        cluster_sync_all();
+        if (threadIdx.x == 0 && s.recv_armed > 0) mbar_drain(&s.recv_full, (s.recv_armed - 1) & 1u, ab.limit);
+        __syncthreads();
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+    // As a programmatic dependent of a preceding kernel: complete only after it has completed.
+    pdl_wait_primary();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -839,6 +875,7 @@ ttt_status launch_linear(const Call& c) {
         p.W0 = c.W0;
         p.W1_out = c.W1_out;
         p.err = reinterpret_cast<uint32_t*>(c.ws);
+        p.wait_ns = c.wait_ns;
         CUtensorMap tmK, tmV, tmQ, tmZ;
         if (!make_tmap_tokens(&tmK, c.K, c, TOK) || !make_tmap_tokens(&tmV, c.V, c, TOK) ||
             !make_tmap_tokens(&tmQ, c.Q, c, Q2) || !make_tmap_tokens(&tmZ, c.Z, c, TOK))

@@ -70,6 +70,7 @@ struct Params {
     const float* W0;                // [heads][64][64]
     float* W1_out;                  // nullable [units][64][64]
     uint32_t* err;                  // workspace error word
+    unsigned long long wait_ns;     // bound of every device-side wait
 };
 
 // Dynamic shared memory: Ctl, then Tiles, then the ring of raw stages (K, Q, V tiles as loaded).
@@ -199,7 +200,7 @@ lin_minibatch(const Params p) {
     const int rl = tid >> 3;                        // row of this lane within the CTA's 8 rows
     const int m = tid & 7;                          // feature group; tokens 2m, 2m+1 after a transpose-sum
     const int gbase = lane & 24;                    // first lane of this row's group of 8
-    const Abort ab{&ctl.abort_flag, p.err};
+    const Abort ab{&ctl.abort_flag, p.err, p.wait_ns};
     if (tid == 0) {
         ctl.abort_flag = 0;
         for (int i = 0; i < kStages; ++i) mbar_init(&ctl.full[i], 1);
@@ -356,6 +357,7 @@ static ttt_status launch(const Call& c, int b, int mode) {
     p.W0 = c.W0;
     p.W1_out = c.W1_out;
     p.err = reinterpret_cast<uint32_t*>(c.ws);
+    p.wait_ns = c.wait_ns;
     const size_t smem = smem_bytes<E>();
     cudaFuncSetAttribute(lin_minibatch<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int per_sm = 0;

@@ -58,6 +58,7 @@ struct Params {
     float* Wa_out;                          // nullable [units][256][64]
     float* Wb_out;                          // nullable [units][64][256]
     uint32_t* err;
+    unsigned long long wait_ns;     // bound of every device-side wait
 };
 
 struct Smem {
@@ -110,7 +111,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
     extern __shared__ uint8_t smem_raw[];
     Smem& s = *reinterpret_cast<Smem*>(align1024(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Abort ab{&s.abort_flag, p.err};
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
 
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
@@ -589,6 +590,7 @@ ttt_status launch_mlp(const Call& c) {
     p.Wa_out = c.W1_out;
     p.Wb_out = c.W1b_out;
     p.err = reinterpret_cast<uint32_t*>(c.ws);
+    p.wait_ns = c.wait_ns;
     CUtensorMap tmK, tmV, tmQ, tmZ;
     if (!make_tmap_tokens(&tmK, c.K, c, TOK) || !make_tmap_tokens(&tmV, c.V, c, TOK) ||
         !make_tmap_tokens(&tmQ, c.Q, c, TOK) || !make_tmap_tokens(&tmZ, c.Z, c, TOK))

@@ -32,6 +32,7 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
 struct Abort {
     volatile int* flag;     // shared memory, one per CTA
     uint32_t* err;          // global error word
+    unsigned long long limit = kWaitLimitNs;   // bound of each wait (ns)
     __device__ __forceinline__ bool raised() const { return *flag != 0; }
     __device__ __forceinline__ void raise() const {
         *flag = 1;
@@ -94,10 +95,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
         for (int i = 0; i < 4; ++i)
             if (mbar_test_suspend(a, parity)) return true;
         if (ab.raised()) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > ab.limit) {
             ab.raise();
             return false;
         }
+    }
+}
+
+// Loads from shared memory by 32-bit shared address (ld.shared: no generic-address resolution).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
+}
+
+// Waits, for at most limit_ns and whatever the CTA's abort flag says, for the phase with the given
+// parity to complete: used on the way out of a kernel, so that no copy or MMA the CTA issued is still
+// in flight when it exits.  Returns false if the bound ran out.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_test(a, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_test_suspend(a, parity)) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -141,7 +167,7 @@ __device__ __forceinline__ bool wait_flag(const uint32_t* flag, const Abort& ab)
         __nanosleep(64);
         if (ld_acquire_gpu(flag) != 0u) return true;
         if (ab.raised()) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > ab.limit) {
             ab.raise();
             return false;
         }
@@ -214,7 +240,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         for (int i = 0; i < 4; ++i)
             if (mbar_test_cluster(a, parity)) return true;
         if (ab.raised()) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > ab.limit) {
             ab.raise();
             return false;
         }

@@ -39,7 +39,11 @@ struct Call {
     int overlap_previous;    // launch as a programmatic dependent of the preceding kernel in the stream
     uint8_t* err_ws;         // workspace whose error word the kernels report to (nullptr: ws itself)
     int* grid_out;           // nullable: the launch writes the number of CTAs it launched
+    unsigned long long wait_ns;   // bound of every device-side wait of the launch (ns)
 };
+
+// Bound of the device-side waits of every launch (ns), process-wide (ttt_set_wait_limit).
+unsigned long long wait_limit_ns();
 
 // Encodes a rank-4 bf16 tensor map over [batch][heads][N][64] with a 64 x box_rows box,
 // 128-byte swizzle, zero fill out of bounds.  Returns false on failure.
@@ -77,6 +81,14 @@ ttt_status launch_linear_minibatch(const Call& c, int batch_tokens, int mode);
 // Full synchronous validation of a call (the checks every entry point runs before launching).
 ttt_status validate_call(int kind, const void* Q, const void* K, const void* V, const float* W0, const float* W0b,
                          void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, size_t need, void* stream);
+
+// The validation of ttt_forward_linear (shape, pointers, workspace of ws_bytes, W1_out) into *c.
+ttt_status prepare_linear(const void* Q, const void* K, const void* V, const float* W0, void* Z, float eta,
+                          const ttt_shape* s, void* ws, size_t ws_bytes, float* W1_out, void* stream, Call* c);
+
+// Synchronises `stream`, reads the error word at the start of device buffer ws; a recorded timeout
+// is cleared and reported as TTT_ERR_TIMEOUT.
+ttt_status read_error_word(void* ws, void* stream);
 
 // Records a launch error in the library's sticky error and maps it to a status.
 ttt_status check_launch(cudaError_t e);
