@@ -9,6 +9,7 @@ Functions and the definitions they follow (page titles and sections; see ``ttt_o
   linear(...)       L2 loss, one full-batch gradient step on W (d x d), z = W1 q  -- per-pair form
   linear_gram(...)  the same step written as W0 - eta (2/N) (W0 K K^T - V K^T)
   dwconv(...)       the same loss with a 3x3 depthwise cross-correlation inner model
+  conv3x3(...)      the same loss with a full 3x3 cross-correlation (d -> d channels) inner model
   mlp(...)          the same loss with f(x) = Wb gelu_tanh(Wa x)
   linear_dot(...), dwconv_dot(...)
                     the linear and conv heads under the dot-product inner loss -(1/N) sum <f(k), v>
@@ -47,11 +48,12 @@ def _load():
         lib.oracle_linear_backward.argtypes = [i, i, i, i, dp, dp, dp, dp, d, dp, dp, dp, dp, dp, dp, i]
         lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv_dot.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_conv3x3.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
         for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_linear_minibatch,
                   lib.oracle_linear_backward,
                   lib.oracle_dwconv,
-                  lib.oracle_dwconv_dot, lib.oracle_mlp):
+                  lib.oracle_dwconv_dot, lib.oracle_conv3x3, lib.oracle_mlp):
             f.restype = ctypes.c_int
         lib.oracle_gelu_tanh.argtypes = [d]
         lib.oracle_gelu_tanh.restype = d
@@ -153,6 +155,19 @@ def dwconv(Q, K, V, W0, eta, Hg, Wg, threads=None):
     W1 = np.empty((B, H, d, 3, 3))
     _check(_load().oracle_dwconv(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1),
                                  _p(Z), threads or default_threads()), "dwconv")
+    return Z, W1
+
+
+def conv3x3(Q, K, V, W0, eta, Hg, Wg, threads=None):
+    """Full 3x3 conv inner model.  Q, K, V: [B][h][Hg*Wg][d]; W0: [h][d][d][3][3].
+    Returns (Z, W1 [B][h][d][d][3][3])."""
+    Q, K, V, W0 = _f64(Q), _f64(K), _f64(V), _f64(W0)
+    B, H, N, d = Q.shape
+    assert N == Hg * Wg and K.shape == Q.shape and V.shape == Q.shape and W0.shape == (H, d, d, 3, 3)
+    Z = np.empty_like(Q)
+    W1 = np.empty((B, H, d, d, 3, 3))
+    _check(_load().oracle_conv3x3(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1),
+                                  _p(Z), threads or default_threads()), "conv3x3")
     return Z, W1
 
 

@@ -26,6 +26,8 @@
  *     - the gradient is the MEAN over the N pairs (factor 2/N), not the sum;
  *     - the conv head is a cross-correlation with zero padding, stride 1, no bias, one 3x3 kernel
  *       per channel, tokens in raster order n = y*W + x, channel c = feature c of the head;
+ *       the full 3x3 conv head (the article's other variant) has the same conventions with a
+ *       d x d x 3 x 3 kernel, every output channel reading every input channel;
  *     - the MLP head is f(x) = Wb * gelu_tanh(Wa * x) with no biases, and both matrices take one
  *       simultaneous step from gradients evaluated at the initial weights.
  *     - the dot-product inner loss of the ViT3 recipe (press article, section on the ViT3 model;
@@ -42,6 +44,8 @@
  *   Q, K, V, Z : [B][heads][N][d]     (token n, feature c at ((b*heads + h)*N + n)*d + c)
  *   linear W   : [heads][d][d]        W[i][j] maps input feature j to output feature i
  *   conv W     : [heads][d][3][3]     W[c][a][b] multiplies the input at offset (a-1, b-1)
+ *   dense conv W: [heads][d][d][3][3] W[c][c'][a][b] maps input channel c' at offset (a-1, b-1)
+ *                                     to output channel c
  *   mlp Wa     : [heads][hidden][d],  Wb : [heads][d][hidden]
  *   updated weights are returned per unit: [B][heads][...]
  *
@@ -494,6 +498,74 @@ int oracle_dwconv(int B, int heads, int Hg, int Wg, int d, const double* Q, cons
         const size_t off = (size_t)u * N * d;
         int s = dwconv_unit(Hg, Wg, d, Q + off, K + off, V + off, W0 + (size_t)h * d * 9, eta,
                             W1 + (size_t)u * d * 9, Z + off);
+        if (s != ORACLE_OK) {
+#pragma omp atomic write
+            status = s;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Full (dense) 3x3 convolution inner model over the token grid (press article, Observation 6   */
+/* and Fig. 5 part 3: the inner model implemented as a 3x3 convolution or as a depthwise one).  */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One unit.  f(X;W)[c,y,x] = sum_{c'} sum_{a,b in 0..2} W[c][c'][a][b] * X[c', y+a-1, x+b-1]
+ * (every output channel reads every input channel; zero padding; no bias).
+ * r = f(K;W0) - V;  g[c][c'][a][b] = (2/N) sum_{y,x} r[c,y,x] * K[c', y+a-1, x+b-1];
+ * W1 = W0 - eta*g;  Z = f(Q;W1).  W: [d][d][3][3]. */
+static int conv3x3_unit(int Hg, int Wg, int d, const double* Q, const double* K, const double* V,
+                        const double* W0, double eta, double* W1, double* Z)
+{
+    const int N = Hg * Wg;
+    double* g = (double*)calloc((size_t)d * d * 9, sizeof(double));
+    if (!g) return ORACLE_ERR_NOMEM;
+    for (int c = 0; c < d; ++c)
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double f = 0.0;
+                for (int cp = 0; cp < d; ++cp)
+                    for (int a = 0; a < 3; ++a)
+                        for (int b = 0; b < 3; ++b)
+                            f += W0[((size_t)c * d + cp) * 9 + a * 3 + b] * grid_at(K, Hg, Wg, d, cp, y + a - 1, x + b - 1);
+                const double r = f - V[((size_t)y * Wg + x) * d + c];
+                for (int cp = 0; cp < d; ++cp)
+                    for (int a = 0; a < 3; ++a)
+                        for (int b = 0; b < 3; ++b)
+                            g[((size_t)c * d + cp) * 9 + a * 3 + b] += r * grid_at(K, Hg, Wg, d, cp, y + a - 1, x + b - 1);
+            }
+    const double scale = 2.0 / (double)N;
+    for (size_t i = 0; i < (size_t)d * d * 9; ++i) W1[i] = W0[i] - eta * scale * g[i];
+    for (int c = 0; c < d; ++c)
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double f = 0.0;
+                for (int cp = 0; cp < d; ++cp)
+                    for (int a = 0; a < 3; ++a)
+                        for (int b = 0; b < 3; ++b)
+                            f += W1[((size_t)c * d + cp) * 9 + a * 3 + b] * grid_at(Q, Hg, Wg, d, cp, y + a - 1, x + b - 1);
+                Z[((size_t)y * Wg + x) * d + c] = f;
+            }
+    free(g);
+    return ORACLE_OK;
+}
+
+int oracle_conv3x3(int B, int heads, int Hg, int Wg, int d, const double* Q, const double* K,
+                   const double* V, const double* W0, double eta, double* W1, double* Z, int nthreads)
+{
+    if (B < 0 || heads < 0 || Hg < 1 || Wg < 1 || d < 1 || !Q || !K || !V || !W0 || !W1 || !Z)
+        return ORACLE_ERR_ARG;
+    const long units = (long)B * heads;
+    const size_t N = (size_t)Hg * Wg;
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long u = 0; u < units; ++u) {
+        const int h = (int)(u % heads);
+        const size_t off = (size_t)u * N * d;
+        int s = conv3x3_unit(Hg, Wg, d, Q + off, K + off, V + off, W0 + (size_t)h * d * d * 9, eta,
+                             W1 + (size_t)u * d * d * 9, Z + off);
         if (s != ORACLE_OK) {
 #pragma omp atomic write
             status = s;

@@ -6,8 +6,10 @@
   solution (numpy.linalg.lstsq) whatever W0 is;
 * invariants: eta = 0 gives z = f(q; W0); values that the initial model already reproduces give a
   zero update; the identity conv kernel with V = K reproduces Q;
-* library special cases: torch conv2d(groups=d), torch gelu(approximate="tanh") and torch float64
-  autograd of the pages' L2 loss;
+* library special cases: torch conv2d (groups=d for the depthwise head, groups=1 for the full 3x3
+  head), torch gelu(approximate="tanh") and torch float64 autograd of the pages' L2 loss;
+* reductions between heads: a channel-diagonal full 3x3 kernel is the depthwise head, and a full 3x3
+  kernel on a one-token grid is the linear head;
 * planted mistakes (a transposed gradient, a flipped sign, a 1/N instead of 2/N factor, a dropped
   update) are shown to fail the pins.
 """
@@ -523,6 +525,153 @@ def test_dwconv_centre_tap_matches_diagonal_linear_gradient():
     _, W1l = oracle.linear(Q, K, V, np.diag(w)[None], eta)
     np.testing.assert_allclose((Wc[0, :, 1, 1] - W1c[0, 0, :, 1, 1]),
                                np.diag(np.diag(w) - W1l[0, 0]), atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------------------------------------------
+# full 3x3 conv head: f(X;W)[c,y,x] = sum_{c',a,b} W[c][c'][a][b] X[c', y+a-1, x+b-1]
+# ------------------------------------------------------------------------------------------------
+def _frac_loss_conv3x3(W, K, V, Hg, Wg):
+    """(1/N) sum_{c,y,x} (f(K;W)[c,y,x] - V[c,y,x])^2 in exact rational arithmetic, the dense
+    cross-correlation written from its definition (every output channel reads every input one)."""
+    d = len(K[0])
+    tot = Fraction(0)
+    for c in range(d):
+        for y in range(Hg):
+            for x in range(Wg):
+                f = Fraction(0)
+                for cp in range(d):
+                    for a in range(3):
+                        for b in range(3):
+                            yy, xx = y + a - 1, x + b - 1
+                            if 0 <= yy < Hg and 0 <= xx < Wg:
+                                f += W[c][cp][a][b] * K[yy * Wg + xx][cp]
+                r = f - V[y * Wg + x][c]
+                tot += r * r
+    return tot / (Hg * Wg)
+
+
+def _conv3x3_fd_grad(W0, K, V, Hg, Wg, entries):
+    """Exact central differences (step 1; the loss is quadratic in W) at the listed entries."""
+    Kf = [[Fraction(int(v)) for v in row] for row in K]
+    Vf = [[Fraction(int(v)) for v in row] for row in V]
+    Wf = [[[[Fraction(int(v)) for v in r] for r in W0[c][cp]] for cp in range(W0.shape[1])] for c in range(W0.shape[0])]
+    out = {}
+    for (c, cp, a, b) in entries:
+        Wp = [[[r[:] for r in k] for k in ch] for ch in Wf]
+        Wm = [[[r[:] for r in k] for k in ch] for ch in Wf]
+        Wp[c][cp][a][b] += 1
+        Wm[c][cp][a][b] -= 1
+        out[(c, cp, a, b)] = float((_frac_loss_conv3x3(Wp, Kf, Vf, Hg, Wg) - _frac_loss_conv3x3(Wm, Kf, Vf, Hg, Wg)) / 2)
+    return out
+
+
+def _torch_conv3x3_f(X, W, Hg, Wg):
+    """Full 3x3 cross-correlation through torch.conv2d (groups=1): X [N][d] -> [N][d]."""
+    N, d = X.shape
+    img = X.T.reshape(1, d, Hg, Wg)
+    return F.conv2d(img, W, padding=1).reshape(W.shape[0], N).T
+
+
+def test_conv3x3_gradient_exact_rational_fd():
+    Hg, Wg, d, eta = 3, 4, 2, 1.0
+    N = Hg * Wg
+    K = _small_ints((N, d)); V = _small_ints((N, d)); Q = _small_ints((N, d))
+    W0 = _small_ints((d, d, 3, 3))
+    _, W1 = oracle.conv3x3(Q[None, None], K[None, None], V[None, None], W0[None], eta, Hg, Wg)
+    grad = (W0 - W1[0, 0]) / eta
+    entries = [(c, cp, a, b) for c in range(d) for cp in range(d) for a in range(3) for b in range(3)]
+    fd = _conv3x3_fd_grad(W0, K, V, Hg, Wg, entries)
+    for e, exact in fd.items():
+        assert abs(grad[e] - exact) <= 1e-12 * max(1.0, abs(exact)), e
+
+
+@pytest.mark.parametrize("mistake", ["sign", "transposed_channels", "flipped_taps", "half_scale"])
+def test_planted_mistakes_fail_the_conv3x3_pin(mistake):
+    """A copy of the oracle's gradient with a planted mistake must disagree with the exact
+    differences: the pin detects sign, channel-transpose, tap-flip and scale errors."""
+    Hg, Wg, d, eta = 3, 4, 2, 1.0
+    N = Hg * Wg
+    K = _small_ints((N, d)); V = _small_ints((N, d)); Q = _small_ints((N, d))
+    W0 = _small_ints((d, d, 3, 3))
+    _, W1 = oracle.conv3x3(Q[None, None], K[None, None], V[None, None], W0[None], eta, Hg, Wg)
+    grad = (W0 - W1[0, 0]) / eta
+    bad = {"sign": -grad, "transposed_channels": grad.transpose(1, 0, 2, 3),
+           "flipped_taps": grad[:, :, ::-1, ::-1], "half_scale": grad / 2}[mistake]
+    entries = [(c, cp, a, b) for c in range(d) for cp in range(d) for a in range(3) for b in range(3)]
+    fd = _conv3x3_fd_grad(W0, K, V, Hg, Wg, entries)
+    assert max(abs(bad[e] - v) for e, v in fd.items()) > 1e-6
+
+
+@pytest.mark.parametrize("Hg,Wg", [(5, 7), (1, 6), (6, 1), (1, 1)])
+def test_conv3x3_eta_zero_is_torch_conv2d(Hg, Wg):
+    d = 6
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 2, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((2, d, d, 3, 3))
+    Z, W1 = oracle.conv3x3(Q, K, V, W0, 0.0, Hg, Wg)
+    for h in range(2):
+        ref = _torch_conv3x3_f(torch.tensor(Q[0, h]), torch.tensor(W0[h]), Hg, Wg).numpy()
+        np.testing.assert_allclose(Z[0, h], ref, atol=1e-12, rtol=0)
+        np.testing.assert_array_equal(W1[0, h], W0[h])
+
+
+@pytest.mark.parametrize("Hg,Wg", [(6, 5), (1, 9), (4, 1)])
+def test_conv3x3_matches_torch_autograd(Hg, Wg):
+    d, eta = 5, 0.5
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((1, 1, N, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, d, 3, 3)) * 0.3
+    Z, W1 = oracle.conv3x3(Q, K, V, W0, eta, Hg, Wg)
+    W = torch.tensor(W0[0], requires_grad=True)
+    r = _torch_conv3x3_f(torch.tensor(K[0, 0]), W, Hg, Wg) - torch.tensor(V[0, 0])
+    loss = (r ** 2).sum(-1).mean()
+    loss.backward()
+    W1_ref = (W - eta * W.grad).detach()
+    np.testing.assert_allclose(W1[0, 0], W1_ref.numpy(), atol=1e-12, rtol=0)
+    Zref = _torch_conv3x3_f(torch.tensor(Q[0, 0]), W1_ref, Hg, Wg).numpy()
+    np.testing.assert_allclose(Z[0, 0], Zref, atol=1e-12, rtol=0)
+
+
+def test_conv3x3_channel_diagonal_kernel_reduces_to_depthwise_head():
+    """With W0[c][c'] = 0 for c != c', the residual is the depthwise head's, so the diagonal of the
+    dense update equals the depthwise update (the off-diagonal entries move too)."""
+    Hg, Wg, d, eta = 6, 5, 6, 0.7
+    N = Hg * Wg
+    Q, K, V = (RNG.standard_normal((2, 1, N, d)) for _ in range(3))
+    Wdw = RNG.standard_normal((1, d, 3, 3))
+    Wfull = np.zeros((1, d, d, 3, 3))
+    for c in range(d):
+        Wfull[0, c, c] = Wdw[0, c]
+    _, W1f = oracle.conv3x3(Q, K, V, Wfull, eta, Hg, Wg)
+    _, W1d = oracle.dwconv(Q, K, V, Wdw, eta, Hg, Wg)
+    for c in range(d):
+        np.testing.assert_allclose(W1f[:, 0, c, c], W1d[:, 0, c], atol=1e-12, rtol=0)
+    off = W1f[:, 0] - Wfull[0][None]
+    assert np.abs(off[:, 0, 1]).max() > 0.0
+
+
+def test_conv3x3_single_token_grid_is_the_linear_head():
+    """On a 1 x 1 grid only the centre tap sees a token: the centre taps are the linear head's W
+    (same update, same readout) and every other tap gets no update."""
+    d, eta = 6, 0.8
+    Q, K, V = (RNG.standard_normal((3, 1, 1, d)) for _ in range(3))
+    W0 = RNG.standard_normal((1, d, d, 3, 3))
+    Z, W1 = oracle.conv3x3(Q, K, V, W0, eta, 1, 1)
+    Zl, W1l = oracle.linear(Q, K, V, W0[:, :, :, 1, 1], eta)
+    np.testing.assert_allclose(W1[:, 0, :, :, 1, 1], W1l[:, 0], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(Z, Zl, atol=1e-12, rtol=0)
+    mask = np.ones((3, 3), bool); mask[1, 1] = False
+    assert np.all(W1[:, 0][..., mask] == np.broadcast_to(W0[0][..., mask], W1[:, 0][..., mask].shape))
+
+
+def test_conv3x3_reproduced_values_give_no_update():
+    Hg, Wg, d = 5, 6, 4
+    N = Hg * Wg
+    Q, K = RNG.standard_normal((1, 1, N, d)), RNG.standard_normal((1, 1, N, d))
+    W0 = RNG.standard_normal((1, d, d, 3, 3))
+    V = _torch_conv3x3_f(torch.tensor(K[0, 0]), torch.tensor(W0[0]), Hg, Wg).numpy()[None, None]
+    _, W1 = oracle.conv3x3(Q, K, V, W0, 1.0, Hg, Wg)
+    np.testing.assert_allclose(W1[0, 0], W0[0], atol=1e-12, rtol=0)
 
 
 # ------------------------------------------------------------------------------------------------
