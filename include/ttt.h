@@ -70,7 +70,8 @@ typedef enum {
     TTT_HEAD_LINEAR = 0,
     TTT_HEAD_DWCONV = 1,
     TTT_HEAD_MLP = 2,
-    TTT_HEAD_LINEAR_BACKWARD = 3   /* the workspace of ttt_backward_linear */
+    TTT_HEAD_LINEAR_BACKWARD = 3,  /* the workspace of ttt_backward_linear */
+    TTT_HEAD_CONV3X3 = 4           /* the workspace of ttt_forward_conv3x3 */
 } ttt_head_kind;
 
 /* Inner loss of the one-step training.
@@ -136,6 +137,25 @@ ttt_status ttt_forward_linear(const void* Q, const void* K, const void* V, const
 ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const float* W0,
                               void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes,
                               float* W1_out, void* stream);
+
+/* Full 3x3 convolution inner model over the H x W grid (press article, Observation 6 and Fig. 5
+ * part 3: the inner model implemented as a 3x3 convolution, beside the depthwise variant above):
+ * cross-correlation, zero padding, stride 1, no bias, every output channel reading every input one:
+ *   f(X;W)[c,y,x] = sum_{c'} sum_{a,b=0..2} W[c][c'][a][b] X[c', y+a-1, x+b-1].
+ *   r = f(K;W0) - V;  g[c][c'][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c', y+a-1, x+b-1];  W1 = W0 - eta g;
+ *   Z = f(Q;W1).
+ *   W0: [heads][d][d][3][3] fp32.  W1_out: optional [batch][heads][d][d][3][3] fp32.
+ *   The three contractions (576 input features per position) run on the tensor cores with bf16
+ *   operands and fp32 accumulation: W0 is rounded to bf16 for the residual, the residual is carried
+ *   as two bf16 parts (about 16 significant bits), W1 is rounded once to bf16 for the readout.
+ *   bf16 and TTT_LOSS_L2 only (fp32 or TTT_LOSS_DOT returns TTT_ERR_UNSUPPORTED).
+ *   ws: ttt_workspace_bytes(TTT_HEAD_CONV3X3, s) bytes (per-CTA partial gradients of 144 KB each and
+ *   the updated weights as bf16 operand images); it needs no zero fill, every call writes what it reads.
+ *   Work is split over CTAs in fixed ranges: results are bitwise reproducible for a fixed SM budget.
+ */
+ttt_status ttt_forward_conv3x3(const void* Q, const void* K, const void* V, const float* W0,
+                               void* Z, float eta, const ttt_shape* s, void* ws, size_t ws_bytes,
+                               float* W1_out, void* stream);
 
 /* One-hidden-layer MLP inner model f(x) = Wb gelu_tanh(Wa x) (press article, Observation 4 and
  * Fig. 5 part 1: width ratio up to 4), gelu_tanh(u) = u/2 (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3))).

@@ -76,6 +76,23 @@ bool make_tmap_grid(CUtensorMap* m, const void* base, const Call& c, int box_col
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_grid_sw128(CUtensorMap* m, const void* base, const Call& c, int box_cols, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const long long esz = 2;   // bf16
+    const long long hs = (c.heads > 1) ? c.hs : (long long)c.N * c.d;
+    const long long bs = (c.batch > 1) ? c.bs : hs * c.heads;
+    cuuint64_t dims[5] = {(cuuint64_t)c.d, (cuuint64_t)c.W, (cuuint64_t)c.H, (cuuint64_t)c.heads, (cuuint64_t)c.batch};
+    cuuint64_t strides[4] = {(cuuint64_t)(c.d * esz), (cuuint64_t)((long long)c.W * c.d * esz), (cuuint64_t)(hs * esz),
+                             (cuuint64_t)(bs * esz)};
+    cuuint32_t box[5] = {(cuuint32_t)c.d, (cuuint32_t)box_cols, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -101,6 +118,10 @@ static ttt_status check_shape(int kind, const ttt_shape* s) {
     if (s->loss != TTT_LOSS_L2 && s->loss != TTT_LOSS_DOT) return TTT_ERR_INVALID_ARG;
     if ((long long)s->batch * s->heads > (1LL << 24)) return TTT_ERR_INVALID_ARG;
     if (s->d != 64) return TTT_ERR_UNSUPPORTED;
+    if (kind == TTT_HEAD_CONV3X3) {
+        if (s->dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+        if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
+    }
     if (kind == TTT_HEAD_MLP) {
         if (s->hidden < 64 || s->hidden % 64 != 0) return TTT_ERR_INVALID_ARG;
         if (s->hidden > 256) return TTT_ERR_UNSUPPORTED;
@@ -236,6 +257,7 @@ size_t ttt_workspace_bytes(int kind, const ttt_shape* s) {
         case TTT_HEAD_DWCONV: return dwconv_ws_bytes(*s);
         case TTT_HEAD_MLP: return mlp_ws_bytes(*s);
         case TTT_HEAD_LINEAR_BACKWARD: return linear_backward_ws_bytes(*s);
+        case TTT_HEAD_CONV3X3: return conv3x3_ws_bytes(*s);
         default: return 0;
     }
 }
@@ -269,6 +291,17 @@ ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const
     if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
     c.W1_out = W1_out;
     return launch_dwconv(c);
+}
+
+ttt_status ttt_forward_conv3x3(const void* Q, const void* K, const void* V, const float* W0, void* Z, float eta,
+                               const ttt_shape* s, void* ws, size_t ws_bytes, float* W1_out, void* stream) {
+    Call c;
+    const size_t need = (check_shape(TTT_HEAD_CONV3X3, s) == TTT_OK) ? conv3x3_ws_bytes(*s) : 0;
+    ttt_status st = prepare(TTT_HEAD_CONV3X3, Q, K, V, W0, nullptr, Z, eta, s, ws, ws_bytes, need, stream, &c);
+    if (st != TTT_OK) return st;
+    if (W1_out && (reinterpret_cast<uintptr_t>(W1_out) % 16 || !is_device_ptr(W1_out))) return TTT_ERR_INVALID_ARG;
+    c.W1_out = W1_out;
+    return launch_conv3x3(c);
 }
 
 ttt_status ttt_forward_mlp(const void* Q, const void* K, const void* V, const float* Wa, const float* Wb, void* Z,

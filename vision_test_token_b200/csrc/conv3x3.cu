@@ -1,0 +1,671 @@
+// conv3x3.cu -- full 3x3 convolution inner model of the TTT layer over the H x W token grid (press
+// article "CVPR 2026 Oral | 清華+阿里發布ViT3", Observation 6 and Fig. 5 part 3: the inner model
+// implemented as a 3x3 convolution, beside the depthwise one).  Every output channel reads every
+// input channel:
+//     f(X;W)[c,y,x] = sum_{c'} sum_{a,b} W[c][c'][a][b] X[c', y+a-1, x+b-1]      (zero padding)
+//     r = f(K;W0) - V,   g[c][c'][a][b] = (2/N) sum_{y,x} r[c,y,x] K[c', y+a-1, x+b-1],
+//     W1 = W0 - eta g,   Z = f(Q;W1).
+// With the 576 features of a position's 3 x 3 neighbourhood (im2col, K~ = [K_0 | ... | K_8], K_t the
+// grid shifted by tap t), f is the linear map W~ (64 x 576) and the step is three dense contractions,
+// which go to the tensor cores (tcgen05, bf16 operands, fp32 accumulation in tensor memory):
+//     R = K~ W0~^T - V          (positions x 64,   K = 576: nine taps of 64 channels)
+//     G = sum_pos K~^T R        (576 x 64: the gradient, transposed)
+//     Z = Q~ W1~^T              (positions x 64)
+// The tap shifts are never materialised: each tap's operand is a TMA box of the grid at the shifted
+// origin, whose out-of-bounds zero fill is the zero padding.  Tiles are 8 rows x 16 columns of the
+// grid (128 positions, the MMA's M).
+//
+// Three kernels on one stream, each a programmatic dependent of the one before:
+//   conv3_grad    (per CTA, a contiguous range of tiles; per tile) TMA loads V and the 9 K boxes
+//                 (two taps per 32 KB ring stage); R = K~ W0~^T accumulates over the taps (A = K box,
+//                 K-major; B = W0 tap image, rows c, K = c'); the epilogue forms r = R - V, zeroes
+//                 positions outside the grid and splits r into bf16 hi + lo (about 16 significant
+//                 bits); the 9 K boxes are streamed again and G^T += [K_t | K_t+1]^T (r_hi + r_lo)
+//                 accumulates in five tap-pair accumulators (A MN-major, M = 128 = two taps' channels;
+//                 B = r, MN-major).  At the end of each unit's part of the range the accumulators
+//                 are written to the workspace slot of (CTA, unit).
+//   conv3_merge   per (unit, tap): the unit's slots summed in CTA order (a fixed order: bitwise
+//                 reproducible for a given grid), W1 = W0 - eta (2/N) g in fp32 (W1_out), and W1
+//                 rounded once to bf16 as the tap's operand image for the readout.
+//   conv3_readout (per CTA, a contiguous range of tiles) Z = sum_t Q_t W1_t^T over the 9 shifted Q
+//                 boxes, drained to bf16 and stored with TMA (the store clips positions outside the
+//                 grid).
+// The weights are read in bf16 for R (their rounding changes r by about 2^-9 of |f(K;W0)|) and r is
+// carried as hi + lo, so the update keeps close to fp32 accuracy relative to the gradient's terms.
+#include <algorithm>
+
+#include "sm100.cuh"
+#include "ttt_internal.h"
+
+namespace ttt {
+namespace c3 {
+
+constexpr int D = 64;
+constexpr int TAPS = 9;
+constexpr int TR = 8, TC = 16;              // a tile: 8 grid rows x 16 grid columns
+constexpr int TILE = TR * TC;               // 128 positions (the MMA's M)
+constexpr int BOX = TILE * D * 2;           // one tap box: 16 KB (128 bytes per position)
+constexpr int PAIR = 2 * BOX;               // one ring stage: two taps
+constexpr int NPAIR = 5;                    // taps (0,1) (2,3) (4,5) (6,7) (8)
+constexpr int S1 = 3;                       // ring stages of the gradient kernel
+constexpr int S3 = 3;                       // ring stages of the readout kernel
+constexpr int kWImg = D * D * 2;            // one tap's weights as a bf16 operand image: 8 KB
+constexpr int kThreads = 192;
+constexpr int kMaxGrid = 160;               // slots of the workspace: (kMaxGrid + units)
+constexpr int kSlotFloats = TAPS * D * D;   // one gradient partial, G^T [tap][c'][c]
+constexpr uint32_t kIdescRow = idesc_bf16_f32(128, 64, false, false);  // D[pos][c] = sum_k A[pos][k] B[c][k]
+constexpr uint32_t kIdescCol = idesc_bf16_f32(128, 64, true, true);    // D[m][c] = sum_pos A[pos][m] B[pos][c]
+constexpr uint32_t kColR = 0;               // tensor memory: two R accumulators,
+constexpr uint32_t kColG = 128;             //   five tap-pair gradient accumulators (448 columns)
+
+__host__ __device__ __forceinline__ int taps_in_pair(int k) { return k < 4 ? 2 : 1; }
+
+struct Geo {
+    int heads, H, W;
+    int tiles_x, tpu;                        // tiles along x, tiles per unit
+    long long T;                             // tiles of the call
+    float eta_scale;                         // eta * 2 / N
+};
+
+// CTA c of G owns tiles [start(c), start(c + 1)); the CTA that owns tile t.
+__host__ __device__ __forceinline__ long long part_start(long long T, int G, int c) { return (long long)c * T / G; }
+__host__ __device__ __forceinline__ int part_cta(long long T, int G, long long t) { return (int)(((t + 1) * G - 1) / T); }
+
+struct TileXY {
+    int u, b, h, x0, y0;
+};
+__device__ __forceinline__ TileXY tile_xy(const Geo& g, long long t) {
+    TileXY r;
+    r.u = (int)(t / g.tpu);
+    const int i = (int)(t % g.tpu);
+    r.b = r.u / g.heads;
+    r.h = r.u % g.heads;
+    r.x0 = (i % g.tiles_x) * TC;
+    r.y0 = (i / g.tiles_x) * TR;
+    return r;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// 16-byte chunk j (channels 8j .. 8j+7) of position row `row` of a 128-byte swizzled operand image.
+__device__ __forceinline__ uint32_t sw_off(int row, int j) { return (uint32_t)(row * 128 + ((j ^ (row & 7)) << 4)); }
+
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    uint4 pk;
+    pk.x = pack_bf16x2(v[0], v[1]); pk.y = pack_bf16x2(v[2], v[3]);
+    pk.z = pack_bf16x2(v[4], v[5]); pk.w = pack_bf16x2(v[6], v[7]);
+    return pk;
+}
+
+// ------------------------------------------------------------------------------------------------
+// conv3_grad
+// ------------------------------------------------------------------------------------------------
+struct GradParams {
+    Geo g;
+    int G;                                   // CTAs
+    const float* W0;                         // [heads][64][64][9]
+    float* slots;                            // [(kMaxGrid + U)][9][64][64]: G^T of a (CTA, unit) part
+    uint32_t* err;
+    unsigned long long wait_ns;
+};
+
+struct GradSmem {
+    uint8_t ring[S1][PAIR];                  // 1024-aligned operand buffers
+    uint8_t w0img[TAPS][kWImg];              // W0 of the part's head, bf16 (row c, K = c')
+    uint8_t vbuf[BOX];                       // the tile's V
+    uint8_t rhi[BOX], rlo[BOX];              // r = R - V as bf16 hi and lo (position-major)
+    uint64_t full[S1], empty[S1];
+    uint64_t vfull, vempty;
+    uint64_t dr_full[2], dr_empty[2];        // R accumulators
+    uint64_t r_full, r_empty;                // r operands written / read by every MMA of the tile
+    uint64_t w_full, w_empty;                // W0 images written / no longer read
+    uint64_t g_full, g_empty;                // a part's gradient accumulators complete / drained
+    uint64_t drain_bar;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ void grad_producer(GradSmem& s, const GradParams& p, const CUtensorMap* tmK,
+                                              const CUtensorMap* tmV, const Abort& ab) {
+    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    uint32_t issued = 0, vq = 0;
+    int st = 0; uint32_t ph = 0;
+    bool ok = true;
+    for (long long t = t0; t < t1 && ok; ++t) {
+        const TileXY x = tile_xy(p.g, t);
+        if (!(ok = mbar_wait(&s.vempty, (vq & 1u) ^ 1u, ab))) break;
+        mbar_arrive_expect_tx(&s.vfull, BOX);
+        tma_load_5d(s.vbuf, tmV, &s.vfull, 0, x.x0, x.y0, x.h, x.b);
+        ++vq;
+        for (int pass = 0; pass < 2 && ok; ++pass)          // taps for R, then again for the gradient
+            for (int k = 0; k < NPAIR; ++k) {
+                if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
+                const int nt = taps_in_pair(k);
+                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(nt * BOX));
+                for (int j = 0; j < nt; ++j) {
+                    const int t9 = 2 * k + j, a = t9 / 3, bb = t9 % 3;
+                    tma_load_5d(s.ring[st] + j * BOX, tmK, &s.full[st], 0, x.x0 + bb - 1, x.y0 + a - 1, x.h, x.b);
+                }
+                ++issued;
+                if (++st == S1) { st = 0; ph ^= 1u; }
+            }
+    }
+    // every copy issued has landed before the CTA may exit
+    for (uint32_t k = issued > (uint32_t)S1 ? issued - S1 : 0u; k < issued; ++k)
+        mbar_drain(&s.full[k % S1], (k / S1) & 1u, ab.limit);
+    if (vq > 0) mbar_drain(&s.vfull, (vq - 1) & 1u, ab.limit);
+}
+
+__device__ __forceinline__ void grad_mma(GradSmem& s, const GradParams& p, uint32_t tmem, const Abort& ab) {
+    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    int st = 0; uint32_t ph = 0;
+    uint32_t n = 0, part = 0;                                // tiles and parts so far
+    for (long long t = t0; t < t1;) {
+        const int u = (int)(t / p.g.tpu);
+        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
+        if (!mbar_wait(&s.w_full, part & 1u, ab)) return;
+        for (long long tt = t; tt < pe; ++tt, ++n) {
+            // R = sum_t K_t W0_t^T (A: K box, K-major; B: W0 tap image)
+            const uint32_t dr = n & 1u;
+            if (!mbar_wait(&s.dr_empty[dr], ((n >> 1) & 1u) ^ 1u, ab)) return;
+            tc_fence_after();
+            for (int k = 0; k < NPAIR; ++k) {
+                if (!mbar_wait(&s.full[st], ph, ab)) return;
+                tc_fence_after();
+                for (int j = 0; j < taps_in_pair(k); ++j) {
+                    const uint32_t sa = smem_u32(s.ring[st] + j * BOX), sb = smem_u32(s.w0img[2 * k + j]);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16_ss(tmem + kColR + dr * 64u, sdesc_sw128(sa + kk * 32, 16, 1024),
+                                    sdesc_sw128(sb + kk * 32, 16, 1024), kIdescRow, (k | j | kk) ? 1u : 0u);
+                }
+                mma_commit(&s.empty[st]);
+                if (++st == S1) { st = 0; ph ^= 1u; }
+            }
+            mma_commit(&s.dr_full[dr]);
+            if (tt + 1 == pe) mma_commit(&s.w_empty);        // the part's last reads of the W0 images
+            // G^T[pair k] += [K_2k | K_2k+1]^T (r_hi + r_lo)  (A MN-major, M = 128; B = r, MN-major)
+            if (!mbar_wait(&s.r_full, n & 1u, ab)) return;
+            const bool first = (tt == t);
+            if (first && !mbar_wait(&s.g_empty, (part & 1u) ^ 1u, ab)) return;
+            tc_fence_after();
+            const uint32_t shi = smem_u32(s.rhi), slo = smem_u32(s.rlo);
+            for (int k = 0; k < NPAIR; ++k) {
+                if (!mbar_wait(&s.full[st], ph, ab)) return;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(s.ring[st]);
+                const uint32_t dg = tmem + kColG + (uint32_t)k * 64u;
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(sa + kk * 2048, BOX, 1024);
+                    mma_bf16_ss(dg, ad, sdesc_sw128(shi + kk * 2048, BOX, 1024), kIdescCol, (first && kk == 0) ? 0u : 1u);
+                    mma_bf16_ss(dg, ad, sdesc_sw128(slo + kk * 2048, BOX, 1024), kIdescCol, 1u);
+                }
+                mma_commit(&s.empty[st]);
+                if (++st == S1) { st = 0; ph ^= 1u; }
+            }
+            mma_commit(&s.r_empty);
+        }
+        mma_commit(&s.g_full);
+        ++part;
+        t = pe;
+    }
+}
+
+__device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, uint32_t tmem, const Abort& ab) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                              // accumulator row = tile position
+    const int tid = threadIdx.x - 64;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    uint32_t n = 0, part = 0;
+    bool failed = false;
+    for (long long t = t0; t < t1 && !failed;) {
+        const int u = (int)(t / p.g.tpu);
+        const int h = u % p.g.heads;
+        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
+        // the head's W0 as nine bf16 operand images (row c, K = c'), once the previous part's R MMAs
+        // are done reading them
+        bool ok = mbar_wait(&s.w_empty, (part & 1u) ^ 1u, ab);
+        if (named_bar_or(1, 128, !ok)) break;
+        {
+            const int c = tid >> 1, cp0 = (tid & 1) * 32;
+            const float* w = p.W0 + (((size_t)h * D + c) * D + cp0) * TAPS;
+            for (int t9 = 0; t9 < TAPS; ++t9) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = __ldg(w + (size_t)(8 * j + e) * TAPS + t9);
+                    *reinterpret_cast<uint4*>(s.w0img[t9] + sw_off(c, cp0 / 8 + j)) = pack8(v);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0) mbar_arrive(&s.w_full);
+        for (long long tt = t; tt < pe; ++tt, ++n) {
+            const TileXY x = tile_xy(p.g, tt);
+            const uint32_t dr = n & 1u;
+            ok = mbar_wait(&s.dr_full[dr], (n >> 1) & 1u, ab) && mbar_wait(&s.vfull, n & 1u, ab);
+            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+            __syncwarp();
+            tc_fence_after();
+            float v[4][16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColR + dr * 64u + (uint32_t)(j * 16) + lane_off, v[j]);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&s.dr_empty[dr]);
+            // r = R - V; positions outside the grid contribute nothing
+            const bool inside = (x.y0 + r / TC) < p.g.H && (x.x0 + r % TC) < p.g.W;
+            float res[64];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 w = *reinterpret_cast<const uint4*>(s.vbuf + sw_off(r, j));
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 8 * j + 2 * e;
+                    res[c] = inside ? v[c / 16][c % 16] - bf16lo_to_f32(ww[e]) : 0.f;
+                    res[c + 1] = inside ? v[(c + 1) / 16][(c + 1) % 16] - bf16hi_to_f32(ww[e]) : 0.f;
+                }
+            }
+            mbar_arrive(&s.vempty);
+            ok = mbar_wait(&s.r_empty, (n & 1u) ^ 1u, ab);   // the previous tile's MMAs read r
+            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float hi[8], lo[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    hi[e] = __bfloat162float(__float2bfloat16_rn(res[8 * j + e]));
+                    lo[e] = res[8 * j + e] - hi[e];
+                }
+                *reinterpret_cast<uint4*>(s.rhi + sw_off(r, j)) = pack8(hi);
+                *reinterpret_cast<uint4*>(s.rlo + sw_off(r, j)) = pack8(lo);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (tid == 0) mbar_arrive(&s.r_full);
+        }
+        if (failed) break;
+        // the part's gradient: accumulator k, row r is channel c' = r % 64 of tap 2k + r / 64
+        ok = mbar_wait(&s.g_full, part & 1u, ab);
+        if (named_bar_or(1, 128, !ok)) break;
+        __syncwarp();
+        tc_fence_after();
+        float* slot = p.slots + (size_t)(blockIdx.x + u) * kSlotFloats;
+        for (int k = 0; k < NPAIR; ++k) {
+            float g[4][16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColG + (uint32_t)(k * 64 + j * 16) + lane_off, g[j]);
+            tmem_ld_wait();
+            const int t9 = 2 * k + r / D;
+            if (t9 < TAPS) {
+                float4* dst = reinterpret_cast<float4*>(slot + ((size_t)t9 * D + (r % D)) * D);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) dst[j] = make_float4(g[j / 4][(j % 4) * 4], g[j / 4][(j % 4) * 4 + 1],
+                                                                  g[j / 4][(j % 4) * 4 + 2], g[j / 4][(j % 4) * 4 + 3]);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&s.g_empty);
+        ++part;
+        t = pe;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+conv3_grad(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const GradParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    GradSmem& s = *reinterpret_cast<GradSmem*>(align1024(smem_raw));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
+    if (threadIdx.x == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < S1; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        mbar_init(&s.vfull, 1); mbar_init(&s.vempty, 128);
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.dr_full[i], 1); mbar_init(&s.dr_empty[i], 128); }
+        mbar_init(&s.r_full, 1); mbar_init(&s.r_empty, 1);
+        mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
+        mbar_init(&s.g_full, 1); mbar_init(&s.g_empty, 128);
+        mbar_init(&s.drain_bar, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+    }
+    if (warp == 1) { tmem_alloc(&s.tmem_base, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch_dependents();                                 // the merge kernel may be scheduled
+    const uint32_t tmem = s.tmem_base;
+    if (warp == 0) {
+        if (lane == 0) grad_producer(s, p, &tmK, &tmV, ab);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            grad_mma(s, p, tmem, ab);
+            mma_commit(&s.drain_bar);                        // every MMA issued has completed
+            mbar_drain(&s.drain_bar, 0u, ab.limit);
+        }
+        __syncwarp();
+    } else {
+        grad_epilogue(s, p, tmem, ab);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// conv3_merge: one CTA per (unit, tap)
+// ------------------------------------------------------------------------------------------------
+struct MergeParams {
+    Geo g;
+    int G;                                   // CTAs of conv3_grad
+    float eta;
+    const float* W0;                         // [heads][64][64][9]
+    const float* slots;
+    float* W1_out;                           // nullable [units][64][64][9]
+    uint8_t* w1img;                          // [units][9][kWImg]
+};
+
+__global__ void __launch_bounds__(256)
+conv3_merge(const MergeParams p) {
+    const int u = blockIdx.x / TAPS, t9 = blockIdx.x % TAPS, h = u % p.g.heads;
+    pdl_launch_dependents();
+    pdl_wait_primary();                                      // every gradient slot is written
+    const int cf = part_cta(p.g.T, p.G, (long long)u * p.g.tpu);
+    const int cl = part_cta(p.g.T, p.G, (long long)(u + 1) * p.g.tpu - 1);
+    uint8_t* img = p.w1img + ((size_t)u * TAPS + t9) * kWImg;
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+        const int cp = e / D, c = e % D;                     // slot element G^T[t9][cp][c]
+        float acc = 0.f;
+        for (int cta = cf; cta <= cl; ++cta) acc += __ldcg(p.slots + (size_t)(cta + u) * kSlotFloats + (size_t)t9 * D * D + e);
+        const size_t wi = (((size_t)h * D + c) * D + cp) * TAPS + t9;
+        const float w1 = __ldg(p.W0 + wi) - p.g.eta_scale * acc;
+        if (p.W1_out) p.W1_out[(((size_t)u * D + c) * D + cp) * TAPS + t9] = w1;
+        *reinterpret_cast<__nv_bfloat16*>(img + sw_off(c, cp / 8) + (cp % 8) * 2) = __float2bfloat16_rn(w1);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// conv3_readout
+// ------------------------------------------------------------------------------------------------
+struct ReadParams {
+    Geo g;
+    int G;                                   // CTAs of this kernel
+    const uint8_t* w1img;                    // [units][9][kWImg]
+    uint32_t* err;
+    unsigned long long wait_ns;
+};
+
+struct ReadSmem {
+    uint8_t ring[S3][PAIR];
+    uint8_t w1img[TAPS][kWImg];
+    uint8_t zbuf[2][BOX];
+    uint64_t full[S3], empty[S3];
+    uint64_t w_full, w_empty;
+    uint64_t dz_full[2], dz_empty[2];
+    uint64_t drain_bar;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ void read_producer(ReadSmem& s, const ReadParams& p, const CUtensorMap* tmQ,
+                                              const Abort& ab) {
+    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    uint32_t issued = 0, parts = 0;
+    int st = 0; uint32_t ph = 0;
+    bool ok = true, waited = false;
+    for (long long t = t0; t < t1 && ok;) {
+        const int u = (int)(t / p.g.tpu);
+        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
+        // W1 of the unit (written by the merge kernel): one bulk copy of its nine tap images
+        if (!waited) { pdl_wait_primary(); waited = true; }
+        if (!(ok = mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab))) break;
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
+        bulk_g2s(s.w1img, p.w1img + (size_t)u * TAPS * kWImg, TAPS * kWImg, &s.w_full);
+        ++parts;
+        for (long long tt = t; tt < pe && ok; ++tt) {
+            const TileXY x = tile_xy(p.g, tt);
+            for (int k = 0; k < NPAIR; ++k) {
+                if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
+                const int nt = taps_in_pair(k);
+                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(nt * BOX));
+                for (int j = 0; j < nt; ++j) {
+                    const int t9 = 2 * k + j, a = t9 / 3, bb = t9 % 3;
+                    tma_load_5d(s.ring[st] + j * BOX, tmQ, &s.full[st], 0, x.x0 + bb - 1, x.y0 + a - 1, x.h, x.b);
+                }
+                ++issued;
+                if (++st == S3) { st = 0; ph ^= 1u; }
+            }
+        }
+        t = pe;
+    }
+    for (uint32_t k = issued > (uint32_t)S3 ? issued - S3 : 0u; k < issued; ++k)
+        mbar_drain(&s.full[k % S3], (k / S3) & 1u, ab.limit);
+    if (parts > 0) mbar_drain(&s.w_full, (parts - 1) & 1u, ab.limit);
+}
+
+__device__ __forceinline__ void read_mma(ReadSmem& s, const ReadParams& p, uint32_t tmem, const Abort& ab) {
+    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    int st = 0; uint32_t ph = 0;
+    uint32_t n = 0, part = 0;
+    for (long long t = t0; t < t1;) {
+        const int u = (int)(t / p.g.tpu);
+        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
+        if (!mbar_wait(&s.w_full, part & 1u, ab)) return;
+        for (long long tt = t; tt < pe; ++tt, ++n) {
+            const uint32_t dz = n & 1u;
+            if (!mbar_wait(&s.dz_empty[dz], ((n >> 1) & 1u) ^ 1u, ab)) return;
+            tc_fence_after();
+            for (int k = 0; k < NPAIR; ++k) {
+                if (!mbar_wait(&s.full[st], ph, ab)) return;
+                tc_fence_after();
+                for (int j = 0; j < taps_in_pair(k); ++j) {
+                    const uint32_t sa = smem_u32(s.ring[st] + j * BOX), sb = smem_u32(s.w1img[2 * k + j]);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16_ss(tmem + dz * 64u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024),
+                                    kIdescRow, (k | j | kk) ? 1u : 0u);
+                }
+                mma_commit(&s.empty[st]);
+                if (++st == S3) { st = 0; ph ^= 1u; }
+            }
+            mma_commit(&s.dz_full[dz]);
+        }
+        mma_commit(&s.w_empty);
+        ++part;
+        t = pe;
+    }
+}
+
+__device__ __forceinline__ void read_epilogue(ReadSmem& s, const ReadParams& p, uint32_t tmem, const CUtensorMap* tmZ,
+                                              const Abort& ab) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int tid = threadIdx.x - 64;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    uint32_t n = 0;
+    for (long long t = t0; t < t1; ++t, ++n) {
+        const TileXY x = tile_xy(p.g, t);
+        const uint32_t dz = n & 1u;
+        const bool ok = mbar_wait(&s.dz_full[dz], (n >> 1) & 1u, ab);
+        if (tid == 0 && n >= 2) bulk_wait_read<1>();          // staging buffer dz is free again
+        if (named_bar_or(1, 128, !ok)) break;
+        __syncwarp();
+        tc_fence_after();
+        float v[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld16(tmem + dz * 64u + (uint32_t)(j * 16) + lane_off, v[j]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s.dz_empty[dz]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(s.zbuf[dz] + sw_off(r, j)) = pack8(&v[j / 2][(j % 2) * 8]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0) {
+            asm volatile("cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(tmZ),
+                         "r"(smem_u32(s.zbuf[dz])), "r"(0), "r"(x.x0), "r"(x.y0), "r"(x.h), "r"(x.b)
+                         : "memory");
+            bulk_commit();
+        }
+    }
+    if (tid == 0) bulk_wait<0>();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+conv3_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmZ, const ReadParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    ReadSmem& s = *reinterpret_cast<ReadSmem*>(align1024(smem_raw));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
+    if (threadIdx.x == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < S3; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.dz_full[i], 1); mbar_init(&s.dz_empty[i], 128); }
+        mbar_init(&s.drain_bar, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
+    }
+    if (warp == 1) { tmem_alloc(&s.tmem_base, 128); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    if (warp == 0) {
+        if (lane == 0) read_producer(s, p, &tmQ, ab);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            read_mma(s, p, tmem, ab);
+            mma_commit(&s.drain_bar);
+            mbar_drain(&s.drain_bar, 0u, ab.limit);
+        }
+        __syncwarp();
+    } else {
+        read_epilogue(s, p, tmem, &tmZ, ab);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------------
+struct WsLayout {
+    size_t slots, w1img, total;
+};
+static WsLayout ws_layout(long long units) {
+    WsLayout L;
+    L.slots = kWsHeader;
+    L.w1img = align_up(L.slots + (size_t)(kMaxGrid + units) * kSlotFloats * sizeof(float), 1024);
+    L.total = L.w1img + (size_t)units * TAPS * kWImg;
+    return L;
+}
+
+static Geo make_geo(const Call& c) {
+    Geo g;
+    g.heads = c.heads;
+    g.H = c.H;
+    g.W = c.W;
+    g.tiles_x = (c.W + TC - 1) / TC;
+    g.tpu = g.tiles_x * ((c.H + TR - 1) / TR);
+    g.T = (long long)c.batch * c.heads * g.tpu;
+    g.eta_scale = c.eta * (2.0f / (float)c.N);
+    return g;
+}
+
+}  // namespace c3
+
+size_t conv3x3_ws_bytes(const ttt_shape& s) { return c3::ws_layout((long long)s.batch * s.heads).total; }
+
+ttt_status launch_conv3x3(const Call& c) {
+    using namespace c3;
+    if (c.dtype != TTT_BF16 || c.loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
+    const long long units = (long long)c.batch * c.heads;
+    const WsLayout L = ws_layout(units);
+    if (c.ws_bytes < L.total) return TTT_ERR_WORKSPACE;
+    const Geo g = make_geo(c);
+    if (g.T > (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+    CUtensorMap tmK, tmV, tmQ, tmZ;
+    if (!make_tmap_grid_sw128(&tmK, c.K, c, TC, TR) || !make_tmap_grid_sw128(&tmV, c.V, c, TC, TR) ||
+        !make_tmap_grid_sw128(&tmQ, c.Q, c, TC, TR) || !make_tmap_grid_sw128(&tmZ, c.Z, c, TC, TR))
+        return TTT_ERR_INVALID_ARG;
+    const int G1 = (int)std::max<long long>(1, std::min<long long>(std::min(c.num_sms, kMaxGrid), g.T));
+    const int G3 = (int)std::max<long long>(1, std::min<long long>(c.num_sms, g.T));
+    uint32_t* err = reinterpret_cast<uint32_t*>(c.ws);
+
+    GradParams gp{};
+    gp.g = g;
+    gp.G = G1;
+    gp.W0 = c.W0;
+    gp.slots = reinterpret_cast<float*>(c.ws + L.slots);
+    gp.err = err;
+    gp.wait_ns = c.wait_ns;
+    const size_t sm1 = sizeof(GradSmem) + 1024, sm3 = sizeof(ReadSmem) + 1024;
+    if (sm1 > 227 * 1024 || sm3 > 227 * 1024) return TTT_ERR_UNSUPPORTED;
+    cudaFuncSetAttribute(conv3_grad, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+    cudaFuncSetAttribute(conv3_readout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3);
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)G1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sm1;
+    cfg.stream = c.stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = c.overlap_previous ? 1 : 0;
+    ttt_status st = check_launch(cudaLaunchKernelEx(&cfg, conv3_grad, tmK, tmV, gp));
+    if (st != TTT_OK) return st;
+
+    MergeParams mp{};
+    mp.g = g;
+    mp.G = G1;
+    mp.eta = c.eta;
+    mp.W0 = c.W0;
+    mp.slots = gp.slots;
+    mp.W1_out = c.W1_out;
+    mp.w1img = c.ws + L.w1img;
+    cfg.gridDim = dim3((unsigned)(units * TAPS));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.numAttrs = 1;
+    st = check_launch(cudaLaunchKernelEx(&cfg, conv3_merge, mp));
+    if (st != TTT_OK) return st;
+
+    ReadParams rp{};
+    rp.g = g;
+    rp.G = G3;
+    rp.w1img = mp.w1img;
+    rp.err = err;
+    rp.wait_ns = c.wait_ns;
+    cfg.gridDim = dim3((unsigned)G3);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sm3;
+    return check_launch(cudaLaunchKernelEx(&cfg, conv3_readout, tmQ, tmZ, rp));
+}
+
+}  // namespace ttt

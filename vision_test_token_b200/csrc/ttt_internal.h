@@ -51,6 +51,9 @@ bool make_tmap_tokens(CUtensorMap* m, const void* base, const Call& c, int box_r
 // Rank-5 tensor map over [batch][heads][H][W][64] (the token grid), no swizzle, zero fill out of bounds,
 // box = 64 channels x box_cols x box_rows of one unit.  Element type from c.dtype.
 bool make_tmap_grid(CUtensorMap* m, const void* base, const Call& c, int box_cols, int box_rows);
+// As make_tmap_grid, bf16 with 128-byte swizzle (a box of 64 channels is one 128-byte swizzled row
+// per position, the layout of a K-major tensor-core operand).
+bool make_tmap_grid_sw128(CUtensorMap* m, const void* base, const Call& c, int box_cols, int box_rows);
 // Rank-2 bf16 tensor map over a contiguous [rows][cols] matrix with a cols x box_rows box (cols*2 = 128).
 bool make_tmap_matrix(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);
 
@@ -64,6 +67,10 @@ size_t dwconv_ws_bytes(const ttt_shape& s);
 // Bytes at the start of a conv workspace that must be zero before a call (every call leaves them zero).
 size_t dwconv_ws_control_bytes(const ttt_shape& s);
 ttt_status launch_dwconv(const Call& c);
+
+// Full 3x3 conv head (bf16, L2 loss).
+size_t conv3x3_ws_bytes(const ttt_shape& s);
+ttt_status launch_conv3x3(const Call& c);
 
 size_t mlp_ws_bytes(const ttt_shape& s);
 ttt_status launch_mlp(const Call& c);

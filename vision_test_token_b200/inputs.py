@@ -7,6 +7,7 @@ Recipe (one torch CPU generator, ``manual_seed(seed)``, float32 draws in this or
   Q, K, V  : [B][heads][N][d] standard normal; every q and k row (length d) is then divided by its
              L2 norm (keys and queries are L2-normalised rows, values stay N(0, 1));
   weights  : linear W0 [heads_lin][d][d] ~ N(0, 1/d); conv W0 [heads_conv][d][3][3] ~ N(0, 1/9);
+             full 3x3 conv W0 [heads][d][d][3][3] ~ N(0, 1/(9d)) (its fan-in is 9d);
              MLP Wa [heads][4d][d] ~ N(0, 1/d), Wb [heads][d][4d] ~ N(0, 1/(4d));
   dZ       : (kind "backward", the upstream gradient of Z) [B][heads][N][d] standard normal, drawn
              after the weights;
@@ -27,6 +28,8 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
                    consecutive batches of 16 tokens (causal prefix inside a batch), eta 0.25
   bwd6084_bf16     backward pass of the linear heads of mixed6084_bf16: B 8, 5 heads, 78 x 78,
                    bf16, eta 0.5
+  conv3x3_6084_bf16  the full 3x3 conv head (the press article's other conv variant) in place of the
+                   depthwise head of mixed6084_bf16: B 8, 1 head, 78 x 78, bf16, eta 0.5
 """
 from dataclasses import dataclass
 import math
@@ -44,7 +47,7 @@ class Workload:
     dtype: str            # "fp32" or "bf16"
     eta: float
     kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp", "minibatch" (linear),
-                          # "backward" (linear)
+                          # "backward" (linear), "conv3x3" (full 3x3 conv heads)
     conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
     d: int = 64
     hidden_ratio: int = 4
@@ -75,6 +78,7 @@ WORKLOADS = {
                                    loss="dot"),
     "mb16_6084_bf16": Workload("mb16_6084_bf16", 8, 6, 78, 78, "bf16", 0.25, "minibatch", mb_tokens=16),
     "bwd6084_bf16": Workload("bwd6084_bf16", 8, 5, 78, 78, "bf16", 0.5, "backward"),
+    "conv3x3_6084_bf16": Workload("conv3x3_6084_bf16", 8, 1, 78, 78, "bf16", 0.5, "conv3x3"),
 }
 
 TORCH_DTYPE = {"fp32": torch.float32, "bf16": torch.bfloat16}
@@ -98,6 +102,8 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
             out["W0_lin"] = torch.randn((w.lin_heads, w.d, w.d), generator=g) / math.sqrt(w.d)
         if w.conv_heads:
             out["W0_conv"] = torch.randn((w.conv_heads, w.d, 3, 3), generator=g) / 3.0
+    elif w.kind == "conv3x3":
+        out["W0_c3"] = torch.randn((w.heads, w.d, w.d, 3, 3), generator=g) / math.sqrt(9 * w.d)
     elif w.kind == "mlp":
         hid = w.hidden_ratio * w.d
         out["Wa"] = torch.randn((w.heads, hid, w.d), generator=g) / math.sqrt(w.d)

@@ -164,6 +164,21 @@ def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=
     return Z
 
 
+def forward_conv3x3(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0):
+    """Full 3x3 conv inner model (every output channel reads every input channel).  W0:
+    [heads][d][d][3][3] fp32 CUDA tensor; bf16 Q, K, V.  Returns Z."""
+    shape = _shape_of(Q, H, W, max_sms=max_sms)
+    Z = _out_like(Q, Z)
+    _same_layout(Q, K, V, Z)
+    W0 = W0.contiguous()
+    if ws is None:
+        ws = workspace(capi.TTT_HEAD_CONV3X3, shape, Q.device)
+    st = capi.ttt_forward_conv3x3(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(Z), float(eta), shape, *_ws_args(ws),
+                                  _ptr(W1_out), _stream_handle(stream))
+    _check(st, "ttt_forward_conv3x3")
+    return Z
+
+
 def forward_mlp(Q, K, V, Wa, Wb, eta, H, W, Z=None, Wa_out=None, Wb_out=None, ws=None, stream=None, max_sms=0,
                 loss="l2"):
     """One-hidden-layer GELU MLP inner model.  Wa: [heads][hidden][d], Wb: [heads][d][hidden].
