@@ -16,8 +16,9 @@ Functions and the definitions they follow (page titles and sections; see ``ttt_o
   linear_minibatch(...)
                     the linear head trained by mini-batch gradient descent over consecutive token
                     batches (prefix: causal prefix sums inside a batch; epoch: one mean step per batch)
-  linear_backward(...)
-                    the chain rule through the full-batch linear step: dQ, dK, dV, dW0, deta
+  linear_backward(...), dwconv_backward(...)
+                    the chain rule through the full-batch linear / depthwise-conv step: dQ, dK, dV,
+                    dW0, deta
   gelu_tanh(u), gelu_tanh_deriv(u)
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py (closed forms,
@@ -49,11 +50,12 @@ def _load():
         lib.oracle_dwconv.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv_dot.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_conv3x3.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
+        lib.oracle_dwconv_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, dp, dp, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
         for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_linear_minibatch,
                   lib.oracle_linear_backward,
                   lib.oracle_dwconv,
-                  lib.oracle_dwconv_dot, lib.oracle_conv3x3, lib.oracle_mlp):
+                  lib.oracle_dwconv_dot, lib.oracle_conv3x3, lib.oracle_dwconv_backward, lib.oracle_mlp):
             f.restype = ctypes.c_int
         lib.oracle_gelu_tanh.argtypes = [d]
         lib.oracle_gelu_tanh.restype = d
@@ -143,6 +145,23 @@ def linear_backward(Q, K, V, W0, eta, dZ, threads=None):
     _check(_load().oracle_linear_backward(B, H, N, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(dZ), _p(dQ),
                                           _p(dK), _p(dV), _p(dW0), _p(deta), threads or default_threads()),
            "linear_backward")
+    return dQ, dK, dV, dW0, float(deta[0])
+
+
+def dwconv_backward(Q, K, V, W0, eta, dZ, Hg, Wg, threads=None):
+    """Backward pass of the depthwise-conv head (L2 loss) for the upstream gradient dZ.
+    Returns (dQ, dK, dV [B][h][N][d], dW0 [h][d][3][3] summed over images, deta: a float summed over
+    every unit) in float64."""
+    Q, K, V, W0, dZ = _f64(Q), _f64(K), _f64(V), _f64(W0), _f64(dZ)
+    B, H, N, d = Q.shape
+    assert N == Hg * Wg and K.shape == Q.shape and V.shape == Q.shape and dZ.shape == Q.shape
+    assert W0.shape == (H, d, 3, 3)
+    dQ, dK, dV = np.empty_like(Q), np.empty_like(Q), np.empty_like(Q)
+    dW0 = np.empty((H, d, 3, 3))
+    deta = np.zeros(1)
+    _check(_load().oracle_dwconv_backward(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(dZ), _p(dQ),
+                                          _p(dK), _p(dV), _p(dW0), _p(deta), threads or default_threads()),
+           "dwconv_backward")
     return dQ, dK, dV, dW0, float(deta[0])
 
 

@@ -37,8 +37,8 @@
  *       from; inside a batch the notes' prefix sum carries no 1/b, while the press article's
  *       B = N/k ablation takes one step of each batch's mean loss and reads out with the final
  *       weights;
- *     - the backward pass differentiates the full-batch linear step; W0 and eta are shared by
- *       every unit, so their gradients are summed (over images, over units).
+ *     - the backward pass differentiates the full-batch linear step and the depthwise-conv step;
+ *       W0 and eta are shared by every unit, so their gradients are summed (over images, over units).
  *
  * Memory layout of every array (contiguous, row-major, fp64):
  *   Q, K, V, Z : [B][heads][N][d]     (token n, feature c at ((b*heads + h)*N + n)*d + c)
@@ -571,6 +571,114 @@ int oracle_conv3x3(int B, int heads, int Hg, int Wg, int d, const double* Q, con
             status = s;
         }
     }
+    return status;
+}
+
+/* Backward pass of the depthwise-conv head (press article, Observation 1: the outer gradient    */
+/* flows through the inner step).  Per channel c, with taps t = (a, b), shifts s_t = (a-1, b-1),  */
+/* K[c, p + s_t] zero outside the grid, and the forward                                          */
+/*     r_p = sum_t W0_t K_{p+s_t} - V_p,   g_t = (2/N) sum_p r_p K_{p+s_t},   W1 = W0 - eta g,    */
+/*     Z_p = sum_t W1_t Q_{p+s_t},                                                               */
+/* the chain rule for the upstream gradient dZ gives, with dg = -eta dW1:                        */
+/*     dW1_t = sum_p dZ_p Q_{p+s_t},          dQ_q = sum_t W1_t dZ_{q-s_t},                      */
+/*     dr_p = (2/N) sum_t dg_t K_{p+s_t},     dV_p = -dr_p,                                      */
+/*     dK_q = (2/N) sum_t dg_t r_{q-s_t} + sum_t W0_t dr_{q-s_t},                                 */
+/*     dW0_t = dW1_t + sum_p dr_p K_{p+s_t},  deta = -sum_t dW1_t g_t                            */
+/* (positions q - s_t outside the grid contribute nothing).  As for the linear head, dW0 is      */
+/* summed over the images of each head and deta over every unit, in index order.                 */
+static int dwconv_backward_unit(int Hg, int Wg, int d, const double* Q, const double* K, const double* V,
+                                const double* W0, double eta, const double* dZ, double* dQ, double* dK,
+                                double* dV, double* dW0, double* deta)
+{
+    const int N = Hg * Wg;
+    double* r = (double*)malloc((size_t)N * sizeof(double));
+    double* dr = (double*)malloc((size_t)N * sizeof(double));
+    if (!r || !dr) { free(r); free(dr); return ORACLE_ERR_NOMEM; }
+    const double scale = 2.0 / (double)N;
+    double de = 0.0;
+    for (int c = 0; c < d; ++c) {
+        const double* w0 = W0 + (size_t)c * 9;
+        double g[9] = {0}, dW1[9] = {0}, w1[9], dg[9];
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double f = 0.0;
+                for (int t = 0; t < 9; ++t) f += w0[t] * grid_at(K, Hg, Wg, d, c, y + t / 3 - 1, x + t % 3 - 1);
+                r[y * Wg + x] = f - V[((size_t)y * Wg + x) * d + c];
+            }
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x)
+                for (int t = 0; t < 9; ++t) {
+                    g[t] += r[y * Wg + x] * grid_at(K, Hg, Wg, d, c, y + t / 3 - 1, x + t % 3 - 1);
+                    dW1[t] += dZ[((size_t)y * Wg + x) * d + c] * grid_at(Q, Hg, Wg, d, c, y + t / 3 - 1, x + t % 3 - 1);
+                }
+        for (int t = 0; t < 9; ++t) {
+            g[t] *= scale;
+            w1[t] = w0[t] - eta * g[t];
+            dg[t] = -eta * dW1[t];
+            de += -dW1[t] * g[t];
+        }
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                double a = 0.0;
+                for (int t = 0; t < 9; ++t) a += dg[t] * grid_at(K, Hg, Wg, d, c, y + t / 3 - 1, x + t % 3 - 1);
+                dr[y * Wg + x] = scale * a;
+            }
+        double dw0[9];
+        for (int t = 0; t < 9; ++t) dw0[t] = dW1[t];
+        for (int y = 0; y < Hg; ++y)
+            for (int x = 0; x < Wg; ++x) {
+                const size_t o = ((size_t)y * Wg + x) * d + c;
+                double aq = 0.0, ak = 0.0;
+                for (int t = 0; t < 9; ++t) {
+                    const int yy = y - (t / 3 - 1), xx = x - (t % 3 - 1);   /* q - s_t */
+                    if (yy < 0 || yy >= Hg || xx < 0 || xx >= Wg) continue;
+                    aq += w1[t] * dZ[((size_t)yy * Wg + xx) * d + c];
+                    ak += scale * dg[t] * r[yy * Wg + xx] + w0[t] * dr[yy * Wg + xx];
+                }
+                dQ[o] = aq;
+                dK[o] = ak;
+                dV[o] = -dr[y * Wg + x];
+                for (int t = 0; t < 9; ++t) dw0[t] += dr[y * Wg + x] * grid_at(K, Hg, Wg, d, c, y + t / 3 - 1, x + t % 3 - 1);
+            }
+        for (int t = 0; t < 9; ++t) dW0[(size_t)c * 9 + t] += dw0[t];
+    }
+    *deta += de;
+    free(r);
+    free(dr);
+    return ORACLE_OK;
+}
+
+/* dW0: [heads][d][3][3] (summed over images), deta: one value (summed over units), as for the
+ * linear head's backward. */
+int oracle_dwconv_backward(int B, int heads, int Hg, int Wg, int d, const double* Q, const double* K,
+                           const double* V, const double* W0, double eta, const double* dZ, double* dQ,
+                           double* dK, double* dV, double* dW0, double* deta, int nthreads)
+{
+    if (B < 0 || heads < 0 || Hg < 1 || Wg < 1 || d < 1 || !Q || !K || !V || !W0 || !dZ || !dQ || !dK || !dV ||
+        !dW0 || !deta)
+        return ORACLE_ERR_ARG;
+    const size_t N = (size_t)Hg * Wg;
+    double* deta_h = (double*)calloc(heads > 0 ? (size_t)heads : 1, sizeof(double));
+    if (!deta_h) return ORACLE_ERR_NOMEM;
+    memset(dW0, 0, (size_t)heads * d * 9 * sizeof(double));
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int h = 0; h < heads; ++h) {
+        for (int b = 0; b < B; ++b) {
+            const size_t off = ((size_t)b * heads + h) * N * d;
+            int st = dwconv_backward_unit(Hg, Wg, d, Q + off, K + off, V + off, W0 + (size_t)h * d * 9, eta, dZ + off,
+                                          dQ + off, dK + off, dV + off, dW0 + (size_t)h * d * 9, &deta_h[h]);
+            if (st != ORACLE_OK) {
+#pragma omp atomic write
+                status = st;
+            }
+        }
+    }
+    double total = 0.0;
+    for (int h = 0; h < heads; ++h) total += deta_h[h];
+    *deta = total;
+    free(deta_h);
     return status;
 }
 

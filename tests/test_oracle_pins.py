@@ -439,6 +439,135 @@ def test_planted_mistake_fails_the_backward_pin():
 
 
 # ------------------------------------------------------------------------------------------------
+# backward pass of the depthwise-conv head
+# ------------------------------------------------------------------------------------------------
+def _cbwd_case(B=2, H=2, Hg=4, Wg=5, d=3, seed=0):
+    r = np.random.default_rng(200 + seed)
+    N = Hg * Wg
+    Q, K, V, dZ = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    W0 = r.standard_normal((H, d, 3, 3)) / 3.0
+    return Q, K, V, W0, dZ
+
+
+def _cfwd_loss(Q, K, V, W0, eta, dZ, Hg, Wg):
+    """L = sum dZ * Z with Z from the pinned forward oracle of the depthwise-conv head."""
+    Z, _ = oracle.dwconv(Q, K, V, W0, eta, Hg, Wg)
+    return float(np.sum(dZ * Z))
+
+
+@pytest.mark.parametrize("Hg,Wg", [(4, 5), (1, 6), (3, 1)])
+def test_dwconv_backward_matches_central_differences_of_the_forward_oracle(Hg, Wg):
+    Q, K, V, W0, dZ = _cbwd_case(Hg=Hg, Wg=Wg)
+    eta, h = 0.7, 1e-5
+    dQ, dK, dV, dW0, deta = oracle.dwconv_backward(Q, K, V, W0, eta, dZ, Hg, Wg)
+    grads = {"Q": dQ, "K": dK, "V": dV, "W0": dW0}
+    args = {"Q": Q, "K": K, "V": V, "W0": W0}
+    r = np.random.default_rng(7)
+    for name, g in grads.items():
+        for _ in range(8):
+            idx = tuple(int(r.integers(0, n)) for n in args[name].shape)
+            plus = {k: v.copy() for k, v in args.items()}
+            minus = {k: v.copy() for k, v in args.items()}
+            plus[name][idx] += h
+            minus[name][idx] -= h
+            fd = (_cfwd_loss(plus["Q"], plus["K"], plus["V"], plus["W0"], eta, dZ, Hg, Wg) -
+                  _cfwd_loss(minus["Q"], minus["K"], minus["V"], minus["W0"], eta, dZ, Hg, Wg)) / (2 * h)
+            assert abs(g[idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, g[idx], fd)
+    fd = (_cfwd_loss(Q, K, V, W0, eta + h, dZ, Hg, Wg) - _cfwd_loss(Q, K, V, W0, eta - h, dZ, Hg, Wg)) / (2 * h)
+    assert abs(deta - fd) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_dwconv_backward_matches_torch_autograd():
+    Hg, Wg = 6, 7
+    Q, K, V, W0, dZ = _cbwd_case(B=2, H=2, Hg=Hg, Wg=Wg, d=5, seed=1)
+    eta = 0.4
+    dQ, dK, dV, dW0, deta = oracle.dwconv_backward(Q, K, V, W0, eta, dZ, Hg, Wg)
+    tQ, tK, tV, tW = (torch.tensor(a, requires_grad=True) for a in (Q, K, V, W0))
+    te = torch.tensor(eta, dtype=torch.float64, requires_grad=True)
+    B, H, N, d = Q.shape
+    tot = 0.0
+    for b in range(B):
+        for hh in range(H):
+            r = _torch_conv_f(tK[b, hh], tW[hh], Hg, Wg) - tV[b, hh]
+            Wv = tW[hh]
+            g = torch.stack([torch.stack([
+                (r * _shifted(tK[b, hh], a, bb, Hg, Wg)).sum(0) for bb in range(3)], -1) for a in range(3)], -2)
+            W1 = Wv - te * (2.0 / N) * g
+            Z = _torch_conv_f(tQ[b, hh], W1, Hg, Wg)
+            tot = tot + (Z * torch.tensor(dZ[b, hh])).sum()
+    tot.backward()
+    np.testing.assert_allclose(dQ, tQ.grad.numpy(), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(dK, tK.grad.numpy(), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(dV, tV.grad.numpy(), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(dW0, tW.grad.numpy(), atol=1e-10, rtol=0)
+    assert abs(deta - te.grad.item()) <= 1e-10 * max(1.0, abs(deta))
+
+
+def _shifted(X, a, b, Hg, Wg):
+    """X [N][d] read at grid offset (a-1, b-1) with zero padding: row p holds X[p + s]."""
+    N, d = X.shape
+    img = X.T.reshape(d, Hg, Wg)
+    pad = F.pad(img, (1, 1, 1, 1))
+    return pad[:, a:a + Hg, b:b + Wg].reshape(d, N).T
+
+
+def test_dwconv_backward_special_cases():
+    """dZ = 0 gives zero gradients; eta = 0 makes the head Z = f(Q; W0): dK = dV = 0, dQ is the
+    transposed depthwise conv of dZ (torch conv_transpose2d) and dW0 = sum dZ Q[shifted]."""
+    Hg, Wg = 5, 6
+    Q, K, V, W0, dZ = _cbwd_case(B=3, H=2, Hg=Hg, Wg=Wg, d=4, seed=2)
+    out = oracle.dwconv_backward(Q, K, V, W0, 0.9, np.zeros_like(dZ), Hg, Wg)
+    for a in out[:4]:
+        assert np.all(a == 0.0)
+    assert out[4] == 0.0
+    dQ, dK, dV, dW0, deta = oracle.dwconv_backward(Q, K, V, W0, 0.0, dZ, Hg, Wg)
+    assert np.all(dK == 0.0) and np.all(dV == 0.0)
+    d = Q.shape[3]
+    for b in range(3):
+        for h in range(2):
+            img = torch.tensor(dZ[b, h].T.reshape(1, d, Hg, Wg))
+            ref = F.conv_transpose2d(img, torch.tensor(W0[h]).reshape(d, 1, 3, 3), padding=1, groups=d)
+            np.testing.assert_allclose(dQ[b, h], ref.reshape(d, Hg * Wg).T.numpy(), atol=1e-12, rtol=0)
+    ref_w = np.zeros_like(W0)
+    for b in range(3):
+        for h in range(2):
+            for a in range(3):
+                for bb in range(3):
+                    ref_w[h, :, a, bb] += (dZ[b, h] * _shifted(torch.tensor(Q[b, h]), a, bb, Hg, Wg).numpy()).sum(0)
+    np.testing.assert_allclose(dW0, ref_w, atol=1e-12, rtol=0)
+
+
+def test_planted_mistake_fails_the_conv_backward_pin():
+    """Dropping the term of dK that flows through the gradient's own K factor ((2/N) dg r[q - s]),
+    planted in a CPU copy, disagrees with the central differences."""
+    Hg, Wg = 4, 4
+    Q, K, V, W0, dZ = _cbwd_case(B=1, H=1, Hg=Hg, Wg=Wg, d=2, seed=3)
+    eta, h = 0.7, 1e-5
+    dQ, dK, dV, _, _ = oracle.dwconv_backward(Q, K, V, W0, eta, dZ, Hg, Wg)
+    N = Hg * Wg
+    c, qy, qx = 1, 2, 1
+    Kt = torch.tensor(K[0, 0])
+    r = (_torch_conv_f(Kt, torch.tensor(W0[0]), Hg, Wg) - torch.tensor(V[0, 0])).numpy()
+    dW1 = np.array([[(dZ[0, 0][:, c] * _shifted(torch.tensor(Q[0, 0]), a, b, Hg, Wg).numpy()[:, c]).sum()
+                     for b in range(3)] for a in range(3)])
+    dg = -eta * dW1
+    term = 0.0
+    for a in range(3):
+        for b in range(3):
+            yy, xx = qy - (a - 1), qx - (b - 1)
+            if 0 <= yy < Hg and 0 <= xx < Wg:
+                term += (2.0 / N) * dg[a, b] * r[yy * Wg + xx, c]
+    idx = (0, 0, qy * Wg + qx, c)
+    bad = dK[idx] - term
+    plus, minus = K.copy(), K.copy()
+    plus[idx] += h
+    minus[idx] -= h
+    fd = (_cfwd_loss(Q, plus, V, W0, eta, dZ, Hg, Wg) - _cfwd_loss(Q, minus, V, W0, eta, dZ, Hg, Wg)) / (2 * h)
+    assert abs(dK[idx] - fd) <= 1e-6 * max(1.0, abs(fd))
+    assert abs(bad - fd) > 1e-4
+
+
+# ------------------------------------------------------------------------------------------------
 # depthwise 3x3 conv head
 # ------------------------------------------------------------------------------------------------
 def test_dwconv_gradient_exact_rational_fd():
