@@ -71,7 +71,8 @@ typedef enum {
     TTT_HEAD_DWCONV = 1,
     TTT_HEAD_MLP = 2,
     TTT_HEAD_LINEAR_BACKWARD = 3,  /* the workspace of ttt_backward_linear */
-    TTT_HEAD_CONV3X3 = 4           /* the workspace of ttt_forward_conv3x3 */
+    TTT_HEAD_CONV3X3 = 4,          /* the workspace of ttt_forward_conv3x3 */
+    TTT_HEAD_DWCONV_BACKWARD = 5   /* the workspace of ttt_backward_dwconv */
 } ttt_head_kind;
 
 /* Inner loss of the one-step training.
@@ -238,6 +239,22 @@ ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void
  * Computed in fp32 from bf16 or fp32 inputs (outputs rounded to the input dtype); deterministic.
  * s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED). */
 ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
+                               float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
+                               void* dV, float* dW0_out, float* deta_out, void* stream);
+
+/* Backward pass of the 3x3 depthwise-conv head (L2 loss; the head of ttt_forward_dwconv), the outer
+ * gradient through its inner step (press article, Observation 1).  Per channel c, taps t with shifts
+ * s_t = (a-1, b-1), dg = -eta dW1, and positions q - s_t outside the grid contributing nothing:
+ *   dW1_t = sum_p dZ_p Q_{p+s_t},          dQ_q = sum_t W1_t dZ_{q-s_t},
+ *   dr_p = (2/N) sum_t dg_t K_{p+s_t},     dV_p = -dr_p,
+ *   dK_q = (2/N) sum_t dg_t r_{q-s_t} + sum_t W0_t dr_{q-s_t}   (r = f(K;W0) - V),
+ *   dW0_t = dW1_t + sum_p dr_p K_{p+s_t},  deta = -sum_t dW1_t g_t.
+ *   Layouts, outputs and rules as ttt_backward_linear: dQ, dK, dV like Q; dW0_out optional
+ *   [heads][d][3][3] fp32 summed over the images of each head in image order; deta_out optional, summed
+ *   over every unit in index order.  ws: ttt_workspace_bytes(TTT_HEAD_DWCONV_BACKWARD, s) bytes (per-tile
+ *   partial sums and per-unit coefficients; needs no zero fill).  fp32 arithmetic from bf16 or fp32
+ *   inputs; deterministic.  s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED). */
+ttt_status ttt_backward_dwconv(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
                                float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
                                void* dV, float* dW0_out, float* deta_out, void* stream);
 

@@ -258,6 +258,7 @@ size_t ttt_workspace_bytes(int kind, const ttt_shape* s) {
         case TTT_HEAD_MLP: return mlp_ws_bytes(*s);
         case TTT_HEAD_LINEAR_BACKWARD: return linear_backward_ws_bytes(*s);
         case TTT_HEAD_CONV3X3: return conv3x3_ws_bytes(*s);
+        case TTT_HEAD_DWCONV_BACKWARD: return dwconv_backward_ws_bytes(*s);
         default: return 0;
     }
 }
@@ -333,17 +334,17 @@ ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void
     return launch_linear_minibatch(c, batch_tokens, mode);
 }
 
-ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
-                               float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
-                               void* dV, float* dW0_out, float* deta_out, void* stream) {
-    ttt_status st = check_shape(TTT_HEAD_LINEAR_BACKWARD, s);
+static ttt_status backward_common(int kind, const void* Q, const void* K, const void* V, const float* W0,
+                                  const void* dZ, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ,
+                                  void* dK, void* dV, float* dW0_out, float* deta_out, void* stream) {
+    ttt_status st = check_shape(kind, s);
     if (st != TTT_OK) return st;
     if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
     if (!dZ || !dK || !dV) return TTT_ERR_INVALID_ARG;
     Call c;
+    const size_t need = (kind == TTT_HEAD_LINEAR_BACKWARD) ? linear_backward_ws_bytes(*s) : dwconv_backward_ws_bytes(*s);
     // Q, K, V, W0, the workspace and dQ (as the output Z: apart from Q, K and V)
-    st = prepare(TTT_HEAD_LINEAR_BACKWARD, Q, K, V, W0, nullptr, dQ, eta, s, ws, ws_bytes, linear_backward_ws_bytes(*s),
-                 stream, &c);
+    st = prepare(kind, Q, K, V, W0, nullptr, dQ, eta, s, ws, ws_bytes, need, stream, &c);
     if (st != TTT_OK) return st;
     for (const void* p : {dZ, (const void*)dK, (const void*)dV}) {
         if (reinterpret_cast<uintptr_t>(p) % 16) return TTT_ERR_ALIGNMENT;
@@ -358,7 +359,22 @@ ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, cons
     if (overlaps(dQ, dK, ext) || overlaps(dQ, dV, ext) || overlaps(dK, dV, ext)) return TTT_ERR_INVALID_ARG;
     if (dW0_out && (reinterpret_cast<uintptr_t>(dW0_out) % 16 || !is_device_ptr(dW0_out))) return TTT_ERR_INVALID_ARG;
     if (deta_out && (reinterpret_cast<uintptr_t>(deta_out) % 4 || !is_device_ptr(deta_out))) return TTT_ERR_INVALID_ARG;
-    return launch_linear_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
+    if (kind == TTT_HEAD_LINEAR_BACKWARD) return launch_linear_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
+    return launch_dwconv_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
+}
+
+ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
+                               float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
+                               void* dV, float* dW0_out, float* deta_out, void* stream) {
+    return backward_common(TTT_HEAD_LINEAR_BACKWARD, Q, K, V, W0, dZ, eta, s, ws, ws_bytes, dQ, dK, dV, dW0_out,
+                           deta_out, stream);
+}
+
+ttt_status ttt_backward_dwconv(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
+                               float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
+                               void* dV, float* dW0_out, float* deta_out, void* stream) {
+    return backward_common(TTT_HEAD_DWCONV_BACKWARD, Q, K, V, W0, dZ, eta, s, ws, ws_bytes, dQ, dK, dV, dW0_out,
+                           deta_out, stream);
 }
 
 constexpr double kConvHeadWeight = 2.0;

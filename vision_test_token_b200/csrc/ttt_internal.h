@@ -81,6 +81,11 @@ size_t linear_backward_ws_control_bytes(const ttt_shape& s);
 ttt_status launch_linear_backward(const Call& c, const void* dZ, void* dQ, void* dK, void* dV, float* dW0_out,
                                   float* deta_out);
 
+// Backward pass of the depthwise-conv head.
+size_t dwconv_backward_ws_bytes(const ttt_shape& s);
+ttt_status launch_dwconv_backward(const Call& c, const void* dZ, void* dQ, void* dK, void* dV, float* dW0_out,
+                                  float* deta_out);
+
 // Mini-batch linear head (its workspace is the error word only): batch_tokens >= 1, mode
 // TTT_MB_PREFIX or TTT_MB_EPOCH.
 ttt_status launch_linear_minibatch(const Call& c, int batch_tokens, int mode);

@@ -28,6 +28,8 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
                    consecutive batches of 16 tokens (causal prefix inside a batch), eta 0.25
   bwd6084_bf16     backward pass of the linear heads of mixed6084_bf16: B 8, 5 heads, 78 x 78,
                    bf16, eta 0.5
+  bwdconv6084_bf16 backward pass of the depthwise-conv head of mixed6084_bf16: B 8, 1 head, 78 x 78,
+                   bf16, eta 0.5 (conv W0 and dZ as above)
   conv3x3_6084_bf16  the full 3x3 conv head (the press article's other conv variant) in place of the
                    depthwise head of mixed6084_bf16: B 8, 1 head, 78 x 78, bf16, eta 0.5
 """
@@ -47,7 +49,7 @@ class Workload:
     dtype: str            # "fp32" or "bf16"
     eta: float
     kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp", "minibatch" (linear),
-                          # "backward" (linear), "conv3x3" (full 3x3 conv heads)
+                          # "backward" (linear), "backward_conv" (depthwise conv), "conv3x3" (full 3x3 conv heads)
     conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
     d: int = 64
     hidden_ratio: int = 4
@@ -78,6 +80,7 @@ WORKLOADS = {
                                    loss="dot"),
     "mb16_6084_bf16": Workload("mb16_6084_bf16", 8, 6, 78, 78, "bf16", 0.25, "minibatch", mb_tokens=16),
     "bwd6084_bf16": Workload("bwd6084_bf16", 8, 5, 78, 78, "bf16", 0.5, "backward"),
+    "bwdconv6084_bf16": Workload("bwdconv6084_bf16", 8, 1, 78, 78, "bf16", 0.5, "backward_conv", conv_heads=1),
     "conv3x3_6084_bf16": Workload("conv3x3_6084_bf16", 8, 1, 78, 78, "bf16", 0.5, "conv3x3"),
 }
 
@@ -97,7 +100,7 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
     K = _unit_rows(torch.randn(shape, generator=g, dtype=torch.float32))
     V = torch.randn(shape, generator=g, dtype=torch.float32)
     out = {}
-    if w.kind in ("linear", "mixed", "minibatch", "backward"):
+    if w.kind in ("linear", "mixed", "minibatch", "backward", "backward_conv"):
         if w.lin_heads:
             out["W0_lin"] = torch.randn((w.lin_heads, w.d, w.d), generator=g) / math.sqrt(w.d)
         if w.conv_heads:
@@ -109,7 +112,7 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
         out["Wa"] = torch.randn((w.heads, hid, w.d), generator=g) / math.sqrt(w.d)
         out["Wb"] = torch.randn((w.heads, w.d, hid), generator=g) / math.sqrt(hid)
     dt = TORCH_DTYPE[w.dtype]
-    if w.kind == "backward":
+    if w.kind in ("backward", "backward_conv"):
         out["dZ"] = torch.randn(shape, generator=g, dtype=torch.float32).to(dt)
     out["Q"], out["K"], out["V"] = Q.to(dt), K.to(dt), V.to(dt)
     if device != "cpu":

@@ -150,6 +150,29 @@ def backward_linear(Q, K, V, W0, eta, H, W, dZ, out=None, ws=None, stream=None, 
     return dQ, dK, dV, dW0, deta
 
 
+def backward_dwconv(Q, K, V, W0, eta, H, W, dZ, out=None, ws=None, stream=None):
+    """Backward pass of the depthwise-conv head (L2 loss) for the upstream gradient dZ of Z.
+    Returns (dQ, dK, dV, dW0 [heads][d][3][3] fp32 summed over images, deta: a 1-element fp32 tensor
+    summed over every unit); `out` may supply those five tensors."""
+    shape = _shape_of(Q, H, W)
+    _same_layout(Q, K, V, dZ)
+    heads = Q.shape[1]
+    if out is None:
+        dQ, dK, dV = (_out_like(Q, None) for _ in range(3))
+        dW0 = torch.empty((heads, Q.shape[3], 3, 3), dtype=torch.float32, device=Q.device)
+        deta = torch.empty(1, dtype=torch.float32, device=Q.device)
+    else:
+        dQ, dK, dV, dW0, deta = out
+    _same_layout(Q, dQ, dK, dV)
+    W0 = W0.contiguous()
+    if ws is None:
+        ws = workspace(capi.TTT_HEAD_DWCONV_BACKWARD, shape, Q.device)
+    st = capi.ttt_backward_dwconv(_ptr(Q), _ptr(K), _ptr(V), _ptr(W0), _ptr(dZ), float(eta), shape, *_ws_args(ws),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dW0), _ptr(deta), _stream_handle(stream))
+    _check(st, "ttt_backward_dwconv")
+    return dQ, dK, dV, dW0, deta
+
+
 def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0, loss="l2"):
     """3x3 depthwise-conv inner model.  W0: [heads][d][3][3] fp32 CUDA tensor.  Returns Z."""
     shape = _shape_of(Q, H, W, max_sms=max_sms, loss=loss)
