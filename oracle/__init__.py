@@ -16,10 +16,10 @@ Functions and the definitions they follow (page titles and sections; see ``ttt_o
   linear_minibatch(...)
                     the linear head trained by mini-batch gradient descent over consecutive token
                     batches (prefix: causal prefix sums inside a batch; epoch: one mean step per batch)
-  linear_backward(...), dwconv_backward(...)
-                    the chain rule through the full-batch linear / depthwise-conv step: dQ, dK, dV,
-                    dW0, deta
-  gelu_tanh(u), gelu_tanh_deriv(u)
+  linear_backward(...), dwconv_backward(...), mlp_backward(...)
+                    the chain rule through the full-batch linear / depthwise-conv / MLP step: dQ, dK,
+                    dV, the weights' gradients, deta
+  gelu_tanh(u), gelu_tanh_deriv(u), gelu_tanh_deriv2(u)
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py (closed forms,
 invariants, exact finite differences, autograd and library special cases).
@@ -51,16 +51,20 @@ def _load():
         lib.oracle_dwconv_dot.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_conv3x3.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, i]
         lib.oracle_dwconv_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, d, dp, dp, dp, dp, dp, dp, i]
+        lib.oracle_mlp_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, dp, dp, dp, dp, i]
         lib.oracle_mlp.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp, i]
         for f in (lib.oracle_linear, lib.oracle_linear_gram, lib.oracle_linear_dot, lib.oracle_linear_minibatch,
                   lib.oracle_linear_backward,
                   lib.oracle_dwconv,
-                  lib.oracle_dwconv_dot, lib.oracle_conv3x3, lib.oracle_dwconv_backward, lib.oracle_mlp):
+                  lib.oracle_dwconv_dot, lib.oracle_conv3x3, lib.oracle_dwconv_backward, lib.oracle_mlp_backward,
+                  lib.oracle_mlp):
             f.restype = ctypes.c_int
         lib.oracle_gelu_tanh.argtypes = [d]
         lib.oracle_gelu_tanh.restype = d
         lib.oracle_gelu_tanh_deriv.argtypes = [d]
         lib.oracle_gelu_tanh_deriv.restype = d
+        lib.oracle_gelu_tanh_deriv2.argtypes = [d]
+        lib.oracle_gelu_tanh_deriv2.restype = d
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -201,6 +205,27 @@ def dwconv_dot(Q, K, V, W0, eta, Hg, Wg, threads=None):
     _check(_load().oracle_dwconv_dot(B, H, Hg, Wg, d, _p(Q), _p(K), _p(V), _p(W0), float(eta), _p(W1),
                                      _p(Z), threads or default_threads()), "dwconv_dot")
     return Z, W1
+
+
+def mlp_backward(Q, K, V, Wa, Wb, eta, dZ, threads=None):
+    """Backward pass of the MLP head (L2 loss) for the upstream gradient dZ.  Returns (dQ, dK, dV
+    [B][h][N][d], dWa [h][hidden][d], dWb [h][d][hidden] summed over images, deta: a float summed over
+    every unit) in float64."""
+    Q, K, V, Wa, Wb, dZ = _f64(Q), _f64(K), _f64(V), _f64(Wa), _f64(Wb), _f64(dZ)
+    B, H, N, d = Q.shape
+    hidden = Wa.shape[1]
+    assert Wa.shape == (H, hidden, d) and Wb.shape == (H, d, hidden) and dZ.shape == Q.shape
+    dQ, dK, dV = np.empty_like(Q), np.empty_like(Q), np.empty_like(Q)
+    dWa, dWb = np.empty((H, hidden, d)), np.empty((H, d, hidden))
+    deta = np.zeros(1)
+    _check(_load().oracle_mlp_backward(B, H, N, d, hidden, _p(Q), _p(K), _p(V), _p(Wa), _p(Wb), float(eta), _p(dZ),
+                                       _p(dQ), _p(dK), _p(dV), _p(dWa), _p(dWb), _p(deta),
+                                       threads or default_threads()), "mlp_backward")
+    return dQ, dK, dV, dWa, dWb, float(deta[0])
+
+
+def gelu_tanh_deriv2(u):
+    return _load().oracle_gelu_tanh_deriv2(float(u))
 
 
 def mlp(Q, K, V, Wa, Wb, eta, threads=None):

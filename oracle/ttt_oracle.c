@@ -37,7 +37,7 @@
  *       from; inside a batch the notes' prefix sum carries no 1/b, while the press article's
  *       B = N/k ablation takes one step of each batch's mean loss and reads out with the final
  *       weights;
- *     - the backward pass differentiates the full-batch linear step and the depthwise-conv step;
+ *     - the backward pass differentiates the full-batch linear, depthwise-conv and MLP steps;
  *       W0 and eta are shared by every unit, so their gradients are summed (over images, over units).
  *
  * Memory layout of every array (contiguous, row-major, fp64):
@@ -849,6 +849,185 @@ int oracle_mlp(int B, int heads, int N, int d, int hidden, const double* Q, cons
             status = s;
         }
     }
+    return status;
+}
+
+/* Second derivative of gelu_tanh (needed by the MLP head's backward pass): with
+ * t = tanh(c (u + a u^3)) and w = c (1 + 3 a u^2),  gelu'' = (1 - t^2) (w - u t w^2 + 3 a c u^2). */
+double oracle_gelu_tanh_deriv2(double u)
+{
+    const double c = sqrt(2.0 / M_PI), a = 0.044715;
+    const double t = tanh(c * (u + a * u * u * u));
+    const double w = c * (1.0 + 3.0 * a * u * u);
+    return (1.0 - t * t) * (w - u * t * w * w + 3.0 * a * c * u * u);
+}
+
+/* Backward pass of the MLP head (press article, Observation 1: the outer gradient flows through the */
+/* inner step; the head: Observation 4).  With s = 2/N and, per key token,                         */
+/*   h = Wa k, a = gelu(h), D = gelu'(h), r = Wb a - v, b = Wb^T r, e = b * D  (* elementwise),     */
+/*   gWb = s sum r a^T, gWa = s sum e k^T, Wa1 = Wa - eta gWa, Wb1 = Wb - eta gWb,                 */
+/* and per query token hq = Wa1 q, aq = gelu(hq), z = Wb1 aq, the chain rule for dZ gives          */
+/*   readout:  dWb1 = sum dz aq^T,  dhq = (Wb1^T dz) * gelu'(hq),  dq = Wa1^T dhq,                 */
+/*             dWa1 = sum dhq q^T;                                                               */
+/*   update:   dgWa = -eta dWa1, dgWb = -eta dWb1, deta = -sum dWa1 * gWa - sum dWb1 * gWb,        */
+/*             and per key token                                                                 */
+/*             de = s dgWa k,  db = de * D,  dD = de * b,  dr = s dgWb a + Wb db,                   */
+/*             da = s dgWb^T r + Wb^T dr,  dh = da * D + dD * gelu''(h),                          */
+/*             dk = s dgWa^T e + Wa^T dh,  dv = -dr,                                              */
+/*             dWa += dh k^T,  dWb += dr a^T + r db^T;                                           */
+/*   dWa_total = dWa1 + dWa,  dWb_total = dWb1 + dWb.                                            */
+/* Wa, Wb and eta are shared by every unit: dWa, dWb are summed over the images of each head and   */
+/* deta over every unit, in index order.                                                         */
+static int mlp_backward_unit(int N, int d, int hid, const double* Q, const double* K, const double* V,
+                             const double* Wa, const double* Wb, double eta, const double* dZ, double* dQ,
+                             double* dK, double* dV, double* dWa, double* dWb, double* deta)
+{
+    const size_t wsz = (size_t)hid * d;
+    double* buf = (double*)calloc(8 * wsz + 12 * (size_t)hid, sizeof(double));
+    if (!buf) return ORACLE_ERR_NOMEM;
+    double *gA = buf, *gB = buf + wsz, *Wa1 = buf + 2 * wsz, *Wb1 = buf + 3 * wsz;
+    double *dWa1 = buf + 4 * wsz, *dWb1 = buf + 5 * wsz, *dgA = buf + 6 * wsz, *dgB = buf + 7 * wsz;
+    double* vec = buf + 8 * wsz;
+    double *h = vec, *a = vec + hid, *D = vec + 2 * hid, *bb = vec + 3 * hid, *e = vec + 4 * hid;
+    double *de = vec + 5 * hid, *db = vec + 6 * hid, *dD = vec + 7 * hid, *da = vec + 8 * hid, *dh = vec + 9 * hid;
+    double r[256], dr[256], dz[256];
+    if (d > 256) { free(buf); return ORACLE_ERR_ARG; }
+    const double s = 2.0 / (double)N;
+    /* (1) the inner step's gradients at (Wa, Wb) and the updated weights */
+    for (int n = 0; n < N; ++n) {
+        const double *k = K + (size_t)n * d, *v = V + (size_t)n * d;
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0;
+            for (int i = 0; i < d; ++i) t += Wa[(size_t)j * d + i] * k[i];
+            h[j] = t; a[j] = oracle_gelu_tanh(t); D[j] = oracle_gelu_tanh_deriv(t);
+        }
+        for (int i = 0; i < d; ++i) {
+            double t = 0.0;
+            for (int j = 0; j < hid; ++j) t += Wb[(size_t)i * hid + j] * a[j];
+            r[i] = t - v[i];
+        }
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0;
+            for (int i = 0; i < d; ++i) t += Wb[(size_t)i * hid + j] * r[i];
+            e[j] = t * D[j];
+        }
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < hid; ++j) gB[(size_t)i * hid + j] += s * r[i] * a[j];
+        for (int j = 0; j < hid; ++j)
+            for (int i = 0; i < d; ++i) gA[(size_t)j * d + i] += s * e[j] * k[i];
+    }
+    for (size_t i = 0; i < wsz; ++i) { Wa1[i] = Wa[i] - eta * gA[i]; Wb1[i] = Wb[i] - eta * gB[i]; }
+    /* (2) the readout */
+    for (int n = 0; n < N; ++n) {
+        const double* q = Q + (size_t)n * d;
+        for (int i = 0; i < d; ++i) dz[i] = dZ[(size_t)n * d + i];
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0;
+            for (int i = 0; i < d; ++i) t += Wa1[(size_t)j * d + i] * q[i];
+            h[j] = t; a[j] = oracle_gelu_tanh(t); D[j] = oracle_gelu_tanh_deriv(t);
+        }
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0;
+            for (int i = 0; i < d; ++i) t += Wb1[(size_t)i * hid + j] * dz[i];
+            dh[j] = t * D[j];
+        }
+        for (int i = 0; i < d; ++i) {
+            double t = 0.0;
+            for (int j = 0; j < hid; ++j) t += Wa1[(size_t)j * d + i] * dh[j];
+            dQ[(size_t)n * d + i] = t;
+        }
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < hid; ++j) dWb1[(size_t)i * hid + j] += dz[i] * a[j];
+        for (int j = 0; j < hid; ++j)
+            for (int i = 0; i < d; ++i) dWa1[(size_t)j * d + i] += dh[j] * q[i];
+    }
+    double dsum = 0.0;
+    for (size_t i = 0; i < wsz; ++i) {
+        dgA[i] = -eta * dWa1[i];
+        dgB[i] = -eta * dWb1[i];
+        dsum += -dWa1[i] * gA[i] - dWb1[i] * gB[i];
+        dWa[i] += dWa1[i];
+        dWb[i] += dWb1[i];
+    }
+    *deta += dsum;
+    /* (3) through the inner step, per key token */
+    for (int n = 0; n < N; ++n) {
+        const double *k = K + (size_t)n * d, *v = V + (size_t)n * d;
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0;
+            for (int i = 0; i < d; ++i) t += Wa[(size_t)j * d + i] * k[i];
+            h[j] = t; a[j] = oracle_gelu_tanh(t); D[j] = oracle_gelu_tanh_deriv(t);
+        }
+        for (int i = 0; i < d; ++i) {
+            double t = 0.0;
+            for (int j = 0; j < hid; ++j) t += Wb[(size_t)i * hid + j] * a[j];
+            r[i] = t - v[i];
+        }
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0, u = 0.0;
+            for (int i = 0; i < d; ++i) { t += Wb[(size_t)i * hid + j] * r[i]; u += dgA[(size_t)j * d + i] * k[i]; }
+            bb[j] = t; e[j] = t * D[j];
+            de[j] = s * u; db[j] = de[j] * D[j]; dD[j] = de[j] * t;
+        }
+        for (int i = 0; i < d; ++i) {
+            double t = 0.0;
+            for (int j = 0; j < hid; ++j) t += s * dgB[(size_t)i * hid + j] * a[j] + Wb[(size_t)i * hid + j] * db[j];
+            dr[i] = t;
+        }
+        for (int j = 0; j < hid; ++j) {
+            double t = 0.0;
+            for (int i = 0; i < d; ++i) t += s * dgB[(size_t)i * hid + j] * r[i] + Wb[(size_t)i * hid + j] * dr[i];
+            da[j] = t;
+            dh[j] = t * D[j] + dD[j] * oracle_gelu_tanh_deriv2(h[j]);
+        }
+        for (int i = 0; i < d; ++i) {
+            double t = 0.0;
+            for (int j = 0; j < hid; ++j) t += s * dgA[(size_t)j * d + i] * e[j] + Wa[(size_t)j * d + i] * dh[j];
+            dK[(size_t)n * d + i] = t;
+            dV[(size_t)n * d + i] = -dr[i];
+        }
+        for (int j = 0; j < hid; ++j)
+            for (int i = 0; i < d; ++i) dWa[(size_t)j * d + i] += dh[j] * k[i];
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < hid; ++j) dWb[(size_t)i * hid + j] += dr[i] * a[j] + r[i] * db[j];
+    }
+    free(buf);
+    return ORACLE_OK;
+}
+
+/* dWa: [heads][hidden][d], dWb: [heads][d][hidden] (summed over images), deta: one value (summed over
+ * units), as for the linear head's backward. */
+int oracle_mlp_backward(int B, int heads, int N, int d, int hidden, const double* Q, const double* K,
+                        const double* V, const double* Wa, const double* Wb, double eta, const double* dZ,
+                        double* dQ, double* dK, double* dV, double* dWa, double* dWb, double* deta, int nthreads)
+{
+    if (B < 0 || heads < 0 || N < 1 || d < 1 || d > 256 || hidden < 1 || !Q || !K || !V || !Wa || !Wb || !dZ ||
+        !dQ || !dK || !dV || !dWa || !dWb || !deta)
+        return ORACLE_ERR_ARG;
+    const size_t wsz = (size_t)hidden * d;
+    double* deta_h = (double*)calloc(heads > 0 ? (size_t)heads : 1, sizeof(double));
+    if (!deta_h) return ORACLE_ERR_NOMEM;
+    memset(dWa, 0, (size_t)heads * wsz * sizeof(double));
+    memset(dWb, 0, (size_t)heads * wsz * sizeof(double));
+    int status = ORACLE_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int h = 0; h < heads; ++h) {
+        for (int b = 0; b < B; ++b) {
+            const size_t off = ((size_t)b * heads + h) * N * d;
+            int st = mlp_backward_unit(N, d, hidden, Q + off, K + off, V + off, Wa + h * wsz, Wb + h * wsz, eta,
+                                       dZ + off, dQ + off, dK + off, dV + off, dWa + h * wsz, dWb + h * wsz,
+                                       &deta_h[h]);
+            if (st != ORACLE_OK) {
+#pragma omp atomic write
+                status = st;
+            }
+        }
+    }
+    double total = 0.0;
+    for (int h = 0; h < heads; ++h) total += deta_h[h];
+    *deta = total;
+    free(deta_h);
     return status;
 }
 

@@ -965,6 +965,123 @@ def test_mlp_reproduced_values_give_no_update():
     np.testing.assert_allclose(Wb1[0], Wb, atol=1e-13, rtol=0)
 
 
+# ------------------------------------------------------------------------------------------------
+# backward pass of the MLP head
+# ------------------------------------------------------------------------------------------------
+def test_gelu_tanh_second_derivative_matches_torch():
+    us = np.concatenate([np.linspace(-8, 8, 201), RNG.standard_normal(100) * 3])
+    for u in us:
+        ut = torch.tensor(u, dtype=torch.float64, requires_grad=True)
+        (g1,) = torch.autograd.grad(F.gelu(ut, approximate="tanh"), ut, create_graph=True)
+        (g2,) = torch.autograd.grad(g1, ut)
+        assert abs(oracle.gelu_tanh_deriv2(u) - g2.item()) <= 1e-12 * max(1.0, abs(g2.item()))
+
+
+def _mbwd_case(B=2, H=2, N=7, d=4, hid=8, seed=0):
+    r = np.random.default_rng(300 + seed)
+    Q, K, V, dZ = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    Wa = r.standard_normal((H, hid, d)) / np.sqrt(d)
+    Wb = r.standard_normal((H, d, hid)) / np.sqrt(hid)
+    return Q, K, V, Wa, Wb, dZ
+
+
+def _mfwd_loss(Q, K, V, Wa, Wb, eta, dZ):
+    """L = sum dZ * Z with Z from the pinned forward oracle of the MLP head."""
+    Z, _, _ = oracle.mlp(Q, K, V, Wa, Wb, eta)
+    return float(np.sum(dZ * Z))
+
+
+def test_mlp_backward_matches_central_differences_of_the_forward_oracle():
+    Q, K, V, Wa, Wb, dZ = _mbwd_case()
+    eta, h = 0.6, 1e-5
+    dQ, dK, dV, dWa, dWb, deta = oracle.mlp_backward(Q, K, V, Wa, Wb, eta, dZ)
+    grads = {"Q": dQ, "K": dK, "V": dV, "Wa": dWa, "Wb": dWb}
+    args = {"Q": Q, "K": K, "V": V, "Wa": Wa, "Wb": Wb}
+    r = np.random.default_rng(11)
+    for name, g in grads.items():
+        for _ in range(8):
+            idx = tuple(int(r.integers(0, n)) for n in args[name].shape)
+            plus = {k: v.copy() for k, v in args.items()}
+            minus = {k: v.copy() for k, v in args.items()}
+            plus[name][idx] += h
+            minus[name][idx] -= h
+            fd = (_mfwd_loss(plus["Q"], plus["K"], plus["V"], plus["Wa"], plus["Wb"], eta, dZ) -
+                  _mfwd_loss(minus["Q"], minus["K"], minus["V"], minus["Wa"], minus["Wb"], eta, dZ)) / (2 * h)
+            assert abs(g[idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, g[idx], fd)
+    fd = (_mfwd_loss(Q, K, V, Wa, Wb, eta + h, dZ) - _mfwd_loss(Q, K, V, Wa, Wb, eta - h, dZ)) / (2 * h)
+    assert abs(deta - fd) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_mlp_backward_matches_torch_autograd():
+    Q, K, V, Wa, Wb, dZ = _mbwd_case(B=2, H=2, N=13, d=6, hid=12, seed=1)
+    eta = 0.4
+    dQ, dK, dV, dWa, dWb, deta = oracle.mlp_backward(Q, K, V, Wa, Wb, eta, dZ)
+    tQ, tK, tV, tA, tB = (torch.tensor(a, requires_grad=True) for a in (Q, K, V, Wa, Wb))
+    te = torch.tensor(eta, dtype=torch.float64, requires_grad=True)
+    N = Q.shape[2]
+    tot = 0.0
+    for b in range(Q.shape[0]):
+        for hh in range(Q.shape[1]):
+            A, Bm = tA[hh], tB[hh]
+            r = _torch_mlp(tK[b, hh], A, Bm) - tV[b, hh]
+            loss = (r ** 2).sum(-1).mean()
+            gA, gB = torch.autograd.grad(loss, (A, Bm), create_graph=True)
+            Z = _torch_mlp(tQ[b, hh], A - te * gA, Bm - te * gB)
+            tot = tot + (Z * torch.tensor(dZ[b, hh])).sum()
+    tot.backward()
+    for got, t in ((dQ, tQ), (dK, tK), (dV, tV), (dWa, tA), (dWb, tB)):
+        np.testing.assert_allclose(got, t.grad.numpy(), atol=1e-10, rtol=0)
+    assert abs(deta - te.grad.item()) <= 1e-10 * max(1.0, abs(deta))
+
+
+def test_mlp_backward_special_cases():
+    """dZ = 0 gives zero gradients; eta = 0 makes the head z = Wb gelu(Wa q): dK = dV = 0 and dQ,
+    dWa, dWb are the plain MLP's gradients (torch autograd)."""
+    Q, K, V, Wa, Wb, dZ = _mbwd_case(B=2, H=1, N=9, d=4, hid=8, seed=2)
+    out = oracle.mlp_backward(Q, K, V, Wa, Wb, 0.8, np.zeros_like(dZ))
+    for a in out[:5]:
+        assert np.all(a == 0.0)
+    assert out[5] == 0.0
+    dQ, dK, dV, dWa, dWb, _ = oracle.mlp_backward(Q, K, V, Wa, Wb, 0.0, dZ)
+    assert np.all(dK == 0.0) and np.all(dV == 0.0)
+    tQ, tA, tB = (torch.tensor(a, requires_grad=True) for a in (Q, Wa[0], Wb[0]))
+    (_torch_mlp(tQ[:, 0], tA, tB) * torch.tensor(dZ[:, 0])).sum().backward()
+    np.testing.assert_allclose(dQ[:, 0], tQ.grad.numpy()[:, 0], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dWa[0], tA.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dWb[0], tB.grad.numpy(), atol=1e-12, rtol=0)
+
+
+def test_planted_mistake_fails_the_mlp_backward_pin():
+    """Dropping the gelu'' term of dh (the path through gelu' inside the inner gradient) changes
+    the key gradient by more than the central differences allow."""
+    Q, K, V, Wa, Wb, dZ = _mbwd_case(B=1, H=1, N=5, d=3, hid=6, seed=3)
+    eta, h = 0.9, 1e-5
+    dQ, dK, _, _, _, _ = oracle.mlp_backward(Q, K, V, Wa, Wb, eta, dZ)
+    N, s = Q.shape[2], 2.0 / Q.shape[2]
+    _, Wa1, Wb1 = oracle.mlp(Q, K, V, Wa, Wb, eta)
+    # the readout's dWa1, then the dropped term for key token n
+    gel = lambda u: 0.5 * u * (1 + np.tanh(np.sqrt(2 / np.pi) * (u + 0.044715 * u ** 3)))
+    d1 = np.vectorize(oracle.gelu_tanh_deriv)
+    d2 = np.vectorize(oracle.gelu_tanh_deriv2)
+    Hq = Q[0, 0] @ Wa1[0, 0].T
+    dHq = (dZ[0, 0] @ Wb1[0, 0]) * d1(Hq)
+    dWa1 = dHq.T @ Q[0, 0]
+    n, i = 2, 1
+    k, v = K[0, 0, n], V[0, 0, n]
+    hvec = Wa[0] @ k
+    rvec = Wb[0] @ gel(hvec) - v
+    bvec = Wb[0].T @ rvec
+    de = s * (-eta * dWa1) @ k
+    dropped = (de * bvec * d2(hvec)) @ Wa[0][:, i]
+    bad = dK[0, 0, n, i] - dropped
+    plus, minus = K.copy(), K.copy()
+    plus[0, 0, n, i] += h
+    minus[0, 0, n, i] -= h
+    fd = (_mfwd_loss(Q, plus, V, Wa, Wb, eta, dZ) - _mfwd_loss(Q, minus, V, Wa, Wb, eta, dZ)) / (2 * h)
+    assert abs(dK[0, 0, n, i] - fd) <= 1e-6 * max(1.0, abs(fd))
+    assert abs(bad - fd) > 1e-5
+
+
 def test_threads_do_not_change_results():
     B, H, N, d = 3, 2, 40, 8
     Q, K, V = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
