@@ -72,7 +72,8 @@ typedef enum {
     TTT_HEAD_MLP = 2,
     TTT_HEAD_LINEAR_BACKWARD = 3,  /* the workspace of ttt_backward_linear */
     TTT_HEAD_CONV3X3 = 4,          /* the workspace of ttt_forward_conv3x3 */
-    TTT_HEAD_DWCONV_BACKWARD = 5   /* the workspace of ttt_backward_dwconv */
+    TTT_HEAD_DWCONV_BACKWARD = 5,  /* the workspace of ttt_backward_dwconv */
+    TTT_HEAD_MLP_BACKWARD = 6      /* the workspace of ttt_backward_mlp */
 } ttt_head_kind;
 
 /* Inner loss of the one-step training.
@@ -257,6 +258,24 @@ ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, cons
 ttt_status ttt_backward_dwconv(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
                                float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
                                void* dV, float* dW0_out, float* deta_out, void* stream);
+
+/* Backward pass of the MLP head (L2 loss; the head of ttt_forward_mlp), the outer gradient through its
+ * inner step (press article, Observation 1).  With s = 2/N, per key token h = Wa k, a = gelu(h),
+ * D = gelu'(h), r = Wb a - v, b = Wb^T r, e = b * D, the step gWb = s sum r a^T, gWa = s sum e k^T,
+ * Wa1 = Wa - eta gWa, Wb1 = Wb - eta gWb, and per query token hq = Wa1 q, aq = gelu(hq):
+ *   readout: dWb1 = sum dz aq^T, dhq = (Wb1^T dz) * gelu'(hq), dq = Wa1^T dhq, dWa1 = sum dhq q^T;
+ *   update:  dgWa = -eta dWa1, dgWb = -eta dWb1, and per key token de = s dgWa k, db = de * D,
+ *            dD = de * b, dr = s dgWb a + Wb db, da = s dgWb^T r + Wb^T dr, dh = da * D + dD * gelu''(h),
+ *            dk = s dgWa^T e + Wa^T dh, dv = -dr, dWa += dh k^T, dWb += dr a^T + r db^T;
+ *   dWa_out = sum over images of (dWa1 + dWa), dWb_out likewise, deta = -sum dWa1 * gWa - sum dWb1 * gWb
+ *   summed over every unit.
+ *   Wa: [heads][hidden][d], Wb: [heads][d][hidden] fp32; dWa_out / dWb_out optional, same shapes.
+ *   dQ, dK, dV like Q.  hidden a multiple of 64 up to 256; bf16 or fp32 inputs, fp32 arithmetic;
+ *   ws: ttt_workspace_bytes(TTT_HEAD_MLP_BACKWARD, s) bytes (needs no zero fill); deterministic.
+ *   s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED). */
+ttt_status ttt_backward_mlp(const void* Q, const void* K, const void* V, const float* Wa, const float* Wb,
+                            const void* dZ, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ,
+                            void* dK, void* dV, float* dWa_out, float* dWb_out, float* deta_out, void* stream);
 
 /* A layer whose heads [0, heads - conv_heads) are linear heads and whose last conv_heads heads are
  * depthwise-conv heads (ViT^3 keeps one conv head among its linear heads: press article,

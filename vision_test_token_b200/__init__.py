@@ -6,8 +6,8 @@ package holds its ctypes binding (``capi``), torch-facing wrappers (``layer``), 
 generator (``inputs``) and the build script (``build``).
 """
 from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
-from .layer import (backward_dwconv, backward_linear, forward_conv3x3, forward_dwconv, forward_layer, forward_linear,  # noqa: F401
+from .layer import (backward_dwconv, backward_linear, backward_mlp, forward_conv3x3, forward_dwconv, forward_layer, forward_linear,  # noqa: F401
                     forward_linear_minibatch, forward_mlp, workspace, workspace_status)
 
 __all__ = ["WORKLOADS", "Workload", "make_inputs", "forward_linear", "forward_linear_minibatch", "forward_dwconv",
-           "forward_conv3x3", "forward_mlp", "forward_layer", "backward_linear", "backward_dwconv", "workspace", "workspace_status"]
+           "forward_conv3x3", "forward_mlp", "forward_layer", "backward_linear", "backward_dwconv", "backward_mlp", "workspace", "workspace_status"]

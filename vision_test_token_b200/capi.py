@@ -11,7 +11,7 @@ TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_ALIGNMENT = 0, 1, 2, 3
 TTT_ERR_WORKSPACE, TTT_ERR_CUDA, TTT_ERR_TIMEOUT = 4, 5, 6
 TTT_FP32, TTT_BF16 = 0, 1
 TTT_HEAD_LINEAR, TTT_HEAD_DWCONV, TTT_HEAD_MLP, TTT_HEAD_LINEAR_BACKWARD, TTT_HEAD_CONV3X3 = 0, 1, 2, 3, 4
-TTT_HEAD_DWCONV_BACKWARD = 5
+TTT_HEAD_DWCONV_BACKWARD, TTT_HEAD_MLP_BACKWARD = 5, 6
 TTT_LOSS_L2, TTT_LOSS_DOT = 0, 1
 TTT_MB_PREFIX, TTT_MB_EPOCH = 0, 1
 
@@ -19,7 +19,7 @@ TTT_MB_PREFIX, TTT_MB_EPOCH = 0, 1
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_workspace_init", "ttt_workspace_status",
     "ttt_forward_linear", "ttt_forward_dwconv", "ttt_forward_conv3x3", "ttt_forward_mlp", "ttt_forward_linear_noalloc", "ttt_noalloc_status",
-    "ttt_forward_linear_minibatch", "ttt_backward_linear", "ttt_backward_dwconv",
+    "ttt_forward_linear_minibatch", "ttt_backward_linear", "ttt_backward_dwconv", "ttt_backward_mlp",
     "ttt_layer_workspace_bytes", "ttt_forward_layer", "ttt_selftest_wait_timeout", "ttt_set_wait_limit",
     "ttt_status_string", "ttt_last_error", "ttt_version",
 )
@@ -69,6 +69,8 @@ def lib():
         L.ttt_backward_linear.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp, vp, vp, vp, vp]
         L.ttt_backward_dwconv.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp, vp, vp, vp, vp]
         L.ttt_backward_dwconv.restype = i
+        L.ttt_backward_mlp.argtypes = [vp, vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp, vp, vp, vp, vp, vp]
+        L.ttt_backward_mlp.restype = i
         L.ttt_backward_linear.restype = i
         L.ttt_forward_dwconv.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
         L.ttt_forward_conv3x3.argtypes = [vp, vp, vp, vp, vp, f, shp, vp, sz, vp, vp]
@@ -141,6 +143,11 @@ def ttt_backward_linear(Q, K, V, W0, dZ, eta, shape, ws, ws_bytes, dQ, dK, dV, d
 def ttt_backward_dwconv(Q, K, V, W0, dZ, eta, shape, ws, ws_bytes, dQ, dK, dV, dW0_out, deta_out, stream):
     return lib().ttt_backward_dwconv(Q, K, V, W0, dZ, eta, ctypes.byref(shape), ws, ws_bytes, dQ, dK, dV, dW0_out,
                                      deta_out, stream)
+
+
+def ttt_backward_mlp(Q, K, V, Wa, Wb, dZ, eta, shape, ws, ws_bytes, dQ, dK, dV, dWa_out, dWb_out, deta_out, stream):
+    return lib().ttt_backward_mlp(Q, K, V, Wa, Wb, dZ, eta, ctypes.byref(shape), ws, ws_bytes, dQ, dK, dV, dWa_out,
+                                  dWb_out, deta_out, stream)
 
 
 def ttt_forward_dwconv(Q, K, V, W0, Z, eta, shape, ws, ws_bytes, W1_out, stream):

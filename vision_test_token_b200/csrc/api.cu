@@ -122,6 +122,11 @@ static ttt_status check_shape(int kind, const ttt_shape* s) {
         if (s->dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
         if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
     }
+    if (kind == TTT_HEAD_MLP_BACKWARD) {
+        if (s->hidden < 64 || s->hidden % 64 != 0) return TTT_ERR_INVALID_ARG;
+        if (s->hidden > 256) return TTT_ERR_UNSUPPORTED;
+        if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
+    }
     if (kind == TTT_HEAD_MLP) {
         if (s->hidden < 64 || s->hidden % 64 != 0) return TTT_ERR_INVALID_ARG;
         if (s->hidden > 256) return TTT_ERR_UNSUPPORTED;
@@ -165,7 +170,8 @@ static ttt_status prepare(int kind, const void* Q, const void* K, const void* V,
                           void* stream, Call* c) {
     ttt_status st = check_shape(kind, s);
     if (st != TTT_OK) return st;
-    if (!Q || !K || !V || !W0 || !Z || (kind == TTT_HEAD_MLP && !W0b)) return TTT_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !W0 || !Z || ((kind == TTT_HEAD_MLP || kind == TTT_HEAD_MLP_BACKWARD) && !W0b))
+        return TTT_ERR_INVALID_ARG;
     if (!std::isfinite(eta)) return TTT_ERR_INVALID_ARG;
     if (need > 0 && (!ws || ws_bytes < need)) return TTT_ERR_WORKSPACE;   // need 0: the call takes no workspace
     for (const void* p : {Q, K, V, (const void*)Z})
@@ -259,6 +265,7 @@ size_t ttt_workspace_bytes(int kind, const ttt_shape* s) {
         case TTT_HEAD_LINEAR_BACKWARD: return linear_backward_ws_bytes(*s);
         case TTT_HEAD_CONV3X3: return conv3x3_ws_bytes(*s);
         case TTT_HEAD_DWCONV_BACKWARD: return dwconv_backward_ws_bytes(*s);
+        case TTT_HEAD_MLP_BACKWARD: return mlp_backward_ws_bytes(*s);
         default: return 0;
     }
 }
@@ -335,16 +342,19 @@ ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void
 }
 
 static ttt_status backward_common(int kind, const void* Q, const void* K, const void* V, const float* W0,
-                                  const void* dZ, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ,
-                                  void* dK, void* dV, float* dW0_out, float* deta_out, void* stream) {
+                                  const float* W0b, const void* dZ, float eta, const ttt_shape* s, void* ws,
+                                  size_t ws_bytes, void* dQ, void* dK, void* dV, float* dW0_out, float* dW0b_out,
+                                  float* deta_out, void* stream) {
     ttt_status st = check_shape(kind, s);
     if (st != TTT_OK) return st;
     if (s->loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
     if (!dZ || !dK || !dV) return TTT_ERR_INVALID_ARG;
     Call c;
-    const size_t need = (kind == TTT_HEAD_LINEAR_BACKWARD) ? linear_backward_ws_bytes(*s) : dwconv_backward_ws_bytes(*s);
-    // Q, K, V, W0, the workspace and dQ (as the output Z: apart from Q, K and V)
-    st = prepare(kind, Q, K, V, W0, nullptr, dQ, eta, s, ws, ws_bytes, need, stream, &c);
+    const size_t need = (kind == TTT_HEAD_LINEAR_BACKWARD) ? linear_backward_ws_bytes(*s)
+                        : (kind == TTT_HEAD_DWCONV_BACKWARD) ? dwconv_backward_ws_bytes(*s)
+                                                             : mlp_backward_ws_bytes(*s);
+    // Q, K, V, the weights, the workspace and dQ (as the output Z: apart from Q, K and V)
+    st = prepare(kind, Q, K, V, W0, W0b, dQ, eta, s, ws, ws_bytes, need, stream, &c);
     if (st != TTT_OK) return st;
     for (const void* p : {dZ, (const void*)dK, (const void*)dV}) {
         if (reinterpret_cast<uintptr_t>(p) % 16) return TTT_ERR_ALIGNMENT;
@@ -357,24 +367,33 @@ static ttt_status backward_common(int kind, const void* Q, const void* K, const 
         for (const void* in : ins)
             if (overlaps(o, in, ext)) return TTT_ERR_INVALID_ARG;
     if (overlaps(dQ, dK, ext) || overlaps(dQ, dV, ext) || overlaps(dK, dV, ext)) return TTT_ERR_INVALID_ARG;
-    if (dW0_out && (reinterpret_cast<uintptr_t>(dW0_out) % 16 || !is_device_ptr(dW0_out))) return TTT_ERR_INVALID_ARG;
+    for (float* o : {dW0_out, dW0b_out})
+        if (o && (reinterpret_cast<uintptr_t>(o) % 16 || !is_device_ptr(o))) return TTT_ERR_INVALID_ARG;
     if (deta_out && (reinterpret_cast<uintptr_t>(deta_out) % 4 || !is_device_ptr(deta_out))) return TTT_ERR_INVALID_ARG;
     if (kind == TTT_HEAD_LINEAR_BACKWARD) return launch_linear_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
-    return launch_dwconv_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
+    if (kind == TTT_HEAD_DWCONV_BACKWARD) return launch_dwconv_backward(c, dZ, dQ, dK, dV, dW0_out, deta_out);
+    return launch_mlp_backward(c, *s, dZ, dQ, dK, dV, dW0_out, dW0b_out, deta_out);
 }
 
 ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
                                float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
                                void* dV, float* dW0_out, float* deta_out, void* stream) {
-    return backward_common(TTT_HEAD_LINEAR_BACKWARD, Q, K, V, W0, dZ, eta, s, ws, ws_bytes, dQ, dK, dV, dW0_out,
-                           deta_out, stream);
+    return backward_common(TTT_HEAD_LINEAR_BACKWARD, Q, K, V, W0, nullptr, dZ, eta, s, ws, ws_bytes, dQ, dK, dV,
+                           dW0_out, nullptr, deta_out, stream);
 }
 
 ttt_status ttt_backward_dwconv(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
                                float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
                                void* dV, float* dW0_out, float* deta_out, void* stream) {
-    return backward_common(TTT_HEAD_DWCONV_BACKWARD, Q, K, V, W0, dZ, eta, s, ws, ws_bytes, dQ, dK, dV, dW0_out,
-                           deta_out, stream);
+    return backward_common(TTT_HEAD_DWCONV_BACKWARD, Q, K, V, W0, nullptr, dZ, eta, s, ws, ws_bytes, dQ, dK, dV,
+                           dW0_out, nullptr, deta_out, stream);
+}
+
+ttt_status ttt_backward_mlp(const void* Q, const void* K, const void* V, const float* Wa, const float* Wb,
+                            const void* dZ, float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ,
+                            void* dK, void* dV, float* dWa_out, float* dWb_out, float* deta_out, void* stream) {
+    return backward_common(TTT_HEAD_MLP_BACKWARD, Q, K, V, Wa, Wb, dZ, eta, s, ws, ws_bytes, dQ, dK, dV, dWa_out,
+                           dWb_out, deta_out, stream);
 }
 
 constexpr double kConvHeadWeight = 2.0;

@@ -86,6 +86,11 @@ size_t dwconv_backward_ws_bytes(const ttt_shape& s);
 ttt_status launch_dwconv_backward(const Call& c, const void* dZ, void* dQ, void* dK, void* dV, float* dW0_out,
                                   float* deta_out);
 
+// Backward pass of the MLP head (s: the validated shape, for the workspace layout).
+size_t mlp_backward_ws_bytes(const ttt_shape& s);
+ttt_status launch_mlp_backward(const Call& c, const ttt_shape& s, const void* dZ, void* dQ, void* dK, void* dV,
+                               float* dWa_out, float* dWb_out, float* deta_out);
+
 // Mini-batch linear head (its workspace is the error word only): batch_tokens >= 1, mode
 // TTT_MB_PREFIX or TTT_MB_EPOCH.
 ttt_status launch_linear_minibatch(const Call& c, int batch_tokens, int mode);

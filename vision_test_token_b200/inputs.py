@@ -30,6 +30,7 @@ Workloads (token counts are the pages' image sizes divided into 16 x 16 patches:
                    bf16, eta 0.5
   bwdconv6084_bf16 backward pass of the depthwise-conv head of mixed6084_bf16: B 8, 1 head, 78 x 78,
                    bf16, eta 0.5 (conv W0 and dZ as above)
+  bwdmlp1024_bf16  backward pass of mlp1024_bf16's MLP head: B 16, 4 heads, 32 x 32, bf16, eta 0.5
   conv3x3_6084_bf16  the full 3x3 conv head (the press article's other conv variant) in place of the
                    depthwise head of mixed6084_bf16: B 8, 1 head, 78 x 78, bf16, eta 0.5
 """
@@ -49,7 +50,8 @@ class Workload:
     dtype: str            # "fp32" or "bf16"
     eta: float
     kind: str             # "linear", "mixed" (linear heads + conv heads last), "mlp", "minibatch" (linear),
-                          # "backward" (linear), "backward_conv" (depthwise conv), "conv3x3" (full 3x3 conv heads)
+                          # "backward" (linear), "backward_conv" (depthwise conv), "backward_mlp" (MLP),
+                          # "conv3x3" (full 3x3 conv heads)
     conv_heads: int = 0   # number of depthwise-conv heads (the last ones) for "mixed"
     d: int = 64
     hidden_ratio: int = 4
@@ -81,6 +83,7 @@ WORKLOADS = {
     "mb16_6084_bf16": Workload("mb16_6084_bf16", 8, 6, 78, 78, "bf16", 0.25, "minibatch", mb_tokens=16),
     "bwd6084_bf16": Workload("bwd6084_bf16", 8, 5, 78, 78, "bf16", 0.5, "backward"),
     "bwdconv6084_bf16": Workload("bwdconv6084_bf16", 8, 1, 78, 78, "bf16", 0.5, "backward_conv", conv_heads=1),
+    "bwdmlp1024_bf16": Workload("bwdmlp1024_bf16", 16, 4, 32, 32, "bf16", 0.5, "backward_mlp"),
     "conv3x3_6084_bf16": Workload("conv3x3_6084_bf16", 8, 1, 78, 78, "bf16", 0.5, "conv3x3"),
 }
 
@@ -107,12 +110,12 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu"):
             out["W0_conv"] = torch.randn((w.conv_heads, w.d, 3, 3), generator=g) / 3.0
     elif w.kind == "conv3x3":
         out["W0_c3"] = torch.randn((w.heads, w.d, w.d, 3, 3), generator=g) / math.sqrt(9 * w.d)
-    elif w.kind == "mlp":
+    elif w.kind in ("mlp", "backward_mlp"):
         hid = w.hidden_ratio * w.d
         out["Wa"] = torch.randn((w.heads, hid, w.d), generator=g) / math.sqrt(w.d)
         out["Wb"] = torch.randn((w.heads, w.d, hid), generator=g) / math.sqrt(hid)
     dt = TORCH_DTYPE[w.dtype]
-    if w.kind in ("backward", "backward_conv"):
+    if w.kind in ("backward", "backward_conv", "backward_mlp"):
         out["dZ"] = torch.randn(shape, generator=g, dtype=torch.float32).to(dt)
     out["Q"], out["K"], out["V"] = Q.to(dt), K.to(dt), V.to(dt)
     if device != "cpu":

@@ -173,6 +173,30 @@ def backward_dwconv(Q, K, V, W0, eta, H, W, dZ, out=None, ws=None, stream=None):
     return dQ, dK, dV, dW0, deta
 
 
+def backward_mlp(Q, K, V, Wa, Wb, eta, H, W, dZ, out=None, ws=None, stream=None):
+    """Backward pass of the MLP head (L2 loss) for the upstream gradient dZ of Z.  Returns (dQ, dK, dV,
+    dWa [heads][hidden][d], dWb [heads][d][hidden] fp32 summed over images, deta: a 1-element fp32 tensor
+    summed over every unit); `out` may supply those six tensors."""
+    shape = _shape_of(Q, H, W, hidden=Wa.shape[1])
+    _same_layout(Q, K, V, dZ)
+    if out is None:
+        dQ, dK, dV = (_out_like(Q, None) for _ in range(3))
+        dWa = torch.empty(Wa.shape, dtype=torch.float32, device=Q.device)
+        dWb = torch.empty(Wb.shape, dtype=torch.float32, device=Q.device)
+        deta = torch.empty(1, dtype=torch.float32, device=Q.device)
+    else:
+        dQ, dK, dV, dWa, dWb, deta = out
+    _same_layout(Q, dQ, dK, dV)
+    Wa, Wb = Wa.contiguous(), Wb.contiguous()
+    if ws is None:
+        ws = workspace(capi.TTT_HEAD_MLP_BACKWARD, shape, Q.device)
+    st = capi.ttt_backward_mlp(_ptr(Q), _ptr(K), _ptr(V), _ptr(Wa), _ptr(Wb), _ptr(dZ), float(eta), shape,
+                               *_ws_args(ws), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dWa), _ptr(dWb), _ptr(deta),
+                               _stream_handle(stream))
+    _check(st, "ttt_backward_mlp")
+    return dQ, dK, dV, dWa, dWb, deta
+
+
 def forward_dwconv(Q, K, V, W0, eta, H, W, Z=None, W1_out=None, ws=None, stream=None, max_sms=0, loss="l2"):
     """3x3 depthwise-conv inner model.  W0: [heads][d][3][3] fp32 CUDA tensor.  Returns Z."""
     shape = _shape_of(Q, H, W, max_sms=max_sms, loss=loss)
