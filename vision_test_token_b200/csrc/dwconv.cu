@@ -149,6 +149,15 @@ __device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
 
+// Waits for fill number q of a ring slot (q = sequence number / slots).  A group reads only some of
+// the fills, so the fill before q -- another group's -- may still be in flight, and a parity wait on
+// `full` alone would then pass one phase early.  Waiting first for that fill's release on `empty`
+// (which needs this reader's own arrival before it can move past fill q) leaves the `full` wait
+// unambiguous.
+__device__ __forceinline__ bool ring_wait(uint64_t* full, uint64_t* empty, uint32_t q, const Abort& ab) {
+    return mbar_wait(empty, (q & 1u) ^ 1u, ab) && mbar_wait(full, q & 1u, ab);
+}
+
 // The 4 staged rows around an output row pair: rows 0, 1 from one group, rows 2, 3 from the next
 // (32-bit shared addresses of the lane's channel pair in column 0 of each group).
 struct Rows {
@@ -393,9 +402,9 @@ dw_band(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtenso
             for (int j = 0; j < n; ++j) {
                 if (j % CG != grp || failed) continue;
                 const uint32_t k0 = kq + j, k1 = kq + j + 1, v0 = vq + j;
-                bool okb = mbar_wait(&s.kfull[k0 % NK], (k0 / NK) & 1u, ab);
-                okb = okb && mbar_wait(&s.kfull[k1 % NK], (k1 / NK) & 1u, ab);
-                okb = okb && mbar_wait(&s.vfull[v0 % NV], (v0 / NV) & 1u, ab);
+                bool okb = ring_wait(&s.kfull[k0 % NK], &s.kempty[k0 % NK], k0 / NK, ab);
+                okb = okb && ring_wait(&s.kfull[k1 % NK], &s.kempty[k1 % NK], k1 / NK, ab);
+                okb = okb && ring_wait(&s.vfull[v0 % NV], &s.vempty[v0 % NV], v0 / NV, ab);
                 if (!okb) { failed = true; continue; }
                 __syncwarp();
                 if (xa < xb) {
@@ -496,8 +505,8 @@ dw_band(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtenso
             for (int j = 0; j < n; ++j) {
                 if (j % CG != grp || failed) continue;
                 const uint32_t k0 = kq + j, k1 = kq + j + 1;
-                bool okb = mbar_wait(&s.kfull[k0 % NK], (k0 / NK) & 1u, ab);
-                okb = okb && mbar_wait(&s.kfull[k1 % NK], (k1 / NK) & 1u, ab);
+                bool okb = ring_wait(&s.kfull[k0 % NK], &s.kempty[k0 % NK], k0 / NK, ab);
+                okb = okb && ring_wait(&s.kfull[k1 % NK], &s.kempty[k1 % NK], k1 / NK, ab);
                 if (!okb) { failed = true; continue; }
                 __syncwarp();
                 const int y0 = 2 * (tk.pa + j);
