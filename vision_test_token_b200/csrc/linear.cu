@@ -3,25 +3,31 @@
 // Oral | 清華+阿里發布ViT3", Observation 2) written in Gram form:
 //     G = sum_n k_n k_n^T,   C = sum_n v_n k_n^T,   W1 = W0 - eta (2/N) (W0 G - C),   z_n = W1 q_n.
 //
-// bf16 path (lin_cluster_bf16): one thread-block cluster of CS CTAs (one CTA per SM) per unit.
-//   Phase 1: each CTA of the cluster streams its share of the unit's 128-token K/V tiles (TMA,
-//     128-byte swizzle) and accumulates [K | V]^T K  (128 x 64 fp32: rows 0..63 = G, rows 64..127
-//     = C) in tensor memory with tcgen05.mma: A = [K | V]^T (M = 128, MN-major straight from the
-//     token-major tiles), B = K (N = 64, MN-major), K-dim = tokens.
+// bf16 path (lin_cluster_bf16): one thread-block cluster of CS <= 4 CTAs (one CTA per SM) per group
+// of units; each CTA takes a 1/CS share of every unit's tokens.
+//   Phase 1: each CTA streams its share of the unit's 128-token K/V tiles (TMA, 128-byte swizzle) and
+//     accumulates [K | V]^T K  (128 x 64 fp32: rows 0..63 = G, rows 64..127 = C) in tensor memory with
+//     tcgen05.mma: A = [K | V]^T (M = 128, MN-major straight from the token-major tiles), B = K
+//     (N = 64, MN-major), K-dim = tokens.
 //   Exchange: each CTA turns its own partial (G_r, C_r) into P_r = W0 G_r - C_r.  The product runs
 //     on the tensor cores with both operands split into bf16 hi + lo parts (M = 128 rows
 //     [W0_hi ; W0_lo], B = G_hi and then G_lo), so that it carries about 16 mantissa bits, close to
 //     fp32.  P_r (16 KB) is pushed with one bulk copy into every other CTA of the cluster (distributed
 //     shared memory, completion counted on the receiver's mbarrier); each CTA then forms
 //     W1 = W0 - eta (2/N) sum_r P_r, summing in rank order (a fixed order: bitwise deterministic),
-//     and rounds W1 once to bf16 into the shared-memory B operand of phase 2.  No global-memory
+//     and rounds W1 once to bf16 into a shared-memory B operand of phase 2.  No global-memory
 //     round trip, no grid-wide wait.
-//   Phase 2: the CTA streams its share of 256-token Q tiles (they are prefetched while the cluster
-//     reduces) and writes Z = Q W1^T: A = Q tile (M = 128 tokens, K-major), B = W1 (K-major), the
-//     epilogue drains tensor memory to bf16 and stores Z with TMA.
-//   Roles (192 threads): warp 0 lane 0 TMA producer, warp 1 lane 0 MMA issuer, warps 2..5 epilogue
-//   and reduction.  CS is chosen so that all clusters are co-resident (units > SMs: CS = 1 and each
-//   CTA loops over units).
+//   Phase 2: the CTA streams its share of 256-token Q tiles and writes Z = Q W1^T: A = Q tile
+//     (M = 128 tokens, K-major), B = W1 (K-major); the epilogue drains tensor memory to bf16 and
+//     stores Z with TMA.
+//   Two units in flight: a cluster with several units streams K/V of unit k+1 before Q of unit k;
+//     with two phase-1 accumulators and two W1 operands, the exchange of unit k runs while unit
+//     k+1's keys stream in, and the exchange of unit k+1 while unit k is read out, so the exchange
+//     leaves no gap in the streaming.
+//   Roles (320 threads): warp 0 lane 0 TMA producer, warp 1 lane 0 MMA issuer, warps 2..5 drain the
+//   phase-2 accumulators and store Z, warps 6..9 run the exchanges.  CS and the number of clusters
+//   are chosen so that all clusters are co-resident (units > SMs: CS = 1 and each CTA loops over
+//   units).
 //
 // fp32 path (lin_p1_f32 / lin_p2_f32): plain fp32 FMA kernels (fp32 accuracy), static partition,
 // the same deterministic last-CTA merge.
@@ -42,7 +48,7 @@ constexpr int D = 64;
 constexpr int TOK = 128;                    // tokens per tile
 constexpr int TILE_BYTES = TOK * D * 2;     // one bf16 tile: 16 KB
 constexpr int kPartialFloats = 2 * D * D;   // [G ; C] = 128 x 64
-constexpr int kThreadsTc = 192;
+constexpr int kThreadsTc = 320;         // producer warp, MMA warp, 4 Z warps, 4 exchange warps
 constexpr int kW0tPitch = D + 4;           // row pitch of the transposed W0 in shared memory (fp32 path)
 constexpr uint32_t kIdescP1 = idesc_bf16_f32(128, 64, true, true);
 constexpr uint32_t kIdescP2 = idesc_bf16_f32(128, 64, false, false);
@@ -173,14 +179,19 @@ __device__ void merge_unit(const MergeOut& m, int u, int h, size_t slot0, int ns
 }
 
 // ------------------------------------------------------------------------------------------------
-// bf16: one thread-block cluster per unit
+// bf16: one thread-block cluster per group of units, two units in flight per cluster
 // ------------------------------------------------------------------------------------------------
 constexpr int STAGES = 4;                   // 32 KB each: a K+V tile pair, or one 256-token Q tile
 constexpr int ACC = 4;                      // phase-2 accumulators (64 columns each)
 constexpr int Q2 = 256;                     // tokens per phase-2 stage
-constexpr int kMaxCluster = 3;                // receive slots of the exchange live in the Z staging area
+constexpr int kMaxCluster = 4;
+constexpr int kRecvBytes = 12288;           // the peers' rows of my P block: (CS - 1) x ceil(64 / CS) x 256 B
+constexpr uint32_t kColPacc = 0;            // tensor memory: two phase-1 accumulators,
+constexpr uint32_t kColAcc = 128;           //   ACC phase-2 accumulators,
+constexpr uint32_t kColProd = 384;          //   the W0 G product (448 of 512 columns)
+constexpr uint32_t kBarZ = 1, kBarX = 2;    // named barriers of the two epilogue warpgroups
 
-// [G ; C] rows in shared memory: 16-byte chunks XOR-swizzled by (row & 15) against bank conflicts.
+// [G ; C] or P rows in shared memory: 16-byte chunks XOR-swizzled by (row & 15) against bank conflicts.
 __device__ __forceinline__ float4* gc_chunk(float* gc, int row, int chunk) {
     return reinterpret_cast<float4*>(gc + row * D) + (chunk ^ (row & 15));
 }
@@ -214,33 +225,43 @@ struct ClusterParams {
 };
 
 struct ClusterSmem {
-    uint8_t stage[STAGES][2 * TILE_BYTES];   // 1024-aligned
-    uint8_t zbuf[2][TILE_BYTES];             // Z staging; doubles as the receive slots of the peers' P
-    uint8_t w1[D * D * 2];                   // W1, bf16, 128-byte swizzled K-major B operand
-    uint8_t a01[2 * D * D * 2];              // [W0_hi ; W0_lo] (bf16 A operand), then D rows 64.. (fp32)
-    float gc[2 * D * D];                     // G as bf16 hi/lo B operands, then C; C rows become P (sent)
+    uint8_t stage[STAGES][2 * TILE_BYTES];   // 1024-aligned operand buffers
+    uint8_t zbuf[2][TILE_BYTES];             // Z staging of the TMA stores
+    uint8_t recv[kRecvBytes];                // the peers' rows of this CTA's block of P
+    uint8_t w1[2][D * D * 2];                // W1 of two units, bf16, 128-byte swizzled K-major B operand
+    uint8_t a01[2 * D * D * 2];              // [W0_hi ; W0_lo] (bf16 A operand of the product)
+    uint8_t gb[2 * D * D * 2];               // G_hi, G_lo (bf16 B operands); then P = W0 G - C (fp32)
     uint64_t full[STAGES], empty[STAGES];
-    uint64_t pacc_full, pacc_empty;          // phase-1 accumulator
+    uint64_t pacc_full[2], pacc_empty[2];    // phase-1 accumulators
     uint64_t acc_full[ACC], acc_empty[ACC];  // phase-2 accumulators
-    uint64_t w_full, w_empty;                // W1 in shared memory
+    uint64_t w_full[2], w_empty[2];          // W1 operands
     uint64_t prod_bar;                       // the W0 G product on the tensor cores is done
-    uint64_t recv_full;                      // the peers' P have landed in zbuf (bytes via complete_tx)
-    uint64_t peer_free;                      // every peer has finished the previous unit: its slots are free
-    uint64_t drain_bar, pdrain_bar;          // the MMAs of the MMA lane / of the epilogue's products (exit)
+    uint64_t recv_full;                      // the peers' rows of my P block have landed in recv
+    uint64_t w1_full;                        // the peers' W1 rows have landed in the W1 operand
+    uint64_t peer_free;                      // every peer has finished the previous exchange
+    uint64_t drain_bar, pdrain_bar;          // the MMAs of the MMA lane / of the products (exit)
     uint32_t tmem_base;
-    uint32_t recv_armed;                     // phases of recv_full armed so far
+    uint32_t recv_armed;                     // phases of recv_full (and of w1_full) armed so far
     int abort_flag;
 };
 
 __device__ __forceinline__ int split_lo(int n, int r, int parts) { return (int)((long long)n * r / parts); }
 
+// Units of this cluster: u_k = cid + k * ncl for k < units_of(cid).
+__device__ __forceinline__ int units_of(const ClusterParams& p, int cid, int ncl) {
+    return cid < p.U ? (p.U - cid + ncl - 1) / ncl : 0;
+}
+
+// The producer streams K/V of unit k+1 before Q of unit k, so that the cluster's exchange for unit k
+// runs while unit k+1's keys stream in, and unit k+1's exchange while unit k is read out.
 __device__ __forceinline__ void cl_producer(ClusterSmem& s, const ClusterParams& p, const CUtensorMap* tmK,
                                             const CUtensorMap* tmV, const CUtensorMap* tmQ, int rank, int cid,
                                             int ncl, const Abort& ab) {
     int st = 0; uint32_t ph = 0;
     uint32_t issued = 0;
     bool ok = true;
-    for (int u = cid; u < p.U && ok; u += ncl) {
+    const int m = units_of(p, cid, ncl);
+    auto load_kv = [&](int u) {
         const int b = u / p.heads, h = u % p.heads;
         const int t1b = split_lo(p.tpu1, rank, p.CS), t1e = split_lo(p.tpu1, rank + 1, p.CS);
         for (int t = t1b; t < t1e && ok; ++t) {
@@ -251,7 +272,9 @@ __device__ __forceinline__ void cl_producer(ClusterSmem& s, const ClusterParams&
             ++issued;
             if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
-        // Q does not depend on W1: it streams in while the cluster reduces and forms W1.
+    };
+    auto load_q = [&](int u) {
+        const int b = u / p.heads, h = u % p.heads;
         const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
         for (int t = t2b; t < t2e && ok; ++t) {
             if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
@@ -260,6 +283,11 @@ __device__ __forceinline__ void cl_producer(ClusterSmem& s, const ClusterParams&
             ++issued;
             if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
+    };
+    if (m > 0) load_kv(cid);
+    for (int k = 0; k < m && ok; ++k) {
+        if (k + 1 < m) load_kv(cid + (k + 1) * ncl);
+        load_q(cid + k * ncl);
     }
     // Before the CTA may exit, every tile load it issued has landed (on a normal exit they were all
     // consumed already; after a wait gave up, some may still be in flight).
@@ -271,13 +299,17 @@ __device__ __forceinline__ void cl_mma(ClusterSmem& s, const ClusterParams& p, u
                                        int ncl, const Abort& ab) {
     int st = 0; uint32_t ph = 0;
     int ai = 0; uint32_t aph = 0;
-    uint32_t k = 0;
-    for (int u = cid; u < p.U; u += ncl, ++k) {
-        if (!mbar_wait(&s.pacc_empty, (k & 1u) ^ 1u, ab)) return;
+    const int m = units_of(p, cid, ncl);
+    // phase 1 of unit k: [K | V]^T K into accumulator k & 1 (A = [K | V]^T, M = 128, and B = K, N = 64,
+    // both MN-major straight from the token-major tiles; 16 tokens per MMA)
+    auto p1 = [&](int k) -> bool {
+        const uint32_t a = (uint32_t)k & 1u, n = (uint32_t)k >> 1;
+        if (!mbar_wait(&s.pacc_empty[a], (n & 1u) ^ 1u, ab)) return false;
         tc_fence_after();
+        const uint32_t d = tmem + kColPacc + a * 64u;
         const int t1b = split_lo(p.tpu1, rank, p.CS), t1e = split_lo(p.tpu1, rank + 1, p.CS);
         for (int t = t1b; t < t1e; ++t) {
-            if (!mbar_wait(&s.full[st], ph, ab)) return;
+            if (!mbar_wait(&s.full[st], ph, ab)) return false;
             tc_fence_after();
             const uint32_t sK = smem_u32(s.stage[st]);
 #pragma unroll
@@ -285,28 +317,33 @@ __device__ __forceinline__ void cl_mma(ClusterSmem& s, const ClusterParams& p, u
                 // 16 tokens per MMA = two 8-row groups (2 x 1024 bytes); V sits TILE_BYTES after K
                 const uint64_t ad = sdesc_sw128(sK + kk * 2048, TILE_BYTES, 1024);
                 const uint64_t bd = sdesc_sw128(sK + kk * 2048, TILE_BYTES, 1024);
-                mma_bf16_ss(tmem, ad, bd, kIdescP1, (t > t1b || kk > 0) ? 1u : 0u);
+                mma_bf16_ss(d, ad, bd, kIdescP1, (t > t1b || kk > 0) ? 1u : 0u);
             }
             mma_commit(&s.empty[st]);
             if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
-        mma_commit(&s.pacc_full);
-        if (!mbar_wait(&s.w_full, k & 1u, ab)) return;
+        mma_commit(&s.pacc_full[a]);
+        return true;
+    };
+    // phase 2 of unit k: Z = Q W1^T per 128-token half tile (A = Q, M = 128, K-major; B = W1, K-major)
+    auto p2 = [&](int k) -> bool {
+        const uint32_t wb = (uint32_t)k & 1u, n = (uint32_t)k >> 1;
+        if (!mbar_wait(&s.w_full[wb], n & 1u, ab)) return false;
         tc_fence_after();
-        const uint32_t sW = smem_u32(s.w1);
+        const uint32_t sW = smem_u32(s.w1[wb]);
         const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
         for (int t = t2b; t < t2e; ++t) {
-            if (!mbar_wait(&s.full[st], ph, ab)) return;
+            if (!mbar_wait(&s.full[st], ph, ab)) return false;
             tc_fence_after();
             for (int hf = 0; hf < 2; ++hf) {
-                if (!mbar_wait(&s.acc_empty[ai], aph ^ 1u, ab)) return;
+                if (!mbar_wait(&s.acc_empty[ai], aph ^ 1u, ab)) return false;
                 tc_fence_after();
                 const uint32_t sQ = smem_u32(s.stage[st]) + hf * TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = sdesc_sw128(sQ + kk * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(sW + kk * 32, 16, 1024);
-                    mma_bf16_ss(tmem + 64u + (uint32_t)(ai * 64), ad, bd, kIdescP2, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColAcc + (uint32_t)(ai * 64), ad, bd, kIdescP2, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s.acc_full[ai]);
                 if (++ai == ACC) { ai = 0; aph ^= 1u; }
@@ -314,211 +351,47 @@ __device__ __forceinline__ void cl_mma(ClusterSmem& s, const ClusterParams& p, u
             mma_commit(&s.empty[st]);
             if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
-        mma_commit(&s.w_empty);
+        mma_commit(&s.w_empty[wb]);
+        return true;
+    };
+    if (m > 0 && !p1(0)) return;
+    for (int k = 0; k < m; ++k) {
+        if (k + 1 < m && !p1(k + 1)) return;
+        if (!p2(k)) return;
     }
 }
 
-__device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams& p, uint32_t tmem,
-                                            const CUtensorMap* tmZ, int rank, int cid, int ncl, const Abort& ab) {
+// Warps 2..5: drain the phase-2 accumulators of every unit in turn and store Z with TMA.
+__device__ __forceinline__ void cl_zepi(ClusterSmem& s, const ClusterParams& p, uint32_t tmem, const CUtensorMap* tmZ,
+                                        int rank, int cid, int ncl, const Abort& ab) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;                                   // tensor-memory lane quarter of this warp
     const int r = q * 32 + lane;                              // accumulator row
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const bool multi = p.CS > 1;
     int ai = 0; uint32_t aph = 0;
     int zn = 0;
-    uint32_t k = 0;
-    bool failed = false;
-    for (int u = cid; u < p.U; u += ncl, ++k) {
+    const int m = units_of(p, cid, ncl);
+    for (int k = 0; k < m; ++k) {
+        const int u = cid + k * ncl;
         const int b = u / p.heads, h = u % p.heads;
-        // W0 row (tid >> 1), columns c0w .. c0w+31, kept in registers until W1 is formed
-        const int wrow = tid >> 1, c0w = (tid & 1) * 32;
-        float w0r[32];
-        {
-            const float4* src = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + wrow) * D + c0w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 v = __ldg(src + i);
-                w0r[4 * i] = v.x; w0r[4 * i + 1] = v.y; w0r[4 * i + 2] = v.z; w0r[4 * i + 3] = v.w;
-            }
-        }
-        // (0) my receive slots (the Z staging area) are free once my Z stores have read it: arm the
-        //     receive barrier, then tell the peers they may push
-        if (tid == 0) bulk_wait_read<0>();
-        // A operand of the product: rows 0..63 = bf16(W0), rows 64..127 = bf16(W0 - bf16(W0))
-        if (!p.dot) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float hi[8], lo[8];
-                split_bf16(w0r + 8 * c, hi, lo);
-                put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
-                put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
-            }
-        }
-        named_bar_sync(1, 128);
-        if (multi && tid == 0) {
-            ++s.recv_armed;
-            mbar_arrive_expect_tx(&s.recv_full, (uint32_t)((p.CS - 1) * D * D * 4));
-            for (int pr = 0; pr < p.CS; ++pr)
-                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
-        }
-        // (1) wait for my phase-1 accumulator and for every peer to be done with the previous unit
-        //     (then my earlier pushes have landed and gc may be overwritten)
-        bool ok = mbar_wait(&s.pacc_full, k & 1u, ab);
-        if (multi) ok = ok && mbar_wait_cluster(&s.peer_free, k & 1u, ab);
-        if (named_bar_or(1, 128, !ok)) { failed = true; break; }
-        __syncwarp();
-        tc_fence_after();
-        // (2) accumulator rows -> G as bf16 hi/lo B operands (rows r < 64) and C in fp32 (rows 64..)
-        uint8_t* bhi = reinterpret_cast<uint8_t*>(s.gc);
-        uint8_t* blo = bhi + D * D * 2;
-        const bool has_p1 = split_lo(p.tpu1, rank + 1, p.CS) > split_lo(p.tpu1, rank, p.CS);
-        {
-            float v[4][16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + (uint32_t)(j * 16) + lane_off, v[j]);
-            tmem_ld_wait();
-            if (!has_p1) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[j][e] = 0.f;
-            }
-            if (r < D) {                                      // G is symmetric: row r of G = column r
-                if (!p.dot) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float hi[8], lo[8];
-                        split_bf16(&v[c / 2][(c & 1) * 8], hi, lo);
-                        put_bf16_chunk(bhi, r, c, hi);
-                        put_bf16_chunk(blo, r, c, lo);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-#pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *gc_chunk(s.gc, r, (j * 16 + e) / 4) = make_float4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
-            }
-        }
-        tc_fence_before();
-        mbar_arrive(&s.pacc_empty);
-        fence_proxy_async_smem();                             // the operands are read by the tensor cores
-        named_bar_sync(1, 128);
-        // (3) D = [W0_hi ; W0_lo] (G_hi + G_lo) on the tensor cores (M = 128, N = 64, K = 64 twice);
-        //     steps (3) and (4) only for the L2 loss (the dot-product loss sends P = C)
-        if (!p.dot) {
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t sa = smem_u32(s.a01), sh = smem_u32(bhi), sl = smem_u32(blo);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sh + kk * 32, 16, 1024),
-                                kIdescP2, kk > 0 ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16_ss(tmem + 320u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sl + kk * 32, 16, 1024),
-                                kIdescP2, 1u);
-                mma_commit(&s.prod_bar);
-            }
-            ok = mbar_wait(&s.prod_bar, k & 1u, ab);
-            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
-            __syncwarp();
-            tc_fence_after();
-            // (4) P = D[0:64] + D[64:128] - C  (= W0 G - C), written over the C rows of gc
-            float* dlo = reinterpret_cast<float*>(s.a01);          // the A operand is consumed: reuse it
-            {
-                float v[4][16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 320u + (uint32_t)(j * 16) + lane_off, v[j]);
-                tmem_ld_wait();
-                tc_fence_before();
-                if (r >= D) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-#pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            *gc_chunk(dlo, r - D, (j * 16 + e) / 4) = make_float4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
-                }
-                named_bar_sync(1, 128);
-                if (r < D) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-#pragma unroll
-                        for (int e = 0; e < 16; e += 4) {
-                            const int c = (j * 16 + e) / 4;
-                            const float4 l = *gc_chunk(dlo, r, c);
-                            float4* cp = gc_chunk(s.gc, D + r, c);
-                            const float4 cv = *cp;
-                            *cp = make_float4(v[j][e] + l.x - cv.x, v[j][e + 1] + l.y - cv.y, v[j][e + 2] + l.z - cv.z,
-                                              v[j][e + 3] + l.w - cv.w);
-                        }
-                }
-            }
-        }
-        const float* Pme = s.gc + D * D;                      // rows 64..127 of gc
-        // (5) push P to every peer (bulk copies into the peers' receive slots), then wait for theirs
-        if (multi) {
-            fence_proxy_async_smem();                         // P is read next by the bulk-copy engine
-            named_bar_sync(1, 128);
-            if (tid == 0)
-                for (int pr = 0; pr < p.CS; ++pr) {
-                    if (pr == rank) continue;
-                    const int slot = (rank < pr) ? rank : rank - 1;   // my slot in the peer's receive area
-                    bulk_s2cluster(map_to_rank(smem_u32(s.zbuf[slot]), (uint32_t)pr), Pme, D * D * 4,
-                                   map_to_rank(smem_u32(&s.recv_full), (uint32_t)pr));
-                }
-            ok = mbar_wait_cluster(&s.recv_full, k & 1u, ab);
-        } else {
-            named_bar_sync(1, 128);
-        }
-        // (6) W1 = W0 - eta_scale sum_r P_r  (ranks in order: deterministic); W1_out from rank 0
-        ok = ok && mbar_wait(&s.w_empty, (k & 1u) ^ 1u, ab);  // phase 2 of the previous unit is done with w1
-        if (named_bar_or(1, 128, !ok)) { failed = true; break; }
-        {
-            float sum[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sum[e] = 0.f;
-            for (int pr = 0; pr < p.CS; ++pr) {
-                float* src = (pr == rank) ? const_cast<float*>(Pme)
-                                          : reinterpret_cast<float*>(s.zbuf[(pr < rank) ? pr : pr - 1]);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 v = *gc_chunk(src, wrow, c0w / 4 + c);
-                    sum[4 * c] += v.x; sum[4 * c + 1] += v.y; sum[4 * c + 2] += v.z; sum[4 * c + 3] += v.w;
-                }
-            }
-            float w1[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w1[e] = w0r[e] - p.eta_scale * sum[e];
-            if (p.W1_out && rank == 0) {
-                float4* o = reinterpret_cast<float4*>(p.W1_out + ((size_t)u * D + wrow) * D + c0w);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) o[c] = make_float4(w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) put_bf16_chunk(s.w1, wrow, c0w / 8 + c, w1 + 8 * c);
-        }
-        fence_proxy_async_smem();                             // w1 is read next by the tensor cores
-        named_bar_sync(1, 128);
-        if (tid == 0) mbar_arrive(&s.w_full);
-        // (5) phase 2: Z tiles
         const int t2b = split_lo(p.tpu2, rank, p.CS), t2e = split_lo(p.tpu2, rank + 1, p.CS);
-        for (int t = t2b; t < t2e && !failed; ++t) {
+        for (int t = t2b; t < t2e; ++t) {
             for (int hf = 0; hf < 2; ++hf) {
-                ok = mbar_wait(&s.acc_full[ai], aph, ab);
+                const bool ok = mbar_wait(&s.acc_full[ai], aph, ab);
                 const int zb = zn & 1;
                 if (tid == 0 && zn >= 2) bulk_wait_read<1>();  // staging buffer zb is free again
-                if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                if (named_bar_or(kBarZ, 128, !ok)) { if (tid == 0) bulk_wait<0>(); return; }
                 __syncwarp();
                 tc_fence_after();
                 uint8_t* zrow = s.zbuf[zb] + r * 128;
                 float va[4][16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 64u + (uint32_t)(ai * 64 + j * 16) + lane_off, va[j]);
+                for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColAcc + (uint32_t)(ai * 64 + j * 16) + lane_off, va[j]);
                 tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&s.acc_empty[ai]);
+                if (++ai == ACC) { ai = 0; aph ^= 1u; }
 #pragma unroll
                 for (int j = 0; j < D; j += 16) {
                     const float* v = va[j / 16];
@@ -531,11 +404,8 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
                     *reinterpret_cast<uint4*>(zrow + ((c0 ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(zrow + (((c0 + 1) ^ (r & 7)) << 4)) = hi;
                 }
-                tc_fence_before();
-                mbar_arrive(&s.acc_empty[ai]);
-                if (++ai == ACC) { ai = 0; aph ^= 1u; }
                 fence_proxy_async_smem();
-                named_bar_sync(1, 128);
+                named_bar_sync(kBarZ, 128);
                 const int row0 = t * Q2 + hf * TOK;
                 if (tid == 0 && row0 < p.N) {
                     tma_store_4d(tmZ, s.zbuf[zb], 0, row0, h, b);
@@ -544,23 +414,222 @@ __device__ __forceinline__ void cl_epilogue(ClusterSmem& s, const ClusterParams&
                 ++zn;
             }
         }
-        if (failed) break;
     }
-    // Final handshake: once every peer has finished its last unit, all pushes from this CTA have
-    // landed and nobody will push into it again; only then may it exit.
+    if (tid == 0) bulk_wait<0>();
+}
+
+// Warps 6..9: the cluster exchange of every unit in turn.  Each CTA turns its partial (G_r, C_r) into
+// P_r = W0 G_r - C_r on the tensor cores (both operands split into bf16 hi + lo: about 16 mantissa
+// bits).  Rows of W1 are then formed in blocks, one per CTA (rank j owns rows [64 j / CS, 64 (j+1) / CS)):
+// every CTA pushes block j of its P into CTA j (reduce-scatter), sums the blocks it receives for its
+// own rows in rank order (a fixed order: bitwise deterministic), forms those rows of
+// W1 = W0 - eta (2/N) sum_r P_r rounded once to bf16 into the unit's W1 operand, and pushes them into
+// the same place in every peer's operand (all-gather).
+__device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, uint32_t tmem, int rank, int cid,
+                                        int ncl, const Abort& ab) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int tid = threadIdx.x - 192;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool multi = p.CS > 1;
+    const int m = units_of(p, cid, ncl);
+    float* pb = reinterpret_cast<float*>(s.gb);               // P (fp32 64 x 64, swizzled chunks)
+    uint8_t* bhi = s.gb;
+    uint8_t* blo = s.gb + D * D * 2;
+    const bool has_p1 = split_lo(p.tpu1, rank + 1, p.CS) > split_lo(p.tpu1, rank, p.CS);
+    const int rb0 = split_lo(D, rank, p.CS), rb1 = split_lo(D, rank + 1, p.CS);   // my block of rows
+    const int slot_rows = (D + p.CS - 1) / p.CS;                                  // rows per receive slot
+    int k = 0;
+    bool failed = false;
+    for (; k < m; ++k) {
+        const int u = cid + k * ncl;
+        const int h = u % p.heads;
+        const uint32_t a = (uint32_t)k & 1u, n = (uint32_t)k >> 1;
+        // (0) the A operand of the product: rows 0..63 = bf16(W0), rows 64..127 = bf16(W0 - bf16(W0))
+        if (!p.dot) {
+            const int wrow = tid >> 1, c0w = (tid & 1) * 32;
+            const float4* src = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + wrow) * D + c0w);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 x0 = __ldg(src + 2 * c), x1 = __ldg(src + 2 * c + 1);
+                const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                float hi[8], lo[8];
+                split_bf16(x, hi, lo);
+                put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
+                put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
+            }
+        }
+        //     my W1 buffer a is free once the MMAs of unit k - 2 have read it; then arm the receive
+        //     barriers and tell the peers they may push (into recv and into W1 buffer a)
+        bool ok = mbar_wait(&s.w_empty[a], (n & 1u) ^ 1u, ab);
+        if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
+        if (multi && tid == 0) {
+            ++s.recv_armed;
+            mbar_arrive_expect_tx(&s.recv_full, (uint32_t)((p.CS - 1) * (rb1 - rb0) * D * 4));
+            mbar_arrive_expect_tx(&s.w1_full, (uint32_t)((D - (rb1 - rb0)) * 128));
+            for (int pr = 0; pr < p.CS; ++pr)
+                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
+        }
+        // (1) my phase-1 accumulator, and every peer ready for this exchange (then my earlier pushes,
+        //     which read gb and W1, have landed)
+        ok = mbar_wait(&s.pacc_full[a], n & 1u, ab);
+        if (multi) ok = ok && mbar_wait_cluster(&s.peer_free, (uint32_t)k & 1u, ab);
+        if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
+        __syncwarp();
+        tc_fence_after();
+        // (2) accumulator rows: G (r < 64) as bf16 hi / lo B operands; C (r >= 64) stays in registers
+        float v[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColPacc + a * 64u + (uint32_t)(j * 16) + lane_off, v[j]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s.pacc_empty[a]);                        // the MMA lane may start unit k + 2
+        if (!has_p1) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[j][e] = 0.f;
+        }
+        if (!p.dot) {
+            if (r < D) {                                      // G is symmetric: row r of G = column r
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float hi[8], lo[8];
+                    split_bf16(&v[c / 2][(c & 1) * 8], hi, lo);
+                    put_bf16_chunk(bhi, r, c, hi);
+                    put_bf16_chunk(blo, r, c, lo);
+                }
+            }
+            fence_proxy_async_smem();                         // the operands are read by the tensor cores
+            named_bar_sync(kBarX, 128);
+            // (3) D = [W0_hi ; W0_lo] (G_hi + G_lo) (M = 128, N = 64, K = 64 twice)
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t sa = smem_u32(s.a01), sh = smem_u32(bhi), sl = smem_u32(blo);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(tmem + kColProd, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sh + kk * 32, 16, 1024),
+                                kIdescP2, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(tmem + kColProd, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sl + kk * 32, 16, 1024),
+                                kIdescP2, 1u);
+                mma_commit(&s.prod_bar);
+            }
+            ok = mbar_wait(&s.prod_bar, (uint32_t)k & 1u, ab);
+            if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
+            __syncwarp();
+            tc_fence_after();
+            // (4) P = D[0:64] + D[64:128] - C into gb (the G operands are consumed)
+            float dd[4][16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColProd + (uint32_t)(j * 16) + lane_off, dd[j]);
+            tmem_ld_wait();
+            tc_fence_before();
+            if (r >= D) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    *gc_chunk(pb, r - D, c) = make_float4(dd[c / 4][(c % 4) * 4] - v[c / 4][(c % 4) * 4],
+                                                          dd[c / 4][(c % 4) * 4 + 1] - v[c / 4][(c % 4) * 4 + 1],
+                                                          dd[c / 4][(c % 4) * 4 + 2] - v[c / 4][(c % 4) * 4 + 2],
+                                                          dd[c / 4][(c % 4) * 4 + 3] - v[c / 4][(c % 4) * 4 + 3]);
+            }
+            named_bar_sync(kBarX, 128);
+            if (r < D) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    float4* x = gc_chunk(pb, r, c);
+                    const float4 l = *x;
+                    *x = make_float4(dd[c / 4][(c % 4) * 4] + l.x, dd[c / 4][(c % 4) * 4 + 1] + l.y,
+                                     dd[c / 4][(c % 4) * 4 + 2] + l.z, dd[c / 4][(c % 4) * 4 + 3] + l.w);
+                }
+            }
+        } else if (r >= D) {
+            // dot-product loss: P = C
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *gc_chunk(pb, r - D, c) = make_float4(v[c / 4][(c % 4) * 4], v[c / 4][(c % 4) * 4 + 1],
+                                                      v[c / 4][(c % 4) * 4 + 2], v[c / 4][(c % 4) * 4 + 3]);
+        }
+        // (5) reduce-scatter: block j of my P into CTA j's receive slot for my rank
+        if (multi) {
+            fence_proxy_async_smem();                         // P is read next by the bulk-copy engine
+            named_bar_sync(kBarX, 128);
+            if (tid == 0)
+                for (int pr = 0; pr < p.CS; ++pr) {
+                    if (pr == rank) continue;
+                    const int b0 = split_lo(D, pr, p.CS), b1 = split_lo(D, pr + 1, p.CS);
+                    const int slot = (rank < pr) ? rank : rank - 1;   // my slot in the peer's receive area
+                    bulk_s2cluster(map_to_rank(smem_u32(s.recv + slot * slot_rows * D * 4), (uint32_t)pr),
+                                   reinterpret_cast<const uint8_t*>(pb) + b0 * D * 4, (uint32_t)((b1 - b0) * D * 4),
+                                   map_to_rank(smem_u32(&s.recv_full), (uint32_t)pr));
+                }
+            ok = mbar_wait_cluster(&s.recv_full, (uint32_t)k & 1u, ab);
+        } else {
+            named_bar_sync(kBarX, 128);
+        }
+        if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
+        // (6) my rows of W1 = W0 - eta_scale sum_r P_r (ranks in order); thread tid: row rb0 + tid / 8,
+        //     columns 8 (tid % 8) .. + 8; W1_out rows from their owner
+        for (int i = rb0 + (tid >> 3); i < rb1; i += 16) {
+            const int c8 = tid & 7;
+            float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int pr = 0; pr < p.CS; ++pr) {
+                const float* src = (pr == rank)
+                    ? pb + i * D
+                    : reinterpret_cast<const float*>(s.recv + ((pr < rank) ? pr : pr - 1) * slot_rows * D * 4) + (i - rb0) * D;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c = 2 * c8 + hh;                    // 16-byte chunk of columns 4c .. 4c+3
+                    const float4 x = reinterpret_cast<const float4*>(src)[c ^ (i & 15)];
+                    sum[4 * hh] += x.x; sum[4 * hh + 1] += x.y; sum[4 * hh + 2] += x.z; sum[4 * hh + 3] += x.w;
+                }
+            }
+            float w1[8];
+            const float4* w0 = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + i) * D + 8 * c8);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const float4 w = __ldg(w0 + hh);
+                w1[4 * hh] = w.x - p.eta_scale * sum[4 * hh];
+                w1[4 * hh + 1] = w.y - p.eta_scale * sum[4 * hh + 1];
+                w1[4 * hh + 2] = w.z - p.eta_scale * sum[4 * hh + 2];
+                w1[4 * hh + 3] = w.w - p.eta_scale * sum[4 * hh + 3];
+            }
+            if (p.W1_out) {
+                float4* o = reinterpret_cast<float4*>(p.W1_out + ((size_t)u * D + i) * D + 8 * c8);
+                o[0] = make_float4(w1[0], w1[1], w1[2], w1[3]);
+                o[1] = make_float4(w1[4], w1[5], w1[6], w1[7]);
+            }
+            put_bf16_chunk(s.w1[a], i, c8, w1);
+        }
+        fence_proxy_async_smem();                             // W1 rows: read by the tensor cores and
+        named_bar_sync(kBarX, 128);                           // by the bulk-copy engine
+        // (7) all-gather: my rows of W1 into every peer's W1 buffer a; then wait for theirs
+        if (multi) {
+            if (tid == 0)
+                for (int pr = 0; pr < p.CS; ++pr) {
+                    if (pr == rank) continue;
+                    bulk_s2cluster(map_to_rank(smem_u32(s.w1[a] + rb0 * 128), (uint32_t)pr), s.w1[a] + rb0 * 128,
+                                   (uint32_t)((rb1 - rb0) * 128), map_to_rank(smem_u32(&s.w1_full), (uint32_t)pr));
+                }
+            ok = mbar_wait_cluster(&s.w1_full, (uint32_t)k & 1u, ab);
+            if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
+        }
+        if (tid == 0) mbar_arrive(&s.w_full[a]);
+    }
+    // Final handshake: once every peer has finished its last exchange, all pushes from this CTA have
+    // landed and nobody will push into it again.
     if (multi && !failed) {
-        named_bar_sync(1, 128);
+        named_bar_sync(kBarX, 128);
         if (tid == 0)
             for (int pr = 0; pr < p.CS; ++pr)
                 if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
-        mbar_wait_cluster(&s.peer_free, k & 1u, ab);
+        mbar_wait_cluster(&s.peer_free, (uint32_t)k & 1u, ab);
     }
-    if (tid == 0) {
-        bulk_wait<0>();
-        if (!p.dot) {                                         // the product MMAs this thread issued
-            mma_commit(&s.pdrain_bar);
-            mbar_drain(&s.pdrain_bar, 0u, ab.limit);
-        }
+    if (tid == 0 && !p.dot && k > 0) {                       // the product MMAs this thread issued
+        mma_commit(&s.pdrain_bar);
+        mbar_drain(&s.pdrain_bar, 0u, ab.limit);
     }
 }
 
@@ -582,13 +651,16 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         s.abort_flag = 0;
         s.recv_armed = 0;
         for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
-        mbar_init(&s.drain_bar, 1); mbar_init(&s.pdrain_bar, 1);
-        mbar_init(&s.pacc_full, 1); mbar_init(&s.pacc_empty, 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.pacc_full[i], 1); mbar_init(&s.pacc_empty[i], 128);
+            mbar_init(&s.w_full[i], 1); mbar_init(&s.w_empty[i], 1);
+        }
         for (int i = 0; i < ACC; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
-        mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
         mbar_init(&s.prod_bar, 1);
         mbar_init(&s.recv_full, 1);
+        mbar_init(&s.w1_full, 1);
         mbar_init(&s.peer_free, (uint32_t)(p.CS > 1 ? p.CS - 1 : 1));
+        mbar_init(&s.drain_bar, 1); mbar_init(&s.pdrain_bar, 1);
         fence_barrier_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
     }
@@ -603,8 +675,7 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const uint32_t tmem = s.tmem_base;
 
     // Lane 0 of warps 0 and 1 carries the producer and MMA roles; the rest of each warp waits for it
-    // here, so that every warp reaches the block barrier below converged (a block barrier reached by
-    // a partly diverged warp does not hold the warp's other lanes).
+    // here, so that every warp reaches the block barrier below converged.
     if (warp == 0) {
         if (lane == 0) cl_producer(s, p, &tmK, &tmV, &tmQ, rank, cid, ncl, ab);
         __syncwarp();
@@ -616,8 +687,10 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             mbar_drain(&s.drain_bar, 0u, ab.limit);
         }
         __syncwarp();
+    } else if (warp < 6) {
+        cl_zepi(s, p, tmem, &tmZ, rank, cid, ncl, ab);
     } else {
-        cl_epilogue(s, p, tmem, &tmZ, rank, cid, ncl, ab);
+        cl_xepi(s, p, tmem, rank, cid, ncl, ab);
     }
 
     tc_fence_before();
@@ -626,7 +699,10 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         // No CTA leaves while a peer may still push into it: every CTA of the cluster gets here after
         // issuing its last push, and then each waits (bounded) for the pushes it was promised to land.
         cluster_sync_all();
-        if (threadIdx.x == 0 && s.recv_armed > 0) mbar_drain(&s.recv_full, (s.recv_armed - 1) & 1u, ab.limit);
+        if (threadIdx.x == 0 && s.recv_armed > 0) {
+            mbar_drain(&s.recv_full, (s.recv_armed - 1) & 1u, ab.limit);
+            mbar_drain(&s.w1_full, (s.recv_armed - 1) & 1u, ab.limit);
+        }
         __syncthreads();
     }
     if (warp == 1) {
@@ -858,11 +934,20 @@ ttt_status launch_linear(const Call& c) {
     if (c.dtype == TTT_BF16) {
         const size_t smem = sizeof(ClusterSmem) + 1024;
         cudaFuncSetAttribute(lin_cluster_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        // CTAs per cluster: spread each unit over up to kMaxCluster SMs while every cluster stays
-        // co-resident (clusters never wait on one another, but a second wave would double the time).
-        int cs = (int)std::max<long long>(1, std::min<long long>(kMaxCluster, c.num_sms / std::max<long long>(1, units)));
-        while (cs > 1 && max_active_clusters(cs, smem) < (int)std::min<long long>(units, c.num_sms / cs)) --cs;
-        const int ncl = (int)std::min<long long>(units, cs == 1 ? c.num_sms : c.num_sms / cs);
+        // CTAs per cluster (cs) and clusters (ncl): every cluster co-resident (a second wave would
+        // double the time), and the least streaming per CTA: the most units a cluster takes, over cs.
+        // A cluster with one unit cannot hide its exchange behind another unit's streaming, which
+        // costs about a quarter of a unit's time; a tie goes to the larger cluster.
+        int cs = 1, ncl = (int)std::min<long long>(units, std::max(1, c.num_sms));
+        double best = 1e30;
+        for (int k = 1; k <= kMaxCluster; ++k) {
+            const long long n = std::min<long long>(units, c.num_sms / k);
+            if (n < 1) break;
+            if (k > 1 && max_active_clusters(k, smem) < n) continue;
+            const long long upc = (units + n - 1) / n;
+            const double score = (double)upc / k * (upc == 1 ? 1.25 : 1.0);
+            if (score <= best) { best = score; cs = k; ncl = (int)((units + upc - 1) / upc); }
+        }
         ClusterParams p{};
         p.heads = c.heads;
         p.U = (int)units;
