@@ -3,7 +3,7 @@
 // Oral | 清華+阿里發布ViT3", Observation 2) written in Gram form:
 //     G = sum_n k_n k_n^T,   C = sum_n v_n k_n^T,   W1 = W0 - eta (2/N) (W0 G - C),   z_n = W1 q_n.
 //
-// bf16 path (lin_cluster_bf16): one thread-block cluster of CS <= 4 CTAs (one CTA per SM) per group
+// bf16 path (lin_cluster_bf16): one thread-block cluster of CS <= 8 CTAs (one CTA per SM) per group
 // of units; each CTA takes a 1/CS share of every unit's tokens.
 //   Phase 1: each CTA streams its share of the unit's 128-token K/V tiles (TMA, 128-byte swizzle) and
 //     accumulates [K | V]^T K  (128 x 64 fp32: rows 0..63 = G, rows 64..127 = C) in tensor memory with
@@ -12,11 +12,12 @@
 //   Exchange: each CTA turns its own partial (G_r, C_r) into P_r = W0 G_r - C_r.  The product runs
 //     on the tensor cores with both operands split into bf16 hi + lo parts (M = 128 rows
 //     [W0_hi ; W0_lo], B = G_hi and then G_lo), so that it carries about 16 mantissa bits, close to
-//     fp32.  P_r (16 KB) is pushed with one bulk copy into every other CTA of the cluster (distributed
-//     shared memory, completion counted on the receiver's mbarrier); each CTA then forms
-//     W1 = W0 - eta (2/N) sum_r P_r, summing in rank order (a fixed order: bitwise deterministic),
-//     and rounds W1 once to bf16 into a shared-memory B operand of phase 2.  No global-memory
-//     round trip, no grid-wide wait.
+//     fp32.  Then a reduce-scatter and an all-gather over distributed shared memory: CTA j owns a
+//     block of about 64 / CS rows of W1; every CTA pushes block j of its P_r into CTA j with one bulk
+//     copy (completion counted on the receiver's mbarrier), CTA j sums its blocks in rank order (a
+//     fixed order: bitwise deterministic), forms those rows of W1 = W0 - eta (2/N) sum_r P_r rounded
+//     once to bf16, and pushes them into every peer's phase-2 B operand.  No global-memory round
+//     trip, no grid-wide wait.
 //   Phase 2: the CTA streams its share of 256-token Q tiles and writes Z = Q W1^T: A = Q tile
 //     (M = 128 tokens, K-major), B = W1 (K-major); the epilogue drains tensor memory to bf16 and
 //     stores Z with TMA.
@@ -184,8 +185,8 @@ __device__ void merge_unit(const MergeOut& m, int u, int h, size_t slot0, int ns
 constexpr int STAGES = 4;                   // 32 KB each: a K+V tile pair, or one 256-token Q tile
 constexpr int ACC = 4;                      // phase-2 accumulators (64 columns each)
 constexpr int Q2 = 256;                     // tokens per phase-2 stage
-constexpr int kMaxCluster = 4;
-constexpr int kRecvBytes = 12288;           // the peers' rows of my P block: (CS - 1) x ceil(64 / CS) x 256 B
+constexpr int kMaxCluster = 8;             // the portable limit
+constexpr int kRecvBytes = 15360;           // the peers' rows of my P block: (CS - 1) x ceil(64 / CS) x 256 B, CS <= 8
 constexpr uint32_t kColPacc = 0;            // tensor memory: two phase-1 accumulators,
 constexpr uint32_t kColAcc = 128;           //   ACC phase-2 accumulators,
 constexpr uint32_t kColProd = 384;          //   the W0 G product (448 of 512 columns)
@@ -418,13 +419,60 @@ __device__ __forceinline__ void cl_zepi(ClusterSmem& s, const ClusterParams& p, 
     if (tid == 0) bulk_wait<0>();
 }
 
+// The product's A operand [bf16(W0) ; bf16(W0 - bf16(W0))] (rows 0..63, 64..127): each exchange
+// thread fetches row wrow, columns c0w .. c0w + 31 of W0 into registers, and later writes its share.
+__device__ __forceinline__ void load_w0_share(const ClusterParams& p, int h, int wrow, int c0w, float4 (&wa)[8]) {
+    const float4* src = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + wrow) * D + c0w);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) wa[c] = __ldg(src + c);
+}
+__device__ __forceinline__ void put_w0_share(ClusterSmem& s, int wrow, int c0w, const float4 (&wa)[8]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float x[8] = {wa[2 * c].x, wa[2 * c].y, wa[2 * c].z, wa[2 * c].w,
+                            wa[2 * c + 1].x, wa[2 * c + 1].y, wa[2 * c + 1].z, wa[2 * c + 1].w};
+        float hi[8], lo[8];
+        split_bf16(x, hi, lo);
+        put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
+        put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
+    }
+}
+
+// Where row i of P goes: this CTA's pb (own = true), or the owner's receive slot for this rank (same
+// chunk swizzle as pb), counted on the owner's recv_full.
+struct PRowDst {
+    bool own;
+    uint32_t row, bar;                       // shared::cluster addresses of the row and of the barrier
+};
+__device__ __forceinline__ PRowDst p_row_dst(ClusterSmem& s, const ClusterParams& p, int rank, int i) {
+    int o = 0;
+    while (o + 1 < p.CS && split_lo(D, o + 1, p.CS) <= i) ++o;
+    PRowDst d;
+    d.own = o == rank;
+    const int slot_rows = (D + p.CS - 1) / p.CS;
+    const int slot = (rank < o) ? rank : rank - 1;
+    d.row = d.own ? 0u
+                  : map_to_rank(smem_u32(s.recv) + (uint32_t)((slot * slot_rows + i - split_lo(D, o, p.CS)) * D * 4),
+                                (uint32_t)o);
+    d.bar = d.own ? 0u : map_to_rank(smem_u32(&s.recv_full), (uint32_t)o);
+    return d;
+}
+// Chunk c (columns 4c .. 4c+3) of row i of P to its destination.
+__device__ __forceinline__ void put_p_chunk(const PRowDst& d, float* pb, int i, int c, float4 v) {
+    if (d.own) *gc_chunk(pb, i, c) = v;
+    else st_async_f4(d.row + (uint32_t)((c ^ (i & 15)) << 4), v, d.bar);
+}
+
 // Warps 6..9: the cluster exchange of every unit in turn.  Each CTA turns its partial (G_r, C_r) into
 // P_r = W0 G_r - C_r on the tensor cores (both operands split into bf16 hi + lo: about 16 mantissa
 // bits).  Rows of W1 are then formed in blocks, one per CTA (rank j owns rows [64 j / CS, 64 (j+1) / CS)):
-// every CTA pushes block j of its P into CTA j (reduce-scatter), sums the blocks it receives for its
-// own rows in rank order (a fixed order: bitwise deterministic), forms those rows of
-// W1 = W0 - eta (2/N) sum_r P_r rounded once to bf16 into the unit's W1 operand, and pushes them into
-// the same place in every peer's operand (all-gather).
+// the thread holding row i of P stores it straight into the receive slot of the row's owner
+// (reduce-scatter), the owner sums the rows it receives in rank order (a fixed order: bitwise
+// deterministic), forms its rows of W1 = W0 - eta (2/N) sum_r P_r rounded once to bf16 into the unit's
+// W1 operand, and stores them into the same place in every peer's operand (all-gather).  All
+// transfers are st.async stores whose bytes the receiver's mbarrier counts: no bulk-copy queue (busy
+// with the streaming loads) and no release fence on the way.  W0 for the next unit's product and for
+// this unit's W1 rows is fetched while the peers' rows are in flight.
 __device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, uint32_t tmem, int rank, int cid,
                                         int ncl, const Abort& ab) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -434,34 +482,27 @@ __device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, 
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool multi = p.CS > 1;
     const int m = units_of(p, cid, ncl);
-    float* pb = reinterpret_cast<float*>(s.gb);               // P (fp32 64 x 64, swizzled chunks)
+    float* pb = reinterpret_cast<float*>(s.gb);               // my rows of P (fp32, swizzled chunks)
     uint8_t* bhi = s.gb;
     uint8_t* blo = s.gb + D * D * 2;
     const bool has_p1 = split_lo(p.tpu1, rank + 1, p.CS) > split_lo(p.tpu1, rank, p.CS);
     const int rb0 = split_lo(D, rank, p.CS), rb1 = split_lo(D, rank + 1, p.CS);   // my block of rows
     const int slot_rows = (D + p.CS - 1) / p.CS;                                  // rows per receive slot
+    // this thread's share of the product's A operand: row wrow of W0, columns c0w .. c0w + 31
+    const int wrow = tid >> 1, c0w = (tid & 1) * 32;
+    float4 wa[8];
+    if (!p.dot && m > 0) {
+        load_w0_share(p, cid % p.heads, wrow, c0w, wa);
+        put_w0_share(s, wrow, c0w, wa);
+    }
     int k = 0;
     bool failed = false;
     for (; k < m; ++k) {
         const int u = cid + k * ncl;
         const int h = u % p.heads;
         const uint32_t a = (uint32_t)k & 1u, n = (uint32_t)k >> 1;
-        // (0) the A operand of the product: rows 0..63 = bf16(W0), rows 64..127 = bf16(W0 - bf16(W0))
-        if (!p.dot) {
-            const int wrow = tid >> 1, c0w = (tid & 1) * 32;
-            const float4* src = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + wrow) * D + c0w);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4 x0 = __ldg(src + 2 * c), x1 = __ldg(src + 2 * c + 1);
-                const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                float hi[8], lo[8];
-                split_bf16(x, hi, lo);
-                put_bf16_chunk(s.a01, wrow, c0w / 8 + c, hi);
-                put_bf16_chunk(s.a01, D + wrow, c0w / 8 + c, lo);
-            }
-        }
-        //     my W1 buffer a is free once the MMAs of unit k - 2 have read it; then arm the receive
-        //     barriers and tell the peers they may push (into recv and into W1 buffer a)
+        // (0) my W1 buffer a is free once the MMAs of unit k - 2 have read it; then arm the receive
+        //     barriers and tell the peers they may store into recv and into W1 buffer a
         bool ok = mbar_wait(&s.w_empty[a], (n & 1u) ^ 1u, ab);
         if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
         if (multi && tid == 0) {
@@ -469,37 +510,37 @@ __device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, 
             mbar_arrive_expect_tx(&s.recv_full, (uint32_t)((p.CS - 1) * (rb1 - rb0) * D * 4));
             mbar_arrive_expect_tx(&s.w1_full, (uint32_t)((D - (rb1 - rb0)) * 128));
             for (int pr = 0; pr < p.CS; ++pr)
-                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
+                if (pr != rank) mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
         }
-        // (1) my phase-1 accumulator, and every peer ready for this exchange (then my earlier pushes,
-        //     which read gb and W1, have landed)
+        // (1) my phase-1 accumulator, and every peer ready for this exchange
         ok = mbar_wait(&s.pacc_full[a], n & 1u, ab);
         if (multi) ok = ok && mbar_wait_cluster(&s.peer_free, (uint32_t)k & 1u, ab);
         if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
         __syncwarp();
         tc_fence_after();
-        // (2) accumulator rows: G (r < 64) as bf16 hi / lo B operands; C (r >= 64) stays in registers
-        float v[4][16];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColPacc + a * 64u + (uint32_t)(j * 16) + lane_off, v[j]);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&s.pacc_empty[a]);                        // the MMA lane may start unit k + 2
-        if (!has_p1) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[j][e] = 0.f;
-        }
+        // (2) accumulator rows 0..63 (G, warps 8 and 9) as bf16 hi / lo B operands; rows 64..127 (C)
+        //     stay in tensor memory until P is formed
+        const uint32_t pacc = tmem + kColPacc + a * 64u + lane_off;
         if (!p.dot) {
             if (r < D) {                                      // G is symmetric: row r of G = column r
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int j = 0; j < 4; ++j) {
+                    float g[16];
+                    tmem_ld16(pacc + (uint32_t)(j * 16), g);
+                    tmem_ld_wait();
+                    if (!has_p1)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) g[e] = 0.f;
                     float hi[8], lo[8];
-                    split_bf16(&v[c / 2][(c & 1) * 8], hi, lo);
-                    put_bf16_chunk(bhi, r, c, hi);
-                    put_bf16_chunk(blo, r, c, lo);
+                    split_bf16(g, hi, lo);
+                    put_bf16_chunk(bhi, r, 2 * j, hi);
+                    put_bf16_chunk(blo, r, 2 * j, lo);
+                    split_bf16(g + 8, hi, lo);
+                    put_bf16_chunk(bhi, r, 2 * j + 1, hi);
+                    put_bf16_chunk(blo, r, 2 * j + 1, lo);
                 }
+                tc_fence_before();
+                mbar_arrive(&s.pacc_empty[a]);
             }
             fence_proxy_async_smem();                         // the operands are read by the tensor cores
             named_bar_sync(kBarX, 128);
@@ -521,58 +562,86 @@ __device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, 
             if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
             __syncwarp();
             tc_fence_after();
-            // (4) P = D[0:64] + D[64:128] - C into gb (the G operands are consumed)
-            float dd[4][16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColProd + (uint32_t)(j * 16) + lane_off, dd[j]);
-            tmem_ld_wait();
-            tc_fence_before();
+            // (4) P = D[0:64] + D[64:128] - C: warps 6, 7 (rows 64..127: the lo half, and C from the
+            //     phase-1 accumulator) put D_lo - C into pb, then warps 8, 9 (rows 0..63) complete
+            //     their rows in registers and send them (the G operands in gb are consumed); 16
+            //     columns at a time
             if (r >= D) {
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    *gc_chunk(pb, r - D, c) = make_float4(dd[c / 4][(c % 4) * 4] - v[c / 4][(c % 4) * 4],
-                                                          dd[c / 4][(c % 4) * 4 + 1] - v[c / 4][(c % 4) * 4 + 1],
-                                                          dd[c / 4][(c % 4) * 4 + 2] - v[c / 4][(c % 4) * 4 + 2],
-                                                          dd[c / 4][(c % 4) * 4 + 3] - v[c / 4][(c % 4) * 4 + 3]);
-            }
-            named_bar_sync(kBarX, 128);
-            if (r < D) {
+                for (int j = 0; j < 4; ++j) {
+                    float dd[16], c16[16];
+                    tmem_ld16(tmem + kColProd + lane_off + (uint32_t)(j * 16), dd);
+                    tmem_ld16(pacc + (uint32_t)(j * 16), c16);
+                    tmem_ld_wait();
+                    if (!has_p1)
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    float4* x = gc_chunk(pb, r, c);
-                    const float4 l = *x;
-                    *x = make_float4(dd[c / 4][(c % 4) * 4] + l.x, dd[c / 4][(c % 4) * 4 + 1] + l.y,
-                                     dd[c / 4][(c % 4) * 4 + 2] + l.z, dd[c / 4][(c % 4) * 4 + 3] + l.w);
-                }
-            }
-        } else if (r >= D) {
-            // dot-product loss: P = C
+                        for (int e = 0; e < 16; ++e) c16[e] = 0.f;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                *gc_chunk(pb, r - D, c) = make_float4(v[c / 4][(c % 4) * 4], v[c / 4][(c % 4) * 4 + 1],
-                                                      v[c / 4][(c % 4) * 4 + 2], v[c / 4][(c % 4) * 4 + 3]);
-        }
-        // (5) reduce-scatter: block j of my P into CTA j's receive slot for my rank
-        if (multi) {
-            fence_proxy_async_smem();                         // P is read next by the bulk-copy engine
-            named_bar_sync(kBarX, 128);
-            if (tid == 0)
-                for (int pr = 0; pr < p.CS; ++pr) {
-                    if (pr == rank) continue;
-                    const int b0 = split_lo(D, pr, p.CS), b1 = split_lo(D, pr + 1, p.CS);
-                    const int slot = (rank < pr) ? rank : rank - 1;   // my slot in the peer's receive area
-                    bulk_s2cluster(map_to_rank(smem_u32(s.recv + slot * slot_rows * D * 4), (uint32_t)pr),
-                                   reinterpret_cast<const uint8_t*>(pb) + b0 * D * 4, (uint32_t)((b1 - b0) * D * 4),
-                                   map_to_rank(smem_u32(&s.recv_full), (uint32_t)pr));
+                    for (int c = 0; c < 4; ++c)
+                        *gc_chunk(pb, r - D, 4 * j + c) = make_float4(dd[4 * c] - c16[4 * c], dd[4 * c + 1] - c16[4 * c + 1],
+                                                                      dd[4 * c + 2] - c16[4 * c + 2],
+                                                                      dd[4 * c + 3] - c16[4 * c + 3]);
                 }
-            ok = mbar_wait_cluster(&s.recv_full, (uint32_t)k & 1u, ab);
+                tc_fence_before();
+                mbar_arrive(&s.pacc_empty[a]);                // the MMA lane may start unit k + 2
+                named_bar_sync(kBarX, 128);
+            } else {
+                const PRowDst dst = p_row_dst(s, p, rank, r);
+                named_bar_sync(kBarX, 128);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float x[16];
+                    tmem_ld16(tmem + kColProd + lane_off + (uint32_t)(j * 16), x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float4 l = *gc_chunk(pb, r, 4 * j + c);
+                        put_p_chunk(dst, pb, r, 4 * j + c,
+                                    make_float4(x[4 * c] + l.x, x[4 * c + 1] + l.y, x[4 * c + 2] + l.z, x[4 * c + 3] + l.w));
+                    }
+                }
+                tc_fence_before();
+            }
         } else {
-            named_bar_sync(kBarX, 128);
+            // dot-product loss: P = C, sent by the threads of rows 64..127
+            if (r >= D) {
+                const PRowDst dst = p_row_dst(s, p, rank, r - D);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float x[16];
+                    tmem_ld16(pacc + (uint32_t)(j * 16), x);
+                    tmem_ld_wait();
+                    if (!has_p1)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) x[e] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        put_p_chunk(dst, pb, r - D, 4 * j + c, make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&s.pacc_empty[a]);
         }
+        // (5) W0 for my rows of W1 (the first two passes: all of them when CS > 1), fetched while the
+        //     rows travel
+        float4 w0r[2][2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = rb0 + (tid >> 3) + 16 * j;
+            if (i < rb1) {
+                const float4* w0 = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + i) * D + 8 * (tid & 7));
+                w0r[j][0] = __ldg(w0);
+                w0r[j][1] = __ldg(w0 + 1);
+            }
+        }
+        if (multi) ok = mbar_wait_cluster(&s.recv_full, (uint32_t)k & 1u, ab);
         if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
-        // (6) my rows of W1 = W0 - eta_scale sum_r P_r (ranks in order); thread tid: row rb0 + tid / 8,
-        //     columns 8 (tid % 8) .. + 8; W1_out rows from their owner
-        for (int i = rb0 + (tid >> 3); i < rb1; i += 16) {
+        // (6) my rows of W1 = W0 - eta_scale sum_r P_r (ranks in order); thread tid: row rb0 + tid / 8
+        //     (+ 16 j), columns 8 (tid % 8) .. + 8; W1_out rows from their owner
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = rb0 + (tid >> 3) + 16 * j;
+            if (i >= rb1) continue;
             const int c8 = tid & 7;
             float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             for (int pr = 0; pr < p.CS; ++pr) {
@@ -587,10 +656,10 @@ __device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, 
                 }
             }
             float w1[8];
-            const float4* w0 = reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + i) * D + 8 * c8);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const float4 w = __ldg(w0 + hh);
+                const float4 w = j < 2 ? w0r[j < 2 ? j : 0][hh]
+                                       : __ldg(reinterpret_cast<const float4*>(p.W0 + ((size_t)h * D + i) * D + 8 * c8) + hh);
                 w1[4 * hh] = w.x - p.eta_scale * sum[4 * hh];
                 w1[4 * hh + 1] = w.y - p.eta_scale * sum[4 * hh + 1];
                 w1[4 * hh + 2] = w.z - p.eta_scale * sum[4 * hh + 2];
@@ -601,30 +670,37 @@ __device__ __forceinline__ void cl_xepi(ClusterSmem& s, const ClusterParams& p, 
                 o[0] = make_float4(w1[0], w1[1], w1[2], w1[3]);
                 o[1] = make_float4(w1[4], w1[5], w1[6], w1[7]);
             }
-            put_bf16_chunk(s.w1[a], i, c8, w1);
+            uint4 pk;
+            pk.x = pack_bf16x2(w1[0], w1[1]); pk.y = pack_bf16x2(w1[2], w1[3]);
+            pk.z = pack_bf16x2(w1[4], w1[5]); pk.w = pack_bf16x2(w1[6], w1[7]);
+            const uint32_t off = (uint32_t)(i * 128 + ((c8 ^ (i & 7)) << 4));   // 128-byte swizzled K-major
+            *reinterpret_cast<uint4*>(s.w1[a] + off) = pk;
+            for (int pr = 0; pr < p.CS; ++pr)
+                if (pr != rank)
+                    st_async_u4(map_to_rank(smem_u32(s.w1[a]) + off, (uint32_t)pr), pk,
+                                map_to_rank(smem_u32(&s.w1_full), (uint32_t)pr));
         }
-        fence_proxy_async_smem();                             // W1 rows: read by the tensor cores and
-        named_bar_sync(kBarX, 128);                           // by the bulk-copy engine
-        // (7) all-gather: my rows of W1 into every peer's W1 buffer a; then wait for theirs
+        // (7) the next unit's product operand when its head differs (the product of this unit has read
+        //     a01); then my W1 rows and the peers' rows, once landed, go to the tensor cores
+        if (!p.dot && k + 1 < m && (cid + (k + 1) * ncl) % p.heads != h) {
+            load_w0_share(p, (cid + (k + 1) * ncl) % p.heads, wrow, c0w, wa);
+            put_w0_share(s, wrow, c0w, wa);
+        }
+        fence_proxy_async_smem();
         if (multi) {
-            if (tid == 0)
-                for (int pr = 0; pr < p.CS; ++pr) {
-                    if (pr == rank) continue;
-                    bulk_s2cluster(map_to_rank(smem_u32(s.w1[a] + rb0 * 128), (uint32_t)pr), s.w1[a] + rb0 * 128,
-                                   (uint32_t)((rb1 - rb0) * 128), map_to_rank(smem_u32(&s.w1_full), (uint32_t)pr));
-                }
             ok = mbar_wait_cluster(&s.w1_full, (uint32_t)k & 1u, ab);
-            if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
+            fence_proxy_async_smem();                         // rows stored by the peers, now observed here
         }
+        if (named_bar_or(kBarX, 128, !ok)) { failed = true; break; }
         if (tid == 0) mbar_arrive(&s.w_full[a]);
     }
-    // Final handshake: once every peer has finished its last exchange, all pushes from this CTA have
-    // landed and nobody will push into it again.
+    // Final handshake: once every peer has finished its last exchange, nobody stores into this CTA
+    // again (each CTA's own stores are then known to have landed: every receiver waited for them).
     if (multi && !failed) {
         named_bar_sync(kBarX, 128);
         if (tid == 0)
             for (int pr = 0; pr < p.CS; ++pr)
-                if (pr != rank) mbar_arrive_remote(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
+                if (pr != rank) mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s.peer_free), (uint32_t)pr));
         mbar_wait_cluster(&s.peer_free, (uint32_t)k & 1u, ab);
     }
     if (tid == 0 && !p.dot && k > 0) {                       // the product MMAs this thread issued
@@ -943,10 +1019,11 @@ ttt_status launch_linear(const Call& c) {
         for (int k = 1; k <= kMaxCluster; ++k) {
             const long long n = std::min<long long>(units, c.num_sms / k);
             if (n < 1) break;
-            if (k > 1 && max_active_clusters(k, smem) < n) continue;
             const long long upc = (units + n - 1) / n;
+            const long long need = (units + upc - 1) / upc;
+            if (k > 1 && max_active_clusters(k, smem) < need) continue;
             const double score = (double)upc / k * (upc == 1 ? 1.25 : 1.0);
-            if (score <= best) { best = score; cs = k; ncl = (int)((units + upc - 1) / upc); }
+            if (score <= best) { best = score; cs = k; ncl = (int)need; }
         }
         ClusterParams p{};
         p.heads = c.heads;

@@ -218,6 +218,25 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
+// The same arrival without release semantics: for a signal that orders no memory writes of this
+// thread (a cluster-scope release waits for all of the thread's outstanding memory operations, which
+// costs microseconds while the SM streams from HBM).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// Asynchronous 16-byte store into a peer CTA's shared memory (addresses from map_to_rank); the
+// peer's mbarrier `bar_caddr` counts the bytes when they land (complete_tx), so the receiver learns
+// of the data by waiting on that barrier, without a fence on the sender's side.
+__device__ __forceinline__ void st_async_f4(uint32_t caddr, float4 v, uint32_t bar_caddr) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(caddr),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar_caddr)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_u4(uint32_t caddr, uint4 v, uint32_t bar_caddr) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(caddr),
+                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_caddr)
+                 : "memory");
+}
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 __device__ __forceinline__ bool mbar_test_cluster(uint32_t addr, uint32_t parity) {
     uint32_t ok;
