@@ -53,9 +53,8 @@ def test_workspace_sizes(lib):
     assert 40 * 64 * 64 * 4 < nf < 16 << 20           # fp32: counters, W1 and partial slots
     nc = capi.ttt_workspace_bytes(capi.TTT_HEAD_DWCONV, s)
     # conv: header, control words (done, 40 unit counters, 40 ready flags) padded to 256 B,
-    # then per unit room for one task per row pair (39) x 3 compute groups of 576-float partials,
-    # then W1 per unit
-    assert nc == 256 + 512 + 40 * 39 * 3 * 576 * 4 + 40 * 576 * 4
+    # then per unit room for one task per row pair (39) of 576-float partials, then W1 per unit
+    assert nc == 256 + 512 + 40 * 39 * 576 * 4 + 40 * 576 * 4
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(d=32)) == 0
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, _shape(batch=0)) == 0
     assert capi.ttt_workspace_bytes(7, s) == 0
@@ -64,7 +63,7 @@ def test_workspace_sizes(lib):
 def test_layer_workspace_sizes(lib):
     s = _shape(heads=6)
     # the linear range's workspace (bf16: the error word), then the conv range's (8 units)
-    assert capi.ttt_layer_workspace_bytes(s, 1) == 256 + (256 + 256 + 8 * 39 * 3 * 576 * 4 + 8 * 576 * 4)
+    assert capi.ttt_layer_workspace_bytes(s, 1) == 256 + (256 + 256 + 8 * 39 * 576 * 4 + 8 * 576 * 4)
     assert capi.ttt_layer_workspace_bytes(s, 0) == 256
     assert capi.ttt_layer_workspace_bytes(s, 6) == capi.ttt_workspace_bytes(capi.TTT_HEAD_DWCONV, s)
     assert capi.ttt_layer_workspace_bytes(s, 7) == 0

@@ -27,12 +27,14 @@
 //     and a 4 x 3 register window slides along the columns (unrolled by 3, so the window never moves
 //     between registers), fed by explicit shared-memory loads.  The residual is carried negated
 //     (s = V - W0 (*) K, from the negated taps), which saves a negation per token.
-//   Merge: each group folds its warps' 64 x 9 sums in a fixed order into its partial for the task,
-//     written to the workspace slot of (unit, task, group).  The group that writes a unit's last
-//     partial sums all of the unit's partials in slot order -- a fixed order, so W1 is bitwise
-//     reproducible whichever CTA ran which task (for a given grid) -- writes W1 and raises the unit's
-//     ready flag; the readout of the unit's tasks waits for that flag (bounded).  Z is written
-//     straight from registers (128 coalesced bytes per token and warp).
+//   Merge: each group folds its warps' 64 x 9 sums in a fixed order, the CTA adds the three groups'
+//     sums in group order into the task's partial, written to the workspace slot of (unit, task).
+//     The CTA that writes a unit's last partial sums all of the unit's partials with all its compute
+//     threads (three slices of tasks, each summed in task order with its loads in flight at once, then
+//     the slices in order: a fixed order, so W1 is bitwise reproducible whichever CTA ran which task,
+//     for a given grid), writes W1 and raises the unit's ready flag; the readout of the unit's tasks
+//     waits for that flag (bounded).  Z is written straight from registers (128 coalesced bytes per
+//     token and warp).
 //   The last CTA to finish returns the workspace's counters and flags to zero for the next call.
 //   When launched as a programmatic dependent of the preceding kernel (the linear heads of the same
 //   layer), the kernel starts while that kernel runs and, at its very end, waits for it, so the
@@ -56,6 +58,7 @@ constexpr int NV = 4;                       // V ring slots (2-row groups)
 constexpr int kPart = D * TAPS;             // 576 floats: a 64 x 9 gradient or kernel, tap-major
 constexpr int kRed = (GW + 1) / 2;          // a group's per-warp gradients are folded pairwise into kRed slots
 constexpr int kTasksPerCta = 1;             // tasks a launch aims for per CTA
+constexpr uint32_t kComputeBar = 4;         // named barrier of all compute warps (groups use 1..3)
 
 template <typename T>
 struct Elem;
@@ -100,7 +103,7 @@ struct Params {
     uint32_t* done;                  // CTAs finished
     uint32_t* unit_count;            // [U] gradient partials written per unit
     uint32_t* ready;                 // [U] 1 once the unit's W1 is formed
-    float* partials;                 // [U][mtpu][CG][576] negated gradient sums per task and group, tap-major
+    float* partials;                 // [U][mtpu][576] negated gradient sums per task, tap-major
     int mtpu;                        // partial slots per unit (one task per row pair, the most a call uses)
     float* w1g;                      // [U][576] W1 per unit, tap-major
     unsigned long long wait_ns;      // bound of every device-side wait
@@ -115,7 +118,7 @@ static WsLayout ws_layout(long long U, int tpu) {
     WsLayout l;
     l.ctl = kWsHeader;
     l.partials = l.ctl + align_up((size_t)(1 + 2 * U) * 4, 256);
-    l.w1g = l.partials + align_up((size_t)U * tpu * CG * kPart * 4, 256);
+    l.w1g = l.partials + align_up((size_t)U * tpu * kPart * 4, 256);
     l.total = l.w1g + (size_t)U * kPart * 4;
     return l;
 }
@@ -123,7 +126,6 @@ static WsLayout ws_layout(long long U, int tpu) {
 struct SmemTail {                            // follows the rings
     float red[CG][kRed][kPart];              // per-warp gradients of each group, folded pairwise
     uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV];
-    int flag[CG];                            // per-group decision broadcast
     int last;
     int abort_flag;
 };
@@ -422,9 +424,10 @@ dw_band(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtenso
                 }
             }
             kq += (uint32_t)n + 1; vq += (uint32_t)n;
-            // the group stops on a failure anywhere in it (a uniform decision)
-            if (named_bar_or(gbar, GW * 32, failed)) { failed = true; break; }
-            // ---- the group's partial, summed over its warps in a fixed order
+            // every compute warp stops on a failure anywhere in the CTA (a uniform decision: the
+            // groups meet at CTA-wide barriers below)
+            if (named_bar_or(kComputeBar, CW * 32, failed)) { failed = true; break; }
+            // ---- the group's partial, summed over its warps in a fixed order, into red[grp][0]
             float(*red)[kPart] = s.red[grp];
             if (seg >= kRed) {                                       // warps kRed.. store, warps 0.. add
 #pragma unroll
@@ -442,48 +445,65 @@ dw_band(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtenso
                 }
             }
             named_bar_sync(gbar, GW * 32);
-            float* part = p.partials + (((size_t)tk.u * p.mtpu + tk.r) * CG + grp) * kPart;
             for (int e = gtid; e < kPart; e += GW * 32) {
                 float acc = 0.f;
 #pragma unroll
                 for (int ww = 0; ww < kRed; ++ww) acc += red[ww][e];
-                part[e] = acc;
+                red[0][e] = acc;                                     // this thread's own element only
             }
+            // ---- the task's partial: the three groups' partials in group order (all compute warps
+            //      of the CTA take the same tasks in the same order, so they meet here once per task)
+            named_bar_sync(kComputeBar, CW * 32);
+            float* part = p.partials + ((size_t)tk.u * p.mtpu + tk.r) * kPart;
+            for (int e = tid; e < kPart; e += CW * 32)
+                part[e] = (s.red[0][0][e] + s.red[1][0][e]) + s.red[2][0][e];
             __threadfence();
-            named_bar_sync(gbar, GW * 32);
-            if (gtid == 0) s.flag[grp] = (atomicAdd(p.unit_count + tk.u, 1u) == (uint32_t)(g.tpu * CG - 1)) ? 1 : 0;
-            named_bar_sync(gbar, GW * 32);
-            if (s.flag[grp]) {
+            named_bar_sync(kComputeBar, CW * 32);
+            if (tid == 0) s.last = (atomicAdd(p.unit_count + tk.u, 1u) == (uint32_t)(g.tpu - 1)) ? 1 : 0;
+            named_bar_sync(kComputeBar, CW * 32);
+            if (s.last) {
                 // ---- the unit's last partial: W1 = W0 - eta (2/N) g = W0 + eta_scale * (sum of the
-                //      partials in (task, group) order)
+                //      unit's task partials in task order).  Thread (e4, sl) sums slice sl of the tasks
+                //      (about a third, all loads in flight), then the slices are added in order.
                 __threadfence();
-                const float* pu = p.partials + (size_t)tk.u * p.mtpu * CG * kPart;
-                const int R = g.tpu * CG;
-                for (int e4 = gtid; e4 < kPart / 4; e4 += GW * 32) {
+                const float* pu = p.partials + (size_t)tk.u * p.mtpu * kPart;
+                const int R = g.tpu;
+                constexpr int kE4 = kPart / 4;                       // 144 float4 per partial
+                float4* sl_sum = reinterpret_cast<float4*>(&s.red[1][0][0]);   // [3][144] (red[1], red[2] free)
+                const int e4 = tid % kE4, sl = tid / kE4;
+                if (sl < 3) {
+                    const int r0 = split_lo(R, sl, 3), r1 = split_lo(R, sl + 1, 3);
                     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int r0 = 0; r0 < R; r0 += 8) {                // 8 loads in flight, added in order
+                    for (int rb = r0; rb < r1; rb += 8) {            // 8 loads in flight, added in order
                         float4 v[8];
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
-                            v[q] = (r0 + q < R) ? __ldcg(reinterpret_cast<const float4*>(pu + (size_t)(r0 + q) * kPart) + e4)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                            v[q] = (rb + q < r1) ? __ldcg(reinterpret_cast<const float4*>(pu + (size_t)(rb + q) * kPart) + e4)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
-                            if (r0 + q < R) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
+                            if (rb + q < r1) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
                     }
-                    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+                    sl_sum[sl * kE4 + e4] = acc;
+                }
+                named_bar_sync(kComputeBar, CW * 32);
+                if (tid < kE4) {
+                    const float4 x0 = sl_sum[tid], x1 = sl_sum[kE4 + tid], x2 = sl_sum[2 * kE4 + tid];
+                    const float a4[4] = {(x0.x + x1.x) + x2.x, (x0.y + x1.y) + x2.y, (x0.z + x1.z) + x2.z,
+                                         (x0.w + x1.w) + x2.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int e = 4 * e4 + i, t9 = e / D, ch = e % D;   // tap-major index
+                        const int e = 4 * tid + i, t9 = e / D, ch = e % D;   // tap-major index
                         const float w1 = __ldg(p.W0 + ((size_t)h * D + ch) * TAPS + t9) + p.eta_scale * a4[i];
                         p.w1g[(size_t)tk.u * kPart + e] = w1;
                         if (p.W1_out) p.W1_out[((size_t)tk.u * D + ch) * TAPS + t9] = w1;
                     }
                 }
                 __threadfence();
-                named_bar_sync(gbar, GW * 32);
-                if (gtid == 0) st_release_gpu(p.ready + tk.u, 1u);
+                named_bar_sync(kComputeBar, CW * 32);
+                if (tid == 0) st_release_gpu(p.ready + tk.u, 1u);
             }
+            named_bar_sync(kComputeBar, CW * 32);                    // s.last and red are reused by the next task
         }
         // ---- phase 2 of every task of this CTA: Z = W1 (*) Q over this group's row pairs
         for (int t = blockIdx.x; t < p.T && !failed; t += gridDim.x) {
