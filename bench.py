@@ -1,15 +1,17 @@
-"""Benchmark of the TTT-layer forward on B200.
+"""Benchmark of the TTT layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
-One step = one forward of the whole layer over one batch: for the default workload
-(mixed6084_bf16: 8 images x 6 heads x 78x78 = 6084 tokens, d = 64, bf16, eta = 0.5) the five linear
-heads and the depthwise-conv head, i.e. the Gram/cross accumulation, the deterministic merge and
-update, and the readout of every head.  --workload mixed6084_dot_bf16 runs the same layer trained
-with the dot-product inner loss (eta = 1.0).  Inputs are synthetic (seeded, the pages' shapes and
-distributions) and already resident in HBM when the timed region starts; three input sets of
-149.5 MB each (more than the 126 MB L2) are rotated so every step reads cold data.  Steps are replayed
-from CUDA graphs (one graph per input set) and timed with CUDA events on the launching stream.
+One step = one pass of the hot path over one batch.  For the default workload (mixed6084_bf16:
+8 images x 6 heads x 78x78 = 6084 tokens, d = 64, bf16, eta = 0.5) that is one ttt_forward_layer call:
+the five linear heads and the depthwise-conv head, i.e. the Gram/cross accumulation, the
+deterministic merge and update, and the readout of every head.  The other workloads time their own
+entry point (linear heads alone, the MLP head, the dense 3x3 conv head, the mini-batch variant, the
+backward passes).  Inputs are synthetic (seeded, the pages' shapes and distributions) and already
+resident in HBM when the timed region starts; enough input sets are rotated that together they exceed
+twice the 126 MB L2, so every step reads cold data.  Steps are replayed from CUDA graphs (each graph
+holds a run of consecutive steps over the rotating sets) and timed with CUDA events on the launching
+stream; a second pass times single-step replays one by one for the p10 / p50 / p90 spread.
 
 Metric: token*heads per second (B * heads * N per step), whole job over all ranks.  Under torchrun
 every rank runs the same per-GPU workload on its own GPU (weak scaling; no data-path collective).
@@ -18,7 +20,9 @@ every rank runs the same per-GPU workload on its own GPU (weak scaling; no data-
 host's cores for the same workload, metric and unit.
 """
 import argparse
+import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -34,34 +38,99 @@ import torch  # noqa: E402
 from vision_test_token_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "TTT-layer fwd tokens*heads/s at 6084 tokens"
-METRIC_BWD = "TTT-layer bwd (linear heads) tokens*heads/s at 6084 tokens"
+METRIC_BWD = "TTT-layer bwd tokens*heads/s"
 UNIT = "token*heads/s"
-# dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures summarised under
-# profiles/.  Valid only for the kernel builds those captures were taken on: an entry is removed
-# whenever its kernel changes.  Mixed layer: the two kernels of one step, summed.
-STEP_TRAFFIC = {"mixed6084_bf16": (93.597184e6 + 3.062272e6) + (18.751488e6 + 0.0),   # profiles/traffic_mixed6084_bf16.md
-                "mixed6084_dot_bf16": (93.595904e6 + 4.063488e6) + (18.747392e6 + 0.002816e6)}
-                # profiles/layer_kernels_mixed6084_dot_bf16.md
-MLP_TRAFFIC = {"mlp1024_bf16": 25.809664e6 + 0.0}                                   # profiles/mlp_fused_mlp1024.md
+L2_BYTES = 126 * 2 ** 20
+
+# DRAM traffic per launch (dram__bytes_read.sum, dram__bytes_write.sum) from ncu, keyed by workload,
+# with the hash of the kernel sources the capture was taken on (kernel_source_hash below).  An entry
+# whose hash differs from the running build's is stale and is not reported.  Captured with
+# --cache-control none on the third of three consecutive steps, so that the previous step's Z
+# write-back (which lands during the next step) is counted as it is in steady state.
+TRAFFIC = {}
+
+# Kernels of this library launched per step, by workload kind (bf16; fp32 where it differs).
+LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backward": 3, "backward_conv": 4,
+                     "backward_mlp": 7, "conv3x3": 3}
+LAUNCHES_PER_STEP_FP32 = {"linear": 2, "mixed": 3}
 
 
-def parse():
+def kernel_source_hash():
+    """sha256 over the CUDA sources and headers of the library (sorted by name)."""
+    d = os.path.join(ROOT, "vision_test_token_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mixed6084_bf16", choices=sorted(WORKLOADS))
-    ap.add_argument("--sets", type=int, default=3, help="rotating input sets (total must exceed L2)")
+    ap.add_argument("--sets", type=int, default=0,
+                    help="rotating input sets (0: enough that together they exceed twice the L2)")
+    ap.add_argument("--graph-steps", type=int, default=30, help="consecutive steps captured in one CUDA graph")
+    ap.add_argument("--spread-reps", type=int, default=200, help="single-step replays timed one by one")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-oracle", action="store_true", help="skip the CPU-oracle baseline leg")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def workload_bytes(w):
+    """Algorithmic HBM bytes per step: every input token row read once and every output row written
+    once (forward: Q, K, V in, Z out; backward: Q, K, V, dZ in, dQ, dK, dV out)."""
     esz = 2 if w.dtype == "bf16" else 4
     units = w.batch * w.heads
-    return 4 * units * w.N * w.d * esz          # read Q, K, V once, write Z once
+    rows = 7 if w.kind.startswith("backward") else 4
+    return rows * units * w.N * w.d * esz
+
+
+def workload_flops(w):
+    """Algorithmic FLOPs per step for the kinds whose bound is arithmetic (None otherwise).
+      conv3x3: three 9-tap d x d contractions per token (residual, gradient, readout): 54 d^2.
+      mlp: seven d x 4d products per token (five in the inner step, two in the readout).
+      backward (linear): 14 d^2 per token (G, C, dW1; dq, dk, dv maps).
+      backward_conv: eight 9-tap sums per token and channel (r, g, dW1, dq, dr, two dk terms, dW0).
+      backward_mlp: 23 d x 4d products per token (5 in the step, 5 through the readout, 13 back
+        through the step), as the chain rule is written out.
+      minibatch: 6 d^2 + 4 b d per token."""
+    n = w.batch * w.heads * w.N
+    d = w.d
+    hid = getattr(w, "hidden_ratio", 4) * d
+    if w.kind == "conv3x3":
+        return n * 54 * d * d
+    if w.kind == "mlp":
+        return n * 7 * 2 * d * hid
+    if w.kind == "backward":
+        return n * 14 * d * d
+    if w.kind == "backward_conv":
+        return n * 8 * 9 * 2 * d
+    if w.kind == "backward_mlp":
+        return n * 23 * 2 * d * hid
+    if w.kind == "minibatch":
+        return n * (6 * d * d + 4 * w.mb_tokens * d)
+    return None
+
+
+MAX_SETS = 64
+
+
+def default_sets(w, cap_bytes=6 << 30):
+    """Rotating input sets: at least 3, and enough that together they exceed twice the L2 (within
+    cap_bytes of device memory and MAX_SETS).  A workload too small for that (its sets together stay
+    within 2 x L2) is timed step by step with the L2 flushed between steps instead."""
+    per = max(1, workload_bytes(w))
+    return int(max(3, min(math.ceil(2 * L2_BYTES / per), cap_bytes // per, MAX_SETS)))
+
+
+def needs_flush(w, n_sets):
+    return n_sets * workload_bytes(w) <= 2 * L2_BYTES
 
 
 def peaks():
@@ -181,40 +250,42 @@ def _np64(t):
     return t.detach().cpu().double().numpy()
 
 
-def oracle_units(w, x, units, threads):
-    """Runs the oracle on the listed (image, head) units of the workload (inputs already float64)."""
+def oracle_units(w, x, images, threads, heads=None):
+    """Runs the oracle on `images` whole images of the workload (inputs already float64; image i of x
+    is used for i < x's batch, then again from the start), on the heads in range `heads` (lo, hi), or
+    all heads."""
     import oracle
-    if w.kind == "backward":
-        for (b, h) in units:
-            sl = (slice(b, b + 1), slice(h, h + 1))
-            oracle.linear_backward(x["Q"][sl], x["K"][sl], x["V"][sl], x["W0_lin"][h:h + 1], w.eta, x["dZ"][sl],
-                                   threads=threads)
-        return
-    if w.kind == "minibatch":
-        for (b, h) in units:
-            oracle.linear_minibatch(x["Q"][b:b + 1, h:h + 1], x["K"][b:b + 1, h:h + 1], x["V"][b:b + 1, h:h + 1],
-                                    x["W0_lin"][h:h + 1], w.eta, w.mb_tokens, w.mb_mode, threads=threads)
-        return
-    if w.kind == "mlp":
-        for (b, h) in units:
-            oracle.mlp(x["Q"][b:b + 1, h:h + 1], x["K"][b:b + 1, h:h + 1], x["V"][b:b + 1, h:h + 1],
-                       x["Wa"][h:h + 1], x["Wb"][h:h + 1], w.eta, threads=threads)
-        return
-    nl = w.lin_heads
-    imgs = sorted({b for b, _ in units})
-    for b in imgs:
-        hs = [h for bb, h in units if bb == b]
-        lin = [h for h in hs if h < nl]
-        conv = [h for h in hs if h >= nl]
+    lo, hi = heads if heads else (0, w.heads)
+    nb = x["Q"].shape[0]
+    idx = [i % nb for i in range(images)]
+    take = lambda k, a, b: x[k][idx][:, a:b]
+    if w.kind == "mixed":
+        nl = w.lin_heads
         lin_fn, conv_fn = (oracle.linear_dot, oracle.dwconv_dot) if w.loss == "dot" else (oracle.linear, oracle.dwconv)
-        if lin:
-            lo, hi = min(lin), max(lin) + 1
-            lin_fn(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
-                   x["W0_lin"][lo:hi], w.eta, threads=threads)
-        if conv:
-            lo, hi = min(conv), max(conv) + 1
-            conv_fn(x["Q"][b:b + 1, lo:hi], x["K"][b:b + 1, lo:hi], x["V"][b:b + 1, lo:hi],
-                    x["W0_conv"][lo - nl:hi - nl], w.eta, w.H, w.W, threads=threads)
+        if lo < nl:
+            a, b = lo, min(hi, nl)
+            lin_fn(take("Q", a, b), take("K", a, b), take("V", a, b), x["W0_lin"][a:b], w.eta, threads=threads)
+        if hi > nl:
+            a, b = max(lo, nl), hi
+            conv_fn(take("Q", a, b), take("K", a, b), take("V", a, b), x["W0_conv"][a - nl:b - nl], w.eta, w.H, w.W,
+                    threads=threads)
+        return
+    Q, K, V = take("Q", lo, hi), take("K", lo, hi), take("V", lo, hi)
+    if w.kind == "backward":
+        oracle.linear_backward(Q, K, V, x["W0_lin"][lo:hi], w.eta, take("dZ", lo, hi), threads=threads)
+    elif w.kind == "backward_conv":
+        oracle.dwconv_backward(Q, K, V, x["W0_conv"][lo:hi], w.eta, take("dZ", lo, hi), w.H, w.W, threads=threads)
+    elif w.kind == "backward_mlp":
+        oracle.mlp_backward(Q, K, V, x["Wa"][lo:hi], x["Wb"][lo:hi], w.eta, take("dZ", lo, hi), threads=threads)
+    elif w.kind == "conv3x3":
+        oracle.conv3x3(Q, K, V, x["W0_c3"][lo:hi], w.eta, w.H, w.W, threads=threads)
+    elif w.kind == "minibatch":
+        oracle.linear_minibatch(Q, K, V, x["W0_lin"][lo:hi], w.eta, w.mb_tokens, w.mb_mode, threads=threads)
+    elif w.kind == "mlp":
+        oracle.mlp(Q, K, V, x["Wa"][lo:hi], x["Wb"][lo:hi], w.eta, threads=threads)
+    else:                                                    # linear heads only
+        fn = oracle.linear_dot if w.loss == "dot" else oracle.linear
+        fn(Q, K, V, x["W0_lin"][lo:hi], w.eta, threads=threads)
 
 
 def oracle_inputs(w, x, images):
@@ -222,30 +293,51 @@ def oracle_inputs(w, x, images):
             if k not in ("Z", "grads")}
 
 
-def time_oracle(w, x, budget_s=12.0):
-    """cpu_baseline: whole images of the workload (all heads, OpenMP over units) until budget_s."""
-    import oracle
-    threads = oracle.default_threads()
-    xs = oracle_inputs(w, x, 1)
-    units = [(0, h) for h in range(w.heads)]
-    t0 = time.perf_counter()
-    reps = 0
+def _time_oracle_leg(w, x, images, threads, budget_s):
+    reps, t0 = 0, time.perf_counter()
     while True:
-        oracle_units(w, xs, units, threads)
+        oracle_units(w, x, images, threads)
         reps += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
-            break
-    return {"value": len(units) * w.N * reps / el, "unit": UNIT, "cores": min(threads, len(units)),
-            "kind": "oracle",
-            "sample": f"image 0 of {w.name} ({w.heads} heads x {w.N} tokens) repeated {reps} times, "
-                      f"{el:.1f} s, fp64, OpenMP over the {len(units)} (image, head) units"}
+            return images * w.heads * w.N * reps / el, reps, el
+
+
+def time_oracle(w, x, budget_s=10.0, single_budget_s=6.0):
+    """cpu_baseline: the fp64 oracle on this host's cores.  All-core: enough whole images that their
+    (image, head) units occupy every core of os.sched_getaffinity (images of the workload's batch,
+    reused when the batch has fewer), OpenMP over the units.  Single-core: one image, one thread."""
+    import oracle
+    cores = oracle.default_threads()
+    images = max(1, math.ceil(cores / w.heads))
+    xs = oracle_inputs(w, x, min(images, x["Q"].shape[0]))
+    v_all, reps, el = _time_oracle_leg(w, xs, images, cores, budget_s)
+    v_one, reps1, el1 = _time_oracle_leg(w, xs, 1, 1, single_budget_s)
+    return {"value": v_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{images} image(s) of {w.name} ({images * w.heads} (image, head) units of {w.N} tokens) "
+                      f"repeated {reps} times in {el:.1f} s, fp64, OpenMP over the units on {cores} cores",
+            "single_core": {"value": v_one, "unit": UNIT, "cores": 1,
+                            "sample": f"1 image of {w.name} ({w.heads} units) repeated {reps1} times in "
+                                      f"{el1:.1f} s, one thread"}}
+
+
+def config_of(w, world):
+    """The config object of a bench line (the same keys for both arms)."""
+    cfg = {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads,
+           "lin_heads": w.lin_heads, "conv_heads": w.conv_heads, "grid": [w.H, w.W], "tokens": w.N, "d": w.d,
+           "eta": w.eta, "loss": w.loss, "kind": w.kind, "parallelism": f"batch-sharded x{world}"}
+    if w.kind == "minibatch":
+        cfg.update({"mb_tokens": w.mb_tokens, "mb_mode": w.mb_mode})
+    if w.kind in ("mlp", "backward_mlp"):
+        cfg["hidden"] = w.hidden_ratio * w.d
+    return cfg
 
 
 def run_reference(args):
-    """The reference arm: the fp64 oracle on this host's cores.  One step = one image of the
-    workload (all heads), or one (image, head) unit per step when K whole images would not finish
-    within about two and a half minutes."""
+    """The reference arm: the fp64 oracle on this host's cores, on the same workload, metric and unit.
+    One step = one whole image of the workload (all heads, OpenMP over them), or one (image, head)
+    unit per step, heads in turn, when K whole images would not finish within about two and a half
+    minutes.  Under torchrun rank 0 alone runs; the other ranks exit without work."""
     import oracle
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -254,30 +346,28 @@ def run_reference(args):
     w = WORKLOADS[args.workload]
     x = oracle_inputs(w, make_inputs(w, seed=0), 1)
     threads = oracle.default_threads()
-    all_units = [(0, h) for h in range(w.heads)]
     t0 = time.perf_counter()
-    oracle_units(w, x, all_units, threads)                  # warm-up: one whole image
+    oracle_units(w, x, 1, threads)                           # warm-up: one whole image
     t_img = time.perf_counter() - t0
     per_image = args.steps * t_img <= 150.0
-    for _ in range(max(0, min(args.warmup, 3) - 1)):
-        oracle_units(w, x, all_units if per_image else all_units[:1], threads)
+    step_heads = (lambda i: None) if per_image else (lambda i: (i % w.heads, i % w.heads + 1))
+    for i in range(max(0, min(args.warmup, 3) - 1)):
+        oracle_units(w, x, 1, threads, step_heads(i))
     t0 = time.perf_counter()
     th = 0
     for i in range(args.steps):
-        units = all_units if per_image else [all_units[i % len(all_units)]]
-        oracle_units(w, x, units, threads)
-        th += len(units) * w.N
+        oracle_units(w, x, 1, threads, step_heads(i))
+        th += (w.heads if per_image else 1) * w.N
     el = time.perf_counter() - t0
     value = th / el
+    used = min(threads, w.heads) if per_image else 1
     sample = (f"{'one image (' + str(w.heads) + ' heads)' if per_image else 'one (image, head) unit, heads in turn'}"
               f" of {w.name} per step, {args.steps} steps, {el:.1f} s, fp64")
-    cb = {"value": value, "unit": UNIT, "kind": "oracle", "cores": min(threads, w.heads if per_image else 1),
-          "sample": sample}
-    line = {"impl": "reference", "metric": METRIC_BWD if w.kind == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(1, args.steps) * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads, "tokens": w.N, "d": w.d,
-                       "eta": w.eta, "loss": w.loss, "device": "host CPU"},
+    cb = {"value": value, "unit": UNIT, "kind": "oracle", "cores": used, "sample": sample}
+    line = {"impl": "reference", "metric": METRIC_BWD if w.kind.startswith("backward") else METRIC, "value": value,
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / max(1, args.steps) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_of(w, world), "device": "host CPU",
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -286,24 +376,48 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------------
-def make_step(w, xs, dev):
-    """Returns fn(i) running one layer forward on input set i (all device tensors)."""
-    from vision_test_token_b200 import layer
-    weights = {k: v for k, v in xs[0].items() if k.startswith("W")}
+def alloc_outputs(w, x, dev):
+    """Output buffers of one input set: Z for the forward kinds, the gradient tuple for the backward
+    kinds."""
+    if w.kind == "backward":
+        x["grads"] = (torch.empty_like(x["Q"]), torch.empty_like(x["Q"]), torch.empty_like(x["Q"]),
+                      torch.empty((w.heads, w.d, w.d), device=dev), torch.empty(1, device=dev))
+    elif w.kind == "backward_conv":
+        x["grads"] = (torch.empty_like(x["Q"]), torch.empty_like(x["Q"]), torch.empty_like(x["Q"]),
+                      torch.empty((w.heads, w.d, 3, 3), device=dev), torch.empty(1, device=dev))
+    elif w.kind == "backward_mlp":
+        hid = w.hidden_ratio * w.d
+        x["grads"] = (torch.empty_like(x["Q"]), torch.empty_like(x["Q"]), torch.empty_like(x["Q"]),
+                      torch.empty((w.heads, hid, w.d), device=dev), torch.empty((w.heads, w.d, hid), device=dev),
+                      torch.empty(1, device=dev))
+    else:
+        x["Z"] = torch.empty_like(x["Q"])
 
-    def step(i):
-        x = xs[i]
-        if w.kind == "mlp":
-            layer.forward_mlp(x["Q"], x["K"], x["V"], weights["Wa"], weights["Wb"], w.eta, w.H, w.W, Z=x["Z"])
-        elif w.kind == "minibatch":
-            layer.forward_linear_minibatch(x["Q"], x["K"], x["V"], weights["W0_lin"], w.eta, w.H, w.W, w.mb_tokens,
-                                           w.mb_mode, Z=x["Z"])
-        elif w.kind == "backward":
-            layer.backward_linear(x["Q"], x["K"], x["V"], weights["W0_lin"], w.eta, w.H, w.W, x["dZ"], out=x["grads"])
-        else:
-            layer.forward_layer(x["Q"], x["K"], x["V"], weights, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=x["Z"],
-                                loss=w.loss)
-    return step
+
+def run_step(w, x, d=None, out=None):
+    """One step of the workload through the public Python API: inputs from x (or d, a dict of
+    device tensors with the same keys), outputs into x's buffers (or out)."""
+    from vision_test_token_b200 import layer
+    d = x if d is None else d
+    if out is None:
+        out = x["grads"] if w.kind.startswith("backward") else x["Z"]
+    Q, K, V = d["Q"], d["K"], d["V"]
+    if w.kind == "mlp":
+        layer.forward_mlp(Q, K, V, d["Wa"], d["Wb"], w.eta, w.H, w.W, Z=out)
+    elif w.kind == "minibatch":
+        layer.forward_linear_minibatch(Q, K, V, d["W0_lin"], w.eta, w.H, w.W, w.mb_tokens, w.mb_mode, Z=out)
+    elif w.kind == "conv3x3":
+        layer.forward_conv3x3(Q, K, V, d["W0_c3"], w.eta, w.H, w.W, Z=out)
+    elif w.kind == "backward":
+        layer.backward_linear(Q, K, V, d["W0_lin"], w.eta, w.H, w.W, d["dZ"], out=out)
+    elif w.kind == "backward_conv":
+        layer.backward_dwconv(Q, K, V, d["W0_conv"], w.eta, w.H, w.W, d["dZ"], out=out)
+    elif w.kind == "backward_mlp":
+        layer.backward_mlp(Q, K, V, d["Wa"], d["Wb"], w.eta, w.H, w.W, d["dZ"], out=out)
+    elif w.kind == "linear":
+        layer.forward_linear(Q, K, V, d["W0_lin"], w.eta, w.H, w.W, Z=out, loss=w.loss)
+    else:
+        layer.forward_layer(Q, K, V, d, w.eta, w.H, w.W, conv_heads=w.conv_heads, Z=out, loss=w.loss)
 
 
 def capture(fn, stream):
@@ -313,15 +427,52 @@ def capture(fn, stream):
     return g
 
 
-def time_graphs(graphs, steps, stream):
+def capture_steps(w, xs, first, count, stream):
+    """One CUDA graph holding `count` consecutive steps over the rotating input sets, from set
+    `first`."""
+    def fn():
+        for i in range(count):
+            run_step(w, xs[(first + i) % len(xs)])
+    return capture(fn, stream)
+
+
+def replay(plan, stream):
+    """Replays a list of (graph, times) on `stream` between two CUDA events; returns seconds."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         start.record(stream)
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        for g, times in plan:
+            for _ in range(times):
+                g.replay()
         end.record(stream)
     end.synchronize()
     return start.elapsed_time(end) / 1e3
+
+
+def time_graphs(graphs, steps, stream):
+    return replay([(graphs[i % len(graphs)], 1) for i in range(steps)], stream)
+
+
+def time_steps(graphs, reps, stream, flush=None):
+    """Single-step replays timed one by one (events around each replay, issued back to back, read
+    after the last); with `flush` (a device buffer larger than the L2) it is overwritten between
+    steps, outside the timed intervals.  Returns the per-step times in microseconds."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for i, (a, b) in enumerate(evs):
+            if flush is not None:
+                flush.fill_(float(i % 7))
+            a.record(stream)
+            graphs[i % len(graphs)].replay()
+            b.record(stream)
+    evs[-1][1].synchronize()
+    return [a.elapsed_time(b) * 1e3 for a, b in evs]
+
+
+def spread_of(us):
+    us = sorted(us)
+    q = lambda f: us[min(len(us) - 1, int(f * len(us)))]
+    return {"p10_us": q(0.1), "p50_us": q(0.5), "p90_us": q(0.9), "reps": len(us)}
 
 
 def time_calls_alone(w, xs, stream, n):
@@ -348,186 +499,189 @@ def time_calls_alone(w, xs, stream, n):
     return out[0], out[1]
 
 
+def traffic_entry(w):
+    """The DRAM traffic capture of this workload, if it was taken on the running kernel sources."""
+    e = TRAFFIC.get(w.name)
+    if not e:
+        return None, "no ncu capture for this workload"
+    if e["src_sha"] != kernel_source_hash():
+        return None, f"stale: the capture was taken on kernel sources {e['src_sha']}, not on this build"
+    return e, None
+
+
+def fp32_peak_tflops(mhz):
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def roofline(w, t_step, pk, clocks, xs, stream, args):
+    """The roofline block of the step: HBM-bound kinds against the measured copy bandwidth,
+    contractions against the measured bf16 tensor peak, plain FP32 FMA paths against the FP32 peak
+    derived from the SM count, the FP32 lanes per SM and the SM clock sampled under load."""
+    nbytes, flops = workload_bytes(w), workload_flops(w)
+    hbm = nbytes / t_step / 1e9
+    tr, tr_note = traffic_entry(w)
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    common = {"us_per_launch": t_step * 1e6, "algorithmic_bytes": nbytes,
+              "traffic": (tr["read"] + tr["write"]) if tr else None}
+    if tr:
+        common["traffic_read"], common["traffic_write"] = tr["read"], tr["write"]
+        common["traffic_src_sha"] = tr["src_sha"]
+    else:
+        common["traffic_note"] = tr_note
+    conv_name = "dw_band<bf16, dot>" if w.loss == "dot" else "dw_band<bf16>"
+    if w.kind in ("mixed", "linear"):
+        if w.kind == "mixed":
+            kern = f"layer step: lin_cluster_bf16 and {conv_name} running at the same time (one ttt_forward_layer call)"
+        else:
+            kern = "lin_cluster_bf16 (the whole ttt_forward_linear call)" if w.dtype == "bf16" else \
+                   "lin_p1_f32 + lin_p2_f32 (the whole ttt_forward_linear call)"
+        roof = {"bound": "hbm", "kernel": kern, "achieved": hbm, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm / pk["hbm_gbs"], "peak_source": pk["source"] + " (copy bandwidth)", **common}
+        if w.kind == "mixed":
+            esz = 2 if w.dtype == "bf16" else 4
+            lin_bytes = 4 * w.batch * w.lin_heads * w.N * w.d * esz
+            conv_bytes = 4 * w.batch * w.conv_heads * w.N * w.d * esz
+            t_lin, t_conv = time_calls_alone(w, xs, stream, n=max(200, args.steps // 4))
+            roof["kernels_alone"] = {
+                "lin_cluster_bf16": {"us_per_launch": t_lin * 1e6, "algorithmic_bytes": lin_bytes,
+                                     "achieved_gbs": lin_bytes / t_lin / 1e9,
+                                     "frac": lin_bytes / t_lin / 1e9 / pk["hbm_gbs"]},
+                conv_name: {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
+                            "achieved_gbs": conv_bytes / t_conv / 1e9,
+                            "frac": conv_bytes / t_conv / 1e9 / pk["hbm_gbs"]}}
+        return roof
+    if w.kind in ("mlp", "conv3x3"):
+        kern = "mlp_fused (the whole ttt_forward_mlp call)" if w.kind == "mlp" else \
+               "conv3_grad + conv3_merge + conv3_readout (the whole ttt_forward_conv3x3 call)"
+        tf = flops / t_step / 1e12
+        return {"bound": "tensor", "kernel": kern, "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tf / pk["bf16_tflops"], "peak_source": pk["source"] + " (bf16 burst)",
+                "algorithmic_flops": flops, "hbm_gbs": hbm, "hbm_frac": hbm / pk["hbm_gbs"], **common}
+    names = {"backward": "lin_bwd_p1 + lin_bwd_p2 + lin_bwd_sum (the whole ttt_backward_linear call)",
+             "backward_conv": "cb_reduce + cb_unit + cb_map + cb_final (the whole ttt_backward_dwconv call)",
+             "backward_mlp": "mb_prep .. mb_final, 7 kernels (the whole ttt_backward_mlp call)",
+             "minibatch": "lin_minibatch (the whole ttt_forward_linear_minibatch call)"}
+    peak = fp32_peak_tflops(mhz)
+    tf = flops / t_step / 1e12
+    return {"bound": "alu", "kernel": names[w.kind], "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+            "frac": tf / peak, "peak_source": f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {mhz:.0f} MHz "
+                                                "(median SM clock under load)",
+            "algorithmic_flops": flops, "hbm_gbs": hbm, "hbm_frac": hbm / pk["hbm_gbs"], **common}
+
+
 def run_ours(args):
     world, rank, local = dist_init(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    from vision_test_token_b200 import build as _build, capi, layer
+    from vision_test_token_b200 import build as _build, capi
     _build.build()
     capi.lib()
     w = WORKLOADS[args.workload]
     pk = peaks()
-
     # this rank's images of the global batch (weak scaling: w.batch images per GPU), one input set per
-    # seed; Z buffers, workspaces
+    # seed, with its output buffers
     first, count = shard_batch(w.batch * world, rank, world)
     assert count == w.batch
+    n_sets = args.sets or default_sets(w)
     xs = []
-    for s in range(args.sets):
+    for s in range(n_sets):
         x = make_inputs(w, seed=1000 * first + s, device=dev)
-        x["Z"] = torch.empty_like(x["Q"])
-        if w.kind == "backward":
-            x["grads"] = (torch.empty_like(x["Q"]), torch.empty_like(x["Q"]), torch.empty_like(x["Q"]),
-                          torch.empty((w.heads, w.d, w.d), device=dev), torch.empty(1, device=dev))
+        alloc_outputs(w, x, dev)
         xs.append(x)
     stream = torch.cuda.Stream(device=dev)
-    step = make_step(w, xs, dev)
     with torch.cuda.stream(stream):
         for i in range(3):                      # eager warm-up (workspaces, attributes)
-            step(i % args.sets)
+            run_step(w, xs[i % n_sets])
     stream.synchronize()
-    graphs = [capture(lambda i=i: step(i), stream) for i in range(args.sets)]
+    # graphs: single steps (one per set), and runs of G consecutive steps (G a multiple of the sets)
+    singles = [capture_steps(w, xs, i, 1, stream) for i in range(n_sets)]
+    G = n_sets * max(1, math.ceil(min(args.graph_steps, max(1, args.steps)) / n_sets))
+    run_g = capture_steps(w, xs, 0, G, stream)
+    q, r = divmod(args.steps, G)
+    plan = [(run_g, q)] + ([(capture_steps(w, xs, 0, r, stream), 1)] if r else [])
 
     sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
     sampler.start()
     time.sleep(0.3)
 
-    # warm-up (graph replays), then the timed region
-    time_graphs(graphs, max(3, args.warmup), stream)
+    # warm-up (W single-step replays), then exactly K steps in the timed region: runs of G steps, or,
+    # for a workload whose sets fit in the L2, single steps with the L2 flushed between them (the
+    # flushes outside the timed intervals)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if needs_flush(w, n_sets) else None
+    time_graphs(singles, max(3, args.warmup), stream)
     barrier(world)
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    el = time_graphs(graphs, args.steps, stream)
+    if flush is None:
+        el = replay(plan, stream)
+    else:
+        el = sum(time_steps(singles, args.steps, stream, flush)) / 1e6
     torch.cuda.synchronize(dev)
     barrier(world)
     t_wall1 = time.time()
     el_max = max_over_ranks(el, world, dev)
+    spread = spread_of(time_steps(singles, args.spread_reps, stream, flush))
     # keep the GPU loaded a little longer so the clock record covers the load
     if t_wall1 - t_wall0 < 1.0:
-        soak_steps = min(20000, int(args.steps * (1.2 / max(t_wall1 - t_wall0, 1e-3))))
+        t_est = max((t_wall1 - t_wall0) / max(1, args.steps), 1e-7)
+        soak = max(1, min(2000, math.ceil(1.2 / (t_est * G))))
         t_wall0 = time.time()
-        time_graphs(graphs, soak_steps, stream)
+        replay([(run_g, soak)], stream)
         t_wall1 = time.time()
     time.sleep(0.25)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
 
-    ms_per_step = el_max / args.steps * 1e3
-    th_step = w.token_heads
-    value = th_step * world / (el_max / args.steps)
+    t_step = el_max / args.steps
+    value = w.token_heads * world / t_step
+    roof = roofline(w, t_step, pk, clocks, xs, stream, args)
 
-    # roofline.  Mixed layer: one ttt_forward_layer call runs the linear kernel and the conv kernel at
-    # the same time (they share HBM), so the bound applies to the layer step as a whole: its
-    # algorithmic bytes over its device time.  Each kernel's time when it runs alone on the whole GPU
-    # is given beside it.
-    roof = None
-    if w.kind == "mixed":
-        esz = 2 if w.dtype == "bf16" else 4
-        lin_bytes = 4 * w.batch * w.lin_heads * w.N * w.d * esz
-        conv_bytes = 4 * w.batch * w.conv_heads * w.N * w.d * esz
-        t_lin, t_conv = time_calls_alone(w, xs, stream, n=max(200, args.steps // 4))
-        step_s = el_max / args.steps
-        achieved = workload_bytes(w) / step_s / 1e9
-        conv_name = "dw_band<bf16, dot>" if w.loss == "dot" else "dw_band<bf16>"
-        roof = {"bound": "hbm",
-                "kernel": f"layer step: lin_cluster_bf16 and {conv_name} running at the same time "
-                          "(one ttt_forward_layer call)",
-                "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                "traffic": STEP_TRAFFIC.get(w.name), "peak_source": pk["source"],
-                "algorithmic_bytes": workload_bytes(w), "us_per_launch": step_s * 1e6,
-                "kernels_alone": {
-                    "lin_cluster_bf16": {"us_per_launch": t_lin * 1e6, "algorithmic_bytes": lin_bytes,
-                                         "achieved_gbs": lin_bytes / t_lin / 1e9,
-                                         "frac": lin_bytes / t_lin / 1e9 / pk["hbm_gbs"]},
-                    conv_name: {"us_per_launch": t_conv * 1e6, "algorithmic_bytes": conv_bytes,
-                                       "achieved_gbs": conv_bytes / t_conv / 1e9,
-                                       "frac": conv_bytes / t_conv / 1e9 / pk["hbm_gbs"]}}}
-    elif w.kind == "backward":
-        # plain FP32 FMA kernels: 14 d^2 FLOP per token and head (6 d^2 for G, C, dW1; 8 d^2 for dq, dk,
-        # dv); algorithmic bytes: read Q, K, V, dZ and write dQ, dK, dV once (7 N d elements per unit)
-        n = max(100, args.steps // 4)
-        time_graphs(graphs, 10, stream)
-        t_b = time_graphs(graphs, n, stream) / n
-        flops = w.batch * w.heads * w.N * 14 * w.d * w.d
-        esz = 2 if w.dtype == "bf16" else 4
-        nbytes = 7 * w.batch * w.heads * w.N * w.d * esz
-        mhz = clocks.get("sm_max_mhz") or 1965.0
-        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-        achieved = flops / t_b / 1e12
-        roof = {"bound": "alu", "kernel": "lin_bwd_p1 + lin_bwd_p2 + lin_bwd_sum (the whole ttt_backward_linear call)",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                "peak_source": f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {mhz:.0f} MHz",
-                "algorithmic_flops": flops, "algorithmic_bytes": nbytes, "us_per_launch": t_b * 1e6,
-                "hbm_gbs": nbytes / t_b / 1e9, "hbm_frac": nbytes / t_b / 1e9 / pk["hbm_gbs"]}
-    elif w.kind == "minibatch":
-        # a sequential FP32 recurrence: bound by plain FMA issue, not by HBM.  Algorithmic FLOPs per
-        # (token, head) are the mini-batch TTT terms 6 d^2 + 4 b d; the peak is 148 SMs x 128 FP32
-        # lanes x 2 FLOP per FMA at the SM clock sampled during the run (its maximum if no sample).
-        n = max(100, args.steps // 4)
-        time_graphs(graphs, 10, stream)
-        t_mb = time_graphs(graphs, n, stream) / n
-        flops = w.batch * w.heads * w.N * (6 * w.d * w.d + 4 * w.mb_tokens * w.d)
-        mhz = clocks.get("sm_max_mhz") or 1965.0
-        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-        achieved = flops / t_mb / 1e12
-        roof = {"bound": "alu", "kernel": "lin_minibatch (the whole ttt_forward_linear_minibatch call)",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                "peak_source": f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {mhz:.0f} MHz",
-                "algorithmic_flops": flops, "us_per_launch": t_mb * 1e6,
-                "hbm_gbs": workload_bytes(w) / t_mb / 1e9}
-    elif w.kind == "mlp":
-        n = max(100, args.steps // 4)
-        time_graphs(graphs, 10, stream)
-        t_mlp = time_graphs(graphs, n, stream) / n
-        d, hid = w.d, w.hidden_ratio * w.d
-        flops = w.batch * w.heads * w.N * (2 * d * hid * 5 + 2 * d * hid * 2)   # 5 products in the step, 2 in the readout
-        achieved = flops / t_mlp / 1e12
-        roof = {"bound": "tensor", "kernel": "mlp_fused (the whole ttt_forward_mlp call)", "achieved": achieved,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                "traffic": MLP_TRAFFIC.get(w.name),
-                "peak_source": pk["source"] + " (bf16 burst)", "algorithmic_flops": flops,
-                "us_per_launch": t_mlp * 1e6}
-
-    # end to end through the public API: pinned host inputs -> device -> layer -> host result
+    # end to end through the public API: pinned host inputs -> device -> step -> host result
     e2e = run_e2e(w, xs[0], dev, stream, args.e2e_steps, world)
 
-    line = {"metric": METRIC_BWD if w.kind == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "global_batch": w.batch * world, "heads": w.heads,
-                       "lin_heads": w.lin_heads, "conv_heads": w.conv_heads, "grid": [w.H, w.W],
-                       "tokens": w.N, "d": w.d, "eta": w.eta, "loss": w.loss,
-                       **({"mb_tokens": w.mb_tokens, "mb_mode": w.mb_mode} if w.kind == "minibatch" else {}),
-                       "parallelism": f"batch-sharded x{world}",
-                       "l2": f"{args.sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB (> 126 MB L2)",
-                       "algorithmic_bytes_per_step": workload_bytes(w),
-                       "launch": "CUDA graph per input set" + ("; one ttt_forward_layer call per step: the conv kernel "
-                                                               "launched behind the linear kernel as a programmatic "
-                                                               "dependent, the two running at the same time"
-                                                               if w.kind == "mixed" else "")},
-            "gbs_per_step": workload_bytes(w) / (el_max / args.steps) / 1e9,
-            "gpu_launches": args.steps * (3 if w.kind == "backward" else 2 if (w.kind == "mixed" or w.dtype == "fp32")
-                                          else 1),
-            "clocks": clocks, "e2e": e2e}
-    if roof:
-        line["roofline"] = roof
+    per_step = (LAUNCHES_PER_STEP_FP32 if w.dtype == "fp32" else {}).get(w.kind, LAUNCHES_PER_STEP[w.kind])
+    line = {"metric": METRIC_BWD if w.kind.startswith("backward") else METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": config_of(w, world), "device": torch.cuda.get_device_name(dev),
+            "l2": (f"{n_sets} rotating input sets of {workload_bytes(w) / 1e6:.1f} MB "
+                   f"({n_sets * workload_bytes(w) / 1e6:.0f} MB in all, > 2 x 126 MB L2)") if flush is None else
+                  (f"{n_sets} rotating input sets of {workload_bytes(w) / 1e6:.2f} MB (within the L2): L2 flushed "
+                   f"between steps by overwriting a {2 * L2_BYTES / 1e6:.0f} MB buffer, outside the timed intervals"),
+            "launch": (f"CUDA graphs of {G} consecutive steps over the rotating sets" if flush is None else
+                       "one CUDA graph per step, each timed by its own pair of events")
+                      + ("; one ttt_forward_layer call per step: the conv kernel launched behind the linear kernel "
+                         "as a programmatic dependent, the two running at the same time" if w.kind == "mixed" else ""),
+            "step_spread": spread, "gbs_per_step": workload_bytes(w) / t_step / 1e9,
+            "gpu_launches": args.steps * per_step, "gpu_launches_per_step": per_step,
+            "kernel_src_sha": kernel_source_hash(), "clocks": clocks, "e2e": e2e, "roofline": roof}
     if rank == 0 and world == 1 and not args.no_oracle:
-        line["cpu_baseline"] = time_oracle(w, xs[0], budget_s=12.0)
+        line["cpu_baseline"] = time_oracle(w, xs[0])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graphs
+        del singles, run_g, plan
         dist.destroy_process_group()
 
 
 def run_e2e(w, x, dev, stream, steps, world):
     """The same metric through the public API with the inputs on the host: every step copies its Q, K,
-    V and weights from pinned host memory to the device, runs the layer and copies Z back.  Steps are
-    pipelined over two buffer sets and three streams, as a serving loop would run them: the
-    host-to-device copy of step i+1 overlaps the compute and the device-to-host copy of step i (PCIe
-    moves both directions at once).  Every step's copies are inside the timed region."""
-    from vision_test_token_b200 import layer
-    names = ["Q", "K", "V"] + (["dZ"] if w.kind == "backward" else []) + sorted(k for k in x if k.startswith("W"))
+    V (and dZ) and weights from pinned host memory to the device, runs the step and copies its outputs
+    (Z, or dQ, dK, dV and the weight gradients) back.  Steps are pipelined over two buffer sets and
+    three streams, as a serving loop would run them: the host-to-device copy of step i+1 overlaps the
+    compute and the device-to-host copy of step i (PCIe moves both directions at once).  Every step's
+    copies are inside the timed region."""
+    bwd = w.kind.startswith("backward")
+    names = ["Q", "K", "V"] + (["dZ"] if bwd else []) + sorted(k for k in x if k.startswith("W"))
     host = {k: x[k].cpu().pin_memory() for k in names}
     dev_in = [{k: torch.empty_like(x[k]) for k in names} for _ in range(2)]
-    n_out = 3 if w.kind == "backward" else 1                 # dQ, dK, dV, or Z
-    z_dev = [[torch.empty_like(x["Q"]) for _ in range(n_out)] for _ in range(2)]
-    z_host = [[torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory() for _ in range(n_out)] for _ in range(2)]
-    small = [(torch.empty((w.heads, w.d, w.d), device=dev), torch.empty(1, device=dev)) for _ in range(2)]
+    outs = list(x["grads"]) if bwd else [x["Z"]]
+    o_dev = [[torch.empty_like(t) for t in outs] for _ in range(2)]
+    o_host = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs] for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in z_host[0])
+    d2h = sum(t.numel() * t.element_size() for t in o_host[0])
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev = lambda: torch.cuda.Event()
     loaded, computed, drained = [ev(), ev()], [ev(), ev()], [ev(), ev()]
@@ -544,24 +698,14 @@ def run_e2e(w, x, dev, stream, steps, world):
             loaded[bsel].record(s_in)
         stream.wait_event(loaded[bsel])
         if started[bsel]:
-            stream.wait_event(drained[bsel])                 # step i-2's Z has left this buffer
+            stream.wait_event(drained[bsel])                 # step i-2's outputs have left this buffer
         with torch.cuda.stream(stream):
-            if w.kind == "mlp":
-                layer.forward_mlp(d["Q"], d["K"], d["V"], d["Wa"], d["Wb"], w.eta, w.H, w.W, Z=z_dev[bsel][0])
-            elif w.kind == "minibatch":
-                layer.forward_linear_minibatch(d["Q"], d["K"], d["V"], d["W0_lin"], w.eta, w.H, w.W, w.mb_tokens,
-                                               w.mb_mode, Z=z_dev[bsel][0])
-            elif w.kind == "backward":
-                layer.backward_linear(d["Q"], d["K"], d["V"], d["W0_lin"], w.eta, w.H, w.W, d["dZ"],
-                                      out=(*z_dev[bsel], *small[bsel]))
-            else:
-                layer.forward_layer(d["Q"], d["K"], d["V"], d, w.eta, w.H, w.W, conv_heads=w.conv_heads,
-                                    Z=z_dev[bsel][0], loss=w.loss)
+            run_step(w, x, d=d, out=tuple(o_dev[bsel]) if bwd else o_dev[bsel][0])
             computed[bsel].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(computed[bsel])
-            for zh, zd in zip(z_host[bsel], z_dev[bsel]):
-                zh.copy_(zd, non_blocking=True)
+            for oh, od in zip(o_host[bsel], o_dev[bsel]):
+                oh.copy_(od, non_blocking=True)
             drained[bsel].record(s_out)
         started[bsel] = True
 

@@ -189,3 +189,11 @@ def test_header_is_plain_c(tmp_path):
     r = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Werror", "-fsyntax-only",
                         "-I", os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_wait_limit_bounds(lib):
+    """The bound of every device-side wait is settable from the host (1 ns .. 1 s); other values are
+    rejected and leave it unchanged."""
+    assert capi.ttt_set_wait_limit(0) == capi.TTT_ERR_INVALID_ARG
+    assert capi.ttt_set_wait_limit(10 ** 10) == capi.TTT_ERR_INVALID_ARG
+    assert capi.ttt_set_wait_limit(1_000_000_000) == capi.TTT_OK

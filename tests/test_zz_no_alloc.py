@@ -42,6 +42,45 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_dev, dtype, B, h, H, W
         assert rel_max_err(W1, W1_ref.double().cpu().numpy()) <= TOL[dtype]
 
 
+def test_noalloc_allocates_nothing(cuda_dev):
+    """Around a pair of calls (the first one on this shape included) neither PyTorch's allocator nor
+    the device's free memory changes: the entry point draws only on its library-owned array.  (One
+    call on another shape first, so that the kernel's code is already loaded on the device.)"""
+    _noalloc(random_unit(1, 1, 9, 9, dtype="bf16", seed=4)[1], 0.5, 9, 9, cuda_dev)
+    _, x = random_unit(2, 3, 16, 16, dtype="bf16", seed=5)
+    Q, K, V = (x[k].to(cuda_dev) for k in ("Q", "K", "V"))
+    W0 = x["W0_lin"].to(cuda_dev).contiguous()
+    Z = torch.empty_like(Q)
+    W1 = torch.empty((2, 3, 64, 64), device=cuda_dev)
+    shape = capi.make_shape(2, 3, 16, 16, 64, Q.stride(0), Q.stride(1), capi.TTT_BF16)
+    stream = torch.cuda.current_stream().cuda_stream
+    torch.cuda.synchronize()
+    n0 = torch.cuda.memory_stats(cuda_dev).get("allocation.all.allocated", 0)
+    f0, _ = torch.cuda.mem_get_info(cuda_dev)
+    for _ in range(2):
+        st = capi.ttt_forward_linear_noalloc(Q.data_ptr(), K.data_ptr(), V.data_ptr(), W0.data_ptr(), Z.data_ptr(),
+                                             0.5, shape, W1.data_ptr(), stream)
+        assert st == capi.TTT_OK
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_stats(cuda_dev).get("allocation.all.allocated", 0) == n0
+    assert torch.cuda.mem_get_info(cuda_dev)[0] == f0
+    assert capi.ttt_noalloc_status(stream) == capi.TTT_OK
+
+
+def test_noalloc_fp32_counters_left_by_a_larger_call(cuda_dev):
+    """fp32 keeps counters and partial slots in the scratch: a call over 6 units, then one over 1 unit
+    (which finds the first call's leftovers), both correct."""
+    for (B, h) in [(2, 3), (1, 1)]:
+        _, x = random_unit(B, h, 14, 14, dtype="fp32", seed=40 + B)
+        Q, K, V = (x[k].to(cuda_dev) for k in ("Q", "K", "V"))
+        W1_ref = torch.empty((B, h, 64, 64), device=cuda_dev)
+        Z_ref = forward_linear(Q, K, V, x["W0_lin"].to(cuda_dev), 0.5, 14, 14, W1_out=W1_ref)
+        torch.cuda.synchronize()
+        Z, W1 = _noalloc(x, 0.5, 14, 14, cuda_dev)
+        assert rel_max_err(Z, Z_ref.double().cpu().numpy()) <= TOL["fp32"]
+        assert rel_max_err(W1, W1_ref.double().cpu().numpy()) <= TOL["fp32"]
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_dev):
     big = torch.zeros(1, device=cuda_dev)
     p = big.data_ptr()

@@ -186,7 +186,10 @@ constexpr int STAGES = 4;                   // 32 KB each: a K+V tile pair, or o
 constexpr int ACC = 4;                      // phase-2 accumulators (64 columns each)
 constexpr int Q2 = 256;                     // tokens per phase-2 stage
 constexpr int kMaxCluster = 8;             // the portable limit
-constexpr int kRecvBytes = 15360;           // the peers' rows of my P block: (CS - 1) x ceil(64 / CS) x 256 B, CS <= 8
+constexpr int kRecvBytes = 15360;
+// Cost model of the cluster-size choice (host): the per-SM streaming rate, the HBM rate the SMs
+// share, and one unit's exchange latency with peers and alone (measured on B200, in GB/s and us).
+constexpr double kCtaGBs = 62.0, kHbmGBs = 6400.0, kExchangeUs = 4.5, kExchangeUs1 = 2.5;           // the peers' rows of my P block: (CS - 1) x ceil(64 / CS) x 256 B, CS <= 8
 constexpr uint32_t kColPacc = 0;            // tensor memory: two phase-1 accumulators,
 constexpr uint32_t kColAcc = 128;           //   ACC phase-2 accumulators,
 constexpr uint32_t kColProd = 384;          //   the W0 G product (448 of 512 columns)
@@ -845,14 +848,31 @@ lin_p1_f32(TokenView Kv, TokenView Vv, const F32Params p) {
         for (int i = 0; i < 32; ++i) acc[i] = 0.f;
         const int n_begin = (int)(t % p.tpu) * TOK;
         const int n_end = min(p.N, (int)((seg_end - (long long)u * p.tpu) * TOK));
-        for (int n0 = n_begin; n0 < n_end; n0 += F32_CHUNK) {
-            for (int e = tid; e < F32_CHUNK * D; e += kThreadsF32) {
-                const int tk = e / D, cc = e % D;
+        // the chunk's K and V rows as 16-byte loads into registers, all issued before any is used;
+        // the next chunk's loads are in flight while the current chunk is accumulated
+        constexpr int F4 = F32_CHUNK * D / 4 / kThreadsF32;   // float4 of K (and of V) per thread
+        float4 fk[F4], fv[F4];
+        auto fetch = [&](int n0) {
+#pragma unroll
+            for (int q = 0; q < F4; ++q) {
+                const int e4 = q * kThreadsF32 + tid, tk = e4 / (D / 4), c4 = e4 % (D / 4);
                 const int n = n0 + tk;
-                s.k[tk][cc] = (n < n_end) ? Kv.row(u, p.heads, n)[cc] : 0.f;
-                s.v[tk][cc] = (n < n_end) ? Vv.row(u, p.heads, n)[cc] : 0.f;
+                fk[q] = n < n_end ? __ldg(reinterpret_cast<const float4*>(Kv.row(u, p.heads, n)) + c4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                fv[q] = n < n_end ? __ldg(reinterpret_cast<const float4*>(Vv.row(u, p.heads, n)) + c4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
+        fetch(n_begin);
+        for (int n0 = n_begin; n0 < n_end; n0 += F32_CHUNK) {
+#pragma unroll
+            for (int q = 0; q < F4; ++q) {
+                const int e4 = q * kThreadsF32 + tid, tk = e4 / (D / 4), c4 = e4 % (D / 4);
+                *reinterpret_cast<float4*>(&s.k[tk][4 * c4]) = fk[q];
+                *reinterpret_cast<float4*>(&s.v[tk][4 * c4]) = fv[q];
             }
             __syncthreads();
+            if (n0 + F32_CHUNK < n_end) fetch(n0 + F32_CHUNK);
             for (int tk = 0; tk < F32_CHUNK; ++tk) {
                 const float x = (r < D) ? s.k[tk][r] : s.v[tk][r - D];
 #pragma unroll
@@ -890,7 +910,7 @@ lin_p1_f32(TokenView Kv, TokenView Vv, const F32Params p) {
 
 struct P2SmemF32 {
     float w1t[D][D];            // W1 transposed: w1t[k][o] = W1[o][k]
-    float q[TOK][D + 1];
+    float q[TOK][D + 4];        // row pitch 272 B: 16-byte aligned rows for the vector stores
 };
 
 __global__ void __launch_bounds__(kThreadsF32)
@@ -901,10 +921,21 @@ lin_p2_f32(TokenView Qv, float* Z, long long zbs, long long zhs, const float* W1
     const long long t = blockIdx.x;                        // one tile per CTA
     const int u = (int)(t / tpu), ti = (int)(t % tpu);
     const int n0 = ti * TOK;
-    for (int e = tid; e < TOK * D; e += kThreadsF32) {
-        const int tk = e / D, cc = e % D;
-        const int n = n0 + tk;
-        s.q[tk][cc] = (n < N) ? Qv.row(u, heads, n)[cc] : 0.f;
+    {
+        // the Q tile as 16-byte loads, all issued before any is stored
+        constexpr int F4 = TOK * D / 4 / kThreadsF32;
+        float4 fq[F4];
+#pragma unroll
+        for (int q = 0; q < F4; ++q) {
+            const int e4 = q * kThreadsF32 + tid, tk = e4 / (D / 4), c4 = e4 % (D / 4);
+            const int n = n0 + tk;
+            fq[q] = n < N ? __ldg(reinterpret_cast<const float4*>(Qv.row(u, heads, n)) + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < F4; ++q) {
+            const int e4 = q * kThreadsF32 + tid, tk = e4 / (D / 4), c4 = e4 % (D / 4);
+            *reinterpret_cast<float4*>(&s.q[tk][4 * c4]) = fq[q];
+        }
     }
     pdl_wait_primary();
     const float* W1u = W1 + (size_t)u * D * D;
@@ -1011,19 +1042,28 @@ ttt_status launch_linear(const Call& c) {
         const size_t smem = sizeof(ClusterSmem) + 1024;
         cudaFuncSetAttribute(lin_cluster_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         // CTAs per cluster (cs) and clusters (ncl): every cluster co-resident (a second wave would
-        // double the time), and the least streaming per CTA: the most units a cluster takes, over cs.
-        // A cluster with one unit cannot hide its exchange behind another unit's streaming, which
-        // costs about a quarter of a unit's time; a tie goes to the larger cluster.
+        // double the time), and the least estimated time.  A CTA streams its 1/cs share of each of its
+        // cluster's units (32 KB stages at the per-SM rate, or at its share of HBM when the SMs
+        // together would exceed it), and each unit's exchange takes a latency of its own; with two
+        // units in flight a unit costs the larger of the two, and the first unit's streaming and the
+        // last unit's exchange are not overlapped.  Large units are streaming-bound (fewer units per
+        // cluster over more CTAs wins); small ones are exchange-bound (fewest units per cluster wins).
         int cs = 1, ncl = (int)std::min<long long>(units, std::max(1, c.num_sms));
         double best = 1e30;
+        const int tpu2 = (c.N + Q2 - 1) / Q2;
         for (int k = 1; k <= kMaxCluster; ++k) {
             const long long n = std::min<long long>(units, c.num_sms / k);
             if (n < 1) break;
             const long long upc = (units + n - 1) / n;
             const long long need = (units + upc - 1) / upc;
             if (k > 1 && max_active_clusters(k, smem) < need) continue;
-            const double score = (double)upc / k * (upc == 1 ? 1.25 : 1.0);
-            if (score <= best) { best = score; cs = k; ncl = (int)need; }
+            const double ctas = (double)need * k;
+            const double gbs = std::min(kCtaGBs, kHbmGBs / ctas);                 // per-CTA rate
+            const double t_stage = 32768.0 / (gbs * 1e3);                         // us per 32 KB stage
+            const double ts = ((tpu + k - 1) / k + (tpu2 + k - 1) / k) * t_stage;  // one unit's share
+            const double tx = k > 1 ? kExchangeUs : kExchangeUs1;
+            const double cost = (double)upc * std::max(ts, tx) + std::min(ts, tx);
+            if (cost <= best * 1.001) { best = std::min(best, cost); cs = k; ncl = (int)need; }   // ties: larger
         }
         ClusterParams p{};
         p.heads = c.heads;
