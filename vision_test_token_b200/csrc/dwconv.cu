@@ -329,6 +329,9 @@ dw_band(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtenso
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ);
     }
     __syncthreads();
+    // A kernel queued behind this one as a programmatic dependent (the next call's linear heads) may
+    // be scheduled as SMs free up; it waits for this grid to complete before it reads anything.
+    pdl_launch_dependents();
 
     if (warp == CW) {                                                // producer
         if (lane == 0) {

@@ -748,8 +748,11 @@ lin_cluster_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     cluster_sync_all();                  // every CTA's barriers exist before any peer arrives on them
-    // A kernel queued behind this one as a programmatic dependent (the conv heads of the same layer)
-    // may start once every CTA of this grid is resident: it takes the SMs this grid leaves free.
+    // Launched as a programmatic dependent of the preceding kernel in the stream: the prologue above
+    // overlaps that kernel's tail, and nothing is read from global memory before it has completed
+    // (with its memory visible).  Only then may a kernel queued behind this one as a programmatic
+    // dependent (the conv heads of the same layer) start: it takes the SMs this grid leaves free.
+    pdl_wait_primary();
     pdl_launch_dependents();
     const uint32_t tmem = s.tmem_base;
 
@@ -1088,11 +1091,13 @@ ttt_status launch_linear(const Call& c) {
         cfg.blockDim = dim3(kThreadsTc);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = c.stream;
-        cudaLaunchAttribute at[1];
+        cudaLaunchAttribute at[2];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = cs; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+        at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see the kernel's prologue
+        at[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         return check_launch(cudaLaunchKernelEx(&cfg, lin_cluster_bf16, tmK, tmV, tmQ, tmZ, p));
     }
 
