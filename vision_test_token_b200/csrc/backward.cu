@@ -116,9 +116,7 @@ __device__ void merge_unit(const Params& p, P1Smem& s, int u, int slot0, int nsl
     const int h = u % p.view.heads;
     // fixed-order sum of the unit's partial slots
     for (int e = tid; e < kPartial; e += P1_THREADS) {
-        float a = 0.f;
-        for (int j = 0; j < nslots; ++j) a += __ldcg(p.partials + (size_t)(slot0 + j) * kPartial + e);
-        (&s.mg.acc[0][0])[e] = a;
+        (&s.mg.acc[0][0])[e] = add_strided_in_order(0.f, p.partials + (size_t)slot0 * kPartial + e, kPartial, nslots);
     }
     for (int e = tid; e < D * D; e += P1_THREADS) s.mg.w0[e / D][e % D] = __ldg(p.W0 + (size_t)h * D * D + e);
     __syncthreads();

@@ -165,11 +165,8 @@ cb_unit(const Params p) {
     pdl_launch_dependents();
     pdl_wait_primary();                                       // every tile partial is written
     const float* src = p.red + (size_t)u * g.tpu * 2 * kPart;
-    float sk = 0.f, zq = 0.f;
-    for (int i = 0; i < g.tpu; ++i) {
-        sk += __ldcg(src + (size_t)i * 2 * kPart + e);
-        zq += __ldcg(src + (size_t)i * 2 * kPart + kPart + e);
-    }
+    const float sk = add_strided_in_order(0.f, src + e, 2 * kPart, g.tpu);
+    const float zq = add_strided_in_order(0.f, src + kPart + e, 2 * kPart, g.tpu);
     const float w0 = __ldg(p.W0 + ((size_t)h * D + c) * TAPS + t);
     const float gr = g.scale * sk;                            // g_t = (2/N) sum r K_t
     float* cf = p.coef + (size_t)u * 3 * kPart;
@@ -283,14 +280,13 @@ cb_final(const Params p) {
     const int h = blockIdx.x, e = threadIdx.x, t = e / D, c = e % D;
     pdl_wait_primary();
     if (p.dW0_out) {
+        // images in order: per image dW1, then the image's tile partials in order
         const int B = g.U / g.heads;
         float acc = 0.f;
-        for (int b = 0; b < B; ++b) {                          // images in order
+        for (int b = 0; b < B; ++b) {
             const int u = b * g.heads + h;
-            float unit = __ldcg(p.coef + (size_t)u * 3 * kPart + 2 * kPart + e);   // dW1
-            const float* mp = p.mapp + (size_t)u * g.tpu * kPart;
-            for (int i = 0; i < g.tpu; ++i) unit += __ldcg(mp + (size_t)i * kPart + e);
-            acc += unit;
+            acc += add_strided_in_order(__ldcg(p.coef + (size_t)u * 3 * kPart + 2 * kPart + e),   // dW1
+                                        p.mapp + (size_t)u * g.tpu * kPart + e, kPart, g.tpu);
         }
         p.dW0_out[((size_t)h * D + c) * TAPS + t] = acc;
     }

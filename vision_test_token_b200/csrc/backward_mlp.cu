@@ -274,7 +274,7 @@ mb_read(const T* __restrict__ Q, const T* __restrict__ dZ, T* __restrict__ dQ, c
 }
 
 // ---- mb_merge2: per unit, dgWa, dgWb and the unit's deta term -------------------------------------
-__global__ void mb_merge2(const Params p) {
+__global__ void __launch_bounds__(1024) mb_merge2(const Params p) {
     __shared__ float red[1024];
     const int u = blockIdx.x;
     const size_t w = (size_t)p.hid * D;
@@ -423,18 +423,15 @@ __global__ void mb_final(const Params p) {
     const size_t w = (size_t)p.hid * D;
     const int B = p.U / p.heads;
     pdl_wait_primary();
-    for (size_t e = threadIdx.x; e < 2 * w; e += blockDim.x) {
-        float acc = 0.f;
-        for (int b = 0; b < B; ++b) {                        // images in order
-            const int u = b * p.heads + h;
-            float unit = __ldcg(p.dw1 + (size_t)u * 2 * w + e);
-            for (int c = 0; c < p.nch; ++c) unit += __ldcg(p.upd + ((size_t)u * p.nch + c) * 2 * w + e);
-            acc += unit;
-        }
+    for (size_t e = (size_t)blockIdx.y * blockDim.x + threadIdx.x; e < 2 * w; e += (size_t)gridDim.y * blockDim.x) {
+        // images in order: per image dW1, then the image's chunk partials in order
+        const float acc = nested_sum_in_order(
+            B, p.nch, [&](int b) { return p.dw1 + (size_t)(b * p.heads + h) * 2 * w + e; },
+            [&](int b, int c) { return p.upd + ((size_t)(b * p.heads + h) * p.nch + c) * 2 * w + e; });
         if (e < w) { if (p.dWa_out) p.dWa_out[h * w + e] = acc; }
         else if (p.dWb_out) p.dWb_out[h * w + (e - w)] = acc;
     }
-    if (h == 0 && threadIdx.x == 0 && p.deta_out) {
+    if (h == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.deta_out) {
         float acc = 0.f;
         for (int u = 0; u < p.U; ++u) acc += __ldcg(p.deta_u + u);
         *p.deta_out = acc;
@@ -513,7 +510,10 @@ static ttt_status launch(const Call& c, const ttt_shape& sh, const void* dZ, voi
         cfg.blockDim = dim3(kThreads);
         st = check_launch(cudaLaunchKernelEx(&cfg, mb_upd<T>, K, V, static_cast<T*>(dK), static_cast<T*>(dV), p));
     }
-    if (st == TTT_OK) { cfg.gridDim = dim3((unsigned)c.heads); st = check_launch(cudaLaunchKernelEx(&cfg, mb_final, p)); }
+    if (st == TTT_OK) {                                     // per head, the 2 hidden x d elements over 32 CTAs
+        cfg.gridDim = dim3((unsigned)c.heads, 32u);
+        st = check_launch(cudaLaunchKernelEx(&cfg, mb_final, p));
+    }
     return st;
 }
 

@@ -366,7 +366,8 @@ conv3_grad(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 }
 
 // ------------------------------------------------------------------------------------------------
-// conv3_merge: one CTA per (unit, tap)
+// conv3_merge: four CTAs per (unit, tap), each a quarter of the tap's 64 x 64 matrix: one float4
+// of it per thread, summed over the unit's slots in slot order with 16 loads in flight at a time
 // ------------------------------------------------------------------------------------------------
 struct MergeParams {
     Geo g;
@@ -380,18 +381,31 @@ struct MergeParams {
 
 __global__ void __launch_bounds__(256)
 conv3_merge(const MergeParams p) {
-    const int u = blockIdx.x / TAPS, t9 = blockIdx.x % TAPS, h = u % p.g.heads;
+    const int q4 = blockIdx.x & 3, ut = blockIdx.x >> 2;
+    const int u = ut / TAPS, t9 = ut % TAPS, h = u % p.g.heads;
     pdl_launch_dependents();
     pdl_wait_primary();                                      // every gradient slot is written
     const int cf = part_cta(p.g.T, p.G, (long long)u * p.g.tpu);
     const int cl = part_cta(p.g.T, p.G, (long long)(u + 1) * p.g.tpu - 1);
     uint8_t* img = p.w1img + ((size_t)u * TAPS + t9) * kWImg;
-    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
-        const int cp = e / D, c = e % D;                     // slot element G^T[t9][cp][c]
-        float acc = 0.f;
-        for (int cta = cf; cta <= cl; ++cta) acc += __ldcg(p.slots + (size_t)(cta + u) * kSlotFloats + (size_t)t9 * D * D + e);
+    const int e4 = q4 * 256 + (int)threadIdx.x;              // float4 of the tap's matrix: elements 4 e4 ..
+    const float4* src = reinterpret_cast<const float4*>(p.slots + (size_t)t9 * D * D) + e4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = cf; c0 <= cl; c0 += 16) {
+        float4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            v[i] = (c0 + i <= cl) ? __ldcg(src + (size_t)(c0 + i + u) * (kSlotFloats / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (c0 + i <= cl) { acc.x += v[i].x; acc.y += v[i].y; acc.z += v[i].z; acc.w += v[i].w; }
+    }
+    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = 4 * e4 + i, cp = e / D, c = e % D;     // slot element G^T[t9][cp][c]
         const size_t wi = (((size_t)h * D + c) * D + cp) * TAPS + t9;
-        const float w1 = __ldg(p.W0 + wi) - p.g.eta_scale * acc;
+        const float w1 = __ldg(p.W0 + wi) - p.g.eta_scale * a4[i];
         if (p.W1_out) p.W1_out[(((size_t)u * D + c) * D + cp) * TAPS + t9] = w1;
         *reinterpret_cast<__nv_bfloat16*>(img + sw_off(c, cp / 8) + (cp % 8) * 2) = __float2bfloat16_rn(w1);
     }
@@ -649,7 +663,7 @@ ttt_status launch_conv3x3(const Call& c) {
     mp.slots = gp.slots;
     mp.W1_out = c.W1_out;
     mp.w1img = c.ws + L.w1img;
-    cfg.gridDim = dim3((unsigned)(units * TAPS));
+    cfg.gridDim = dim3((unsigned)(units * TAPS * 4));
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.numAttrs = 1;

@@ -102,6 +102,57 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
 }
 
+// init + base[0] + base[stride] + ... + base[(n-1) stride], added in that order (bitwise the plain
+// loop), with 16 of the L2-resident loads in flight at a time instead of one.
+__device__ __forceinline__ float add_strided_in_order(float init, const float* base, size_t stride, int n) {
+    float acc = init;
+    for (int k0 = 0; k0 < n; k0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[q] = k0 + q < n ? __ldcg(base + (size_t)(k0 + q) * stride) : 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (k0 + q < n) acc += v[q];
+    }
+    return acc;
+}
+
+// sum_b (first(b) + sum_{i < n} rest(b, i)) over b < B, added in exactly the order of the nested
+// loops (unit = first; unit += rest in i order; acc += unit in b order), with up to 16 loads in flight
+// across image boundaries: for many short inner sums.  first and rest return the terms' addresses.
+template <class First, class Rest>
+__device__ __forceinline__ float nested_sum_in_order(int B, int n, First first, Rest rest) {
+    float acc = 0.f, unit = 0.f;
+    bool started = false;
+    int b = 0, i = -1;                       // the next term: first(b) when i < 0, else rest(b, i)
+    while (b < B) {
+        float v[16];
+        bool head[16], live[16];
+        int bb = b, ii = i;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            live[q] = bb < B;
+            head[q] = ii < 0;
+            v[q] = live[q] ? __ldcg(ii < 0 ? first(bb) : rest(bb, ii)) : 0.f;
+            if (++ii == n) { ii = -1; ++bb; }
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (!live[q]) continue;
+            if (head[q]) {
+                if (started) acc += unit;
+                unit = v[q];
+                started = true;
+            } else {
+                unit += v[q];
+            }
+        }
+        b = bb;
+        i = ii;
+    }
+    return started ? acc + unit : 0.f;
+}
+
 // Loads from shared memory by 32-bit shared address (ld.shared: no generic-address resolution).
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     uint32_t v;
