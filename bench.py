@@ -47,7 +47,18 @@ L2_BYTES = 126 * 2 ** 20
 # whose hash differs from the running build's is stale and is not reported.  Captured with
 # --cache-control none on the third of three consecutive steps, so that the previous step's Z
 # write-back (which lands during the next step) is counted as it is in steady state.
-TRAFFIC = {}
+TRAFFIC = {
+    "mixed6084_bf16": {"read": 112356352, "write": 38231040, "src_sha": "88e63fe44a5cadc0"},
+    "mixed6084_dot_bf16": {"read": 112324352, "write": 38272256, "src_sha": "88e63fe44a5cadc0"},
+    "lin6400_bf16": {"read": 118183168, "write": 40068864, "src_sha": "e252f1ffc5b63f16"},
+    "lin196_bf16": {"read": 14328832, "write": 599040, "src_sha": "e252f1ffc5b63f16"},
+    "mlp1024_bf16": {"read": 25482752, "write": 6326784, "src_sha": "f33d5474b3e7c44e"},
+    "conv3x3_6084_bf16": {"read": 18741504, "write": 7558144, "src_sha": "2385ceaf5d3c5c3d"},
+    "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
+    "bwd6084_bf16": {"read": 208251136, "write": 113136640, "src_sha": "6ed6afd58a0eb27a"},
+    "bwdconv6084_bf16": {"read": 24883456, "write": 17042944, "src_sha": "1dfe7c0812e5935d"},
+    "bwdmlp1024_bf16": {"read": 67329024, "write": 145303808, "src_sha": "a33fe42962dd5335"},
+}
 
 # Kernels of this library launched per step, by workload kind (bf16; fp32 where it differs).
 LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backward": 3, "backward_conv": 4,
@@ -55,11 +66,20 @@ LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backwar
 LAUNCHES_PER_STEP_FP32 = {"linear": 2, "mixed": 3}
 
 
-def kernel_source_hash():
-    """sha256 over the CUDA sources and headers of the library (sorted by name)."""
+# The CUDA sources each workload kind runs (besides the shared headers and the host entry points).
+KIND_SOURCES = {"linear": ["linear.cu"], "mixed": ["linear.cu", "dwconv.cu"], "mlp": ["mlp.cu"],
+                "minibatch": ["minibatch.cu"], "backward": ["backward.cu"], "backward_conv": ["backward_conv.cu"],
+                "backward_mlp": ["backward_mlp.cu"], "conv3x3": ["conv3x3.cu"]}
+COMMON_SOURCES = ["sm100.cuh", "ttt_internal.h", "api.cu"]
+
+
+def kernel_source_hash(kind=None):
+    """sha256 over the CUDA sources a workload kind runs and the shared headers and host entry points
+    (every source of the library when kind is None), sorted by name."""
     d = os.path.join(ROOT, "vision_test_token_b200", "csrc")
+    names = sorted(os.listdir(d)) if kind is None else sorted(COMMON_SOURCES + KIND_SOURCES[kind])
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
+    for name in names:
         if name.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(d, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
@@ -504,7 +524,7 @@ def traffic_entry(w):
     e = TRAFFIC.get(w.name)
     if not e:
         return None, "no ncu capture for this workload"
-    if e["src_sha"] != kernel_source_hash():
+    if e["src_sha"] != kernel_source_hash(w.kind):
         return None, f"stale: the capture was taken on kernel sources {e['src_sha']}, not on this build"
     return e, None
 
@@ -655,7 +675,7 @@ def run_ours(args):
                          "as a programmatic dependent, the two running at the same time" if w.kind == "mixed" else ""),
             "step_spread": spread, "gbs_per_step": workload_bytes(w) / t_step / 1e9,
             "gpu_launches": args.steps * per_step, "gpu_launches_per_step": per_step,
-            "kernel_src_sha": kernel_source_hash(), "clocks": clocks, "e2e": e2e, "roofline": roof}
+            "kernel_src_sha": kernel_source_hash(w.kind), "clocks": clocks, "e2e": e2e, "roofline": roof}
     if rank == 0 and world == 1 and not args.no_oracle:
         line["cpu_baseline"] = time_oracle(w, xs[0])
     if rank == 0:

@@ -62,11 +62,14 @@ def test_traffic_entry_refuses_a_stale_capture(monkeypatch):
     monkeypatch.setattr(bench, "TRAFFIC", {w.name: {"read": 1.0, "write": 2.0, "src_sha": "0" * 16}})
     e, note = bench.traffic_entry(w)
     assert e is None and note.startswith("stale")
-    monkeypatch.setattr(bench, "TRAFFIC", {w.name: {"read": 1.0, "write": 2.0, "src_sha": bench.kernel_source_hash()}})
+    monkeypatch.setattr(bench, "TRAFFIC", {w.name: {"read": 1.0, "write": 2.0,
+                                                    "src_sha": bench.kernel_source_hash(w.kind)}})
     e, note = bench.traffic_entry(w)
     assert e["read"] == 1.0 and note is None
 
 
-def test_kernel_source_hash_is_stable():
+def test_kernel_source_hash_is_stable_and_per_kind():
     assert bench.kernel_source_hash() == bench.kernel_source_hash()
     assert len(bench.kernel_source_hash()) == 16
+    assert set(bench.KIND_SOURCES) >= {w.kind for w in WORKLOADS.values()}
+    assert bench.kernel_source_hash("mixed") != bench.kernel_source_hash("mlp")
