@@ -329,13 +329,20 @@ def time_oracle(w, x, budget_s=10.0, single_budget_s=6.0):
     reused when the batch has fewer), OpenMP over the units.  Single-core: one image, one thread."""
     import oracle
     cores = oracle.default_threads()
-    images = max(1, math.ceil(cores / w.heads))
+    if w.kind.startswith("backward"):
+        # the backward oracles sum the weight gradients over the images of each head in order: OpenMP
+        # over the heads only
+        images, used, over = 1, min(cores, w.heads), "heads"
+    else:
+        images = max(1, math.ceil(cores / w.heads))
+        used, over = min(cores, images * w.heads), "(image, head) units"
     xs = oracle_inputs(w, x, min(images, x["Q"].shape[0]))
     v_all, reps, el = _time_oracle_leg(w, xs, images, cores, budget_s)
     v_one, reps1, el1 = _time_oracle_leg(w, xs, 1, 1, single_budget_s)
-    return {"value": v_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": v_all, "unit": UNIT, "cores": used, "kind": "oracle",
             "sample": f"{images} image(s) of {w.name} ({images * w.heads} (image, head) units of {w.N} tokens) "
-                      f"repeated {reps} times in {el:.1f} s, fp64, OpenMP over the units on {cores} cores",
+                      f"repeated {reps} times in {el:.1f} s, fp64, OpenMP over the {over}: {used} of the "
+                      f"{cores} cores of the affinity mask busy",
             "single_core": {"value": v_one, "unit": UNIT, "cores": 1,
                             "sample": f"1 image of {w.name} ({w.heads} units) repeated {reps1} times in "
                                       f"{el1:.1f} s, one thread"}}
