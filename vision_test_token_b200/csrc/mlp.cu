@@ -9,8 +9,10 @@
 //
 // Every product is a dense contraction and runs on tcgen05 (bf16 operands, fp32 accumulation in
 // tensor memory).  A unit is owned by a cluster of two CTAs, each taking half of the tokens (one CTA
-// per unit, persistent over units, when there are more units than SM pairs).  Per 128-token tile of
-// phase 1:
+// per unit, persistent over units, when there are more units than SM pairs).  A CTA has a TMA
+// producer warp and 8 compute warps: tid 0 issues the MMAs, and the two warps of each tensor-memory
+// lane quarter split every elementwise pass's columns (GELU in packed half precision).  Per 128-token
+// tile of phase 1:
 //   H  = K Wa^T            M=128 tokens, N=256, K=64       -> TMEM cols 256..511
 //   A  = gelu(H) (bf16, shared memory), gelu'(H) packed bf16x2 back into TMEM cols 256..383
 //   Y  = A Wb^T            M=128, N=64, K=256             -> TMEM cols 384..447
@@ -29,6 +31,8 @@
 // another (both use the 128-byte swizzled layout TMA writes), so nothing is transposed.
 #include <algorithm>
 
+#include <cuda_fp16.h>
+
 #include "sm100.cuh"
 #include "ttt_internal.h"
 
@@ -40,7 +44,8 @@ constexpr int HID = 256;
 constexpr int TOK = 128;
 constexpr int TILE = TOK * D * 2;           // 16 KB bf16 tile
 constexpr int STAGES = 2;                   // each holds a K tile + V tile, or a Q tile
-constexpr int THREADS = 160;                // warp 0: TMA producer, warps 1..4: MMA + elementwise
+constexpr int THREADS = 288;                // warp 0: TMA producer, warps 1..8: MMA + elementwise
+constexpr int kCT = 256;                    // compute threads: two warps per tensor-memory lane quarter
 constexpr float kGeluC = 0.7978845608028654f;   // sqrt(2 / pi)
 constexpr float kGeluA = 0.044715f;
 
@@ -87,22 +92,36 @@ __device__ __forceinline__ uint32_t sw_off(int row, int col) {
     return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
 }
 
-__device__ __forceinline__ float tanh_fast(float x) {
-    float y;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
+// gelu(u) and its derivative, from t = tanh(c (u + a u^3)):
+//     gelu(u) = u/2 (1 + t),   gelu'(u) = (1 + t)/2 + u/2 (1 - t^2) c (1 + 3 a u^2),
+// evaluated on a pair of values in packed half precision (10-bit mantissa, finer than
+// the bf16 the results are rounded to), returned as packed bf16 pairs: about half the instructions
+// of the fp32 form.
+__device__ __forceinline__ __half2 tanh_fast_h2(__half2 x) {
+    uint32_t y;
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(y) : "r"(*reinterpret_cast<const uint32_t*>(&x)));
+    return *reinterpret_cast<const __half2*>(&y);
 }
-
-// gelu(u) and its derivative, from t = tanh(c (u + a u^3)).
-__device__ __forceinline__ void gelu_and_grad(float u, float& g, float& dg) {
-    const float u2 = u * u;
-    const float t = tanh_fast(kGeluC * fmaf(kGeluA * u2, u, u));
-    g = 0.5f * u * (1.f + t);
-    dg = 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * kGeluC * fmaf(3.f * kGeluA, u2, 1.f);
+__device__ __forceinline__ uint32_t h2_to_bf16x2(__half2 v) {
+    const float2 f = __half22float2(v);
+    return pack_bf16x2(f.x, f.y);
 }
-__device__ __forceinline__ float gelu_only(float u) {
-    const float t = tanh_fast(kGeluC * fmaf(kGeluA * u * u, u, u));
-    return 0.5f * u * (1.f + t);
+__device__ __forceinline__ void gelu_and_grad2(float u0, float u1, uint32_t& g, uint32_t& dg) {
+    const __half2 one = __float2half2_rn(1.f), half = __float2half2_rn(0.5f);
+    const __half2 u = __floats2half2_rn(u0, u1);
+    const __half2 u2 = __hmul2(u, u);
+    const __half2 t = tanh_fast_h2(__hmul2(__float2half2_rn(kGeluC), __hfma2(__hmul2(__float2half2_rn(kGeluA), u2), u, u)));
+    const __half2 opt = __hadd2(one, t);
+    g = h2_to_bf16x2(__hmul2(__hmul2(half, u), opt));
+    const __half2 omt2 = __hfma2(__hneg2(t), t, one);                            // 1 - t^2
+    const __half2 poly = __hfma2(__float2half2_rn(3.f * kGeluA), u2, one);      // 1 + 3 a u^2
+    dg = h2_to_bf16x2(__hfma2(__hmul2(__hmul2(__float2half2_rn(0.5f * kGeluC), u), omt2), poly, __hmul2(half, opt)));
+}
+__device__ __forceinline__ uint32_t gelu_only2(float u0, float u1) {
+    const __half2 u = __floats2half2_rn(u0, u1);
+    const __half2 t = tanh_fast_h2(__hmul2(__float2half2_rn(kGeluC),
+                                           __hfma2(__hmul2(__float2half2_rn(kGeluA), __hmul2(u, u)), u, u)));
+    return h2_to_bf16x2(__hmul2(__hmul2(__float2half2_rn(0.5f), u), __hadd2(__float2half2_rn(1.f), t)));
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -118,8 +137,8 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
         for (int i = 0; i < STAGES; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
         mbar_init(&s.mma_bar, 1);
         mbar_init(&s.free_bar, 1);
-        mbar_init(&s.xbar, 128);
-        mbar_init(&s.wbar, 128);
+        mbar_init(&s.xbar, kCT);
+        mbar_init(&s.wbar, kCT);
         fence_barrier_init();
         prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
     }
@@ -159,12 +178,14 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
         __syncwarp();                                          // the warp reaches the block barrier converged
     } else {
         // ---------------------------------------------------------------------------------------
-        // warps 1..4: tid 0 issues the MMAs, all 128 threads do the elementwise work.  Thread tid
-        // reads and writes accumulator row r (its TMEM lane): a token (or a hidden unit).
+        // warps 1..8: tid 0 issues the MMAs, all 256 threads do the elementwise work.  Thread tid
+        // reads and writes accumulator row r (its TMEM lane): a token (or a hidden unit); the two
+        // warps of a lane quarter take the two halves (hw) of each elementwise pass's columns.
         // ---------------------------------------------------------------------------------------
         const int tid = threadIdx.x - 32;
         const int q = warp & 3;
         const int r = q * 32 + lane;
+        const int hw = (warp - 1) >> 2;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const uint32_t sact = smem_u32(s.act[0]), swa = smem_u32(s.wa), swb = smem_u32(s.wb[0]), srz = smem_u32(s.rz);
         uint32_t mph = 0;                                       // mma_bar phase
@@ -177,7 +198,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
             if (tid == 0) mma_commit(&s.mma_bar);
             ok = mbar_wait(&s.mma_bar, mph, ab);
             mph ^= 1u;
-            if (named_bar_or(1, 128, !ok)) return false;
+            if (named_bar_or(1, kCT, !ok)) return false;
             __syncwarp();
             tc_fence_after();
             return true;
@@ -189,28 +210,34 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
             // ---- Wa, Wb of the head -> bf16 operands (coalesced float4 loads: consecutive threads read
             //      consecutive 16-byte pieces of a row)
             {
+                // all 16 of a thread's float4 of each matrix in flight before any is converted
                 const float4* Wa4 = reinterpret_cast<const float4*>(p.Wa + (size_t)h * HID * D);
                 const float4* Wb4 = reinterpret_cast<const float4*>(p.Wb + (size_t)h * D * HID);
-#pragma unroll 4
-                for (int f = tid; f < HID * D / 4; f += 128) {             // Wa: row = hidden unit, 16 float4 a row
-                    const float4 v = __ldg(Wa4 + f);
-                    const int row = f >> 4, col = (f & 15) * 4;
-                    *reinterpret_cast<uint2*>(s.wa + sw_off(row, col)) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+                constexpr int F4 = HID * D / 4 / kCT;
+                float4 v[F4];
+#pragma unroll
+                for (int i = 0; i < F4; ++i) v[i] = __ldg(Wa4 + i * kCT + tid);
+#pragma unroll
+                for (int i = 0; i < F4; ++i) {                             // Wa: row = hidden unit, 16 float4 a row
+                    const int f = i * kCT + tid, row = f >> 4, col = (f & 15) * 4;
+                    *reinterpret_cast<uint2*>(s.wa + sw_off(row, col)) =
+                        make_uint2(pack_bf16x2(v[i].x, v[i].y), pack_bf16x2(v[i].z, v[i].w));
                 }
-#pragma unroll 4
-                for (int f = tid; f < D * HID / 4; f += 128) {             // Wb: row = d, 64 float4 a row
-                    const float4 v = __ldg(Wb4 + f);
-                    const int d = f >> 6, col = (f & 63) * 4;
+#pragma unroll
+                for (int i = 0; i < F4; ++i) v[i] = __ldg(Wb4 + i * kCT + tid);
+#pragma unroll
+                for (int i = 0; i < F4; ++i) {                             // Wb: row = d, 64 float4 a row
+                    const int f = i * kCT + tid, d = f >> 6, col = (f & 63) * 4;
                     *reinterpret_cast<uint2*>(s.wb[col / 64] + sw_off(d, col % 64)) =
-                        make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+                        make_uint2(pack_bf16x2(v[i].x, v[i].y), pack_bf16x2(v[i].z, v[i].w));
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
             }
             // ---- phase 1 over this CTA's tiles
             for (int t = t0; t < t1 && !failed; ++t) {
                 bool ok = mbar_wait(&s.full[st], ph, ab);
-                if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                if (named_bar_or(1, kCT, !ok)) { failed = true; break; }
                 const uint32_t sK = smem_u32(s.stage[st]);
                 const uint8_t* vtile = s.stage[st] + TILE;
                 // H = K Wa^T
@@ -222,39 +249,38 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                                     kIdH, kk > 0 ? 1u : 0u);
                 }
                 if (!mma_sync(ok)) { failed = true; break; }
-                // A = gelu(H) -> act (bf16); gelu'(H) packed bf16x2 -> TMEM cols 256 + hid/2
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {                          // 64 hidden units per chunk
-                    float hv[4][16];
+                // A = gelu(H) -> act (bf16); gelu'(H) packed bf16x2 -> TMEM cols 256 + hid/2.  Half hw
+                // takes the 64-hidden chunks 2 hw and 2 hw + 1; the packed gelu' overwrites H columns
+                // the other half may still read, so it is written back after a barrier
+                uint32_t gp[2][2][16];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 256u + (uint32_t)(c * 64 + j * 16) + lane_off, hv[j]);
-                    tmem_ld_wait();
-                    uint32_t gp[32];
+                for (int ci = 0; ci < 2; ++ci) {
+                    const int c = 2 * hw + ci;                         // 64 hidden units per chunk
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        float a[16], dg[16];
+                        float hv[16];
+                        tmem_ld16(tmem + 256u + (uint32_t)(c * 64 + j * 16) + lane_off, hv);
+                        tmem_ld_wait();
+                        uint32_t aw[8];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) gelu_and_grad(hv[j][e], a[e], dg[e]);
-#pragma unroll
-                        for (int e = 0; e < 16; e += 8) {
-                            uint4 pk;
-                            pk.x = pack_bf16x2(a[e], a[e + 1]); pk.y = pack_bf16x2(a[e + 2], a[e + 3]);
-                            pk.z = pack_bf16x2(a[e + 4], a[e + 5]); pk.w = pack_bf16x2(a[e + 6], a[e + 7]);
-                            *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16 + e)) = pk;
-                        }
-#pragma unroll
-                        for (int e = 0; e < 16; e += 2) gp[j * 8 + e / 2] = pack_bf16x2(dg[e], dg[e + 1]);
+                        for (int e = 0; e < 16; e += 2) gelu_and_grad2(hv[e], hv[e + 1], aw[e / 2], gp[ci][j / 2][(j % 2) * 8 + e / 2]);
+                        *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16)) = make_uint4(aw[0], aw[1], aw[2], aw[3]);
+                        *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16 + 8)) = make_uint4(aw[4], aw[5], aw[6], aw[7]);
                     }
-                    uint32_t g0[16], g1[16];
+                }
+                tc_fence_before();
+                named_bar_sync(1, kCT);                                // every H column has been read
+                tc_fence_after();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) { g0[e] = gp[e]; g1[e] = gp[16 + e]; }
-                    tmem_st16(tmem + 256u + (uint32_t)(c * 32) + lane_off, g0);
-                    tmem_st16(tmem + 256u + (uint32_t)(c * 32 + 16) + lane_off, g1);
+                for (int ci = 0; ci < 2; ++ci) {
+                    const int c = 2 * hw + ci;
+                    tmem_st16(tmem + 256u + (uint32_t)(c * 32) + lane_off, gp[ci][0]);
+                    tmem_st16(tmem + 256u + (uint32_t)(c * 32 + 16) + lane_off, gp[ci][1]);
                 }
                 tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
                 // Y = A Wb^T
                 if (tid == 0) {
                     tc_fence_after();
@@ -265,21 +291,22 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                                     kk > 0 ? 1u : 0u);
                 }
                 if (!mma_sync(ok)) { failed = true; break; }
-                // R = Y - V -> rz (bf16)
+                // R = Y - V -> rz (bf16); half hw takes columns 32 hw .. 32 hw + 31
                 {
-                    float yv[4][16];
+                    float yv[2][16];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 384u + (uint32_t)(j * 16) + lane_off, yv[j]);
+                    for (int j = 0; j < 2; ++j) tmem_ld16(tmem + 384u + (uint32_t)(hw * 32 + j * 16) + lane_off, yv[j]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < D; c += 8) {
+                    for (int cc = 0; cc < 32; cc += 8) {
+                        const int c = hw * 32 + cc;
                         const uint4 vv = *reinterpret_cast<const uint4*>(vtile + sw_off(r, c));
                         const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
                         float rr[8];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            rr[2 * e] = yv[c / 16][(c % 16) + 2 * e] - bf16lo_to_f32(vw[e]);
-                            rr[2 * e + 1] = yv[c / 16][(c % 16) + 2 * e + 1] - bf16hi_to_f32(vw[e]);
+                            rr[2 * e] = yv[cc / 16][(cc % 16) + 2 * e] - bf16lo_to_f32(vw[e]);
+                            rr[2 * e + 1] = yv[cc / 16][(cc % 16) + 2 * e + 1] - bf16hi_to_f32(vw[e]);
                         }
                         uint4 pk;
                         pk.x = pack_bf16x2(rr[0], rr[1]); pk.y = pack_bf16x2(rr[2], rr[3]);
@@ -289,7 +316,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
                 // gWb^T += A^T R (two hidden halves) and dA_0 = R Wb (hidden 0..127)
                 if (tid == 0) {
                     tc_fence_after();
@@ -320,34 +347,37 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                         }
                         if (!mma_sync(ok)) { failed = true; break; }
                     }
-#pragma unroll 1
-                    for (int c = 0; c < 2; ++c) {                       // 64 hidden units per chunk
-                        float da[4][16];
-                        float gq[2][16];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 384u + (uint32_t)(c * 64 + j * 16) + lane_off, da[j]);
-                        tmem_ld16(tmem + 256u + (uint32_t)(half * 64 + c * 32) + lane_off, gq[0]);
-                        tmem_ld16(tmem + 256u + (uint32_t)(half * 64 + c * 32 + 16) + lane_off, gq[1]);
-                        tmem_ld_wait();
+                    {
+                        const int c = hw;                                // 64 hidden units per chunk
                         const int panel = half * 2 + c;
 #pragma unroll
-                        for (int e = 0; e < 64; e += 8) {
-                            float dh[8];
+                        for (int sub = 0; sub < 2; ++sub) {              // 32 hidden units at a time
+                            float da[2][16];
+                            float gq[16];
 #pragma unroll
-                            for (int i = 0; i < 8; i += 2) {
-                                const uint32_t w = __float_as_uint(gq[(e + i) / 32][((e + i) % 32) / 2]);
-                                dh[i] = da[(e + i) / 16][(e + i) % 16] * bf16lo_to_f32(w);
-                                dh[i + 1] = da[(e + i + 1) / 16][(e + i + 1) % 16] * bf16hi_to_f32(w);
+                            for (int j = 0; j < 2; ++j)
+                                tmem_ld16(tmem + 384u + (uint32_t)(c * 64 + sub * 32 + j * 16) + lane_off, da[j]);
+                            tmem_ld16(tmem + 256u + (uint32_t)(half * 64 + c * 32 + sub * 16) + lane_off, gq);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; e += 8) {
+                                float dh[8];
+#pragma unroll
+                                for (int i = 0; i < 8; i += 2) {
+                                    const uint32_t w = __float_as_uint(gq[(e + i) / 2]);
+                                    dh[i] = da[(e + i) / 16][(e + i) % 16] * bf16lo_to_f32(w);
+                                    dh[i + 1] = da[(e + i + 1) / 16][(e + i + 1) % 16] * bf16hi_to_f32(w);
+                                }
+                                uint4 pk;
+                                pk.x = pack_bf16x2(dh[0], dh[1]); pk.y = pack_bf16x2(dh[2], dh[3]);
+                                pk.z = pack_bf16x2(dh[4], dh[5]); pk.w = pack_bf16x2(dh[6], dh[7]);
+                                *reinterpret_cast<uint4*>(s.act[panel] + sw_off(r, sub * 32 + e)) = pk;
                             }
-                            uint4 pk;
-                            pk.x = pack_bf16x2(dh[0], dh[1]); pk.y = pack_bf16x2(dh[2], dh[3]);
-                            pk.z = pack_bf16x2(dh[4], dh[5]); pk.w = pack_bf16x2(dh[6], dh[7]);
-                            *reinterpret_cast<uint4*>(s.act[panel] + sw_off(r, e)) = pk;
                         }
                     }
                     fence_proxy_async_smem();
                     tc_fence_before();
-                    named_bar_sync(1, 128);
+                    named_bar_sync(1, kCT);
                 }
                 if (failed) break;
                 // gWa += dH^T K (two hidden halves); frees the K/V stage when done
@@ -385,13 +415,13 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                     if (tid == 0) mbar_arrive_remote(map_to_rank(smem_u32(&s.free_bar), (uint32_t)peer));
                     // (2) and the peer's phase 1 is over
                     ok = mbar_wait_cluster(&s.free_bar, k & 1u, ab);
-                    if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                    if (named_bar_or(1, kCT, !ok)) { failed = true; break; }
                     tc_fence_after();
                     // (3) push my partials for the peer's half into the peer's act
                     const int ob = peer;
                     const uint32_t rb = map_to_rank(smem_u32(recv), (uint32_t)peer);
 #pragma unroll 1
-                    for (int j = 0; j < 4; ++j) {
+                    for (int j = 2 * hw; j < 2 * hw + 2; ++j) {
                         float ga[16], gb[16];
                         tmem_ld16(tmem + 128u + (uint32_t)(ob * 64 + j * 16) + lane_off, ga);
                         tmem_ld16(tmem + (uint32_t)(ob * 64 + j * 16) + lane_off, gb);
@@ -411,7 +441,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                     mbar_arrive_remote(map_to_rank(smem_u32(&s.xbar), (uint32_t)peer));   // after my stores
                     // (4) the peer's partials for my half
                     ok = mbar_wait_cluster(&s.xbar, k & 1u, ab);
-                    if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                    if (named_bar_or(1, kCT, !ok)) { failed = true; break; }
                 }
                 const float* Wa = p.Wa + (size_t)h * HID * D;
                 const float* Wb = p.Wb + (size_t)h * D * HID;
@@ -420,37 +450,45 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
 #pragma unroll 1
                 for (int hb = multi ? rank : 0; hb < (multi ? rank + 1 : 2); ++hb) {
                     const int hid = hb * 128 + r;
-                    float ga[4][16], gb[4][16];
+                    const int c0 = hw * 32;                           // this half's 32 columns
+                    // the initial weights of this thread's entries, all loads in flight at once
+                    float4 wa0[8];
+                    float wb0[32];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tmem_ld16(tmem + 128u + (uint32_t)(hb * 64 + j * 16) + lane_off, ga[j]);
-                        tmem_ld16(tmem + (uint32_t)(hb * 64 + j * 16) + lane_off, gb[j]);
+                    for (int i = 0; i < 8; ++i) wa0[i] = __ldg(reinterpret_cast<const float4*>(Wa + (size_t)hid * D + c0) + i);
+#pragma unroll
+                    for (int dd = 0; dd < 32; ++dd) wb0[dd] = __ldg(Wb + (size_t)(c0 + dd) * HID + hid);
+                    float ga[2][16], gb[2][16];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        tmem_ld16(tmem + 128u + (uint32_t)(hb * 64 + c0 + j * 16) + lane_off, ga[j]);
+                        tmem_ld16(tmem + (uint32_t)(hb * 64 + c0 + j * 16) + lane_off, gb[j]);
                     }
                     tmem_ld_wait();
                     if (!has) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < 2; ++j)
 #pragma unroll
                             for (int e = 0; e < 16; ++e) { ga[j][e] = 0.f; gb[j][e] = 0.f; }
                     }
                     if (multi) {                                      // + the peer's partial (two terms: any order)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < 2; ++j)
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                ga[j][e] += *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(recv) + roff(0, r, j * 16 + e));
-                                gb[j][e] += *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(recv) + roff(1, r, j * 16 + e));
+                                ga[j][e] += *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(recv) + roff(0, r, c0 + j * 16 + e));
+                                gb[j][e] += *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(recv) + roff(1, r, c0 + j * 16 + e));
                             }
                     }
 #pragma unroll
-                    for (int c = 0; c < D; c += 8) {
+                    for (int cc = 0; cc < 32; cc += 8) {
+                        const int c = c0 + cc;
                         float w[8];
-                        const float4 w0a = __ldg(reinterpret_cast<const float4*>(Wa + (size_t)hid * D + c));
-                        const float4 w0b = __ldg(reinterpret_cast<const float4*>(Wa + (size_t)hid * D + c + 4));
+                        const float4 w0a = wa0[cc / 4], w0b = wa0[cc / 4 + 1];
                         const float w0[8] = {w0a.x, w0a.y, w0a.z, w0a.w, w0b.x, w0b.y, w0b.z, w0b.w};
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            w[e] = w0[e] - p.eta_scale * ga[(c + e) / 16][(c + e) % 16];
+                            w[e] = w0[e] - p.eta_scale * ga[(cc + e) / 16][(cc + e) % 16];
                             if (p.Wa_out) p.Wa_out[((size_t)u * HID + hid) * D + c + e] = w[e];
                         }
                         uint4 pk;
@@ -460,8 +498,9 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                         if (multi) st_cluster_v4(pwa + sw_off(hid, c), pk);
                     }
 #pragma unroll
-                    for (int d = 0; d < D; ++d) {
-                        const float w = __ldg(Wb + (size_t)d * HID + hid) - p.eta_scale * gb[d / 16][d % 16];
+                    for (int dd = 0; dd < 32; ++dd) {
+                        const int d = c0 + dd;
+                        const float w = wb0[dd] - p.eta_scale * gb[dd / 16][dd % 16];
                         if (p.Wb_out) p.Wb_out[((size_t)u * D + d) * HID + hid] = w;
                         const __nv_bfloat16 wb16 = __float2bfloat16_rn(w);
                         const uint32_t off = (uint32_t)((hid / 64) * (D * 128)) + sw_off(d, hid % 64);
@@ -476,16 +515,16 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                     mbar_arrive_remote(map_to_rank(smem_u32(&s.wbar), (uint32_t)peer));   // after my stores
                     // (5) the peer's half of the operands
                     ok = mbar_wait_cluster(&s.wbar, k & 1u, ab);
-                    if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                    if (named_bar_or(1, kCT, !ok)) { failed = true; break; }
                 }
                 fence_proxy_async_smem();                             // the operands are read by the tensor cores
                 tc_fence_before();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
             }
             // ---- phase 2: Z = gelu(Q Wa1^T) Wb1^T over this CTA's tiles
             for (int t = t0; t < t1 && !failed; ++t) {
                 bool ok = mbar_wait(&s.full[st], ph, ab);
-                if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+                if (named_bar_or(1, kCT, !ok)) { failed = true; break; }
                 const uint32_t sQ = smem_u32(s.stage[st]);
                 if (tid == 0) {
                     tc_fence_after();
@@ -496,27 +535,22 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                 }
                 if (!mma_sync(ok)) { failed = true; break; }
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float hv[4][16];
+                for (int c = 2 * hw; c < 2 * hw + 2; ++c) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 256u + (uint32_t)(c * 64 + j * 16) + lane_off, hv[j]);
-                    tmem_ld_wait();
+                    for (int j = 0; j < 4; ++j) {
+                        float hv[16];
+                        tmem_ld16(tmem + 256u + (uint32_t)(c * 64 + j * 16) + lane_off, hv);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-#pragma unroll
-                        for (int e = 0; e < 16; e += 8) {
-                            float a[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) a[i] = gelu_only(hv[j][e + i]);
-                            uint4 pk;
-                            pk.x = pack_bf16x2(a[0], a[1]); pk.y = pack_bf16x2(a[2], a[3]);
-                            pk.z = pack_bf16x2(a[4], a[5]); pk.w = pack_bf16x2(a[6], a[7]);
-                            *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16 + e)) = pk;
-                        }
+                        for (int e = 0; e < 16; e += 8)
+                            *reinterpret_cast<uint4*>(s.act[c] + sw_off(r, j * 16 + e)) =
+                                make_uint4(gelu_only2(hv[e], hv[e + 1]), gelu_only2(hv[e + 2], hv[e + 3]),
+                                           gelu_only2(hv[e + 4], hv[e + 5]), gelu_only2(hv[e + 6], hv[e + 7]));
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
                 if (tid == 0) {
                     tc_fence_after();
 #pragma unroll
@@ -528,25 +562,26 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                 }
                 if (!mma_sync(ok)) { failed = true; break; }
                 if (tid == 0 && zn > 0) bulk_wait_read<0>();          // the previous Z tile has left rz
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
                 {
-                    float zv[4][16];
+                    float zv[2][16];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) tmem_ld16(tmem + 384u + (uint32_t)(j * 16) + lane_off, zv[j]);
+                    for (int j = 0; j < 2; ++j) tmem_ld16(tmem + 384u + (uint32_t)(hw * 32 + j * 16) + lane_off, zv[j]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < D; c += 8) {
+                    for (int cc = 0; cc < 32; cc += 8) {
+                        const int c = hw * 32 + cc;
                         uint4 pk;
-                        pk.x = pack_bf16x2(zv[c / 16][c % 16], zv[c / 16][c % 16 + 1]);
-                        pk.y = pack_bf16x2(zv[c / 16][c % 16 + 2], zv[c / 16][c % 16 + 3]);
-                        pk.z = pack_bf16x2(zv[c / 16][c % 16 + 4], zv[c / 16][c % 16 + 5]);
-                        pk.w = pack_bf16x2(zv[c / 16][c % 16 + 6], zv[c / 16][c % 16 + 7]);
+                        pk.x = pack_bf16x2(zv[cc / 16][cc % 16], zv[cc / 16][cc % 16 + 1]);
+                        pk.y = pack_bf16x2(zv[cc / 16][cc % 16 + 2], zv[cc / 16][cc % 16 + 3]);
+                        pk.z = pack_bf16x2(zv[cc / 16][cc % 16 + 4], zv[cc / 16][cc % 16 + 5]);
+                        pk.w = pack_bf16x2(zv[cc / 16][cc % 16 + 6], zv[cc / 16][cc % 16 + 7]);
                         *reinterpret_cast<uint4*>(s.rz + sw_off(r, c)) = pk;
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kCT);
                 if (tid == 0) {
                     tma_store_4d(&tmZ, s.rz, 0, t * TOK, h, bi);
                     bulk_commit();
@@ -555,7 +590,7 @@ mlp_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUten
                 if (++st == STAGES) { st = 0; ph ^= 1u; }
             }
             if (tid == 0) bulk_wait<0>();                          // rz is reused by the next unit
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kCT);
         }
         if (tid == 0) bulk_wait<0>();
     }
