@@ -62,7 +62,7 @@ TRAFFIC = {
 
 # Kernels of this library launched per step, by workload kind (bf16; fp32 where it differs).
 LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backward": 3, "backward_conv": 4,
-                     "backward_mlp": 7, "conv3x3": 3}
+                     "backward_mlp": 7, "conv3x3": 4}
 LAUNCHES_PER_STEP_FP32 = {"linear": 2, "mixed": 3}
 
 
@@ -579,7 +579,7 @@ def roofline(w, t_step, pk, clocks, xs, stream, args):
         return roof
     if w.kind in ("mlp", "conv3x3"):
         kern = "mlp_fused (the whole ttt_forward_mlp call)" if w.kind == "mlp" else \
-               "conv3_grad + conv3_merge + conv3_readout (the whole ttt_forward_conv3x3 call)"
+               "conv3_wprep + conv3_grad + conv3_merge + conv3_readout (the whole ttt_forward_conv3x3 call)"
         tf = flops / t_step / 1e12
         return {"bound": "tensor", "kernel": kern, "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tf / pk["bf16_tflops"], "peak_source": pk["source"] + " (bf16 burst)",

@@ -151,8 +151,9 @@ ttt_status ttt_forward_dwconv(const void* Q, const void* K, const void* V, const
  *   operands and fp32 accumulation: W0 is rounded to bf16 for the residual, the residual is carried
  *   as two bf16 parts (about 16 significant bits), W1 is rounded once to bf16 for the readout.
  *   bf16 and TTT_LOSS_L2 only (fp32 or TTT_LOSS_DOT returns TTT_ERR_UNSUPPORTED).
- *   ws: ttt_workspace_bytes(TTT_HEAD_CONV3X3, s) bytes (per-CTA partial gradients of 144 KB each and
- *   the updated weights as bf16 operand images); it needs no zero fill, every call writes what it reads.
+ *   ws: ttt_workspace_bytes(TTT_HEAD_CONV3X3, s) bytes (per-CTA partial gradients of 144 KB each, and
+ *   W0 and the updated weights as bf16 operand images); it needs no zero fill, every call writes what
+ *   it reads.
  *   Work is split over CTAs in fixed ranges: results are bitwise reproducible for a fixed SM budget.
  */
 ttt_status ttt_forward_conv3x3(const void* Q, const void* K, const void* V, const float* W0,

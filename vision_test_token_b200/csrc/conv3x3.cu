@@ -15,7 +15,10 @@
 // origin, whose out-of-bounds zero fill is the zero padding.  Tiles are 8 rows x 16 columns of the
 // grid (128 positions, the MMA's M).
 //
-// Three kernels on one stream, each a programmatic dependent of the one before:
+// Four kernels on one stream, each a programmatic dependent of the one before:
+//   conv3_wprep   W0 rounded to bf16 and laid out as nine swizzled tap operand images per head (row
+//                 c, K = c'), once per call, so that each gradient CTA loads its head's weights with
+//                 one bulk copy instead of gathering them from the [c][c'][a][b] layout.
 //   conv3_grad    (per CTA, a contiguous range of tiles; per tile) TMA loads V and the 9 K boxes
 //                 (two taps per 32 KB ring stage); R = K~ W0~^T accumulates over the taps (A = K box,
 //                 K-major; B = W0 tap image, rows c, K = c'); the epilogue forms r = R - V, zeroes
@@ -23,7 +26,8 @@
 //                 bits); the 9 K boxes are streamed again and G^T += [K_t | K_t+1]^T (r_hi + r_lo)
 //                 accumulates in five tap-pair accumulators (A MN-major, M = 128 = two taps' channels;
 //                 B = r, MN-major).  At the end of each unit's part of the range the accumulators
-//                 are written to the workspace slot of (CTA, unit).
+//                 are written to the workspace slot of (CTA, unit), as G[tap][c][c'] so that the
+//                 32 lanes of a warp (32 consecutive c') store one 128-byte line per instruction.
 //   conv3_merge   per (unit, tap): the unit's slots summed in CTA order (a fixed order: bitwise
 //                 reproducible for a given grid), W1 = W0 - eta (2/N) g in fp32 (W1_out), and W1
 //                 rounded once to bf16 as the tap's operand image for the readout.
@@ -52,7 +56,7 @@ constexpr int S3 = 3;                       // ring stages of the readout kernel
 constexpr int kWImg = D * D * 2;            // one tap's weights as a bf16 operand image: 8 KB
 constexpr int kThreads = 192;
 constexpr int kMaxGrid = 160;               // slots of the workspace: (kMaxGrid + units)
-constexpr int kSlotFloats = TAPS * D * D;   // one gradient partial, G^T [tap][c'][c]
+constexpr int kSlotFloats = TAPS * D * D;   // one gradient partial, G [tap][c][c']
 constexpr uint32_t kIdescRow = idesc_bf16_f32(128, 64, false, false);  // D[pos][c] = sum_k A[pos][k] B[c][k]
 constexpr uint32_t kIdescCol = idesc_bf16_f32(128, 64, true, true);    // D[m][c] = sum_pos A[pos][m] B[pos][c]
 constexpr uint32_t kColR = 0;               // tensor memory: two R accumulators,
@@ -102,11 +106,29 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // ------------------------------------------------------------------------------------------------
 // conv3_grad
 // ------------------------------------------------------------------------------------------------
+// ------------------------------------------------------------------------------------------------
+// conv3_wprep: one CTA per (head, output channel c), one thread per input channel c'
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(D)
+conv3_wprep(const float* __restrict__ W0, uint8_t* __restrict__ w0img) {
+    const int h = blockIdx.x / D, c = blockIdx.x % D, cp = threadIdx.x;
+    pdl_wait_primary();                                      // the previous call's kernels are done with the images
+    pdl_launch_dependents();
+    const float* w = W0 + (((size_t)h * D + c) * D + cp) * TAPS;
+    float v[TAPS];
+#pragma unroll
+    for (int t9 = 0; t9 < TAPS; ++t9) v[t9] = __ldg(w + t9);
+#pragma unroll
+    for (int t9 = 0; t9 < TAPS; ++t9)
+        *reinterpret_cast<__nv_bfloat16*>(w0img + ((size_t)h * TAPS + t9) * kWImg + sw_off(c, cp / 8) + (cp % 8) * 2) =
+            __float2bfloat16_rn(v[t9]);
+}
+
 struct GradParams {
     Geo g;
     int G;                                   // CTAs
-    const float* W0;                         // [heads][64][64][9]
-    float* slots;                            // [(kMaxGrid + U)][9][64][64]: G^T of a (CTA, unit) part
+    const uint8_t* w0img;                    // [heads][9][kWImg], written by conv3_wprep
+    float* slots;                            // [(kMaxGrid + U)][9][64][64]: G of a (CTA, unit) part
     uint32_t* err;
     unsigned long long wait_ns;
 };
@@ -130,11 +152,20 @@ struct GradSmem {
 __device__ __forceinline__ void grad_producer(GradSmem& s, const GradParams& p, const CUtensorMap* tmK,
                                               const CUtensorMap* tmV, const Abort& ab) {
     const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    uint32_t issued = 0, vq = 0;
+    uint32_t issued = 0, vq = 0, parts = 0;
     int st = 0; uint32_t ph = 0;
     bool ok = true;
     for (long long t = t0; t < t1 && ok; ++t) {
         const TileXY x = tile_xy(p.g, t);
+        if (t == t0 || x.u != (int)((t - 1) / p.g.tpu)) {
+            // a part starts: the head's W0 tap images, once the previous part's R MMAs are done with them
+            if (t == t0) pdl_wait_primary();                 // conv3_wprep has written the images
+            if (!(ok = mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab))) break;
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
+            bulk_g2s(s.w0img, p.w0img + (size_t)x.h * TAPS * kWImg, TAPS * kWImg, &s.w_full);
+            ++parts;
+        }
         if (!(ok = mbar_wait(&s.vempty, (vq & 1u) ^ 1u, ab))) break;
         mbar_arrive_expect_tx(&s.vfull, BOX);
         tma_load_5d(s.vbuf, tmV, &s.vfull, 0, x.x0, x.y0, x.h, x.b);
@@ -156,6 +187,7 @@ __device__ __forceinline__ void grad_producer(GradSmem& s, const GradParams& p, 
     for (uint32_t k = issued > (uint32_t)S1 ? issued - S1 : 0u; k < issued; ++k)
         mbar_drain(&s.full[k % S1], (k / S1) & 1u, ab.limit);
     if (vq > 0) mbar_drain(&s.vfull, (vq - 1) & 1u, ab.limit);
+    if (parts > 0) mbar_drain(&s.w_full, (parts - 1) & 1u, ab.limit);
 }
 
 __device__ __forceinline__ void grad_mma(GradSmem& s, const GradParams& p, uint32_t tmem, const Abort& ab) {
@@ -225,28 +257,8 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
     bool failed = false;
     for (long long t = t0; t < t1 && !failed;) {
         const int u = (int)(t / p.g.tpu);
-        const int h = u % p.g.heads;
         const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
-        // the head's W0 as nine bf16 operand images (row c, K = c'), once the previous part's R MMAs
-        // are done reading them
-        bool ok = mbar_wait(&s.w_empty, (part & 1u) ^ 1u, ab);
-        if (named_bar_or(1, 128, !ok)) break;
-        {
-            const int c = tid >> 1, cp0 = (tid & 1) * 32;
-            const float* w = p.W0 + (((size_t)h * D + c) * D + cp0) * TAPS;
-            for (int t9 = 0; t9 < TAPS; ++t9) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float v[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __ldg(w + (size_t)(8 * j + e) * TAPS + t9);
-                    *reinterpret_cast<uint4*>(s.w0img[t9] + sw_off(c, cp0 / 8 + j)) = pack8(v);
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (tid == 0) mbar_arrive(&s.w_full);
+        bool ok = true;
         for (long long tt = t; tt < pe; ++tt, ++n) {
             const TileXY x = tile_xy(p.g, tt);
             const uint32_t dr = n & 1u;
@@ -306,10 +318,9 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
             tmem_ld_wait();
             const int t9 = 2 * k + r / D;
             if (t9 < TAPS) {
-                float4* dst = reinterpret_cast<float4*>(slot + ((size_t)t9 * D + (r % D)) * D);
+                float* dst = slot + (size_t)t9 * D * D + (r % D);    // G[t9][c][c' = r % 64]
 #pragma unroll
-                for (int j = 0; j < 16; ++j) dst[j] = make_float4(g[j / 4][(j % 4) * 4], g[j / 4][(j % 4) * 4 + 1],
-                                                                  g[j / 4][(j % 4) * 4 + 2], g[j / 4][(j % 4) * 4 + 3]);
+                for (int c = 0; c < D; ++c) __stcg(dst + (size_t)c * D, g[c / 16][c % 16]);
             }
         }
         tc_fence_before();
@@ -403,7 +414,7 @@ conv3_merge(const MergeParams p) {
     const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int e = 4 * e4 + i, cp = e / D, c = e % D;     // slot element G^T[t9][cp][c]
+        const int e = 4 * e4 + i, c = e / D, cp = e % D;     // slot element G[t9][c][cp]
         const size_t wi = (((size_t)h * D + c) * D + cp) * TAPS + t9;
         const float w1 = __ldg(p.W0 + wi) - p.g.eta_scale * a4[i];
         if (p.W1_out) p.W1_out[(((size_t)u * D + c) * D + cp) * TAPS + t9] = w1;
@@ -588,13 +599,14 @@ conv3_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 // Host side
 // ------------------------------------------------------------------------------------------------
 struct WsLayout {
-    size_t slots, w1img, total;
+    size_t slots, w1img, w0img, total;
 };
-static WsLayout ws_layout(long long units) {
+static WsLayout ws_layout(long long units, int heads) {
     WsLayout L;
     L.slots = kWsHeader;
     L.w1img = align_up(L.slots + (size_t)(kMaxGrid + units) * kSlotFloats * sizeof(float), 1024);
-    L.total = L.w1img + (size_t)units * TAPS * kWImg;
+    L.w0img = L.w1img + (size_t)units * TAPS * kWImg;
+    L.total = L.w0img + (size_t)heads * TAPS * kWImg;
     return L;
 }
 
@@ -612,13 +624,13 @@ static Geo make_geo(const Call& c) {
 
 }  // namespace c3
 
-size_t conv3x3_ws_bytes(const ttt_shape& s) { return c3::ws_layout((long long)s.batch * s.heads).total; }
+size_t conv3x3_ws_bytes(const ttt_shape& s) { return c3::ws_layout((long long)s.batch * s.heads, s.heads).total; }
 
 ttt_status launch_conv3x3(const Call& c) {
     using namespace c3;
     if (c.dtype != TTT_BF16 || c.loss != TTT_LOSS_L2) return TTT_ERR_UNSUPPORTED;
     const long long units = (long long)c.batch * c.heads;
-    const WsLayout L = ws_layout(units);
+    const WsLayout L = ws_layout(units, c.heads);
     if (c.ws_bytes < L.total) return TTT_ERR_WORKSPACE;
     const Geo g = make_geo(c);
     if (g.T > (1LL << 40)) return TTT_ERR_UNSUPPORTED;
@@ -633,7 +645,7 @@ ttt_status launch_conv3x3(const Call& c) {
     GradParams gp{};
     gp.g = g;
     gp.G = G1;
-    gp.W0 = c.W0;
+    gp.w0img = c.ws + L.w0img;
     gp.slots = reinterpret_cast<float*>(c.ws + L.slots);
     gp.err = err;
     gp.wait_ns = c.wait_ns;
@@ -646,13 +658,20 @@ ttt_status launch_conv3x3(const Call& c) {
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
 
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)G1);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = sm1;
+    cfg.gridDim = dim3((unsigned)(c.heads * D));
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = c.stream;
     cfg.attrs = pdl;
     cfg.numAttrs = c.overlap_previous ? 1 : 0;
-    ttt_status st = check_launch(cudaLaunchKernelEx(&cfg, conv3_grad, tmK, tmV, gp));
+    ttt_status st = check_launch(cudaLaunchKernelEx(&cfg, conv3_wprep, c.W0, c.ws + L.w0img));
+    if (st != TTT_OK) return st;
+
+    cfg.gridDim = dim3((unsigned)G1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sm1;
+    cfg.numAttrs = 1;
+    st = check_launch(cudaLaunchKernelEx(&cfg, conv3_grad, tmK, tmV, gp));
     if (st != TTT_OK) return st;
 
     MergeParams mp{};
