@@ -52,7 +52,7 @@ TRAFFIC = {
     "mixed6084_dot_bf16": {"read": 112324352, "write": 38272256, "src_sha": "88e63fe44a5cadc0"},
     "lin6400_bf16": {"read": 118183168, "write": 40068864, "src_sha": "e252f1ffc5b63f16"},
     "lin196_bf16": {"read": 14328832, "write": 599040, "src_sha": "e252f1ffc5b63f16"},
-    "mlp1024_bf16": {"read": 25482752, "write": 6326784, "src_sha": "f33d5474b3e7c44e"},
+    "mlp1024_bf16": {"read": 25533440, "write": 6981376, "src_sha": "e351f2e6a0775778"},
     "conv3x3_6084_bf16": {"read": 18741504, "write": 7558144, "src_sha": "2385ceaf5d3c5c3d"},
     "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
     "bwd6084_bf16": {"read": 208251136, "write": 113136640, "src_sha": "6ed6afd58a0eb27a"},
