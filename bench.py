@@ -61,9 +61,9 @@ TRAFFIC = {
 }
 
 # Kernels of this library launched per step, by workload kind (bf16; fp32 where it differs).
-LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backward": 3, "backward_conv": 4,
+LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backward": 4, "backward_conv": 4,
                      "backward_mlp": 7, "conv3x3": 4}
-LAUNCHES_PER_STEP_FP32 = {"linear": 2, "mixed": 3}
+LAUNCHES_PER_STEP_FP32 = {"linear": 2, "mixed": 3, "backward": 3}
 
 
 # The CUDA sources each workload kind runs (besides the shared headers and the host entry points).
@@ -584,6 +584,12 @@ def roofline(w, t_step, pk, clocks, xs, stream, args):
         return {"bound": "tensor", "kernel": kern, "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tf / pk["bf16_tflops"], "peak_source": pk["source"] + " (bf16 burst)",
                 "algorithmic_flops": flops, "hbm_gbs": hbm, "hbm_frac": hbm / pk["hbm_gbs"], **common}
+    if w.kind == "backward" and w.dtype == "bf16":
+        # two token-streaming phases on the tensor cores: HBM-bound (48 FLOP per byte at most)
+        kern = "lin_bwd_p1_tc + lin_bwd_merge_tc + lin_bwd_p2_tc + lin_bwd_sum (the whole ttt_backward_linear call)"
+        return {"bound": "hbm", "kernel": kern, "achieved": hbm, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm / pk["hbm_gbs"], "peak_source": pk["source"] + " (copy bandwidth)",
+                "algorithmic_flops": flops, "tflops": flops / t_step / 1e12, **common}
     names = {"backward": "lin_bwd_p1 + lin_bwd_p2 + lin_bwd_sum (the whole ttt_backward_linear call)",
              "backward_conv": "cb_reduce + cb_unit + cb_map + cb_final (the whole ttt_backward_dwconv call)",
              "backward_mlp": "mb_prep .. mb_final, 7 kernels (the whole ttt_backward_mlp call)",

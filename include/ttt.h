@@ -238,8 +238,10 @@ ttt_status ttt_forward_linear_minibatch(const void* Q, const void* K, const void
  *   deta_out: optional, one fp32, summed over every (image, head) unit in index order.
  *   ws: ttt_workspace_bytes(TTT_HEAD_LINEAR_BACKWARD, s) bytes, zero-filled once
  *   (ttt_workspace_init); it holds per-unit partial sums and matrices.
- * Computed in fp32 from bf16 or fp32 inputs (outputs rounded to the input dtype); deterministic.
- * s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED). */
+ * fp32 inputs: computed in fp32 throughout.  bf16 inputs (tensor cores): the token sums G, C, dW1 are
+ * exact products accumulated in fp32, the unit matrices are formed in fp32, and the per-token maps
+ * multiply by them split into two bf16 parts (about 16 significant bits).  Outputs are rounded to the
+ * input dtype; deterministic.  s->loss must be TTT_LOSS_L2 (else TTT_ERR_UNSUPPORTED). */
 ttt_status ttt_backward_linear(const void* Q, const void* K, const void* V, const float* W0, const void* dZ,
                                float eta, const ttt_shape* s, void* ws, size_t ws_bytes, void* dQ, void* dK,
                                void* dV, float* dW0_out, float* deta_out, void* stream);

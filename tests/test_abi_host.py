@@ -160,8 +160,9 @@ def test_backward_workspace_and_validation(lib):
     n = capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR_BACKWARD, s)
     units = 8 * 5
     # counters, then partial slots for up to 320 CTAs + one per unit ([G ; C ; dW1] = 192 x 64 fp32),
-    # the unit matrices (4 x 64 x 64), each unit's dW0 and deta
-    assert n > (320 + units) * 192 * 64 * 4 + units * 5 * 64 * 64 * 4
+    # the unit matrices (4 x 64 x 64), each unit's dW0 and deta, and the bf16 operand images of the
+    # per-token maps (8 x 64 x 64 bf16 per unit)
+    assert n > (320 + units) * 192 * 64 * 4 + units * 5 * 64 * 64 * 4 + units * 8 * 64 * 64 * 2
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR_BACKWARD, _shape(batch=0)) == 0
     fake = ctypes.c_void_p(1 << 20)
     far = ctypes.c_void_p(1 << 40)

@@ -8,8 +8,9 @@
 //     deta = -(2/N) sum_ij dW1_ij (W0 G - C)_ij,
 // dW0 summed over the images of each head and deta over every unit.
 //
-// Three kernels, plain fp32 FMA (a first, exact-arithmetic path; the contractions are the same
-// shapes as the forward's, so the tensor-core route of the forward applies to them):
+// bf16 runs on the tensor cores (lin_bwd_p1_tc, lin_bwd_merge_tc, lin_bwd_p2_tc below: the token sums
+// and the per-token maps are the forward's contraction shapes).  fp32 keeps three plain fp32 FMA
+// kernels, for fp32 accuracy:
 //   lin_bwd_p1  static partition of 128-token tiles over CTAs; each CTA accumulates its share of
 //               [G ; C ; dW1] (192 x 64) and writes it to a partial slot; the CTA that completes a
 //               unit sums the unit's slots in slot order (deterministic) and forms W1, dC, dC^T,
@@ -21,6 +22,7 @@
 // memory under half an SM's, so that two CTAs share every SM.
 //   lin_bwd_sum dW0 over images and deta over units, in index order.
 #include <algorithm>
+#include <type_traits>
 
 #include "sm100.cuh"
 #include "ttt_internal.h"
@@ -326,10 +328,420 @@ lin_bwd_sum(const Params p, int batch) {
 }
 
 // ------------------------------------------------------------------------------------------------
+// bf16 on the tensor cores (tcgen05, fp32 accumulation in tensor memory, tiles moved by TMA)
+//   lin_bwd_p1_tc     static partition of 128-token tiles over one CTA per SM.  Per tile the four
+//                     token boxes [K | V | dZ | Q] land in one 64 KB ring stage; two MMAs per
+//                     16-token step accumulate [K | V]^T K (M = 128: the G rows, then the C rows)
+//                     and [dZ | Q]^T Q (M = 128, of which the dZ rows are dW1).  At the end of each
+//                     unit's run of tiles the accumulators go to the (CTA, unit) partial slot.
+//   lin_bwd_merge_tc  one CTA per unit (programmatic dependent of p1): the slot sum and the unit's
+//                     matrices as in merge_unit, then the four maps of phase 2 as bf16 hi + lo
+//                     operand images (128-byte swizzled rows c, K = i).
+//   lin_bwd_p2_tc     static partition of 128-token tiles over one CTA per SM (programmatic
+//                     dependent of the merge): per tile the boxes dZ, K, V; dQ = dZ W1, dV = K dC^T,
+//                     dK = V dC + K (dG + dG^T), each against the hi and lo image; the
+//                     accumulators are drained to bf16 and stored by TMA.
+// ------------------------------------------------------------------------------------------------
+namespace tc {
+
+constexpr int BOX = TOK * D * 2;             // one 128-token box of one tensor: 16 KB
+constexpr int S1 = 3;                        // ring stages of p1 (four boxes each)
+constexpr int S2 = 2;                        // ring stages of p2 (three boxes each)
+constexpr int kImg = D * D * 2;              // one 64 x 64 bf16 operand image: 8 KB
+constexpr int kImgs = 8;                     // W1^T, dC, dC^T, dG + dG^T, each hi and lo
+constexpr int kThreads = 192;                // producer warp, MMA warp, four drain warps
+constexpr uint32_t kIdescSum = idesc_bf16_f32(128, 64, true, true);     // D[m][n] = sum_tok A[tok][m] B[tok][n]
+constexpr uint32_t kIdescMap = idesc_bf16_f32(128, 64, false, false);   // D[tok][c] = sum_i A[tok][i] B[c][i]
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+// 16-byte chunk j (elements 8j .. 8j+7) of row `row` of a 128-byte swizzled operand image.
+__device__ __forceinline__ uint32_t sw_off(int row, int j) { return (uint32_t)(row * 128 + ((j ^ (row & 7)) << 4)); }
+
+struct TcParams {
+    int tpu, heads;
+    Partition part;
+    float* partials;                         // [(G + units)][192][64]
+    const uint8_t* imgs;                     // [units][kImgs][kImg] (p2)
+    uint32_t* err;
+    unsigned long long wait_ns;
+};
+
+// ---------------------------------------------------------------- p1
+struct P1TcSmem {
+    uint8_t ring[S1][4 * BOX];               // K, V, dZ, Q
+    uint64_t full[S1], empty[S1];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t drain_bar;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ void p1_producer(P1TcSmem& s, const TcParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                            const CUtensorMap* tmZ, const CUtensorMap* tmQ, const Abort& ab) {
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    int st = 0; uint32_t ph = 0, issued = 0;
+    for (long long t = t0; t < t1; ++t) {
+        const int u = (int)(t / p.tpu), n0 = (int)(t % p.tpu) * TOK, h = u % p.heads, b = u / p.heads;
+        if (!mbar_wait(&s.empty[st], ph ^ 1u, ab)) break;
+        mbar_arrive_expect_tx(&s.full[st], 4 * BOX);
+        uint8_t* dst = s.ring[st];
+        tma_load_4d(dst + 0 * BOX, tmK, &s.full[st], 0, n0, h, b);
+        tma_load_4d(dst + 1 * BOX, tmV, &s.full[st], 0, n0, h, b);
+        tma_load_4d(dst + 2 * BOX, tmZ, &s.full[st], 0, n0, h, b);
+        tma_load_4d(dst + 3 * BOX, tmQ, &s.full[st], 0, n0, h, b);
+        ++issued;
+        if (++st == S1) { st = 0; ph ^= 1u; }
+    }
+    for (uint32_t k = issued > (uint32_t)S1 ? issued - S1 : 0u; k < issued; ++k)
+        mbar_drain(&s.full[k % S1], (k / S1) & 1u, ab.limit);
+}
+
+__device__ __forceinline__ void p1_mma(P1TcSmem& s, const TcParams& p, uint32_t tmem, const Abort& ab) {
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    int st = 0; uint32_t ph = 0, seg = 0;
+    for (long long t = t0; t < t1;) {
+        const int u = (int)(t / p.tpu);
+        const long long se = min(t1, (long long)(u + 1) * p.tpu);
+        const uint32_t ab2 = seg & 1u;
+        if (!mbar_wait(&s.acc_empty[ab2], ((seg >> 1) & 1u) ^ 1u, ab)) return;
+        tc_fence_after();
+        const uint32_t d1 = tmem + ab2 * 128u, d2 = d1 + 64u;
+        for (long long tt = t; tt < se; ++tt) {
+            if (!mbar_wait(&s.full[st], ph, ab)) return;
+            tc_fence_after();
+            const uint32_t k = smem_u32(s.ring[st]), z = k + 2 * BOX;
+#pragma unroll
+            for (int kk = 0; kk < TOK / 16; ++kk) {
+                const uint32_t acc = (tt == t && kk == 0) ? 0u : 1u;
+                const uint64_t bk = sdesc_sw128(k + kk * 2048, BOX, 1024);
+                mma_bf16_ss(d1, sdesc_sw128(k + kk * 2048, BOX, 1024), bk, kIdescSum, acc);   // [K | V]^T K
+                mma_bf16_ss(d2, sdesc_sw128(z + kk * 2048, BOX, 1024),
+                            sdesc_sw128(z + BOX + kk * 2048, BOX, 1024), kIdescSum, acc);     // [dZ | Q]^T Q
+            }
+            mma_commit(&s.empty[st]);
+            if (++st == S1) { st = 0; ph ^= 1u; }
+        }
+        mma_commit(&s.acc_full[ab2]);
+        ++seg;
+        t = se;
+    }
+}
+
+// Drain warps: TMEM lane r of the accumulators is row r of [G ; C] and (r < 64) row r of dW1.
+__device__ __forceinline__ void p1_drain(P1TcSmem& s, const TcParams& p, uint32_t tmem, const Abort& ab) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3, r = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    uint32_t seg = 0;
+    for (long long t = t0; t < t1;) {
+        const int u = (int)(t / p.tpu);
+        const long long se = min(t1, (long long)(u + 1) * p.tpu);
+        const uint32_t ab2 = seg & 1u;
+        const bool ok = mbar_wait(&s.acc_full[ab2], (seg >> 1) & 1u, ab);
+        if (named_bar_or(1, 128, !ok)) break;
+        __syncwarp();
+        tc_fence_after();
+        float g[4][16], w[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld16(tmem + ab2 * 128u + (uint32_t)(j * 16) + lane_off, g[j]);
+        if (q < 2) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + ab2 * 128u + 64u + (uint32_t)(j * 16) + lane_off, w[j]);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s.acc_empty[ab2]);
+        float* slot = p.partials + (size_t)(blockIdx.x + u) * kPartial;
+        float4* d1 = reinterpret_cast<float4*>(slot + (size_t)r * D);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) d1[j] = make_float4(g[j / 4][(j % 4) * 4], g[j / 4][(j % 4) * 4 + 1],
+                                                         g[j / 4][(j % 4) * 4 + 2], g[j / 4][(j % 4) * 4 + 3]);
+        if (q < 2) {
+            float4* d2 = reinterpret_cast<float4*>(slot + (size_t)(2 * D + r) * D);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) d2[j] = make_float4(w[j / 4][(j % 4) * 4], w[j / 4][(j % 4) * 4 + 1],
+                                                             w[j / 4][(j % 4) * 4 + 2], w[j / 4][(j % 4) * 4 + 3]);
+        }
+        ++seg;
+        t = se;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+lin_bwd_p1_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+              const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    P1TcSmem& s = *reinterpret_cast<P1TcSmem*>(align1024(smem_raw));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
+    if (threadIdx.x == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < S1; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
+        mbar_init(&s.drain_bar, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmZ); prefetch_tmap(&tmQ);
+    }
+    if (warp == 1) { tmem_alloc(&s.tmem_base, 256); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch_dependents();
+    const uint32_t tmem = s.tmem_base;
+    if (warp == 0) {
+        if (lane == 0) p1_producer(s, p, &tmK, &tmV, &tmZ, &tmQ, ab);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            p1_mma(s, p, tmem, ab);
+            mma_commit(&s.drain_bar);
+            mbar_drain(&s.drain_bar, 0u, ab.limit);
+        }
+        __syncwarp();
+    } else {
+        p1_drain(s, p, tmem, ab);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------- merge
+// The unit's matrices (merge_unit), then the operand images of phase 2, image x holding X[c][i]:
+//   0/1 W1^T (dQ = dZ W1),  2/3 dC (dV = K dC^T),  4/5 dC^T (dK = V dC + ..),  6/7 dG + dG^T (symmetric),
+// each rounded to bf16 (hi) with the rounding error rounded again (lo).
+__global__ void __launch_bounds__(P1_THREADS)
+lin_bwd_merge_tc(const Params p, uint8_t* imgs) {
+    extern __shared__ uint8_t smem_raw[];
+    P1Smem& s = *reinterpret_cast<P1Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int u = blockIdx.x;
+    pdl_wait_primary();                      // every partial slot is written
+    pdl_launch_dependents();
+    const int cf = p.part.cta_of((long long)u * p.tpu), cl = p.part.cta_of((long long)(u + 1) * p.tpu - 1);
+    merge_unit<__nv_bfloat16>(p, s, u, cf + u, cl - cf + 1);
+    __syncthreads();                         // the unit's matrices are in global memory
+    const float* M = p.mats + (size_t)u * kMats * D * D;
+    uint8_t* out = imgs + (size_t)u * kImgs * kImg;
+    for (int e = threadIdx.x; e < 4 * D * (D / 8); e += P1_THREADS) {
+        const int m = e / (D * (D / 8)), c = (e / (D / 8)) % D, j = e % (D / 8);
+        float hi[8], lo[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = 8 * j + k;
+            const float x = (m == 0) ? M[(size_t)i * D + c] : M[(size_t)m * D * D + (size_t)c * D + i];
+            hi[k] = __bfloat162float(__float2bfloat16_rn(x));
+            lo[k] = x - hi[k];
+        }
+        uint4 h4, l4;
+        h4.x = pack_bf16x2(hi[0], hi[1]); h4.y = pack_bf16x2(hi[2], hi[3]);
+        h4.z = pack_bf16x2(hi[4], hi[5]); h4.w = pack_bf16x2(hi[6], hi[7]);
+        l4.x = pack_bf16x2(lo[0], lo[1]); l4.y = pack_bf16x2(lo[2], lo[3]);
+        l4.z = pack_bf16x2(lo[4], lo[5]); l4.w = pack_bf16x2(lo[6], lo[7]);
+        *reinterpret_cast<uint4*>(out + (size_t)(2 * m) * kImg + sw_off(c, j)) = h4;
+        *reinterpret_cast<uint4*>(out + (size_t)(2 * m + 1) * kImg + sw_off(c, j)) = l4;
+    }
+}
+
+// ---------------------------------------------------------------- p2
+struct P2TcSmem {
+    uint8_t ring[S2][3 * BOX];               // dZ, K, V
+    uint8_t img[kImgs][kImg];                // the unit's operand images
+    uint8_t stage[3][BOX];                   // dQ, dK, dV of a tile as bf16, for the TMA stores
+    uint64_t full[S2], empty[S2];
+    uint64_t img_full, img_empty;
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t drain_bar;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ bool p2_load_imgs(P2TcSmem& s, const TcParams& p, int u, uint32_t& parts, const Abort& ab) {
+    if (parts == 0) pdl_wait_primary();      // the merge kernel has written the images
+    if (!mbar_wait(&s.img_empty, (parts & 1u) ^ 1u, ab)) return false;
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(&s.img_full, kImgs * kImg);
+    bulk_g2s(s.img, p.imgs + (size_t)u * kImgs * kImg, kImgs * kImg, &s.img_full);
+    ++parts;
+    return true;
+}
+
+__device__ __forceinline__ void p2_producer(P2TcSmem& s, const TcParams& p, const CUtensorMap* tmZ, const CUtensorMap* tmK,
+                                            const CUtensorMap* tmV, const Abort& ab) {
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    int st = 0; uint32_t ph = 0, issued = 0, parts = 0;
+    int pending = -1;                        // unit whose images are not requested yet
+    bool ok = true;
+    for (long long t = t0; t < t1 && ok; ++t) {
+        const int u = (int)(t / p.tpu), n0 = (int)(t % p.tpu) * TOK, h = u % p.heads, b = u / p.heads;
+        if (t == t0) {
+            pending = u;                     // the first tiles (inputs) load while the merge runs
+        } else if (t % p.tpu == 0) {         // a new unit: its images, after the first unit's
+            if (pending >= 0 && !(ok = p2_load_imgs(s, p, pending, parts, ab))) break;
+            pending = -1;
+            if (!(ok = p2_load_imgs(s, p, u, parts, ab))) break;
+        }
+        if (pending >= 0 && issued == (uint32_t)S2) {
+            if (!(ok = p2_load_imgs(s, p, pending, parts, ab))) break;
+            pending = -1;
+        }
+        if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
+        mbar_arrive_expect_tx(&s.full[st], 3 * BOX);
+        uint8_t* dst = s.ring[st];
+        tma_load_4d(dst + 0 * BOX, tmZ, &s.full[st], 0, n0, h, b);
+        tma_load_4d(dst + 1 * BOX, tmK, &s.full[st], 0, n0, h, b);
+        tma_load_4d(dst + 2 * BOX, tmV, &s.full[st], 0, n0, h, b);
+        ++issued;
+        if (++st == S2) { st = 0; ph ^= 1u; }
+    }
+    if (ok && pending >= 0) p2_load_imgs(s, p, pending, parts, ab);
+    for (uint32_t k = issued > (uint32_t)S2 ? issued - S2 : 0u; k < issued; ++k)
+        mbar_drain(&s.full[k % S2], (k / S2) & 1u, ab.limit);
+    if (parts > 0) mbar_drain(&s.img_full, (parts - 1) & 1u, ab.limit);
+}
+
+__device__ __forceinline__ void p2_mma(P2TcSmem& s, const TcParams& p, uint32_t tmem, const Abort& ab) {
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    int st = 0; uint32_t ph = 0, parts = 0, n = 0;
+    const uint32_t img = smem_u32(s.img);
+    for (long long t = t0; t < t1; ++t, ++n) {
+        if (t == t0 || t % p.tpu == 0) {
+            if (!mbar_wait(&s.img_full, parts & 1u, ab)) return;
+            ++parts;
+        }
+        const uint32_t ab2 = n & 1u;
+        if (!mbar_wait(&s.acc_empty[ab2], ((n >> 1) & 1u) ^ 1u, ab)) return;
+        if (!mbar_wait(&s.full[st], ph, ab)) return;
+        tc_fence_after();
+        const uint32_t z = smem_u32(s.ring[st]), k = z + BOX, v = z + 2 * BOX;
+        const uint32_t dq = tmem + ab2 * 192u, dv = dq + 64u, dk = dq + 128u;
+        // (A box, image pair, accumulator): dQ = dZ W1, dV = K dC^T, dK = V dC + K (dG + dG^T)
+        const uint32_t a_of[4] = {z, k, v, k};
+        const uint32_t d_of[4] = {dq, dv, dk, dk};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+#pragma unroll
+            for (int hl = 0; hl < 2; ++hl) {
+                const uint32_t bimg = img + (uint32_t)((2 * m + hl) * kImg);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(d_of[m], sdesc_sw128(a_of[m] + kk * 32, 16, 1024), sdesc_sw128(bimg + kk * 32, 16, 1024),
+                                kIdescMap, (m == 3 || hl || kk) ? 1u : 0u);
+            }
+        }
+        mma_commit(&s.empty[st]);
+        mma_commit(&s.acc_full[ab2]);
+        if (t + 1 == t1 || (t + 1) % p.tpu == 0) mma_commit(&s.img_empty);
+        if (++st == S2) { st = 0; ph ^= 1u; }
+    }
+}
+
+// Drain warps: TMEM lane r is token row r of the tile; each output goes to its staging box as bf16
+// (128-byte swizzled rows, the TMA store's layout), then one TMA store per output.
+__device__ __forceinline__ void p2_drain(P2TcSmem& s, const TcParams& p, uint32_t tmem, const CUtensorMap* tmdQ,
+                                         const CUtensorMap* tmdK, const CUtensorMap* tmdV, const Abort& ab) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3, r = q * 32 + lane;
+    const int tid = threadIdx.x - 64;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    uint32_t n = 0;
+    for (long long t = t0; t < t1; ++t, ++n) {
+        const int u = (int)(t / p.tpu), n0 = (int)(t % p.tpu) * TOK, h = u % p.heads, b = u / p.heads;
+        const uint32_t ab2 = n & 1u;
+        const bool ok = mbar_wait(&s.acc_full[ab2], (n >> 1) & 1u, ab);
+        if (tid == 0 && n > 0) bulk_wait_read<0>();          // the previous tile's stores have read the staging boxes
+        if (named_bar_or(1, 128, !ok)) break;
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll 1
+        for (int o = 0; o < 3; ++o) {                         // dQ, dV, dK: accumulator columns 64 o
+            float v[4][16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(tmem + ab2 * 192u + (uint32_t)(64 * o + 16 * j) + lane_off, v[j]);
+            tmem_ld_wait();
+            uint8_t* dst = s.stage[o];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float* x = &v[j / 2][(j % 2) * 8];
+                uint4 pk;
+                pk.x = pack_bf16x2(x[0], x[1]); pk.y = pack_bf16x2(x[2], x[3]);
+                pk.z = pack_bf16x2(x[4], x[5]); pk.w = pack_bf16x2(x[6], x[7]);
+                *reinterpret_cast<uint4*>(dst + sw_off(r, j)) = pk;
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&s.acc_empty[ab2]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0) {
+            tma_store_4d(tmdQ, s.stage[0], 0, n0, h, b);
+            tma_store_4d(tmdV, s.stage[1], 0, n0, h, b);
+            tma_store_4d(tmdK, s.stage[2], 0, n0, h, b);
+            bulk_commit();
+        }
+    }
+    if (tid == 0) bulk_wait<0>();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+lin_bwd_p2_tc(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdQ,
+              const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    P2TcSmem& s = *reinterpret_cast<P2TcSmem*>(align1024(smem_raw));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
+    if (threadIdx.x == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < S2; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        mbar_init(&s.img_full, 1); mbar_init(&s.img_empty, 1);
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
+        mbar_init(&s.drain_bar, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmZ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdQ); prefetch_tmap(&tmdK); prefetch_tmap(&tmdV);
+    }
+    if (warp == 1) { tmem_alloc(&s.tmem_base, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    if (warp == 0) {
+        if (lane == 0) p2_producer(s, p, &tmZ, &tmK, &tmV, ab);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            p2_mma(s, p, tmem, ab);
+            mma_commit(&s.drain_bar);
+            mbar_drain(&s.drain_bar, 0u, ab.limit);
+        }
+        __syncwarp();
+    } else {
+        p2_drain(s, p, tmem, &tmdQ, &tmdK, &tmdV, ab);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
 struct WsLayout {
-    size_t counters, partials, mats, dw0, deta, total;
+    size_t counters, partials, mats, dw0, deta, imgs, total;
 };
 
 static WsLayout ws_layout(long long units) {
@@ -339,8 +751,58 @@ static WsLayout ws_layout(long long units) {
     L.mats = align_up(L.partials + (size_t)(kMaxGrid + units) * kPartial * sizeof(float), 1024);
     L.dw0 = align_up(L.mats + (size_t)units * kMats * D * D * sizeof(float), 1024);
     L.deta = align_up(L.dw0 + (size_t)units * D * D * sizeof(float), 256);
-    L.total = align_up(L.deta + (size_t)units * sizeof(float), 256);
+    L.imgs = align_up(L.deta + (size_t)units * sizeof(float), 1024);
+    L.total = L.imgs + (size_t)units * tc::kImgs * tc::kImg;
     return L;
+}
+
+// bf16: the tensor-core kernels, one CTA per SM for the two streaming phases.
+static ttt_status launch_tc(const Call& c, Params p, const WsLayout& L) {
+    using namespace tc;
+    CUtensorMap tmK, tmV, tmZ, tmQ, tmdQ, tmdK, tmdV;
+    if (!make_tmap_tokens(&tmK, c.K, c, TOK) || !make_tmap_tokens(&tmV, c.V, c, TOK) ||
+        !make_tmap_tokens(&tmZ, p.dZ, c, TOK) || !make_tmap_tokens(&tmQ, c.Q, c, TOK) ||
+        !make_tmap_tokens(&tmdQ, p.dQ, c, TOK) || !make_tmap_tokens(&tmdK, p.dK, c, TOK) ||
+        !make_tmap_tokens(&tmdV, p.dV, c, TOK))
+        return TTT_ERR_INVALID_ARG;
+    const long long T = p.part.T;
+    const int G = (int)std::max<long long>(1, std::min<long long>(std::min(c.num_sms, kMaxGrid), T));
+    p.part = Partition{T, G};
+    TcParams tp{};
+    tp.tpu = p.tpu;
+    tp.heads = c.heads;
+    tp.part = p.part;
+    tp.partials = p.partials;
+    tp.imgs = c.ws + L.imgs;
+    tp.err = reinterpret_cast<uint32_t*>(c.ws);
+    tp.wait_ns = c.wait_ns;
+    const size_t sm1 = sizeof(P1TcSmem) + 1024, smm = sizeof(P1Smem) + 128, sm2 = sizeof(P2TcSmem) + 1024;
+    if (sm1 > 227 * 1024 || sm2 > 227 * 1024) return TTT_ERR_UNSUPPORTED;
+    cudaFuncSetAttribute(lin_bwd_p1_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+    cudaFuncSetAttribute(lin_bwd_merge_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smm);
+    cudaFuncSetAttribute(lin_bwd_p2_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    lin_bwd_p1_tc<<<G, kThreads, sm1, c.stream>>>(tmK, tmV, tmZ, tmQ, tp);
+    ttt_status st = check_launch(cudaGetLastError());
+    if (st != TTT_OK) return st;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)p.units);
+    cfg.blockDim = dim3(P1_THREADS);
+    cfg.dynamicSmemBytes = smm;
+    cfg.stream = c.stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_merge_tc, p, c.ws + L.imgs));
+    if (st != TTT_OK) return st;
+    cfg.gridDim = dim3((unsigned)G);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sm2;
+    st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2_tc, tmZ, tmK, tmV, tmdQ, tmdK, tmdV, tp));
+    if (st != TTT_OK || (!p.dW0_out && !p.deta_out)) return st;
+    lin_bwd_sum<<<c.heads, 256, 0, c.stream>>>(p, c.batch);
+    return check_launch(cudaGetLastError());
 }
 
 template <typename E>
@@ -369,28 +831,31 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
     p.deta_unit = reinterpret_cast<float*>(c.ws + L.deta);
     p.dW0_out = dW0_out;
     p.deta_out = deta_out;
-
-    const size_t sm1 = sizeof(P1Smem) + 128, sm2 = sizeof(P2Smem) + 128;
-    cudaFuncSetAttribute(lin_bwd_p1<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-    cudaFuncSetAttribute(lin_bwd_p2<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    lin_bwd_p1<E><<<G, P1_THREADS, sm1, c.stream>>>(p);
-    ttt_status st = check_launch(cudaGetLastError());
-    if (st != TTT_OK) return st;
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    const int tiles2 = (c.N + P2_TOK - 1) / P2_TOK;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)(units * tiles2));
-    cfg.blockDim = dim3(P2_THREADS);
-    cfg.dynamicSmemBytes = sm2;
-    cfg.stream = c.stream;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2<E>, p, tiles2));
-    if (st != TTT_OK || (!dW0_out && !deta_out)) return st;
-    lin_bwd_sum<<<c.heads, 256, 0, c.stream>>>(p, c.batch);
-    return check_launch(cudaGetLastError());
+    if constexpr (std::is_same<E, __nv_bfloat16>::value) {
+        return launch_tc(c, p, L);
+    } else {
+        const size_t sm1 = sizeof(P1Smem) + 128, sm2 = sizeof(P2Smem) + 128;
+        cudaFuncSetAttribute(lin_bwd_p1<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+        cudaFuncSetAttribute(lin_bwd_p2<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+        lin_bwd_p1<E><<<G, P1_THREADS, sm1, c.stream>>>(p);
+        ttt_status st = check_launch(cudaGetLastError());
+        if (st != TTT_OK) return st;
+        cudaLaunchAttribute pdl[1];
+        pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pdl[0].val.programmaticStreamSerializationAllowed = 1;
+        const int tiles2 = (c.N + P2_TOK - 1) / P2_TOK;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(units * tiles2));
+        cfg.blockDim = dim3(P2_THREADS);
+        cfg.dynamicSmemBytes = sm2;
+        cfg.stream = c.stream;
+        cfg.attrs = pdl;
+        cfg.numAttrs = 1;
+        st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2<E>, p, tiles2));
+        if (st != TTT_OK || (!dW0_out && !deta_out)) return st;
+        lin_bwd_sum<<<c.heads, 256, 0, c.stream>>>(p, c.batch);
+        return check_launch(cudaGetLastError());
+    }
 }
 
 }  // namespace bwd

@@ -149,100 +149,141 @@ struct GradSmem {
     int abort_flag;
 };
 
+// The CTA's tiles n = 0 .. N-1 go through the tensor pipe in the order R(0), R(1), G(0), R(2), G(1),
+// ..., R(N-1), G(N-2), G(N-1): while the epilogue turns R(n) into the residual operand of G(n), the
+// MMAs of R(n+1) run.  The producer loads in the same order: V(n) and the nine K boxes of R(n), then
+// the nine K boxes of G(n-1) again.
+__host__ __device__ __forceinline__ bool first_of_part(const Geo& g, long long t0, long long t) {
+    return t == t0 || t % g.tpu == 0;
+}
+__host__ __device__ __forceinline__ bool last_of_part(const Geo& g, long long t1, long long t) {
+    return t + 1 == t1 || (t + 1) % g.tpu == 0;
+}
+
+struct Ring {
+    int st = 0;
+    uint32_t ph = 0, issued = 0;
+    __device__ __forceinline__ void advance() {
+        ++issued;
+        if (++st == S1) { st = 0; ph ^= 1u; }
+    }
+};
+
+// The nine K boxes of tile t at their tap shifts, two taps per ring stage.
+__device__ __forceinline__ bool load_taps(GradSmem& s, const CUtensorMap* tmK, const TileXY& x, Ring& rg,
+                                          const Abort& ab) {
+    for (int k = 0; k < NPAIR; ++k) {
+        if (!mbar_wait(&s.empty[rg.st], rg.ph ^ 1u, ab)) return false;
+        const int nt = taps_in_pair(k);
+        mbar_arrive_expect_tx(&s.full[rg.st], (uint32_t)(nt * BOX));
+        for (int j = 0; j < nt; ++j) {
+            const int t9 = 2 * k + j, a = t9 / 3, bb = t9 % 3;
+            tma_load_5d(s.ring[rg.st] + j * BOX, tmK, &s.full[rg.st], 0, x.x0 + bb - 1, x.y0 + a - 1, x.h, x.b);
+        }
+        rg.advance();
+    }
+    return true;
+}
+
 __device__ __forceinline__ void grad_producer(GradSmem& s, const GradParams& p, const CUtensorMap* tmK,
                                               const CUtensorMap* tmV, const Abort& ab) {
     const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    uint32_t issued = 0, vq = 0, parts = 0;
-    int st = 0; uint32_t ph = 0;
+    uint32_t vq = 0, parts = 0;
+    Ring rg;
     bool ok = true;
-    for (long long t = t0; t < t1 && ok; ++t) {
-        const TileXY x = tile_xy(p.g, t);
-        if (t == t0 || x.u != (int)((t - 1) / p.g.tpu)) {
-            // a part starts: the head's W0 tap images, once the previous part's R MMAs are done with them
-            if (t == t0) pdl_wait_primary();                 // conv3_wprep has written the images
-            if (!(ok = mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab))) break;
-            fence_proxy_async_global();
-            mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
-            bulk_g2s(s.w0img, p.w0img + (size_t)x.h * TAPS * kWImg, TAPS * kWImg, &s.w_full);
-            ++parts;
-        }
-        if (!(ok = mbar_wait(&s.vempty, (vq & 1u) ^ 1u, ab))) break;
-        mbar_arrive_expect_tx(&s.vfull, BOX);
-        tma_load_5d(s.vbuf, tmV, &s.vfull, 0, x.x0, x.y0, x.h, x.b);
-        ++vq;
-        for (int pass = 0; pass < 2 && ok; ++pass)          // taps for R, then again for the gradient
-            for (int k = 0; k < NPAIR; ++k) {
-                if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
-                const int nt = taps_in_pair(k);
-                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(nt * BOX));
-                for (int j = 0; j < nt; ++j) {
-                    const int t9 = 2 * k + j, a = t9 / 3, bb = t9 % 3;
-                    tma_load_5d(s.ring[st] + j * BOX, tmK, &s.full[st], 0, x.x0 + bb - 1, x.y0 + a - 1, x.h, x.b);
-                }
-                ++issued;
-                if (++st == S1) { st = 0; ph ^= 1u; }
+    for (long long t = t0; t <= t1 && ok; ++t) {
+        if (t < t1) {
+            const TileXY x = tile_xy(p.g, t);
+            if (first_of_part(p.g, t0, t)) {
+                // the head's W0 tap images, once the previous part's R MMAs are done with them
+                if (t == t0) pdl_wait_primary();             // conv3_wprep has written the images
+                if (!(ok = mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab))) break;
+                fence_proxy_async_global();
+                mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
+                bulk_g2s(s.w0img, p.w0img + (size_t)x.h * TAPS * kWImg, TAPS * kWImg, &s.w_full);
+                ++parts;
             }
+            if (!(ok = mbar_wait(&s.vempty, (vq & 1u) ^ 1u, ab))) break;
+            mbar_arrive_expect_tx(&s.vfull, BOX);
+            tma_load_5d(s.vbuf, tmV, &s.vfull, 0, x.x0, x.y0, x.h, x.b);
+            ++vq;
+            if (!(ok = load_taps(s, tmK, x, rg, ab))) break;
+        }
+        if (t > t0) ok = load_taps(s, tmK, tile_xy(p.g, t - 1), rg, ab);
     }
     // every copy issued has landed before the CTA may exit
-    for (uint32_t k = issued > (uint32_t)S1 ? issued - S1 : 0u; k < issued; ++k)
+    for (uint32_t k = rg.issued > (uint32_t)S1 ? rg.issued - S1 : 0u; k < rg.issued; ++k)
         mbar_drain(&s.full[k % S1], (k / S1) & 1u, ab.limit);
     if (vq > 0) mbar_drain(&s.vfull, (vq - 1) & 1u, ab.limit);
     if (parts > 0) mbar_drain(&s.w_full, (parts - 1) & 1u, ab.limit);
 }
 
+// R(t) = sum_t9 K_t9 W0_t9^T into R accumulator n & 1 (A: K box, K-major; B: W0 tap image).
+__device__ __forceinline__ bool mma_R(GradSmem& s, const GradParams& p, uint32_t tmem, long long t0, long long t1,
+                                      long long t, uint32_t n, uint32_t& wparts, Ring& rg, const Abort& ab) {
+    if (first_of_part(p.g, t0, t)) {
+        if (!mbar_wait(&s.w_full, wparts & 1u, ab)) return false;
+        ++wparts;
+    }
+    const uint32_t dr = n & 1u;
+    if (!mbar_wait(&s.dr_empty[dr], ((n >> 1) & 1u) ^ 1u, ab)) return false;
+    tc_fence_after();
+    for (int k = 0; k < NPAIR; ++k) {
+        if (!mbar_wait(&s.full[rg.st], rg.ph, ab)) return false;
+        tc_fence_after();
+        for (int j = 0; j < taps_in_pair(k); ++j) {
+            const uint32_t sa = smem_u32(s.ring[rg.st] + j * BOX), sb = smem_u32(s.w0img[2 * k + j]);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16_ss(tmem + kColR + dr * 64u, sdesc_sw128(sa + kk * 32, 16, 1024),
+                            sdesc_sw128(sb + kk * 32, 16, 1024), kIdescRow, (k | j | kk) ? 1u : 0u);
+        }
+        mma_commit(&s.empty[rg.st]);
+        rg.advance();
+    }
+    mma_commit(&s.dr_full[dr]);
+    if (last_of_part(p.g, t1, t)) mma_commit(&s.w_empty);    // the part's last reads of the W0 images
+    return true;
+}
+
+// G^T[pair k] += [K_2k | K_2k+1]^T (r_hi + r_lo) for tile t (A MN-major, M = 128; B = r, MN-major).
+__device__ __forceinline__ bool mma_G(GradSmem& s, const GradParams& p, uint32_t tmem, long long t0, long long t1,
+                                      long long t, uint32_t n, uint32_t& gparts, Ring& rg, const Abort& ab) {
+    if (!mbar_wait(&s.r_full, n & 1u, ab)) return false;
+    const bool first = first_of_part(p.g, t0, t);
+    if (first && !mbar_wait(&s.g_empty, (gparts & 1u) ^ 1u, ab)) return false;
+    tc_fence_after();
+    const uint32_t shi = smem_u32(s.rhi), slo = smem_u32(s.rlo);
+    for (int k = 0; k < NPAIR; ++k) {
+        if (!mbar_wait(&s.full[rg.st], rg.ph, ab)) return false;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(s.ring[rg.st]);
+        const uint32_t dg = tmem + kColG + (uint32_t)k * 64u;
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sa + kk * 2048, BOX, 1024);
+            mma_bf16_ss(dg, ad, sdesc_sw128(shi + kk * 2048, BOX, 1024), kIdescCol, (first && kk == 0) ? 0u : 1u);
+            mma_bf16_ss(dg, ad, sdesc_sw128(slo + kk * 2048, BOX, 1024), kIdescCol, 1u);
+        }
+        mma_commit(&s.empty[rg.st]);
+        rg.advance();
+    }
+    mma_commit(&s.r_empty);
+    if (last_of_part(p.g, t1, t)) {
+        mma_commit(&s.g_full);
+        ++gparts;
+    }
+    return true;
+}
+
 __device__ __forceinline__ void grad_mma(GradSmem& s, const GradParams& p, uint32_t tmem, const Abort& ab) {
     const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    int st = 0; uint32_t ph = 0;
-    uint32_t n = 0, part = 0;                                // tiles and parts so far
-    for (long long t = t0; t < t1;) {
-        const int u = (int)(t / p.g.tpu);
-        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
-        if (!mbar_wait(&s.w_full, part & 1u, ab)) return;
-        for (long long tt = t; tt < pe; ++tt, ++n) {
-            // R = sum_t K_t W0_t^T (A: K box, K-major; B: W0 tap image)
-            const uint32_t dr = n & 1u;
-            if (!mbar_wait(&s.dr_empty[dr], ((n >> 1) & 1u) ^ 1u, ab)) return;
-            tc_fence_after();
-            for (int k = 0; k < NPAIR; ++k) {
-                if (!mbar_wait(&s.full[st], ph, ab)) return;
-                tc_fence_after();
-                for (int j = 0; j < taps_in_pair(k); ++j) {
-                    const uint32_t sa = smem_u32(s.ring[st] + j * BOX), sb = smem_u32(s.w0img[2 * k + j]);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_bf16_ss(tmem + kColR + dr * 64u, sdesc_sw128(sa + kk * 32, 16, 1024),
-                                    sdesc_sw128(sb + kk * 32, 16, 1024), kIdescRow, (k | j | kk) ? 1u : 0u);
-                }
-                mma_commit(&s.empty[st]);
-                if (++st == S1) { st = 0; ph ^= 1u; }
-            }
-            mma_commit(&s.dr_full[dr]);
-            if (tt + 1 == pe) mma_commit(&s.w_empty);        // the part's last reads of the W0 images
-            // G^T[pair k] += [K_2k | K_2k+1]^T (r_hi + r_lo)  (A MN-major, M = 128; B = r, MN-major)
-            if (!mbar_wait(&s.r_full, n & 1u, ab)) return;
-            const bool first = (tt == t);
-            if (first && !mbar_wait(&s.g_empty, (part & 1u) ^ 1u, ab)) return;
-            tc_fence_after();
-            const uint32_t shi = smem_u32(s.rhi), slo = smem_u32(s.rlo);
-            for (int k = 0; k < NPAIR; ++k) {
-                if (!mbar_wait(&s.full[st], ph, ab)) return;
-                tc_fence_after();
-                const uint32_t sa = smem_u32(s.ring[st]);
-                const uint32_t dg = tmem + kColG + (uint32_t)k * 64u;
-#pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(sa + kk * 2048, BOX, 1024);
-                    mma_bf16_ss(dg, ad, sdesc_sw128(shi + kk * 2048, BOX, 1024), kIdescCol, (first && kk == 0) ? 0u : 1u);
-                    mma_bf16_ss(dg, ad, sdesc_sw128(slo + kk * 2048, BOX, 1024), kIdescCol, 1u);
-                }
-                mma_commit(&s.empty[st]);
-                if (++st == S1) { st = 0; ph ^= 1u; }
-            }
-            mma_commit(&s.r_empty);
-        }
-        mma_commit(&s.g_full);
-        ++part;
-        t = pe;
+    Ring rg;
+    uint32_t wparts = 0, gparts = 0;
+    for (long long t = t0; t <= t1; ++t) {
+        const uint32_t n = (uint32_t)(t - t0);
+        if (t < t1 && !mma_R(s, p, tmem, t0, t1, t, n, wparts, rg, ab)) return;
+        if (t > t0 && !mma_G(s, p, tmem, t0, t1, t - 1, n - 1, gparts, rg, ab)) return;
     }
 }
 
@@ -445,25 +486,39 @@ struct ReadSmem {
     int abort_flag;
 };
 
+// W1 of unit u (written by the merge kernel): one bulk copy of its nine tap images, once the
+// previous part's MMAs are done with the images.
+__device__ __forceinline__ bool load_w1(ReadSmem& s, const ReadParams& p, int u, uint32_t& parts, const Abort& ab) {
+    if (parts == 0) pdl_wait_primary();
+    if (!mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab)) return false;
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
+    bulk_g2s(s.w1img, p.w1img + (size_t)u * TAPS * kWImg, TAPS * kWImg, &s.w_full);
+    ++parts;
+    return true;
+}
+
 __device__ __forceinline__ void read_producer(ReadSmem& s, const ReadParams& p, const CUtensorMap* tmQ,
                                               const Abort& ab) {
     const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
     uint32_t issued = 0, parts = 0;
     int st = 0; uint32_t ph = 0;
-    bool ok = true, waited = false;
+    bool ok = true;
+    int pending = -1;                                        // unit whose W1 images are not requested yet
     for (long long t = t0; t < t1 && ok;) {
         const int u = (int)(t / p.g.tpu);
         const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
-        // W1 of the unit (written by the merge kernel): one bulk copy of its nine tap images
-        if (!waited) { pdl_wait_primary(); waited = true; }
-        if (!(ok = mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab))) break;
-        fence_proxy_async_global();
-        mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
-        bulk_g2s(s.w1img, p.w1img + (size_t)u * TAPS * kWImg, TAPS * kWImg, &s.w_full);
-        ++parts;
+        // the first part's images are requested once the ring's stages are in flight: the Q boxes (an
+        // input) load while the merge kernel is still writing W1
+        if (t == t0) pending = u;
+        else if (!(ok = load_w1(s, p, u, parts, ab))) break;
         for (long long tt = t; tt < pe && ok; ++tt) {
             const TileXY x = tile_xy(p.g, tt);
             for (int k = 0; k < NPAIR; ++k) {
+                if (pending >= 0 && issued == (uint32_t)S3) {
+                    if (!(ok = load_w1(s, p, pending, parts, ab))) break;
+                    pending = -1;
+                }
                 if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
                 const int nt = taps_in_pair(k);
                 mbar_arrive_expect_tx(&s.full[st], (uint32_t)(nt * BOX));
@@ -477,6 +532,7 @@ __device__ __forceinline__ void read_producer(ReadSmem& s, const ReadParams& p, 
         }
         t = pe;
     }
+    if (ok && pending >= 0) load_w1(s, p, pending, parts, ab);
     for (uint32_t k = issued > (uint32_t)S3 ? issued - S3 : 0u; k < issued; ++k)
         mbar_drain(&s.full[k % S3], (k / S3) & 1u, ab.limit);
     if (parts > 0) mbar_drain(&s.w_full, (parts - 1) & 1u, ab.limit);
