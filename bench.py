@@ -55,7 +55,7 @@ TRAFFIC = {
     "mlp1024_bf16": {"read": 25533440, "write": 6981376, "src_sha": "e351f2e6a0775778"},
     "conv3x3_6084_bf16": {"read": 18741504, "write": 7558144, "src_sha": "2385ceaf5d3c5c3d"},
     "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
-    "bwd6084_bf16": {"read": 208251136, "write": 113136640, "src_sha": "6ed6afd58a0eb27a"},
+    "bwd6084_bf16": {"read": 218148352, "write": 105013504, "src_sha": "c97c5f030b248cf5"},
     "bwdconv6084_bf16": {"read": 24883456, "write": 17042944, "src_sha": "1dfe7c0812e5935d"},
     "bwdmlp1024_bf16": {"read": 67329024, "write": 145303808, "src_sha": "a33fe42962dd5335"},
 }

@@ -87,7 +87,8 @@ struct Params {
     float* partials;                         // [(G + units)][192][64], slot = cta + unit
     float* mats;                             // [units][4][64][64]: W1, dC, dC^T, dG + dG^T
     float* dW0_unit;                         // [units][64][64]
-    float* deta_unit;                        // [units]
+    float* deta_unit;                        // [deta_terms]: per unit (fp32), per merge CTA (bf16)
+    int deta_terms;
     float* dW0_out;                          // nullable [heads][64][64]
     float* deta_out;                         // nullable, one float
 };
@@ -310,20 +311,39 @@ lin_bwd_p2(const Params p, int tiles_per_unit) {
 // ------------------------------------------------------------------------------------------------
 // dW0 over images, deta over units (index order)
 // ------------------------------------------------------------------------------------------------
+// Four CTAs per head, one float4 of dW0 per thread, the images' terms eight at a time in flight.
 __global__ void __launch_bounds__(256)
 lin_bwd_sum(const Params p, int batch) {
-    const int h = blockIdx.x, heads = p.view.heads;
+    const int h = blockIdx.x >> 2, heads = p.view.heads;
+    const int e4 = (blockIdx.x & 3) * 256 + (int)threadIdx.x;        // float4 of the head's 64 x 64
+    pdl_wait_primary();                      // launched as a programmatic dependent of phase 2
     if (p.dW0_out) {
-        for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
-            float a = 0.f;
-            for (int b = 0; b < batch; ++b) a += p.dW0_unit[((size_t)b * heads + h) * D * D + e];
-            p.dW0_out[(size_t)h * D * D + e] = a;
+        const float4* src = reinterpret_cast<const float4*>(p.dW0_unit) + (size_t)h * (D * D / 4) + e4;
+        const size_t stride = (size_t)heads * (D * D / 4);
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int b0 = 0; b0 < batch; b0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = b0 + q < batch ? __ldcg(src + (size_t)(b0 + q) * stride) : a;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (b0 + q < batch) { a.x += v[q].x; a.y += v[q].y; a.z += v[q].z; a.w += v[q].w; }
         }
+        reinterpret_cast<float4*>(p.dW0_out + (size_t)h * D * D)[e4] = a;
     }
-    if (p.deta_out && h == 0 && threadIdx.x == 0) {
-        float a = 0.f;
-        for (int u = 0; u < p.units; ++u) a += p.deta_unit[u];
-        *p.deta_out = a;
+    if (p.deta_out && blockIdx.x == 0) {
+        // the terms of deta loaded by the whole block (one round trip per 1024), summed in index order
+        __shared__ float terms[1024];
+        float acc = 0.f;
+        for (int t0 = 0; t0 < p.deta_terms; t0 += 1024) {
+            const int n = min(1024, p.deta_terms - t0);
+            __syncthreads();
+            for (int k = threadIdx.x; k < n; k += blockDim.x) terms[k] = __ldcg(p.deta_unit + t0 + k);
+            __syncthreads();
+            if (threadIdx.x == 0)
+                for (int k = 0; k < n; ++k) acc += terms[k];
+        }
+        if (threadIdx.x == 0) *p.deta_out = acc;
     }
 }
 
@@ -514,38 +534,178 @@ lin_bwd_p1_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 }
 
 // ---------------------------------------------------------------- merge
-// The unit's matrices (merge_unit), then the operand images of phase 2, image x holding X[c][i]:
+// SPLIT CTAs per unit (1, 2 or 4: as many as keep one CTA per SM), each 64 / SPLIT rows i of the
+// unit's matrices; a thread takes 4 / SPLIT of those rows and four columns j0 .. j0+3 of the products
+// P = W0 G - C, M = W0^T dW1 (row i and column i) and dW1 G:
+//   W1 = W0 - s P,  dC = s dW1,  dG + dG^T = -s (M + M^T),  dW0 = dW1 - s dW1 G,
+//   deta = -(2/N) sum dW1 * P  (per CTA: warp sums, then the warps in order; the CTAs' partials are
+//   summed in index order by lin_bwd_sum).
+constexpr int kMergeThreads = 256;
+constexpr int kMaxSplit = 4;
+// Dynamic shared memory of a merge CTA: more than half an SM's, so that the block scheduler places
+// one merge CTA per SM (packed four to an SM they ran four times slower).
+constexpr size_t kMergeSmem = 120 * 1024;
+struct MergeTcSmem {
+    float g[D][MP];                              // G, summed over the unit's slots
+    float dw1[D][MP];                            // dW1
+    float c[D][MP];                              // the CTA's rows of C
+    float w0[D][MP];
+    __nv_bfloat16 tr[4][D][D];                   // W1^T and dC^T (hi, lo): rows c, the CTA's K = i
+    float red[kMergeThreads / 32];
+};
+static_assert(sizeof(MergeTcSmem) + 128 <= kMergeSmem, "merge shared memory");
+
+// Elements K = k0 .. k0+3 of row `row` of an operand image pair (8-byte stores, k0 a multiple of 4).
+__device__ __forceinline__ void put_hi_lo4(uint8_t* hi, int row, int k0, const float (&v)[4]) {
+    float h[4], l[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        h[k] = __bfloat162float(__float2bfloat16_rn(v[k]));
+        l[k] = v[k] - h[k];
+    }
+    const uint32_t off = sw_off(row, k0 / 8) + (uint32_t)(k0 % 8) * 2;
+    *reinterpret_cast<uint2*>(hi + off) = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+    *reinterpret_cast<uint2*>(hi + kImg + off) = make_uint2(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]));
+}
+
+// Row r (0 .. 143) of what a merge CTA sums: G rows 0..63, its 16 rows of C, then dW1 rows 0..63;
+// returns the slot row and the shared-memory row.
+template <int ROWS>
+__device__ __forceinline__ void merge_row(MergeTcSmem& s, int r, int i0, int& slot_row, float*& dst) {
+    if (r < D) { slot_row = r; dst = s.g[r]; }
+    else if (r < D + ROWS) { slot_row = D + i0 + (r - D); dst = s.c[r - D]; }
+    else { slot_row = 2 * D + (r - D - ROWS); dst = s.dw1[r - D - ROWS]; }
+}
+
+// The unit's matrices, then the operand images of phase 2, image x holding X[c][i]:
 //   0/1 W1^T (dQ = dZ W1),  2/3 dC (dV = K dC^T),  4/5 dC^T (dK = V dC + ..),  6/7 dG + dG^T (symmetric),
 // each rounded to bf16 (hi) with the rounding error rounded again (lo).
-__global__ void __launch_bounds__(P1_THREADS)
+template <int SPLIT>
+__global__ void __launch_bounds__(kMergeThreads, 1)
 lin_bwd_merge_tc(const Params p, uint8_t* imgs) {
+    constexpr int ROWS = D / SPLIT, RPT = ROWS / 16;     // rows per CTA, rows per thread
     extern __shared__ uint8_t smem_raw[];
-    P1Smem& s = *reinterpret_cast<P1Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    const int u = blockIdx.x;
+    MergeTcSmem& s = *reinterpret_cast<MergeTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int u = blockIdx.x / SPLIT, i0 = (blockIdx.x % SPLIT) * ROWS;
+    const int tid = threadIdx.x, h = u % p.view.heads;
     pdl_wait_primary();                      // every partial slot is written
     pdl_launch_dependents();
     const int cf = p.part.cta_of((long long)u * p.tpu), cl = p.part.cta_of((long long)(u + 1) * p.tpu - 1);
-    merge_unit<__nv_bfloat16>(p, s, u, cf + u, cl - cf + 1);
-    __syncthreads();                         // the unit's matrices are in global memory
-    const float* M = p.mats + (size_t)u * kMats * D * D;
-    uint8_t* out = imgs + (size_t)u * kImgs * kImg;
-    for (int e = threadIdx.x; e < 4 * D * (D / 8); e += P1_THREADS) {
-        const int m = e / (D * (D / 8)), c = (e / (D / 8)) % D, j = e % (D / 8);
-        float hi[8], lo[8];
+    const int nslots = cl - cf + 1;
+    // the slot sums in slot order: three float4 per thread at a time, eight slots of each in flight
+    constexpr int F4 = (2 * D + ROWS) * (D / 4);
+    const float4* src = reinterpret_cast<const float4*>(p.partials + (size_t)(cf + u) * kPartial);
+    for (int f0 = tid; f0 < F4; f0 += 3 * kMergeThreads) {
+        float4 acc[3];
+        size_t off[3];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int i = 8 * j + k;
-            const float x = (m == 0) ? M[(size_t)i * D + c] : M[(size_t)m * D * D + (size_t)c * D + i];
-            hi[k] = __bfloat162float(__float2bfloat16_rn(x));
-            lo[k] = x - hi[k];
+        for (int g = 0; g < 3; ++g) {
+            acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int f = min(f0 + g * kMergeThreads, F4 - 1);
+            int sr; float* d;
+            merge_row<ROWS>(s, f / (D / 4), i0, sr, d);
+            off[g] = (size_t)sr * (D / 4) + f % (D / 4);
         }
-        uint4 h4, l4;
-        h4.x = pack_bf16x2(hi[0], hi[1]); h4.y = pack_bf16x2(hi[2], hi[3]);
-        h4.z = pack_bf16x2(hi[4], hi[5]); h4.w = pack_bf16x2(hi[6], hi[7]);
-        l4.x = pack_bf16x2(lo[0], lo[1]); l4.y = pack_bf16x2(lo[2], lo[3]);
-        l4.z = pack_bf16x2(lo[4], lo[5]); l4.w = pack_bf16x2(lo[6], lo[7]);
-        *reinterpret_cast<uint4*>(out + (size_t)(2 * m) * kImg + sw_off(c, j)) = h4;
-        *reinterpret_cast<uint4*>(out + (size_t)(2 * m + 1) * kImg + sw_off(c, j)) = l4;
+        for (int k0 = 0; k0 < nslots; k0 += 8) {
+            float4 v[3][8];
+#pragma unroll
+            for (int g = 0; g < 3; ++g)
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    v[g][q] = k0 + q < nslots ? __ldcg(src + (size_t)(k0 + q) * (kPartial / 4) + off[g])
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int g = 0; g < 3; ++g)
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (k0 + q < nslots) {
+                        acc[g].x += v[g][q].x; acc[g].y += v[g][q].y; acc[g].z += v[g][q].z; acc[g].w += v[g][q].w;
+                    }
+        }
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            const int f = f0 + g * kMergeThreads;
+            if (f < F4) {
+                int sr; float* d;
+                merge_row<ROWS>(s, f / (D / 4), i0, sr, d);
+                *reinterpret_cast<float4*>(d + 4 * (f % (D / 4))) = acc[g];
+            }
+        }
+    }
+    const float4* w04 = reinterpret_cast<const float4*>(p.W0 + (size_t)h * D * D);
+#pragma unroll
+    for (int k = 0; k < D * D / 4 / kMergeThreads; ++k) {
+        const int e = 4 * (tid + k * kMergeThreads);
+        *reinterpret_cast<float4*>(&s.w0[e / D][e % D]) = __ldg(w04 + tid + k * kMergeThreads);
+    }
+    __syncthreads();
+    const int a0 = (tid >> 4) * RPT, j0 = (tid & 15) * 4;     // rows i0 + a0 .. i0 + a0 + RPT - 1
+    float P[RPT][4], Mr[RPT][4], Mc[RPT][4], WG[RPT][4];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) { P[r][b] = 0.f; Mr[r][b] = 0.f; Mc[r][b] = 0.f; WG[r][b] = 0.f; }
+#pragma unroll 4
+    for (int m = 0; m < D; ++m) {
+        const float4 g4 = *reinterpret_cast<const float4*>(&s.g[m][j0]);
+        const float4 d4 = *reinterpret_cast<const float4*>(&s.dw1[m][j0]);
+        const float4 w4 = *reinterpret_cast<const float4*>(&s.w0[m][j0]);
+        const float gv[4] = {g4.x, g4.y, g4.z, g4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w}, wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int i = i0 + a0 + r;
+            const float wim = s.w0[i][m], wmi = s.w0[m][i], dmi = s.dw1[m][i], dim = s.dw1[i][m];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                P[r][b] = fmaf(wim, gv[b], P[r][b]);       // (W0 G)[i][j]
+                Mr[r][b] = fmaf(wmi, dv[b], Mr[r][b]);     // M[i][j] = sum_m W0[m][i] dW1[m][j]
+                Mc[r][b] = fmaf(wv[b], dmi, Mc[r][b]);     // M[j][i]
+                WG[r][b] = fmaf(dim, gv[b], WG[r][b]);     // (dW1 G)[i][j]
+            }
+        }
+    }
+    uint8_t* out = imgs + (size_t)u * kImgs * kImg;
+    float part = 0.f;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = i0 + a0 + r;
+        float dc[4], dg[4], dw0[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int j = j0 + b;
+            const float pij = P[r][b] - s.c[a0 + r][j], g = s.dw1[i][j];
+            const float w1 = s.w0[i][j] - p.s * pij;
+            dc[b] = p.s * g;
+            dg[b] = -p.s * (Mr[r][b] + Mc[r][b]);
+            dw0[b] = g - p.s * WG[r][b];
+            part = fmaf(g, pij, part);
+            // W1^T and dC^T (row c = j, K = i): staged, stored below as 16-byte chunks
+            const __nv_bfloat16 wh = __float2bfloat16_rn(w1), ch = __float2bfloat16_rn(dc[b]);
+            s.tr[0][j][i - i0] = wh;
+            s.tr[1][j][i - i0] = __float2bfloat16_rn(w1 - __bfloat162float(wh));
+            s.tr[2][j][i - i0] = ch;
+            s.tr[3][j][i - i0] = __float2bfloat16_rn(dc[b] - __bfloat162float(ch));
+        }
+        put_hi_lo4(out + 2 * kImg, i, j0, dc);                // dC: row c = i, K = j
+        put_hi_lo4(out + 6 * kImg, i, j0, dg);                // dG + dG^T: row c = i, K = j
+        *reinterpret_cast<float4*>(p.dW0_unit + (size_t)u * D * D + (size_t)i * D + j0) =
+            make_float4(dw0[0], dw0[1], dw0[2], dw0[3]);
+    }
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((tid & 31) == 0) s.red[tid >> 5] = part;
+    __syncthreads();
+    // the staged chunks: images 0, 1 (W1^T hi, lo) and 4, 5 (dC^T hi, lo), rows c, chunks of K = i
+    constexpr int CH = ROWS / 8;
+    for (int e = tid; e < 4 * D * CH; e += kMergeThreads) {
+        const int x = e / (D * CH), c = (e / CH) % D, k = e % CH;
+        const int img = (x < 2) ? x : x + 2;
+        *reinterpret_cast<uint4*>(out + (size_t)img * kImg + sw_off(c, i0 / 8 + k)) =
+            *reinterpret_cast<const uint4*>(&s.tr[x][c][8 * k]);
+    }
+    if (tid == 0) {
+        float t = 0.f;
+        for (int w = 0; w < kMergeThreads / 32; ++w) t += s.red[w];
+        p.deta_unit[blockIdx.x] = p.eta_grad_scale * t;
     }
 }
 
@@ -712,6 +872,7 @@ lin_bwd_p2_tc(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_launch_dependents();                 // lin_bwd_sum waits for this grid's completion itself
     const uint32_t tmem = s.tmem_base;
     if (warp == 0) {
         if (lane == 0) p2_producer(s, p, &tmZ, &tmK, &tmV, ab);
@@ -751,7 +912,7 @@ static WsLayout ws_layout(long long units) {
     L.mats = align_up(L.partials + (size_t)(kMaxGrid + units) * kPartial * sizeof(float), 1024);
     L.dw0 = align_up(L.mats + (size_t)units * kMats * D * D * sizeof(float), 1024);
     L.deta = align_up(L.dw0 + (size_t)units * D * D * sizeof(float), 256);
-    L.imgs = align_up(L.deta + (size_t)units * sizeof(float), 1024);
+    L.imgs = align_up(L.deta + (size_t)units * tc::kMaxSplit * sizeof(float), 1024);
     L.total = L.imgs + (size_t)units * tc::kImgs * tc::kImg;
     return L;
 }
@@ -776,10 +937,12 @@ static ttt_status launch_tc(const Call& c, Params p, const WsLayout& L) {
     tp.imgs = c.ws + L.imgs;
     tp.err = reinterpret_cast<uint32_t*>(c.ws);
     tp.wait_ns = c.wait_ns;
-    const size_t sm1 = sizeof(P1TcSmem) + 1024, smm = sizeof(P1Smem) + 128, sm2 = sizeof(P2TcSmem) + 1024;
+    const size_t sm1 = sizeof(P1TcSmem) + 1024, sm2 = sizeof(P2TcSmem) + 1024;
     if (sm1 > 227 * 1024 || sm2 > 227 * 1024) return TTT_ERR_UNSUPPORTED;
     cudaFuncSetAttribute(lin_bwd_p1_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-    cudaFuncSetAttribute(lin_bwd_merge_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smm);
+    cudaFuncSetAttribute(lin_bwd_merge_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMergeSmem);
+    cudaFuncSetAttribute(lin_bwd_merge_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMergeSmem);
+    cudaFuncSetAttribute(lin_bwd_merge_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMergeSmem);
     cudaFuncSetAttribute(lin_bwd_p2_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
     lin_bwd_p1_tc<<<G, kThreads, sm1, c.stream>>>(tmK, tmV, tmZ, tmQ, tp);
     ttt_status st = check_launch(cudaGetLastError());
@@ -788,21 +951,28 @@ static ttt_status launch_tc(const Call& c, Params p, const WsLayout& L) {
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)p.units);
-    cfg.blockDim = dim3(P1_THREADS);
-    cfg.dynamicSmemBytes = smm;
+    // merge CTAs per unit: the most of 4, 2, 1 that keeps every merge CTA on an SM of its own
+    const int split = (p.units * 4 <= c.num_sms) ? 4 : (p.units * 2 <= c.num_sms) ? 2 : 1;
+    p.deta_terms = p.units * split;
+    cfg.gridDim = dim3((unsigned)(p.units * split));
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = kMergeSmem;
     cfg.stream = c.stream;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_merge_tc, p, c.ws + L.imgs));
+    st = check_launch(split == 4 ? cudaLaunchKernelEx(&cfg, lin_bwd_merge_tc<4>, p, c.ws + L.imgs)
+                      : split == 2 ? cudaLaunchKernelEx(&cfg, lin_bwd_merge_tc<2>, p, c.ws + L.imgs)
+                                   : cudaLaunchKernelEx(&cfg, lin_bwd_merge_tc<1>, p, c.ws + L.imgs));
     if (st != TTT_OK) return st;
     cfg.gridDim = dim3((unsigned)G);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = sm2;
     st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2_tc, tmZ, tmK, tmV, tmdQ, tmdK, tmdV, tp));
     if (st != TTT_OK || (!p.dW0_out && !p.deta_out)) return st;
-    lin_bwd_sum<<<c.heads, 256, 0, c.stream>>>(p, c.batch);
-    return check_launch(cudaGetLastError());
+    cfg.gridDim = dim3((unsigned)(c.heads * 4));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    return check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_sum, p, c.batch));
 }
 
 template <typename E>
@@ -829,6 +999,7 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
     p.mats = reinterpret_cast<float*>(c.ws + L.mats);
     p.dW0_unit = reinterpret_cast<float*>(c.ws + L.dw0);
     p.deta_unit = reinterpret_cast<float*>(c.ws + L.deta);
+    p.deta_terms = (int)units;
     p.dW0_out = dW0_out;
     p.deta_out = deta_out;
     if constexpr (std::is_same<E, __nv_bfloat16>::value) {
@@ -853,7 +1024,7 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
         cfg.numAttrs = 1;
         st = check_launch(cudaLaunchKernelEx(&cfg, lin_bwd_p2<E>, p, tiles2));
         if (st != TTT_OK || (!dW0_out && !deta_out)) return st;
-        lin_bwd_sum<<<c.heads, 256, 0, c.stream>>>(p, c.batch);
+        lin_bwd_sum<<<c.heads * 4, 256, 0, c.stream>>>(p, c.batch);
         return check_launch(cudaGetLastError());
     }
 }
