@@ -49,10 +49,8 @@ constexpr int TAPS = 9;
 constexpr int TR = 8, TC = 16;              // a tile: 8 grid rows x 16 grid columns
 constexpr int TILE = TR * TC;               // 128 positions (the MMA's M)
 constexpr int BOX = TILE * D * 2;           // one tap box: 16 KB (128 bytes per position)
-constexpr int PAIR = 2 * BOX;               // one ring stage: two taps
-constexpr int NPAIR = 5;                    // taps (0,1) (2,3) (4,5) (6,7) (8)
-constexpr int S1 = 3;                       // ring stages of the gradient kernel
-constexpr int S3 = 3;                       // ring stages of the readout kernel
+constexpr int HALO = (TR + 2) * TC * 128;   // a tile's rows -1 .. 8 at one x shift: 20 KB
+constexpr int NPAIR = 5;                    // gradient accumulators: two taps each (the last one tap)
 constexpr int kWImg = D * D * 2;            // one tap's weights as a bf16 operand image: 8 KB
 constexpr int kThreads = 192;
 constexpr int kMaxGrid = 160;               // slots of the workspace: (kMaxGrid + units)
@@ -62,7 +60,18 @@ constexpr uint32_t kIdescCol = idesc_bf16_f32(128, 64, true, true);    // D[m][c
 constexpr uint32_t kColR = 0;               // tensor memory: two R accumulators,
 constexpr uint32_t kColG = 128;             //   five tap-pair gradient accumulators (448 columns)
 
-__host__ __device__ __forceinline__ int taps_in_pair(int k) { return k < 4 ? 2 : 1; }
+// A tile's operands are three halo buffers: buffer b holds grid rows y0-1 .. y0+8 at columns
+// x0+b-1 .. x0+b+14 (a 10 x 16 TMA box, 128-byte swizzled rows of 64 channels).  Tap t = 3a + b
+// (shift (a-1, b-1)) is the 128 rows of buffer b starting at row 16a: 1024-byte aligned, so every
+// tap is an ordinary operand box and the nine taps cost three loads.
+__device__ __forceinline__ uint32_t tap_box(uint32_t halo0, int t9) {
+    return halo0 + (uint32_t)((t9 % 3) * HALO + (t9 / 3) * TC * 128);
+}
+// The gradient's tap pairs: the two taps of pair k are one M = 128 operand whose second half lies
+// kPairLbo[k] bytes after the first (the same x shift one grid row further, or the next buffer);
+// the last accumulator's second half reads rows nothing uses.
+__constant__ int kPairTap[NPAIR][2] = {{0, 3}, {1, 4}, {2, 5}, {6, 7}, {8, 8}};
+__constant__ uint32_t kPairLbo[NPAIR] = {TC * 128, TC * 128, TC * 128, (uint32_t)HALO, TC * 128};
 
 struct Geo {
     int heads, H, W;
@@ -74,6 +83,25 @@ struct Geo {
 // CTA c of G owns tiles [start(c), start(c + 1)); the CTA that owns tile t.
 __host__ __device__ __forceinline__ long long part_start(long long T, int G, int c) { return (long long)c * T / G; }
 __host__ __device__ __forceinline__ int part_cta(long long T, int G, long long t) { return (int)(((t + 1) * G - 1) / T); }
+
+// The gradient kernel's tiles: with cpu > 0, cpu CTAs per unit, CTA c taking a contiguous share of
+// unit c / cpu's tiles only (no CTA drains two units' gradients); with cpu = 0 (more units than CTAs),
+// the contiguous split above.
+struct GradPart {
+    long long T;
+    int G, cpu, tpu;
+    __host__ __device__ __forceinline__ long long start(int c) const {
+        if (cpu == 0) return part_start(T, G, c);
+        const int u = c / cpu, k = c % cpu;
+        return (long long)u * tpu + (long long)k * tpu / cpu;
+    }
+    __host__ __device__ __forceinline__ int first_cta(int u) const {
+        return cpu ? u * cpu : part_cta(T, G, (long long)u * tpu);
+    }
+    __host__ __device__ __forceinline__ int last_cta(int u) const {
+        return cpu ? (u + 1) * cpu - 1 : part_cta(T, G, (long long)(u + 1) * tpu - 1);
+    }
+};
 
 struct TileXY {
     int u, b, h, x0, y0;
@@ -126,20 +154,20 @@ conv3_wprep(const float* __restrict__ W0, uint8_t* __restrict__ w0img) {
 
 struct GradParams {
     Geo g;
-    int G;                                   // CTAs
+    GradPart part;                           // the CTAs' tile ranges
     const uint8_t* w0img;                    // [heads][9][kWImg], written by conv3_wprep
+    const __nv_bfloat16* V;                  // V, read directly by the epilogue
+    long long bs, hs;                        // V's element strides of an image and of a head
     float* slots;                            // [(kMaxGrid + U)][9][64][64]: G of a (CTA, unit) part
     uint32_t* err;
     unsigned long long wait_ns;
 };
 
 struct GradSmem {
-    uint8_t ring[S1][PAIR];                  // 1024-aligned operand buffers
+    uint8_t kh[2][3][HALO];                  // two tiles' K halo buffers (x shift b = 0, 1, 2)
     uint8_t w0img[TAPS][kWImg];              // W0 of the part's head, bf16 (row c, K = c')
-    uint8_t vbuf[BOX];                       // the tile's V
     uint8_t rhi[BOX], rlo[BOX];              // r = R - V as bf16 hi and lo (position-major)
-    uint64_t full[S1], empty[S1];
-    uint64_t vfull, vempty;
+    uint64_t kfull[2], kempty[2];
     uint64_t dr_full[2], dr_empty[2];        // R accumulators
     uint64_t r_full, r_empty;                // r operands written / read by every MMA of the tile
     uint64_t w_full, w_empty;                // W0 images written / no longer read
@@ -151,8 +179,7 @@ struct GradSmem {
 
 // The CTA's tiles n = 0 .. N-1 go through the tensor pipe in the order R(0), R(1), G(0), R(2), G(1),
 // ..., R(N-1), G(N-2), G(N-1): while the epilogue turns R(n) into the residual operand of G(n), the
-// MMAs of R(n+1) run.  The producer loads in the same order: V(n) and the nine K boxes of R(n), then
-// the nine K boxes of G(n-1) again.
+// MMAs of R(n+1) run.  Tile n's K halo (three boxes) sits in buffer n & 1 from R(n) to G(n).
 __host__ __device__ __forceinline__ bool first_of_part(const Geo& g, long long t0, long long t) {
     return t == t0 || t % g.tpu == 0;
 }
@@ -160,114 +187,76 @@ __host__ __device__ __forceinline__ bool last_of_part(const Geo& g, long long t1
     return t + 1 == t1 || (t + 1) % g.tpu == 0;
 }
 
-struct Ring {
-    int st = 0;
-    uint32_t ph = 0, issued = 0;
-    __device__ __forceinline__ void advance() {
-        ++issued;
-        if (++st == S1) { st = 0; ph ^= 1u; }
-    }
-};
-
-// The nine K boxes of tile t at their tap shifts, two taps per ring stage.
-__device__ __forceinline__ bool load_taps(GradSmem& s, const CUtensorMap* tmK, const TileXY& x, Ring& rg,
-                                          const Abort& ab) {
-    for (int k = 0; k < NPAIR; ++k) {
-        if (!mbar_wait(&s.empty[rg.st], rg.ph ^ 1u, ab)) return false;
-        const int nt = taps_in_pair(k);
-        mbar_arrive_expect_tx(&s.full[rg.st], (uint32_t)(nt * BOX));
-        for (int j = 0; j < nt; ++j) {
-            const int t9 = 2 * k + j, a = t9 / 3, bb = t9 % 3;
-            tma_load_5d(s.ring[rg.st] + j * BOX, tmK, &s.full[rg.st], 0, x.x0 + bb - 1, x.y0 + a - 1, x.h, x.b);
+__device__ __forceinline__ void grad_producer(GradSmem& s, const GradParams& p, const CUtensorMap* tmH,
+                                              const Abort& ab) {
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
+    uint32_t parts = 0, n = 0;
+    for (long long t = t0; t < t1; ++t, ++n) {
+        const TileXY x = tile_xy(p.g, t);
+        if (first_of_part(p.g, t0, t)) {
+            // the head's W0 tap images, once the previous part's R MMAs are done with them
+            if (t == t0) pdl_wait_primary();                 // conv3_wprep has written the images
+            if (!mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab)) break;
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
+            bulk_g2s(s.w0img, p.w0img + (size_t)x.h * TAPS * kWImg, TAPS * kWImg, &s.w_full);
+            ++parts;
         }
-        rg.advance();
-    }
-    return true;
-}
-
-__device__ __forceinline__ void grad_producer(GradSmem& s, const GradParams& p, const CUtensorMap* tmK,
-                                              const CUtensorMap* tmV, const Abort& ab) {
-    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    uint32_t vq = 0, parts = 0;
-    Ring rg;
-    bool ok = true;
-    for (long long t = t0; t <= t1 && ok; ++t) {
-        if (t < t1) {
-            const TileXY x = tile_xy(p.g, t);
-            if (first_of_part(p.g, t0, t)) {
-                // the head's W0 tap images, once the previous part's R MMAs are done with them
-                if (t == t0) pdl_wait_primary();             // conv3_wprep has written the images
-                if (!(ok = mbar_wait(&s.w_empty, (parts & 1u) ^ 1u, ab))) break;
-                fence_proxy_async_global();
-                mbar_arrive_expect_tx(&s.w_full, TAPS * kWImg);
-                bulk_g2s(s.w0img, p.w0img + (size_t)x.h * TAPS * kWImg, TAPS * kWImg, &s.w_full);
-                ++parts;
-            }
-            if (!(ok = mbar_wait(&s.vempty, (vq & 1u) ^ 1u, ab))) break;
-            mbar_arrive_expect_tx(&s.vfull, BOX);
-            tma_load_5d(s.vbuf, tmV, &s.vfull, 0, x.x0, x.y0, x.h, x.b);
-            ++vq;
-            if (!(ok = load_taps(s, tmK, x, rg, ab))) break;
-        }
-        if (t > t0) ok = load_taps(s, tmK, tile_xy(p.g, t - 1), rg, ab);
+        const uint32_t kb = n & 1u;
+        if (!mbar_wait(&s.kempty[kb], ((n >> 1) & 1u) ^ 1u, ab)) break;
+        mbar_arrive_expect_tx(&s.kfull[kb], 3 * HALO);
+        for (int b = 0; b < 3; ++b)
+            tma_load_5d(s.kh[kb][b], tmH, &s.kfull[kb], 0, x.x0 + b - 1, x.y0 - 1, x.h, x.b);
     }
     // every copy issued has landed before the CTA may exit
-    for (uint32_t k = rg.issued > (uint32_t)S1 ? rg.issued - S1 : 0u; k < rg.issued; ++k)
-        mbar_drain(&s.full[k % S1], (k / S1) & 1u, ab.limit);
-    if (vq > 0) mbar_drain(&s.vfull, (vq - 1) & 1u, ab.limit);
+    for (uint32_t k = n > 2u ? n - 2u : 0u; k < n; ++k) mbar_drain(&s.kfull[k & 1u], (k >> 1) & 1u, ab.limit);
     if (parts > 0) mbar_drain(&s.w_full, (parts - 1) & 1u, ab.limit);
 }
 
-// R(t) = sum_t9 K_t9 W0_t9^T into R accumulator n & 1 (A: K box, K-major; B: W0 tap image).
+// R(t) = sum_t9 K_t9 W0_t9^T into R accumulator n & 1 (A: the tap's rows of the K halo, K-major;
+// B: W0 tap image).
 __device__ __forceinline__ bool mma_R(GradSmem& s, const GradParams& p, uint32_t tmem, long long t0, long long t1,
-                                      long long t, uint32_t n, uint32_t& wparts, Ring& rg, const Abort& ab) {
+                                      long long t, uint32_t n, uint32_t& wparts, const Abort& ab) {
     if (first_of_part(p.g, t0, t)) {
         if (!mbar_wait(&s.w_full, wparts & 1u, ab)) return false;
         ++wparts;
     }
-    const uint32_t dr = n & 1u;
+    const uint32_t dr = n & 1u, kb = n & 1u;
     if (!mbar_wait(&s.dr_empty[dr], ((n >> 1) & 1u) ^ 1u, ab)) return false;
+    if (!mbar_wait(&s.kfull[kb], (n >> 1) & 1u, ab)) return false;
     tc_fence_after();
-    for (int k = 0; k < NPAIR; ++k) {
-        if (!mbar_wait(&s.full[rg.st], rg.ph, ab)) return false;
-        tc_fence_after();
-        for (int j = 0; j < taps_in_pair(k); ++j) {
-            const uint32_t sa = smem_u32(s.ring[rg.st] + j * BOX), sb = smem_u32(s.w0img[2 * k + j]);
+    for (int t9 = 0; t9 < TAPS; ++t9) {
+        const uint32_t sa = tap_box(smem_u32(s.kh[kb][0]), t9), sb = smem_u32(s.w0img[t9]);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                mma_bf16_ss(tmem + kColR + dr * 64u, sdesc_sw128(sa + kk * 32, 16, 1024),
-                            sdesc_sw128(sb + kk * 32, 16, 1024), kIdescRow, (k | j | kk) ? 1u : 0u);
-        }
-        mma_commit(&s.empty[rg.st]);
-        rg.advance();
+        for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + kColR + dr * 64u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024),
+                        kIdescRow, (t9 | kk) ? 1u : 0u);
     }
     mma_commit(&s.dr_full[dr]);
     if (last_of_part(p.g, t1, t)) mma_commit(&s.w_empty);    // the part's last reads of the W0 images
     return true;
 }
 
-// G^T[pair k] += [K_2k | K_2k+1]^T (r_hi + r_lo) for tile t (A MN-major, M = 128; B = r, MN-major).
+// G^T[pair k] += [K_a | K_b]^T (r_hi + r_lo) for tile t, the pair's two taps as one M = 128 operand
+// (MN-major: the second tap's rows lie kPairLbo[k] bytes after the first's); frees the K halo.
 __device__ __forceinline__ bool mma_G(GradSmem& s, const GradParams& p, uint32_t tmem, long long t0, long long t1,
-                                      long long t, uint32_t n, uint32_t& gparts, Ring& rg, const Abort& ab) {
+                                      long long t, uint32_t n, uint32_t& gparts, const Abort& ab) {
     if (!mbar_wait(&s.r_full, n & 1u, ab)) return false;
     const bool first = first_of_part(p.g, t0, t);
     if (first && !mbar_wait(&s.g_empty, (gparts & 1u) ^ 1u, ab)) return false;
     tc_fence_after();
-    const uint32_t shi = smem_u32(s.rhi), slo = smem_u32(s.rlo);
+    const uint32_t shi = smem_u32(s.rhi), slo = smem_u32(s.rlo), kh = smem_u32(s.kh[n & 1u][0]);
     for (int k = 0; k < NPAIR; ++k) {
-        if (!mbar_wait(&s.full[rg.st], rg.ph, ab)) return false;
-        tc_fence_after();
-        const uint32_t sa = smem_u32(s.ring[rg.st]);
+        const uint32_t sa = tap_box(kh, kPairTap[k][0]), lbo = kPairLbo[k];
         const uint32_t dg = tmem + kColG + (uint32_t)k * 64u;
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sa + kk * 2048, BOX, 1024);
+            const uint64_t ad = sdesc_sw128(sa + kk * 2048, lbo, 1024);
             mma_bf16_ss(dg, ad, sdesc_sw128(shi + kk * 2048, BOX, 1024), kIdescCol, (first && kk == 0) ? 0u : 1u);
             mma_bf16_ss(dg, ad, sdesc_sw128(slo + kk * 2048, BOX, 1024), kIdescCol, 1u);
         }
-        mma_commit(&s.empty[rg.st]);
-        rg.advance();
     }
+    mma_commit(&s.kempty[n & 1u]);
     mma_commit(&s.r_empty);
     if (last_of_part(p.g, t1, t)) {
         mma_commit(&s.g_full);
@@ -277,13 +266,12 @@ __device__ __forceinline__ bool mma_G(GradSmem& s, const GradParams& p, uint32_t
 }
 
 __device__ __forceinline__ void grad_mma(GradSmem& s, const GradParams& p, uint32_t tmem, const Abort& ab) {
-    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    Ring rg;
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
     uint32_t wparts = 0, gparts = 0;
     for (long long t = t0; t <= t1; ++t) {
         const uint32_t n = (uint32_t)(t - t0);
-        if (t < t1 && !mma_R(s, p, tmem, t0, t1, t, n, wparts, rg, ab)) return;
-        if (t > t0 && !mma_G(s, p, tmem, t0, t1, t - 1, n - 1, gparts, rg, ab)) return;
+        if (t < t1 && !mma_R(s, p, tmem, t0, t1, t, n, wparts, ab)) return;
+        if (t > t0 && !mma_G(s, p, tmem, t0, t1, t - 1, n - 1, gparts, ab)) return;
     }
 }
 
@@ -293,7 +281,7 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
     const int r = q * 32 + lane;                              // accumulator row = tile position
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
+    const long long t0 = p.part.start(blockIdx.x), t1 = p.part.start(blockIdx.x + 1);
     uint32_t n = 0, part = 0;
     bool failed = false;
     for (long long t = t0; t < t1 && !failed;) {
@@ -302,8 +290,17 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
         bool ok = true;
         for (long long tt = t; tt < pe; ++tt, ++n) {
             const TileXY x = tile_xy(p.g, tt);
+            // this position's V row (positions outside the grid contribute nothing), loaded before the
+            // wait for R
+            const int y = x.y0 + r / TC, xx = x.x0 + r % TC;
+            const bool inside = y < p.g.H && xx < p.g.W;
+            uint4 vw[8];
+            const uint4* vrow = reinterpret_cast<const uint4*>(
+                p.V + (size_t)x.b * p.bs + (size_t)x.h * p.hs + ((size_t)y * p.g.W + xx) * D);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) vw[j] = inside ? __ldg(vrow + j) : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t dr = n & 1u;
-            ok = mbar_wait(&s.dr_full[dr], (n >> 1) & 1u, ab) && mbar_wait(&s.vfull, n & 1u, ab);
+            ok = mbar_wait(&s.dr_full[dr], (n >> 1) & 1u, ab);
             if (named_bar_or(1, 128, !ok)) { failed = true; break; }
             __syncwarp();
             tc_fence_after();
@@ -313,13 +310,11 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&s.dr_empty[dr]);
-            // r = R - V; positions outside the grid contribute nothing
-            const bool inside = (x.y0 + r / TC) < p.g.H && (x.x0 + r % TC) < p.g.W;
+            // r = R - V
             float res[64];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint4 w = *reinterpret_cast<const uint4*>(s.vbuf + sw_off(r, j));
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                const uint32_t ww[4] = {vw[j].x, vw[j].y, vw[j].z, vw[j].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = 8 * j + 2 * e;
@@ -327,7 +322,6 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
                     res[c + 1] = inside ? v[(c + 1) / 16][(c + 1) % 16] - bf16hi_to_f32(ww[e]) : 0.f;
                 }
             }
-            mbar_arrive(&s.vempty);
             ok = mbar_wait(&s.r_empty, (n & 1u) ^ 1u, ab);   // the previous tile's MMAs read r
             if (named_bar_or(1, 128, !ok)) { failed = true; break; }
 #pragma unroll
@@ -346,7 +340,7 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
             if (tid == 0) mbar_arrive(&s.r_full);
         }
         if (failed) break;
-        // the part's gradient: accumulator k, row r is channel c' = r % 64 of tap 2k + r / 64
+        // the part's gradient: accumulator k, row r is channel c' = r % 64 of tap kPairTap[k][r / 64]
         ok = mbar_wait(&s.g_full, part & 1u, ab);
         if (named_bar_or(1, 128, !ok)) break;
         __syncwarp();
@@ -357,8 +351,8 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
 #pragma unroll
             for (int j = 0; j < 4; ++j) tmem_ld16(tmem + kColG + (uint32_t)(k * 64 + j * 16) + lane_off, g[j]);
             tmem_ld_wait();
-            const int t9 = 2 * k + r / D;
-            if (t9 < TAPS) {
+            if (k < NPAIR - 1 || r < D) {
+                const int t9 = kPairTap[k][r / D];
                 float* dst = slot + (size_t)t9 * D * D + (r % D);    // G[t9][c][c' = r % 64]
 #pragma unroll
                 for (int c = 0; c < D; ++c) __stcg(dst + (size_t)c * D, g[c / 16][c % 16]);
@@ -372,22 +366,21 @@ __device__ __forceinline__ void grad_epilogue(GradSmem& s, const GradParams& p, 
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-conv3_grad(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const GradParams p) {
+conv3_grad(const __grid_constant__ CUtensorMap tmH, const GradParams p) {
     extern __shared__ uint8_t smem_raw[];
     GradSmem& s = *reinterpret_cast<GradSmem*>(align1024(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Abort ab{&s.abort_flag, p.err, p.wait_ns};
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
-        for (int i = 0; i < S1; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
-        mbar_init(&s.vfull, 1); mbar_init(&s.vempty, 128);
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.kfull[i], 1); mbar_init(&s.kempty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&s.dr_full[i], 1); mbar_init(&s.dr_empty[i], 128); }
         mbar_init(&s.r_full, 1); mbar_init(&s.r_empty, 1);
         mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
         mbar_init(&s.g_full, 1); mbar_init(&s.g_empty, 128);
         mbar_init(&s.drain_bar, 1);
         fence_barrier_init();
-        prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+        prefetch_tmap(&tmH);
     }
     if (warp == 1) { tmem_alloc(&s.tmem_base, 512); tmem_relinquish(); }
     tc_fence_before();
@@ -396,7 +389,7 @@ conv3_grad(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     pdl_launch_dependents();                                 // the merge kernel may be scheduled
     const uint32_t tmem = s.tmem_base;
     if (warp == 0) {
-        if (lane == 0) grad_producer(s, p, &tmK, &tmV, ab);
+        if (lane == 0) grad_producer(s, p, &tmH, ab);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
@@ -423,7 +416,7 @@ conv3_grad(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 // ------------------------------------------------------------------------------------------------
 struct MergeParams {
     Geo g;
-    int G;                                   // CTAs of conv3_grad
+    GradPart part;                           // the tile ranges of conv3_grad's CTAs
     float eta;
     const float* W0;                         // [heads][64][64][9]
     const float* slots;
@@ -437,8 +430,7 @@ conv3_merge(const MergeParams p) {
     const int u = ut / TAPS, t9 = ut % TAPS, h = u % p.g.heads;
     pdl_launch_dependents();
     pdl_wait_primary();                                      // every gradient slot is written
-    const int cf = part_cta(p.g.T, p.G, (long long)u * p.g.tpu);
-    const int cl = part_cta(p.g.T, p.G, (long long)(u + 1) * p.g.tpu - 1);
+    const int cf = p.part.first_cta(u), cl = p.part.last_cta(u);
     uint8_t* img = p.w1img + ((size_t)u * TAPS + t9) * kWImg;
     const int e4 = q4 * 256 + (int)threadIdx.x;              // float4 of the tap's matrix: elements 4 e4 ..
     const float4* src = reinterpret_cast<const float4*>(p.slots + (size_t)t9 * D * D) + e4;
@@ -475,10 +467,10 @@ struct ReadParams {
 };
 
 struct ReadSmem {
-    uint8_t ring[S3][PAIR];
+    uint8_t qh[2][3][HALO];                  // two tiles' Q halo buffers (x shift b = 0, 1, 2)
     uint8_t w1img[TAPS][kWImg];
     uint8_t zbuf[2][BOX];
-    uint64_t full[S3], empty[S3];
+    uint64_t qfull[2], qempty[2];
     uint64_t w_full, w_empty;
     uint64_t dz_full[2], dz_empty[2];
     uint64_t drain_bar;
@@ -498,76 +490,58 @@ __device__ __forceinline__ bool load_w1(ReadSmem& s, const ReadParams& p, int u,
     return true;
 }
 
-__device__ __forceinline__ void read_producer(ReadSmem& s, const ReadParams& p, const CUtensorMap* tmQ,
+__device__ __forceinline__ void read_producer(ReadSmem& s, const ReadParams& p, const CUtensorMap* tmH,
                                               const Abort& ab) {
     const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    uint32_t issued = 0, parts = 0;
-    int st = 0; uint32_t ph = 0;
-    bool ok = true;
+    uint32_t parts = 0, n = 0;
     int pending = -1;                                        // unit whose W1 images are not requested yet
-    for (long long t = t0; t < t1 && ok;) {
-        const int u = (int)(t / p.g.tpu);
-        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
-        // the first part's images are requested once the ring's stages are in flight: the Q boxes (an
-        // input) load while the merge kernel is still writing W1
-        if (t == t0) pending = u;
-        else if (!(ok = load_w1(s, p, u, parts, ab))) break;
-        for (long long tt = t; tt < pe && ok; ++tt) {
-            const TileXY x = tile_xy(p.g, tt);
-            for (int k = 0; k < NPAIR; ++k) {
-                if (pending >= 0 && issued == (uint32_t)S3) {
-                    if (!(ok = load_w1(s, p, pending, parts, ab))) break;
-                    pending = -1;
-                }
-                if (!(ok = mbar_wait(&s.empty[st], ph ^ 1u, ab))) break;
-                const int nt = taps_in_pair(k);
-                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(nt * BOX));
-                for (int j = 0; j < nt; ++j) {
-                    const int t9 = 2 * k + j, a = t9 / 3, bb = t9 % 3;
-                    tma_load_5d(s.ring[st] + j * BOX, tmQ, &s.full[st], 0, x.x0 + bb - 1, x.y0 + a - 1, x.h, x.b);
-                }
-                ++issued;
-                if (++st == S3) { st = 0; ph ^= 1u; }
-            }
+    bool ok = true;
+    for (long long t = t0; t < t1 && ok; ++t, ++n) {
+        const TileXY x = tile_xy(p.g, t);
+        if (t == t0) {
+            pending = x.u;          // the first Q halos (an input) load while the merge kernel still writes W1
+        } else if (t % p.g.tpu == 0) {
+            if (pending >= 0 && !(ok = load_w1(s, p, pending, parts, ab))) break;
+            pending = -1;
+            if (!(ok = load_w1(s, p, x.u, parts, ab))) break;
         }
-        t = pe;
+        if (pending >= 0 && n == 2u) {                       // the next buffer is freed by the MMAs
+            if (!(ok = load_w1(s, p, pending, parts, ab))) break;
+            pending = -1;
+        }
+        const uint32_t qb = n & 1u;
+        if (!(ok = mbar_wait(&s.qempty[qb], ((n >> 1) & 1u) ^ 1u, ab))) break;
+        mbar_arrive_expect_tx(&s.qfull[qb], 3 * HALO);
+        for (int b = 0; b < 3; ++b)
+            tma_load_5d(s.qh[qb][b], tmH, &s.qfull[qb], 0, x.x0 + b - 1, x.y0 - 1, x.h, x.b);
     }
     if (ok && pending >= 0) load_w1(s, p, pending, parts, ab);
-    for (uint32_t k = issued > (uint32_t)S3 ? issued - S3 : 0u; k < issued; ++k)
-        mbar_drain(&s.full[k % S3], (k / S3) & 1u, ab.limit);
+    for (uint32_t k = n > 2u ? n - 2u : 0u; k < n; ++k) mbar_drain(&s.qfull[k & 1u], (k >> 1) & 1u, ab.limit);
     if (parts > 0) mbar_drain(&s.w_full, (parts - 1) & 1u, ab.limit);
 }
 
 __device__ __forceinline__ void read_mma(ReadSmem& s, const ReadParams& p, uint32_t tmem, const Abort& ab) {
     const long long t0 = part_start(p.g.T, p.G, blockIdx.x), t1 = part_start(p.g.T, p.G, blockIdx.x + 1);
-    int st = 0; uint32_t ph = 0;
-    uint32_t n = 0, part = 0;
-    for (long long t = t0; t < t1;) {
-        const int u = (int)(t / p.g.tpu);
-        const long long pe = (t1 < (long long)(u + 1) * p.g.tpu) ? t1 : (long long)(u + 1) * p.g.tpu;
-        if (!mbar_wait(&s.w_full, part & 1u, ab)) return;
-        for (long long tt = t; tt < pe; ++tt, ++n) {
-            const uint32_t dz = n & 1u;
-            if (!mbar_wait(&s.dz_empty[dz], ((n >> 1) & 1u) ^ 1u, ab)) return;
-            tc_fence_after();
-            for (int k = 0; k < NPAIR; ++k) {
-                if (!mbar_wait(&s.full[st], ph, ab)) return;
-                tc_fence_after();
-                for (int j = 0; j < taps_in_pair(k); ++j) {
-                    const uint32_t sa = smem_u32(s.ring[st] + j * BOX), sb = smem_u32(s.w1img[2 * k + j]);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_bf16_ss(tmem + dz * 64u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024),
-                                    kIdescRow, (k | j | kk) ? 1u : 0u);
-                }
-                mma_commit(&s.empty[st]);
-                if (++st == S3) { st = 0; ph ^= 1u; }
-            }
-            mma_commit(&s.dz_full[dz]);
+    uint32_t n = 0, parts = 0;
+    for (long long t = t0; t < t1; ++t, ++n) {
+        if (first_of_part(p.g, t0, t)) {
+            if (!mbar_wait(&s.w_full, parts & 1u, ab)) return;
+            ++parts;
         }
-        mma_commit(&s.w_empty);
-        ++part;
-        t = pe;
+        const uint32_t dz = n & 1u, qb = n & 1u;
+        if (!mbar_wait(&s.dz_empty[dz], ((n >> 1) & 1u) ^ 1u, ab)) return;
+        if (!mbar_wait(&s.qfull[qb], (n >> 1) & 1u, ab)) return;
+        tc_fence_after();
+        for (int t9 = 0; t9 < TAPS; ++t9) {
+            const uint32_t sa = tap_box(smem_u32(s.qh[qb][0]), t9), sb = smem_u32(s.w1img[t9]);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16_ss(tmem + dz * 64u, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024),
+                            kIdescRow, (t9 | kk) ? 1u : 0u);
+        }
+        mma_commit(&s.qempty[qb]);
+        mma_commit(&s.dz_full[dz]);
+        if (last_of_part(p.g, t1, t)) mma_commit(&s.w_empty);
     }
 }
 
@@ -610,19 +584,19 @@ __device__ __forceinline__ void read_epilogue(ReadSmem& s, const ReadParams& p, 
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-conv3_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmZ, const ReadParams p) {
+conv3_readout(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmZ, const ReadParams p) {
     extern __shared__ uint8_t smem_raw[];
     ReadSmem& s = *reinterpret_cast<ReadSmem*>(align1024(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Abort ab{&s.abort_flag, p.err, p.wait_ns};
     if (threadIdx.x == 0) {
         s.abort_flag = 0;
-        for (int i = 0; i < S3; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.qfull[i], 1); mbar_init(&s.qempty[i], 1); }
         mbar_init(&s.w_full, 1); mbar_init(&s.w_empty, 1);
         for (int i = 0; i < 2; ++i) { mbar_init(&s.dz_full[i], 1); mbar_init(&s.dz_empty[i], 128); }
         mbar_init(&s.drain_bar, 1);
         fence_barrier_init();
-        prefetch_tmap(&tmQ); prefetch_tmap(&tmZ);
+        prefetch_tmap(&tmH); prefetch_tmap(&tmZ);
     }
     if (warp == 1) { tmem_alloc(&s.tmem_base, 128); tmem_relinquish(); }
     tc_fence_before();
@@ -630,7 +604,7 @@ conv3_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
     if (warp == 0) {
-        if (lane == 0) read_producer(s, p, &tmQ, ab);
+        if (lane == 0) read_producer(s, p, &tmH, ab);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
@@ -690,18 +664,30 @@ ttt_status launch_conv3x3(const Call& c) {
     if (c.ws_bytes < L.total) return TTT_ERR_WORKSPACE;
     const Geo g = make_geo(c);
     if (g.T > (1LL << 40)) return TTT_ERR_UNSUPPORTED;
-    CUtensorMap tmK, tmV, tmQ, tmZ;
-    if (!make_tmap_grid_sw128(&tmK, c.K, c, TC, TR) || !make_tmap_grid_sw128(&tmV, c.V, c, TC, TR) ||
-        !make_tmap_grid_sw128(&tmQ, c.Q, c, TC, TR) || !make_tmap_grid_sw128(&tmZ, c.Z, c, TC, TR))
+    CUtensorMap tmKH, tmQH, tmZ;
+    if (!make_tmap_grid_sw128(&tmKH, c.K, c, TC, TR + 2) || !make_tmap_grid_sw128(&tmQH, c.Q, c, TC, TR + 2) ||
+        !make_tmap_grid_sw128(&tmZ, c.Z, c, TC, TR))
         return TTT_ERR_INVALID_ARG;
-    const int G1 = (int)std::max<long long>(1, std::min<long long>(std::min(c.num_sms, kMaxGrid), g.T));
+    // gradient CTAs: as many per unit as fit, each within one unit, when there are fewer units than SMs
+    const int S = std::min(c.num_sms, kMaxGrid);
+    GradPart gpart{g.T, 0, 0, g.tpu};
+    if (units <= S) {
+        gpart.cpu = std::max(1, std::min(S / (int)units, g.tpu));
+        gpart.G = (int)units * gpart.cpu;
+    } else {
+        gpart.G = (int)std::max<long long>(1, std::min<long long>(S, g.T));
+    }
+    const int G1 = gpart.G;
     const int G3 = (int)std::max<long long>(1, std::min<long long>(c.num_sms, g.T));
     uint32_t* err = reinterpret_cast<uint32_t*>(c.ws);
 
     GradParams gp{};
     gp.g = g;
-    gp.G = G1;
+    gp.part = gpart;
     gp.w0img = c.ws + L.w0img;
+    gp.V = static_cast<const __nv_bfloat16*>(c.V);
+    gp.bs = c.bs;
+    gp.hs = c.hs;
     gp.slots = reinterpret_cast<float*>(c.ws + L.slots);
     gp.err = err;
     gp.wait_ns = c.wait_ns;
@@ -727,12 +713,12 @@ ttt_status launch_conv3x3(const Call& c) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = sm1;
     cfg.numAttrs = 1;
-    st = check_launch(cudaLaunchKernelEx(&cfg, conv3_grad, tmK, tmV, gp));
+    st = check_launch(cudaLaunchKernelEx(&cfg, conv3_grad, tmKH, gp));
     if (st != TTT_OK) return st;
 
     MergeParams mp{};
     mp.g = g;
-    mp.G = G1;
+    mp.part = gpart;
     mp.eta = c.eta;
     mp.W0 = c.W0;
     mp.slots = gp.slots;
@@ -754,7 +740,7 @@ ttt_status launch_conv3x3(const Call& c) {
     cfg.gridDim = dim3((unsigned)G3);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = sm3;
-    return check_launch(cudaLaunchKernelEx(&cfg, conv3_readout, tmQ, tmZ, rp));
+    return check_launch(cudaLaunchKernelEx(&cfg, conv3_readout, tmQH, tmZ, rp));
 }
 
 }  // namespace ttt
