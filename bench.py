@@ -53,7 +53,7 @@ TRAFFIC = {
     "lin6400_bf16": {"read": 118183168, "write": 40068864, "src_sha": "e252f1ffc5b63f16"},
     "lin196_bf16": {"read": 14328832, "write": 599040, "src_sha": "e252f1ffc5b63f16"},
     "mlp1024_bf16": {"read": 25533440, "write": 6981376, "src_sha": "e351f2e6a0775778"},
-    "conv3x3_6084_bf16": {"read": 18741504, "write": 7558144, "src_sha": "2385ceaf5d3c5c3d"},
+    "conv3x3_6084_bf16": {"read": 18785024, "write": 7295744, "src_sha": "0d0c9febef88a717"},
     "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
     "bwd6084_bf16": {"read": 218148352, "write": 105013504, "src_sha": "c97c5f030b248cf5"},
     "bwdconv6084_bf16": {"read": 24883456, "write": 17042944, "src_sha": "1dfe7c0812e5935d"},
