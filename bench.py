@@ -64,6 +64,7 @@ TRAFFIC = {
 LAUNCHES_PER_STEP = {"linear": 1, "mixed": 2, "mlp": 1, "minibatch": 1, "backward": 4, "backward_conv": 4,
                      "backward_mlp": 7, "conv3x3": 4}
 LAUNCHES_PER_STEP_FP32 = {"linear": 2, "mixed": 3, "backward": 3}
+SMALL_F32_TOKENS = 384                       # fp32 linear units up to this many tokens: lin_small_f32
 
 
 # The CUDA sources each workload kind runs (besides the shared headers and the host entry points).
@@ -561,6 +562,7 @@ def roofline(w, t_step, pk, clocks, xs, stream, args):
             kern = f"layer step: lin_cluster_bf16 and {conv_name} running at the same time (one ttt_forward_layer call)"
         else:
             kern = "lin_cluster_bf16 (the whole ttt_forward_linear call)" if w.dtype == "bf16" else \
+                   "lin_small_f32 (the whole ttt_forward_linear call)" if w.N <= SMALL_F32_TOKENS else \
                    "lin_p1_f32 + lin_p2_f32 (the whole ttt_forward_linear call)"
         roof = {"bound": "hbm", "kernel": kern, "achieved": hbm, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": hbm / pk["hbm_gbs"], "peak_source": pk["source"] + " (copy bandwidth)", **common}
@@ -674,6 +676,8 @@ def run_ours(args):
     e2e = run_e2e(w, xs[0], dev, stream, args.e2e_steps, world)
 
     per_step = (LAUNCHES_PER_STEP_FP32 if w.dtype == "fp32" else {}).get(w.kind, LAUNCHES_PER_STEP[w.kind])
+    if w.dtype == "fp32" and w.kind in ("linear", "mixed") and w.N <= SMALL_F32_TOKENS:
+        per_step -= 1                        # one cluster kernel instead of the two tile kernels
     line = {"metric": METRIC_BWD if w.kind.startswith("backward") else METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",

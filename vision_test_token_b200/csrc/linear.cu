@@ -971,6 +971,192 @@ lin_p2_f32(TokenView Qv, float* Z, long long zbs, long long zhs, const float* W1
 // ------------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------------
+// ------------------------------------------------------------------------------------------------
+// lin_small_f32: fp32 units of at most kSmallN tokens (the 1e-5 case of a few hundred tokens, where
+// the tile kernels above are pure latency).  One cluster of kSmallCS CTAs per unit (a persistent loop
+// when there are more units than clusters).  Each CTA holds the unit's keys in shared memory and forms
+// kSmallRows rows of G = sum k k^T and C = sum v k^T; its G rows go to every CTA of the cluster
+// (distributed shared memory), each CTA forms its rows of W1 = W0 - eta_scale (W0 G - C) and sends
+// them likewise, then reads out its share of the tokens, z = W1 q.  Two cluster barriers per unit,
+// no workspace, every sum in a fixed order (bitwise reproducible).
+// ------------------------------------------------------------------------------------------------
+constexpr int kSmallCS = 8;
+constexpr int kSmallN = 384;
+constexpr int kSmallThreads = 512;
+constexpr int kSmallRows = D / kSmallCS;            // 8 rows of G, C, W1 per CTA
+constexpr int kSmallQ = kSmallN / kSmallCS + 1;     // tokens read out per CTA, at most
+
+struct SmallSmem {
+    float k[kSmallN][D];                 // the unit's keys
+    float v[kSmallN][kSmallRows];        // this CTA's columns of V
+    float q[kSmallQ][D];                 // this CTA's query tokens
+    float g[D][D];                       // G, gathered from the cluster
+    float w1t[D][D];                     // W1 transposed (w1t[m][j] = W1[j][m]), gathered
+    float w0[kSmallRows][D];             // this CTA's rows of W0
+    float part[kSmallRows][2][kSmallRows][D];   // the token groups' rows of G and C
+    float c[kSmallRows][D];              // this CTA's rows of C
+    uint64_t bar;                        // the bulk copies of a unit's rows
+    int abort_flag;
+};
+
+struct SmallParams {
+    TokenView Kv, Vv, Qv;
+    float* Z;
+    long long zbs, zhs;
+    const float* W0;
+    float* W1_out;
+    int heads, N, units, dot;
+    float eta_scale;                     // W1 = W0 - eta_scale (W0 G - C); dot loss: no W0 G term
+    uint32_t* err;
+    unsigned long long wait_ns;
+};
+
+__global__ void __launch_bounds__(kSmallThreads, 1)
+lin_small_f32(const SmallParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    SmallSmem& s = *reinterpret_cast<SmallSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int rank = (int)cluster_ctarank();
+    const int N = p.N;
+    const int n0 = rank * N / kSmallCS, n1 = (rank + 1) * N / kSmallCS;    // this CTA's query tokens
+    const Abort ab{&s.abort_flag, p.err, p.wait_ns};
+    if (tid == 0) {
+        s.abort_flag = 0;
+        mbar_init(&s.bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    uint32_t it = 0;
+    for (int u = (int)cluster_id_x(); u < p.units; u += (int)cluster_count_x(), ++it) {
+        const int h = u % p.heads;
+        // ---- the unit's keys, its query tokens and this CTA's rows of W0 by bulk copies (the rows
+        //      are contiguous), this CTA's columns of V by loads
+        if (tid == 0) {
+            const uint32_t nq = (uint32_t)(n1 - n0) * D * 4;
+            mbar_arrive_expect_tx(&s.bar, (uint32_t)N * D * 4 + nq + kSmallRows * D * 4);
+            bulk_g2s(&s.k[0][0], p.Kv.row(u, p.heads, 0), (uint32_t)N * D * 4, &s.bar);
+            if (nq) bulk_g2s(&s.q[0][0], p.Qv.row(u, p.heads, n0), nq, &s.bar);
+            bulk_g2s(&s.w0[0][0], p.W0 + ((size_t)h * D + rank * kSmallRows) * D, kSmallRows * D * 4, &s.bar);
+        }
+        {
+            float4 v4[(2 * kSmallN + kSmallThreads - 1) / kSmallThreads];
+#pragma unroll
+            for (int k = 0; k < (2 * kSmallN + kSmallThreads - 1) / kSmallThreads; ++k) {
+                const int e = tid + k * kSmallThreads;
+                if (e < 2 * N)
+                    v4[k] = __ldg(reinterpret_cast<const float4*>(p.Vv.row(u, p.heads, e >> 1) + rank * kSmallRows) + (e & 1));
+            }
+#pragma unroll
+            for (int k = 0; k < (2 * kSmallN + kSmallThreads - 1) / kSmallThreads; ++k) {
+                const int e = tid + k * kSmallThreads;
+                if (e < 2 * N) reinterpret_cast<float4*>(&s.v[e >> 1][0])[e & 1] = v4[k];
+            }
+        }
+        // every CTA of the cluster runs before any peer writes into it (first unit); peers are done
+        // reading what this unit's gathers overwrite (later units)
+        if (it == 0) cluster_sync_all();
+        mbar_wait(&s.bar, it & 1u, ab);  // on a timeout the error word says so; the cluster stays in step
+        __syncthreads();
+        // ---- rows of G and C: warp tg (< 8) sums tokens [tg N / 8, (tg + 1) N / 8) for all of this
+        //      CTA's rows and the lane's columns 2 lane, 2 lane + 1: per token one pair of key columns
+        //      and the CTA's eight key and value entries feed 32 FMAs
+        {
+            const int tg = tid >> 5;
+            if (tg < kSmallRows) {
+                float ag[kSmallRows][2], ac[kSmallRows][2];
+#pragma unroll
+                for (int a = 0; a < kSmallRows; ++a) { ag[a][0] = ag[a][1] = 0.f; ac[a][0] = ac[a][1] = 0.f; }
+                const int na = tg * N / kSmallRows, nb = (tg + 1) * N / kSmallRows;
+                for (int n = na; n < nb; ++n) {
+                    const float2 kj = *reinterpret_cast<const float2*>(&s.k[n][2 * lane]);
+                    const float4 k0 = *reinterpret_cast<const float4*>(&s.k[n][rank * kSmallRows]);
+                    const float4 k1 = *reinterpret_cast<const float4*>(&s.k[n][rank * kSmallRows + 4]);
+                    const float4 v0 = *reinterpret_cast<const float4*>(&s.v[n][0]);
+                    const float4 v1 = *reinterpret_cast<const float4*>(&s.v[n][4]);
+                    const float kr[kSmallRows] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    const float vr[kSmallRows] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                    for (int a = 0; a < kSmallRows; ++a) {
+                        ag[a][0] = fmaf(kr[a], kj.x, ag[a][0]); ag[a][1] = fmaf(kr[a], kj.y, ag[a][1]);
+                        ac[a][0] = fmaf(vr[a], kj.x, ac[a][0]); ac[a][1] = fmaf(vr[a], kj.y, ac[a][1]);
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < kSmallRows; ++a) {
+                    *reinterpret_cast<float2*>(&s.part[tg][0][a][2 * lane]) = make_float2(ag[a][0], ag[a][1]);
+                    *reinterpret_cast<float2*>(&s.part[tg][1][a][2 * lane]) = make_float2(ac[a][0], ac[a][1]);
+                }
+            }
+        }
+        __syncthreads();
+        // the token groups added in order: this CTA's rows of G (into the gathered G) and of C
+        for (int e = tid; e < 2 * kSmallRows * D; e += kSmallThreads) {
+            const int x = e / (kSmallRows * D), a = (e / D) % kSmallRows, j = e % D;
+            float acc = s.part[0][x][a][j];
+#pragma unroll
+            for (int t = 1; t < kSmallRows; ++t) acc += s.part[t][x][a][j];
+            if (x == 0) s.g[rank * kSmallRows + a][j] = acc;
+            else s.c[a][j] = acc;
+        }
+        __syncthreads();
+        // ---- this CTA's rows of G into every other CTA of the cluster, 16 bytes a store
+        for (int e = tid; e < (kSmallCS - 1) * kSmallRows * (D / 4); e += kSmallThreads) {
+            const int r = (rank + 1 + e / (kSmallRows * (D / 4))) % kSmallCS, f = e % (kSmallRows * (D / 4));
+            const uint32_t la = smem_u32(&s.g[rank * kSmallRows][0]) + (uint32_t)f * 16;
+            st_cluster_v4(map_to_rank(la, (uint32_t)r), *reinterpret_cast<const uint4*>(&s.g[rank * kSmallRows][4 * f]));
+        }
+        cluster_sync_all();
+        // ---- W1[i][j] = W0[i][j] - eta_scale ((W0 G)[i][j] - C[i][j]): thread (row a, column j)
+        {
+            const int a = tid >> 6, j = tid & (D - 1), i = rank * kSmallRows + a;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (!p.dot) {
+#pragma unroll 4
+                for (int m = 0; m < D; m += 4)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[q] = fmaf(s.w0[a][m + q], s.g[m + q][j], acc[q]);
+            }
+            const float w1 = s.w0[a][j] - p.eta_scale * (((acc[0] + acc[1]) + (acc[2] + acc[3])) - s.c[a][j]);
+            if (p.W1_out) p.W1_out[((size_t)u * D + i) * D + j] = w1;
+            s.w1t[j][i] = w1;
+        }
+        __syncthreads();
+        // ---- this CTA's rows of W1 are columns 8 rank .. 8 rank + 7 of w1t: two 16-byte pieces of each
+        //      of its 64 rows, into every other CTA of the cluster
+        for (int e = tid; e < (kSmallCS - 1) * D * 2; e += kSmallThreads) {
+            const int r = (rank + 1 + e / (D * 2)) % kSmallCS, m = (e / 2) % D, half = e & 1;
+            float* src = &s.w1t[m][rank * kSmallRows + 4 * half];
+            st_cluster_v4(map_to_rank(smem_u32(src), (uint32_t)r), *reinterpret_cast<const uint4*>(src));
+        }
+        cluster_sync_all();
+        // ---- z = W1 q for this CTA's tokens: thread (token group tg, output channel j) holds row j of
+        //      W1 in registers; the token's q comes as broadcast float4
+        {
+            const int j = tid & (D - 1), tg = tid >> 6;
+            float wr[D];
+#pragma unroll
+            for (int m = 0; m < D; ++m) wr[m] = s.w1t[m][j];
+            float* zb = p.Z + (long long)(u / p.heads) * p.zbs + (long long)h * p.zhs;
+            for (int t = tg; t < n1 - n0; t += kSmallThreads / D) {
+                float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m = 0; m < D; m += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(&s.q[t][m]);
+                    z[0] = fmaf(wr[m], q4.x, z[0]); z[1] = fmaf(wr[m + 1], q4.y, z[1]);
+                    z[2] = fmaf(wr[m + 2], q4.z, z[2]); z[3] = fmaf(wr[m + 3], q4.w, z[3]);
+                }
+                zb[(long long)(n0 + t) * D + j] = (z[0] + z[1]) + (z[2] + z[3]);
+            }
+        }
+        // s.k, s.v, s.q, s.w0 are reloaded for the next unit, and the peers' gathers of the next
+        // unit overwrite s.g and s.w1t: every CTA of the cluster is done with this unit first
+        cluster_sync_all();
+    }
+    // after a wait that gave up, the last unit's copies may still be landing
+    if (tid == 0 && it > 0) mbar_drain(&s.bar, (it - 1) & 1u, ab.limit);
+}
+
 constexpr int kMaxGridF32 = 160;
 
 struct WsLayout {
@@ -1033,6 +1219,48 @@ size_t linear_ws_bytes(const ttt_shape& s) {
 
 size_t linear_ws_control_bytes(const ttt_shape& s) {
     return lin::ws_layout((long long)s.batch * s.heads, s.dtype).w1;   // error word (and fp32 counters)
+}
+
+// fp32 units of at most kSmallN tokens: one kSmallCS-CTA cluster per unit (lin_small_f32).
+static ttt_status launch_small_f32(const Call& c, long long units) {
+    using namespace lin;
+    const size_t smem = sizeof(SmallSmem) + 128;
+    cudaFuncSetAttribute(lin_small_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(kSmallThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = kSmallCS; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    // every cluster co-resident: a persistent loop takes the units beyond them
+    long long ncl = std::min<long long>(units, c.num_sms / kSmallCS);
+    cfg.gridDim = dim3((unsigned)(ncl * kSmallCS));
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, lin_small_f32, &cfg) == cudaSuccess && active > 0)
+        ncl = std::min<long long>(ncl, active);
+    cudaGetLastError();
+    cfg.gridDim = dim3((unsigned)(ncl * kSmallCS));
+    if (c.grid_out) *c.grid_out = (int)(ncl * kSmallCS);
+    SmallParams p{};
+    p.Kv = TokenView{static_cast<const float*>(c.K), c.bs, c.hs};
+    p.Vv = TokenView{static_cast<const float*>(c.V), c.bs, c.hs};
+    p.Qv = TokenView{static_cast<const float*>(c.Q), c.bs, c.hs};
+    p.Z = static_cast<float*>(c.Z);
+    p.zbs = c.bs;
+    p.zhs = c.hs;
+    p.W0 = c.W0;
+    p.W1_out = c.W1_out;
+    p.heads = c.heads;
+    p.N = c.N;
+    p.units = (int)units;
+    p.dot = c.loss == TTT_LOSS_DOT;
+    p.eta_scale = p.dot ? c.eta / (float)c.N : c.eta * (2.0f / (float)c.N);
+    p.err = reinterpret_cast<uint32_t*>(c.err_ws ? c.err_ws : c.ws);
+    p.wait_ns = c.wait_ns;
+    return check_launch(cudaLaunchKernelEx(&cfg, lin_small_f32, p));
 }
 
 ttt_status launch_linear(const Call& c) {
@@ -1109,6 +1337,7 @@ ttt_status launch_linear(const Call& c) {
     m.W1_out = c.W1_out;
 
     // fp32
+    if (c.N <= kSmallN && c.num_sms >= kSmallCS) return launch_small_f32(c, units);
     const long long T = units * tpu;
     const int G = (int)std::min<long long>(std::min(c.num_sms, kMaxGridF32), T);
     m.W1_f32 = reinterpret_cast<float*>(c.ws + L.w1);
