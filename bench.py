@@ -56,7 +56,7 @@ TRAFFIC = {
     "conv3x3_6084_bf16": {"read": 18785024, "write": 7295744, "src_sha": "0d0c9febef88a717"},
     "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
     "bwd6084_bf16": {"read": 218148352, "write": 105013504, "src_sha": "c97c5f030b248cf5"},
-    "bwdconv6084_bf16": {"read": 24883456, "write": 17042944, "src_sha": "1dfe7c0812e5935d"},
+    "bwdconv6084_bf16": {"read": 24807936, "write": 16324864, "src_sha": "5f3347347183751c"},
     "bwdmlp1024_bf16": {"read": 67329024, "write": 145303808, "src_sha": "a33fe42962dd5335"},
 }
 

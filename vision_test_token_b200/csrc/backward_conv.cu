@@ -16,13 +16,15 @@
 // 2l+1, a 3 x 3 register window sliding along a grid row.  Four kernels on one stream, each a
 // programmatic dependent of the one before; every sum has a fixed order, so the results are bitwise
 // reproducible.  Positions are taken in tiles of 8 grid rows x 16 columns (warp w: row w of a tile).
+// Each tile's inputs (with the margins its taps reach) are first staged in shared memory with all of
+// their loads in flight, so that the per-position loops read no global memory.
 //   cb_reduce    per tile: the partial sums sum_p r_p K_{p+s_t} and sum_p dZ_p Q_{p+s_t} (2 x 64 x 9)
 //   cb_unit      per unit: the tile partials summed in tile order -> g, W1, dg, dW1 and the unit's
 //                deta term
 //   cb_map       per tile: r and dr on the tile and a one-position halo (shared memory), then dQ, dK,
 //                dV for the tile's positions and the tile's partial sum_p dr_p K_{p+s_t}
-//   cb_final     per head: dW0 = sum over images of (dW1 + the unit's map partials in tile order);
-//                block 0 also sums deta over the units
+//   cb_final     per (head, tap): dW0 = sum over images of (dW1 + the unit's map partials in tile
+//                order), the images' terms formed in parallel; block 0 also sums deta over the units
 #include <algorithm>
 
 #include "sm100.cuh"
@@ -88,12 +90,54 @@ __device__ __forceinline__ long long unit_off(const Geo& g, int u) {
     return (long long)(u / g.heads) * g.bs + (long long)(u % g.heads) * g.hs;
 }
 
+// The positions (y0 - MR .. y0 + TR - 1 + MR) x (x0 - MR .. x0 + TC - 1 + MR) of one unit's X, staged in
+// shared memory as rows of 64 channels (zero outside the grid), with all of the 16-byte loads in
+// flight before any is stored.
+template <typename T, int MR>
+__device__ __forceinline__ void stage_halo(T* dst, const T* base, const Geo& g, int y0, int x0) {
+    constexpr int RW = TC + 2 * MR, CH = D * (int)sizeof(T) / 16;
+    constexpr int TOT = (TR + 2 * MR) * RW * CH, PER = (TOT + kThreads - 1) / kThreads;
+    uint4 v[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int e = threadIdx.x + k * kThreads, pos = e / CH, ch = e % CH;
+        const int y = y0 - MR + pos / RW, x = x0 - MR + pos % RW;
+        v[k] = (e < TOT && y >= 0 && y < g.H && x >= 0 && x < g.W)
+                   ? __ldg(reinterpret_cast<const uint4*>(base + ((long long)y * g.W + x) * D) + ch)
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int e = threadIdx.x + k * kThreads;
+        if (e < TOT) reinterpret_cast<uint4*>(dst)[e] = v[k];
+    }
+}
+// Channel pair `lane` at staged row r, column c of a region RW positions wide.
+template <typename T>
+__device__ __forceinline__ float2 sat(const T* st, int RW, int r, int c, int lane);
+template <>
+__device__ __forceinline__ float2 sat<__nv_bfloat16>(const __nv_bfloat16* st, int RW, int r, int c, int lane) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(st + (r * RW + c) * D)[lane];
+    return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+}
+template <>
+__device__ __forceinline__ float2 sat<float>(const float* st, int RW, int r, int c, int lane) {
+    return reinterpret_cast<const float2*>(st + (r * RW + c) * D)[lane];
+}
+constexpr int KRW = TC + 4, ZRW = TC + 2;    // staged K (two-position margin), staged dZ (one)
+constexpr int kMaxFinalImages = 64;          // images whose terms cb_final holds at a time
+
 // ---- cb_reduce: one CTA per tile -----------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 cb_reduce(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ dZ,
           const Params p) {
-    __shared__ float red[TR][2][kPart];
+    extern __shared__ uint8_t smem_raw[];
+    float (*red)[2][kPart] = reinterpret_cast<float (*)[2][kPart]>(smem_raw);   // [TR][2][576]
+    T* ks = reinterpret_cast<T*>(smem_raw + sizeof(float) * TR * 2 * kPart);    // [TR+2][TC+2][64] K
+    T* qs = ks + (TR + 2) * ZRW * D;                                            // [TR+2][TC+2][64] Q
+    T* vs = qs + (TR + 2) * ZRW * D;                                            // [TR][TC][64] V
+    T* zs = vs + TR * TC * D;                                                   // [TR][TC][64] dZ
     const Geo& g = p.g;
     const int u = blockIdx.x / g.tpu, i = blockIdx.x % g.tpu;
     const int h = u % g.heads;
@@ -102,6 +146,11 @@ cb_reduce(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict_
     pdl_launch_dependents();
     const long long off = unit_off(g, u);
     const T *Ku = K + off, *Vu = V + off, *Qu = Q + off, *dZu = dZ + off;
+    stage_halo<T, 1>(ks, Ku, g, y0, x0);
+    stage_halo<T, 1>(qs, Qu, g, y0, x0);
+    stage_halo<T, 0>(vs, Vu, g, y0, x0);
+    stage_halo<T, 0>(zs, dZu, g, y0, x0);
+    __syncthreads();
     float2 w0[TAPS], sk[TAPS], zq[TAPS];
 #pragma unroll
     for (int t = 0; t < TAPS; ++t) {
@@ -114,17 +163,17 @@ cb_reduce(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict_
         const int xe = min(g.W, x0 + TC);
         float2 kw[3][3], qw[3][3];                           // [tap row][column x-1, x, x+1]
 #pragma unroll
-        for (int a = 0; a < 3; ++a) {
-            kw[a][0] = at(Ku, g, y + a - 1, x0 - 1, lane); kw[a][1] = at(Ku, g, y + a - 1, x0, lane);
-            qw[a][0] = at(Qu, g, y + a - 1, x0 - 1, lane); qw[a][1] = at(Qu, g, y + a - 1, x0, lane);
+        for (int a = 0; a < 3; ++a) {                        // staged row warp + a is grid row y + a - 1
+            kw[a][0] = sat<T>(ks, ZRW, warp + a, 0, lane); kw[a][1] = sat<T>(ks, ZRW, warp + a, 1, lane);
+            qw[a][0] = sat<T>(qs, ZRW, warp + a, 0, lane); qw[a][1] = sat<T>(qs, ZRW, warp + a, 1, lane);
         }
         for (int x = x0; x < xe; ++x) {
 #pragma unroll
             for (int a = 0; a < 3; ++a) {
-                kw[a][2] = at(Ku, g, y + a - 1, x + 1, lane);
-                qw[a][2] = at(Qu, g, y + a - 1, x + 1, lane);
+                kw[a][2] = sat<T>(ks, ZRW, warp + a, x - x0 + 2, lane);
+                qw[a][2] = sat<T>(qs, ZRW, warp + a, x - x0 + 2, lane);
             }
-            const float2 v = at(Vu, g, y, x, lane), dz = at(dZu, g, y, x, lane);
+            const float2 v = sat<T>(vs, TC, warp, x - x0, lane), dz = sat<T>(zs, TC, warp, x - x0, lane);
             float2 r = make_float2(-v.x, -v.y);
 #pragma unroll
             for (int t = 0; t < TAPS; ++t) r = fma2(w0[t], kw[t / 3][t % 3], r);
@@ -191,6 +240,8 @@ cb_map(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ d
     float2* rs = reinterpret_cast<float2*>(smem_raw);          // [HR*HC][32] r at the halo tile
     float2* drs = rs + HR * HC * 32;                           // [HR*HC][32] dr
     float* red = reinterpret_cast<float*>(drs + HR * HC * 32); // [TR][576]
+    T* ks = reinterpret_cast<T*>(red + TR * kPart);            // [TR+4][TC+4][64] K
+    T* zs = ks + (TR + 4) * KRW * D;                           // [TR+2][TC+2][64] dZ
     const Geo& g = p.g;
     const int u = blockIdx.x / g.tpu, i = blockIdx.x % g.tpu;
     const int h = u % g.heads;
@@ -199,11 +250,14 @@ cb_map(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ d
     pdl_launch_dependents();
     const long long off = unit_off(g, u);
     const T *Ku = K + off, *Vu = V + off, *dZu = dZ + off;
+    stage_halo<T, 2>(ks, Ku, g, y0, x0);                      // inputs: loaded before the wait
+    stage_halo<T, 1>(zs, dZu, g, y0, x0);
     float2 w0[TAPS];
 #pragma unroll
     for (int t = 0; t < TAPS; ++t)
         w0[t] = make_float2(__ldg(p.W0 + ((size_t)h * D + 2 * lane) * TAPS + t),
                             __ldg(p.W0 + ((size_t)h * D + 2 * lane + 1) * TAPS + t));
+    __syncthreads();
     pdl_wait_primary();                                       // W1, dg of the unit are formed
     const float* cf = p.coef + (size_t)u * 3 * kPart;
     float2 w1[TAPS], dgs[TAPS];                               // dgs = (2/N) dg
@@ -213,24 +267,30 @@ cb_map(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ d
         const float2 dg = __ldcg(reinterpret_cast<const float2*>(cf + kPart + t * D) + lane);
         dgs[t] = make_float2(g.scale * dg.x, g.scale * dg.y);
     }
-    // (1) r and dr at the tile and its halo (zero outside the grid)
+    // (1) r and dr at the tile and its halo (zero outside the grid); V six positions at a time, all
+    //     six loads in flight
     for (int hr = warp; hr < HR; hr += TR) {
         const int y = y0 - 1 + hr;
-        for (int hc = 0; hc < HC; ++hc) {
-            const int x = x0 - 1 + hc;
-            float2 r = make_float2(0.f, 0.f), dr = make_float2(0.f, 0.f);
-            if (y >= 0 && y < g.H && x >= 0 && x < g.W) {
-                const float2 v = at(Vu, g, y, x, lane);
-                r = make_float2(-v.x, -v.y);
+        for (int hc0 = 0; hc0 < HC; hc0 += 6) {
+            float2 v[6];
 #pragma unroll
-                for (int t = 0; t < TAPS; ++t) {
-                    const float2 k = at(Ku, g, y + t / 3 - 1, x + t % 3 - 1, lane);
-                    r = fma2(w0[t], k, r);
-                    dr = fma2(dgs[t], k, dr);
+            for (int q = 0; q < 6; ++q) v[q] = at(Vu, g, y, x0 - 1 + hc0 + q, lane);
+#pragma unroll
+            for (int q = 0; q < 6; ++q) {
+                const int hc = hc0 + q, x = x0 - 1 + hc;
+                float2 r = make_float2(0.f, 0.f), dr = make_float2(0.f, 0.f);
+                if (y >= 0 && y < g.H && x >= 0 && x < g.W) {
+                    r = make_float2(-v[q].x, -v[q].y);
+#pragma unroll
+                    for (int t = 0; t < TAPS; ++t) {
+                        const float2 k = sat<T>(ks, KRW, hr + t / 3, hc + t % 3, lane);
+                        r = fma2(w0[t], k, r);
+                        dr = fma2(dgs[t], k, dr);
+                    }
                 }
+                rs[(hr * HC + hc) * 32 + lane] = r;
+                drs[(hr * HC + hc) * 32 + lane] = dr;
             }
-            rs[(hr * HC + hc) * 32 + lane] = r;
-            drs[(hr * HC + hc) * 32 + lane] = dr;
         }
     }
     __syncthreads();
@@ -247,14 +307,14 @@ cb_map(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ d
 #pragma unroll
             for (int t = 0; t < TAPS; ++t) {
                 const int ay = t / 3 - 1, bx = t % 3 - 1;      // q - s_t
-                aq = fma2(w1[t], at(dZu, g, y - ay, x - bx, lane), aq);
+                aq = fma2(w1[t], sat<T>(zs, ZRW, warp + 1 - ay, x - x0 + 1 - bx, lane), aq);
                 const int hidx = ((hr - ay) * HC + (hc - bx)) * 32 + lane;
                 ak = fma2(dgs[t], rs[hidx], ak);
                 ak = fma2(w0[t], drs[hidx], ak);
             }
             const float2 dr = drs[(hr * HC + hc) * 32 + lane];
 #pragma unroll
-            for (int t = 0; t < TAPS; ++t) acc[t] = fma2(dr, at(Ku, g, y + t / 3 - 1, x + t % 3 - 1, lane), acc[t]);
+            for (int t = 0; t < TAPS; ++t) acc[t] = fma2(dr, sat<T>(ks, KRW, warp + 1 + t / 3, x - x0 + 1 + t % 3, lane), acc[t]);
             const long long o = ((long long)y * g.W + x) * D + 2 * lane;
             Elem<T>::st(dQ + off + o, aq);
             Elem<T>::st(dK + off + o, ak);
@@ -273,27 +333,50 @@ cb_map(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ d
     }
 }
 
-// ---- cb_final: one CTA per head (block 0 also sums deta) -----------------------------------------
-__global__ void __launch_bounds__(kPart)
+// ---- cb_final: per (head, tap) 64 channels; block 0 also sums deta ---------------------------------
+// dW0 = sum over images in order of (dW1 + the unit's tile partials in tile order).  Thread (c, b0)
+// forms the per-image terms of images b0, b0 + 8, ... (each with its tile loads in flight), then
+// thread c adds the images' terms in image order: the same sums, in the same order, as one thread
+// walking the images.
+constexpr int kFinalLanes = 8;
+__global__ void __launch_bounds__(D * kFinalLanes)
 cb_final(const Params p) {
     const Geo& g = p.g;
-    const int h = blockIdx.x, e = threadIdx.x, t = e / D, c = e % D;
+    __shared__ float img[kMaxFinalImages][D];
+    __shared__ float dterms[kFinalLanes * D];
+    const int h = blockIdx.x / TAPS, t = blockIdx.x % TAPS;
+    const int c = threadIdx.x % D, b0 = threadIdx.x / D, e = t * D + c;
     pdl_wait_primary();
+    const int B = g.U / g.heads;
     if (p.dW0_out) {
-        // images in order: per image dW1, then the image's tile partials in order
-        const int B = g.U / g.heads;
-        float acc = 0.f;
-        for (int b = 0; b < B; ++b) {
-            const int u = b * g.heads + h;
-            acc += add_strided_in_order(__ldcg(p.coef + (size_t)u * 3 * kPart + 2 * kPart + e),   // dW1
-                                        p.mapp + (size_t)u * g.tpu * kPart + e, kPart, g.tpu);
+        for (int bc = 0; bc < B; bc += kMaxFinalImages) {
+            const int nb = min(kMaxFinalImages, B - bc);
+            for (int b = b0; b < nb; b += kFinalLanes) {
+                const int u = (bc + b) * g.heads + h;
+                img[b][c] = add_strided_in_order(__ldcg(p.coef + (size_t)u * 3 * kPart + 2 * kPart + e),   // dW1
+                                                 p.mapp + (size_t)u * g.tpu * kPart + e, kPart, g.tpu);
+            }
+            __syncthreads();
+            if (b0 == 0) {
+                float acc = (bc == 0) ? 0.f : p.dW0_out[((size_t)h * D + c) * TAPS + t];
+                for (int b = 0; b < nb; ++b) acc += img[b][c];
+                p.dW0_out[((size_t)h * D + c) * TAPS + t] = acc;
+            }
+            __syncthreads();
         }
-        p.dW0_out[((size_t)h * D + c) * TAPS + t] = acc;
     }
-    if (h == 0 && e == 0 && p.deta_out) {
+    if (blockIdx.x == 0 && p.deta_out) {
+        // the units' terms loaded by the whole block, summed in unit order
         float acc = 0.f;
-        for (int u = 0; u < g.U; ++u) acc += __ldcg(p.deta_u + u);
-        *p.deta_out = acc;
+        for (int u0 = 0; u0 < g.U; u0 += kFinalLanes * D) {
+            const int n = min(kFinalLanes * D, g.U - u0);
+            __syncthreads();
+            if ((int)threadIdx.x < n) dterms[threadIdx.x] = __ldcg(p.deta_u + u0 + threadIdx.x);
+            __syncthreads();
+            if (threadIdx.x == 0)
+                for (int k = 0; k < n; ++k) acc += dterms[k];
+        }
+        if (threadIdx.x == 0) *p.deta_out = acc;
     }
 }
 
@@ -346,14 +429,19 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
     cfg.gridDim = dim3((unsigned)(U * tpu));
     cfg.blockDim = dim3(kThreads);
     cfg.numAttrs = 0;
+    const size_t smem_r = sizeof(float) * TR * 2 * kPart + ((size_t)2 * (TR + 2) * ZRW + 2 * TR * TC) * D * sizeof(T);
+    cudaFuncSetAttribute(cb_reduce<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
+    cfg.dynamicSmemBytes = smem_r;
     ttt_status st = check_launch(cudaLaunchKernelEx(&cfg, cb_reduce<T>, Q, K, V, dz, p));
     if (st != TTT_OK) return st;
     cfg.numAttrs = 1;
     cfg.gridDim = dim3((unsigned)U);
     cfg.blockDim = dim3(kPart);
+    cfg.dynamicSmemBytes = 0;
     st = check_launch(cudaLaunchKernelEx(&cfg, cb_unit, p));
     if (st != TTT_OK) return st;
-    const size_t smem = (size_t)2 * HR * HC * 32 * sizeof(float2) + (size_t)TR * kPart * sizeof(float);
+    const size_t smem = (size_t)2 * HR * HC * 32 * sizeof(float2) + (size_t)TR * kPart * sizeof(float) +
+                        ((size_t)(TR + 4) * KRW + (size_t)(TR + 2) * ZRW) * D * sizeof(T);
     cudaFuncSetAttribute(cb_map<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cfg.gridDim = dim3((unsigned)(U * tpu));
     cfg.blockDim = dim3(kThreads);
@@ -361,8 +449,8 @@ static ttt_status launch(const Call& c, const void* dZ, void* dQ, void* dK, void
     st = check_launch(cudaLaunchKernelEx(&cfg, cb_map<T>, K, V, dz, static_cast<T*>(dQ), static_cast<T*>(dK),
                                          static_cast<T*>(dV), p));
     if (st != TTT_OK) return st;
-    cfg.gridDim = dim3((unsigned)c.heads);
-    cfg.blockDim = dim3(kPart);
+    cfg.gridDim = dim3((unsigned)(c.heads * TAPS));
+    cfg.blockDim = dim3(D * kFinalLanes);
     cfg.dynamicSmemBytes = 0;
     return check_launch(cudaLaunchKernelEx(&cfg, cb_final, p));
 }
