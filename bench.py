@@ -48,15 +48,15 @@ L2_BYTES = 126 * 2 ** 20
 # --cache-control none on the third of three consecutive steps, so that the previous step's Z
 # write-back (which lands during the next step) is counted as it is in steady state.
 TRAFFIC = {
-    "mixed6084_bf16": {"read": 112356352, "write": 38231040, "src_sha": "88e63fe44a5cadc0"},
-    "mixed6084_dot_bf16": {"read": 112324352, "write": 38272256, "src_sha": "88e63fe44a5cadc0"},
-    "lin6400_bf16": {"read": 118183168, "write": 40068864, "src_sha": "e252f1ffc5b63f16"},
-    "lin196_bf16": {"read": 14328832, "write": 599040, "src_sha": "e252f1ffc5b63f16"},
+    "mixed6084_bf16": {"read": 112345856, "write": 38357504, "src_sha": "abb1454f1edc678c"},
+    "mixed6084_dot_bf16": {"read": 112343040, "write": 38928384, "src_sha": "abb1454f1edc678c"},
+    "lin6400_bf16": {"read": 118186240, "write": 39789312, "src_sha": "e54e80ef8998d239"},
+    "lin196_bf16": {"read": 14328576, "write": 824832, "src_sha": "e54e80ef8998d239"},
     "mlp1024_bf16": {"read": 25533440, "write": 6981376, "src_sha": "e351f2e6a0775778"},
     "conv3x3_6084_bf16": {"read": 18785024, "write": 7295744, "src_sha": "0d0c9febef88a717"},
     "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
     "bwd6084_bf16": {"read": 218148352, "write": 105013504, "src_sha": "c97c5f030b248cf5"},
-    "bwdconv6084_bf16": {"read": 24807936, "write": 16324864, "src_sha": "5f3347347183751c"},
+    "bwdconv6084_bf16": {"read": 24875776, "write": 16282112, "src_sha": "1518b59fd12bbd54"},
     "bwdmlp1024_bf16": {"read": 67329024, "write": 145303808, "src_sha": "a33fe42962dd5335"},
 }
 
