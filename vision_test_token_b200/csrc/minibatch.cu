@@ -11,10 +11,9 @@
 //     final weights.
 //
 // The loss decomposes over output features, so every row of W is an independent recurrence: row i
-// needs only k_t, q_t and the i-th value feature of each token.  A CTA of 64 threads takes 8 rows of
-// one unit (8 CTAs per unit), 8 lanes per row and 8 features per lane (4m..4m+3 and 32+4m..32+4m+3
-// for lane m, so that a row's 8 lanes read 128 contiguous bytes of a token).  Each lane keeps, for
-// its 8 weights, W_s (the weights the mini-batch started from: the residuals are taken there) and dW,
+// needs only k_t, q_t and the i-th value feature of each token.  A CTA of 128 threads takes 8 rows of
+// one unit (8 CTAs per unit), 16 lanes per row and 4 features per lane (4m..4m+3 for lane m, so that
+// a row's 16 lanes read a token's 256 contiguous bytes).  Each lane keeps, for its 4 weights, W_s (the weights the mini-batch started from: the residuals are taken there) and dW,
 // the update accumulated since, at its own scale (many small per-token terms added straight into W_s
 // would each be rounded at the scale of W).  No CTA waits on another.
 //
@@ -24,12 +23,12 @@
 // the memory latency).  Each sub-block is first converted to fp32 tiles.
 //
 // Per sub-block (sub-blocks never straddle a mini-batch):
-//   - each lane forms partial dot products W_s k_t over its 8 features for the 16 tokens, and a
-//     transpose-sum over the row's 8 lanes (14 shuffles) leaves lane m with the residuals of tokens
-//     2m and 2m+1, r_t = W_s k_t - v_t, which are then broadcast to the row's lanes;
+//   - each lane forms partial dot products W_s k_t over its 4 features for the 16 tokens, and a
+//     transpose-sum over the row's 16 lanes (15 shuffles) leaves lane m with the residual of token
+//     m, r_t = W_s k_t - v_t, which is then broadcast to the row's lanes;
 //   - token by token, dW -= scale r_t k_t (scale 2 eta, or 2 eta / |batch| in epoch mode), and in
-//     prefix mode the partial readout W_s . q_t + dW . q_t is formed right after token t's own
-//     update, so that z_t = W_t q_t; a second transpose-sum completes z;
+//     prefix mode the partial readout (W_s + dW) . q_t is formed right after token t's own update,
+//     so that z_t = W_t q_t; a second transpose-sum completes z;
 //   - at the end of a mini-batch W_s += dW, dW = 0.
 // Epoch mode then streams Q once more and reads out with the final weights.
 //
@@ -46,17 +45,17 @@ namespace mb {
 
 constexpr int D = 64;
 constexpr int RB = 8;               // rows of W per CTA
-constexpr int LPR = 8;              // lanes per row
+constexpr int LPR = 16;             // lanes per row
 constexpr int FPL = D / LPR;        // features per lane
 constexpr int T = 16;               // tokens per sub-block
-constexpr int THREADS = RB * LPR;   // 64
+constexpr int THREADS = RB * LPR;   // 128
 constexpr int kStages = 4;          // bulk-copy ring depth (sub-blocks in flight)
 constexpr int KP = D + 4;           // padded row pitch (floats) of the fp32 K and Q tiles
 constexpr int VP = RB + 1;
 constexpr int ZP = RB + 1;
 constexpr int kCtasPerUnit = D / RB;
 constexpr int kTileChunks = T * D / 8;                  // 8-element chunks of a K or Q tile: 128
-constexpr int kChunksPerThread = kTileChunks / THREADS; // 2
+constexpr int kChunksPerThread = kTileChunks / THREADS; // 1
 
 struct Params {
     const void* Q;
@@ -145,39 +144,42 @@ __device__ __forceinline__ Sub next_sub(const Params& p, const Sub& s) {
 
 __device__ __forceinline__ bool reads_q(const Params& p, const Sub& s) { return s.phase == 1 || p.mode == 0; }
 
-// v[0..15]: this lane's partials for tokens 0..15.  Afterwards v[0] and v[1] hold, in lane m of each
-// group of 8 lanes (m = lane & 7), the sums over the group's 8 lanes for tokens 2m and 2m + 1.
-__device__ __forceinline__ void transpose_sum8(float (&v)[T], int lane) {
+// v[0..15]: this lane's partials for tokens 0..15.  Afterwards v[0] holds, in lane m of each group
+// of 16 lanes (m = lane & 15), the sum over the group's 16 lanes for token m.
+__device__ __forceinline__ void transpose_sum16(float (&v)[T], int lane) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const bool up = lane & 4;
+        const bool up = lane & 8;
         const float send = up ? v[i] : v[i + 8];
         const float keep = up ? v[i + 8] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const bool up = lane & 2;
+        const bool up = lane & 4;
         const float send = up ? v[i] : v[i + 4];
         const float keep = up ? v[i + 4] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const bool up = lane & 1;
+        const bool up = lane & 2;
         const float send = up ? v[i] : v[i + 2];
         const float keep = up ? v[i + 2] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    {
+        const bool up = lane & 1;
+        const float send = up ? v[0] : v[1];
+        const float keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
     }
 }
 
-// Lane m's 8 features of a 64-wide fp32 row: 4m..4m+3 and 32+4m..32+4m+3.
-__device__ __forceinline__ float dot8(const float (&w)[FPL], const float* row, int m) {
+// Lane m's 4 features (4m .. 4m+3) of a 64-wide fp32 row.
+__device__ __forceinline__ float dot4(const float (&w)[FPL], const float* row, int m) {
     const float4 a = *reinterpret_cast<const float4*>(row + 4 * m);
-    const float4 b = *reinterpret_cast<const float4*>(row + 32 + 4 * m);
-    const float lo = fmaf(w[3], a.w, fmaf(w[2], a.z, fmaf(w[1], a.y, w[0] * a.x)));
-    const float hi = fmaf(w[7], b.w, fmaf(w[6], b.z, fmaf(w[5], b.y, w[4] * b.x)));
-    return lo + hi;
+    return fmaf(w[3], a.w, fmaf(w[2], a.z, fmaf(w[1], a.y, w[0] * a.x)));
 }
 
 // Bounded wait that ignores the abort flag (draining copies that are still in flight).
@@ -197,9 +199,9 @@ lin_minibatch(const Params p) {
     constexpr uint32_t kTileBytes = T * D * sizeof(E);
     uint8_t* ring = smem_raw + kCtlBytes + ((sizeof(Tiles) + 127) / 128) * 128;
     const int tid = threadIdx.x, lane = tid & 31;
-    const int rl = tid >> 3;                        // row of this lane within the CTA's 8 rows
-    const int m = tid & 7;                          // feature group; tokens 2m, 2m+1 after a transpose-sum
-    const int gbase = lane & 24;                    // first lane of this row's group of 8
+    const int rl = tid >> 4;                        // row of this lane within the CTA's 8 rows
+    const int m = tid & 15;                         // feature group; token m after a transpose-sum
+    const int gbase = lane & 16;                    // first lane of this row's group of 16
     const Abort ab{&ctl.abort_flag, p.err, p.wait_ns};
     if (tid == 0) {
         ctl.abort_flag = 0;
@@ -242,8 +244,7 @@ lin_minibatch(const Params p) {
         {
             const float* src = p.W0 + ((size_t)h * D + i) * D;
             const float4 a = __ldg(reinterpret_cast<const float4*>(src + 4 * m));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 32 + 4 * m));
-            ws[0] = a.x; ws[1] = a.y; ws[2] = a.z; ws[3] = a.w; ws[4] = b.x; ws[5] = b.y; ws[6] = b.z; ws[7] = b.w;
+            ws[0] = a.x; ws[1] = a.y; ws[2] = a.z; ws[3] = a.w;
 #pragma unroll
             for (int c = 0; c < FPL; ++c) dw[c] = 0.f;
         }
@@ -291,23 +292,19 @@ lin_minibatch(const Params p) {
             if (cur.phase == 0) {
                 // residuals at the mini-batch's start weights
 #pragma unroll
-                for (int t = 0; t < T; ++t) acc[t] = dot8(ws, s.k[t], m);
-                transpose_sum8(acc, lane);
-                float r0 = acc[0] - s.v[2 * m][rl], r1 = acc[1] - s.v[2 * m + 1][rl];
-                if (2 * m >= cur.cnt) r0 = 0.f;
-                if (2 * m + 1 >= cur.cnt) r1 = 0.f;
+                for (int t = 0; t < T; ++t) acc[t] = dot4(ws, s.k[t], m);
+                transpose_sum16(acc, lane);
+                const float r = (m < cur.cnt) ? acc[0] - s.v[m][rl] : 0.f;
                 const float scale = (p.mode == 0) ? 2.0f * p.eta : 2.0f * p.eta / (float)cur.batch_len;
-                // token by token: dW -= scale r_t k_t, then (prefix mode) the partial readout W_t . q_t
+                // token by token: dW -= scale r_t k_t, then (prefix mode) the partial readout
+                // W_s . q_t + dW . q_t, so that z_t = W_t q_t
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
-                    const float rt = __shfl_sync(0xffffffffu, (t & 1) ? r1 : r0, gbase + (t >> 1));
-                    const float c = -scale * rt;
+                    const float c = -scale * __shfl_sync(0xffffffffu, r, gbase + t);
                     const float4 ka = *reinterpret_cast<const float4*>(&s.k[t][4 * m]);
-                    const float4 kb = *reinterpret_cast<const float4*>(&s.k[t][32 + 4 * m]);
-                    dw[0] = fmaf(c, ka.x, dw[0]); dw[1] = fmaf(c, ka.y, dw[1]); dw[2] = fmaf(c, ka.z, dw[2]);
-                    dw[3] = fmaf(c, ka.w, dw[3]); dw[4] = fmaf(c, kb.x, dw[4]); dw[5] = fmaf(c, kb.y, dw[5]);
-                    dw[6] = fmaf(c, kb.z, dw[6]); dw[7] = fmaf(c, kb.w, dw[7]);
-                    if (p.mode == 0) acc[t] = dot8(ws, s.q[t], m) + dot8(dw, s.q[t], m);
+                    dw[0] = fmaf(c, ka.x, dw[0]); dw[1] = fmaf(c, ka.y, dw[1]);
+                    dw[2] = fmaf(c, ka.z, dw[2]); dw[3] = fmaf(c, ka.w, dw[3]);
+                    if (p.mode == 0) acc[t] = dot4(ws, s.q[t], m) + dot4(dw, s.q[t], m);
                 }
                 if (cur.batch_end) {
 #pragma unroll
@@ -316,13 +313,12 @@ lin_minibatch(const Params p) {
             } else {
                 // epoch-mode readout with the final weights
 #pragma unroll
-                for (int t = 0; t < T; ++t) acc[t] = dot8(ws, s.q[t], m);
+                for (int t = 0; t < T; ++t) acc[t] = dot4(ws, s.q[t], m);
             }
             const bool writes_z = reads_q(p, cur);
             if (writes_z) {
-                transpose_sum8(acc, lane);
-                s.z[2 * m][rl] = acc[0];
-                s.z[2 * m + 1][rl] = acc[1];
+                transpose_sum16(acc, lane);
+                s.z[m][rl] = acc[0];
             }
             __syncthreads();
             if (writes_z) {
@@ -336,7 +332,6 @@ lin_minibatch(const Params p) {
         if (p.W1_out) {
             float* dst = p.W1_out + ((size_t)u * D + i) * D;
             *reinterpret_cast<float4*>(dst + 4 * m) = make_float4(ws[0], ws[1], ws[2], ws[3]);
-            *reinterpret_cast<float4*>(dst + 32 + 4 * m) = make_float4(ws[4], ws[5], ws[6], ws[7]);
         }
     }
 }
