@@ -54,7 +54,7 @@ TRAFFIC = {
     "lin196_bf16": {"read": 14328576, "write": 824832, "src_sha": "e54e80ef8998d239"},
     "mlp1024_bf16": {"read": 25533440, "write": 6981376, "src_sha": "e351f2e6a0775778"},
     "conv3x3_6084_bf16": {"read": 18785024, "write": 7295744, "src_sha": "0d0c9febef88a717"},
-    "mb16_6084_bf16": {"read": 112638208, "write": 37697536, "src_sha": "17a7fdb7e5ba2966"},
+    "mb16_6084_bf16": {"read": 112244992, "write": 37442304, "src_sha": "a3a28c9aeba97913"},
     "bwd6084_bf16": {"read": 218148352, "write": 105013504, "src_sha": "c97c5f030b248cf5"},
     "bwdconv6084_bf16": {"read": 24875776, "write": 16282112, "src_sha": "1518b59fd12bbd54"},
     "bwdmlp1024_bf16": {"read": 67329024, "write": 145303808, "src_sha": "a33fe42962dd5335"},

@@ -69,6 +69,8 @@ def test_sm_budget(cuda_dev, max_sms, dtype):
     (37, 1, 15, 20),     # 3 tiles per unit, units spread over several CTAs
     (200, 1, 10, 13),    # many small units: CTAs span several units
     (2, 3, 77, 79),      # ragged large units
+    (1, 2, 16, 24),      # 384 tokens: the largest unit of the fp32 cluster kernel
+    (1, 1, 5, 77),       # 385 tokens: the fp32 tile kernels again
 ])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_odd_shapes(cuda_dev, B, h, H, W, dtype):
