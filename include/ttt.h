@@ -305,8 +305,10 @@ ttt_status ttt_forward_layer(const void* Q, const void* K, const void* V, const 
  * nothing sets, and then takes the steps every bounded wait of the layer kernels takes when it runs
  * out: it records TTT_ERR_TIMEOUT in the workspace error word and returns.  ttt_workspace_status(ws)
  * then reports TTT_ERR_TIMEOUT (and clears it).  ws: any workspace of at least 256 bytes that is
- * zero-filled (ttt_workspace_init); it must not be in use by another call.
- * Errors: TTT_ERR_WORKSPACE (ws NULL or too small), TTT_ERR_ALIGNMENT, TTT_ERR_INVALID_ARG. */
+ * zero-filled (ttt_workspace_init); it must not be in use by another call.  ws = NULL: the
+ * library-owned array of ttt_forward_linear_noalloc on the current device (ws_bytes is ignored), whose
+ * timeout ttt_noalloc_status then reports.
+ * Errors: TTT_ERR_WORKSPACE (ws too small), TTT_ERR_ALIGNMENT, TTT_ERR_INVALID_ARG. */
 ttt_status ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned long long limit_ns, void* stream);
 
 /* Bound, in nanoseconds (1 .. 1e9; 1e9 at load), of every device-side wait of the kernels launched

@@ -133,7 +133,7 @@ def test_dot_loss_shapes_size_like_l2(lib):
 
 def test_selftest_rejects_bad_arguments(lib):
     fake = ctypes.c_void_p(1 << 20)
-    assert capi.ttt_selftest_wait_timeout(None, 256, 1000, None) == capi.TTT_ERR_WORKSPACE
+    assert capi.ttt_selftest_wait_timeout(None, 256, 0, None) == capi.TTT_ERR_INVALID_ARG   # checked first
     assert capi.ttt_selftest_wait_timeout(fake, 100, 1000, None) == capi.TTT_ERR_WORKSPACE
     assert capi.ttt_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 16), 256, 1000, None) == capi.TTT_ERR_ALIGNMENT
     assert capi.ttt_selftest_wait_timeout(fake, 256, 0, None) == capi.TTT_ERR_INVALID_ARG

@@ -88,3 +88,22 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_dev):
     assert capi.ttt_workspace_bytes(capi.TTT_HEAD_LINEAR, shape) > (8 << 20)
     st = capi.ttt_forward_linear_noalloc(p, p, p, p, p, 0.5, shape, None, torch.cuda.current_stream().cuda_stream)
     assert st == capi.TTT_ERR_WORKSPACE
+
+
+def test_noalloc_status_reports_a_timeout_once(cuda_dev):
+    """A bounded wait that runs out on the library-owned array (the self-test kernel pointed at it) is
+    reported by ttt_noalloc_status once, and the next no-alloc call is still correct."""
+    stream = torch.cuda.current_stream().cuda_stream
+    _, x = random_unit(2, 2, 12, 12, dtype="bf16", seed=17)
+    _noalloc(x, 0.5, 12, 12, cuda_dev)
+    assert capi.ttt_noalloc_status(stream) == capi.TTT_OK
+    assert capi.ttt_selftest_wait_timeout(None, 0, 2_000_000, stream) == capi.TTT_OK
+    assert capi.ttt_noalloc_status(stream) == capi.TTT_ERR_TIMEOUT
+    assert capi.ttt_noalloc_status(stream) == capi.TTT_OK
+    Q, K, V = (x[k].to(cuda_dev) for k in ("Q", "K", "V"))
+    W1_ref = torch.empty((2, 2, 64, 64), device=cuda_dev)
+    Z_ref = forward_linear(Q, K, V, x["W0_lin"].to(cuda_dev), 0.5, 12, 12, W1_out=W1_ref)
+    Z, W1 = _noalloc(x, 0.5, 12, 12, cuda_dev)
+    assert rel_max_err(Z, Z_ref.double().cpu().numpy()) <= TOL["bf16"]
+    assert rel_max_err(W1, W1_ref.double().cpu().numpy()) <= TOL["bf16"]
+    assert capi.ttt_noalloc_status(stream) == capi.TTT_OK

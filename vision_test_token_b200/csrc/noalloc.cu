@@ -33,7 +33,7 @@ static CtxGetCurrentFn ctx_get_current() {
 // Device address of the scratch on the current device.  It is looked up on the first use per device
 // and again whenever the device's current context differs from the one the address was taken in
 // (after a cudaDeviceReset the module is loaded anew and the old address is stale).
-static ttt_status noalloc_scratch(void** out) {
+ttt_status noalloc_scratch(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return check_launch(e);

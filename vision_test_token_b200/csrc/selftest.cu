@@ -31,9 +31,14 @@ __global__ void selftest_wait(const uint32_t* flag, uint32_t* err, unsigned long
 using namespace ttt;
 
 extern "C" ttt_status ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned long long limit_ns, void* stream) {
-    if (!ws || ws_bytes < kWsHeader) return TTT_ERR_WORKSPACE;
-    if (reinterpret_cast<uintptr_t>(ws) % 256) return TTT_ERR_ALIGNMENT;
     if (limit_ns == 0 || limit_ns > 1000000000ull) return TTT_ERR_INVALID_ARG;
+    if (!ws) {                       // the no-alloc entry point's array: reported by ttt_noalloc_status
+        const ttt_status st = noalloc_scratch(&ws);
+        if (st != TTT_OK) return st;
+        ws_bytes = kWsHeader;
+    }
+    if (ws_bytes < kWsHeader) return TTT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % 256) return TTT_ERR_ALIGNMENT;
     uint32_t* words = static_cast<uint32_t*>(ws);
     selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(words + kSelftestFlagWord, words, limit_ns);
     return check_launch(cudaGetLastError());

@@ -42,6 +42,10 @@ struct Call {
     unsigned long long wait_ns;   // bound of every device-side wait of the launch (ns)
 };
 
+// The library-owned array of ttt_forward_linear_noalloc on the current device (its first 256 bytes
+// are a workspace header).
+ttt_status noalloc_scratch(void** out);
+
 // Bound of the device-side waits of every launch (ns), process-wide (ttt_set_wait_limit).
 unsigned long long wait_limit_ns();
 
