@@ -57,7 +57,7 @@ TRAFFIC = {
     "mb16_6084_bf16": {"read": 112244992, "write": 37442304, "src_sha": "a3a28c9aeba97913"},
     "bwd6084_bf16": {"read": 218148352, "write": 105013504, "src_sha": "c97c5f030b248cf5"},
     "bwdconv6084_bf16": {"read": 24875776, "write": 16282112, "src_sha": "1518b59fd12bbd54"},
-    "bwdmlp1024_bf16": {"read": 67770368, "write": 145598464, "src_sha": "67c8f10cdb74fb80"},
+    "bwdmlp1024_bf16": {"read": 66835712, "write": 145287168, "src_sha": "82c10e7f21b6b7f8"},
 }
 
 # Kernels of this library launched per step, by workload kind (bf16; fp32 where it differs).

@@ -121,6 +121,19 @@ __device__ __forceinline__ float dot_hidden(float init, const float* px, const f
     for (; jj < n; ++jj) a0 = fmaf(ld(px + (size_t)jj * D), y[jj], a0);
     return (a0 + a1) + (a2 + a3);
 }
+// sum_jj (s1 x1[jj] y1[jj] + x2[jj] y2[jj]) likewise (per term: the x2 product first, then x1's).
+template <class LD1, class LD2>
+__device__ __forceinline__ float dot_hidden2(float s1, const float* px1, const float* y1, LD1 ld1, const float* px2,
+                                             const float* y2, LD2 ld2, int n) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    int jj = 0;
+    for (; jj + 4 <= n; jj += 4)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            a[q] = fmaf(s1 * ld1(px1 + (size_t)(jj + q) * D), y1[jj + q], fmaf(ld2(px2 + (size_t)(jj + q) * D), y2[jj + q], a[q]));
+    for (; jj < n; ++jj) a[0] = fmaf(s1 * ld1(px1 + (size_t)jj * D), y1[jj], fmaf(ld2(px2 + (size_t)jj * D), y2[jj], a[0]));
+    return (a[0] + a[1]) + (a[2] + a[3]);
+}
 __device__ __forceinline__ float ld_nc(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
@@ -392,10 +405,7 @@ mb_upd(const T* __restrict__ K, const T* __restrict__ V, T* __restrict__ dK, T* 
         }
         __syncthreads();
         {                                                    // dr = s dgWb a + Wb db
-            float acc = 0.f;
-            for (int jj = 0; jj < hid; ++jj)
-                acc = fmaf(s * __ldcg(dgBT + (size_t)jj * D + ci), av[0][ti][jj],
-                           fmaf(__ldg(WbT + (size_t)jj * D + ci), av[3][ti][jj], acc));
+            const float acc = dot_hidden2(s, dgBT + ci, av[0][ti], ld_cg, WbT + ci, av[3][ti], ld_nc, hid);
             rv[1][ti][ci] = ti < nt ? acc : 0.f;
             if (ti < nt) stx(dV + off + (long long)(n + ti) * D + ci, -acc);
         }
@@ -421,10 +431,7 @@ mb_upd(const T* __restrict__ K, const T* __restrict__ V, T* __restrict__ dK, T* 
         }
         __syncthreads();
         {                                                    // dk = s dgWa^T e + Wa^T dh
-            float acc = 0.f;
-            for (int jj = 0; jj < hid; ++jj)
-                acc = fmaf(s * __ldcg(dgA + (size_t)jj * D + ci), av[2][ti][jj],
-                           fmaf(__ldg(Wa + (size_t)jj * D + ci), av[4][ti][jj], acc));
+            const float acc = dot_hidden2(s, dgA + ci, av[2][ti], ld_cg, Wa + ci, av[4][ti], ld_nc, hid);
             if (ti < nt) stx(dK + off + (long long)(n + ti) * D + ci, acc);
         }
         __syncthreads();
