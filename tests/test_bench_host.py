@@ -73,3 +73,10 @@ def test_kernel_source_hash_is_stable_and_per_kind():
     assert len(bench.kernel_source_hash()) == 16
     assert set(bench.KIND_SOURCES) >= {w.kind for w in WORKLOADS.values()}
     assert bench.kernel_source_hash("mixed") != bench.kernel_source_hash("mlp")
+
+
+def test_source_hash_sees_code_not_comments():
+    """A capture stays valid across comment edits, and only across them."""
+    assert bench.code_of(b"int a; // one\n\n// two\n  int b;  \n") == bench.code_of(b"int a;\n  int b;")
+    assert bench.code_of(b"int a;\n  int b;") == b"int a;\n  int b;"
+    assert bench.code_of(b"int a = 1;") != bench.code_of(b"int a = 2;")

@@ -354,9 +354,9 @@ lin_bwd_sum(const Params p, int batch) {
 //                     16-token step accumulate [K | V]^T K (M = 128: the G rows, then the C rows)
 //                     and [dZ | Q]^T Q (M = 128, of which the dZ rows are dW1).  At the end of each
 //                     unit's run of tiles the accumulators go to the (CTA, unit) partial slot.
-//   lin_bwd_merge_tc  one CTA per unit (programmatic dependent of p1): the slot sum and the unit's
-//                     matrices as in merge_unit, then the four maps of phase 2 as bf16 hi + lo
-//                     operand images (128-byte swizzled rows c, K = i).
+//   lin_bwd_merge_tc  1, 2 or 4 CTAs per unit (programmatic dependent of p1), each a share of the
+//                     unit's rows: the slot sum, the unit's matrices as in merge_unit, and the four
+//                     maps of phase 2 as bf16 hi + lo operand images (128-byte swizzled rows c, K = i).
 //   lin_bwd_p2_tc     static partition of 128-token tiles over one CTA per SM (programmatic
 //                     dependent of the merge): per tile the boxes dZ, K, V; dQ = dZ W1, dV = K dC^T,
 //                     dK = V dC + K (dG + dG^T), each against the hi and lo image; the

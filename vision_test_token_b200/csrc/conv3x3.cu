@@ -11,29 +11,31 @@
 //     R = K~ W0~^T - V          (positions x 64,   K = 576: nine taps of 64 channels)
 //     G = sum_pos K~^T R        (576 x 64: the gradient, transposed)
 //     Z = Q~ W1~^T              (positions x 64)
-// The tap shifts are never materialised: each tap's operand is a TMA box of the grid at the shifted
-// origin, whose out-of-bounds zero fill is the zero padding.  Tiles are 8 rows x 16 columns of the
-// grid (128 positions, the MMA's M).
+// The tap shifts are never materialised.  Tiles are 8 rows x 16 columns of the grid (128 positions,
+// the MMA's M); a tile's K (or Q) comes as three TMA boxes of its rows -1 .. 8, one per x shift, and
+// tap (a, b) is the 128 rows of box b that start at row 16a (tap_box below).  The boxes' out-of-bounds
+// zero fill is the zero padding.
 //
 // Four kernels on one stream, each a programmatic dependent of the one before:
 //   conv3_wprep   W0 rounded to bf16 and laid out as nine swizzled tap operand images per head (row
 //                 c, K = c'), once per call, so that each gradient CTA loads its head's weights with
 //                 one bulk copy instead of gathering them from the [c][c'][a][b] layout.
-//   conv3_grad    (per CTA, a contiguous range of tiles; per tile) TMA loads V and the 9 K boxes
-//                 (two taps per 32 KB ring stage); R = K~ W0~^T accumulates over the taps (A = K box,
-//                 K-major; B = W0 tap image, rows c, K = c'); the epilogue forms r = R - V, zeroes
-//                 positions outside the grid and splits r into bf16 hi + lo (about 16 significant
-//                 bits); the 9 K boxes are streamed again and G^T += [K_t | K_t+1]^T (r_hi + r_lo)
-//                 accumulates in five tap-pair accumulators (A MN-major, M = 128 = two taps' channels;
-//                 B = r, MN-major).  At the end of each unit's part of the range the accumulators
-//                 are written to the workspace slot of (CTA, unit), as G[tap][c][c'] so that the
-//                 32 lanes of a warp (32 consecutive c') store one 128-byte line per instruction.
+//   conv3_grad    (a fixed number of CTAs per unit, each a contiguous share of one unit's tiles;
+//                 per tile) the three K halo boxes by TMA, two tiles' halos resident; R = K~ W0~^T
+//                 accumulates over the taps (A = the tap's rows of a halo box, K-major; B = W0 tap
+//                 image, rows c, K = c'); the epilogue reads V straight from global memory, forms
+//                 r = R - V, zeroes positions outside the grid and splits r into bf16 hi + lo (about
+//                 16 significant bits); G^T += [K_a | K_b]^T (r_hi + r_lo) accumulates in five
+//                 tap-pair accumulators (A MN-major, M = 128 = two taps' channels; B = r, MN-major).
+//                 The MMAs run R(n+1) before G(n).  At the end of its tiles the CTA writes the
+//                 accumulators to its workspace slot as G[tap][c][c'], so that the 32 lanes of a
+//                 warp (32 consecutive c') store one 128-byte line per instruction.
 //   conv3_merge   per (unit, tap): the unit's slots summed in CTA order (a fixed order: bitwise
 //                 reproducible for a given grid), W1 = W0 - eta (2/N) g in fp32 (W1_out), and W1
 //                 rounded once to bf16 as the tap's operand image for the readout.
-//   conv3_readout (per CTA, a contiguous range of tiles) Z = sum_t Q_t W1_t^T over the 9 shifted Q
-//                 boxes, drained to bf16 and stored with TMA (the store clips positions outside the
-//                 grid).
+//   conv3_readout (per CTA, a contiguous range of tiles) Z = sum_t Q_t W1_t^T over the tile's three
+//                 Q halo boxes, drained to bf16 and stored with TMA (the store clips positions
+//                 outside the grid).
 // The weights are read in bf16 for R (their rounding changes r by about 2^-9 of |f(K;W0)|) and r is
 // carried as hi + lo, so the update keeps close to fp32 accuracy relative to the gradient's terms.
 #include <algorithm>
