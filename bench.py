@@ -76,6 +76,14 @@ KIND_SOURCES = {"linear": ["linear.cu"], "mixed": ["linear.cu", "dwconv.cu"], "m
 COMMON_SOURCES = ["sm100.cuh", "api.cu"]
 
 
+def launches_per_step(w):
+    """Kernels of this library one step of workload w launches (on all SMs)."""
+    n = (LAUNCHES_PER_STEP_FP32 if w.dtype == "fp32" else {}).get(w.kind, LAUNCHES_PER_STEP[w.kind])
+    if w.dtype == "fp32" and w.kind in ("linear", "mixed") and w.N <= SMALL_F32_TOKENS:
+        n -= 1                               # one cluster kernel instead of the two tile kernels
+    return n
+
+
 def code_of(src):
     """A source file's code for the hash: line comments and blank lines removed (the library's sources
     put no comment marker inside a string literal and use no block comments)."""
@@ -685,9 +693,7 @@ def run_ours(args):
     # end to end through the public API: pinned host inputs -> device -> step -> host result
     e2e = run_e2e(w, xs[0], dev, stream, args.e2e_steps, world)
 
-    per_step = (LAUNCHES_PER_STEP_FP32 if w.dtype == "fp32" else {}).get(w.kind, LAUNCHES_PER_STEP[w.kind])
-    if w.dtype == "fp32" and w.kind in ("linear", "mixed") and w.N <= SMALL_F32_TOKENS:
-        per_step -= 1                        # one cluster kernel instead of the two tile kernels
+    per_step = launches_per_step(w)
     line = {"metric": METRIC_BWD if w.kind.startswith("backward") else METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",

@@ -80,3 +80,14 @@ def test_source_hash_sees_code_not_comments():
     assert bench.code_of(b"int a; // one\n\n// two\n  int b;  \n") == bench.code_of(b"int a;\n  int b;")
     assert bench.code_of(b"int a;\n  int b;") == b"int a;\n  int b;"
     assert bench.code_of(b"int a = 1;") != bench.code_of(b"int a = 2;")
+
+
+def test_launches_per_step():
+    """The kernels a step launches, as the bench line's gpu_launches counts them."""
+    counts = {name: bench.launches_per_step(w) for name, w in WORKLOADS.items()}
+    assert counts["mixed6084_bf16"] == 2                      # linear heads and conv head at once
+    assert counts["lin196_fp32"] == 1                         # one cluster kernel for a small fp32 unit
+    assert counts["lin6400_bf16"] == counts["lin196_bf16"] == 1
+    assert counts["conv3x3_6084_bf16"] == 4                   # W0 images, gradient, merge, readout
+    assert counts["bwd6084_bf16"] == 4                        # phase 1, merge, phase 2, sums
+    assert bench.launches_per_step(Workload("big32", 1, 1, 40, 40, "fp32", 0.5, "linear")) == 2
